@@ -1,0 +1,108 @@
+"""Analytic cost model of the LatentMoE layer: the paper's roofline formulas
+and the algorithmic FLOP / byte counts the benchmark divides by.
+
+Paper formulas (LatentMoE, arXiv 2601.18089):
+* Section 2.1: the compute-bound threshold F / BW_HBM, the per-expert cost
+  C_exp = 2 t d m and traffic M_exp = d m + t (d + m), and the arithmetic
+  intensity I = 2 t d m / (d m + t (d + m)) (also the Figure 2 caption).
+* Section 2.2: the communication / compute time ratio 5 F / (4 m BW_NVL).
+* Table 1: the per-expert weight-loading cost d m (standard MoE) versus
+  l m (LatentMoE).
+
+Algorithmic counts (what the layer must compute and move at minimum, used for
+the achieved-throughput figures): only the experts that at least one token
+reaches have their weights read; every other tensor is read or written once;
+the intermediates (latent rows, expert hidden rows, expert outputs, the
+combined rows) are excluded and reported separately as overhead.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+from typing import Optional, Sequence
+
+
+# ---- the paper's closed forms ------------------------------------------------
+
+def compute_bound_threshold(F: float, bw_hbm: float) -> float:
+    """FLOPs per byte above which a kernel is compute bound (Section 2.1)."""
+    return F / bw_hbm
+
+
+def expert_cost(t_exp: float, d: float, m: float):
+    """(C_exp, M_exp) for one expert fed t_exp tokens (Section 2.1)."""
+    return 2.0 * t_exp * d * m, d * m + t_exp * (d + m)
+
+
+def arithmetic_intensity(t_exp: float, d: float, m: float) -> float:
+    """I = 2 t d m / (d m + t (d + m)) (Section 2.1, Figure 2)."""
+    c, mem = expert_cost(t_exp, d, m)
+    return c / mem
+
+
+def threshold_tokens(I: float, d: float, m: float) -> float:
+    """Smallest t_exp with arithmetic_intensity(t_exp, d, m) >= I; the root of
+    2 t d m = I (d m + t (d + m))."""
+    den = 2.0 * d * m - I * (d + m)
+    if den <= 0:
+        return float("inf")
+    return I * d * m / den
+
+
+def comm_compute_ratio(F: float, m: float, bw_nvl: float) -> float:
+    """All-to-all time over expert compute time under expert parallelism with
+    FP4 dispatch and BF16 combine (Section 2.2): 5 F / (4 m BW_NVL)."""
+    return 5.0 * F / (4.0 * m * bw_nvl)
+
+
+def weight_load_per_expert(width: float, m: float) -> float:
+    """Weight-loading memory cost per expert (Table 1): d m for a standard
+    MoE, l m for LatentMoE."""
+    return width * m
+
+
+# ---- algorithmic counts of one forward pass ----------------------------------
+
+@dataclass
+class LayerCounts:
+    flops: float            # whole layer
+    bytes: float            # whole layer, algorithmic
+    expert_flops: float     # the two expert GEMMs
+    fc1_flops: float
+    fc1_bytes: float        # FC1 kernel: touched W1 + latent rows in + hidden rows out
+    fc2_flops: float
+    fc2_bytes: float        # FC2 kernel: touched W2 + hidden rows in + expert rows out
+    expert_weight_bytes: float
+    intermediate_bytes: float
+    touched: int
+    t_exp_mean: float
+
+
+def layer_counts(*, T: int, d: int, l: int, N: int, k: int, m: int, act: str,
+                 shared_m: int = 0, skip_proj: bool = False, elem_bytes: int = 2,
+                 loads: Optional[Sequence[int]] = None) -> LayerCounts:
+    """Counts for one pass over T tokens.  ``loads`` are the per-expert row
+    counts (default: every expert touched)."""
+    m_in = 2 * m if act == "swiglu" else m
+    ms_in = 2 * shared_m if act == "swiglu" else shared_m
+    R = T * k
+    touched = N if loads is None else sum(1 for c in loads if c > 0)
+    eb = elem_bytes
+    fc1_flops = 2.0 * R * l * m_in
+    fc2_flops = 2.0 * R * m * l
+    router_flops = 2.0 * T * d * N
+    proj_flops = 0.0 if skip_proj else 2.0 * (2.0 * T * d * l)
+    shared_flops = 2.0 * T * (d * ms_in + shared_m * d)
+    flops = router_flops + proj_flops + fc1_flops + fc2_flops + shared_flops
+    w1 = touched * l * m_in * eb
+    w2 = touched * m * l * eb
+    other_w = d * N * eb + (0 if skip_proj else 2 * d * l * eb) + (d * ms_in + shared_m * d) * eb
+    io = 2.0 * T * d * eb
+    byts = w1 + w2 + other_w + io
+    fc1_bytes = w1 + T * l * eb + R * m * eb
+    fc2_bytes = w2 + R * m * eb + R * l * eb
+    inter = 2.0 * eb * (R * l + R * m + R * l + T * l)
+    return LayerCounts(flops=flops, bytes=byts, expert_flops=fc1_flops + fc2_flops,
+                       fc1_flops=fc1_flops, fc1_bytes=fc1_bytes, fc2_flops=fc2_flops,
+                       fc2_bytes=fc2_bytes, expert_weight_bytes=w1 + w2,
+                       intermediate_bytes=inter, touched=touched,
+                       t_exp_mean=(R / touched) if touched else 0.0)

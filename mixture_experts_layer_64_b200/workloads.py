@@ -1,0 +1,206 @@
+"""Seeded synthetic workloads for the LatentMoE layer.
+
+This module holds the five workload shapes and the seeded generator of their
+inputs (token activations, router / projection / expert weights, router bias).
+It contains none of the layer's arithmetic: both the CUDA library (through the
+tests and the benchmark) and the CPU oracle consume the exact bytes it
+produces, so the generator never affects parity.
+
+Input recipe
+------------
+* ``x ~ N(0, 1)``.
+* Every weight ``~ N(0, 1/fan_in)``, fan_in being the input width of the
+  matrix: d for the router, the down-projection and the shared expert's first
+  matrix; the latent width l for the expert FC1 and the up-projection; the
+  expert width m for FC2; the shared width for the shared expert's second
+  matrix.  In the standard-MoE shape (l = d, projections skipped) FC1 has
+  fan_in d.
+* Router bias (only where a workload asks for one): ``N(0, variance 0.5)`` for
+  the latent decode shape; for the skewed prefill shape the log of a
+  Zipf(s=1.1) law over experts ranked by index,
+  ``b[e] = ln((e+1)^-1.1 / H_{N,1.1})``, computed in float64 and stored fp32.
+* Storage: fp32 for the tiny shape, bf16 (round-to-nearest-even of the fp32
+  draw) for the others; the bias is always fp32.
+* Weights use the API layout ``[in, out]`` row-major (``y = x @ W``).  The
+  SwiGLU FC1 matrix is ``[l, 2m]``: columns ``[0, m)`` feed the SiLU gate and
+  columns ``[m, 2m)`` are the linear ("up") half.
+
+Every tensor (and, for the expert stacks, every expert) draws from its own
+``torch.Generator`` seeded by ``(workload seed, tensor id, expert)``, so a
+tensor can be produced in pieces, on the CPU or on a CUDA device, and a subset
+of experts can be regenerated without the rest.  Values drawn on different
+device types differ (different Philox streams); any single run draws each
+tensor once and hands the same bytes to both sides.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, replace
+from typing import Dict, Optional
+
+import torch
+
+ACTS = ("silu", "swiglu", "relu2")
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    T: int
+    d: int
+    l: int
+    N: int
+    k: int
+    m: int
+    act: str
+    shared_m: int = 0
+    dtype: str = "bf16"          # "f32" or "bf16"
+    skip_proj: bool = False      # l == d and the two projections are identities
+    bias: Optional[str] = None   # None, "normal0.5" or "zipf1.1"
+    seed: int = 0
+
+    @property
+    def m_in(self) -> int:
+        return 2 * self.m if self.act == "swiglu" else self.m
+
+    @property
+    def ms_in(self) -> int:
+        return 2 * self.shared_m if self.act == "swiglu" else self.shared_m
+
+    @property
+    def torch_dtype(self) -> torch.dtype:
+        return torch.float32 if self.dtype == "f32" else torch.bfloat16
+
+    def with_T(self, T: int) -> "Workload":
+        return replace(self, T=T)
+
+
+# The five workloads: a tiny fp32 layer, the standard-MoE decode shape
+# (projections skipped), the latent decode shape, latent prefill with a
+# full-width shared expert, and high-sparsity skewed prefill.
+WORKLOADS: Dict[str, Workload] = {
+    "tiny-fp32": Workload("tiny-fp32", T=64, d=256, l=64, N=16, k=4, m=128,
+                          act="silu", dtype="f32", seed=0),
+    "std-moe-decode": Workload("std-moe-decode", T=256, d=4096, l=4096, N=128,
+                               k=8, m=1536, act="swiglu", skip_proj=True,
+                               seed=1),
+    "latent-decode": Workload("latent-decode", T=256, d=4096, l=1024, N=512,
+                              k=32, m=1536, act="swiglu", bias="normal0.5",
+                              seed=2),
+    "latent-prefill-shared": Workload("latent-prefill-shared", T=4096, d=4096,
+                                      l=1024, N=512, k=22, m=2048,
+                                      act="relu2", shared_m=3072, seed=3),
+    "latent-prefill-skewed": Workload("latent-prefill-skewed", T=16384,
+                                      d=7168, l=1792, N=896, k=16, m=1024,
+                                      act="swiglu", bias="zipf1.1", seed=4),
+}
+WORKLOAD_ORDER = list(WORKLOADS)
+
+_TID = {"x": 1, "Wg": 2, "bias": 3, "Wdown": 4, "Wup": 5, "W1": 6, "W2": 7,
+        "Ws1": 8, "Ws2": 9}
+
+
+def _gen(seed: int, tid: int, sub: int, device) -> torch.Generator:
+    g = torch.Generator(device=device)
+    g.manual_seed(((seed * 1_000_003 + tid) * 65_537 + sub) & 0x7FFF_FFFF_FFFF_FFFF)
+    return g
+
+
+def _normal(shape, std: float, seed: int, tid: int, sub: int, device,
+            dtype: torch.dtype) -> torch.Tensor:
+    g = _gen(seed, tid, sub, device)
+    t = torch.randn(shape, generator=g, device=device, dtype=torch.float32)
+    if std != 1.0:
+        t.mul_(std)
+    return t.to(dtype)
+
+
+def zipf_log_bias(N: int, s: float = 1.1) -> torch.Tensor:
+    """ln of a Zipf(s) probability law over N experts ranked by index."""
+    H = math.fsum((r + 1) ** -s for r in range(N))
+    return torch.tensor([math.log(((e + 1) ** -s) / H) for e in range(N)],
+                        dtype=torch.float64).to(torch.float32)
+
+
+def make_bias(w: Workload, device="cpu") -> Optional[torch.Tensor]:
+    if w.bias is None:
+        return None
+    if w.bias == "normal0.5":
+        return _normal((w.N,), math.sqrt(0.5), w.seed, _TID["bias"], 0, device,
+                       torch.float32)
+    if w.bias == "zipf1.1":
+        return zipf_log_bias(w.N, 1.1).to(device)
+    raise ValueError(f"unknown bias recipe {w.bias!r}")
+
+
+def make_x(w: Workload, device="cpu", T: Optional[int] = None) -> torch.Tensor:
+    T = w.T if T is None else T
+    return _normal((T, w.d), 1.0, w.seed, _TID["x"], 0, device, w.torch_dtype)
+
+
+def make_expert_W1(w: Workload, e: int, device="cpu") -> torch.Tensor:
+    return _normal((w.l, w.m_in), 1.0 / math.sqrt(w.l), w.seed, _TID["W1"], e,
+                   device, w.torch_dtype)
+
+
+def make_expert_W2(w: Workload, e: int, device="cpu") -> torch.Tensor:
+    return _normal((w.m, w.l), 1.0 / math.sqrt(w.m), w.seed, _TID["W2"], e,
+                   device, w.torch_dtype)
+
+
+def make_weights(w: Workload, device="cpu", experts: bool = True) -> Dict[str, Optional[torch.Tensor]]:
+    """All weights of one layer, API layout.  With ``experts=False`` the expert
+    stacks W1/W2 are left out (use make_expert_W1/W2 per expert)."""
+    dt = w.torch_dtype
+    out: Dict[str, Optional[torch.Tensor]] = {}
+    out["Wg"] = _normal((w.d, w.N), 1.0 / math.sqrt(w.d), w.seed, _TID["Wg"], 0,
+                        device, dt)
+    out["bias"] = make_bias(w, device)
+    if w.skip_proj:
+        out["Wdown"] = None
+        out["Wup"] = None
+    else:
+        out["Wdown"] = _normal((w.d, w.l), 1.0 / math.sqrt(w.d), w.seed,
+                               _TID["Wdown"], 0, device, dt)
+        out["Wup"] = _normal((w.l, w.d), 1.0 / math.sqrt(w.l), w.seed,
+                             _TID["Wup"], 0, device, dt)
+    if experts:
+        W1 = torch.empty((w.N, w.l, w.m_in), dtype=dt, device=device)
+        W2 = torch.empty((w.N, w.m, w.l), dtype=dt, device=device)
+        for e in range(w.N):
+            W1[e] = make_expert_W1(w, e, device)
+            W2[e] = make_expert_W2(w, e, device)
+        out["W1"] = W1
+        out["W2"] = W2
+    if w.shared_m:
+        out["Ws1"] = _normal((w.d, w.ms_in), 1.0 / math.sqrt(w.d), w.seed,
+                             _TID["Ws1"], 0, device, dt)
+        out["Ws2"] = _normal((w.shared_m, w.d), 1.0 / math.sqrt(w.shared_m),
+                             w.seed, _TID["Ws2"], 0, device, dt)
+    else:
+        out["Ws1"] = None
+        out["Ws2"] = None
+    return out
+
+
+def make_logits(T: int, N: int, seed: int, bias: Optional[torch.Tensor] = None,
+                ties: bool = True, device="cpu") -> torch.Tensor:
+    """fp32 router logits for routing-only tests: N(0,1) plus an optional bias,
+    with exact ties, signed zeros and repeated values planted in some rows."""
+    g = _gen(seed, 100, 0, "cpu")
+    lg = torch.randn((T, N), generator=g, dtype=torch.float32)
+    if bias is not None:
+        lg += bias.to("cpu", torch.float32)[None, :]
+    if ties and T > 0:
+        r = torch.randint(0, 4, (T,), generator=g)
+        for t in range(T):
+            if r[t] == 0:      # a block of identical values
+                c = torch.randint(0, N, (max(2, N // 4),), generator=g)
+                lg[t, c] = lg[t, c[0]].item()
+            elif r[t] == 1:    # +0.0 and -0.0 mixed with exact zeros
+                c = torch.randint(0, N, (max(2, N // 3),), generator=g)
+                sign = torch.randint(0, 2, (c.numel(),), generator=g)
+                lg[t, c] = torch.where(sign == 0, torch.tensor(0.0), torch.tensor(-0.0))
+            elif r[t] == 2:    # an entire row of one value
+                lg[t, :] = 0.25
+    return lg.to(device)
