@@ -1,0 +1,428 @@
+#!/usr/bin/env python
+"""Benchmark of the LatentMoE layer forward pass on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--no-cpu-baseline]
+
+One step is one lmoe_forward over the workload's T tokens (router, top-k,
+grouping, down-projection, expert FC1/FC2, combine, up-projection, residual).
+Inputs are seeded synthetic tensors resident in HBM; the expert weights
+(GBs) exceed the 126 MB L2, so every step streams them from HBM.  With N GPUs
+(one process each, launched by torchrun) every rank runs an independent
+replica on its own batch: tokens are independent, so there is no data-path
+collective; the timed region is bracketed by a barrier and
+torch.cuda.synchronize(), and the time is the max over ranks.
+
+Prints one JSON line (rank 0).  --impl reference times the CPU oracle (the
+reference arm of this method: a plain float64 C++ implementation) on a
+bounded token sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import datetime
+import hashlib
+import io
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from mixture_experts_layer_64_b200 import costmodel, workloads  # noqa: E402
+
+METRIC = "LatentMoE layer tokens/sec at decode & prefill T; HBM GB/s / tensor-pipe % of peak"
+UNIT = "tokens/s"
+DEFAULT_WORKLOAD = "std-moe-decode"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNEL_SOURCES = ["mixture_experts_layer_64_b200/csrc/" + f for f in
+                  ("common.cuh", "tc_gemm.cuh", "simt_gemm.cuh", "routing.cuh", "misc.cuh", "lmoe.cu")]
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            d = json.load(fh)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def recorded_traffic(workload: str, stage: str):
+    """DRAM bytes per launch of `stage` from the committed ncu summary, or None
+    when absent or taken on other kernel sources."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as fh:
+        d = json.load(fh)
+    rec = d.get(workload, {}).get(stage)
+    if not rec or rec.get("kernel_sources") != kernel_source_hash():
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{gpu_index}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.fh, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        rows = []
+        with open(self.path) as fh:
+            for r in csv.reader(fh):
+                if len(r) >= 9:
+                    rows.append([c.strip() for c in r])
+        if not rows:
+            return None
+
+        def num(s):
+            try:
+                return float(s)
+            except ValueError:
+                return float("nan")
+
+        sm = [num(r[1]) for r in rows]
+        mx = [num(r[2]) for r in rows]
+        pw = [num(r[3]) for r in rows]
+        # samples under load: the top half by power draw
+        order = sorted(range(len(rows)), key=lambda i: -pw[i] if pw[i] == pw[i] else 0)
+        load = order[: max(1, len(order) // 2)]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[j] for i in load for j in range(4)
+                          if rows[i][5 + j].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm[i] for i in load),
+                "sm_max_mhz": max(x for x in mx if x == x) if any(x == x for x in mx) else None,
+                "reasons": reasons, "samples": len(rows), "samples_under_load": len(load)}
+
+
+# ---------------------------------------------------------------------------
+# oracle (CPU baseline / reference arm)
+# ---------------------------------------------------------------------------
+
+class OracleRunner:
+    """Times the CPU oracle on token samples of a workload.  Host copies of the
+    weights are taken once; expert matrices are copied on first use."""
+
+    def __init__(self, w: workloads.Workload, W_dev, x_dev):
+        import oracle
+
+        self.oracle = oracle
+        self.w = w
+        self.threads = oracle.default_threads()
+        cpu = lambda t: None if t is None else t.detach().cpu()
+        self.W_dev = W_dev
+        self.x = cpu(x_dev)
+        self.base = dict(d=w.d, l=w.l, N=w.N, k=w.k, m=w.m, act=w.act, shared_m=w.shared_m,
+                         dtype=w.dtype, skip_proj=w.skip_proj, Wg=cpu(W_dev["Wg"]),
+                         bias=cpu(W_dev["bias"]), Wdown=cpu(W_dev["Wdown"]),
+                         Wup=cpu(W_dev["Wup"]), Ws1=cpu(W_dev["Ws1"]), Ws2=cpu(W_dev["Ws2"]))
+        self.probe = oracle.OracleLayer(W1={}, W2={}, **self.base)
+        self.W1, self.W2 = {}, {}
+
+    def time_tokens(self, tokens: np.ndarray) -> float:
+        """Seconds the oracle takes for the whole layer on `tokens` (routing
+        probe and weight copies untimed)."""
+        lg = self.probe.router_logits(self.x, tokens).astype(np.float32)
+        idx, _, _, _ = self.oracle.route(lg, self.w.k)
+        for e in np.unique(idx).tolist():
+            if e not in self.W1:
+                self.W1[e] = self.W_dev["W1"][e].cpu()
+                self.W2[e] = self.W_dev["W2"][e].cpu()
+        O = self.oracle.OracleLayer(W1=self.W1, W2=self.W2, **self.base)
+        t0 = time.perf_counter()
+        O.layer(self.x, tokens=tokens)
+        return time.perf_counter() - t0
+
+    def sample(self, n: int, seed: int) -> np.ndarray:
+        rng = np.random.default_rng(seed)
+        n = max(1, min(n, self.w.T))
+        return np.sort(rng.choice(self.w.T, size=n, replace=False)).astype(np.int32)
+
+    def calibrated_rate(self, target_s: float, seed: int = 0):
+        """(tokens/s, tokens, seconds) on a sample sized to take ~target_s."""
+        n = min(self.w.T, 4)
+        dt = self.time_tokens(self.sample(n, seed))
+        n2 = int(min(self.w.T, max(n, n / dt * target_s)))
+        if n2 > n:
+            dt = self.time_tokens(self.sample(n2, seed + 1))
+            n = n2
+        return n / dt, n, dt
+
+
+# ---------------------------------------------------------------------------
+# the arms
+# ---------------------------------------------------------------------------
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def workload_config(w: workloads.Workload, n_gpus: int):
+    c = costmodel.layer_counts(T=w.T, d=w.d, l=w.l, N=w.N, k=w.k, m=w.m, act=w.act,
+                               shared_m=w.shared_m, skip_proj=w.skip_proj)
+    return {"workload": w.name, "T": w.T, "d": w.d, "l": w.l, "N": w.N, "k": w.k, "m": w.m,
+            "act": w.act, "shared_m": w.shared_m, "skip_proj": w.skip_proj, "bias": w.bias,
+            "global_batch": w.T * n_gpus, "parallelism": f"replicas{n_gpus}",
+            "l2": f"inputs larger than L2: {c.expert_weight_bytes / 1e9:.2f} GB of expert "
+                  "weights streamed from HBM every step"}
+
+
+def run_reference(args):
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    w = workloads.WORKLOADS[args.workload]
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    W = workloads.make_weights(w, device=dev)
+    x = workloads.make_x(w, device=dev)
+    runner = OracleRunner(w, W, x)
+    steps = args.steps + args.warmup
+    budget_s = 150.0
+    rate, _, _ = runner.calibrated_rate(target_s=min(10.0, budget_s / steps))
+    per_step = int(min(w.T, max(1, rate * budget_s / steps)))
+    tok, sec = 0, 0.0
+    for s in range(steps):
+        dt = runner.time_tokens(runner.sample(per_step, seed=100 + s))
+        if s >= args.warmup:
+            tok += per_step
+            sec += dt
+    value = tok / sec
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1000.0 * sec / max(1, args.steps), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(w, 1),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": runner.threads,
+                             "kind": "oracle",
+                             "sample": f"{per_step} of {w.T} tokens per step ({w.name}), whole "
+                                       "layer from x (fp64 logits, fp32 selection)"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args):
+    from mixture_experts_layer_64_b200 import build, lmoe
+
+    ws, rank, local = dist_env()
+    pg = None
+    if ws > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+        pg = dist
+    else:
+        torch.cuda.set_device(0)
+    build.build_library()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    w = workloads.WORKLOADS[args.workload]
+    W = workloads.make_weights(w, device=dev)
+    # each replica draws its own batch
+    xw = w if rank == 0 else workloads.Workload(**{**w.__dict__, "seed": w.seed + 1000 * rank})
+    x = workloads.make_x(xw, device=dev)
+    L = lmoe.LatentMoELayer(w.d, w.l, w.N, w.k, w.m, act=w.act, shared_m=w.shared_m,
+                            dtype=w.dtype, skip_proj=w.skip_proj)
+    L.set_weights(W["Wg"], W["bias"], W["Wdown"], W["Wup"], W["W1"], W["W2"], W["Ws1"], W["Ws2"])
+    L.reserve(w.T)
+    out = torch.empty_like(x)
+    stream = torch.cuda.current_stream()
+
+    for _ in range(args.warmup):
+        L.forward(x, out)
+    torch.cuda.synchronize()
+    st, word = L.last_error()
+    if st != lmoe.OK:
+        raise RuntimeError(f"device error after warm-up: {lmoe.status_string(st)} word={word}")
+    launches_per_step = L.last_launch_count
+    loads = np.diff(L.debug_dump("offsets", w.T).cpu().numpy())
+
+    sampler = ClockSampler(local) if rank == 0 else None
+    if sampler:
+        sampler.start()
+    # ---- timed region: K steps, stage events recorded on the launching stream
+    L.profile_begin(args.steps)
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        L.forward(x, out)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    if pg:
+        pg.barrier()
+    clocks = sampler.stop() if sampler else None
+    elapsed_ms = t0.elapsed_time(t1)
+    prof = L.profile_end()
+    if pg:
+        tt = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
+        pg.all_reduce(tt, op=pg.ReduceOp.MAX)
+        elapsed_ms = float(tt.item())
+    ms_per_step = elapsed_ms / args.steps
+    value = w.T * ws / (ms_per_step / 1000.0)
+
+    # ---- end to end through the host-buffer entry point (pinned buffers)
+    xh = x.cpu().pin_memory()
+    oh = torch.empty_like(xh).pin_memory()
+    for _ in range(max(1, args.warmup // 2)):
+        L.forward_host(xh, oh)
+    e_steps = max(3, min(args.steps, 200))
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e_steps):
+        L.forward_host(xh, oh)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e_ms = e0.elapsed_time(e1) / e_steps
+    if pg:
+        tt = torch.tensor([e_ms], device=dev, dtype=torch.float64)
+        pg.all_reduce(tt, op=pg.ReduceOp.MAX)
+        e_ms = float(tt.item())
+    io_bytes = w.T * w.d * (4 if w.dtype == "f32" else 2)
+
+    st, word = L.last_error()
+    if st != lmoe.OK:
+        raise RuntimeError(f"device error: {lmoe.status_string(st)} word={word}")
+
+    # ---- roofline of the dominant kernel (stage averages over the timed steps)
+    stage_ms = {k: statistics.fmean(p[k] for p in prof) for k in prof[0]} if prof else {}
+    counts = costmodel.stage_counts(T=w.T, d=w.d, l=w.l, N=w.N, k=w.k, m=w.m, act=w.act,
+                                    shared_m=w.shared_m, skip_proj=w.skip_proj,
+                                    elem_bytes=4 if w.dtype == "f32" else 2, loads=loads)
+    peaks, peak_src = load_peaks()
+    roofline = None
+    if stage_ms:
+        dom = max(stage_ms, key=stage_ms.get)
+        fl, by = counts[dom]
+        t = stage_ms[dom] / 1000.0
+        ridge = peaks["bf16_tflops_sustained"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+        if by > 0 and (fl / by) < ridge:
+            ach, pk, unit, bound = by / t / 1e9, peaks["hbm_gbs"], "GB/s", "hbm"
+        else:
+            ach, pk, unit, bound = fl / t / 1e12, peaks["bf16_tflops_sustained"], "TFLOP/s", "tensor"
+        roofline = {"bound": bound, "achieved": ach, "peak": pk, "unit": unit, "frac": ach / pk,
+                    "traffic": recorded_traffic(w.name, dom), "kernel": dom,
+                    "algorithmic_per_launch": by if bound == "hbm" else fl,
+                    "launch_ms": stage_ms[dom], "peak_source": f"{peak_src} "
+                    f"({'hbm_gbs' if bound == 'hbm' else 'bf16_tflops_sustained'})",
+                    "stage_ms": {k: round(v, 5) for k, v in stage_ms.items()}}
+        lc = costmodel.layer_counts(T=w.T, d=w.d, l=w.l, N=w.N, k=w.k, m=w.m, act=w.act,
+                                    shared_m=w.shared_m, skip_proj=w.skip_proj, loads=loads)
+        roofline["layer"] = {"alg_bytes": lc.bytes, "alg_flops": lc.flops,
+                             "hbm_frac": lc.bytes / (ms_per_step / 1e3) / 1e9 / peaks["hbm_gbs"],
+                             "touched_experts": lc.touched,
+                             "t_exp_mean": round(lc.t_exp_mean, 2),
+                             "paper_intensity": costmodel.arithmetic_intensity(
+                                 lc.t_exp_mean, w.l, w.m) if lc.touched else None}
+
+    cpu_baseline = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        try:
+            runner = OracleRunner(w, W, x)
+            rate, n, dt = runner.calibrated_rate(target_s=15.0)
+            cpu_baseline = {"value": rate, "unit": UNIT, "cores": runner.threads,
+                            "kind": "oracle",
+                            "sample": f"{n} of {w.T} tokens of {w.name} ({dt:.1f} s), whole "
+                                      "layer from x"}
+        except Exception as e:  # the baseline is reported, never required
+            cpu_baseline = {"value": None, "unit": UNIT, "cores": None, "kind": "oracle",
+                            "sample": f"failed: {e}"}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+                "config": workload_config(w, ws),
+                "e2e": {"value": w.T * ws / (e_ms / 1000.0), "unit": UNIT,
+                        "h2d_bytes_per_step": io_bytes, "d2h_bytes_per_step": io_bytes},
+                "gpu_launches": launches_per_step * args.steps,
+                "roofline": roofline, "cpu_baseline": cpu_baseline, "clocks": clocks,
+                "expert_path": ["cuda-core", "tcgen05 token-tiled",
+                                "tcgen05 weight-stationary"][max(0, L.last_expert_path)]}
+        print(json.dumps(line), flush=True)
+    L.close()
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=workloads.WORKLOAD_ORDER, default=DEFAULT_WORKLOAD)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,234 @@
+/*
+ * lmoe.h -- C ABI of the B200 (sm_100a) LatentMoE layer forward pass.
+ *
+ * The layer (LatentMoE: Toward Optimal Accuracy per FLOP and Parameter in
+ * Mixture of Experts, arXiv 2601.18089, Section 3, Eq. (1) and Eq. (2)):
+ *
+ *   logits = x Wg (+ bias)                     router, full width d
+ *   slots  = top-k of logits, ties to the lowest expert index
+ *   w      = softmax over the k selected logits (renormalised gates)
+ *   z      = x Wdown                           down-projection d -> l
+ *   y_j    = act(z W1[e_j]) W2[e_j]            routed experts in latent width
+ *   comb   = sum_j w_j y_j                     gate-weighted combine
+ *   out    = x + comb Wup + act(x Ws1) Ws2     up-projection, shared expert,
+ *                                              residual add
+ *
+ * act is SiLU (non-gated), SwiGLU (FC1 has 2m columns: [0,m) is the SiLU
+ * gate, [m,2m) the linear half) or squared ReLU (non-gated).  The shared
+ * expert, when present, uses the same act.  With LMOE_SKIP_PROJ the layer is
+ * the paper's standard MoE (Table 1, first row): l == d, z = x, u = comb.
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers on the handle's device, row
+ *     major and contiguous, unless a parameter says "host".  The caller owns
+ *     them; the library never frees or retains them past the call.
+ *   - Weights use the API layout [in, out] (y = x W).
+ *   - dtype (set at create) applies to x, out and every weight; the router
+ *     bias and all logits are fp32; indices are int32.
+ *   - Calls taking a stream are asynchronous on it: they enqueue work and
+ *     return; results are ready when the stream is.  They never allocate and
+ *     never synchronise the host, except where stated.
+ *   - Errors are returned as lmoe_status and never thrown.  Arguments are
+ *     validated before any work is enqueued; on an error nothing is enqueued.
+ *     Device-side failures (a bounded wait that ran out, a failed debug
+ *     check) set a device error word that lmoe_last_error reads.
+ *   - A handle is not thread safe: one host thread at a time per handle.
+ *     Calls on one handle share its workspace, so calls enqueued on
+ *     different streams must not overlap on the GPU.
+ */
+#ifndef LMOE_H
+#define LMOE_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st* lmoe_stream_t;
+
+typedef enum {
+  LMOE_OK = 0,
+  LMOE_ERR_INVALID_ARG = 1,   /* a bad size, pointer, flag or state         */
+  LMOE_ERR_NOT_READY = 2,     /* weights not set / workspace not reserved   */
+  LMOE_ERR_CUDA = 3,          /* a CUDA runtime or driver call failed       */
+  LMOE_ERR_OOM = 4,           /* device allocation failed                   */
+  LMOE_ERR_TIMEOUT = 5,       /* a device-side bounded wait gave up         */
+  LMOE_ERR_UNSUPPORTED = 6,   /* valid but outside this build's limits      */
+  LMOE_ERR_DEVICE = 7         /* a device-side check failed (error word)    */
+} lmoe_status;
+
+typedef enum { LMOE_ACT_SILU = 0, LMOE_ACT_SWIGLU = 1, LMOE_ACT_RELU2 = 2 } lmoe_act;
+typedef enum { LMOE_F32 = 0, LMOE_BF16 = 1 } lmoe_dtype;
+
+/* Flags of lmoe_create. */
+#define LMOE_SKIP_PROJ     0x1u  /* l == d, no projections (standard MoE)       */
+#define LMOE_DEBUG_CHECKS  0x2u  /* device range checks and non-finite checks   */
+#define LMOE_FORCE_SIMT    0x4u  /* bf16: every contraction on the CUDA-core
+                                    kernels instead of tcgen05 (for testing)    */
+#define LMOE_FORCE_SWAP    0x8u  /* always use the weight-stationary (swap-AB)
+                                    expert kernels (for testing)                */
+#define LMOE_FORCE_NOSWAP  0x10u /* never use them (for testing)                */
+
+/* Limits of this build. */
+#define LMOE_MAX_EXPERTS 1024
+#define LMOE_MAX_TOPK    32
+
+/* Bits of the device error word. */
+#define LMOE_DEVERR_WAIT_TIMEOUT 0x1  /* an mbarrier wait ran past its limit     */
+#define LMOE_DEVERR_RANGE        0x2  /* an index out of range (debug checks)    */
+#define LMOE_DEVERR_NONFINITE    0x4  /* a NaN/Inf logit (debug checks)          */
+
+typedef struct lmoe_layer lmoe_layer;
+
+/*
+ * lmoe_create -- a layer handle on the current CUDA device.
+ * d: hidden width; l: latent width (== d with LMOE_SKIP_PROJ); N: routed
+ * experts (1..LMOE_MAX_EXPERTS); k: active experts per token
+ * (1..min(N, LMOE_MAX_TOPK)); m: expert width; shared_m: shared-expert width
+ * (0: none).  Paper: d, l, N', K (or K'), m of Section 3; S shared experts of
+ * Eq. (1) are one expert of S times the width.
+ * Allocates nothing on the device.  *out receives the handle (NULL on error).
+ * Errors: INVALID_ARG for any size out of range or unknown act/dtype/flag;
+ * CUDA if no device is usable.
+ */
+lmoe_status lmoe_create(int d, int l, int N, int k, int m, lmoe_act act, int shared_m,
+                        lmoe_dtype dtype, unsigned flags, lmoe_layer** out);
+
+/*
+ * lmoe_set_weights -- copy the weights into library-owned device storage
+ * (repacked to the kernels' layout; the caller may free its tensors after
+ * the call returns).  Synchronous: returns when the copy is done.
+ *   W_g     [d, N]            router (paper W'_r, transposed)
+ *   bias    [N] fp32 or NULL  additive per-expert router bias
+ *   W_down  [d, l]            down-projection (NULL iff LMOE_SKIP_PROJ)
+ *   W_up    [l, d]            up-projection   (NULL iff LMOE_SKIP_PROJ)
+ *   W1      [N, l, m_in]      expert FC1; m_in = 2m for SwiGLU, else m
+ *   W2      [N, m, l]         expert FC2
+ *   Ws1     [d, ms_in]        shared FC1 (NULL iff shared_m == 0)
+ *   Ws2     [shared_m, d]     shared FC2 (NULL iff shared_m == 0)
+ * May be called again to replace the weights.  Allocates (once) the weight
+ * storage.  Errors: INVALID_ARG (NULL where required or non-NULL where not),
+ * OOM, CUDA.
+ */
+lmoe_status lmoe_set_weights(lmoe_layer* h, const void* W_g, const float* bias,
+                             const void* W_down, const void* W_up, const void* W1,
+                             const void* W2, const void* Ws1, const void* Ws2);
+
+/*
+ * lmoe_reserve -- size the workspace for up to max_T tokens per call.
+ * Allocates; call it before lmoe_forward / lmoe_route_only /
+ * lmoe_router_logits / lmoe_forward_host.  Calling it again with a larger
+ * max_T reallocates (synchronously).  Errors: INVALID_ARG (max_T < 1), OOM.
+ */
+lmoe_status lmoe_reserve(lmoe_layer* h, int max_T);
+
+/*
+ * lmoe_forward -- the layer on T tokens (Eq. (1)/(2) plus the residual):
+ * out[T, d] = x + MoE(x).  x and out must not alias.  0 <= T <= reserved
+ * max_T (T == 0 enqueues nothing).  Errors: NOT_READY (no weights or no
+ * workspace), INVALID_ARG (T out of range, NULL pointer), CUDA.
+ */
+lmoe_status lmoe_forward(lmoe_layer* h, const void* x, void* out, int T, lmoe_stream_t stream);
+
+/*
+ * lmoe_forward_host -- lmoe_forward with HOST buffers: copies x_host (host,
+ * [T, d]) into library staging memory, runs the layer and copies the result
+ * to out_host (host, [T, d]), all enqueued on stream; the caller synchronises
+ * the stream before reading out_host.  Pinned host memory makes the copies
+ * asynchronous.  Errors: as lmoe_forward.
+ */
+lmoe_status lmoe_forward_host(lmoe_layer* h, const void* x_host, void* out_host, int T,
+                              lmoe_stream_t stream);
+
+/*
+ * lmoe_route_only -- the routing steps on given fp32 logits [T, N]
+ * (Section 3: the top-K set and the dispatch grouping):
+ *   idx[T, k]     experts of each token in slot order (logit desc, index asc;
+ *                 +0.0 == -0.0)
+ *   w[T, k]       renormalised gates exp(l_j - l_0) / sum_j' exp(l_j' - l_0)
+ *   offsets[N+1]  first expert-sorted row of each expert; offsets[N] = T*k
+ *   perm[T*k]     expert-sorted row -> pair t*k + j; within one expert rows
+ *                 are in ascending token order
+ * The same kernels lmoe_forward routes with.  Logits must be finite (with
+ * LMOE_DEBUG_CHECKS a non-finite logit sets LMOE_DEVERR_NONFINITE).
+ * Errors: NOT_READY (no workspace), INVALID_ARG.
+ */
+lmoe_status lmoe_route_only(lmoe_layer* h, const float* logits, int T, int* idx, float* w,
+                            int* offsets, int* perm, lmoe_stream_t stream);
+
+/*
+ * lmoe_router_logits -- the router GEMM alone: logits[T, N] (fp32) =
+ * x Wg + bias, computed by the kernel lmoe_forward uses (deterministic run to
+ * run).  Errors: NOT_READY, INVALID_ARG.
+ */
+lmoe_status lmoe_router_logits(lmoe_layer* h, const void* x, float* logits, int T,
+                               lmoe_stream_t stream);
+
+/* Intermediate buffers of the last lmoe_forward, for tests and debugging. */
+typedef enum {
+  LMOE_STAGE_LOGITS = 0,   /* [T, N]   fp32                                  */
+  LMOE_STAGE_IDX = 1,      /* [T, k]   int32                                 */
+  LMOE_STAGE_W = 2,        /* [T, k]   fp32                                  */
+  LMOE_STAGE_OFFSETS = 3,  /* [N+1]    int32                                 */
+  LMOE_STAGE_PERM = 4,     /* [T*k]    int32 sorted row -> t*k+j             */
+  LMOE_STAGE_Z = 5,        /* [T, l]   dtype  latent rows (not with SKIP)    */
+  LMOE_STAGE_H = 6,        /* [T*k, m] dtype  expert hidden rows, sorted     */
+  LMOE_STAGE_YS = 7,       /* [T*k, l] dtype  gate-scaled expert outputs,
+                                             in slot order t*k+j             */
+  LMOE_STAGE_COMB = 8      /* [T, l]   dtype  combined rows (not with SKIP)  */
+} lmoe_stage;
+
+/*
+ * lmoe_stage_bytes -- size in bytes of a stage buffer for T tokens.
+ * lmoe_debug_dump -- copy that buffer of the last forward (T of that call)
+ * into dst (device, at least lmoe_stage_bytes bytes), on stream.
+ * Errors: INVALID_ARG (unknown or absent stage, bytes too small), NOT_READY.
+ */
+lmoe_status lmoe_stage_bytes(const lmoe_layer* h, int stage, int T, size_t* bytes);
+lmoe_status lmoe_debug_dump(lmoe_layer* h, int stage, void* dst, size_t bytes,
+                            lmoe_stream_t stream);
+
+/*
+ * lmoe_last_error -- synchronise the device, read the device error word into
+ * *device_error_word (LMOE_DEVERR_* bits, 0 when clean) and clear it.
+ * Returns TIMEOUT or DEVICE when a bit was set, CUDA if the device itself
+ * reports an error, OK otherwise.
+ */
+lmoe_status lmoe_last_error(lmoe_layer* h, int* device_error_word);
+
+/*
+ * Per-stage timing.  lmoe_profile_begin allocates CUDA events for up to
+ * max_forwards calls (synchronous); afterwards every lmoe_forward records an
+ * event at each stage boundary on its stream.  lmoe_profile_end synchronises,
+ * writes the stage durations in milliseconds to ms[f * n_stages + s] for the
+ * recorded forwards f (at most capacity values), sets *n_forwards and
+ * *n_stages, and stops recording.  Stage s is named by lmoe_stage_name(s).
+ */
+lmoe_status lmoe_profile_begin(lmoe_layer* h, int max_forwards);
+lmoe_status lmoe_profile_end(lmoe_layer* h, float* ms, int capacity, int* n_forwards,
+                             int* n_stages);
+const char* lmoe_stage_name(int stage);
+
+/* Kernel launches the last lmoe_forward enqueued (library kernels only). */
+int lmoe_last_launch_count(const lmoe_layer* h);
+
+/* Which expert kernels the last lmoe_forward used: 0 CUDA-core, 1 tcgen05
+ * token-tiled, 2 tcgen05 weight-stationary (swap-AB). */
+int lmoe_last_expert_path(const lmoe_layer* h);
+
+const char* lmoe_status_string(lmoe_status s);
+
+/* Text of the last host-side failure on h (the failing CUDA call and its
+ * message); "" when none.  Valid until the next call on h. */
+const char* lmoe_error_detail(const lmoe_layer* h);
+
+/* Frees everything the handle owns (synchronises its device). NULL is a no-op. */
+void lmoe_destroy(lmoe_layer* h);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LMOE_H */

@@ -1,13 +1,7 @@
 """B200-native LatentMoE layer forward pass.
 
-``lmoe`` is the Python binding of the C-ABI library ``liblmoe.so`` (imported
-lazily so that the workload generator and the cost model load without it).
+Submodules: ``lmoe`` (Python binding of the C-ABI library ``liblmoe.so``),
+``build`` (compiles it for sm_100a), ``workloads`` (seeded synthetic inputs)
+and ``costmodel`` (the paper's roofline formulas and algorithmic counts).
+Import them explicitly, e.g. ``from mixture_experts_layer_64_b200 import lmoe``.
 """
-__all__ = ["lmoe", "workloads", "costmodel"]
-
-
-def __getattr__(name):
-    if name == "lmoe":
-        from . import lmoe
-        return lmoe
-    raise AttributeError(name)

@@ -106,3 +106,32 @@ def layer_counts(*, T: int, d: int, l: int, N: int, k: int, m: int, act: str,
                        fc2_bytes=fc2_bytes, expert_weight_bytes=w1 + w2,
                        intermediate_bytes=inter, touched=touched,
                        t_exp_mean=(R / touched) if touched else 0.0)
+
+
+def stage_counts(*, T: int, d: int, l: int, N: int, k: int, m: int, act: str,
+                 shared_m: int = 0, skip_proj: bool = False, elem_bytes: int = 2,
+                 loads: Optional[Sequence[int]] = None):
+    """Algorithmic (flops, bytes) of each launch stage of one forward pass:
+    every operand read once and every result written once; expert weights
+    only for touched experts.  Keys follow the library's stage names."""
+    m_in = 2 * m if act == "swiglu" else m
+    ms_in = 2 * shared_m if act == "swiglu" else shared_m
+    R = T * k
+    eb = elem_bytes
+    touched = N if loads is None else sum(1 for c in loads if c > 0)
+    kup = (0 if skip_proj else l) + shared_m
+    s = {
+        "router": (2.0 * T * d * N, T * d * eb + N * d * eb + T * N * 4.0),
+        "topk": (0.0, T * N * 4.0 + R * 8.0),
+        "group": (0.0, R * 4.0 * 4),
+        "down_proj": ((0.0, 0.0) if skip_proj else
+                      (2.0 * T * d * l, T * d * eb + d * l * eb + T * l * eb)),
+        "shared_fc1": ((0.0, 0.0) if not shared_m else
+                       (2.0 * T * d * ms_in, T * d * eb + d * ms_in * eb + T * shared_m * eb)),
+        "expert_fc1": (2.0 * R * l * m_in, touched * l * m_in * eb + T * l * eb + R * m * eb),
+        "expert_fc2": (2.0 * R * m * l, touched * m * l * eb + R * m * eb + R * l * eb),
+        "combine": (0.0, R * l * eb + T * l * eb + (T * d * eb if skip_proj else 0.0)),
+        "up_proj": ((0.0, 0.0) if kup == 0 else
+                    (2.0 * T * kup * d, T * kup * eb + kup * d * eb + 2.0 * T * d * eb)),
+    }
+    return s

@@ -1,0 +1,309 @@
+// Device helpers shared by the library's kernels: element types, activations,
+// the epilogue parameter block, and thin inline-PTX wrappers for mbarriers,
+// TMA (cp.async.bulk.tensor), cp.async and the tcgen05 tensor-core family of
+// sm_100a.  Every wait on an mbarrier is bounded by wall time (globaltimer);
+// on expiry it sets LMOE_DEVERR_WAIT_TIMEOUT in the device error word and
+// reports failure so that the kernel can unwind instead of hanging.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/lmoe.h"
+
+namespace lmoe {
+
+typedef __nv_bfloat16 bf16;
+
+enum EpiKind {
+  EPI_F32_BIAS = 0,      // out_f32[r, f] = acc + bias[f]                      (router)
+  EPI_ACT = 1,           // out[r, col0 + f] = act(acc) / swiglu(acc0, acc1)  (FC1, down-proj)
+  EPI_SCALE_SCATTER = 2, // out[row_slot[r], f] = row_w[r] * acc               (expert FC2)
+  EPI_RESID = 3          // out[r, f] = resid[r, f] + acc                      (up-projection)
+};
+enum ActKind { ACT_NONE = -1, ACT_SILU = 0, ACT_SWIGLU = 1, ACT_RELU2 = 2 };
+
+// Where a GEMM writes and what its epilogue mixes in.
+struct EpiParams {
+  void* out;              // output base (fp32 for EPI_F32_BIAS, else the layer dtype)
+  long ldo;               // output row stride (elements)
+  int col0;               // first output column written (EPI_ACT)
+  int act;                // ActKind for EPI_ACT
+  const float* bias;      // EPI_F32_BIAS, may be NULL
+  const void* resid;      // EPI_RESID, row stride ldr
+  long ldr;
+  const int* row_slot;    // EPI_SCALE_SCATTER: tile row -> output row
+  const float* row_w;     // EPI_SCALE_SCATTER: tile row -> gate weight
+};
+
+// A (possibly grouped) problem D[r, f] = sum_k A[src(r), k] * B[wrow(g, f), k]
+// over the row groups [offsets[g], offsets[g+1]).  Rows are handled in tiles
+// of 128 that never straddle a group; tile_prefix[g] counts the row tiles of
+// the groups before g.  Without offsets the problem is one dense group of M
+// rows.  Weights are K-major: group g's feature f lives in row
+// g * w_group_stride + f of B (for gated FC1 the linear half starts m rows
+// later: f + dual_offset).
+struct GemmProblem {
+  const int* offsets;     // [G+1] device, or NULL for one dense group
+  const int* tile_prefix; // [G+1] device (with offsets)
+  int G;
+  int M;                  // rows of the dense group (offsets == NULL)
+  int max_row_tiles;      // host upper bound on row tiles (grid sizing)
+  const void* A;          // activations, row stride lda
+  long lda;
+  const int* gather;      // row -> source row of A, or NULL (identity)
+  const void* B;          // K-major weights, row stride K
+  long w_group_stride;
+  int dual_offset;        // > 0: gated (two accumulators: f and f + dual_offset)
+  int F;                  // output features
+  int K;                  // reduction length
+  EpiParams epi;
+  int* err;               // device error word
+};
+
+constexpr int kRowTile = 128;
+
+// ---- scalar helpers ---------------------------------------------------------
+
+template <typename T> __device__ __forceinline__ float to_f32(T v);
+template <> __device__ __forceinline__ float to_f32<float>(float v) { return v; }
+template <> __device__ __forceinline__ float to_f32<bf16>(bf16 v) { return __bfloat162float(v); }
+
+template <typename T> __device__ __forceinline__ T from_f32(float v);
+template <> __device__ __forceinline__ float from_f32<float>(float v) { return v; }
+template <> __device__ __forceinline__ bf16 from_f32<bf16>(float v) { return __float2bfloat16_rn(v); }
+
+__device__ __forceinline__ float silu_f(float a) { return a / (1.0f + expf(-a)); }
+
+// act of one output feature; g is the gate (or only) pre-activation and u
+// the linear half for SwiGLU.
+__device__ __forceinline__ float apply_act(int act, float g, float u) {
+  switch (act) {
+    case ACT_SILU: return silu_f(g);
+    case ACT_SWIGLU: return silu_f(g) * u;
+    case ACT_RELU2: return g > 0.0f ? g * g : 0.0f;
+    default: return g;
+  }
+}
+
+// Locates row tile `rt` in a grouped problem: group g, first row and rows.
+__device__ __forceinline__ void locate_row_tile(const GemmProblem& p, int rt, int& g, int& row0,
+                                                int& rows) {
+  if (p.offsets == nullptr) {
+    g = 0;
+    row0 = rt * kRowTile;
+    rows = min(kRowTile, p.M - row0);
+    return;
+  }
+  int lo = 0, hi = p.G - 1;  // largest g with tile_prefix[g] <= rt
+  while (lo < hi) {
+    int mid = (lo + hi + 1) >> 1;
+    if (__ldg(p.tile_prefix + mid) <= rt) lo = mid; else hi = mid - 1;
+  }
+  g = lo;
+  const int start = __ldg(p.offsets + g), end = __ldg(p.offsets + g + 1);
+  row0 = start + (rt - __ldg(p.tile_prefix + g)) * kRowTile;
+  rows = min(kRowTile, end - row0);
+}
+
+__device__ __forceinline__ int total_row_tiles(const GemmProblem& p) {
+  if (p.offsets == nullptr) return (p.M + kRowTile - 1) / kRowTile;
+  return *((volatile const int*)(p.tile_prefix + p.G));
+}
+
+__device__ __forceinline__ void set_error(int* err, int bits) {
+  if (err) atomicOr(err, bits);
+}
+
+// ---- PTX wrappers -----------------------------------------------------------
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t globaltimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
+               : "memory");
+}
+
+__device__ __forceinline__ void fence_barrier_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Wall-time limit of one mbarrier wait (ns).  No legitimate wait in these
+// kernels lasts more than a few milliseconds.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+// Bounded wait on `bar` reaching phase parity `parity`.  Returns false (after
+// flagging the error word and the block-wide abort flag) on expiry, or
+// immediately when another thread of the block has already aborted.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                          int* err) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 255u) == 0) {
+      if (*abort_flag) return false;
+      if (globaltimer() - t0 > kWaitLimitNs) {
+        *abort_flag = 1;
+        set_error(err, LMOE_DEVERR_WAIT_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+
+// Bounded wait that ignores the abort flag: used while draining in-flight
+// asynchronous work before the block exits.
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer();
+  for (uint32_t it = 0;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 255u) == 255u && globaltimer() - t0 > kWaitLimitNs) return false;
+  }
+}
+
+__device__ __forceinline__ void tma_load_2d(const CUtensorMap* map, uint64_t* bar, void* smem_dst,
+                                            int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
+      : "memory");
+}
+
+__device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// 16-byte cp.async with zero fill of the (16 - src_bytes) tail.
+__device__ __forceinline__ void cp_async_16(void* smem_dst, const void* gsrc, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem_dst)),
+               "l"(gsrc), "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// tcgen05 (5th-generation tensor cores, tensor memory).
+__device__ __forceinline__ void tmem_alloc(uint32_t* smem_slot, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                   smem_u32(smem_slot)),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+// D(tmem) (+)= A(smem desc) * B(smem desc)^T, bf16 inputs, fp32 accumulate.
+__device__ __forceinline__ void tc_mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Arrive on `bar` once all previously issued tcgen05.mma of this thread finish.
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+__device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// 32 lanes x 32 consecutive fp32 columns: thread i of the warp receives lane
+// (taddr.lane + i), columns [taddr.col, taddr.col + 32).
+__device__ __forceinline__ void tmem_ld_32x32(uint32_t taddr, float* v) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Shared-memory matrix descriptor of a K-major operand tile written with the
+// 128-byte swizzle (rows of 64 bf16 = 128 B, 8-row atoms of 1024 B): start
+// address, leading-byte offset 16 B (unused for swizzled K-major), stride
+// byte offset 1024 B between 8-row groups, descriptor version 1 (sm_100),
+// layout type 2 = SWIZZLE_128B.
+__device__ __forceinline__ uint64_t smem_desc_sw128(const void* smem_tile) {
+  const uint64_t addr = smem_u32(smem_tile);
+  uint64_t desc = 0;
+  desc |= (addr >> 4) & 0x3FFFull;            // bits [0,14)  start address >> 4
+  desc |= (uint64_t)(16 >> 4) << 16;          // bits [16,30) leading byte offset >> 4
+  desc |= (uint64_t)(1024 >> 4) << 32;        // bits [32,46) stride byte offset >> 4
+  desc |= (uint64_t)1 << 46;                  // bits [46,48) version = 1
+  desc |= (uint64_t)2 << 61;                  // bits [61,64) SWIZZLE_128B
+  return desc;
+}
+
+// Instruction descriptor of tcgen05.mma kind::f16: bf16 A and B, fp32 D,
+// both operands K-major, shape M x N.
+__device__ __forceinline__ uint32_t idesc_bf16_f32(int M, int N) {
+  uint32_t d = 0;
+  d |= 1u << 4;                       // D format: F32
+  d |= 1u << 7;                       // A format: BF16
+  d |= 1u << 10;                      // B format: BF16
+  d |= (uint32_t)(N >> 3) << 17;      // N >> 3
+  d |= (uint32_t)(M >> 4) << 24;      // M >> 4
+  return d;
+}
+
+}  // namespace lmoe

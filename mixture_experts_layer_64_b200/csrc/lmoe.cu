@@ -1,0 +1,826 @@
+// Host side of the LatentMoE layer library: the handle, weight repack,
+// workspace, per-call kernel selection and the C ABI declared in lmoe.h.
+//
+// One forward pass (LatentMoE paper, Section 3, Eq. (1)/(2), plus the
+// residual add) is this sequence of launches on the caller's stream:
+//   1 router GEMM            logits[T,N] fp32 = x Wg + bias
+//   2 top-k + softmax        idx, w, per-expert token bitmaps
+//   3 grouping               word prefixes, offsets, tile counts; sorted rows
+//   4 down-projection GEMM   z[T,l] = x Wdown                 (not when skipped)
+//   5 shared FC1 GEMM        hs = act(x Ws1) into cat[:, l:]  (with a shared expert)
+//   6 expert FC1 (grouped)   h[r] = act(z[tok(r)] W1[e])      rows gathered by token
+//   7 expert FC2 (grouped)   ys[slot(r)] = w(r) * (h[r] W2[e])
+//   8 combine                cat[t, :l] = sum_j ys[t*k + j]   (or out = x + sum, skipped)
+//   9 up-projection GEMM     out = x + [comb | hs] [Wup ; Ws2]
+// Contractions run on the tcgen05 kernel (bf16) or the CUDA-core kernel
+// (fp32, or shapes the tcgen05 kernel does not take).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "../../include/lmoe.h"
+#include "common.cuh"
+#include "misc.cuh"
+#include "routing.cuh"
+#include "simt_gemm.cuh"
+#include "tc_gemm.cuh"
+
+using namespace lmoe;
+
+namespace {
+
+constexpr int kStages = 9;  // profiled stage count (10 boundaries)
+const char* kStageNames[kStages] = {"router",     "topk",       "group",   "down_proj", "shared_fc1",
+                                    "expert_fc1", "expert_fc2", "combine", "up_proj"};
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+}  // namespace
+
+struct lmoe_layer {
+  int d, l, N, k, m, act, shared_m, dtype;
+  unsigned flags;
+  int m_in, ms_in, Kup, es;  // es: element size
+  int device = 0, num_sms = 148;
+  bool weights_set = false;
+  // weights, K-major
+  void* Wg_t = nullptr;   // [N, d]
+  float* bias = nullptr;  // [N]
+  void* Wd_t = nullptr;   // [l, d]
+  void* Wu_t = nullptr;   // [d, Kup]: [Wup^T | Ws2^T]
+  void* Ws1_t = nullptr;  // [ms_in, d]
+  void* W1_t = nullptr;   // [N * m_in, l]
+  void* W2_t = nullptr;   // [N * l, m]
+  // workspace
+  int max_T = 0, W = 0;
+  float* logits = nullptr;
+  int* idx = nullptr;
+  float* w = nullptr;
+  uint32_t* bitmap = nullptr;
+  uint2* wp = nullptr;
+  int *counts = nullptr, *offsets = nullptr, *tile_prefix = nullptr;
+  unsigned* done = nullptr;
+  int* err = nullptr;
+  int *row_tok = nullptr, *row_slot = nullptr;
+  float* row_w = nullptr;
+  void *z = nullptr, *h = nullptr, *ys = nullptr, *cat = nullptr;
+  void *x_stage = nullptr, *out_stage = nullptr;
+  // bookkeeping
+  int last_T = -1, launches = 0, expert_path = -1;
+  std::string detail;
+  // profiling
+  std::vector<cudaEvent_t> events;
+  int prof_cap = 0, prof_count = 0;
+  bool profiling = false;
+};
+
+namespace {
+
+struct DevGuard {
+  int prev = -1;
+  bool changed = false;
+  explicit DevGuard(int dev) {
+    if (cudaGetDevice(&prev) == cudaSuccess && prev != dev) {
+      changed = cudaSetDevice(dev) == cudaSuccess;
+    }
+  }
+  ~DevGuard() {
+    if (changed) cudaSetDevice(prev);
+  }
+};
+
+lmoe_status cuda_fail(lmoe_layer* h, cudaError_t e, const char* what) {
+  if (h) h->detail = std::string(what) + ": " + cudaGetErrorString(e);
+  return e == cudaErrorMemoryAllocation ? LMOE_ERR_OOM : LMOE_ERR_CUDA;
+}
+
+#define LMOE_CUDA(h, call)                                 \
+  do {                                                     \
+    cudaError_t e_ = (call);                               \
+    if (e_ != cudaSuccess) return cuda_fail((h), e_, #call); \
+  } while (0)
+
+#define LMOE_CHECK_LAUNCH(h)                                           \
+  do {                                                                 \
+    cudaError_t e_ = cudaGetLastError();                               \
+    if (e_ != cudaSuccess) return cuda_fail((h), e_, "kernel launch"); \
+    ++(h)->launches;                                                   \
+  } while (0)
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+// ---- GEMM dispatch --------------------------------------------------------------
+
+enum GemmKind { GK_ROUTER, GK_DENSE_ACT, GK_FC1, GK_FC2, GK_UP };
+
+struct GemmCall {
+  GemmProblem p;
+  GemmKind kind;
+  long a_rows;  // rows of A (TMA bounds)
+  long b_rows;  // rows of B (TMA bounds)
+  bool swap;    // weight-stationary expert kernels
+};
+
+bool encode_map(CUtensorMap* map, const void* ptr, long rows, int cols, long ld, int box_rows) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <class Cfg>
+lmoe_status launch_tc(lmoe_layer* h, const GemmCall& c, cudaStream_t st) {
+  static bool attr_done = false;
+  if (!attr_done) {
+    LMOE_CUDA(h, cudaFuncSetAttribute(tc_gemm_kernel<Cfg>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      Cfg::SMEM_BYTES));
+    attr_done = true;
+  }
+  CUtensorMap ta, tb;
+  std::memset(&ta, 0, sizeof ta);
+  std::memset(&tb, 0, sizeof tb);
+  if (!Cfg::kGather &&
+      !encode_map(&ta, c.p.A, c.a_rows, c.p.K, c.p.lda, Cfg::kSwap ? 32 : 128)) {
+    h->detail = "cuTensorMapEncodeTiled (activations) failed";
+    return LMOE_ERR_CUDA;
+  }
+  if (!encode_map(&tb, c.p.B, c.b_rows, c.p.K, c.p.K, Cfg::W_ROWS)) {
+    h->detail = "cuTensorMapEncodeTiled (weights) failed";
+    return LMOE_ERR_CUDA;
+  }
+  const long NT = (c.p.F + Cfg::FT - 1) / Cfg::FT;
+  const long tiles = (long)c.p.max_row_tiles * NT;
+  const int grid = (int)std::max(1L, std::min<long>(h->num_sms, tiles));
+  tc_gemm_kernel<Cfg><<<grid, kTcThreads, Cfg::SMEM_BYTES, st>>>(ta, tb, c.p);
+  LMOE_CHECK_LAUNCH(h);
+  return LMOE_OK;
+}
+
+template <typename T, bool kDual, int kEpi>
+lmoe_status launch_simt(lmoe_layer* h, const GemmCall& c, cudaStream_t st) {
+  const long NT = (c.p.F + kSimtTN - 1) / kSimtTN;
+  const long blocks = (long)c.p.max_row_tiles * NT;
+  if (blocks <= 0) return LMOE_OK;
+  simt_gemm_kernel<T, kDual, kEpi><<<(unsigned)blocks, 256, 0, st>>>(c.p);
+  LMOE_CHECK_LAUNCH(h);
+  return LMOE_OK;
+}
+
+template <typename T>
+lmoe_status dispatch_simt(lmoe_layer* h, const GemmCall& c, cudaStream_t st) {
+  const bool dual = c.p.dual_offset > 0;
+  switch (c.kind) {
+    case GK_ROUTER: return launch_simt<T, false, EPI_F32_BIAS>(h, c, st);
+    case GK_DENSE_ACT:
+    case GK_FC1:
+      return dual ? launch_simt<T, true, EPI_ACT>(h, c, st) : launch_simt<T, false, EPI_ACT>(h, c, st);
+    case GK_FC2: return launch_simt<T, false, EPI_SCALE_SCATTER>(h, c, st);
+    case GK_UP: return launch_simt<T, false, EPI_RESID>(h, c, st);
+  }
+  return LMOE_ERR_INVALID_ARG;
+}
+
+// Whether the tcgen05 kernel can take this call: bf16, K a multiple of 64,
+// 16-byte aligned rows for TMA / cp.async and for the vector epilogue.
+bool tc_eligible(const lmoe_layer* h, const GemmCall& c) {
+  if (h->dtype != LMOE_BF16 || (h->flags & LMOE_FORCE_SIMT)) return false;
+  const GemmProblem& p = c.p;
+  if (p.K % 64 != 0 || p.K <= 0) return false;
+  if (p.lda % 8 != 0 || !aligned16(p.A) || !aligned16(p.B)) return false;
+  if (c.kind == GK_ROUTER) {
+    if (p.epi.ldo % 4 != 0 || !aligned16(p.epi.out)) return false;
+  } else {
+    if (p.epi.ldo % 8 != 0 || p.epi.col0 % 8 != 0 || !aligned16(p.epi.out)) return false;
+  }
+  if (c.kind == GK_UP && (p.epi.ldr % 8 != 0 || !aligned16(p.epi.resid))) return false;
+  return true;
+}
+
+lmoe_status run_gemm(lmoe_layer* h, GemmCall c, cudaStream_t st, int* path = nullptr) {
+  c.p.err = h->err;
+  if (!tc_eligible(h, c)) {
+    if (path) *path = 0;
+    return h->dtype == LMOE_F32 ? dispatch_simt<float>(h, c, st) : dispatch_simt<bf16>(h, c, st);
+  }
+  const bool dual = c.p.dual_offset > 0;
+  if (path) *path = c.swap ? 2 : 1;
+  switch (c.kind) {
+    case GK_ROUTER: return launch_tc<TcCfg<false, false, false, 128, EPI_F32_BIAS>>(h, c, st);
+    case GK_DENSE_ACT:
+      return dual ? launch_tc<TcCfg<false, false, true, 128, EPI_ACT>>(h, c, st)
+                  : launch_tc<TcCfg<false, false, false, 256, EPI_ACT>>(h, c, st);
+    case GK_FC1:
+      if (c.swap)
+        return dual ? launch_tc<TcCfg<true, true, true, 128, EPI_ACT>>(h, c, st)
+                    : launch_tc<TcCfg<true, true, false, 128, EPI_ACT>>(h, c, st);
+      return dual ? launch_tc<TcCfg<false, true, true, 128, EPI_ACT>>(h, c, st)
+                  : launch_tc<TcCfg<false, true, false, 256, EPI_ACT>>(h, c, st);
+    case GK_FC2:
+      return c.swap ? launch_tc<TcCfg<true, false, false, 128, EPI_SCALE_SCATTER>>(h, c, st)
+                    : launch_tc<TcCfg<false, false, false, 256, EPI_SCALE_SCATTER>>(h, c, st);
+    case GK_UP: return launch_tc<TcCfg<false, false, false, 256, EPI_RESID>>(h, c, st);
+  }
+  return LMOE_ERR_INVALID_ARG;
+}
+
+GemmCall dense_call(GemmKind kind, int M, const void* A, long lda, const void* B, int F, int K) {
+  GemmCall c;
+  std::memset(&c, 0, sizeof c);
+  c.kind = kind;
+  c.p.M = M;
+  c.p.G = 1;
+  c.p.max_row_tiles = (M + kRowTile - 1) / kRowTile;
+  c.p.A = A;
+  c.p.lda = lda;
+  c.p.B = B;
+  c.p.F = F;
+  c.p.K = K;
+  c.a_rows = M;
+  c.b_rows = F;
+  c.p.epi.act = ACT_NONE;
+  return c;
+}
+
+GemmCall grouped_call(const lmoe_layer* h, GemmKind kind, int T, const void* A, long lda,
+                      long a_rows, const int* gather, const void* B, long stride, int F, int K) {
+  GemmCall c;
+  std::memset(&c, 0, sizeof c);
+  const long R = (long)T * h->k;
+  c.kind = kind;
+  c.p.offsets = h->offsets;
+  c.p.tile_prefix = h->tile_prefix;
+  c.p.G = h->N;
+  c.p.max_row_tiles = (int)((R + kRowTile - 1) / kRowTile + h->N);
+  c.p.A = A;
+  c.p.lda = lda;
+  c.p.gather = gather;
+  c.p.B = B;
+  c.p.w_group_stride = stride;
+  c.p.F = F;
+  c.p.K = K;
+  c.a_rows = a_rows;
+  c.b_rows = (long)h->N * stride;
+  c.p.epi.act = ACT_NONE;
+  return c;
+}
+
+bool use_swap(const lmoe_layer* h, int T) {
+  if (h->flags & LMOE_FORCE_SWAP) return true;
+  if (h->flags & LMOE_FORCE_NOSWAP) return false;
+  return (long)T * h->k < 64L * h->N;  // fewer than 64 rows per expert on average
+}
+
+void prof_mark(lmoe_layer* h, cudaStream_t st, int i) {
+  if (h->profiling && h->prof_count < h->prof_cap)
+    cudaEventRecord(h->events[(size_t)h->prof_count * (kStages + 1) + i], st);
+}
+
+// ---- the routing steps ---------------------------------------------------------
+
+lmoe_status run_routing(lmoe_layer* h, const float* logits, int T, int* idx, float* w,
+                        int* offsets, int* row_tok, int* row_slot, float* row_w, cudaStream_t st,
+                        bool marks) {
+  const int W = (T + 31) / 32;
+  const int debug = (h->flags & LMOE_DEBUG_CHECKS) ? 1 : 0;
+  topk_softmax_kernel<<<(T + 7) / 8, 256, 0, st>>>(logits, T, h->N, h->k, idx, w, h->bitmap, W,
+                                                   debug, h->err);
+  LMOE_CHECK_LAUNCH(h);
+  if (marks) prof_mark(h, st, 2);
+  group_count_kernel<<<(h->N + 7) / 8, 256, 0, st>>>(h->bitmap, h->wp, h->N, W, h->counts, offsets,
+                                                     h->tile_prefix, h->done);
+  LMOE_CHECK_LAUNCH(h);
+  const long P = (long)T * h->k;
+  group_rank_kernel<<<(unsigned)((P + 255) / 256), 256, 0, st>>>(
+      idx, w, h->wp, offsets, T, h->k, h->N, W, row_tok, row_slot, row_w, debug, h->err);
+  LMOE_CHECK_LAUNCH(h);
+  return LMOE_OK;
+}
+
+lmoe_status run_router(lmoe_layer* h, const void* x, float* logits, int T, cudaStream_t st) {
+  GemmCall c = dense_call(GK_ROUTER, T, x, h->d, h->Wg_t, h->N, h->d);
+  c.p.epi.out = logits;
+  c.p.epi.ldo = h->N;
+  c.p.epi.bias = h->bias;
+  return run_gemm(h, c, st);
+}
+
+#define LMOE_TRY(expr)               \
+  do {                               \
+    lmoe_status s_ = (expr);         \
+    if (s_ != LMOE_OK) return s_;    \
+  } while (0)
+
+lmoe_status run_forward(lmoe_layer* h, const void* x, void* out, int T, cudaStream_t st) {
+  h->launches = 0;
+  const bool skip = (h->flags & LMOE_SKIP_PROJ) != 0;
+  const int d = h->d, l = h->l, k = h->k, m = h->m, ms = h->shared_m;
+  const long R = (long)T * k;
+  prof_mark(h, st, 0);
+  LMOE_TRY(run_router(h, x, h->logits, T, st));
+  prof_mark(h, st, 1);
+  LMOE_TRY(run_routing(h, h->logits, T, h->idx, h->w, h->offsets, h->row_tok, h->row_slot,
+                       h->row_w, st, true));
+  prof_mark(h, st, 3);
+  if (!skip) {
+    GemmCall c = dense_call(GK_DENSE_ACT, T, x, d, h->Wd_t, l, d);
+    c.p.epi.out = h->z;
+    c.p.epi.ldo = l;
+    LMOE_TRY(run_gemm(h, c, st));
+  }
+  prof_mark(h, st, 4);
+  if (ms > 0) {
+    GemmCall c = dense_call(GK_DENSE_ACT, T, x, d, h->Ws1_t, ms, d);
+    c.b_rows = h->ms_in;
+    c.p.dual_offset = h->act == LMOE_ACT_SWIGLU ? ms : 0;
+    c.p.epi.out = h->cat;
+    c.p.epi.ldo = h->Kup;
+    c.p.epi.col0 = skip ? 0 : l;
+    c.p.epi.act = h->act;
+    LMOE_TRY(run_gemm(h, c, st));
+  }
+  prof_mark(h, st, 5);
+  const bool swap = use_swap(h, T);
+  {
+    const void* A = skip ? x : h->z;
+    GemmCall c = grouped_call(h, GK_FC1, T, A, skip ? d : l, T, h->row_tok, h->W1_t, h->m_in, m, l);
+    c.swap = swap;
+    c.p.dual_offset = h->act == LMOE_ACT_SWIGLU ? m : 0;
+    c.p.epi.out = h->h;
+    c.p.epi.ldo = m;
+    c.p.epi.act = h->act;
+    int path = 0;
+    LMOE_TRY(run_gemm(h, c, st, &path));
+    h->expert_path = path;
+  }
+  prof_mark(h, st, 6);
+  {
+    GemmCall c = grouped_call(h, GK_FC2, T, h->h, m, R, nullptr, h->W2_t, l, l, m);
+    c.swap = swap;
+    c.p.epi.out = h->ys;
+    c.p.epi.ldo = l;
+    c.p.epi.row_slot = h->row_slot;
+    c.p.epi.row_w = h->row_w;
+    LMOE_TRY(run_gemm(h, c, st));
+  }
+  prof_mark(h, st, 7);
+  {
+    const void* resid = skip ? x : nullptr;
+    void* dst = skip ? out : h->cat;
+    const long ldo = skip ? d : h->Kup;
+    const int vec = 16 / h->es;
+    const bool vec_ok = (l % vec == 0) && (ldo % vec == 0) && aligned16(dst) && aligned16(h->ys) &&
+                        (!resid || (aligned16(resid) && d % vec == 0));
+    const int threads = std::min(256, std::max(32, (l / vec + 31) / 32 * 32));
+    if (h->dtype == LMOE_BF16) {
+      if (vec_ok)
+        combine_kernel<bf16><<<T, threads, 0, st>>>((const bf16*)h->ys, k, l, (const bf16*)resid,
+                                                    d, (bf16*)dst, ldo);
+      else
+        combine_scalar_kernel<bf16><<<T, 256, 0, st>>>((const bf16*)h->ys, k, l,
+                                                       (const bf16*)resid, d, (bf16*)dst, ldo);
+    } else {
+      if (vec_ok)
+        combine_kernel<float><<<T, threads, 0, st>>>((const float*)h->ys, k, l,
+                                                     (const float*)resid, d, (float*)dst, ldo);
+      else
+        combine_scalar_kernel<float><<<T, 256, 0, st>>>((const float*)h->ys, k, l,
+                                                        (const float*)resid, d, (float*)dst, ldo);
+    }
+    LMOE_CHECK_LAUNCH(h);
+  }
+  prof_mark(h, st, 8);
+  if (!skip || ms > 0) {
+    GemmCall c = dense_call(GK_UP, T, h->cat, h->Kup, h->Wu_t, d, h->Kup);
+    c.p.epi.out = out;
+    c.p.epi.ldo = d;
+    c.p.epi.resid = skip ? out : x;  // skipped projections: out already holds x + comb
+    c.p.epi.ldr = d;
+    LMOE_TRY(run_gemm(h, c, st));
+  }
+  prof_mark(h, st, 9);
+  if (h->profiling && h->prof_count < h->prof_cap) ++h->prof_count;
+  h->last_T = T;
+  return LMOE_OK;
+}
+
+template <typename T>
+void free_ptr(T*& p) {
+  if (p) cudaFree((void*)p);
+  p = nullptr;
+}
+
+void free_workspace(lmoe_layer* h) {
+  free_ptr(h->logits);
+  free_ptr(h->idx);
+  free_ptr(h->w);
+  free_ptr(h->bitmap);
+  free_ptr(h->wp);
+  free_ptr(h->counts);
+  free_ptr(h->offsets);
+  free_ptr(h->tile_prefix);
+  free_ptr(h->done);
+  free_ptr(h->err);
+  free_ptr(h->row_tok);
+  free_ptr(h->row_slot);
+  free_ptr(h->row_w);
+  free_ptr(h->z);
+  free_ptr(h->h);
+  free_ptr(h->ys);
+  free_ptr(h->cat);
+  free_ptr(h->x_stage);
+  free_ptr(h->out_stage);
+  h->max_T = 0;
+}
+
+void free_weights(lmoe_layer* h) {
+  free_ptr(h->Wg_t);
+  free_ptr(h->bias);
+  free_ptr(h->Wd_t);
+  free_ptr(h->Wu_t);
+  free_ptr(h->Ws1_t);
+  free_ptr(h->W1_t);
+  free_ptr(h->W2_t);
+  h->weights_set = false;
+}
+
+void destroy_events(lmoe_layer* h) {
+  for (cudaEvent_t e : h->events) cudaEventDestroy(e);
+  h->events.clear();
+  h->prof_cap = h->prof_count = 0;
+  h->profiling = false;
+}
+
+// API layout [batch][rows][cols] -> K-major [batch][cols][col0 + rows] (row stride ldo).
+lmoe_status repack(lmoe_layer* h, const void* in, int rows, int cols, int batch, void* out, long ldo,
+                   int col0) {
+  dim3 grid((cols + 31) / 32, (rows + 31) / 32, batch), block(32, 8);
+  const long ib = (long)rows * cols, ob = (long)cols * ldo;
+  if (h->dtype == LMOE_BF16)
+    transpose_kernel<bf16><<<grid, block>>>((const bf16*)in, rows, cols, ib, (bf16*)out, ldo, col0, ob);
+  else
+    transpose_kernel<float><<<grid, block>>>((const float*)in, rows, cols, ib, (float*)out, ldo, col0,
+                                             ob);
+  LMOE_CUDA(h, cudaGetLastError());
+  return LMOE_OK;
+}
+
+bool valid_stream_call(const lmoe_layer* h, int T) { return h && T >= 0 && T <= h->max_T; }
+
+}  // namespace
+
+// ================================== C ABI ==================================
+
+extern "C" {
+
+const char* lmoe_status_string(lmoe_status s) {
+  switch (s) {
+    case LMOE_OK: return "ok";
+    case LMOE_ERR_INVALID_ARG: return "invalid argument";
+    case LMOE_ERR_NOT_READY: return "not ready (weights not set or workspace not reserved)";
+    case LMOE_ERR_CUDA: return "CUDA error";
+    case LMOE_ERR_OOM: return "out of device memory";
+    case LMOE_ERR_TIMEOUT: return "device-side wait timed out";
+    case LMOE_ERR_UNSUPPORTED: return "unsupported configuration";
+    case LMOE_ERR_DEVICE: return "device-side check failed";
+  }
+  return "unknown status";
+}
+
+const char* lmoe_stage_name(int stage) {
+  return (stage >= 0 && stage < kStages) ? kStageNames[stage] : "";
+}
+
+const char* lmoe_error_detail(const lmoe_layer* h) { return h ? h->detail.c_str() : ""; }
+
+lmoe_status lmoe_create(int d, int l, int N, int k, int m, lmoe_act act, int shared_m,
+                        lmoe_dtype dtype, unsigned flags, lmoe_layer** out) {
+  if (!out) return LMOE_ERR_INVALID_ARG;
+  *out = nullptr;
+  const unsigned known = LMOE_SKIP_PROJ | LMOE_DEBUG_CHECKS | LMOE_FORCE_SIMT | LMOE_FORCE_SWAP |
+                         LMOE_FORCE_NOSWAP;
+  if (d <= 0 || l <= 0 || N <= 0 || k <= 0 || m <= 0 || shared_m < 0) return LMOE_ERR_INVALID_ARG;
+  if (k > N || (flags & ~known)) return LMOE_ERR_INVALID_ARG;
+  if (act != LMOE_ACT_SILU && act != LMOE_ACT_SWIGLU && act != LMOE_ACT_RELU2) return LMOE_ERR_INVALID_ARG;
+  if (dtype != LMOE_F32 && dtype != LMOE_BF16) return LMOE_ERR_INVALID_ARG;
+  if ((flags & LMOE_SKIP_PROJ) && l != d) return LMOE_ERR_INVALID_ARG;
+  if ((flags & LMOE_FORCE_SWAP) && (flags & LMOE_FORCE_NOSWAP)) return LMOE_ERR_INVALID_ARG;
+  if (N > LMOE_MAX_EXPERTS || k > LMOE_MAX_TOPK) return LMOE_ERR_UNSUPPORTED;
+  // 32-bit row and element indices inside the kernels
+  if ((long)N * (2L * m) * l >= (1L << 31) * 8L) return LMOE_ERR_UNSUPPORTED;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return LMOE_ERR_CUDA;
+  lmoe_layer* h = new lmoe_layer();
+  h->d = d; h->l = l; h->N = N; h->k = k; h->m = m; h->act = act; h->shared_m = shared_m;
+  h->dtype = dtype; h->flags = flags;
+  h->m_in = act == LMOE_ACT_SWIGLU ? 2 * m : m;
+  h->ms_in = act == LMOE_ACT_SWIGLU ? 2 * shared_m : shared_m;
+  h->Kup = ((flags & LMOE_SKIP_PROJ) ? 0 : l) + shared_m;
+  h->es = dtype == LMOE_BF16 ? 2 : 4;
+  h->device = dev;
+  int sms = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && sms > 0)
+    h->num_sms = sms;
+  *out = h;
+  return LMOE_OK;
+}
+
+lmoe_status lmoe_set_weights(lmoe_layer* h, const void* W_g, const float* bias, const void* W_down,
+                             const void* W_up, const void* W1, const void* W2, const void* Ws1,
+                             const void* Ws2) {
+  if (!h || !W_g || !W1 || !W2) return LMOE_ERR_INVALID_ARG;
+  const bool skip = (h->flags & LMOE_SKIP_PROJ) != 0;
+  if (skip != (W_down == nullptr) || skip != (W_up == nullptr)) return LMOE_ERR_INVALID_ARG;
+  if ((h->shared_m > 0) != (Ws1 != nullptr) || (h->shared_m > 0) != (Ws2 != nullptr))
+    return LMOE_ERR_INVALID_ARG;
+  DevGuard g(h->device);
+  LMOE_CUDA(h, cudaDeviceSynchronize());
+  const size_t es = h->es;
+  const int d = h->d, l = h->l, N = h->N, m = h->m;
+  if (!h->weights_set) {
+    LMOE_CUDA(h, cudaMalloc(&h->Wg_t, (size_t)N * d * es));
+    LMOE_CUDA(h, cudaMalloc(&h->W1_t, (size_t)N * h->m_in * l * es));
+    LMOE_CUDA(h, cudaMalloc(&h->W2_t, (size_t)N * l * m * es));
+    if (!skip) LMOE_CUDA(h, cudaMalloc(&h->Wd_t, (size_t)l * d * es));
+    if (h->Kup > 0) LMOE_CUDA(h, cudaMalloc(&h->Wu_t, (size_t)d * h->Kup * es));
+    if (h->shared_m > 0) LMOE_CUDA(h, cudaMalloc(&h->Ws1_t, (size_t)h->ms_in * d * es));
+  }
+  free_ptr(h->bias);
+  if (bias) {
+    LMOE_CUDA(h, cudaMalloc(&h->bias, (size_t)N * sizeof(float)));
+    LMOE_CUDA(h, cudaMemcpy(h->bias, bias, (size_t)N * sizeof(float), cudaMemcpyDeviceToDevice));
+  }
+  LMOE_TRY(repack(h, W_g, d, N, 1, h->Wg_t, d, 0));
+  LMOE_TRY(repack(h, W1, l, h->m_in, N, h->W1_t, l, 0));
+  LMOE_TRY(repack(h, W2, m, l, N, h->W2_t, m, 0));
+  if (!skip) {
+    LMOE_TRY(repack(h, W_down, d, l, 1, h->Wd_t, d, 0));
+    LMOE_TRY(repack(h, W_up, l, d, 1, h->Wu_t, h->Kup, 0));
+  }
+  if (h->shared_m > 0) {
+    LMOE_TRY(repack(h, Ws1, d, h->ms_in, 1, h->Ws1_t, d, 0));
+    LMOE_TRY(repack(h, Ws2, h->shared_m, d, 1, h->Wu_t, h->Kup, skip ? 0 : l));
+  }
+  LMOE_CUDA(h, cudaDeviceSynchronize());
+  h->weights_set = true;
+  return LMOE_OK;
+}
+
+lmoe_status lmoe_reserve(lmoe_layer* h, int max_T) {
+  if (!h || max_T < 1) return LMOE_ERR_INVALID_ARG;
+  if (max_T <= h->max_T) return LMOE_OK;
+  DevGuard g(h->device);
+  LMOE_CUDA(h, cudaDeviceSynchronize());
+  free_workspace(h);
+  const size_t T = max_T, R = T * h->k, es = h->es;
+  const size_t W = (T + 31) / 32;
+  const bool skip = (h->flags & LMOE_SKIP_PROJ) != 0;
+#define ALLOC(ptr, bytes) LMOE_CUDA(h, cudaMalloc((void**)&(ptr), std::max<size_t>(bytes, 16)))
+  ALLOC(h->logits, T * h->N * sizeof(float));
+  ALLOC(h->idx, R * sizeof(int));
+  ALLOC(h->w, R * sizeof(float));
+  ALLOC(h->bitmap, (size_t)h->N * W * sizeof(uint32_t));
+  ALLOC(h->wp, (size_t)h->N * W * sizeof(uint2));
+  ALLOC(h->counts, (size_t)h->N * sizeof(int));
+  ALLOC(h->offsets, (size_t)(h->N + 1) * sizeof(int));
+  ALLOC(h->tile_prefix, (size_t)(h->N + 1) * sizeof(int));
+  ALLOC(h->done, sizeof(unsigned));
+  ALLOC(h->err, sizeof(int));
+  ALLOC(h->row_tok, R * sizeof(int));
+  ALLOC(h->row_slot, R * sizeof(int));
+  ALLOC(h->row_w, R * sizeof(float));
+  if (!skip) ALLOC(h->z, T * h->l * es);
+  ALLOC(h->h, R * h->m * es);
+  ALLOC(h->ys, R * h->l * es);
+  if (h->Kup > 0) ALLOC(h->cat, T * h->Kup * es);
+  ALLOC(h->x_stage, T * h->d * es);
+  ALLOC(h->out_stage, T * h->d * es);
+#undef ALLOC
+  LMOE_CUDA(h, cudaMemset(h->bitmap, 0, (size_t)h->N * W * sizeof(uint32_t)));
+  LMOE_CUDA(h, cudaMemset(h->done, 0, sizeof(unsigned)));
+  LMOE_CUDA(h, cudaMemset(h->err, 0, sizeof(int)));
+  LMOE_CUDA(h, cudaMemset(h->offsets, 0, (size_t)(h->N + 1) * sizeof(int)));
+  LMOE_CUDA(h, cudaMemset(h->tile_prefix, 0, (size_t)(h->N + 1) * sizeof(int)));
+  LMOE_CUDA(h, cudaDeviceSynchronize());
+  h->max_T = max_T;
+  h->W = (int)W;
+  return LMOE_OK;
+}
+
+lmoe_status lmoe_forward(lmoe_layer* h, const void* x, void* out, int T, lmoe_stream_t stream) {
+  if (!h) return LMOE_ERR_INVALID_ARG;
+  if (!h->weights_set || h->max_T == 0) return LMOE_ERR_NOT_READY;
+  if (!valid_stream_call(h, T)) return LMOE_ERR_INVALID_ARG;
+  if (T == 0) return LMOE_OK;
+  if (!x || !out || x == out) return LMOE_ERR_INVALID_ARG;
+  DevGuard g(h->device);
+  return run_forward(h, x, out, T, (cudaStream_t)stream);
+}
+
+lmoe_status lmoe_forward_host(lmoe_layer* h, const void* x_host, void* out_host, int T,
+                              lmoe_stream_t stream) {
+  if (!h) return LMOE_ERR_INVALID_ARG;
+  if (!h->weights_set || h->max_T == 0) return LMOE_ERR_NOT_READY;
+  if (!valid_stream_call(h, T)) return LMOE_ERR_INVALID_ARG;
+  if (T == 0) return LMOE_OK;
+  if (!x_host || !out_host) return LMOE_ERR_INVALID_ARG;
+  DevGuard g(h->device);
+  cudaStream_t st = (cudaStream_t)stream;
+  const size_t bytes = (size_t)T * h->d * h->es;
+  LMOE_CUDA(h, cudaMemcpyAsync(h->x_stage, x_host, bytes, cudaMemcpyHostToDevice, st));
+  LMOE_TRY(run_forward(h, h->x_stage, h->out_stage, T, st));
+  LMOE_CUDA(h, cudaMemcpyAsync(out_host, h->out_stage, bytes, cudaMemcpyDeviceToHost, st));
+  return LMOE_OK;
+}
+
+lmoe_status lmoe_route_only(lmoe_layer* h, const float* logits, int T, int* idx, float* w,
+                            int* offsets, int* perm, lmoe_stream_t stream) {
+  if (!h) return LMOE_ERR_INVALID_ARG;
+  if (h->max_T == 0) return LMOE_ERR_NOT_READY;
+  if (!valid_stream_call(h, T)) return LMOE_ERR_INVALID_ARG;
+  if (!offsets) return LMOE_ERR_INVALID_ARG;
+  if (T > 0 && (!logits || !idx || !w || !perm)) return LMOE_ERR_INVALID_ARG;
+  DevGuard g(h->device);
+  cudaStream_t st = (cudaStream_t)stream;
+  h->launches = 0;
+  if (T == 0) {
+    LMOE_CUDA(h, cudaMemsetAsync(offsets, 0, (size_t)(h->N + 1) * sizeof(int), st));
+    return LMOE_OK;
+  }
+  return run_routing(h, logits, T, idx, w, offsets, nullptr, perm, nullptr, st, false);
+}
+
+lmoe_status lmoe_router_logits(lmoe_layer* h, const void* x, float* logits, int T,
+                               lmoe_stream_t stream) {
+  if (!h) return LMOE_ERR_INVALID_ARG;
+  if (!h->weights_set || h->max_T == 0) return LMOE_ERR_NOT_READY;
+  if (!valid_stream_call(h, T)) return LMOE_ERR_INVALID_ARG;
+  if (T == 0) return LMOE_OK;
+  if (!x || !logits) return LMOE_ERR_INVALID_ARG;
+  DevGuard g(h->device);
+  h->launches = 0;
+  return run_router(h, x, logits, T, (cudaStream_t)stream);
+}
+
+lmoe_status lmoe_stage_bytes(const lmoe_layer* h, int stage, int T, size_t* bytes) {
+  if (!h || !bytes || T < 0) return LMOE_ERR_INVALID_ARG;
+  const size_t t = T, R = t * h->k, es = h->es;
+  const bool skip = (h->flags & LMOE_SKIP_PROJ) != 0;
+  switch (stage) {
+    case LMOE_STAGE_LOGITS: *bytes = t * h->N * 4; break;
+    case LMOE_STAGE_IDX:
+    case LMOE_STAGE_W:
+    case LMOE_STAGE_PERM: *bytes = R * 4; break;
+    case LMOE_STAGE_OFFSETS: *bytes = (size_t)(h->N + 1) * 4; break;
+    case LMOE_STAGE_Z:
+      if (skip) return LMOE_ERR_INVALID_ARG;
+      *bytes = t * h->l * es;
+      break;
+    case LMOE_STAGE_H: *bytes = R * h->m * es; break;
+    case LMOE_STAGE_YS: *bytes = R * h->l * es; break;
+    case LMOE_STAGE_COMB:
+      if (skip) return LMOE_ERR_INVALID_ARG;
+      *bytes = t * h->l * es;
+      break;
+    default: return LMOE_ERR_INVALID_ARG;
+  }
+  return LMOE_OK;
+}
+
+lmoe_status lmoe_debug_dump(lmoe_layer* h, int stage, void* dst, size_t bytes, lmoe_stream_t stream) {
+  if (!h || !dst) return LMOE_ERR_INVALID_ARG;
+  if (h->last_T < 0) return LMOE_ERR_NOT_READY;
+  size_t need = 0;
+  LMOE_TRY(lmoe_stage_bytes(h, stage, h->last_T, &need));
+  if (bytes < need) return LMOE_ERR_INVALID_ARG;
+  if (need == 0) return LMOE_OK;
+  const void* src = nullptr;
+  size_t pitch = 0, width = 0, rows = 0;
+  switch (stage) {
+    case LMOE_STAGE_LOGITS: src = h->logits; break;
+    case LMOE_STAGE_IDX: src = h->idx; break;
+    case LMOE_STAGE_W: src = h->w; break;
+    case LMOE_STAGE_OFFSETS: src = h->offsets; break;
+    case LMOE_STAGE_PERM: src = h->row_slot; break;
+    case LMOE_STAGE_Z: src = h->z; break;
+    case LMOE_STAGE_H: src = h->h; break;
+    case LMOE_STAGE_YS: src = h->ys; break;
+    case LMOE_STAGE_COMB:  // the first l columns of the [T, l + shared_m] operand
+      src = h->cat;
+      pitch = (size_t)h->Kup * h->es;
+      width = (size_t)h->l * h->es;
+      rows = (size_t)h->last_T;
+      break;
+  }
+  DevGuard g(h->device);
+  if (pitch)
+    LMOE_CUDA(h, cudaMemcpy2DAsync(dst, width, src, pitch, width, rows, cudaMemcpyDeviceToDevice,
+                                   (cudaStream_t)stream));
+  else
+    LMOE_CUDA(h, cudaMemcpyAsync(dst, src, need, cudaMemcpyDeviceToDevice, (cudaStream_t)stream));
+  return LMOE_OK;
+}
+
+lmoe_status lmoe_last_error(lmoe_layer* h, int* device_error_word) {
+  if (!h || !device_error_word) return LMOE_ERR_INVALID_ARG;
+  *device_error_word = 0;
+  if (!h->err) return LMOE_OK;
+  DevGuard g(h->device);
+  LMOE_CUDA(h, cudaDeviceSynchronize());
+  int word = 0;
+  LMOE_CUDA(h, cudaMemcpy(&word, h->err, sizeof(int), cudaMemcpyDeviceToHost));
+  LMOE_CUDA(h, cudaMemset(h->err, 0, sizeof(int)));
+  *device_error_word = word;
+  if (word & LMOE_DEVERR_WAIT_TIMEOUT) return LMOE_ERR_TIMEOUT;
+  if (word) return LMOE_ERR_DEVICE;
+  return LMOE_OK;
+}
+
+lmoe_status lmoe_profile_begin(lmoe_layer* h, int max_forwards) {
+  if (!h || max_forwards < 1) return LMOE_ERR_INVALID_ARG;
+  DevGuard g(h->device);
+  LMOE_CUDA(h, cudaDeviceSynchronize());
+  destroy_events(h);
+  const size_t n = (size_t)max_forwards * (kStages + 1);
+  h->events.resize(n, nullptr);
+  for (size_t i = 0; i < n; ++i) {
+    cudaError_t e = cudaEventCreate(&h->events[i]);
+    if (e != cudaSuccess) {
+      h->events.resize(i);
+      destroy_events(h);
+      return cuda_fail(h, e, "cudaEventCreate");
+    }
+  }
+  h->prof_cap = max_forwards;
+  h->prof_count = 0;
+  h->profiling = true;
+  return LMOE_OK;
+}
+
+lmoe_status lmoe_profile_end(lmoe_layer* h, float* ms, int capacity, int* n_forwards, int* n_stages) {
+  if (!h || !n_forwards || !n_stages || (capacity > 0 && !ms)) return LMOE_ERR_INVALID_ARG;
+  DevGuard g(h->device);
+  *n_forwards = 0;
+  *n_stages = kStages;
+  if (!h->profiling) return LMOE_ERR_NOT_READY;
+  LMOE_CUDA(h, cudaDeviceSynchronize());
+  int written = 0;
+  for (int f = 0; f < h->prof_count; ++f) {
+    if ((f + 1) * kStages > capacity) break;
+    for (int s = 0; s < kStages; ++s) {
+      float t = 0.f;
+      cudaEvent_t* ev = &h->events[(size_t)f * (kStages + 1)];
+      LMOE_CUDA(h, cudaEventElapsedTime(&t, ev[s], ev[s + 1]));
+      ms[f * kStages + s] = t;
+    }
+    written = f + 1;
+  }
+  *n_forwards = written;
+  destroy_events(h);
+  return LMOE_OK;
+}
+
+int lmoe_last_launch_count(const lmoe_layer* h) { return h ? h->launches : 0; }
+int lmoe_last_expert_path(const lmoe_layer* h) { return h ? h->expert_path : -1; }
+
+void lmoe_destroy(lmoe_layer* h) {
+  if (!h) return;
+  {
+    DevGuard g(h->device);
+    cudaDeviceSynchronize();
+    destroy_events(h);
+    free_workspace(h);
+    free_weights(h);
+  }
+  delete h;
+}
+
+}  // extern "C"

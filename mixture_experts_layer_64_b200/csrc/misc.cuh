@@ -1,0 +1,81 @@
+// Elementwise kernels: the gate-weighted combine (Eq. (1), the sum over the
+// selected experts, in latent width) and the weight repack into the K-major
+// layout the GEMMs read.
+#pragma once
+
+#include "common.cuh"
+
+namespace lmoe {
+
+// comb[t, c] = (resid[t, c] +) sum_{j < k} ys[t*k + j, c], summed in fp32 in
+// slot order, rounded once.  ys rows are in slot order (t*k + j), so each
+// token's k rows are contiguous.  One block per token, VEC elements per thread
+// per step (16-byte accesses).
+template <typename T>
+__global__ void __launch_bounds__(256) combine_kernel(const T* __restrict__ ys, int k, int l,
+                                                      const T* __restrict__ resid, long ldr,
+                                                      T* __restrict__ out, long ldo) {
+  constexpr int VEC = 16 / sizeof(T);
+  const int t = blockIdx.x;
+  const T* base = ys + (size_t)t * k * l;
+  for (int c = threadIdx.x * VEC; c < l; c += blockDim.x * VEC) {
+    float acc[VEC];
+    if (resid) {
+      const uint4 rv = *reinterpret_cast<const uint4*>(resid + (size_t)t * ldr + c);
+      const T* rb = reinterpret_cast<const T*>(&rv);
+#pragma unroll
+      for (int v = 0; v < VEC; ++v) acc[v] = to_f32<T>(rb[v]);
+    } else {
+#pragma unroll
+      for (int v = 0; v < VEC; ++v) acc[v] = 0.f;
+    }
+    for (int j = 0; j < k; ++j) {
+      const uint4 yv = __ldg(reinterpret_cast<const uint4*>(base + (size_t)j * l + c));
+      const T* yb = reinterpret_cast<const T*>(&yv);
+#pragma unroll
+      for (int v = 0; v < VEC; ++v) acc[v] += to_f32<T>(yb[v]);
+    }
+    uint4 ov;
+    T* ob = reinterpret_cast<T*>(&ov);
+#pragma unroll
+    for (int v = 0; v < VEC; ++v) ob[v] = from_f32<T>(acc[v]);
+    *reinterpret_cast<uint4*>(out + (size_t)t * ldo + c) = ov;
+  }
+}
+
+// Scalar fallback of combine_kernel for widths that are not a multiple of VEC.
+template <typename T>
+__global__ void __launch_bounds__(256) combine_scalar_kernel(const T* __restrict__ ys, int k, int l,
+                                                             const T* __restrict__ resid, long ldr,
+                                                             T* __restrict__ out, long ldo) {
+  const int t = blockIdx.x;
+  for (int c = threadIdx.x; c < l; c += blockDim.x) {
+    float acc = resid ? to_f32<T>(resid[(size_t)t * ldr + c]) : 0.f;
+    for (int j = 0; j < k; ++j) acc += to_f32<T>(ys[((size_t)t * k + j) * l + c]);
+    out[(size_t)t * ldo + c] = from_f32<T>(acc);
+  }
+}
+
+// out[b][c][col0 + r] = in[b][r][c] for r < rows, c < cols: the [in, out]
+// API layout to the K-major [out, in] layout, batched over experts, with a
+// column offset so that two matrices can share one K-concatenated operand.
+template <typename T>
+__global__ void transpose_kernel(const T* __restrict__ in, int rows, int cols, long in_bstride,
+                                 T* __restrict__ out, long ldo, int col0, long out_bstride) {
+  __shared__ T tile[32][33];
+  const int b = blockIdx.z;
+  const int c0 = blockIdx.x * 32, r0 = blockIdx.y * 32;
+  const T* src = in + (size_t)b * in_bstride;
+  T* dst = out + (size_t)b * out_bstride;
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    const int r = r0 + i, c = c0 + threadIdx.x;
+    if (r < rows && c < cols) tile[i][threadIdx.x] = src[(size_t)r * cols + c];
+  }
+  __syncthreads();
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    const int c = c0 + i, r = r0 + threadIdx.x;
+    if (r < rows && c < cols) dst[(size_t)c * ldo + col0 + r] = tile[threadIdx.x][i];
+  }
+}
+
+}  // namespace lmoe

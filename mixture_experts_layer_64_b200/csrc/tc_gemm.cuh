@@ -1,0 +1,386 @@
+// Persistent grouped GEMM on the sm_100a tensor cores (tcgen05.mma, fp32
+// accumulators in tensor memory, operands staged in shared memory by TMA or
+// by a cp.async row gather).
+//
+// One kernel serves every contraction of the layer:
+//   router logits, down-projection, shared FC1, up-projection  (dense)
+//   expert FC1 (+ activation) and FC2 (+ gate scale, slot scatter) (grouped)
+// A problem is D[r, f] = sum_k A[src(r), k] B[wrow(g, f), k] with both
+// operands K-major (B holds the weights transposed to [out, in]).
+//
+// Two operand arrangements:
+//   token-tiled (kSwap = false): the MMA's M = 128 activation rows, N = the
+//     weight tile (128 or 256 features); used when groups hold many rows.
+//   weight-stationary (kSwap = true): the MMA's M = 128 weight rows
+//     (features), N = the group's rows rounded up to 16 (<= 128); used at
+//     decode sizes, where an expert sees ~16 tokens and the kernel is a
+//     stream over the expert weights.
+// Gated FC1 (SwiGLU) loads the gate rows f and the linear rows f + m of the
+// same feature tile and accumulates them into two TMEM accumulators, so the
+// epilogue sees both halves of a feature in one thread.
+//
+// Warp roles (256 threads):
+//   warp 0      TMA producer (weights, and contiguous activation rows)
+//   warp 1      TMEM allocation and the single-thread MMA issuer
+//   warps 2-3   cp.async row gather of activations (gathered problems)
+//   warps 4-7   epilogue: tcgen05.ld -> epilogue math -> global stores
+// The smem ring has STAGES stages of one 64-wide K slice each; TMEM holds two
+// accumulator buffers so the epilogue of tile i overlaps the MMAs of tile i+1.
+#pragma once
+
+#include "common.cuh"
+
+namespace lmoe {
+
+constexpr int kTcThreads = 256;
+constexpr int kTcSmemBudget = 200 * 1024;
+constexpr int kGatherThreads = 64;
+constexpr int kGatherLag = 2;  // stages of cp.async a gather thread keeps in flight
+
+template <bool kSwap_, bool kGather_, bool kDual_, int kWN_, int kEpi_>
+struct TcCfg {
+  static constexpr bool kSwap = kSwap_, kGather = kGather_, kDual = kDual_;
+  static constexpr int kEpi = kEpi_;
+  static constexpr int BK = 64;                       // bf16 per 128-byte swizzled row
+  static constexpr int ACT_ROWS = 128;
+  static constexpr int W_ROWS = kSwap ? 128 : (kDual ? 128 : kWN_);
+  static constexpr int NUM_W = kDual ? 2 : 1;
+  static constexpr int ACT_BYTES = ACT_ROWS * BK * 2;
+  static constexpr int W_BYTES = W_ROWS * BK * 2;
+  static constexpr int STAGE_BYTES = ACT_BYTES + NUM_W * W_BYTES;
+  static constexpr int STAGES_RAW = kTcSmemBudget / STAGE_BYTES;
+  static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
+  static constexpr int ACC_N = kSwap ? 128 : W_ROWS;  // fp32 columns of one accumulator
+  static constexpr int ACC_COLS = ACC_N * NUM_W;      // one TMEM buffer
+  static constexpr int TMEM_COLS = 2 * ACC_COLS;      // double buffered
+  static constexpr int FT = W_ROWS;                   // features per tile
+  static constexpr int SMEM_BYTES = 1024 /*align slack*/ + STAGES * STAGE_BYTES + 512;
+  static_assert(TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM allocation must be a power of two");
+  static_assert(STAGES >= kGatherLag + 2, "pipeline too shallow");
+  static_assert(!kSwap || kEpi == EPI_ACT || kEpi == EPI_SCALE_SCATTER, "swap epilogues");
+  static_assert(kWN_ == 128 || kWN_ == 256, "weight tile");
+};
+
+// ---- epilogue stores ----------------------------------------------------------
+
+// One row (token-tiled mode): 32 consecutive features [f, f+32) of row `row`.
+template <int kEpi>
+__device__ __forceinline__ void store_row32(const GemmProblem& p, int row, int f, const float* v0,
+                                            const float* v1) {
+  const EpiParams& e = p.epi;
+  const bool full = f + 32 <= p.F;
+  if (kEpi == EPI_F32_BIAS) {
+    float* o = static_cast<float*>(e.out) + (size_t)row * e.ldo + f;
+    if (full) {
+#pragma unroll
+      for (int i = 0; i < 32; i += 4) {
+        float4 q;
+        q.x = v0[i] + (e.bias ? __ldg(e.bias + f + i) : 0.f);
+        q.y = v0[i + 1] + (e.bias ? __ldg(e.bias + f + i + 1) : 0.f);
+        q.z = v0[i + 2] + (e.bias ? __ldg(e.bias + f + i + 2) : 0.f);
+        q.w = v0[i + 3] + (e.bias ? __ldg(e.bias + f + i + 3) : 0.f);
+        *reinterpret_cast<float4*>(o + i) = q;
+      }
+    } else {
+      for (int i = 0; i < 32 && f + i < p.F; ++i) o[i] = v0[i] + (e.bias ? e.bias[f + i] : 0.f);
+    }
+    return;
+  }
+  float r[32];
+  const bf16* res = nullptr;
+  size_t orow = (size_t)row;
+  if (kEpi == EPI_ACT) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) r[i] = apply_act(e.act, v0[i], v1 ? v1[i] : 0.f);
+  } else if (kEpi == EPI_SCALE_SCATTER) {
+    const float s = __ldg(e.row_w + row);
+    orow = (size_t)__ldg(e.row_slot + row);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) r[i] = v0[i] * s;
+  } else {  // EPI_RESID
+    res = static_cast<const bf16*>(e.resid) + (size_t)row * e.ldr + f;
+  }
+  bf16* o = static_cast<bf16*>(e.out) + orow * e.ldo + (kEpi == EPI_ACT ? e.col0 : 0) + f;
+  if (full) {
+#pragma unroll
+    for (int i = 0; i < 32; i += 8) {
+      if (kEpi == EPI_RESID) {
+        const uint4 rv = *reinterpret_cast<const uint4*>(res + i);
+        const bf16* rb = reinterpret_cast<const bf16*>(&rv);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) r[i + j] = __bfloat162float(rb[j]) + v0[i + j];
+      }
+      uint4 q;
+      bf16* qb = reinterpret_cast<bf16*>(&q);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) qb[j] = __float2bfloat16_rn(r[i + j]);
+      *reinterpret_cast<uint4*>(o + i) = q;
+    }
+  } else {
+    for (int i = 0; i < 32 && f + i < p.F; ++i) {
+      float v = (kEpi == EPI_RESID) ? __bfloat162float(res[i]) + v0[i] : r[i];
+      o[i] = __float2bfloat16_rn(v);
+    }
+  }
+}
+
+// One element (weight-stationary mode): feature f of row `row`.
+template <int kEpi>
+__device__ __forceinline__ void store_elem(const GemmProblem& p, int row, int f, float v0, float v1) {
+  const EpiParams& e = p.epi;
+  if (kEpi == EPI_ACT) {
+    static_cast<bf16*>(e.out)[(size_t)row * e.ldo + e.col0 + f] =
+        __float2bfloat16_rn(apply_act(e.act, v0, v1));
+  } else {  // EPI_SCALE_SCATTER
+    const size_t orow = (size_t)__ldg(e.row_slot + row);
+    static_cast<bf16*>(e.out)[orow * e.ldo + f] = __float2bfloat16_rn(v0 * __ldg(e.row_w + row));
+  }
+}
+
+// ---- the kernel -----------------------------------------------------------------
+
+template <class Cfg>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const GemmProblem p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + Cfg::STAGES * Cfg::STAGE_BYTES);
+  uint64_t* empty = full + Cfg::STAGES;
+  uint64_t* tfull = empty + Cfg::STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int NT = (p.F + Cfg::FT - 1) / Cfg::FT;
+  const int KB = p.K / Cfg::BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < Cfg::STAGES; ++s) {
+      mbar_init(&full[s], Cfg::kGather ? 1 + kGatherThreads : 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 4);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    if (!Cfg::kGather) prefetch_tensormap(&tmA);
+    prefetch_tensormap(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int num_tiles = total_row_tiles(p) * NT;
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      long armed = 0;
+      for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+        const int rt = t / NT, ft = t - (t / NT) * NT;
+        int g, row0, rows;
+        locate_row_tile(p, rt, g, row0, rows);
+        const int wrow = (int)(g * p.w_group_stride) + ft * Cfg::FT;
+        const int nsub = Cfg::kSwap ? (rows + 31) / 32 : 4;
+        uint32_t bytes = Cfg::NUM_W * Cfg::W_BYTES;
+        if (!Cfg::kGather) bytes += Cfg::kSwap ? nsub * 4096 : Cfg::ACT_BYTES;
+        bool ok = true;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, p.err)) { ok = false; break; }
+          uint8_t* st = smem + s * Cfg::STAGE_BYTES;
+          mbar_arrive_expect_tx(&full[s], bytes);
+          ++armed;
+          tma_load_2d(&tmB, &full[s], st + Cfg::ACT_BYTES, kb * Cfg::BK, wrow);
+          if (Cfg::kDual)
+            tma_load_2d(&tmB, &full[s], st + Cfg::ACT_BYTES + Cfg::W_BYTES, kb * Cfg::BK,
+                        wrow + p.dual_offset);
+          if (!Cfg::kGather) {
+            if (Cfg::kSwap) {
+              for (int sub = 0; sub < nsub; ++sub)
+                tma_load_2d(&tmA, &full[s], st + sub * 4096, kb * Cfg::BK, row0 + sub * 32);
+            } else {
+              tma_load_2d(&tmA, &full[s], st, kb * Cfg::BK, row0);
+            }
+          }
+          if (++s == Cfg::STAGES) { s = 0; ph ^= 1; }
+        }
+        if (!ok) break;
+      }
+      if (*abort_flag) {
+        // Let every armed load land before the block frees its shared memory.
+        int ss = s;
+        uint32_t pp = ph;
+        for (long i = 0; i < armed && i < Cfg::STAGES; ++i) {
+          if (ss == 0) { ss = Cfg::STAGES; pp ^= 1; }
+          --ss;
+          mbar_wait_drain(&full[ss], pp);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      int it = 0;
+      for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++it) {
+        const int rt = t / NT;
+        int g, row0, rows;
+        locate_row_tile(p, rt, g, row0, rows);
+        const int ab = it & 1;
+        const uint32_t aph = (it >> 1) & 1;
+        if (!mbar_wait(&tempty[ab], aph ^ 1, abort_flag, p.err)) break;
+        tc_fence_after();
+        const uint32_t d0 = tmem_base + ab * Cfg::ACC_COLS;
+        const uint32_t d1 = d0 + Cfg::ACC_N;
+        int n = Cfg::ACC_N;
+        if (Cfg::kSwap) n = max(16, (rows + 15) & ~15);
+        const uint32_t idesc = idesc_bf16_f32(128, n);
+        bool ok = true;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(&full[s], ph, abort_flag, p.err)) { ok = false; break; }
+          tc_fence_after();
+          const uint8_t* st = smem + s * Cfg::STAGE_BYTES;
+          const uint64_t da = smem_desc_sw128(st);
+          const uint64_t dw0 = smem_desc_sw128(st + Cfg::ACT_BYTES);
+          const uint64_t dw1 = smem_desc_sw128(st + Cfg::ACT_BYTES + Cfg::W_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < Cfg::BK / 16; ++kk) {
+            const uint32_t acc = (kb | kk) != 0;
+            const uint64_t adv = (uint64_t)(kk * 32) >> 4;  // 16 bf16 = 32 bytes along K
+            if (Cfg::kSwap) {
+              tc_mma_bf16(d0, dw0 + adv, da + adv, idesc, acc);
+              if (Cfg::kDual) tc_mma_bf16(d1, dw1 + adv, da + adv, idesc, acc);
+            } else {
+              tc_mma_bf16(d0, da + adv, dw0 + adv, idesc, acc);
+              if (Cfg::kDual) tc_mma_bf16(d1, da + adv, dw1 + adv, idesc, acc);
+            }
+          }
+          tc_commit(&empty[s]);
+          if (++s == Cfg::STAGES) { s = 0; ph ^= 1; }
+        }
+        if (!ok) break;
+        tc_commit(&tfull[ab]);
+      }
+      // Every MMA this thread issued has completed once `drain` flips.
+      tc_commit(drain);
+      mbar_wait_drain(drain, 0);
+    }
+  } else if (warp < 4) {
+    // ---------------- cp.async row gather ----------------
+    if (Cfg::kGather) {
+      const int gt = threadIdx.x - 64;  // 0..63
+      const int q = gt & 7;             // 16-byte chunk of a 128-byte row
+      const int rsub = gt >> 3;         // rows rsub, rsub + 8, ...
+      const uint32_t swz = (uint32_t)((q ^ rsub) * 16);
+      const bf16* A = static_cast<const bf16*>(p.A);
+      int s = 0, s_ret = 0, pending = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+        const int rt = t / NT;
+        int g, row0, rows;
+        locate_row_tile(p, rt, g, row0, rows);
+        const int nload = Cfg::kSwap ? max(16, (rows + 15) & ~15) : 128;
+        const bf16* src[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int r = rsub + 8 * i;
+          src[i] = (r < rows) ? A + (size_t)__ldg(p.gather + row0 + r) * p.lda + q * 8 : A;
+        }
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, p.err)) { ok = false; break; }
+          uint8_t* act = smem + s * Cfg::STAGE_BYTES;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int r = rsub + 8 * i;
+            if (r < nload)
+              cp_async_16(act + r * 128 + swz, src[i] + kb * Cfg::BK, r < rows ? 16u : 0u);
+          }
+          cp_async_commit();
+          if (pending == kGatherLag) {
+            cp_async_wait<kGatherLag>();
+            fence_proxy_async_smem();
+            mbar_arrive(&full[s_ret]);
+            if (++s_ret == Cfg::STAGES) s_ret = 0;
+          } else {
+            ++pending;
+          }
+          if (++s == Cfg::STAGES) { s = 0; ph ^= 1; }
+        }
+      }
+      cp_async_wait<0>();
+      fence_proxy_async_smem();
+      for (; pending > 0; --pending) {
+        mbar_arrive(&full[s_ret]);
+        if (++s_ret == Cfg::STAGES) s_ret = 0;
+      }
+    }
+  } else {
+    // ---------------- epilogue (warps 4..7) ----------------
+    const int qd = warp & 3;  // TMEM lane quarter this warp may access
+    int it = 0;
+    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++it) {
+      const int rt = t / NT, ft = t - (t / NT) * NT;
+      int g, row0, rows;
+      locate_row_tile(p, rt, g, row0, rows);
+      const int ab = it & 1;
+      const uint32_t aph = (it >> 1) & 1;
+      if (!mbar_wait(&tfull[ab], aph, abort_flag, p.err)) break;
+      tc_fence_after();
+      const uint32_t tb = tmem_base + ((uint32_t)(qd * 32) << 16) + ab * Cfg::ACC_COLS;
+      const int f0 = ft * Cfg::FT;
+      float v0[32], v1[32];
+      if (!Cfg::kSwap) {
+        const int r = qd * 32 + lane;
+        for (int c0 = 0; c0 < Cfg::ACC_N; c0 += 32) {
+          tmem_ld_32x32(tb + c0, v0);
+          if (Cfg::kDual) tmem_ld_32x32(tb + Cfg::ACC_N + c0, v1);
+          tc_wait_ld();
+          if (r < rows && f0 + c0 < p.F)
+            store_row32<Cfg::kEpi>(p, row0 + r, f0 + c0, v0, Cfg::kDual ? v1 : nullptr);
+        }
+      } else {
+        const int f = f0 + qd * 32 + lane;
+        for (int c0 = 0; c0 < rows; c0 += 32) {
+          tmem_ld_32x32(tb + c0, v0);
+          if (Cfg::kDual) tmem_ld_32x32(tb + Cfg::ACC_N + c0, v1);
+          tc_wait_ld();
+          if (f < p.F) {
+            const int cn = min(32, rows - c0);
+#pragma unroll
+            for (int c = 0; c < 32; ++c)
+              if (c < cn)
+                store_elem<Cfg::kEpi>(p, row0 + c0 + c, f, v0[c], Cfg::kDual ? v1[c] : 0.f);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[ab]);
+    }
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
+  }
+}
+
+}  // namespace lmoe

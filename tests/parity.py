@@ -1,0 +1,159 @@
+"""Helpers of the GPU parity tests: build a layer on the device through the
+C-ABI binding, build the CPU oracle from host copies of the same bytes, and
+compare.
+
+The oracle never consumes a GPU result.  It computes its own fp64 router
+logits, rounds them to fp32 and selects on those (the kernel's precision).
+The GPU's logits differ from it by fp32 accumulation error, bounded per logit
+by tau = 64 u sum_i |x_i Wg_ie| (+ u |b_e|), u = 2^-24.  For a token whose
+oracle margin between the k-th and (k+1)-th logit exceeds 2 tau the selected
+set is unique and must match exactly, with its output; for the rest several
+selections are correct, so the test checks that the GPU's choice is one of
+them (every chosen logit within 2 tau of the k-th, every unchosen one below
+it + 2 tau) and leaves their outputs out of the element-wise comparison.
+"""
+from __future__ import annotations
+
+import math
+from typing import Dict, Iterable, Optional
+
+import numpy as np
+import torch
+
+import oracle
+from mixture_experts_layer_64_b200 import lmoe, workloads
+
+U32 = 2.0 ** -24
+BF16_MAX_ABS, BF16_REL_L2 = 2e-2, 5e-3   # stated tolerances for bf16 storage, fp32 accumulation
+F32_REL_L2 = 1e-5                       # stated tolerance for the fp32 layer
+
+
+def gpu_layer(w: workloads.Workload, flags: int = 0, W: Optional[Dict] = None):
+    if W is None:
+        W = workloads.make_weights(w, device="cuda")
+    L = lmoe.LatentMoELayer(w.d, w.l, w.N, w.k, w.m, act=w.act, shared_m=w.shared_m,
+                            dtype=w.dtype, flags=flags, skip_proj=w.skip_proj)
+    L.set_weights(W["Wg"], W["bias"], W["Wdown"], W["Wup"], W["W1"], W["W2"], W["Ws1"], W["Ws2"])
+    L.reserve(w.T)
+    return L, W
+
+
+def _cpu(t):
+    return None if t is None else t.detach().to("cpu")
+
+
+def oracle_layer(w: workloads.Workload, W: Dict, experts: Optional[Iterable[int]] = None):
+    if experts is None:
+        W1, W2 = _cpu(W["W1"]), _cpu(W["W2"])
+    else:
+        ex = sorted(set(int(e) for e in experts))
+        W1 = {e: _cpu(W["W1"][e]) for e in ex}
+        W2 = {e: _cpu(W["W2"][e]) for e in ex}
+    return oracle.OracleLayer(d=w.d, l=w.l, N=w.N, k=w.k, m=w.m, act=w.act,
+                              shared_m=w.shared_m, dtype=w.dtype, skip_proj=w.skip_proj,
+                              Wg=_cpu(W["Wg"]), bias=_cpu(W["bias"]), Wdown=_cpu(W["Wdown"]),
+                              Wup=_cpu(W["Wup"]), W1=W1, W2=W2, Ws1=_cpu(W["Ws1"]),
+                              Ws2=_cpu(W["Ws2"]))
+
+
+def logit_bound(x_host: torch.Tensor, Wg_host: torch.Tensor, bias_host) -> np.ndarray:
+    """tau[t, e] = 64 u sum_i |x_ti Wg_ie| + u |b_e| (float64)."""
+    ax = x_host.to(torch.float64).abs().numpy()
+    aw = Wg_host.to(torch.float64).abs().numpy()
+    tau = 64.0 * U32 * (ax @ aw)
+    if bias_host is not None:
+        tau += U32 * np.abs(bias_host.to(torch.float64).numpy())[None, :]
+    return tau
+
+
+def rel_l2(a: np.ndarray, b: np.ndarray) -> float:
+    den = float(np.linalg.norm(b))
+    return float(np.linalg.norm(a - b)) / (den if den > 0 else 1.0)
+
+
+def check_forward(w: workloads.Workload, flags: int = 0, tokens: Optional[np.ndarray] = None,
+                  x: Optional[torch.Tensor] = None, W: Optional[Dict] = None,
+                  layer=None, stages: bool = True) -> Dict:
+    """Runs lmoe_forward on the workload and compares it with the oracle on
+    `tokens` (all by default).  Returns the measured errors."""
+    if layer is None:
+        L, W = gpu_layer(w, flags, W)
+    else:
+        L = layer
+    if x is None:
+        x = workloads.make_x(w, device="cuda")
+    T = x.shape[0]
+    out = L.forward(x)
+    torch.cuda.synchronize()
+    g_idx = L.debug_dump("idx", T).cpu().numpy()
+    g_w = L.debug_dump("w", T).cpu().numpy()
+    g_lg = L.debug_dump("logits", T).cpu().numpy()
+    g_z = L.debug_dump("z", T).cpu().float().numpy() if (stages and not w.skip_proj) else None
+    g_comb = L.debug_dump("comb", T).cpu().float().numpy() if (stages and not w.skip_proj) else None
+    g_out = out.cpu().to(torch.float64).numpy()
+    st, word = L.last_error()
+    assert st == lmoe.OK and word == 0, (st, word)
+
+    if tokens is None:
+        tokens = np.arange(T, dtype=np.int32)
+    tokens = np.asarray(tokens, dtype=np.int32)
+    x_host = x.cpu()
+    O0 = oracle_layer(w, W, experts=[])
+    lg64 = O0.router_logits(x_host, tokens)
+    lg32 = lg64.astype(np.float32)
+    o_idx, o_w, _, _ = oracle.route(lg32, w.k)
+
+    # logits: within the accumulation bound of the oracle's
+    tau = logit_bound(x_host[tokens], _cpu(W["Wg"]), _cpu(W["bias"]))
+    err = np.abs(g_lg[tokens].astype(np.float64) - lg64)
+    assert np.all(err <= tau), f"router logits off by {err.max():.3e} (bound {tau.min():.3e}..)"
+    logit_rel = rel_l2(g_lg[tokens].astype(np.float64), lg64)
+
+    # routing: unique where the oracle's top-k boundary is wider than 2 tau
+    srt = -np.sort(-lg32.astype(np.float64), axis=1)
+    kth = srt[:, w.k - 1]
+    nxt = srt[:, w.k] if w.k < w.N else np.full(len(tokens), -np.inf)
+    tmax = tau.max(axis=1)
+    uniq = (kth - nxt) > 2 * tmax
+    gi = g_idx[tokens]
+    assert np.array_equal(gi[uniq], o_idx[uniq]), "selected experts differ on unique tokens"
+    assert np.all(np.abs(g_w[tokens][uniq] - o_w[uniq]) <= 1e-3)
+    for r in np.nonzero(~uniq)[0]:
+        chosen = lg32[r, gi[r]].astype(np.float64)
+        assert len(set(gi[r].tolist())) == w.k
+        assert np.all(chosen >= kth[r] - 2 * tmax[r])
+        others = np.setdiff1d(np.arange(w.N), gi[r])
+        if others.size:
+            assert np.all(lg32[r, others] <= kth[r] + 2 * tmax[r])
+
+    # outputs of the unique tokens
+    ut = tokens[uniq]
+    res = {"tokens": len(tokens), "unique": int(uniq.sum()), "logit_rel_l2": logit_rel}
+    if ut.size:
+        experts = np.unique(o_idx[uniq])
+        O = oracle_layer(w, W, experts=experts)
+        ref, z, comb = O.forward(x_host, o_idx[uniq], o_w[uniq], tokens=ut, stages=True)
+        got = g_out[ut]
+        res["max_abs"] = float(np.abs(got - ref).max())
+        res["rel_l2"] = rel_l2(got, ref)
+        if w.dtype == "f32":
+            assert res["rel_l2"] <= F32_REL_L2, res
+        else:
+            assert res["max_abs"] <= BF16_MAX_ABS and res["rel_l2"] <= BF16_REL_L2, res
+        if g_z is not None:
+            res["z_rel_l2"] = rel_l2(g_z[ut].astype(np.float64), z)
+            assert res["z_rel_l2"] <= (1e-5 if w.dtype == "f32" else 5e-3), res
+        if g_comb is not None:
+            res["comb_rel_l2"] = rel_l2(g_comb[ut].astype(np.float64), comb)
+            assert res["comb_rel_l2"] <= (1e-5 if w.dtype == "f32" else 1e-2), res
+    res["expert_path"] = L.last_expert_path
+    res["launches"] = L.last_launch_count
+    return res
+
+
+def sample_tokens(T: int, n: int, seed: int = 0) -> np.ndarray:
+    if n >= T:
+        return np.arange(T, dtype=np.int32)
+    rng = np.random.default_rng(seed)
+    pick = set(rng.choice(T, size=n - 2, replace=False).tolist()) | {0, T - 1}
+    return np.array(sorted(pick), dtype=np.int32)

@@ -1,0 +1,173 @@
+"""GPU parity of the CUDA library against the CPU oracle, through the C ABI.
+
+Routing on shared fp32 logits is compared bit for bit (indices, offsets,
+permutation); floating-point outputs within the stated tolerances (bf16
+storage with fp32 accumulation: max-abs <= 2e-2 and rel-L2 <= 5e-3; the fp32
+layer: rel-L2 <= 1e-5).  See tests/parity.py for how near-ties are handled.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from mixture_experts_layer_64_b200 import lmoe, workloads
+from parity import check_forward, gpu_layer, sample_tokens
+
+pytestmark = pytest.mark.gpu
+
+W_ = workloads.Workload
+
+
+# ---------------------------------------------------------------------------
+# routing on shared logits: bit-exact
+# ---------------------------------------------------------------------------
+
+def _route_case(T, N, k, seed, bias=None):
+    lg = workloads.make_logits(T, N, seed, bias=bias, ties=True)
+    w = W_("route", T=max(T, 1), d=64, l=64, N=N, k=k, m=64, act="silu", dtype="bf16")
+    L = lmoe.LatentMoELayer(w.d, w.l, N, k, w.m, act="silu", dtype="bf16")
+    L.reserve(max(T, 1))
+    r = L.route_only(lg.cuda())
+    torch.cuda.synchronize()
+    if T == 0:
+        assert torch.all(r["offsets"] == 0)
+        return
+    o_idx, o_w, o_off, o_perm = oracle.route(lg.numpy(), k)
+    np.testing.assert_array_equal(r["idx"].cpu().numpy(), o_idx)
+    np.testing.assert_array_equal(r["offsets"].cpu().numpy(), o_off)
+    np.testing.assert_array_equal(r["perm"].cpu().numpy(), o_perm)
+    np.testing.assert_allclose(r["w"].cpu().numpy(), o_w, rtol=2e-6, atol=1e-7)
+    assert L.last_error() == (lmoe.OK, 0)
+
+
+@pytest.mark.parametrize("name", workloads.WORKLOAD_ORDER)
+def test_route_only_bit_exact_workload_shapes(name):
+    w = workloads.WORKLOADS[name]
+    _route_case(w.T, w.N, w.k, seed=w.seed + 10, bias=workloads.make_bias(w))
+
+
+@pytest.mark.parametrize("T,N,k", [(1, 1, 1), (1, 16, 4), (33, 16, 16), (31, 7, 3), (32, 64, 1),
+                                   (1000, 128, 8), (4097, 512, 22), (0, 16, 4), (65, 1024, 32),
+                                   (300, 896, 16)])
+def test_route_only_bit_exact_edges(T, N, k):
+    _route_case(T, N, k, seed=T * 7 + N + k)
+
+
+def test_route_only_rejects_oversized_T():
+    L = lmoe.LatentMoELayer(64, 64, 16, 4, 64, act="silu", dtype="bf16")
+    L.reserve(8)
+    with pytest.raises(lmoe.LmoeError):
+        L.route_only(torch.zeros((9, 16), device="cuda"))
+
+
+# ---------------------------------------------------------------------------
+# small layers that span several tiles with ragged tails
+# ---------------------------------------------------------------------------
+
+SMALL = {
+    # tcgen05 path: K multiples of 64, feature and row tiles with ragged tails
+    "swiglu": W_("s-swiglu", T=300, d=256, l=128, N=8, k=3, m=192, act="swiglu", seed=11),
+    "relu2-shared": W_("s-relu2", T=260, d=256, l=192, N=6, k=2, m=320, act="relu2",
+                       shared_m=320, seed=12),
+    "silu-bias": W_("s-silu", T=200, d=320, l=128, N=12, k=4, m=128, act="silu",
+                    bias="normal0.5", seed=13),
+    "swiglu-shared": W_("s-swiglu-sh", T=150, d=192, l=64, N=5, k=2, m=64, act="swiglu",
+                        shared_m=192, seed=14),
+    "skip": W_("s-skip", T=130, d=256, l=256, N=4, k=2, m=128, act="swiglu", skip_proj=True,
+               seed=15),
+    "skip-shared": W_("s-skip-sh", T=70, d=128, l=128, N=4, k=1, m=64, act="relu2",
+                      skip_proj=True, shared_m=128, seed=16),
+    # shapes the tcgen05 kernel does not take (K % 64 != 0): CUDA-core path
+    "odd-K": W_("s-odd", T=90, d=200, l=72, N=6, k=2, m=40, act="swiglu", shared_m=24, seed=17),
+    "fp32": W_("s-f32", T=100, d=96, l=32, N=8, k=3, m=48, act="relu2", shared_m=16, dtype="f32",
+               seed=18),
+}
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_small_layer_default_path(name):
+    res = check_forward(SMALL[name])
+    assert res["unique"] >= res["tokens"] * 0.9
+
+
+@pytest.mark.parametrize("name", ["swiglu", "relu2-shared", "skip"])
+@pytest.mark.parametrize("flags", [lmoe.FORCE_SWAP, lmoe.FORCE_NOSWAP, lmoe.FORCE_SIMT])
+def test_small_layer_each_expert_kernel(name, flags):
+    res = check_forward(SMALL[name], flags=flags)
+    want = {lmoe.FORCE_SWAP: 2, lmoe.FORCE_NOSWAP: 1, lmoe.FORCE_SIMT: 0}[flags]
+    assert res["expert_path"] == want
+
+
+def test_tcgen05_path_is_taken_for_bf16():
+    res = check_forward(SMALL["swiglu"])
+    assert res["expert_path"] in (1, 2)
+    res = check_forward(SMALL["odd-K"])
+    assert res["expert_path"] == 0
+
+
+def test_single_token_and_empty_batch():
+    w = SMALL["relu2-shared"]
+    L, W = gpu_layer(w)
+    x = workloads.make_x(w, device="cuda")
+    check_forward(w, layer=L, W=W, x=x[:1].contiguous())
+    out = torch.empty((0, w.d), dtype=torch.bfloat16, device="cuda")
+    L.forward(x[:0], out)  # T = 0 enqueues nothing
+    with pytest.raises(lmoe.LmoeError):
+        L.forward(workloads.make_x(w.with_T(w.T + 1), device="cuda"))
+
+
+def test_forward_is_deterministic_and_host_entry_matches():
+    w = SMALL["swiglu-shared"]
+    L, W = gpu_layer(w)
+    x = workloads.make_x(w, device="cuda")
+    a = L.forward(x)
+    b = L.forward(x)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+    xh = x.cpu().pin_memory()
+    oh = torch.empty_like(xh).pin_memory()
+    L.forward_host(xh, oh)
+    torch.cuda.synchronize()
+    assert torch.equal(oh, a.cpu())
+
+
+def test_uniform_router_is_mean_of_experts():
+    """W_g = 0, k = N: every token uses every expert with weight 1/N."""
+    w = W_("uniform", T=64, d=128, l=64, N=4, k=4, m=64, act="relu2", seed=19)
+    W = workloads.make_weights(w, device="cuda")
+    W["Wg"] = torch.zeros_like(W["Wg"])
+    res = check_forward(w, W=W)
+    assert res["unique"] == res["tokens"]
+
+
+def test_device_error_word_clean_and_profile():
+    w = SMALL["swiglu"]
+    L, W = gpu_layer(w)
+    x = workloads.make_x(w, device="cuda")
+    L.profile_begin(3)
+    for _ in range(3):
+        L.forward(x)
+    prof = L.profile_end()
+    assert len(prof) == 3 and all(v >= 0 for p in prof for v in p.values())
+    assert L.last_error() == (lmoe.OK, 0)
+    assert L.last_launch_count >= 8
+
+
+# ---------------------------------------------------------------------------
+# the five workloads at full size (sampled tokens for the large ones)
+# ---------------------------------------------------------------------------
+
+FULL_SAMPLES = {"tiny-fp32": 64, "std-moe-decode": 96, "latent-decode": 96,
+                "latent-prefill-shared": 64, "latent-prefill-skewed": 48}
+
+
+@pytest.mark.parametrize("name", workloads.WORKLOAD_ORDER)
+def test_workload_full_size(name):
+    w = workloads.WORKLOADS[name]
+    toks = sample_tokens(w.T, FULL_SAMPLES[name], seed=w.seed)
+    res = check_forward(w, tokens=toks)
+    print(name, res)
+    assert res["unique"] >= 0.8 * res["tokens"]
+    if w.dtype == "bf16":
+        assert res["expert_path"] in (1, 2)
+    torch.cuda.empty_cache()
