@@ -415,10 +415,22 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=workloads.WORKLOAD_ORDER, default=DEFAULT_WORKLOAD)
+
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--experts", type=int, default=None,
+                    help="override N (reduced cases for profiler captures)")
+    ap.add_argument("--topk", type=int, default=None, help="override k")
+    ap.add_argument("--tokens", type=int, default=None, help="override T")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
+    if args.experts or args.topk or args.tokens:
+        import dataclasses
+        base = workloads.WORKLOADS[args.workload]
+        ch = {k: v for k, v in (("N", args.experts), ("k", args.topk), ("T", args.tokens)) if v}
+        name = base.name + "(" + ",".join(f"{k}={v}" for k, v in ch.items()) + ")"
+        workloads.WORKLOADS[name] = dataclasses.replace(base, name=name, **ch)
+        args.workload = name
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)

@@ -36,6 +36,9 @@ struct EpiParams {
   long ldr;
   const int* row_slot;    // EPI_SCALE_SCATTER: tile row -> output row
   const float* row_w;     // EPI_SCALE_SCATTER: tile row -> gate weight
+  int split_off;          // EPI_ACT, bf16: > 0 also writes v - bf16(v) (rounded) at
+                          // column col0 + split_off + f, so that hi + lo carries the
+                          // value to ~16 significant bits through the next bf16 GEMM
 };
 
 // A (possibly grouped) problem D[r, f] = sum_k A[src(r), k] * B[wrow(g, f), k]
@@ -212,6 +215,12 @@ __device__ __forceinline__ void cp_async_16(void* smem_dst, const void* gsrc, ui
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem_dst)),
                "l"(gsrc), "r"(src_bytes)
                : "memory");
+}
+// Arrive on `bar` once every cp.async this thread issued so far has landed
+// (the pending count is raised first, so the phase waits for the copies; the
+// thread's own mbarrier.arrive is still needed to count it).
+__device__ __forceinline__ void cp_async_mbar_arrive(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>

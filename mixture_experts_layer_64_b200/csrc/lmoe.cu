@@ -7,11 +7,11 @@
 //   2 top-k + softmax        idx, w, per-expert token bitmaps
 //   3 grouping               word prefixes, offsets, tile counts; sorted rows
 //   4 down-projection GEMM   z[T,l] = x Wdown                 (not when skipped)
-//   5 shared FC1 GEMM        hs = act(x Ws1) into cat[:, l:]  (with a shared expert)
+//   5 shared FC1 GEMM        hs = act(x Ws1) into cat[:, l:] as bf16 hi + lo pairs
 //   6 expert FC1 (grouped)   h[r] = act(z[tok(r)] W1[e])      rows gathered by token
 //   7 expert FC2 (grouped)   ys[slot(r)] = w(r) * (h[r] W2[e])
 //   8 combine                cat[t, :l] = sum_j ys[t*k + j]   (or out = x + sum, skipped)
-//   9 up-projection GEMM     out = x + [comb | hs] [Wup ; Ws2]
+//   9 up-projection GEMM     out = x + [comb | hs_hi | hs_lo] [Wup ; Ws2 ; Ws2]
 // Contractions run on the tcgen05 kernel (bf16) or the CUDA-core kernel
 // (fp32, or shapes the tcgen05 kernel does not take).
 #include <cuda.h>
@@ -64,6 +64,7 @@ struct lmoe_layer {
   int d, l, N, k, m, act, shared_m, dtype;
   unsigned flags;
   int m_in, ms_in, Kup, es;  // es: element size
+  bool split_shared = false;  // bf16 shared hidden carried as a hi + lo pair
   int device = 0, num_sms = 148;
   bool weights_set = false;
   // weights, K-major
@@ -219,7 +220,9 @@ bool tc_eligible(const lmoe_layer* h, const GemmCall& c) {
   if (c.kind == GK_ROUTER) {
     if (p.epi.ldo % 4 != 0 || !aligned16(p.epi.out)) return false;
   } else {
-    if (p.epi.ldo % 8 != 0 || p.epi.col0 % 8 != 0 || !aligned16(p.epi.out)) return false;
+    if (p.epi.ldo % 8 != 0 || p.epi.col0 % 8 != 0 || p.epi.split_off % 8 != 0 ||
+        !aligned16(p.epi.out))
+      return false;
   }
   if (c.kind == GK_UP && (p.epi.ldr % 8 != 0 || !aligned16(p.epi.resid))) return false;
   return true;
@@ -365,6 +368,7 @@ lmoe_status run_forward(lmoe_layer* h, const void* x, void* out, int T, cudaStre
     c.p.epi.ldo = h->Kup;
     c.p.epi.col0 = skip ? 0 : l;
     c.p.epi.act = h->act;
+    c.p.epi.split_off = h->split_shared ? ms : 0;
     LMOE_TRY(run_gemm(h, c, st));
   }
   prof_mark(h, st, 5);
@@ -543,7 +547,12 @@ lmoe_status lmoe_create(int d, int l, int N, int k, int m, lmoe_act act, int sha
   h->dtype = dtype; h->flags = flags;
   h->m_in = act == LMOE_ACT_SWIGLU ? 2 * m : m;
   h->ms_in = act == LMOE_ACT_SWIGLU ? 2 * shared_m : shared_m;
-  h->Kup = ((flags & LMOE_SKIP_PROJ) ? 0 : l) + shared_m;
+  // bf16: the shared expert's hidden activations go into the up-projection as
+  // hi + lo bf16 pairs (K grows by shared_m, Ws2 appears twice in the
+  // K-concatenated weight), so their storage rounding no longer dominates the
+  // output error of layers with a large shared contribution.
+  h->split_shared = dtype == LMOE_BF16 && shared_m > 0;
+  h->Kup = ((flags & LMOE_SKIP_PROJ) ? 0 : l) + shared_m * (h->split_shared ? 2 : 1);
   h->es = dtype == LMOE_BF16 ? 2 : 4;
   h->device = dev;
   int sms = 0;
@@ -588,6 +597,8 @@ lmoe_status lmoe_set_weights(lmoe_layer* h, const void* W_g, const float* bias, 
   if (h->shared_m > 0) {
     LMOE_TRY(repack(h, Ws1, d, h->ms_in, 1, h->Ws1_t, d, 0));
     LMOE_TRY(repack(h, Ws2, h->shared_m, d, 1, h->Wu_t, h->Kup, skip ? 0 : l));
+    if (h->split_shared)
+      LMOE_TRY(repack(h, Ws2, h->shared_m, d, 1, h->Wu_t, h->Kup, (skip ? 0 : l) + h->shared_m));
   }
   LMOE_CUDA(h, cudaDeviceSynchronize());
   h->weights_set = true;

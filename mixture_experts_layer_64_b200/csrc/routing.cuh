@@ -7,7 +7,7 @@
 //                         (order-preserving fp32 bits << 32 | ~expert), so one
 //                         integer max picks "largest logit, then lowest
 //                         index"; -0.0 is folded into +0.0 first.  k rounds of
-//                         warp max give the slots; the gates are
+//                         warp max (two redux.sync each) give the slots; the gates are
 //                         exp(l_j - l_0) / sum over the k chosen.  Each choice
 //                         sets bit t of expert e's token bitmap.
 //   group_count_kernel    one warp per expert: popcount prefix over the
@@ -31,15 +31,6 @@ __device__ __forceinline__ uint32_t orderable_bits(float v) {
 }
 __device__ __forceinline__ float from_orderable_bits(uint32_t u) {
   return __uint_as_float((u & 0x80000000u) ? (u & 0x7FFFFFFFu) : ~u);
-}
-
-__device__ __forceinline__ unsigned long long warp_max_u64(unsigned long long v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const unsigned long long w = __shfl_xor_sync(0xffffffffu, v, o);
-    v = w > v ? w : v;
-  }
-  return v;
 }
 
 // logits [T, N] fp32 -> idx [T, k], w [T, k]; bitmap [N, W] gets bit t of
@@ -70,7 +61,12 @@ __global__ void __launch_bounds__(256) topk_softmax_kernel(const float* __restri
   if (debug && __any_sync(0xffffffffu, bad) && lane == 0) set_error(err, LMOE_DEVERR_NONFINITE);
   unsigned long long mine = 0;
   for (int j = 0; j < k; ++j) {
-    const unsigned long long top = warp_max_u64(best);
+    // warp max of the 64-bit keys as two 32-bit reductions: the value bits,
+    // then the inverted index among the lanes holding that value
+    const uint32_t hi = (uint32_t)(best >> 32);
+    const uint32_t vmax = __reduce_max_sync(0xffffffffu, hi);
+    const uint32_t imax = __reduce_max_sync(0xffffffffu, hi == vmax ? (uint32_t)best : 0u);
+    const unsigned long long top = ((unsigned long long)vmax << 32) | imax;
     if (lane == j) mine = top;
     const int e = (int)(0xFFFFFFFFu - (uint32_t)(top & 0xFFFFFFFFull));
     if ((e & 31) == lane) {  // the owner drops it and rescans its keys

@@ -18,7 +18,11 @@ __device__ __forceinline__ void simt_store(const GemmProblem& p, int row, int f,
   if (kEpi == EPI_F32_BIAS) {
     static_cast<float*>(e.out)[(size_t)row * e.ldo + f] = v0 + (e.bias ? e.bias[f] : 0.f);
   } else if (kEpi == EPI_ACT) {
-    static_cast<T*>(e.out)[(size_t)row * e.ldo + e.col0 + f] = from_f32<T>(apply_act(e.act, v0, v1));
+    const float v = apply_act(e.act, v0, v1);
+    T* o = static_cast<T*>(e.out) + (size_t)row * e.ldo + e.col0 + f;
+    const T hi = from_f32<T>(v);
+    o[0] = hi;
+    if (e.split_off) o[e.split_off] = from_f32<T>(v - to_f32<T>(hi));
   } else if (kEpi == EPI_SCALE_SCATTER) {
     const size_t orow = (size_t)e.row_slot[row];
     static_cast<T*>(e.out)[orow * e.ldo + f] = from_f32<T>(v0 * e.row_w[row]);

@@ -22,7 +22,8 @@
 // Warp roles (256 threads):
 //   warp 0      TMA producer (weights, and contiguous activation rows)
 //   warp 1      TMEM allocation and the single-thread MMA issuer
-//   warps 2-3   cp.async row gather of activations (gathered problems)
+//   warps 2-3   cp.async row gather of activations (gathered problems),
+//               completion signalled to the MMA issuer through the mbarrier
 //   warps 4-7   epilogue: tcgen05.ld -> epilogue math -> global stores
 // The smem ring has STAGES stages of one 64-wide K slice each; TMEM holds two
 // accumulator buffers so the epilogue of tile i overlaps the MMAs of tile i+1.
@@ -35,7 +36,6 @@ namespace lmoe {
 constexpr int kTcThreads = 256;
 constexpr int kTcSmemBudget = 200 * 1024;
 constexpr int kGatherThreads = 64;
-constexpr int kGatherLag = 2;  // stages of cp.async a gather thread keeps in flight
 
 template <bool kSwap_, bool kGather_, bool kDual_, int kWN_, int kEpi_>
 struct TcCfg {
@@ -56,7 +56,7 @@ struct TcCfg {
   static constexpr int FT = W_ROWS;                   // features per tile
   static constexpr int SMEM_BYTES = 1024 /*align slack*/ + STAGES * STAGE_BYTES + 512;
   static_assert(TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM allocation must be a power of two");
-  static_assert(STAGES >= kGatherLag + 2, "pipeline too shallow");
+  static_assert(STAGES >= 3, "pipeline too shallow");
   static_assert(!kSwap || kEpi == EPI_ACT || kEpi == EPI_SCALE_SCATTER, "swap epilogues");
   static_assert(kWN_ == 128 || kWN_ == 256, "weight tile");
 };
@@ -101,6 +101,7 @@ __device__ __forceinline__ void store_row32(const GemmProblem& p, int row, int f
     res = static_cast<const bf16*>(e.resid) + (size_t)row * e.ldr + f;
   }
   bf16* o = static_cast<bf16*>(e.out) + orow * e.ldo + (kEpi == EPI_ACT ? e.col0 : 0) + f;
+  const int split = (kEpi == EPI_ACT) ? e.split_off : 0;
   if (full) {
 #pragma unroll
     for (int i = 0; i < 32; i += 8) {
@@ -110,16 +111,23 @@ __device__ __forceinline__ void store_row32(const GemmProblem& p, int row, int f
 #pragma unroll
         for (int j = 0; j < 8; ++j) r[i + j] = __bfloat162float(rb[j]) + v0[i + j];
       }
-      uint4 q;
+      uint4 q, ql;
       bf16* qb = reinterpret_cast<bf16*>(&q);
+      bf16* qlb = reinterpret_cast<bf16*>(&ql);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) qb[j] = __float2bfloat16_rn(r[i + j]);
+      for (int j = 0; j < 8; ++j) {
+        qb[j] = __float2bfloat16_rn(r[i + j]);
+        qlb[j] = __float2bfloat16_rn(r[i + j] - __bfloat162float(qb[j]));
+      }
       *reinterpret_cast<uint4*>(o + i) = q;
+      if (split) *reinterpret_cast<uint4*>(o + split + i) = ql;
     }
   } else {
     for (int i = 0; i < 32 && f + i < p.F; ++i) {
       float v = (kEpi == EPI_RESID) ? __bfloat162float(res[i]) + v0[i] : r[i];
-      o[i] = __float2bfloat16_rn(v);
+      const bf16 hi = __float2bfloat16_rn(v);
+      o[i] = hi;
+      if (split) o[split + i] = __float2bfloat16_rn(v - __bfloat162float(hi));
     }
   }
 }
@@ -129,8 +137,11 @@ template <int kEpi>
 __device__ __forceinline__ void store_elem(const GemmProblem& p, int row, int f, float v0, float v1) {
   const EpiParams& e = p.epi;
   if (kEpi == EPI_ACT) {
-    static_cast<bf16*>(e.out)[(size_t)row * e.ldo + e.col0 + f] =
-        __float2bfloat16_rn(apply_act(e.act, v0, v1));
+    const float v = apply_act(e.act, v0, v1);
+    const bf16 hi = __float2bfloat16_rn(v);
+    bf16* o = static_cast<bf16*>(e.out) + (size_t)row * e.ldo + e.col0 + f;
+    o[0] = hi;
+    if (e.split_off) o[e.split_off] = __float2bfloat16_rn(v - __bfloat162float(hi));
   } else {  // EPI_SCALE_SCATTER
     const size_t orow = (size_t)__ldg(e.row_slot + row);
     static_cast<bf16*>(e.out)[orow * e.ldo + f] = __float2bfloat16_rn(v0 * __ldg(e.row_w + row));
@@ -283,13 +294,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
   } else if (warp < 4) {
     // ---------------- cp.async row gather ----------------
+    // Each thread copies 16-byte chunks of the tile's rows straight into the
+    // 128-byte-swizzled layout, then hands the stage to the MMA issuer with an
+    // mbarrier arrive that the hardware triggers when its copies have landed.
+    // The thread never waits for its own copies, so all STAGES stages can be
+    // in flight.
     if (Cfg::kGather) {
       const int gt = threadIdx.x - 64;  // 0..63
       const int q = gt & 7;             // 16-byte chunk of a 128-byte row
       const int rsub = gt >> 3;         // rows rsub, rsub + 8, ...
       const uint32_t swz = (uint32_t)((q ^ rsub) * 16);
       const bf16* A = static_cast<const bf16*>(p.A);
-      int s = 0, s_ret = 0, pending = 0;
+      int s = 0;
       uint32_t ph = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
@@ -312,24 +328,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             if (r < nload)
               cp_async_16(act + r * 128 + swz, src[i] + kb * Cfg::BK, r < rows ? 16u : 0u);
           }
-          cp_async_commit();
-          if (pending == kGatherLag) {
-            cp_async_wait<kGatherLag>();
-            fence_proxy_async_smem();
-            mbar_arrive(&full[s_ret]);
-            if (++s_ret == Cfg::STAGES) s_ret = 0;
-          } else {
-            ++pending;
-          }
+          cp_async_mbar_arrive(&full[s]);
+          mbar_arrive(&full[s]);
           if (++s == Cfg::STAGES) { s = 0; ph ^= 1; }
         }
       }
       cp_async_wait<0>();
-      fence_proxy_async_smem();
-      for (; pending > 0; --pending) {
-        mbar_arrive(&full[s_ret]);
-        if (++s_ret == Cfg::STAGES) s_ret = 0;
-      }
     }
   } else {
     // ---------------- epilogue (warps 4..7) ----------------

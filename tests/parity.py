@@ -134,12 +134,7 @@ def check_forward(w: workloads.Workload, flags: int = 0, tokens: Optional[np.nda
         O = oracle_layer(w, W, experts=experts)
         ref, z, comb = O.forward(x_host, o_idx[uniq], o_w[uniq], tokens=ut, stages=True)
         got = g_out[ut]
-        res["max_abs"] = float(np.abs(got - ref).max())
-        res["rel_l2"] = rel_l2(got, ref)
-        if w.dtype == "f32":
-            assert res["rel_l2"] <= F32_REL_L2, res
-        else:
-            assert res["max_abs"] <= BF16_MAX_ABS and res["rel_l2"] <= BF16_REL_L2, res
+        res.update(compare_outputs(got, ref, w.dtype))
         if g_z is not None:
             res["z_rel_l2"] = rel_l2(g_z[ut].astype(np.float64), z)
             assert res["z_rel_l2"] <= (1e-5 if w.dtype == "f32" else 5e-3), res
@@ -148,6 +143,34 @@ def check_forward(w: workloads.Workload, flags: int = 0, tokens: Optional[np.nda
             assert res["comb_rel_l2"] <= (1e-5 if w.dtype == "f32" else 1e-2), res
     res["expert_path"] = L.last_expert_path
     res["launches"] = L.last_launch_count
+    return res
+
+
+def compare_outputs(got: np.ndarray, ref: np.ndarray, dtype: str) -> Dict:
+    """Element-wise comparison with the stated tolerances.
+
+    bf16: max-abs <= 2e-2 and rel-L2 <= 5e-3.  Where |ref| >= 8 a bf16 output
+    cannot come within 2e-2 of the exact value whatever the arithmetic (half an
+    ulp there is >= 2^-5), so those elements are held to the same multiple of
+    the storage half-ulp that 2e-2 is of the half-ulp just below 8
+    (2e-2 / 2^-6 = 1.28): err <= 1.28 * half_ulp(ref)."""
+    err = np.abs(got - ref)
+    aref = np.abs(ref)
+    res = {"rel_l2": rel_l2(got, ref)}
+    i = int(np.argmax(err))
+    res["worst"] = (float(aref.flat[i]), float(err.flat[i]))
+    if dtype == "f32":
+        res["max_abs"] = float(err.max())
+        assert res["rel_l2"] <= F32_REL_L2, res
+        return res
+    big = aref >= 8.0
+    res["max_abs"] = float(err[~big].max()) if (~big).any() else 0.0
+    res["n_ge8"] = int(big.sum())
+    if big.any():
+        half_ulp = 2.0 ** (np.floor(np.log2(aref[big])) - 8)
+        res["max_err_over_half_ulp_ge8"] = float((err[big] / half_ulp).max())
+        assert np.all(err[big] <= BF16_MAX_ABS / 2.0 ** -6 * half_ulp), res
+    assert res["max_abs"] <= BF16_MAX_ABS and res["rel_l2"] <= BF16_REL_L2, res
     return res
 
 
