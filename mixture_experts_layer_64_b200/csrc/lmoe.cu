@@ -10,7 +10,8 @@
 //   5 shared FC1 GEMM        hs = act(x Ws1) into cat[:, l:] as bf16 hi + lo pairs
 //   6 expert FC1 (grouped)   h[r] = act(z[tok(r)] W1[e])      rows gathered by token
 //   7 expert FC2 (grouped)   ys[slot(r)] = w(r) * (h[r] W2[e])
-//   8 combine                cat[t, :l] = sum_j ys[t*k + j]   (or out = x + sum, skipped)
+//   8 combine                cat[t, :l] = sum_j ys[t*k + j]   (skipped projections:
+//                            out = x + sum (+ the shared expert, computed in fp32 at 5))
 //   9 up-projection GEMM     out = x + [comb | hs_hi | hs_lo] [Wup ; Ws2 ; Ws2]
 // Contractions run on the tcgen05 kernel (bf16) or the CUDA-core kernel
 // (fp32, or shapes the tcgen05 kernel does not take).
@@ -89,6 +90,7 @@ struct lmoe_layer {
   float* row_w = nullptr;
   void *z = nullptr, *h = nullptr, *ys = nullptr, *cat = nullptr;
   void *x_stage = nullptr, *out_stage = nullptr;
+  float* s32 = nullptr;  // [T, d] fp32 shared-expert output (projection-skip layers)
   // bookkeeping
   int last_T = -1, launches = 0, expert_path = -1;
   std::string detail;
@@ -370,6 +372,15 @@ lmoe_status run_forward(lmoe_layer* h, const void* x, void* out, int T, cudaStre
     c.p.epi.act = h->act;
     c.p.epi.split_off = h->split_shared ? ms : 0;
     LMOE_TRY(run_gemm(h, c, st));
+    if (skip) {
+      // no up-projection GEMM to carry it: s = hs Ws2 in fp32, added by the
+      // combine before the output's single rounding
+      GemmCall c2 = dense_call(GK_ROUTER, T, h->cat, h->Kup, h->Wu_t, d, h->Kup);
+      c2.p.epi.out = h->s32;
+      c2.p.epi.ldo = d;
+      c2.p.epi.bias = nullptr;
+      LMOE_TRY(run_gemm(h, c2, st));
+    }
   }
   prof_mark(h, st, 5);
   const bool swap = use_swap(h, T);
@@ -398,6 +409,7 @@ lmoe_status run_forward(lmoe_layer* h, const void* x, void* out, int T, cudaStre
   prof_mark(h, st, 7);
   {
     const void* resid = skip ? x : nullptr;
+    const float* add32 = (skip && ms > 0) ? h->s32 : nullptr;
     void* dst = skip ? out : h->cat;
     const long ldo = skip ? d : h->Kup;
     const int vec = 16 / h->es;
@@ -407,26 +419,26 @@ lmoe_status run_forward(lmoe_layer* h, const void* x, void* out, int T, cudaStre
     if (h->dtype == LMOE_BF16) {
       if (vec_ok)
         combine_kernel<bf16><<<T, threads, 0, st>>>((const bf16*)h->ys, k, l, (const bf16*)resid,
-                                                    d, (bf16*)dst, ldo);
+                                                    d, add32, (bf16*)dst, ldo);
       else
         combine_scalar_kernel<bf16><<<T, 256, 0, st>>>((const bf16*)h->ys, k, l,
-                                                       (const bf16*)resid, d, (bf16*)dst, ldo);
+                                                       (const bf16*)resid, d, add32, (bf16*)dst, ldo);
     } else {
       if (vec_ok)
         combine_kernel<float><<<T, threads, 0, st>>>((const float*)h->ys, k, l,
-                                                     (const float*)resid, d, (float*)dst, ldo);
+                                                     (const float*)resid, d, add32, (float*)dst, ldo);
       else
         combine_scalar_kernel<float><<<T, 256, 0, st>>>((const float*)h->ys, k, l,
-                                                        (const float*)resid, d, (float*)dst, ldo);
+                                                        (const float*)resid, d, add32, (float*)dst, ldo);
     }
     LMOE_CHECK_LAUNCH(h);
   }
   prof_mark(h, st, 8);
-  if (!skip || ms > 0) {
+  if (!skip) {
     GemmCall c = dense_call(GK_UP, T, h->cat, h->Kup, h->Wu_t, d, h->Kup);
     c.p.epi.out = out;
     c.p.epi.ldo = d;
-    c.p.epi.resid = skip ? out : x;  // skipped projections: out already holds x + comb
+    c.p.epi.resid = x;
     c.p.epi.ldr = d;
     LMOE_TRY(run_gemm(h, c, st));
   }
@@ -462,6 +474,7 @@ void free_workspace(lmoe_layer* h) {
   free_ptr(h->cat);
   free_ptr(h->x_stage);
   free_ptr(h->out_stage);
+  free_ptr(h->s32);
   h->max_T = 0;
 }
 
@@ -634,6 +647,7 @@ lmoe_status lmoe_reserve(lmoe_layer* h, int max_T) {
   if (h->Kup > 0) ALLOC(h->cat, T * h->Kup * es);
   ALLOC(h->x_stage, T * h->d * es);
   ALLOC(h->out_stage, T * h->d * es);
+  if (skip && h->shared_m > 0) ALLOC(h->s32, T * h->d * sizeof(float));
 #undef ALLOC
   LMOE_CUDA(h, cudaMemset(h->bitmap, 0, (size_t)h->N * W * sizeof(uint32_t)));
   LMOE_CUDA(h, cudaMemset(h->done, 0, sizeof(unsigned)));

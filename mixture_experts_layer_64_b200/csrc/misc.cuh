@@ -11,9 +11,12 @@ namespace lmoe {
 // slot order, rounded once.  ys rows are in slot order (t*k + j), so each
 // token's k rows are contiguous.  One block per token, VEC elements per thread
 // per step (16-byte accesses).
+// With add32 (fp32, row stride ldr) that addend joins the sum before the one
+// rounding: the projection-skip layer adds its shared expert this way.
 template <typename T>
 __global__ void __launch_bounds__(256) combine_kernel(const T* __restrict__ ys, int k, int l,
                                                       const T* __restrict__ resid, long ldr,
+                                                      const float* __restrict__ add32,
                                                       T* __restrict__ out, long ldo) {
   constexpr int VEC = 16 / sizeof(T);
   const int t = blockIdx.x;
@@ -28,6 +31,10 @@ __global__ void __launch_bounds__(256) combine_kernel(const T* __restrict__ ys, 
     } else {
 #pragma unroll
       for (int v = 0; v < VEC; ++v) acc[v] = 0.f;
+    }
+    if (add32) {
+#pragma unroll
+      for (int v = 0; v < VEC; ++v) acc[v] += add32[(size_t)t * ldr + c + v];
     }
     for (int j = 0; j < k; ++j) {
       const uint4 yv = __ldg(reinterpret_cast<const uint4*>(base + (size_t)j * l + c));
@@ -47,10 +54,12 @@ __global__ void __launch_bounds__(256) combine_kernel(const T* __restrict__ ys, 
 template <typename T>
 __global__ void __launch_bounds__(256) combine_scalar_kernel(const T* __restrict__ ys, int k, int l,
                                                              const T* __restrict__ resid, long ldr,
+                                                             const float* __restrict__ add32,
                                                              T* __restrict__ out, long ldo) {
   const int t = blockIdx.x;
   for (int c = threadIdx.x; c < l; c += blockDim.x) {
     float acc = resid ? to_f32<T>(resid[(size_t)t * ldr + c]) : 0.f;
+    if (add32) acc += add32[(size_t)t * ldr + c];
     for (int j = 0; j < k; ++j) acc += to_f32<T>(ys[((size_t)t * k + j) * l + c]);
     out[(size_t)t * ldo + c] = from_f32<T>(acc);
   }
