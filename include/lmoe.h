@@ -211,6 +211,38 @@ lmoe_status lmoe_profile_end(lmoe_layer* h, float* ms, int capacity, int* n_forw
                              int* n_stages);
 const char* lmoe_stage_name(int stage);
 
+/*
+ * lmoe_route_only_noalloc -- lmoe_route_only without a handle and without
+ * allocating device memory.  The paper has no counterpart: this is an
+ * interface for callers, not a step of the method.
+ *
+ * Some callers cannot call cudaMalloc: an inference server that reserves all
+ * of HBM for its own pool up front (a driver allocation would fail or
+ * fragment it), or code running where the device-wide synchronisation that
+ * cudaMalloc / cudaFree imply is not allowed.  This call runs the routing
+ * kernels of lmoe_route_only (same arguments and results: idx, w, offsets,
+ * perm for N experts and top-k) with their scratch in a fixed file-scope
+ * device array of LMOE_NOALLOC_SCRATCH_BYTES, which every GPU that loads the
+ * library holds until the process exits.  It calls no cudaMalloc, cudaFree or
+ * other allocating routine.
+ *   Limits: N <= LMOE_MAX_EXPERTS, k <= LMOE_MAX_TOPK and
+ *   N * ceil(T / 32) <= LMOE_NOALLOC_MAX_WORDS (e.g. T <= 8192 with N = 1024,
+ *   T <= 16384 with N = 512); beyond them it returns LMOE_ERR_UNSUPPORTED and
+ *   enqueues nothing.
+ *   Setup: the first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call
+ *   before any stream capture.
+ *   Sharing: every call uses the same array and clears the parts that must
+ *   start at zero, so calls that overlap on the GPU (other streams, other
+ *   host threads) race and must be serialised by the caller.
+ * Errors: INVALID_ARG (bad sizes, NULL pointers), UNSUPPORTED (over the
+ * limits), CUDA.
+ */
+#define LMOE_NOALLOC_MAX_WORDS     262144u
+#define LMOE_NOALLOC_SCRATCH_BYTES 3211264u
+lmoe_status lmoe_route_only_noalloc(const float* logits, int T, int N, int k, int* idx, float* w,
+                                    int* offsets, int* perm, lmoe_stream_t stream);
+
 /* Kernel launches the last lmoe_forward enqueued (library kernels only). */
 int lmoe_last_launch_count(const lmoe_layer* h);
 

@@ -12,7 +12,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB_PATH = os.path.join(HERE, "liblmoe.so")
-SOURCES = [os.path.join(CSRC, "lmoe.cu")]
+SOURCES = [os.path.join(CSRC, "lmoe.cu"), os.path.join(CSRC, "noalloc.cu")]
 DEPS = SOURCES + [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith(".cuh")] + [
     os.path.join(ROOT, "include", "lmoe.h")]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")

@@ -35,7 +35,7 @@ __device__ __forceinline__ float from_orderable_bits(uint32_t u) {
 
 // logits [T, N] fp32 -> idx [T, k], w [T, k]; bitmap [N, W] gets bit t of
 // token t set in the row of every chosen expert (W = ceil(T/32) words).
-__global__ void __launch_bounds__(256) topk_softmax_kernel(const float* __restrict__ logits, int T,
+static __global__ void __launch_bounds__(256) topk_softmax_kernel(const float* __restrict__ logits, int T,
                                                            int N, int k, int* __restrict__ idx,
                                                            float* __restrict__ w,
                                                            uint32_t* __restrict__ bitmap, int W,
@@ -94,7 +94,7 @@ __global__ void __launch_bounds__(256) topk_softmax_kernel(const float* __restri
 
 // Word prefix + bits: wp[e][wd] = {set bits of expert e in words < wd, word wd}.
 // Also zeroes the bitmap.  The last block scans the loads.
-__global__ void __launch_bounds__(256) group_count_kernel(uint32_t* __restrict__ bitmap,
+static __global__ void __launch_bounds__(256) group_count_kernel(uint32_t* __restrict__ bitmap,
                                                           uint2* __restrict__ wp, int N, int W,
                                                           int* __restrict__ counts,
                                                           int* __restrict__ offsets,
@@ -167,7 +167,7 @@ __global__ void __launch_bounds__(256) group_count_kernel(uint32_t* __restrict__
 }
 
 // row(t, j) = offsets[e] + rank of t among the tokens routed to e.
-__global__ void __launch_bounds__(256) group_rank_kernel(
+static __global__ void __launch_bounds__(256) group_rank_kernel(
     const int* __restrict__ idx, const float* __restrict__ w, const uint2* __restrict__ wp,
     const int* __restrict__ offsets, int T, int k, int N, int W, int* __restrict__ row_tok,
     int* __restrict__ row_slot, float* __restrict__ row_w, int debug, int* err) {

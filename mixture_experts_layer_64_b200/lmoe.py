@@ -28,7 +28,8 @@ EXPORTS = ["lmoe_create", "lmoe_set_weights", "lmoe_reserve", "lmoe_forward", "l
            "lmoe_route_only", "lmoe_router_logits", "lmoe_stage_bytes", "lmoe_debug_dump",
            "lmoe_last_error", "lmoe_profile_begin", "lmoe_profile_end", "lmoe_stage_name",
            "lmoe_last_launch_count", "lmoe_last_expert_path", "lmoe_status_string",
-           "lmoe_error_detail", "lmoe_destroy"]
+           "lmoe_error_detail", "lmoe_destroy", "lmoe_route_only_noalloc"]
+NOALLOC_MAX_WORDS = 262144
 
 
 class LmoeError(RuntimeError):
@@ -70,6 +71,7 @@ def lib() -> ctypes.CDLL:
             "lmoe_status_string": ([I], ctypes.c_char_p),
             "lmoe_error_detail": ([P], ctypes.c_char_p),
             "lmoe_destroy": ([P], None),
+            "lmoe_route_only_noalloc": ([P, I, I, I, P, P, P, P, P], I),
         }
         for name, (args, res) in sig.items():
             f = getattr(L, name)
@@ -94,6 +96,27 @@ def _ptr(t: Optional[torch.Tensor]):
 def _stream(stream: Optional[torch.cuda.Stream]):
     s = stream if stream is not None else torch.cuda.current_stream()
     return ctypes.c_void_p(s.cuda_stream)
+
+
+def route_only_noalloc(logits: torch.Tensor, k: int, stream=None) -> Dict[str, torch.Tensor]:
+    """lmoe_route_only_noalloc: the routing steps without a layer handle and
+    without any device allocation inside the library (its scratch is a fixed
+    device array; calls overlapping on the GPU race).  The outputs are
+    allocated here by torch, as a caller that owns its memory would."""
+    if logits.dtype != torch.float32 or logits.dim() != 2 or not logits.is_cuda:
+        raise ValueError("logits must be a [T, N] fp32 CUDA tensor")
+    logits = logits.contiguous()
+    T, N = logits.shape
+    dev = logits.device
+    idx = torch.empty((T, k), dtype=torch.int32, device=dev)
+    w = torch.empty((T, k), dtype=torch.float32, device=dev)
+    offsets = torch.empty((N + 1,), dtype=torch.int32, device=dev)
+    perm = torch.empty((T * k,), dtype=torch.int32, device=dev)
+    st = lib().lmoe_route_only_noalloc(_ptr(logits), T, N, k, _ptr(idx), _ptr(w), _ptr(offsets),
+                                       _ptr(perm), _stream(stream))
+    if st != OK:
+        raise LmoeError(st, "lmoe_route_only_noalloc")
+    return {"idx": idx, "w": w, "offsets": offsets, "perm": perm}
 
 
 class LatentMoELayer:
