@@ -43,17 +43,24 @@ METRIC = "LatentMoE layer tokens/sec at decode & prefill T; HBM GB/s / tensor-pi
 UNIT = "tokens/s"
 DEFAULT_WORKLOAD = "std-moe-decode"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNEL_SOURCES = ["mixture_experts_layer_64_b200/csrc/" + f for f in
-                  ("common.cuh", "tc_gemm.cuh", "simt_gemm.cuh", "routing.cuh", "misc.cuh", "lmoe.cu")]
+_CSRC = "mixture_experts_layer_64_b200/csrc/"
+_GEMM_SRC = (_CSRC + "common.cuh", _CSRC + "tc_gemm.cuh")
+# device code of each stage's kernel: recorded DRAM traffic is trusted only
+# while these files are unchanged since the capture
+STAGE_SOURCES = {"router": _GEMM_SRC, "down_proj": _GEMM_SRC, "shared_fc1": _GEMM_SRC,
+                 "expert_fc1": _GEMM_SRC, "expert_fc2": _GEMM_SRC, "up_proj": _GEMM_SRC,
+                 "topk": (_CSRC + "common.cuh", _CSRC + "routing.cuh"),
+                 "group": (_CSRC + "common.cuh", _CSRC + "routing.cuh"),
+                 "combine": (_CSRC + "common.cuh", _CSRC + "misc.cuh")}
 
 
 def log(*a):
     print(*a, file=sys.stderr, flush=True)
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(stage: str) -> str:
     h = hashlib.sha256()
-    for f in KERNEL_SOURCES:
+    for f in STAGE_SOURCES[stage]:
         with open(os.path.join(ROOT, f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -77,7 +84,7 @@ def recorded_traffic(workload: str, stage: str):
     with open(p) as fh:
         d = json.load(fh)
     rec = d.get(workload, {}).get(stage)
-    if not rec or rec.get("kernel_sources") != kernel_source_hash():
+    if not rec or rec.get("kernel_sources") != kernel_source_hash(stage):
         return None
     return rec.get("dram_bytes_per_launch")
 
@@ -399,7 +406,8 @@ def run_ours(args):
                 "gpu_launches": launches_per_step * args.steps,
                 "roofline": roofline, "cpu_baseline": cpu_baseline, "clocks": clocks,
                 "expert_path": ["cuda-core", "tcgen05 token-tiled",
-                                "tcgen05 weight-stationary"][max(0, L.last_expert_path)]}
+                                "tcgen05 weight-stationary",
+                                "tcgen05 token-tiled, 2-SM CTA pairs"][max(0, L.last_expert_path)]}
         print(json.dumps(line), flush=True)
     L.close()
     if pg:

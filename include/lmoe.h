@@ -70,6 +70,8 @@ typedef enum { LMOE_F32 = 0, LMOE_BF16 = 1 } lmoe_dtype;
 #define LMOE_FORCE_SWAP    0x8u  /* always use the weight-stationary (swap-AB)
                                     expert kernels (for testing)                */
 #define LMOE_FORCE_NOSWAP  0x10u /* never use them (for testing)                */
+#define LMOE_FORCE_NOPAIR  0x20u /* never use the 2-SM (CTA pair) tensor-core
+                                    kernels (for testing)                       */
 
 /* Limits of this build. */
 #define LMOE_MAX_EXPERTS 1024
@@ -247,7 +249,8 @@ lmoe_status lmoe_route_only_noalloc(const float* logits, int T, int N, int k, in
 int lmoe_last_launch_count(const lmoe_layer* h);
 
 /* Which expert kernels the last lmoe_forward used: 0 CUDA-core, 1 tcgen05
- * token-tiled, 2 tcgen05 weight-stationary (swap-AB). */
+ * token-tiled, 2 tcgen05 weight-stationary (swap-AB), 3 tcgen05 token-tiled on
+ * CTA pairs (2-SM MMA). */
 int lmoe_last_expert_path(const lmoe_layer* h);
 
 const char* lmoe_status_string(lmoe_status s);

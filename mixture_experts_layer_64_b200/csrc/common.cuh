@@ -36,6 +36,9 @@ struct EpiParams {
   long ldr;
   const int* row_slot;    // EPI_SCALE_SCATTER: tile row -> output row
   const float* row_w;     // EPI_SCALE_SCATTER: tile row -> gate weight
+  void* scat;             // EPI_ACT: also copy each output row t to rows
+  const int* slot_row;    //   scat[slot_row[t * scat_k + j]], j < scat_k (row stride ldo):
+  int scat_k;             //   latent rows written straight into expert order
   int split_off;          // EPI_ACT, bf16: > 0 also writes v - bf16(v) (rounded) at
                           // column col0 + split_off + f, so that hi + lo carries the
                           // value to ~16 significant bits through the next bf16 GEMM
@@ -54,6 +57,7 @@ struct GemmProblem {
   int G;
   int M;                  // rows of the dense group (offsets == NULL)
   int max_row_tiles;      // host upper bound on row tiles (grid sizing)
+  int row_tile;           // rows per tile: 128, or 256 for CTA pairs (tile_prefix must match)
   const void* A;          // activations, row stride lda
   long lda;
   const int* gather;      // row -> source row of A, or NULL (identity)
@@ -96,8 +100,8 @@ __device__ __forceinline__ void locate_row_tile(const GemmProblem& p, int rt, in
                                                 int& rows) {
   if (p.offsets == nullptr) {
     g = 0;
-    row0 = rt * kRowTile;
-    rows = min(kRowTile, p.M - row0);
+    row0 = rt * p.row_tile;
+    rows = min(p.row_tile, p.M - row0);
     return;
   }
   int lo = 0, hi = p.G - 1;  // largest g with tile_prefix[g] <= rt
@@ -107,12 +111,12 @@ __device__ __forceinline__ void locate_row_tile(const GemmProblem& p, int rt, in
   }
   g = lo;
   const int start = __ldg(p.offsets + g), end = __ldg(p.offsets + g + 1);
-  row0 = start + (rt - __ldg(p.tile_prefix + g)) * kRowTile;
-  rows = min(kRowTile, end - row0);
+  row0 = start + (rt - __ldg(p.tile_prefix + g)) * p.row_tile;
+  rows = min(p.row_tile, end - row0);
 }
 
 __device__ __forceinline__ int total_row_tiles(const GemmProblem& p) {
-  if (p.offsets == nullptr) return (p.M + kRowTile - 1) / kRowTile;
+  if (p.offsets == nullptr) return (p.M + p.row_tile - 1) / p.row_tile;
   return *((volatile const int*)(p.tile_prefix + p.G));
 }
 
@@ -231,6 +235,77 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// ---- clusters (CTA pairs of the 2-SM MMA) ------------------------------------
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_id_x() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_count_x() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%nclusterid.x;" : "=r"(r));
+  return r;
+}
+// shared::cluster address of the same shared variable in CTA `rank` of the cluster
+__device__ __forceinline__ uint32_t cluster_map(const void* smem_ptr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(smem_ptr)), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                   : "memory");
+}
+// arrive on an mbarrier given by its shared::cluster address (possibly in the peer CTA)
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait with cluster-scope acquire (arrivals may come from the peer CTA).
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity,
+                                                  volatile int* abort_flag, int* err) {
+  if (mbar_try_wait_cluster(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    if ((it & 255u) == 0) {
+      if (*abort_flag) return false;
+      if (globaltimer() - t0 > kWaitLimitNs) {
+        *abort_flag = 1;
+        set_error(err, LMOE_DEVERR_WAIT_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+// 2-SM TMA load into this CTA's shared memory; completion is counted on the
+// mbarrier at shared::cluster address `bar_cluster` (the pair's leader).
+__device__ __forceinline__ void tma_load_2d_pair(const CUtensorMap* map, uint32_t bar_cluster,
+                                                 void* smem_dst, int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.cta_group::2"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(c0), "r"(c1)
+      : "memory");
+}
+
 // tcgen05 (5th-generation tensor cores, tensor memory).
 __device__ __forceinline__ void tmem_alloc(uint32_t* smem_slot, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -267,6 +342,40 @@ __device__ __forceinline__ void tc_commit(uint64_t* bar) {
                    smem_u32(bar))
                : "memory");
 }
+// 2-SM variants: the pair's TMEM is allocated by one warp in each CTA; MMAs
+// are issued by the leader and read operands from both CTAs' shared memory.
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* smem_slot, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                   smem_u32(smem_slot)),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tc_mma_bf16_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                                 uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Arrive on `bar` (same offset) in every CTA of ctaMask once the pair's
+// previously issued MMAs finish.
+__device__ __forceinline__ void tc_commit_pair_mc(uint64_t* bar, uint16_t cta_mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 "
+      "[%0], %1;" ::"r"(smem_u32(bar)),
+      "h"(cta_mask)
+      : "memory");
+}
+
 __device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 // 32 lanes x 32 consecutive fp32 columns: thread i of the warp receives lane

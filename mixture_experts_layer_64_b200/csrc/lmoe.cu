@@ -83,12 +83,12 @@ struct lmoe_layer {
   float* w = nullptr;
   uint32_t* bitmap = nullptr;
   uint2* wp = nullptr;
-  int *counts = nullptr, *offsets = nullptr, *tile_prefix = nullptr;
+  int *counts = nullptr, *offsets = nullptr, *tile_prefix = nullptr, *tile_prefix2 = nullptr;
   unsigned* done = nullptr;
   int* err = nullptr;
-  int *row_tok = nullptr, *row_slot = nullptr;
+  int *row_tok = nullptr, *row_slot = nullptr, *slot_row = nullptr;
   float* row_w = nullptr;
-  void *z = nullptr, *h = nullptr, *ys = nullptr, *cat = nullptr;
+  void *z = nullptr, *zs = nullptr, *h = nullptr, *ys = nullptr, *cat = nullptr;
   void *x_stage = nullptr, *out_stage = nullptr;
   float* s32 = nullptr;  // [T, d] fp32 shared-expert output (projection-skip layers)
   // bookkeeping
@@ -145,6 +145,7 @@ struct GemmCall {
   long a_rows;  // rows of A (TMA bounds)
   long b_rows;  // rows of B (TMA bounds)
   bool swap;    // weight-stationary expert kernels
+  bool pair;    // 2-SM token-tiled kernels on CTA pairs (256-row tiles)
 };
 
 bool encode_map(CUtensorMap* map, const void* ptr, long rows, int cols, long ld, int box_rows) {
@@ -185,6 +186,62 @@ lmoe_status launch_tc(lmoe_layer* h, const GemmCall& c, cudaStream_t st) {
   const int grid = (int)std::max(1L, std::min<long>(h->num_sms, tiles));
   tc_gemm_kernel<Cfg><<<grid, kTcThreads, Cfg::SMEM_BYTES, st>>>(ta, tb, c.p);
   LMOE_CHECK_LAUNCH(h);
+  return LMOE_OK;
+}
+
+template <class Cfg>
+lmoe_status launch_pair(lmoe_layer* h, const GemmCall& c, cudaStream_t st) {
+  static bool attr_done = false;
+  static int max_clusters = 0;
+  if (!attr_done) {
+    LMOE_CUDA(h, cudaFuncSetAttribute(tc_gemm_pair_kernel<Cfg>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      Cfg::SMEM_BYTES));
+    LMOE_CUDA(h, cudaFuncSetAttribute(tc_gemm_pair_kernel<Cfg>,
+                                      cudaFuncAttributeNonPortableClusterSizeAllowed, 0));
+    cudaLaunchConfig_t q = {};
+    cudaLaunchAttribute qa[1];
+    qa[0].id = cudaLaunchAttributeClusterDimension;
+    qa[0].val.clusterDim.x = 2;
+    qa[0].val.clusterDim.y = 1;
+    qa[0].val.clusterDim.z = 1;
+    q.gridDim = dim3(2 * (h->num_sms / 2), 1, 1);
+    q.blockDim = dim3(kTcThreads, 1, 1);
+    q.dynamicSmemBytes = Cfg::SMEM_BYTES;
+    q.attrs = qa;
+    q.numAttrs = 1;
+    LMOE_CUDA(h, cudaOccupancyMaxActiveClusters(&max_clusters, tc_gemm_pair_kernel<Cfg>, &q));
+    if (max_clusters < 1) {
+      h->detail = "no CTA pair of the 2-SM kernel fits on the device";
+      return LMOE_ERR_UNSUPPORTED;
+    }
+    attr_done = true;
+  }
+  CUtensorMap ta, tb;
+  std::memset(&ta, 0, sizeof ta);
+  std::memset(&tb, 0, sizeof tb);
+  if (!encode_map(&ta, c.p.A, c.a_rows, c.p.K, c.p.lda, 128) ||
+      !encode_map(&tb, c.p.B, c.b_rows, c.p.K, c.p.K, 128)) {
+    h->detail = "cuTensorMapEncodeTiled failed";
+    return LMOE_ERR_CUDA;
+  }
+  const long NT = (c.p.F + Cfg::FT - 1) / Cfg::FT;
+  const long tiles = (long)c.p.max_row_tiles * NT;
+  const long clusters = std::max(1L, std::min<long>(max_clusters, tiles));
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3((unsigned)(2 * clusters), 1, 1);
+  cfg.blockDim = dim3(kTcThreads, 1, 1);
+  cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  LMOE_CUDA(h, cudaLaunchKernelEx(&cfg, tc_gemm_pair_kernel<Cfg>, ta, tb, c.p));
+  ++h->launches;
   return LMOE_OK;
 }
 
@@ -232,12 +289,36 @@ bool tc_eligible(const lmoe_layer* h, const GemmCall& c) {
 
 lmoe_status run_gemm(lmoe_layer* h, GemmCall c, cudaStream_t st, int* path = nullptr) {
   c.p.err = h->err;
+  if (c.pair && c.p.gather != nullptr) {
+    // the pair kernels read activations with TMA only
+    c.pair = false;
+    c.p.row_tile = kRowTile;
+    c.p.tile_prefix = h->tile_prefix;
+  }
   if (!tc_eligible(h, c)) {
+    if (c.pair) {  // the CUDA-core kernel tiles by 128 rows
+      c.pair = false;
+      c.p.row_tile = kRowTile;
+      c.p.tile_prefix = h->tile_prefix;
+      if (!c.p.offsets) c.p.max_row_tiles = (c.p.M + kRowTile - 1) / kRowTile;
+      else c.p.max_row_tiles = (int)((c.a_rows + kRowTile - 1) / kRowTile + h->N);
+    }
     if (path) *path = 0;
     return h->dtype == LMOE_F32 ? dispatch_simt<float>(h, c, st) : dispatch_simt<bf16>(h, c, st);
   }
   const bool dual = c.p.dual_offset > 0;
-  if (path) *path = c.swap ? 2 : 1;
+  if (path) *path = c.pair ? 3 : (c.swap ? 2 : 1);
+  if (c.pair) {
+    switch (c.kind) {
+      case GK_DENSE_ACT:
+      case GK_FC1:
+        return dual ? launch_pair<TcPairCfg<true, EPI_ACT>>(h, c, st)
+                    : launch_pair<TcPairCfg<false, EPI_ACT>>(h, c, st);
+      case GK_FC2: return launch_pair<TcPairCfg<false, EPI_SCALE_SCATTER>>(h, c, st);
+      case GK_UP: return launch_pair<TcPairCfg<false, EPI_RESID>>(h, c, st);
+      case GK_ROUTER: return launch_pair<TcPairCfg<false, EPI_F32_BIAS>>(h, c, st);
+    }
+  }
   switch (c.kind) {
     case GK_ROUTER: return launch_tc<TcCfg<false, false, false, 128, EPI_F32_BIAS>>(h, c, st);
     case GK_DENSE_ACT:
@@ -264,6 +345,7 @@ GemmCall dense_call(GemmKind kind, int M, const void* A, long lda, const void* B
   c.p.M = M;
   c.p.G = 1;
   c.p.max_row_tiles = (M + kRowTile - 1) / kRowTile;
+  c.p.row_tile = kRowTile;
   c.p.A = A;
   c.p.lda = lda;
   c.p.B = B;
@@ -273,6 +355,19 @@ GemmCall dense_call(GemmKind kind, int M, const void* A, long lda, const void* B
   c.b_rows = F;
   c.p.epi.act = ACT_NONE;
   return c;
+}
+
+// Switches a call to CTA pairs: 256-row tiles (and their tile counts).
+void make_pair(const lmoe_layer* h, GemmCall& c) {
+  c.pair = true;
+  c.p.row_tile = 2 * kRowTile;
+  if (c.p.offsets) {
+    c.p.tile_prefix = h->tile_prefix2;
+    const long R = (long)c.a_rows;
+    c.p.max_row_tiles = (int)((R + 2 * kRowTile - 1) / (2 * kRowTile) + h->N);
+  } else {
+    c.p.max_row_tiles = (c.p.M + 2 * kRowTile - 1) / (2 * kRowTile);
+  }
 }
 
 GemmCall grouped_call(const lmoe_layer* h, GemmKind kind, int T, const void* A, long lda,
@@ -285,6 +380,7 @@ GemmCall grouped_call(const lmoe_layer* h, GemmKind kind, int T, const void* A, 
   c.p.tile_prefix = h->tile_prefix;
   c.p.G = h->N;
   c.p.max_row_tiles = (int)((R + kRowTile - 1) / kRowTile + h->N);
+  c.p.row_tile = kRowTile;
   c.p.A = A;
   c.p.lda = lda;
   c.p.gather = gather;
@@ -312,8 +408,8 @@ void prof_mark(lmoe_layer* h, cudaStream_t st, int i) {
 // ---- the routing steps ---------------------------------------------------------
 
 lmoe_status run_routing(lmoe_layer* h, const float* logits, int T, int* idx, float* w,
-                        int* offsets, int* row_tok, int* row_slot, float* row_w, cudaStream_t st,
-                        bool marks) {
+                        int* offsets, int* row_tok, int* row_slot, float* row_w, int* slot_row,
+                        int* tile_prefix2, cudaStream_t st, bool marks) {
   const int W = (T + 31) / 32;
   const int debug = (h->flags & LMOE_DEBUG_CHECKS) ? 1 : 0;
   topk_softmax_kernel<<<(T + 7) / 8, 256, 0, st>>>(logits, T, h->N, h->k, idx, w, h->bitmap, W,
@@ -321,11 +417,11 @@ lmoe_status run_routing(lmoe_layer* h, const float* logits, int T, int* idx, flo
   LMOE_CHECK_LAUNCH(h);
   if (marks) prof_mark(h, st, 2);
   group_count_kernel<<<(h->N + 7) / 8, 256, 0, st>>>(h->bitmap, h->wp, h->N, W, h->counts, offsets,
-                                                     h->tile_prefix, h->done);
+                                                     h->tile_prefix, tile_prefix2, h->done);
   LMOE_CHECK_LAUNCH(h);
   const long P = (long)T * h->k;
   group_rank_kernel<<<(unsigned)((P + 255) / 256), 256, 0, st>>>(
-      idx, w, h->wp, offsets, T, h->k, h->N, W, row_tok, row_slot, row_w, debug, h->err);
+      idx, w, h->wp, offsets, T, h->k, h->N, W, row_tok, row_slot, row_w, slot_row, debug, h->err);
   LMOE_CHECK_LAUNCH(h);
   return LMOE_OK;
 }
@@ -335,6 +431,8 @@ lmoe_status run_router(lmoe_layer* h, const void* x, float* logits, int T, cudaS
   c.p.epi.out = logits;
   c.p.epi.ldo = h->N;
   c.p.epi.bias = h->bias;
+  if (h->dtype == LMOE_BF16 && T >= 1024 && !(h->flags & (LMOE_FORCE_SIMT | LMOE_FORCE_NOPAIR)))
+    make_pair(h, c);
   return run_gemm(h, c, st);
 }
 
@@ -353,12 +451,25 @@ lmoe_status run_forward(lmoe_layer* h, const void* x, void* out, int T, cudaStre
   LMOE_TRY(run_router(h, x, h->logits, T, st));
   prof_mark(h, st, 1);
   LMOE_TRY(run_routing(h, h->logits, T, h->idx, h->w, h->offsets, h->row_tok, h->row_slot,
-                       h->row_w, st, true));
+                       h->row_w, h->slot_row, h->tile_prefix2, st, true));
   prof_mark(h, st, 3);
+  const bool swap = use_swap(h, T);
+  const bool pairs_ok = h->dtype == LMOE_BF16 && !(h->flags & (LMOE_FORCE_SIMT | LMOE_FORCE_NOPAIR));
+  // CTA pairs for the dense GEMMs once there are enough rows to fill them,
+  // and for the token-tiled expert GEMMs (their FC1 then reads the latent
+  // rows in expert order, written by the down-projection's epilogue)
+  const bool pair_dense = pairs_ok && T >= 1024;
+  const bool pair_experts = pairs_ok && !swap && !skip && h->zs != nullptr;
   if (!skip) {
     GemmCall c = dense_call(GK_DENSE_ACT, T, x, d, h->Wd_t, l, d);
     c.p.epi.out = h->z;
     c.p.epi.ldo = l;
+    if (pair_experts) {
+      c.p.epi.scat = h->zs;
+      c.p.epi.slot_row = h->slot_row;
+      c.p.epi.scat_k = k;
+    }
+    if (pair_dense) make_pair(h, c);
     LMOE_TRY(run_gemm(h, c, st));
   }
   prof_mark(h, st, 4);
@@ -371,6 +482,7 @@ lmoe_status run_forward(lmoe_layer* h, const void* x, void* out, int T, cudaStre
     c.p.epi.col0 = skip ? 0 : l;
     c.p.epi.act = h->act;
     c.p.epi.split_off = h->split_shared ? ms : 0;
+    if (pair_dense) make_pair(h, c);
     LMOE_TRY(run_gemm(h, c, st));
     if (skip) {
       // no up-projection GEMM to carry it: s = hs Ws2 in fp32, added by the
@@ -383,10 +495,13 @@ lmoe_status run_forward(lmoe_layer* h, const void* x, void* out, int T, cudaStre
     }
   }
   prof_mark(h, st, 5);
-  const bool swap = use_swap(h, T);
   {
     const void* A = skip ? x : h->z;
-    GemmCall c = grouped_call(h, GK_FC1, T, A, skip ? d : l, T, h->row_tok, h->W1_t, h->m_in, m, l);
+    GemmCall c = pair_experts
+                     ? grouped_call(h, GK_FC1, T, h->zs, l, R, nullptr, h->W1_t, h->m_in, m, l)
+                     : grouped_call(h, GK_FC1, T, A, skip ? d : l, T, h->row_tok, h->W1_t,
+                                    h->m_in, m, l);
+    if (pair_experts) make_pair(h, c);
     c.swap = swap;
     c.p.dual_offset = h->act == LMOE_ACT_SWIGLU ? m : 0;
     c.p.epi.out = h->h;
@@ -399,6 +514,7 @@ lmoe_status run_forward(lmoe_layer* h, const void* x, void* out, int T, cudaStre
   prof_mark(h, st, 6);
   {
     GemmCall c = grouped_call(h, GK_FC2, T, h->h, m, R, nullptr, h->W2_t, l, l, m);
+    if (pair_experts) make_pair(h, c);
     c.swap = swap;
     c.p.epi.out = h->ys;
     c.p.epi.ldo = l;
@@ -440,6 +556,7 @@ lmoe_status run_forward(lmoe_layer* h, const void* x, void* out, int T, cudaStre
     c.p.epi.ldo = d;
     c.p.epi.resid = x;
     c.p.epi.ldr = d;
+    if (pair_dense) make_pair(h, c);
     LMOE_TRY(run_gemm(h, c, st));
   }
   prof_mark(h, st, 9);
@@ -463,6 +580,9 @@ void free_workspace(lmoe_layer* h) {
   free_ptr(h->counts);
   free_ptr(h->offsets);
   free_ptr(h->tile_prefix);
+  free_ptr(h->tile_prefix2);
+  free_ptr(h->slot_row);
+  free_ptr(h->zs);
   free_ptr(h->done);
   free_ptr(h->err);
   free_ptr(h->row_tok);
@@ -543,7 +663,7 @@ lmoe_status lmoe_create(int d, int l, int N, int k, int m, lmoe_act act, int sha
   if (!out) return LMOE_ERR_INVALID_ARG;
   *out = nullptr;
   const unsigned known = LMOE_SKIP_PROJ | LMOE_DEBUG_CHECKS | LMOE_FORCE_SIMT | LMOE_FORCE_SWAP |
-                         LMOE_FORCE_NOSWAP;
+                         LMOE_FORCE_NOSWAP | LMOE_FORCE_NOPAIR;
   if (d <= 0 || l <= 0 || N <= 0 || k <= 0 || m <= 0 || shared_m < 0) return LMOE_ERR_INVALID_ARG;
   if (k > N || (flags & ~known)) return LMOE_ERR_INVALID_ARG;
   if (act != LMOE_ACT_SILU && act != LMOE_ACT_SWIGLU && act != LMOE_ACT_RELU2) return LMOE_ERR_INVALID_ARG;
@@ -636,12 +756,17 @@ lmoe_status lmoe_reserve(lmoe_layer* h, int max_T) {
   ALLOC(h->counts, (size_t)h->N * sizeof(int));
   ALLOC(h->offsets, (size_t)(h->N + 1) * sizeof(int));
   ALLOC(h->tile_prefix, (size_t)(h->N + 1) * sizeof(int));
+  ALLOC(h->tile_prefix2, (size_t)(h->N + 1) * sizeof(int));
+  ALLOC(h->slot_row, R * sizeof(int));
   ALLOC(h->done, sizeof(unsigned));
   ALLOC(h->err, sizeof(int));
   ALLOC(h->row_tok, R * sizeof(int));
   ALLOC(h->row_slot, R * sizeof(int));
   ALLOC(h->row_w, R * sizeof(float));
   if (!skip) ALLOC(h->z, T * h->l * es);
+  // latent rows in expert order, for the CTA-pair expert kernels (bf16 only)
+  if (!skip && h->dtype == LMOE_BF16 && !(h->flags & (LMOE_FORCE_SIMT | LMOE_FORCE_NOPAIR)))
+    ALLOC(h->zs, R * h->l * es);
   ALLOC(h->h, R * h->m * es);
   ALLOC(h->ys, R * h->l * es);
   if (h->Kup > 0) ALLOC(h->cat, T * h->Kup * es);
@@ -654,6 +779,7 @@ lmoe_status lmoe_reserve(lmoe_layer* h, int max_T) {
   LMOE_CUDA(h, cudaMemset(h->err, 0, sizeof(int)));
   LMOE_CUDA(h, cudaMemset(h->offsets, 0, (size_t)(h->N + 1) * sizeof(int)));
   LMOE_CUDA(h, cudaMemset(h->tile_prefix, 0, (size_t)(h->N + 1) * sizeof(int)));
+  LMOE_CUDA(h, cudaMemset(h->tile_prefix2, 0, (size_t)(h->N + 1) * sizeof(int)));
   LMOE_CUDA(h, cudaDeviceSynchronize());
   h->max_T = max_T;
   h->W = (int)W;
@@ -700,7 +826,8 @@ lmoe_status lmoe_route_only(lmoe_layer* h, const float* logits, int T, int* idx,
     LMOE_CUDA(h, cudaMemsetAsync(offsets, 0, (size_t)(h->N + 1) * sizeof(int), st));
     return LMOE_OK;
   }
-  return run_routing(h, logits, T, idx, w, offsets, nullptr, perm, nullptr, st, false);
+  return run_routing(h, logits, T, idx, w, offsets, nullptr, perm, nullptr, nullptr, nullptr, st,
+                     false);
 }
 
 lmoe_status lmoe_router_logits(lmoe_layer* h, const void* x, float* logits, int T,

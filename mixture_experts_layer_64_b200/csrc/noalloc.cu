@@ -95,10 +95,10 @@ extern "C" lmoe_status lmoe_route_only_noalloc(const float* logits, int T, int N
     return LMOE_ERR_CUDA;
   topk_softmax_kernel<<<(T + 7) / 8, 256, 0, s>>>(logits, T, N, k, idx, w, bitmap, (int)W, 0, err);
   group_count_kernel<<<(N + 7) / 8, 256, 0, s>>>(bitmap, wp, N, (int)W, counts, offsets,
-                                                 tile_prefix, done);
+                                                 tile_prefix, nullptr, done);
   const long P = (long)T * k;
   group_rank_kernel<<<(unsigned)((P + 255) / 256), 256, 0, s>>>(idx, w, wp, offsets, T, k, N,
-                                                                 (int)W, nullptr, perm, nullptr, 0,
-                                                                 err);
+                                                                 (int)W, nullptr, perm, nullptr,
+                                                                 nullptr, 0, err);
   return cudaGetLastError() == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA;
 }

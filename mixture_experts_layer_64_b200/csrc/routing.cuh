@@ -15,7 +15,9 @@
 //                         call); the last block to finish scans the loads
 //                         into offsets and into per-expert 128-row tile counts.
 //   group_rank_kernel     one thread per pair: row = offsets[e] + (tokens < t
-//                         routed to e), read from the word prefix + popcount.
+//                         routed to e), read from the word prefix + popcount;
+//                         writes row -> token, row -> pair, row -> gate and
+//                         pair -> row.
 // Everything is integer work on fixed inputs, so the permutation is the same
 // on every run and equals "sort pairs by expert, then by token".
 #pragma once
@@ -99,6 +101,7 @@ static __global__ void __launch_bounds__(256) group_count_kernel(uint32_t* __res
                                                           int* __restrict__ counts,
                                                           int* __restrict__ offsets,
                                                           int* __restrict__ tile_prefix,
+                                                          int* __restrict__ tile_prefix2,
                                                           unsigned int* done) {
   const int lane = threadIdx.x & 31;
   const int e = blockIdx.x * 8 + (threadIdx.x >> 5);
@@ -130,38 +133,47 @@ static __global__ void __launch_bounds__(256) group_count_kernel(uint32_t* __res
   __syncthreads();
   if (!is_last) return;
   __threadfence();
-  // Block-wide exclusive scans of counts and of ceil(counts / 128).
-  __shared__ int s_c[256], s_t[256];
+  // Block-wide exclusive scans of counts and of ceil(counts / 128) and
+  // ceil(counts / 256) (row tiles of single CTAs and of CTA pairs).
+  __shared__ int s_c[256], s_t[256], s_u[256];
   const int per = (N + 255) / 256;
   const int lo = threadIdx.x * per, hi = min(N, lo + per);
-  int c_sum = 0, t_sum = 0;
+  int c_sum = 0, t_sum = 0, u_sum = 0;
   for (int i = lo; i < hi; ++i) {
     const int c = __ldcg(counts + i);
     c_sum += c;
     t_sum += (c + kRowTile - 1) / kRowTile;
+    u_sum += (c + 2 * kRowTile - 1) / (2 * kRowTile);
   }
   s_c[threadIdx.x] = c_sum;
   s_t[threadIdx.x] = t_sum;
+  s_u[threadIdx.x] = u_sum;
   __syncthreads();
   for (int o = 1; o < 256; o <<= 1) {
     const int a = threadIdx.x >= o ? s_c[threadIdx.x - o] : 0;
     const int b = threadIdx.x >= o ? s_t[threadIdx.x - o] : 0;
+    const int d = threadIdx.x >= o ? s_u[threadIdx.x - o] : 0;
     __syncthreads();
     s_c[threadIdx.x] += a;
     s_t[threadIdx.x] += b;
+    s_u[threadIdx.x] += d;
     __syncthreads();
   }
-  int c_run = s_c[threadIdx.x] - c_sum, t_run = s_t[threadIdx.x] - t_sum;
+  int c_run = s_c[threadIdx.x] - c_sum, t_run = s_t[threadIdx.x] - t_sum,
+      u_run = s_u[threadIdx.x] - u_sum;
   for (int i = lo; i < hi; ++i) {
     const int c = __ldcg(counts + i);
     offsets[i] = c_run;
     tile_prefix[i] = t_run;
+    if (tile_prefix2) tile_prefix2[i] = u_run;
     c_run += c;
     t_run += (c + kRowTile - 1) / kRowTile;
+    u_run += (c + 2 * kRowTile - 1) / (2 * kRowTile);
   }
   if (threadIdx.x == 255) {
     offsets[N] = s_c[255];
     tile_prefix[N] = s_t[255];
+    if (tile_prefix2) tile_prefix2[N] = s_u[255];
     *done = 0u;
   }
 }
@@ -170,7 +182,8 @@ static __global__ void __launch_bounds__(256) group_count_kernel(uint32_t* __res
 static __global__ void __launch_bounds__(256) group_rank_kernel(
     const int* __restrict__ idx, const float* __restrict__ w, const uint2* __restrict__ wp,
     const int* __restrict__ offsets, int T, int k, int N, int W, int* __restrict__ row_tok,
-    int* __restrict__ row_slot, float* __restrict__ row_w, int debug, int* err) {
+    int* __restrict__ row_slot, float* __restrict__ row_w, int* __restrict__ slot_row, int debug,
+    int* err) {
   const long pidx = (long)blockIdx.x * blockDim.x + threadIdx.x;
   if (pidx >= (long)T * k) return;
   const int t = (int)(pidx / k);
@@ -187,6 +200,7 @@ static __global__ void __launch_bounds__(256) group_rank_kernel(
     return;
   }
   if (row_tok) row_tok[row] = t;
+  if (slot_row) slot_row[pidx] = row;
   row_slot[row] = (int)pidx;
   if (row_w) row_w[row] = __ldg(w + pidx);
 }

@@ -121,6 +121,12 @@ __device__ __forceinline__ void store_row32(const GemmProblem& p, int row, int f
       }
       *reinterpret_cast<uint4*>(o + i) = q;
       if (split) *reinterpret_cast<uint4*>(o + split + i) = ql;
+      if (kEpi == EPI_ACT && e.scat) {
+        for (int j = 0; j < e.scat_k; ++j) {
+          const size_t srow = (size_t)__ldg(e.slot_row + (size_t)row * e.scat_k + j);
+          *reinterpret_cast<uint4*>(static_cast<bf16*>(e.scat) + srow * e.ldo + e.col0 + f + i) = q;
+        }
+      }
     }
   } else {
     for (int i = 0; i < 32 && f + i < p.F; ++i) {
@@ -128,6 +134,12 @@ __device__ __forceinline__ void store_row32(const GemmProblem& p, int row, int f
       const bf16 hi = __float2bfloat16_rn(v);
       o[i] = hi;
       if (split) o[split + i] = __float2bfloat16_rn(v - __bfloat162float(hi));
+      if (kEpi == EPI_ACT && e.scat) {
+        for (int j = 0; j < e.scat_k; ++j) {
+          const size_t srow = (size_t)__ldg(e.slot_row + (size_t)row * e.scat_k + j);
+          static_cast<bf16*>(e.scat)[srow * e.ldo + e.col0 + f + i] = hi;
+        }
+      }
     }
   }
 }
@@ -259,7 +271,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         tc_fence_after();
         const uint32_t d0 = tmem_base + ab * Cfg::ACC_COLS;
         const uint32_t d1 = d0 + Cfg::ACC_N;
-        int n = Cfg::ACC_N;
+        // Token-tiled gated tiles: the gate and linear weight tiles sit back to
+        // back in shared memory (rows 0-127 and 128-255 of one 256-row B
+        // operand) and their accumulators back to back in TMEM, so one N = 256
+        // MMA computes both and reads the activation tile once.
+        int n = Cfg::kDual ? 2 * Cfg::ACC_N : Cfg::ACC_N;
         if (Cfg::kSwap) n = max(16, (rows + 15) & ~15);
         const uint32_t idesc = idesc_bf16_f32(128, n);
         bool ok = true;
@@ -279,7 +295,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               if (Cfg::kDual) tc_mma_bf16(d1, dw1 + adv, da + adv, idesc, acc);
             } else {
               tc_mma_bf16(d0, da + adv, dw0 + adv, idesc, acc);
-              if (Cfg::kDual) tc_mma_bf16(d1, da + adv, dw1 + adv, idesc, acc);
             }
           }
           tc_commit(&empty[s]);
@@ -384,6 +399,202 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
+  }
+}
+
+
+// ==== 2-SM (CTA pair) token-tiled GEMM ==========================================
+//
+// The prefill contractions on CTA pairs: one tcgen05.mma.cta_group::2 of
+// M = 256, N = 256 per K step, issued by the pair's leader.  Each CTA stages
+// its own 128 activation rows (A is split by M) and half of the 256 weight
+// rows (B is split by N), so per SM the operand traffic (L2 -> shared memory,
+// shared-memory reads by the tensor core, TMA requests) is two thirds of a
+// single-CTA M = 128, N = 256 tile for the same math; each CTA's TMEM holds
+// its 128 rows x 256 columns.  Gated FC1: CTA 0 stages the 128 gate rows and
+// CTA 1 the 128 linear rows of the same features, which puts gate and linear
+// accumulators side by side in every row as in the single-CTA kernel.
+//
+// Synchronisation: both CTAs' TMA loads complete on the leader's `full`
+// barrier (2-SM TMA); the leader's MMA commits arrive on `empty` and `tfull`
+// in both CTAs (multicast commit); both CTAs' epilogue warps arrive on the
+// leader's `tempty` (remote arrive).  Activations are always TMA tiles of
+// contiguous rows (the expert FC1 reads latent rows already in expert order).
+
+template <bool kDual_, int kEpi_>
+struct TcPairCfg {
+  static constexpr bool kDual = kDual_;
+  static constexpr int kEpi = kEpi_;
+  static constexpr int BK = 64;
+  static constexpr int A_BYTES = 128 * BK * 2;   // this CTA's 128 rows
+  static constexpr int B_BYTES = 128 * BK * 2;   // this CTA's half of the 256 weight rows
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES = 6;
+  static constexpr int ACC_N = 256;              // columns of one accumulator buffer
+  static constexpr int TMEM_COLS = 512;
+  static constexpr int FT = kDual ? 128 : 256;   // output features per tile
+  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 512;
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
+};
+
+template <class Cfg>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    tc_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
+                        const __grid_constant__ CUtensorMap tmB, const GemmProblem p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + Cfg::STAGES * Cfg::STAGE_BYTES);
+  uint64_t* empty = full + Cfg::STAGES;
+  uint64_t* tfull = empty + Cfg::STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int cid = (int)cluster_id_x(), ncl = (int)cluster_count_x();
+  const int NT = (p.F + Cfg::FT - 1) / Cfg::FT;
+  const int KB = p.K / Cfg::BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < Cfg::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 8);  // 4 epilogue warps in each CTA of the pair
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&tmA);
+    prefetch_tensormap(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, Cfg::TMEM_COLS);
+    tmem_relinquish_pair();
+    tc_fence_before();
+  }
+  __syncthreads();
+  cluster_sync();  // both CTAs' barriers exist before any remote arrive
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int num_tiles = total_row_tiles(p) * NT;
+
+  if (warp == 0) {
+    // ---------------- TMA producer (both CTAs) ----------------
+    if (lane == 0) {
+      const uint32_t full_leader = cluster_map(&full[0], 0);
+      int s = 0;
+      uint32_t ph = 0;
+      long armed = 0;
+      for (int t = cid; t < num_tiles; t += ncl) {
+        const int rt = t / NT, ft = t - (t / NT) * NT;
+        int g, row0, rows;
+        locate_row_tile(p, rt, g, row0, rows);
+        int wrow = (int)(g * p.w_group_stride) + ft * Cfg::FT;
+        wrow += Cfg::kDual ? (rank ? p.dual_offset : 0) : (int)rank * 128;
+        const int arow = row0 + (int)rank * 128;
+        bool ok = true;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait_cluster(&empty[s], ph ^ 1, abort_flag, p.err)) { ok = false; break; }
+          uint8_t* st = smem + s * Cfg::STAGE_BYTES;
+          if (rank == 0) {
+            mbar_arrive_expect_tx(&full[s], 2 * Cfg::STAGE_BYTES);
+            ++armed;
+          }
+          const uint32_t fb = full_leader + (uint32_t)s * 8u;
+          tma_load_2d_pair(&tmA, fb, st, kb * Cfg::BK, arow);
+          tma_load_2d_pair(&tmB, fb, st + Cfg::A_BYTES, kb * Cfg::BK, wrow);
+          if (++s == Cfg::STAGES) { s = 0; ph ^= 1; }
+        }
+        if (!ok) break;
+      }
+      if (rank == 0 && *abort_flag) {
+        int ss = s;
+        uint32_t pp = ph;
+        for (long i = 0; i < armed && i < Cfg::STAGES; ++i) {
+          if (ss == 0) { ss = Cfg::STAGES; pp ^= 1; }
+          --ss;
+          mbar_wait_drain(&full[ss], pp);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer (leader only) ----------------
+    if (rank == 0 && lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(256, Cfg::ACC_N);
+      int s = 0;
+      uint32_t ph = 0;
+      int it = 0;
+      for (int t = cid; t < num_tiles; t += ncl, ++it) {
+        const int ab = it & 1;
+        const uint32_t aph = (it >> 1) & 1;
+        if (!mbar_wait_cluster(&tempty[ab], aph ^ 1, abort_flag, p.err)) break;
+        tc_fence_after();
+        const uint32_t d0 = tmem_base + ab * Cfg::ACC_N;
+        bool ok = true;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait_cluster(&full[s], ph, abort_flag, p.err)) { ok = false; break; }
+          tc_fence_after();
+          const uint8_t* st = smem + s * Cfg::STAGE_BYTES;
+          const uint64_t da = smem_desc_sw128(st);
+          const uint64_t db = smem_desc_sw128(st + Cfg::A_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < Cfg::BK / 16; ++kk) {
+            const uint64_t adv = (uint64_t)(kk * 32) >> 4;
+            tc_mma_bf16_pair(d0, da + adv, db + adv, idesc, (kb | kk) != 0);
+          }
+          tc_commit_pair_mc(&empty[s], 0x3);
+          if (++s == Cfg::STAGES) { s = 0; ph ^= 1; }
+        }
+        if (!ok) break;
+        tc_commit_pair_mc(&tfull[ab], 0x3);
+      }
+      tc_commit_pair_mc(drain, 0x1);
+      mbar_wait_drain(drain, 0);
+    }
+  } else if (warp >= 4) {
+    // ---------------- epilogue (warps 4..7 of both CTAs) ----------------
+    const int qd = warp & 3;
+    const uint32_t tempty_leader = cluster_map(&tempty[0], 0);
+    int it = 0;
+    for (int t = cid; t < num_tiles; t += ncl, ++it) {
+      const int rt = t / NT, ft = t - (t / NT) * NT;
+      int g, row0, rows;
+      locate_row_tile(p, rt, g, row0, rows);
+      const int ab = it & 1;
+      const uint32_t aph = (it >> 1) & 1;
+      if (!mbar_wait_cluster(&tfull[ab], aph, abort_flag, p.err)) break;
+      tc_fence_after();
+      const uint32_t tb = tmem_base + ((uint32_t)(qd * 32) << 16) + ab * Cfg::ACC_N;
+      const int f0 = ft * Cfg::FT;
+      const int r = (int)rank * 128 + qd * 32 + lane;  // row within the 256-row tile
+      float v0[32], v1[32];
+      constexpr int NCOL = Cfg::kDual ? 128 : 256;
+      for (int c0 = 0; c0 < NCOL; c0 += 32) {
+        tmem_ld_32x32(tb + c0, v0);
+        if (Cfg::kDual) tmem_ld_32x32(tb + 128 + c0, v1);
+        tc_wait_ld();
+        if (r < rows && f0 + c0 < p.F)
+          store_row32<Cfg::kEpi>(p, row0 + r, f0 + c0, v0, Cfg::kDual ? v1 : nullptr);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(tempty_leader + (uint32_t)ab * 8u);
+    }
+  }
+
+  __syncthreads();
+  cluster_sync();  // no CTA leaves while its peer may still signal its barriers
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, Cfg::TMEM_COLS);
   }
 }
 
