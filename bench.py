@@ -42,6 +42,8 @@ from mixture_experts_layer_64_b200 import costmodel, workloads  # noqa: E402
 METRIC = "LatentMoE layer tokens/sec at decode & prefill T; HBM GB/s / tensor-pipe % of peak"
 UNIT = "tokens/s"
 DEFAULT_WORKLOAD = "std-moe-decode"
+EXPERT_PATHS = ["cuda-core", "tcgen05 token-tiled", "tcgen05 weight-stationary",
+                "tcgen05 token-tiled, 2-SM CTA pairs"]
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 _CSRC = "mixture_experts_layer_64_b200/csrc/"
 _GEMM_SRC = (_CSRC + "common.cuh", _CSRC + "tc_gemm.cuh")
@@ -283,7 +285,7 @@ def run_ours(args):
     xw = w if rank == 0 else workloads.Workload(**{**w.__dict__, "seed": w.seed + 1000 * rank})
     x = workloads.make_x(xw, device=dev)
     L = lmoe.LatentMoELayer(w.d, w.l, w.N, w.k, w.m, act=w.act, shared_m=w.shared_m,
-                            dtype=w.dtype, skip_proj=w.skip_proj)
+                            dtype=w.dtype, skip_proj=w.skip_proj, flags=args.lib_flags)
     L.set_weights(W["Wg"], W["bias"], W["Wdown"], W["Wup"], W["W1"], W["W2"], W["Ws1"], W["Ws2"])
     L.reserve(w.T)
     out = torch.empty_like(x)
@@ -404,10 +406,10 @@ def run_ours(args):
                 "e2e": {"value": w.T * ws / (e_ms / 1000.0), "unit": UNIT,
                         "h2d_bytes_per_step": io_bytes, "d2h_bytes_per_step": io_bytes},
                 "gpu_launches": launches_per_step * args.steps,
+                "lib_flags": args.lib_flags,
                 "roofline": roofline, "cpu_baseline": cpu_baseline, "clocks": clocks,
-                "expert_path": ["cuda-core", "tcgen05 token-tiled",
-                                "tcgen05 weight-stationary",
-                                "tcgen05 token-tiled, 2-SM CTA pairs"][max(0, L.last_expert_path)]}
+                "expert_path": {"fc1": EXPERT_PATHS[max(0, L.last_expert_path) & 3],
+                                "fc2": EXPERT_PATHS[max(0, L.last_expert_path) >> 2]}}
         print(json.dumps(line), flush=True)
     L.close()
     if pg:
@@ -429,6 +431,8 @@ def main():
                     help="override N (reduced cases for profiler captures)")
     ap.add_argument("--topk", type=int, default=None, help="override k")
     ap.add_argument("--tokens", type=int, default=None, help="override T")
+    ap.add_argument("--lib-flags", type=int, default=0,
+                    help="lmoe_create flags (e.g. 32 = never use CTA pairs) for A/B runs")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

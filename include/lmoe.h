@@ -178,7 +178,7 @@ typedef enum {
   LMOE_STAGE_Z = 5,        /* [T, l]   dtype  latent rows (not with SKIP)    */
   LMOE_STAGE_H = 6,        /* [T*k, m] dtype  expert hidden rows, sorted     */
   LMOE_STAGE_YS = 7,       /* [T*k, l] dtype  gate-scaled expert outputs,
-                                             in slot order t*k+j             */
+                                             expert-sorted rows (as H)       */
   LMOE_STAGE_COMB = 8      /* [T, l]   dtype  combined rows (not with SKIP)  */
 } lmoe_stage;
 
@@ -248,9 +248,9 @@ lmoe_status lmoe_route_only_noalloc(const float* logits, int T, int N, int k, in
 /* Kernel launches the last lmoe_forward enqueued (library kernels only). */
 int lmoe_last_launch_count(const lmoe_layer* h);
 
-/* Which expert kernels the last lmoe_forward used: 0 CUDA-core, 1 tcgen05
- * token-tiled, 2 tcgen05 weight-stationary (swap-AB), 3 tcgen05 token-tiled on
- * CTA pairs (2-SM MMA). */
+/* Which expert kernels the last lmoe_forward used, FC1 in bits 0-1 and FC2
+ * in bits 2-3, each: 0 CUDA-core, 1 tcgen05 token-tiled, 2 tcgen05
+ * weight-stationary (swap-AB), 3 tcgen05 token-tiled on CTA pairs (2-SM MMA). */
 int lmoe_last_expert_path(const lmoe_layer* h);
 
 const char* lmoe_status_string(lmoe_status s);

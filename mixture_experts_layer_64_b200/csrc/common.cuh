@@ -20,7 +20,7 @@ typedef __nv_bfloat16 bf16;
 enum EpiKind {
   EPI_F32_BIAS = 0,      // out_f32[r, f] = acc + bias[f]                      (router)
   EPI_ACT = 1,           // out[r, col0 + f] = act(acc) / swiglu(acc0, acc1)  (FC1, down-proj)
-  EPI_SCALE_SCATTER = 2, // out[row_slot[r], f] = row_w[r] * acc               (expert FC2)
+  EPI_SCALE_ROWS = 2,    // out[r, f] = row_w[r] * acc (rows in expert order)   (expert FC2)
   EPI_RESID = 3          // out[r, f] = resid[r, f] + acc                      (up-projection)
 };
 enum ActKind { ACT_NONE = -1, ACT_SILU = 0, ACT_SWIGLU = 1, ACT_RELU2 = 2 };
@@ -34,11 +34,7 @@ struct EpiParams {
   const float* bias;      // EPI_F32_BIAS, may be NULL
   const void* resid;      // EPI_RESID, row stride ldr
   long ldr;
-  const int* row_slot;    // EPI_SCALE_SCATTER: tile row -> output row
-  const float* row_w;     // EPI_SCALE_SCATTER: tile row -> gate weight
-  void* scat;             // EPI_ACT: also copy each output row t to rows
-  const int* slot_row;    //   scat[slot_row[t * scat_k + j]], j < scat_k (row stride ldo):
-  int scat_k;             //   latent rows written straight into expert order
+  const float* row_w;     // EPI_SCALE_ROWS: row -> gate weight
   int split_off;          // EPI_ACT, bf16: > 0 also writes v - bf16(v) (rounded) at
                           // column col0 + split_off + f, so that hi + lo carries the
                           // value to ~16 significant bits through the next bf16 GEMM
@@ -67,6 +63,8 @@ struct GemmProblem {
   int F;                  // output features
   int K;                  // reduction length
   EpiParams epi;
+  int tma_store;          // token-tiled kernels: write full 32-row blocks with TMA stores
+                          // (the output map is the kernel's third tensor map)
   int* err;               // device error word
 };
 
@@ -209,6 +207,22 @@ __device__ __forceinline__ void tma_load_2d(const CUtensorMap* map, uint64_t* ba
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
       : "memory");
 }
+
+// Bulk tensor store of a shared-memory box to global memory (async proxy).
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* smem_src, int c0,
+                                             int c1) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(c0), "r"(c1), "r"(smem_u32(smem_src))
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// wait until the sources of all committed bulk stores have been read
+__device__ __forceinline__ void bulk_wait_read0() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// wait until all committed bulk stores have completed
+__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");

@@ -9,8 +9,8 @@
 //   4 down-projection GEMM   z[T,l] = x Wdown                 (not when skipped)
 //   5 shared FC1 GEMM        hs = act(x Ws1) into cat[:, l:] as bf16 hi + lo pairs
 //   6 expert FC1 (grouped)   h[r] = act(z[tok(r)] W1[e])      rows gathered by token
-//   7 expert FC2 (grouped)   ys[slot(r)] = w(r) * (h[r] W2[e])
-//   8 combine                cat[t, :l] = sum_j ys[t*k + j]   (skipped projections:
+//   7 expert FC2 (grouped)   ys[r] = w(r) * (h[r] W2[e])         rows in expert order
+//   8 combine                cat[t, :l] = sum_j ys[row(t, j)] (skipped projections:
 //                            out = x + sum (+ the shared expert, computed in fp32 at 5))
 //   9 up-projection GEMM     out = x + [comb | hs_hi | hs_lo] [Wup ; Ws2 ; Ws2]
 // Contractions run on the tcgen05 kernel (bf16) or the CUDA-core kernel
@@ -88,7 +88,7 @@ struct lmoe_layer {
   int* err = nullptr;
   int *row_tok = nullptr, *row_slot = nullptr, *slot_row = nullptr;
   float* row_w = nullptr;
-  void *z = nullptr, *zs = nullptr, *h = nullptr, *ys = nullptr, *cat = nullptr;
+  void *z = nullptr, *h = nullptr, *ys = nullptr, *cat = nullptr;
   void *x_stage = nullptr, *out_stage = nullptr;
   float* s32 = nullptr;  // [T, d] fp32 shared-expert output (projection-skip layers)
   // bookkeeping
@@ -144,6 +144,7 @@ struct GemmCall {
   GemmKind kind;
   long a_rows;  // rows of A (TMA bounds)
   long b_rows;  // rows of B (TMA bounds)
+  long out_rows;  // rows of the output (TMA store bounds)
   bool swap;    // weight-stationary expert kernels
   bool pair;    // 2-SM token-tiled kernels on CTA pairs (256-row tiles)
 };
@@ -158,6 +159,35 @@ bool encode_map(CUtensorMap* map, const void* ptr, long rows, int cols, long ld,
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Output map of the TMA-store epilogue: 32 x 32 boxes, 64-byte swizzle for
+// bf16 (64-byte rows), 128-byte swizzle for fp32 (128-byte rows).
+bool encode_out_map(CUtensorMap* map, const GemmCall& c) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return false;
+  const bool f32 = c.kind == GK_ROUTER;
+  const size_t es = f32 ? 4 : 2;
+  const char* base = static_cast<const char*>(c.p.epi.out) +
+                     (c.kind == GK_DENSE_ACT || c.kind == GK_FC1 ? (size_t)c.p.epi.col0 * es : 0);
+  cuuint64_t dims[2] = {(cuuint64_t)c.p.F, (cuuint64_t)c.out_rows};
+  cuuint64_t strides[1] = {(cuuint64_t)c.p.epi.ldo * es};
+  cuuint32_t box[2] = {32, 32};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(map, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+            const_cast<char*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            f32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+            CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Whether a token-tiled call can write its output with TMA stores.
+bool tma_store_ok(const GemmCall& c) {
+  const EpiParams& e = c.p.epi;
+  if (c.swap || e.split_off || c.kind == GK_ROUTER) return false;  // fp32 logits: plain stores
+  const size_t es = 2;
+  const char* base = static_cast<const char*>(e.out) +
+                     (c.kind == GK_DENSE_ACT || c.kind == GK_FC1 ? (size_t)e.col0 * es : 0);
+  return aligned16(base) && ((size_t)e.ldo * es) % 16 == 0 && (c.p.F * es) % 16 == 0;
 }
 
 template <class Cfg>
@@ -181,10 +211,14 @@ lmoe_status launch_tc(lmoe_layer* h, const GemmCall& c, cudaStream_t st) {
     h->detail = "cuTensorMapEncodeTiled (weights) failed";
     return LMOE_ERR_CUDA;
   }
+  CUtensorMap tc;
+  std::memset(&tc, 0, sizeof tc);
+  GemmProblem p = c.p;
+  p.tma_store = (!Cfg::kSwap && tma_store_ok(c) && encode_out_map(&tc, c)) ? 1 : 0;
   const long NT = (c.p.F + Cfg::FT - 1) / Cfg::FT;
   const long tiles = (long)c.p.max_row_tiles * NT;
   const int grid = (int)std::max(1L, std::min<long>(h->num_sms, tiles));
-  tc_gemm_kernel<Cfg><<<grid, kTcThreads, Cfg::SMEM_BYTES, st>>>(ta, tb, c.p);
+  tc_gemm_kernel<Cfg><<<grid, kTcThreads, Cfg::SMEM_BYTES, st>>>(ta, tb, tc, p);
   LMOE_CHECK_LAUNCH(h);
   return LMOE_OK;
 }
@@ -240,7 +274,11 @@ lmoe_status launch_pair(lmoe_layer* h, const GemmCall& c, cudaStream_t st) {
   cfg.stream = st;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  LMOE_CUDA(h, cudaLaunchKernelEx(&cfg, tc_gemm_pair_kernel<Cfg>, ta, tb, c.p));
+  CUtensorMap tc;
+  std::memset(&tc, 0, sizeof tc);
+  GemmProblem p = c.p;
+  p.tma_store = (tma_store_ok(c) && encode_out_map(&tc, c)) ? 1 : 0;
+  LMOE_CUDA(h, cudaLaunchKernelEx(&cfg, tc_gemm_pair_kernel<Cfg>, ta, tb, tc, p));
   ++h->launches;
   return LMOE_OK;
 }
@@ -263,7 +301,7 @@ lmoe_status dispatch_simt(lmoe_layer* h, const GemmCall& c, cudaStream_t st) {
     case GK_DENSE_ACT:
     case GK_FC1:
       return dual ? launch_simt<T, true, EPI_ACT>(h, c, st) : launch_simt<T, false, EPI_ACT>(h, c, st);
-    case GK_FC2: return launch_simt<T, false, EPI_SCALE_SCATTER>(h, c, st);
+    case GK_FC2: return launch_simt<T, false, EPI_SCALE_ROWS>(h, c, st);
     case GK_UP: return launch_simt<T, false, EPI_RESID>(h, c, st);
   }
   return LMOE_ERR_INVALID_ARG;
@@ -314,7 +352,7 @@ lmoe_status run_gemm(lmoe_layer* h, GemmCall c, cudaStream_t st, int* path = nul
       case GK_FC1:
         return dual ? launch_pair<TcPairCfg<true, EPI_ACT>>(h, c, st)
                     : launch_pair<TcPairCfg<false, EPI_ACT>>(h, c, st);
-      case GK_FC2: return launch_pair<TcPairCfg<false, EPI_SCALE_SCATTER>>(h, c, st);
+      case GK_FC2: return launch_pair<TcPairCfg<false, EPI_SCALE_ROWS>>(h, c, st);
       case GK_UP: return launch_pair<TcPairCfg<false, EPI_RESID>>(h, c, st);
       case GK_ROUTER: return launch_pair<TcPairCfg<false, EPI_F32_BIAS>>(h, c, st);
     }
@@ -331,8 +369,8 @@ lmoe_status run_gemm(lmoe_layer* h, GemmCall c, cudaStream_t st, int* path = nul
       return dual ? launch_tc<TcCfg<false, true, true, 128, EPI_ACT>>(h, c, st)
                   : launch_tc<TcCfg<false, true, false, 256, EPI_ACT>>(h, c, st);
     case GK_FC2:
-      return c.swap ? launch_tc<TcCfg<true, false, false, 128, EPI_SCALE_SCATTER>>(h, c, st)
-                    : launch_tc<TcCfg<false, false, false, 256, EPI_SCALE_SCATTER>>(h, c, st);
+      return c.swap ? launch_tc<TcCfg<true, false, false, 128, EPI_SCALE_ROWS>>(h, c, st)
+                    : launch_tc<TcCfg<false, false, false, 256, EPI_SCALE_ROWS>>(h, c, st);
     case GK_UP: return launch_tc<TcCfg<false, false, false, 256, EPI_RESID>>(h, c, st);
   }
   return LMOE_ERR_INVALID_ARG;
@@ -353,6 +391,7 @@ GemmCall dense_call(GemmKind kind, int M, const void* A, long lda, const void* B
   c.p.K = K;
   c.a_rows = M;
   c.b_rows = F;
+  c.out_rows = M;
   c.p.epi.act = ACT_NONE;
   return c;
 }
@@ -390,6 +429,7 @@ GemmCall grouped_call(const lmoe_layer* h, GemmKind kind, int T, const void* A, 
   c.p.K = K;
   c.a_rows = a_rows;
   c.b_rows = (long)h->N * stride;
+  c.out_rows = R;
   c.p.epi.act = ACT_NONE;
   return c;
 }
@@ -456,19 +496,14 @@ lmoe_status run_forward(lmoe_layer* h, const void* x, void* out, int T, cudaStre
   const bool swap = use_swap(h, T);
   const bool pairs_ok = h->dtype == LMOE_BF16 && !(h->flags & (LMOE_FORCE_SIMT | LMOE_FORCE_NOPAIR));
   // CTA pairs for the dense GEMMs once there are enough rows to fill them,
-  // and for the token-tiled expert GEMMs (their FC1 then reads the latent
-  // rows in expert order, written by the down-projection's epilogue)
+  // and for the token-tiled expert FC2 (its input rows are contiguous; the
+  // expert FC1 gathers its rows by token and stays on single CTAs)
   const bool pair_dense = pairs_ok && T >= 1024;
-  const bool pair_experts = pairs_ok && !swap && !skip && h->zs != nullptr;
+  const bool pair_fc2 = pairs_ok && !swap;
   if (!skip) {
     GemmCall c = dense_call(GK_DENSE_ACT, T, x, d, h->Wd_t, l, d);
     c.p.epi.out = h->z;
     c.p.epi.ldo = l;
-    if (pair_experts) {
-      c.p.epi.scat = h->zs;
-      c.p.epi.slot_row = h->slot_row;
-      c.p.epi.scat_k = k;
-    }
     if (pair_dense) make_pair(h, c);
     LMOE_TRY(run_gemm(h, c, st));
   }
@@ -497,11 +532,7 @@ lmoe_status run_forward(lmoe_layer* h, const void* x, void* out, int T, cudaStre
   prof_mark(h, st, 5);
   {
     const void* A = skip ? x : h->z;
-    GemmCall c = pair_experts
-                     ? grouped_call(h, GK_FC1, T, h->zs, l, R, nullptr, h->W1_t, h->m_in, m, l)
-                     : grouped_call(h, GK_FC1, T, A, skip ? d : l, T, h->row_tok, h->W1_t,
-                                    h->m_in, m, l);
-    if (pair_experts) make_pair(h, c);
+    GemmCall c = grouped_call(h, GK_FC1, T, A, skip ? d : l, T, h->row_tok, h->W1_t, h->m_in, m, l);
     c.swap = swap;
     c.p.dual_offset = h->act == LMOE_ACT_SWIGLU ? m : 0;
     c.p.epi.out = h->h;
@@ -514,13 +545,14 @@ lmoe_status run_forward(lmoe_layer* h, const void* x, void* out, int T, cudaStre
   prof_mark(h, st, 6);
   {
     GemmCall c = grouped_call(h, GK_FC2, T, h->h, m, R, nullptr, h->W2_t, l, l, m);
-    if (pair_experts) make_pair(h, c);
+    if (pair_fc2) make_pair(h, c);
     c.swap = swap;
     c.p.epi.out = h->ys;
     c.p.epi.ldo = l;
-    c.p.epi.row_slot = h->row_slot;
     c.p.epi.row_w = h->row_w;
-    LMOE_TRY(run_gemm(h, c, st));
+    int path = 0;
+    LMOE_TRY(run_gemm(h, c, st, &path));
+    h->expert_path |= path << 2;
   }
   prof_mark(h, st, 7);
   {
@@ -534,17 +566,17 @@ lmoe_status run_forward(lmoe_layer* h, const void* x, void* out, int T, cudaStre
     const int threads = std::min(256, std::max(32, (l / vec + 31) / 32 * 32));
     if (h->dtype == LMOE_BF16) {
       if (vec_ok)
-        combine_kernel<bf16><<<T, threads, 0, st>>>((const bf16*)h->ys, k, l, (const bf16*)resid,
+        combine_kernel<bf16><<<T, threads, 0, st>>>((const bf16*)h->ys, h->slot_row, k, l, (const bf16*)resid,
                                                     d, add32, (bf16*)dst, ldo);
       else
-        combine_scalar_kernel<bf16><<<T, 256, 0, st>>>((const bf16*)h->ys, k, l,
+        combine_scalar_kernel<bf16><<<T, 256, 0, st>>>((const bf16*)h->ys, h->slot_row, k, l,
                                                        (const bf16*)resid, d, add32, (bf16*)dst, ldo);
     } else {
       if (vec_ok)
-        combine_kernel<float><<<T, threads, 0, st>>>((const float*)h->ys, k, l,
+        combine_kernel<float><<<T, threads, 0, st>>>((const float*)h->ys, h->slot_row, k, l,
                                                      (const float*)resid, d, add32, (float*)dst, ldo);
       else
-        combine_scalar_kernel<float><<<T, 256, 0, st>>>((const float*)h->ys, k, l,
+        combine_scalar_kernel<float><<<T, 256, 0, st>>>((const float*)h->ys, h->slot_row, k, l,
                                                         (const float*)resid, d, add32, (float*)dst, ldo);
     }
     LMOE_CHECK_LAUNCH(h);
@@ -582,7 +614,6 @@ void free_workspace(lmoe_layer* h) {
   free_ptr(h->tile_prefix);
   free_ptr(h->tile_prefix2);
   free_ptr(h->slot_row);
-  free_ptr(h->zs);
   free_ptr(h->done);
   free_ptr(h->err);
   free_ptr(h->row_tok);
@@ -764,9 +795,6 @@ lmoe_status lmoe_reserve(lmoe_layer* h, int max_T) {
   ALLOC(h->row_slot, R * sizeof(int));
   ALLOC(h->row_w, R * sizeof(float));
   if (!skip) ALLOC(h->z, T * h->l * es);
-  // latent rows in expert order, for the CTA-pair expert kernels (bf16 only)
-  if (!skip && h->dtype == LMOE_BF16 && !(h->flags & (LMOE_FORCE_SIMT | LMOE_FORCE_NOPAIR)))
-    ALLOC(h->zs, R * h->l * es);
   ALLOC(h->h, R * h->m * es);
   ALLOC(h->ys, R * h->l * es);
   if (h->Kup > 0) ALLOC(h->cat, T * h->Kup * es);

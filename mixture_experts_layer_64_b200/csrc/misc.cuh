@@ -7,20 +7,21 @@
 
 namespace lmoe {
 
-// comb[t, c] = (resid[t, c] +) sum_{j < k} ys[t*k + j, c], summed in fp32 in
-// slot order, rounded once.  ys rows are in slot order (t*k + j), so each
-// token's k rows are contiguous.  One block per token, VEC elements per thread
-// per step (16-byte accesses).
+// comb[t, c] = (resid[t, c] +) sum_{j < k} ys[slot_row[t*k + j], c], summed in
+// fp32 in slot order, rounded once.  ys rows are in expert order (as the
+// expert GEMMs wrote them); slot_row maps each (token, slot) pair to its row.
+// One block per token, VEC elements per thread per step (16-byte accesses).
 // With add32 (fp32, row stride ldr) that addend joins the sum before the one
 // rounding: the projection-skip layer adds its shared expert this way.
 template <typename T>
-__global__ void __launch_bounds__(256) combine_kernel(const T* __restrict__ ys, int k, int l,
-                                                      const T* __restrict__ resid, long ldr,
+__global__ void __launch_bounds__(256) combine_kernel(const T* __restrict__ ys,
+                                                      const int* __restrict__ slot_row, int k,
+                                                      int l, const T* __restrict__ resid, long ldr,
                                                       const float* __restrict__ add32,
                                                       T* __restrict__ out, long ldo) {
   constexpr int VEC = 16 / sizeof(T);
   const int t = blockIdx.x;
-  const T* base = ys + (size_t)t * k * l;
+  const int* rows = slot_row + (size_t)t * k;
   for (int c = threadIdx.x * VEC; c < l; c += blockDim.x * VEC) {
     float acc[VEC];
     if (resid) {
@@ -37,7 +38,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const T* __restrict__ ys, 
       for (int v = 0; v < VEC; ++v) acc[v] += add32[(size_t)t * ldr + c + v];
     }
     for (int j = 0; j < k; ++j) {
-      const uint4 yv = __ldg(reinterpret_cast<const uint4*>(base + (size_t)j * l + c));
+      const uint4 yv = __ldg(reinterpret_cast<const uint4*>(ys + (size_t)__ldg(rows + j) * l + c));
       const T* yb = reinterpret_cast<const T*>(&yv);
 #pragma unroll
       for (int v = 0; v < VEC; ++v) acc[v] += to_f32<T>(yb[v]);
@@ -52,7 +53,9 @@ __global__ void __launch_bounds__(256) combine_kernel(const T* __restrict__ ys, 
 
 // Scalar fallback of combine_kernel for widths that are not a multiple of VEC.
 template <typename T>
-__global__ void __launch_bounds__(256) combine_scalar_kernel(const T* __restrict__ ys, int k, int l,
+__global__ void __launch_bounds__(256) combine_scalar_kernel(const T* __restrict__ ys,
+                                                             const int* __restrict__ slot_row,
+                                                             int k, int l,
                                                              const T* __restrict__ resid, long ldr,
                                                              const float* __restrict__ add32,
                                                              T* __restrict__ out, long ldo) {
@@ -60,7 +63,7 @@ __global__ void __launch_bounds__(256) combine_scalar_kernel(const T* __restrict
   for (int c = threadIdx.x; c < l; c += blockDim.x) {
     float acc = resid ? to_f32<T>(resid[(size_t)t * ldr + c]) : 0.f;
     if (add32) acc += add32[(size_t)t * ldr + c];
-    for (int j = 0; j < k; ++j) acc += to_f32<T>(ys[((size_t)t * k + j) * l + c]);
+    for (int j = 0; j < k; ++j) acc += to_f32<T>(ys[(size_t)slot_row[(size_t)t * k + j] * l + c]);
     out[(size_t)t * ldo + c] = from_f32<T>(acc);
   }
 }

@@ -23,12 +23,8 @@ __device__ __forceinline__ void simt_store(const GemmProblem& p, int row, int f,
     const T hi = from_f32<T>(v);
     o[0] = hi;
     if (e.split_off) o[e.split_off] = from_f32<T>(v - to_f32<T>(hi));
-    if (e.scat)
-      for (int j = 0; j < e.scat_k; ++j)
-        static_cast<T*>(e.scat)[(size_t)e.slot_row[(size_t)row * e.scat_k + j] * e.ldo + e.col0 + f] = hi;
-  } else if (kEpi == EPI_SCALE_SCATTER) {
-    const size_t orow = (size_t)e.row_slot[row];
-    static_cast<T*>(e.out)[orow * e.ldo + f] = from_f32<T>(v0 * e.row_w[row]);
+  } else if (kEpi == EPI_SCALE_ROWS) {
+    static_cast<T*>(e.out)[(size_t)row * e.ldo + f] = from_f32<T>(v0 * e.row_w[row]);
   } else {
     const T* rs = static_cast<const T*>(e.resid);
     static_cast<T*>(e.out)[(size_t)row * e.ldo + f] =

@@ -4,7 +4,7 @@
 //
 // One kernel serves every contraction of the layer:
 //   router logits, down-projection, shared FC1, up-projection  (dense)
-//   expert FC1 (+ activation) and FC2 (+ gate scale, slot scatter) (grouped)
+//   expert FC1 (+ activation) and FC2 (+ gate scale)                (grouped)
 // A problem is D[r, f] = sum_k A[src(r), k] B[wrow(g, f), k] with both
 // operands K-major (B holds the weights transposed to [out, in]).
 //
@@ -19,12 +19,14 @@
 // same feature tile and accumulates them into two TMEM accumulators, so the
 // epilogue sees both halves of a feature in one thread.
 //
-// Warp roles (256 threads):
+// Warp roles (384 threads):
 //   warp 0      TMA producer (weights, and contiguous activation rows)
 //   warp 1      TMEM allocation and the single-thread MMA issuer
 //   warps 2-3   cp.async row gather of activations (gathered problems),
 //               completion signalled to the MMA issuer through the mbarrier
-//   warps 4-7   epilogue: tcgen05.ld -> epilogue math -> global stores
+//   warps 4-11  epilogue, two warpgroups taking alternate 32-column chunks:
+//               tcgen05.ld -> epilogue math -> shared-memory staging -> TMA
+//               bulk stores (plain stores for partly covered row blocks)
 // The smem ring has STAGES stages of one 64-wide K slice each; TMEM holds two
 // accumulator buffers so the epilogue of tile i overlaps the MMAs of tile i+1.
 #pragma once
@@ -33,7 +35,8 @@
 
 namespace lmoe {
 
-constexpr int kTcThreads = 256;
+constexpr int kTcThreads = 384;
+constexpr int kEpiWarps = 8;  // two warpgroups; each warp reads its TMEM lane quarter (warp % 4)
 constexpr int kTcSmemBudget = 200 * 1024;
 constexpr int kGatherThreads = 64;
 
@@ -54,19 +57,22 @@ struct TcCfg {
   static constexpr int ACC_COLS = ACC_N * NUM_W;      // one TMEM buffer
   static constexpr int TMEM_COLS = 2 * ACC_COLS;      // double buffered
   static constexpr int FT = W_ROWS;                   // features per tile
-  static constexpr int SMEM_BYTES = 1024 /*align slack*/ + STAGES * STAGE_BYTES + 512;
+  static constexpr int TABLE_BYTES = 2 * (LMOE_MAX_EXPERTS + 1) * 4;  // tile_prefix, offsets
+  static constexpr int STG_BYTES = kSwap ? 0 : kEpiWarps * 2048;  // epilogue staging (bf16 boxes)
+  static constexpr int SMEM_BYTES = 1024 /*align slack*/ + STAGES * STAGE_BYTES + STG_BYTES + 512 +
+                                    TABLE_BYTES;
   static_assert(TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM allocation must be a power of two");
   static_assert(STAGES >= 3, "pipeline too shallow");
-  static_assert(!kSwap || kEpi == EPI_ACT || kEpi == EPI_SCALE_SCATTER, "swap epilogues");
+  static_assert(!kSwap || kEpi == EPI_ACT || kEpi == EPI_SCALE_ROWS, "swap epilogues");
   static_assert(kWN_ == 128 || kWN_ == 256, "weight tile");
 };
 
 // ---- epilogue stores ----------------------------------------------------------
 
 // One row (token-tiled mode): 32 consecutive features [f, f+32) of row `row`.
-template <int kEpi>
-__device__ __forceinline__ void store_row32(const GemmProblem& p, int row, int f, const float* v0,
-                                            const float* v1) {
+template <int kEpi, bool kGated>
+__device__ __forceinline__ void store_row32(const GemmProblem& p, int row, int f,
+                                            const float (&v0)[32], const float (&v1)[32]) {
   const EpiParams& e = p.epi;
   const bool full = f + 32 <= p.F;
   if (kEpi == EPI_F32_BIAS) {
@@ -82,7 +88,9 @@ __device__ __forceinline__ void store_row32(const GemmProblem& p, int row, int f
         *reinterpret_cast<float4*>(o + i) = q;
       }
     } else {
-      for (int i = 0; i < 32 && f + i < p.F; ++i) o[i] = v0[i] + (e.bias ? e.bias[f + i] : 0.f);
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        if (f + i < p.F) o[i] = v0[i] + (e.bias ? e.bias[f + i] : 0.f);
     }
     return;
   }
@@ -91,10 +99,9 @@ __device__ __forceinline__ void store_row32(const GemmProblem& p, int row, int f
   size_t orow = (size_t)row;
   if (kEpi == EPI_ACT) {
 #pragma unroll
-    for (int i = 0; i < 32; ++i) r[i] = apply_act(e.act, v0[i], v1 ? v1[i] : 0.f);
-  } else if (kEpi == EPI_SCALE_SCATTER) {
+    for (int i = 0; i < 32; ++i) r[i] = apply_act(e.act, v0[i], kGated ? v1[i] : 0.f);
+  } else if (kEpi == EPI_SCALE_ROWS) {
     const float s = __ldg(e.row_w + row);
-    orow = (size_t)__ldg(e.row_slot + row);
 #pragma unroll
     for (int i = 0; i < 32; ++i) r[i] = v0[i] * s;
   } else {  // EPI_RESID
@@ -104,7 +111,8 @@ __device__ __forceinline__ void store_row32(const GemmProblem& p, int row, int f
   const int split = (kEpi == EPI_ACT) ? e.split_off : 0;
   if (full) {
 #pragma unroll
-    for (int i = 0; i < 32; i += 8) {
+    for (int c = 0; c < 4; ++c) {
+      const int i = 8 * c;
       if (kEpi == EPI_RESID) {
         const uint4 rv = *reinterpret_cast<const uint4*>(res + i);
         const bf16* rb = reinterpret_cast<const bf16*>(&rv);
@@ -121,24 +129,17 @@ __device__ __forceinline__ void store_row32(const GemmProblem& p, int row, int f
       }
       *reinterpret_cast<uint4*>(o + i) = q;
       if (split) *reinterpret_cast<uint4*>(o + split + i) = ql;
-      if (kEpi == EPI_ACT && e.scat) {
-        for (int j = 0; j < e.scat_k; ++j) {
-          const size_t srow = (size_t)__ldg(e.slot_row + (size_t)row * e.scat_k + j);
-          *reinterpret_cast<uint4*>(static_cast<bf16*>(e.scat) + srow * e.ldo + e.col0 + f + i) = q;
-        }
-      }
     }
   } else {
-    for (int i = 0; i < 32 && f + i < p.F; ++i) {
-      float v = (kEpi == EPI_RESID) ? __bfloat162float(res[i]) + v0[i] : r[i];
-      const bf16 hi = __float2bfloat16_rn(v);
-      o[i] = hi;
-      if (split) o[split + i] = __float2bfloat16_rn(v - __bfloat162float(hi));
-      if (kEpi == EPI_ACT && e.scat) {
-        for (int j = 0; j < e.scat_k; ++j) {
-          const size_t srow = (size_t)__ldg(e.slot_row + (size_t)row * e.scat_k + j);
-          static_cast<bf16*>(e.scat)[srow * e.ldo + e.col0 + f + i] = hi;
-        }
+    // ragged last chunk (F not a multiple of 32): element stores, fully
+    // unrolled so that r and v0 stay in registers
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      if (f + i < p.F) {
+        float v = (kEpi == EPI_RESID) ? __bfloat162float(res[i]) + v0[i] : r[i];
+        const bf16 hi = __float2bfloat16_rn(v);
+        o[i] = hi;
+        if (split) o[split + i] = __float2bfloat16_rn(v - __bfloat162float(hi));
       }
     }
   }
@@ -154,10 +155,115 @@ __device__ __forceinline__ void store_elem(const GemmProblem& p, int row, int f,
     bf16* o = static_cast<bf16*>(e.out) + (size_t)row * e.ldo + e.col0 + f;
     o[0] = hi;
     if (e.split_off) o[e.split_off] = __float2bfloat16_rn(v - __bfloat162float(hi));
-  } else {  // EPI_SCALE_SCATTER
-    const size_t orow = (size_t)__ldg(e.row_slot + row);
-    static_cast<bf16*>(e.out)[orow * e.ldo + f] = __float2bfloat16_rn(v0 * __ldg(e.row_w + row));
+  } else {  // EPI_SCALE_ROWS
+    static_cast<bf16*>(e.out)[(size_t)row * e.ldo + f] =
+        __float2bfloat16_rn(v0 * __ldg(e.row_w + row));
   }
+}
+
+// ---- epilogue through shared memory and TMA stores ------------------------------
+//
+// A TMEM row belongs to one thread, so plain global stores from registers put
+// 32 rows into every store instruction, 16 bytes each: half of a 32-byte
+// sector per row per instruction, which the memory system completes with
+// read-modify-writes.  Instead each epilogue warp stages its 32 rows x 32
+// bf16 columns in shared memory (64-byte rows with the 64-byte swizzle, which
+// keeps the row-per-thread writes free of bank conflicts) and one lane writes
+// the box with a bulk tensor store.  Blocks of 32 rows that a tile only partly
+// covers, and the fp32 router logits, use the plain stores.
+template <int kEpi, bool kGated>
+__device__ __forceinline__ void epi_tma_chunk32_impl(const GemmProblem& p, const CUtensorMap* tmC,
+                                                uint8_t* stg, int lane, int row_base, int f,
+                                                const float (&v0)[32], const float (&v1)[32]) {
+  const EpiParams& e = p.epi;
+  const int row = row_base + lane;
+  float r[32];
+  if (kEpi == EPI_ACT) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) r[i] = apply_act(e.act, v0[i], kGated ? v1[i] : 0.f);
+  } else if (kEpi == EPI_SCALE_ROWS) {
+    const float sc = __ldg(e.row_w + row);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) r[i] = v0[i] * sc;
+  } else if (kEpi == EPI_RESID) {
+    const bf16* rrow = static_cast<const bf16*>(e.resid) + (size_t)row * e.ldr + f;
+    if (f + 32 <= p.F) {
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const uint4 rv = reinterpret_cast<const uint4*>(rrow)[c];
+        const bf16* rb = reinterpret_cast<const bf16*>(&rv);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) r[8 * c + j] = __bfloat162float(rb[j]) + v0[8 * c + j];
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) r[i] = (f + i < p.F) ? __bfloat162float(rrow[i]) + v0[i] : 0.f;
+    }
+  }
+  if (lane == 0) bulk_wait_read0();  // the previous box has left the buffer
+  __syncwarp();
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    uint4 q;
+    bf16* qb = reinterpret_cast<bf16*>(&q);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) qb[j] = __float2bfloat16_rn(r[8 * c + j]);
+    *reinterpret_cast<uint4*>(stg + lane * 64 + ((c ^ ((lane >> 1) & 3)) << 4)) = q;
+  }
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_2d(tmC, stg, f, row_base);
+    bulk_commit();
+  }
+}
+
+template <int kEpi, bool kGated>
+__device__ __forceinline__ void epi_tma_chunk32(const GemmProblem& p, const CUtensorMap* tmC,
+                                                uint8_t* stg, int lane, int row_base, int f,
+                                                const float (&v0)[32], const float (&v1)[32]) {
+  if constexpr (kEpi != EPI_F32_BIAS)
+    epi_tma_chunk32_impl<kEpi, kGated>(p, tmC, stg, lane, row_base, f, v0, v1);
+}
+
+// ---- tile lookup from shared memory -----------------------------------------------
+//
+// Every role of a persistent CTA maps its next tile index to (group, first
+// row, rows) with a binary search over the groups' tile counts.  Done on
+// global memory that is ~10 dependent loads at every tile boundary, longer
+// than the pipeline hides, so the grouped kernels first copy tile_prefix and
+// offsets (G + 1 entries each) into shared memory.
+__device__ __forceinline__ void load_tile_tables(const GemmProblem& p, int* s_tiles) {
+  if (p.offsets == nullptr) return;
+  for (int i = threadIdx.x; i <= p.G; i += blockDim.x) {
+    s_tiles[i] = p.tile_prefix[i];
+    s_tiles[LMOE_MAX_EXPERTS + 1 + i] = p.offsets[i];
+  }
+}
+
+__device__ __forceinline__ void locate_row_tile_s(const GemmProblem& p, const int* s_tiles, int rt,
+                                                  int& g, int& row0, int& rows) {
+  if (p.offsets == nullptr) {
+    g = 0;
+    row0 = rt * p.row_tile;
+    rows = min(p.row_tile, p.M - row0);
+    return;
+  }
+  const int* tp = s_tiles;
+  const int* off = s_tiles + LMOE_MAX_EXPERTS + 1;
+  int lo = 0, hi = p.G - 1;  // largest g with tp[g] <= rt
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (tp[mid] <= rt) lo = mid; else hi = mid - 1;
+  }
+  g = lo;
+  row0 = off[g] + (rt - tp[g]) * p.row_tile;
+  rows = min(p.row_tile, off[g + 1] - row0);
+}
+
+__device__ __forceinline__ int total_row_tiles_s(const GemmProblem& p, const int* s_tiles) {
+  if (p.offsets == nullptr) return (p.M + p.row_tile - 1) / p.row_tile;
+  return s_tiles[p.G];
 }
 
 // ---- the kernel -----------------------------------------------------------------
@@ -165,19 +271,22 @@ __device__ __forceinline__ void store_elem(const GemmProblem& p, int row, int f,
 template <class Cfg>
 __global__ void __launch_bounds__(kTcThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const GemmProblem p) {
+                   const __grid_constant__ CUtensorMap tmC, const GemmProblem p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + Cfg::STAGES * Cfg::STAGE_BYTES);
+  uint8_t* stg_base = smem + Cfg::STAGES * Cfg::STAGE_BYTES;  // epilogue staging (1024-aligned)
+  uint64_t* full = reinterpret_cast<uint64_t*>(stg_base + Cfg::STG_BYTES);
   uint64_t* empty = full + Cfg::STAGES;
   uint64_t* tfull = empty + Cfg::STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* s_tiles = reinterpret_cast<int*>(stg_base + Cfg::STG_BYTES + 512);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  load_tile_tables(p, s_tiles);
   const int NT = (p.F + Cfg::FT - 1) / Cfg::FT;
   const int KB = p.K / Cfg::BK;
 
@@ -188,7 +297,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], 4);
+      mbar_init(&tempty[b], kEpiWarps);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -206,7 +315,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const int num_tiles = total_row_tiles(p) * NT;
+  const int num_tiles = total_row_tiles_s(p, s_tiles) * NT;
 
   if (warp == 0) {
     // ---------------- TMA producer ----------------
@@ -217,7 +326,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
         const int rt = t / NT, ft = t - (t / NT) * NT;
         int g, row0, rows;
-        locate_row_tile(p, rt, g, row0, rows);
+        locate_row_tile_s(p, s_tiles, rt, g, row0, rows);
         const int wrow = (int)(g * p.w_group_stride) + ft * Cfg::FT;
         const int nsub = Cfg::kSwap ? (rows + 31) / 32 : 4;
         uint32_t bytes = Cfg::NUM_W * Cfg::W_BYTES;
@@ -264,7 +373,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++it) {
         const int rt = t / NT;
         int g, row0, rows;
-        locate_row_tile(p, rt, g, row0, rows);
+        locate_row_tile_s(p, s_tiles, rt, g, row0, rows);
         const int ab = it & 1;
         const uint32_t aph = (it >> 1) & 1;
         if (!mbar_wait(&tempty[ab], aph ^ 1, abort_flag, p.err)) break;
@@ -326,7 +435,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
         const int rt = t / NT;
         int g, row0, rows;
-        locate_row_tile(p, rt, g, row0, rows);
+        locate_row_tile_s(p, s_tiles, rt, g, row0, rows);
         const int nload = Cfg::kSwap ? max(16, (rows + 15) & ~15) : 128;
         const bf16* src[16];
 #pragma unroll
@@ -351,13 +460,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       cp_async_wait<0>();
     }
   } else {
-    // ---------------- epilogue (warps 4..7) ----------------
-    const int qd = warp & 3;  // TMEM lane quarter this warp may access
+    // ---------------- epilogue (warps 4..11: two warpgroups) ----------------
+    const int qd = warp & 3;          // TMEM lane quarter this warp may access
+    const int eg = (warp - 4) >> 2;   // warpgroup: even / odd 32-column chunks
     int it = 0;
     for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++it) {
       const int rt = t / NT, ft = t - (t / NT) * NT;
       int g, row0, rows;
-      locate_row_tile(p, rt, g, row0, rows);
+      locate_row_tile_s(p, s_tiles, rt, g, row0, rows);
       const int ab = it & 1;
       const uint32_t aph = (it >> 1) & 1;
       if (!mbar_wait(&tfull[ab], aph, abort_flag, p.err)) break;
@@ -367,16 +477,23 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       float v0[32], v1[32];
       if (!Cfg::kSwap) {
         const int r = qd * 32 + lane;
-        for (int c0 = 0; c0 < Cfg::ACC_N; c0 += 32) {
+        const bool tma = p.tma_store && rows - qd * 32 >= 32;
+        uint8_t* stg = stg_base + (warp - 4) * 2048;
+        for (int c0 = 32 * eg; c0 < Cfg::ACC_N; c0 += 64) {
           tmem_ld_32x32(tb + c0, v0);
           if (Cfg::kDual) tmem_ld_32x32(tb + Cfg::ACC_N + c0, v1);
           tc_wait_ld();
-          if (r < rows && f0 + c0 < p.F)
-            store_row32<Cfg::kEpi>(p, row0 + r, f0 + c0, v0, Cfg::kDual ? v1 : nullptr);
+          if (f0 + c0 < p.F) {
+            if (tma)
+              epi_tma_chunk32<Cfg::kEpi, Cfg::kDual>(p, &tmC, stg, lane, row0 + qd * 32, f0 + c0,
+                                                     v0, v1);
+            else if (r < rows)
+              store_row32<Cfg::kEpi, Cfg::kDual>(p, row0 + r, f0 + c0, v0, v1);
+          }
         }
       } else {
         const int f = f0 + qd * 32 + lane;
-        for (int c0 = 0; c0 < rows; c0 += 32) {
+        for (int c0 = 32 * eg; c0 < rows; c0 += 64) {
           tmem_ld_32x32(tb + c0, v0);
           if (Cfg::kDual) tmem_ld_32x32(tb + Cfg::ACC_N + c0, v1);
           tc_wait_ld();
@@ -393,6 +510,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[ab]);
     }
+    if (lane == 0) bulk_wait0();  // this warp's bulk stores are complete
   }
 
   __syncthreads();
@@ -419,7 +537,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 // barrier (2-SM TMA); the leader's MMA commits arrive on `empty` and `tfull`
 // in both CTAs (multicast commit); both CTAs' epilogue warps arrive on the
 // leader's `tempty` (remote arrive).  Activations are always TMA tiles of
-// contiguous rows (the expert FC1 reads latent rows already in expert order).
+// contiguous rows (dense GEMMs, and the expert FC2 whose input rows are
+// already in expert order).
 
 template <bool kDual_, int kEpi_>
 struct TcPairCfg {
@@ -433,26 +552,32 @@ struct TcPairCfg {
   static constexpr int ACC_N = 256;              // columns of one accumulator buffer
   static constexpr int TMEM_COLS = 512;
   static constexpr int FT = kDual ? 128 : 256;   // output features per tile
-  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 512;
+  static constexpr int STG_BYTES = kEpiWarps * 2048;  // epilogue staging (bf16 boxes)
+  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + STG_BYTES + 512 +
+                                    2 * (LMOE_MAX_EXPERTS + 1) * 4;
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 };
 
 template <class Cfg>
 __global__ void __launch_bounds__(kTcThreads, 1)
     tc_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
-                        const __grid_constant__ CUtensorMap tmB, const GemmProblem p) {
+                        const __grid_constant__ CUtensorMap tmB,
+                        const __grid_constant__ CUtensorMap tmC, const GemmProblem p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + Cfg::STAGES * Cfg::STAGE_BYTES);
+  uint8_t* stg_base = smem + Cfg::STAGES * Cfg::STAGE_BYTES;  // epilogue staging (1024-aligned)
+  uint64_t* full = reinterpret_cast<uint64_t*>(stg_base + Cfg::STG_BYTES);
   uint64_t* empty = full + Cfg::STAGES;
   uint64_t* tfull = empty + Cfg::STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* s_tiles = reinterpret_cast<int*>(stg_base + Cfg::STG_BYTES + 512);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  load_tile_tables(p, s_tiles);
   const uint32_t rank = cluster_ctarank();
   const int cid = (int)cluster_id_x(), ncl = (int)cluster_count_x();
   const int NT = (p.F + Cfg::FT - 1) / Cfg::FT;
@@ -465,7 +590,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], 8);  // 4 epilogue warps in each CTA of the pair
+      mbar_init(&tempty[b], 2 * kEpiWarps);  // the epilogue warps of both CTAs
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -484,7 +609,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   cluster_sync();  // both CTAs' barriers exist before any remote arrive
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const int num_tiles = total_row_tiles(p) * NT;
+  const int num_tiles = total_row_tiles_s(p, s_tiles) * NT;
 
   if (warp == 0) {
     // ---------------- TMA producer (both CTAs) ----------------
@@ -496,7 +621,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       for (int t = cid; t < num_tiles; t += ncl) {
         const int rt = t / NT, ft = t - (t / NT) * NT;
         int g, row0, rows;
-        locate_row_tile(p, rt, g, row0, rows);
+        locate_row_tile_s(p, s_tiles, rt, g, row0, rows);
         int wrow = (int)(g * p.w_group_stride) + ft * Cfg::FT;
         wrow += Cfg::kDual ? (rank ? p.dual_offset : 0) : (int)rank * 128;
         const int arow = row0 + (int)rank * 128;
@@ -560,34 +685,44 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_wait_drain(drain, 0);
     }
   } else if (warp >= 4) {
-    // ---------------- epilogue (warps 4..7 of both CTAs) ----------------
+    // ---------------- epilogue (warps 4..11 of both CTAs) ----------------
     const int qd = warp & 3;
+    const int eg = (warp - 4) >> 2;
     const uint32_t tempty_leader = cluster_map(&tempty[0], 0);
     int it = 0;
     for (int t = cid; t < num_tiles; t += ncl, ++it) {
       const int rt = t / NT, ft = t - (t / NT) * NT;
       int g, row0, rows;
-      locate_row_tile(p, rt, g, row0, rows);
+      locate_row_tile_s(p, s_tiles, rt, g, row0, rows);
       const int ab = it & 1;
       const uint32_t aph = (it >> 1) & 1;
       if (!mbar_wait_cluster(&tfull[ab], aph, abort_flag, p.err)) break;
       tc_fence_after();
       const uint32_t tb = tmem_base + ((uint32_t)(qd * 32) << 16) + ab * Cfg::ACC_N;
       const int f0 = ft * Cfg::FT;
-      const int r = (int)rank * 128 + qd * 32 + lane;  // row within the 256-row tile
+      const int wrow = (int)rank * 128 + qd * 32;  // this warp's first row in the 256-row tile
+      const int r = wrow + lane;
+      const bool tma = p.tma_store && rows - wrow >= 32;
+      uint8_t* stg = stg_base + (warp - 4) * 2048;
       float v0[32], v1[32];
       constexpr int NCOL = Cfg::kDual ? 128 : 256;
-      for (int c0 = 0; c0 < NCOL; c0 += 32) {
+      for (int c0 = 32 * eg; c0 < NCOL; c0 += 64) {
         tmem_ld_32x32(tb + c0, v0);
         if (Cfg::kDual) tmem_ld_32x32(tb + 128 + c0, v1);
         tc_wait_ld();
-        if (r < rows && f0 + c0 < p.F)
-          store_row32<Cfg::kEpi>(p, row0 + r, f0 + c0, v0, Cfg::kDual ? v1 : nullptr);
+        if (f0 + c0 < p.F) {
+          if (tma)
+            epi_tma_chunk32<Cfg::kEpi, Cfg::kDual>(p, &tmC, stg, lane, row0 + wrow, f0 + c0, v0,
+                                                   v1);
+          else if (r < rows)
+            store_row32<Cfg::kEpi, Cfg::kDual>(p, row0 + r, f0 + c0, v0, v1);
+        }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(tempty_leader + (uint32_t)ab * 8u);
     }
+    if (lane == 0) bulk_wait0();
   }
 
   __syncthreads();
