@@ -80,14 +80,21 @@ template <typename T> __device__ __forceinline__ T from_f32(float v);
 template <> __device__ __forceinline__ float from_f32<float>(float v) { return v; }
 template <> __device__ __forceinline__ bf16 from_f32<bf16>(float v) { return __float2bfloat16_rn(v); }
 
-__device__ __forceinline__ float silu_f(float a) { return a / (1.0f + expf(-a)); }
+// SiLU a * sigmoid(a) with the fast exponential and division intrinsics: their
+// few-ulp fp32 error is far below the bf16 rounding every SiLU output gets
+// (for a < -88, __expf(-a) is +inf and the quotient is 0).
+__device__ __forceinline__ float silu_f(float a) { return __fdividef(a, 1.0f + __expf(-a)); }
+
+// SiLU with the correctly rounded exponential and division (fp32 layers).
+__device__ __forceinline__ float silu_precise(float a) { return a / (1.0f + expf(-a)); }
 
 // act of one output feature; g is the gate (or only) pre-activation and u
-// the linear half for SwiGLU.
+// the linear half for SwiGLU.  kPrecise selects silu_precise.
+template <bool kPrecise = false>
 __device__ __forceinline__ float apply_act(int act, float g, float u) {
   switch (act) {
-    case ACT_SILU: return silu_f(g);
-    case ACT_SWIGLU: return silu_f(g) * u;
+    case ACT_SILU: return kPrecise ? silu_precise(g) : silu_f(g);
+    case ACT_SWIGLU: return (kPrecise ? silu_precise(g) : silu_f(g)) * u;
     case ACT_RELU2: return g > 0.0f ? g * g : 0.0f;
     default: return g;
   }

@@ -3,11 +3,11 @@
 // (LatentMoE paper, Section 3: the top-K index set of Eq. (1)/(2) and the
 // dispatch after the down-projection).
 //
-//   topk_softmax_kernel   one warp per token.  Each logit becomes a 64-bit key
-//                         (order-preserving fp32 bits << 32 | ~expert), so one
-//                         integer max picks "largest logit, then lowest
-//                         index"; -0.0 is folded into +0.0 first.  k rounds of
-//                         warp max (two redux.sync each) give the slots; the gates are
+//   topk_softmax_kernel   one warp per token.  Each logit becomes an
+//                         order-preserving 32-bit key (-0.0 folded into +0.0);
+//                         a bitwise binary search finds the k-th largest, ties
+//                         go to the lowest expert index, and a bitonic sort of
+//                         (key, ~expert) gives slot order.  The gates are
 //                         exp(l_j - l_0) / sum over the k chosen.  Each choice
 //                         sets bit t of expert e's token bitmap.
 //   group_count_kernel    one warp per expert: popcount prefix over the
@@ -37,53 +37,97 @@ __device__ __forceinline__ float from_orderable_bits(uint32_t u) {
 
 // logits [T, N] fp32 -> idx [T, k], w [T, k]; bitmap [N, W] gets bit t of
 // token t set in the row of every chosen expert (W = ceil(T/32) words).
-static __global__ void __launch_bounds__(256) topk_softmax_kernel(const float* __restrict__ logits, int T,
-                                                           int N, int k, int* __restrict__ idx,
-                                                           float* __restrict__ w,
-                                                           uint32_t* __restrict__ bitmap, int W,
-                                                           int debug, int* err) {
-  const int lane = threadIdx.x & 31;
-  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+//
+// One warp per token; lane L holds the logits of experts L, L+32, ... as
+// order-preserving 32-bit keys.  The k-th largest key tau is found by a
+// bitwise binary search (32 steps of per-lane counts and one warp sum); the
+// selection is every key above tau plus the lowest-indexed keys equal to tau;
+// a 32-lane bitonic sort of (key << 32 | ~expert) puts the k winners in slot
+// order.  Selection and order are exact integer operations.
+static __global__ void __launch_bounds__(256) topk_softmax_kernel(const float* __restrict__ logits,
+                                                                  int T, int N, int k,
+                                                                  int* __restrict__ idx,
+                                                                  float* __restrict__ w,
+                                                                  uint32_t* __restrict__ bitmap,
+                                                                  int W, int debug, int* err) {
+  __shared__ unsigned long long s_sel[8][32];
+  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+  const int t = blockIdx.x * (blockDim.x >> 5) + wib;
   if (t >= T) return;
   const float* lg = logits + (size_t)t * N;
-  unsigned long long key[32];
-  unsigned long long best = 0;
+  uint32_t key[32];
   bool bad = false;
 #pragma unroll
   for (int i = 0; i < 32; ++i) {
     const int e = lane + 32 * i;
-    key[i] = 0;
+    key[i] = 0u;
     if (e < N) {
       const float v = __ldg(lg + e);
       if (debug && !isfinite(v)) bad = true;
-      key[i] = ((unsigned long long)orderable_bits(v) << 32) | (0xFFFFFFFFu - (uint32_t)e);
-      best = key[i] > best ? key[i] : best;
+      key[i] = orderable_bits(v);  // >= 1 for every non-NaN value
     }
   }
   if (debug && __any_sync(0xffffffffu, bad) && lane == 0) set_error(err, LMOE_DEVERR_NONFINITE);
-  unsigned long long mine = 0;
-  for (int j = 0; j < k; ++j) {
-    // warp max of the 64-bit keys as two 32-bit reductions: the value bits,
-    // then the inverted index among the lanes holding that value
-    const uint32_t hi = (uint32_t)(best >> 32);
-    const uint32_t vmax = __reduce_max_sync(0xffffffffu, hi);
-    const uint32_t imax = __reduce_max_sync(0xffffffffu, hi == vmax ? (uint32_t)best : 0u);
-    const unsigned long long top = ((unsigned long long)vmax << 32) | imax;
-    if (lane == j) mine = top;
-    const int e = (int)(0xFFFFFFFFu - (uint32_t)(top & 0xFFFFFFFFull));
-    if ((e & 31) == lane) {  // the owner drops it and rescans its keys
-      best = 0;
+
+  // tau: the largest value with at least k keys >= tau
+  uint32_t tau = 0u;
+#pragma unroll 1
+  for (int b = 31; b >= 0; --b) {
+    const uint32_t cand = tau | (1u << b);
+    uint32_t c = 0;
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        if (key[i] == top) key[i] = 0;
-        best = key[i] > best ? key[i] : best;
-      }
+    for (int i = 0; i < 32; ++i) c += key[i] >= cand ? 1u : 0u;
+    if ((int)__reduce_add_sync(0xffffffffu, c) >= k) tau = cand;
+  }
+  uint32_t gt = 0, sel = 0;
+#pragma unroll
+  for (int i = 0; i < 32; ++i)
+    if (key[i] > tau) {
+      ++gt;
+      sel |= 1u << i;
+    }
+  int need = k - (int)__reduce_add_sync(0xffffffffu, gt);  // ties to take, lowest index first
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const uint32_t tie = __ballot_sync(0xffffffffu, key[i] == tau && lane + 32 * i < N);
+    if (need > 0 && tie) {
+      if (((tie >> lane) & 1u) && __popc(tie & ((1u << lane) - 1u)) < need) sel |= 1u << i;
+      need -= min(need, __popc(tie));
     }
   }
+  // compact the k selected keys into s_sel[wib][0..k) (lane-major), then sort
+  const uint32_t cnt = __popc(sel);
+  uint32_t incl = cnt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  uint32_t pos = incl - cnt;
+#pragma unroll
+  for (int i = 0; i < 32; ++i)
+    if ((sel >> i) & 1u)
+      s_sel[wib][pos++] = ((unsigned long long)key[i] << 32) |
+                          (0xFFFFFFFFu - (uint32_t)(lane + 32 * i));
+  __syncwarp();
+  unsigned long long v = lane < k ? s_sel[wib][lane] : 0ull;
+  // bitonic sort, descending over the 32 lanes
+#pragma unroll
+  for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      const unsigned long long o = __shfl_xor_sync(0xffffffffu, v, stride);
+      const bool desc = (lane & size) == 0;
+      const bool lower = (lane & stride) == 0;
+      const unsigned long long hi = v > o ? v : o, lo = v > o ? o : v;
+      v = (lower == desc) ? hi : lo;
+    }
+  }
+  const unsigned long long mine = v;
   const int e = (int)(0xFFFFFFFFu - (uint32_t)(mine & 0xFFFFFFFFull));
-  const float v = from_orderable_bits((uint32_t)(mine >> 32));
-  const float l0 = __shfl_sync(0xffffffffu, v, 0);
-  const float ex = lane < k ? expf(v - l0) : 0.f;
+  const float val = from_orderable_bits((uint32_t)(mine >> 32));
+  const float l0 = __shfl_sync(0xffffffffu, val, 0);
+  const float ex = lane < k ? expf(val - l0) : 0.f;
   float sum = ex;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);

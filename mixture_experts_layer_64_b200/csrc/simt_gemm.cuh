@@ -18,7 +18,7 @@ __device__ __forceinline__ void simt_store(const GemmProblem& p, int row, int f,
   if (kEpi == EPI_F32_BIAS) {
     static_cast<float*>(e.out)[(size_t)row * e.ldo + f] = v0 + (e.bias ? e.bias[f] : 0.f);
   } else if (kEpi == EPI_ACT) {
-    const float v = apply_act(e.act, v0, v1);
+    const float v = apply_act<sizeof(T) == 4>(e.act, v0, v1);
     T* o = static_cast<T*>(e.out) + (size_t)row * e.ldo + e.col0 + f;
     const T hi = from_f32<T>(v);
     o[0] = hi;
