@@ -43,7 +43,7 @@ METRIC = "LatentMoE layer tokens/sec at decode & prefill T; HBM GB/s / tensor-pi
 UNIT = "tokens/s"
 DEFAULT_WORKLOAD = "std-moe-decode"
 EXPERT_PATHS = ["cuda-core", "tcgen05 token-tiled", "tcgen05 weight-stationary",
-                "tcgen05 token-tiled, 2-SM CTA pairs"]
+                "tcgen05 token-tiled, 2-SM CTA pairs", "tcgen05 weight-stationary, 2-SM CTA pairs"]
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 _CSRC = "mixture_experts_layer_64_b200/csrc/"
 _GEMM_SRC = (_CSRC + "common.cuh", _CSRC + "tc_gemm.cuh")
@@ -408,8 +408,8 @@ def run_ours(args):
                 "gpu_launches": launches_per_step * args.steps,
                 "lib_flags": args.lib_flags,
                 "roofline": roofline, "cpu_baseline": cpu_baseline, "clocks": clocks,
-                "expert_path": {"fc1": EXPERT_PATHS[max(0, L.last_expert_path) & 3],
-                                "fc2": EXPERT_PATHS[max(0, L.last_expert_path) >> 2]}}
+                "expert_path": {"fc1": EXPERT_PATHS[max(0, L.last_expert_path) & 7],
+                                "fc2": EXPERT_PATHS[max(0, L.last_expert_path) >> 3]}}
         print(json.dumps(line), flush=True)
     L.close()
     if pg:

@@ -67,11 +67,19 @@ typedef enum { LMOE_F32 = 0, LMOE_BF16 = 1 } lmoe_dtype;
 #define LMOE_DEBUG_CHECKS  0x2u  /* device range checks and non-finite checks   */
 #define LMOE_FORCE_SIMT    0x4u  /* bf16: every contraction on the CUDA-core
                                     kernels instead of tcgen05 (for testing)    */
-#define LMOE_FORCE_SWAP    0x8u  /* always use the weight-stationary (swap-AB)
-                                    expert kernels (for testing)                */
-#define LMOE_FORCE_NOSWAP  0x10u /* never use them (for testing)                */
+#define LMOE_FORCE_SWAP    0x8u  /* always use the single-CTA weight-stationary
+                                    (swap-AB) expert kernels (for testing)      */
+#define LMOE_FORCE_NOSWAP  0x10u /* never use the weight-stationary expert
+                                    kernels (for testing)                       */
 #define LMOE_FORCE_NOPAIR  0x20u /* never use the 2-SM (CTA pair) tensor-core
                                     kernels (for testing)                       */
+#define LMOE_FORCE_WS_PAIR 0x40u /* expert FC1 and FC2 on the weight-stationary
+                                    kernel on CTA pairs wherever the single-CTA
+                                    weight-stationary kernel is not used.  It
+                                    pads an expert's last tile to 16 rows, not
+                                    to 128/256, but its 2-SM MMAs with N < 256
+                                    run below full rate, which makes it slower
+                                    at a few hundred rows per expert.           */
 
 /* Limits of this build. */
 #define LMOE_MAX_EXPERTS 1024
@@ -248,9 +256,11 @@ lmoe_status lmoe_route_only_noalloc(const float* logits, int T, int N, int k, in
 /* Kernel launches the last lmoe_forward enqueued (library kernels only). */
 int lmoe_last_launch_count(const lmoe_layer* h);
 
-/* Which expert kernels the last lmoe_forward used, FC1 in bits 0-1 and FC2
- * in bits 2-3, each: 0 CUDA-core, 1 tcgen05 token-tiled, 2 tcgen05
- * weight-stationary (swap-AB), 3 tcgen05 token-tiled on CTA pairs (2-SM MMA). */
+/* Which expert kernels the last lmoe_forward used, FC1 in bits 0-2 and FC2
+ * in bits 3-5, each: 0 CUDA-core, 1 tcgen05 token-tiled, 2 tcgen05
+ * weight-stationary (swap-AB), 3 tcgen05 token-tiled on CTA pairs (2-SM MMA),
+ * 4 tcgen05 weight-stationary on CTA pairs (the expert's rows as the MMA's N,
+ * split into tiles of nearly equal size in units of 16 rows). */
 int lmoe_last_expert_path(const lmoe_layer* h);
 
 const char* lmoe_status_string(lmoe_status s);

@@ -120,6 +120,12 @@ lmoe_status cuda_fail(lmoe_layer* h, cudaError_t e, const char* what) {
   return e == cudaErrorMemoryAllocation ? LMOE_ERR_OOM : LMOE_ERR_CUDA;
 }
 
+#define LMOE_TRY(expr)               \
+  do {                               \
+    lmoe_status s_ = (expr);         \
+    if (s_ != LMOE_OK) return s_;    \
+  } while (0)
+
 #define LMOE_CUDA(h, call)                                 \
   do {                                                     \
     cudaError_t e_ = (call);                               \
@@ -147,6 +153,7 @@ struct GemmCall {
   long out_rows;  // rows of the output (TMA store bounds)
   bool swap;    // weight-stationary expert kernels
   bool pair;    // 2-SM token-tiled kernels on CTA pairs (256-row tiles)
+  bool ws_pair;  // grouped: weight-stationary kernel on CTA pairs (rows on N)
 };
 
 bool encode_map(CUtensorMap* map, const void* ptr, long rows, int cols, long ld, int box_rows) {
@@ -223,34 +230,56 @@ lmoe_status launch_tc(lmoe_layer* h, const GemmCall& c, cudaStream_t st) {
   return LMOE_OK;
 }
 
+// Largest number of co-resident CTA pairs of a 2-SM kernel (cluster size 2).
+template <typename Kern>
+lmoe_status pair_setup(lmoe_layer* h, Kern kern, int smem_bytes, int* max_clusters) {
+  LMOE_CUDA(h, cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes));
+  LMOE_CUDA(h, cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 0));
+  cudaLaunchConfig_t q = {};
+  cudaLaunchAttribute qa[1];
+  qa[0].id = cudaLaunchAttributeClusterDimension;
+  qa[0].val.clusterDim.x = 2;
+  qa[0].val.clusterDim.y = 1;
+  qa[0].val.clusterDim.z = 1;
+  q.gridDim = dim3(2 * (h->num_sms / 2), 1, 1);
+  q.blockDim = dim3(kTcThreads, 1, 1);
+  q.dynamicSmemBytes = smem_bytes;
+  q.attrs = qa;
+  q.numAttrs = 1;
+  LMOE_CUDA(h, cudaOccupancyMaxActiveClusters(max_clusters, kern, &q));
+  if (*max_clusters < 1) {
+    h->detail = "no CTA pair of the 2-SM kernel fits on the device";
+    return LMOE_ERR_UNSUPPORTED;
+  }
+  return LMOE_OK;
+}
+
+// Launches `clusters` CTA pairs of a 2-SM kernel.
+template <typename Kern, typename... Args>
+lmoe_status pair_launch(lmoe_layer* h, Kern kern, int smem_bytes, long clusters, cudaStream_t st,
+                        Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3((unsigned)(2 * clusters), 1, 1);
+  cfg.blockDim = dim3(kTcThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem_bytes;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  LMOE_CUDA(h, cudaLaunchKernelEx(&cfg, kern, args...));
+  ++h->launches;
+  return LMOE_OK;
+}
+
 template <class Cfg>
 lmoe_status launch_pair(lmoe_layer* h, const GemmCall& c, cudaStream_t st) {
-  static bool attr_done = false;
   static int max_clusters = 0;
-  if (!attr_done) {
-    LMOE_CUDA(h, cudaFuncSetAttribute(tc_gemm_pair_kernel<Cfg>,
-                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      Cfg::SMEM_BYTES));
-    LMOE_CUDA(h, cudaFuncSetAttribute(tc_gemm_pair_kernel<Cfg>,
-                                      cudaFuncAttributeNonPortableClusterSizeAllowed, 0));
-    cudaLaunchConfig_t q = {};
-    cudaLaunchAttribute qa[1];
-    qa[0].id = cudaLaunchAttributeClusterDimension;
-    qa[0].val.clusterDim.x = 2;
-    qa[0].val.clusterDim.y = 1;
-    qa[0].val.clusterDim.z = 1;
-    q.gridDim = dim3(2 * (h->num_sms / 2), 1, 1);
-    q.blockDim = dim3(kTcThreads, 1, 1);
-    q.dynamicSmemBytes = Cfg::SMEM_BYTES;
-    q.attrs = qa;
-    q.numAttrs = 1;
-    LMOE_CUDA(h, cudaOccupancyMaxActiveClusters(&max_clusters, tc_gemm_pair_kernel<Cfg>, &q));
-    if (max_clusters < 1) {
-      h->detail = "no CTA pair of the 2-SM kernel fits on the device";
-      return LMOE_ERR_UNSUPPORTED;
-    }
-    attr_done = true;
-  }
+  if (max_clusters == 0)
+    LMOE_TRY(pair_setup(h, tc_gemm_pair_kernel<Cfg>, Cfg::SMEM_BYTES, &max_clusters));
   CUtensorMap ta, tb;
   std::memset(&ta, 0, sizeof ta);
   std::memset(&tb, 0, sizeof tb);
@@ -262,25 +291,36 @@ lmoe_status launch_pair(lmoe_layer* h, const GemmCall& c, cudaStream_t st) {
   const long NT = (c.p.F + Cfg::FT - 1) / Cfg::FT;
   const long tiles = (long)c.p.max_row_tiles * NT;
   const long clusters = std::max(1L, std::min<long>(max_clusters, tiles));
-  cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.gridDim = dim3((unsigned)(2 * clusters), 1, 1);
-  cfg.blockDim = dim3(kTcThreads, 1, 1);
-  cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
-  cfg.stream = st;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
   CUtensorMap tc;
   std::memset(&tc, 0, sizeof tc);
   GemmProblem p = c.p;
   p.tma_store = (tma_store_ok(c) && encode_out_map(&tc, c)) ? 1 : 0;
-  LMOE_CUDA(h, cudaLaunchKernelEx(&cfg, tc_gemm_pair_kernel<Cfg>, ta, tb, tc, p));
-  ++h->launches;
-  return LMOE_OK;
+  return pair_launch(h, tc_gemm_pair_kernel<Cfg>, Cfg::SMEM_BYTES, clusters, st, ta, tb, tc, p);
+}
+
+// Grouped expert GEMM, weight-stationary on CTA pairs: the expert's rows are
+// split into ceil(rows / NMAX) tiles, whose counts are the 128- or 256-row
+// tile prefix of the grouping step.
+template <class Cfg>
+lmoe_status launch_pair_ws(lmoe_layer* h, const GemmCall& c, cudaStream_t st) {
+  static int max_clusters = 0;
+  if (max_clusters == 0)
+    LMOE_TRY(pair_setup(h, tc_gemm_pair_ws_kernel<Cfg>, Cfg::SMEM_BYTES, &max_clusters));
+  CUtensorMap ta, tb;
+  std::memset(&ta, 0, sizeof ta);
+  std::memset(&tb, 0, sizeof tb);
+  if ((!Cfg::kGather && !encode_map(&ta, c.p.A, c.a_rows, c.p.K, c.p.lda, 32)) ||
+      !encode_map(&tb, c.p.B, c.b_rows, c.p.K, c.p.K, 128)) {
+    h->detail = "cuTensorMapEncodeTiled failed";
+    return LMOE_ERR_CUDA;
+  }
+  GemmProblem p = c.p;
+  p.tile_prefix = Cfg::NMAX == 2 * kRowTile ? h->tile_prefix2 : h->tile_prefix;
+  p.row_tile = Cfg::NMAX;
+  const long max_row_tiles = (long)c.out_rows / Cfg::NMAX + h->N;
+  const long NT = (c.p.F + Cfg::FT - 1) / Cfg::FT;
+  const long clusters = std::max(1L, std::min<long>(max_clusters, max_row_tiles * NT));
+  return pair_launch(h, tc_gemm_pair_ws_kernel<Cfg>, Cfg::SMEM_BYTES, clusters, st, ta, tb, p);
 }
 
 template <typename T, bool kDual, int kEpi>
@@ -345,6 +385,14 @@ lmoe_status run_gemm(lmoe_layer* h, GemmCall c, cudaStream_t st, int* path = nul
     return h->dtype == LMOE_F32 ? dispatch_simt<float>(h, c, st) : dispatch_simt<bf16>(h, c, st);
   }
   const bool dual = c.p.dual_offset > 0;
+  if (c.ws_pair && c.p.offsets) {
+    if (path) *path = 4;
+    if (c.kind == GK_FC1 && c.p.gather)
+      return dual ? launch_pair_ws<TcPairWsCfg<true, true, EPI_ACT>>(h, c, st)
+                  : launch_pair_ws<TcPairWsCfg<true, false, EPI_ACT>>(h, c, st);
+    if (c.kind == GK_FC2 && !c.p.gather)
+      return launch_pair_ws<TcPairWsCfg<false, false, EPI_SCALE_ROWS>>(h, c, st);
+  }
   if (path) *path = c.pair ? 3 : (c.swap ? 2 : 1);
   if (c.pair) {
     switch (c.kind) {
@@ -452,9 +500,11 @@ lmoe_status run_routing(lmoe_layer* h, const float* logits, int T, int* idx, flo
                         int* tile_prefix2, cudaStream_t st, bool marks) {
   const int W = (T + 31) / 32;
   const int debug = (h->flags & LMOE_DEBUG_CHECKS) ? 1 : 0;
-  topk_softmax_kernel<<<(T + 7) / 8, 256, 0, st>>>(logits, T, h->N, h->k, idx, w, h->bitmap, W,
-                                                   debug, h->err);
-  LMOE_CHECK_LAUNCH(h);
+  {
+    const cudaError_t e = launch_topk(logits, T, h->N, h->k, idx, w, h->bitmap, W, debug, h->err, st);
+    if (e != cudaSuccess) return cuda_fail(h, e, "top-k launch");
+    ++h->launches;
+  }
   if (marks) prof_mark(h, st, 2);
   group_count_kernel<<<(h->N + 7) / 8, 256, 0, st>>>(h->bitmap, h->wp, h->N, W, h->counts, offsets,
                                                      h->tile_prefix, tile_prefix2, h->done);
@@ -476,12 +526,6 @@ lmoe_status run_router(lmoe_layer* h, const void* x, float* logits, int T, cudaS
   return run_gemm(h, c, st);
 }
 
-#define LMOE_TRY(expr)               \
-  do {                               \
-    lmoe_status s_ = (expr);         \
-    if (s_ != LMOE_OK) return s_;    \
-  } while (0)
-
 lmoe_status run_forward(lmoe_layer* h, const void* x, void* out, int T, cudaStream_t st) {
   h->launches = 0;
   const bool skip = (h->flags & LMOE_SKIP_PROJ) != 0;
@@ -500,6 +544,10 @@ lmoe_status run_forward(lmoe_layer* h, const void* x, void* out, int T, cudaStre
   // expert FC1 gathers its rows by token and stays on single CTAs)
   const bool pair_dense = pairs_ok && T >= 1024;
   const bool pair_fc2 = pairs_ok && !swap;
+  // on request: the expert GEMMs weight-stationary on CTA pairs (rows on the
+  // MMA's N, so an expert's last tile is padded to 16 rows, not 128 or 256)
+  const bool ws_pair = pairs_ok && !swap && (h->flags & LMOE_FORCE_WS_PAIR) &&
+                       !(h->flags & LMOE_FORCE_NOSWAP);
   if (!skip) {
     GemmCall c = dense_call(GK_DENSE_ACT, T, x, d, h->Wd_t, l, d);
     c.p.epi.out = h->z;
@@ -534,6 +582,7 @@ lmoe_status run_forward(lmoe_layer* h, const void* x, void* out, int T, cudaStre
     const void* A = skip ? x : h->z;
     GemmCall c = grouped_call(h, GK_FC1, T, A, skip ? d : l, T, h->row_tok, h->W1_t, h->m_in, m, l);
     c.swap = swap;
+    c.ws_pair = ws_pair;
     c.p.dual_offset = h->act == LMOE_ACT_SWIGLU ? m : 0;
     c.p.epi.out = h->h;
     c.p.epi.ldo = m;
@@ -545,14 +594,15 @@ lmoe_status run_forward(lmoe_layer* h, const void* x, void* out, int T, cudaStre
   prof_mark(h, st, 6);
   {
     GemmCall c = grouped_call(h, GK_FC2, T, h->h, m, R, nullptr, h->W2_t, l, l, m);
-    if (pair_fc2) make_pair(h, c);
+    if (pair_fc2 && !ws_pair) make_pair(h, c);
     c.swap = swap;
+    c.ws_pair = ws_pair;
     c.p.epi.out = h->ys;
     c.p.epi.ldo = l;
     c.p.epi.row_w = h->row_w;
     int path = 0;
     LMOE_TRY(run_gemm(h, c, st, &path));
-    h->expert_path |= path << 2;
+    h->expert_path |= path << 3;
   }
   prof_mark(h, st, 7);
   {
@@ -694,7 +744,7 @@ lmoe_status lmoe_create(int d, int l, int N, int k, int m, lmoe_act act, int sha
   if (!out) return LMOE_ERR_INVALID_ARG;
   *out = nullptr;
   const unsigned known = LMOE_SKIP_PROJ | LMOE_DEBUG_CHECKS | LMOE_FORCE_SIMT | LMOE_FORCE_SWAP |
-                         LMOE_FORCE_NOSWAP | LMOE_FORCE_NOPAIR;
+                         LMOE_FORCE_NOSWAP | LMOE_FORCE_NOPAIR | LMOE_FORCE_WS_PAIR;
   if (d <= 0 || l <= 0 || N <= 0 || k <= 0 || m <= 0 || shared_m < 0) return LMOE_ERR_INVALID_ARG;
   if (k > N || (flags & ~known)) return LMOE_ERR_INVALID_ARG;
   if (act != LMOE_ACT_SILU && act != LMOE_ACT_SWIGLU && act != LMOE_ACT_RELU2) return LMOE_ERR_INVALID_ARG;

@@ -5,11 +5,12 @@
 //
 //   topk_softmax_kernel   one warp per token.  Each logit becomes an
 //                         order-preserving 32-bit key (-0.0 folded into +0.0);
-//                         a bitwise binary search finds the k-th largest, ties
-//                         go to the lowest expert index, and a bitonic sort of
-//                         (key, ~expert) gives slot order.  The gates are
-//                         exp(l_j - l_0) / sum over the k chosen.  Each choice
-//                         sets bit t of expert e's token bitmap.
+//                         the keys that can be in the top k (at or above the
+//                         k-th largest lane maximum) are sorted by (key,
+//                         ~expert); a radix select takes over when too many
+//                         pass.  Ties go to the lowest expert index.  The
+//                         gates are exp(l_j - l_0) / sum over the k chosen.
+//                         Each choice sets bit t of expert e's token bitmap.
 //   group_count_kernel    one warp per expert: popcount prefix over the
 //                         expert's bitmap words (also clears them for the next
 //                         call); the last block to finish scans the loads
@@ -35,67 +36,165 @@ __device__ __forceinline__ float from_orderable_bits(uint32_t u) {
   return __uint_as_float((u & 0x80000000u) ? (u & 0x7FFFFFFFu) : ~u);
 }
 
+// Bitonic sort of 32 values across a warp (one per lane), descending.
+template <typename V>
+__device__ __forceinline__ V warp_sort_desc32(V v, int lane) {
+#pragma unroll
+  for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      const V o = __shfl_xor_sync(0xffffffffu, v, stride);
+      const bool keep_hi = ((lane & stride) == 0) == ((lane & size) == 0);
+      v = keep_hi ? (v > o ? v : o) : (v > o ? o : v);
+    }
+  }
+  return v;
+}
+
+// Bitonic sort of 64 values across a warp, descending: lane L holds elements
+// L (a) and L + 32 (b).  On return a holds the 32 largest in order.
+__device__ __forceinline__ void warp_sort_desc64(unsigned long long& a, unsigned long long& b,
+                                                 int lane) {
+#pragma unroll
+  for (int size = 2; size <= 64; size <<= 1) {
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      if (stride == 32) {  // a and b are partners; size 64 sorts descending
+        const unsigned long long hi = a > b ? a : b, lo = a > b ? b : a;
+        a = hi;
+        b = lo;
+      } else {
+        const unsigned long long oa = __shfl_xor_sync(0xffffffffu, a, stride);
+        const unsigned long long ob = __shfl_xor_sync(0xffffffffu, b, stride);
+        const bool lower = (lane & stride) == 0;
+        const bool keep_a = lower == ((lane & size) == 0);
+        const bool keep_b = lower == (((lane + 32) & size) == 0);
+        a = keep_a ? (a > oa ? a : oa) : (a > oa ? oa : a);
+        b = keep_b ? (b > ob ? b : ob) : (b > ob ? ob : b);
+      }
+    }
+  }
+}
+
 // logits [T, N] fp32 -> idx [T, k], w [T, k]; bitmap [N, W] gets bit t of
 // token t set in the row of every chosen expert (W = ceil(T/32) words).
 //
-// One warp per token; lane L holds the logits of experts L, L+32, ... as
-// order-preserving 32-bit keys.  The k-th largest key tau is found by a
-// bitwise binary search (32 steps of per-lane counts and one warp sum); the
-// selection is every key above tau plus the lowest-indexed keys equal to tau;
-// a 32-lane bitonic sort of (key << 32 | ~expert) puts the k winners in slot
-// order.  Selection and order are exact integer operations.
-static __global__ void __launch_bounds__(256) topk_softmax_kernel(const float* __restrict__ logits,
-                                                                  int T, int N, int k,
-                                                                  int* __restrict__ idx,
-                                                                  float* __restrict__ w,
-                                                                  uint32_t* __restrict__ bitmap,
-                                                                  int W, int debug, int* err) {
-  __shared__ unsigned long long s_sel[8][32];
+// One warp per token; lane L holds the logits of experts L, L+32, ...
+// (NPL >= ceil(N/32) slots) as order-preserving 32-bit keys.
+//
+// Candidates: with theta the k-th largest of the 32 lane maxima, at least k
+// keys are >= theta, so every one of the top k is >= theta.  When at most 64
+// keys pass, they are sorted by (key, lowest expert first) and the first k
+// are the answer.  Otherwise (many equal or crowded logits) a radix select
+// finds the k-th largest key tau exactly (four passes over 8-bit digits, each
+// a 256-bin histogram in shared memory of the keys matching the digits
+// decided so far); the selection is every key above tau plus the
+// lowest-indexed keys equal to tau.  Selection and order are exact integer
+// operations in both branches.
+template <int NPL>
+__global__ void __launch_bounds__(256) topk_softmax_kernel(const float* __restrict__ logits, int T,
+                                                           int N, int k, int* __restrict__ idx,
+                                                           float* __restrict__ w,
+                                                           uint32_t* __restrict__ bitmap, int W,
+                                                           int debug, int* err) {
+  __shared__ uint32_t s_hist[8][256];
+  __shared__ unsigned long long s_sel[8][64];
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
   const int t = blockIdx.x * (blockDim.x >> 5) + wib;
   if (t >= T) return;
   const float* lg = logits + (size_t)t * N;
-  uint32_t key[32];
+  uint32_t key[NPL];
   bool bad = false;
 #pragma unroll
-  for (int i = 0; i < 32; ++i) {
+  for (int i = 0; i < NPL; ++i) {
     const int e = lane + 32 * i;
-    key[i] = 0u;
+    key[i] = 0u;  // absent experts: 0, never above a real key and never counted
     if (e < N) {
       const float v = __ldg(lg + e);
       if (debug && !isfinite(v)) bad = true;
-      key[i] = orderable_bits(v);  // >= 1 for every non-NaN value
+      key[i] = orderable_bits(v);
     }
   }
   if (debug && __any_sync(0xffffffffu, bad) && lane == 0) set_error(err, LMOE_DEVERR_NONFINITE);
 
-  // tau: the largest value with at least k keys >= tau
-  uint32_t tau = 0u;
+  uint32_t lmax = 0u;
+#pragma unroll
+  for (int i = 0; i < NPL; ++i) lmax = max(lmax, key[i]);
+  const uint32_t theta = __shfl_sync(0xffffffffu, warp_sort_desc32(lmax, lane), k - 1);
+  uint32_t sel = 0;
+#pragma unroll
+  for (int i = 0; i < NPL; ++i)
+    if (lane + 32 * i < N && key[i] >= theta) sel |= 1u << i;
+  int ncand = (int)__reduce_add_sync(0xffffffffu, (uint32_t)__popc(sel));
+
+  if (ncand > 64) {
+    // radix select of the k-th largest key
+    uint32_t* hist = s_hist[wib];
+    uint32_t tau = 0u, tmask = 0u;
+    int kk = k;  // rank of tau among the keys that match the decided digits
 #pragma unroll 1
-  for (int b = 31; b >= 0; --b) {
-    const uint32_t cand = tau | (1u << b);
-    uint32_t c = 0;
+    for (int shift = 24; shift >= 0; shift -= 8) {
 #pragma unroll
-    for (int i = 0; i < 32; ++i) c += key[i] >= cand ? 1u : 0u;
-    if ((int)__reduce_add_sync(0xffffffffu, c) >= k) tau = cand;
-  }
-  uint32_t gt = 0, sel = 0;
+      for (int j = 0; j < 8; ++j) hist[lane * 8 + j] = 0u;
+      __syncwarp();
 #pragma unroll
-  for (int i = 0; i < 32; ++i)
-    if (key[i] > tau) {
-      ++gt;
-      sel |= 1u << i;
+      for (int i = 0; i < NPL; ++i)
+        if (lane + 32 * i < N && (key[i] & tmask) == tau)
+          atomicAdd(&hist[(key[i] >> shift) & 255u], 1u);
+      __syncwarp();
+      // lane L owns digits 255 - 8L ... 248 - 8L (descending across the warp)
+      uint32_t h[8], sum = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        h[j] = hist[255 - 8 * lane - j];
+        sum += h[j];
+      }
+      uint32_t incl = sum;  // keys with digit >= this lane's lowest digit
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      const uint32_t before = incl - sum;  // keys with digit above this lane's bins
+      const bool here = before < (uint32_t)kk && incl >= (uint32_t)kk;
+      const int src = __ffs(__ballot_sync(0xffffffffu, here)) - 1;
+      uint32_t digit = 0, above = 0;
+      if (lane == src) {
+        uint32_t run = before;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if (run + h[j] >= (uint32_t)kk) {
+            digit = 255 - 8 * lane - j;
+            above = run;
+            break;
+          }
+          run += h[j];
+        }
+      }
+      digit = __shfl_sync(0xffffffffu, digit, src);
+      above = __shfl_sync(0xffffffffu, above, src);
+      tau |= digit << shift;
+      tmask |= 255u << shift;
+      kk -= (int)above;
+      __syncwarp();
     }
-  int need = k - (int)__reduce_add_sync(0xffffffffu, gt);  // ties to take, lowest index first
+    sel = 0;
 #pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    const uint32_t tie = __ballot_sync(0xffffffffu, key[i] == tau && lane + 32 * i < N);
-    if (need > 0 && tie) {
-      if (((tie >> lane) & 1u) && __popc(tie & ((1u << lane) - 1u)) < need) sel |= 1u << i;
-      need -= min(need, __popc(tie));
+    for (int i = 0; i < NPL; ++i)
+      if (key[i] > tau) sel |= 1u << i;
+    int need = kk;  // keys equal to tau still to take, lowest index first
+#pragma unroll
+    for (int i = 0; i < NPL; ++i) {
+      if (need > 0) {
+        const uint32_t tie = __ballot_sync(0xffffffffu, key[i] == tau && lane + 32 * i < N);
+        if (((tie >> lane) & 1u) && __popc(tie & ((1u << lane) - 1u)) < need) sel |= 1u << i;
+        need -= min(need, __popc(tie));
+      }
     }
+    ncand = k;
   }
-  // compact the k selected keys into s_sel[wib][0..k) (lane-major), then sort
+
+  // compact the selected keys into s_sel[wib][0..ncand) (lane-major), then sort
   const uint32_t cnt = __popc(sel);
   uint32_t incl = cnt;
 #pragma unroll
@@ -105,27 +204,20 @@ static __global__ void __launch_bounds__(256) topk_softmax_kernel(const float* _
   }
   uint32_t pos = incl - cnt;
 #pragma unroll
-  for (int i = 0; i < 32; ++i)
+  for (int i = 0; i < NPL; ++i)
     if ((sel >> i) & 1u)
       s_sel[wib][pos++] = ((unsigned long long)key[i] << 32) |
                           (0xFFFFFFFFu - (uint32_t)(lane + 32 * i));
   __syncwarp();
-  unsigned long long v = lane < k ? s_sel[wib][lane] : 0ull;
-  // bitonic sort, descending over the 32 lanes
-#pragma unroll
-  for (int size = 2; size <= 32; size <<= 1) {
-#pragma unroll
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      const unsigned long long o = __shfl_xor_sync(0xffffffffu, v, stride);
-      const bool desc = (lane & size) == 0;
-      const bool lower = (lane & stride) == 0;
-      const unsigned long long hi = v > o ? v : o, lo = v > o ? o : v;
-      v = (lower == desc) ? hi : lo;
-    }
+  unsigned long long v = lane < ncand ? s_sel[wib][lane] : 0ull;
+  if (ncand <= 32) {
+    v = warp_sort_desc32(v, lane);
+  } else {
+    unsigned long long b = lane + 32 < ncand ? s_sel[wib][lane + 32] : 0ull;
+    warp_sort_desc64(v, b, lane);
   }
-  const unsigned long long mine = v;
-  const int e = (int)(0xFFFFFFFFu - (uint32_t)(mine & 0xFFFFFFFFull));
-  const float val = from_orderable_bits((uint32_t)(mine >> 32));
+  const int e = (int)(0xFFFFFFFFu - (uint32_t)(v & 0xFFFFFFFFull));
+  const float val = from_orderable_bits((uint32_t)(v >> 32));
   const float l0 = __shfl_sync(0xffffffffu, val, 0);
   const float ex = lane < k ? expf(val - l0) : 0.f;
   float sum = ex;
@@ -136,6 +228,33 @@ static __global__ void __launch_bounds__(256) topk_softmax_kernel(const float* _
     w[(size_t)t * k + lane] = ex / sum;
     atomicOr(bitmap + (size_t)e * W + (t >> 5), 1u << (t & 31));
   }
+}
+
+// Launches topk_softmax_kernel with the smallest multiple of 4 slots per lane
+// that covers N.
+static inline cudaError_t launch_topk(const float* logits, int T, int N, int k, int* idx, float* w,
+                                      uint32_t* bitmap, int W, int debug, int* err,
+                                      cudaStream_t st) {
+  const dim3 grid((T + 7) / 8), block(256);
+#define LMOE_TOPK_CASE(S)                                                                      \
+  case S:                                                                                      \
+    topk_softmax_kernel<S><<<grid, block, 0, st>>>(logits, T, N, k, idx, w, bitmap, W, debug, \
+                                                   err);                                       \
+    break;
+  switch ((N + 127) / 128 * 4) {
+    LMOE_TOPK_CASE(4)
+    LMOE_TOPK_CASE(8)
+    LMOE_TOPK_CASE(12)
+    LMOE_TOPK_CASE(16)
+    LMOE_TOPK_CASE(20)
+    LMOE_TOPK_CASE(24)
+    LMOE_TOPK_CASE(28)
+    LMOE_TOPK_CASE(32)
+    default:
+      return cudaErrorInvalidValue;
+  }
+#undef LMOE_TOPK_CASE
+  return cudaGetLastError();
 }
 
 // Word prefix + bits: wp[e][wd] = {set bits of expert e in words < wd, word wd}.

@@ -733,4 +733,329 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   }
 }
 
+
+// ==== weight-stationary grouped GEMM on CTA pairs ================================
+//
+// The prefill expert GEMMs.  Token-tiled tiles have 128 (or, on pairs, 256)
+// rows, and an expert's last tile is padded to that size: with a few hundred
+// rows per expert a fifth to two fifths of the tensor-core work is padding.
+// Here the expert's rows are the MMA's N dimension, which only needs a
+// multiple of 16: one tcgen05.mma.cta_group::2 of M = 256 weight rows
+// (features; each CTA stages 128) and N = the tile's rows (each CTA stages
+// half), with an expert's rows split into ceil(rows / NMAX) tiles of nearly
+// equal size in units of 16.  Splitting the rows across the pair keeps the
+// shared-memory operand reads at or below those of a 1-CTA 128 x 256 tile
+// for N >= ~100.
+//
+// Gated FC1 (SwiGLU) issues two MMAs per K step, gate rows and linear rows of
+// the same 256 features, into accumulators at TMEM columns [0, N) and
+// [128, 128 + N): NMAX = 128 keeps two buffers in 512 columns.  Ungated
+// problems use NMAX = 256.
+//
+// Rows reach shared memory by TMA (contiguous rows: FC2) or by the cp.async
+// gather of both CTAs (FC1 reads the down-projected tokens by index).  The
+// peer CTA's gather completes on its own mbarrier (cp.async can only signal
+// the executing CTA's barriers), and its warp 1 relays each completed stage
+// to the leader's `full` barrier with a remote arrive.
+//
+// Epilogue: TMEM lane = feature, column = row, so each thread holds one
+// feature of 32 rows and a warp writes 64 contiguous bytes of every row.
+
+template <bool kGather_, bool kDual_, int kEpi_>
+struct TcPairWsCfg {
+  static constexpr bool kGather = kGather_, kDual = kDual_;
+  static constexpr int kEpi = kEpi_;
+  static constexpr int BK = 64;
+  static constexpr int NUM_W = kDual ? 2 : 1;
+  static constexpr int NMAX = kDual ? 128 : 256;  // rows per tile (the MMA's N), at most
+  static constexpr int W_BYTES = 128 * BK * 2;    // this CTA's 128 weight rows
+  static constexpr int B_ROWS = NMAX / 2;         // this CTA's rows of a tile, at most
+  static constexpr int B_BYTES = B_ROWS * BK * 2;
+  static constexpr int STAGE_BYTES = NUM_W * W_BYTES + B_BYTES;
+  static constexpr int STAGES_RAW = kTcSmemBudget / STAGE_BYTES;
+  static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
+  static constexpr int ACC_COLS = 256;            // one accumulator buffer
+  static constexpr int TMEM_COLS = 512;
+  static constexpr int FT = 256;                  // output features per tile (128 per CTA)
+  static constexpr int TABLE_BYTES = 2 * (LMOE_MAX_EXPERTS + 1) * 4;
+  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 512 + TABLE_BYTES;
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
+  static_assert(STAGES >= 3, "pipeline too shallow");
+  static_assert(kEpi == EPI_ACT || kEpi == EPI_SCALE_ROWS, "grouped epilogues");
+  static_assert(kGather || B_ROWS % 32 == 0, "row boxes of 32");
+};
+
+// Row tile rt of a grouped problem split into nearly equal tiles: group g,
+// first row row0, valid rows n, and the MMA's N (n rounded up to 16; at most
+// NMAX when the tile counts are ceil(rows / NMAX)).
+__device__ __forceinline__ void locate_ws_tile(const GemmProblem& p, const int* s_tiles, int rt,
+                                               int& g, int& row0, int& n, int& nmma) {
+  const int* tp = s_tiles;
+  const int* off = s_tiles + LMOE_MAX_EXPERTS + 1;
+  int lo = 0, hi = p.G - 1;  // largest g with tp[g] <= rt
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (tp[mid] <= rt) lo = mid; else hi = mid - 1;
+  }
+  g = lo;
+  const int j = rt - tp[g], nt = tp[g + 1] - tp[g];
+  const int rows_g = off[g + 1] - off[g];
+  const int units = (rows_g + 15) >> 4;
+  const int s16 = j * units / nt, e16 = (j + 1) * units / nt;
+  row0 = off[g] + 16 * s16;
+  n = min(16 * e16, rows_g) - 16 * s16;
+  nmma = 16 * (e16 - s16);
+}
+
+template <class Cfg>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    tc_gemm_pair_ws_kernel(const __grid_constant__ CUtensorMap tmA,
+                           const __grid_constant__ CUtensorMap tmB, const GemmProblem p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + Cfg::STAGES * Cfg::STAGE_BYTES);
+  uint64_t* empty = full + Cfg::STAGES;
+  uint64_t* gfull = empty + Cfg::STAGES;  // peer CTA: its own gather's completion
+  uint64_t* tfull = gfull + Cfg::STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* s_tiles = reinterpret_cast<int*>(smem + Cfg::STAGES * Cfg::STAGE_BYTES + 512);
+  static_assert(3 * Cfg::STAGES * 8 + 5 * 8 + 8 <= 512, "barrier area");
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  load_tile_tables(p, s_tiles);
+  const uint32_t rank = cluster_ctarank();
+  const int cid = (int)cluster_id_x(), ncl = (int)cluster_count_x();
+  const int NT = (p.F + Cfg::FT - 1) / Cfg::FT;
+  const int KB = p.K / Cfg::BK;
+  constexpr int W_OFF = Cfg::NUM_W * Cfg::W_BYTES;  // rows follow the weight tile(s)
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < Cfg::STAGES; ++s) {
+      // leader: its TMA arrive + (gather) its 64 gather threads + the peer's relay
+      mbar_init(&full[s], Cfg::kGather ? 2 + kGatherThreads : 1);
+      mbar_init(&empty[s], 1);
+      mbar_init(&gfull[s], kGatherThreads);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 2 * kEpiWarps);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    if (!Cfg::kGather) prefetch_tensormap(&tmA);
+    prefetch_tensormap(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, Cfg::TMEM_COLS);
+    tmem_relinquish_pair();
+    tc_fence_before();
+  }
+  __syncthreads();
+  cluster_sync();  // both CTAs' barriers exist before any remote arrive
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int num_tiles = s_tiles[p.G] * NT;
+
+  if (warp == 0) {
+    // ---------------- TMA producer (both CTAs) ----------------
+    if (lane == 0) {
+      const uint32_t full_leader = cluster_map(&full[0], 0);
+      int s = 0;
+      uint32_t ph = 0;
+      long armed = 0;
+      for (int t = cid; t < num_tiles; t += ncl) {
+        const int rt = t / NT, ft = t - (t / NT) * NT;
+        int g, row0, n, nmma;
+        locate_ws_tile(p, s_tiles, rt, g, row0, n, nmma);
+        const int hb = nmma >> 1;  // rows per CTA
+        const int wrow = (int)(g * p.w_group_stride) + ft * Cfg::FT + (int)rank * 128;
+        const int nsub = Cfg::kGather ? 0 : (hb + 31) / 32;
+        const uint32_t bytes = 2u * (uint32_t)(W_OFF + nsub * 4096);
+        bool ok = true;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait_cluster(&empty[s], ph ^ 1, abort_flag, p.err)) { ok = false; break; }
+          uint8_t* st = smem + s * Cfg::STAGE_BYTES;
+          if (rank == 0) {
+            mbar_arrive_expect_tx(&full[s], bytes);
+            ++armed;
+          }
+          const uint32_t fb = full_leader + (uint32_t)s * 8u;
+          tma_load_2d_pair(&tmB, fb, st, kb * Cfg::BK, wrow);
+          if (Cfg::kDual)
+            tma_load_2d_pair(&tmB, fb, st + Cfg::W_BYTES, kb * Cfg::BK, wrow + p.dual_offset);
+          for (int sub = 0; sub < nsub; ++sub)
+            tma_load_2d_pair(&tmA, fb, st + W_OFF + sub * 4096, kb * Cfg::BK,
+                             row0 + (int)rank * hb + sub * 32);
+          if (++s == Cfg::STAGES) { s = 0; ph ^= 1; }
+        }
+        if (!ok) break;
+      }
+      if (rank == 0 && *abort_flag) {
+        int ss = s;
+        uint32_t pp = ph;
+        for (long i = 0; i < armed && i < Cfg::STAGES; ++i) {
+          if (ss == 0) { ss = Cfg::STAGES; pp ^= 1; }
+          --ss;
+          mbar_wait_drain(&full[ss], pp);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (rank == 0 && lane == 0) {
+      // ---------------- MMA issuer (leader) ----------------
+      int s = 0;
+      uint32_t ph = 0;
+      int it = 0;
+      for (int t = cid; t < num_tiles; t += ncl, ++it) {
+        const int rt = t / NT;
+        int g, row0, n, nmma;
+        locate_ws_tile(p, s_tiles, rt, g, row0, n, nmma);
+        const uint32_t idesc = idesc_bf16_f32(256, nmma);
+        const int ab = it & 1;
+        const uint32_t aph = (it >> 1) & 1;
+        if (!mbar_wait_cluster(&tempty[ab], aph ^ 1, abort_flag, p.err)) break;
+        tc_fence_after();
+        const uint32_t d0 = tmem_base + ab * Cfg::ACC_COLS;
+        bool ok = true;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait_cluster(&full[s], ph, abort_flag, p.err)) { ok = false; break; }
+          tc_fence_after();
+          const uint8_t* st = smem + s * Cfg::STAGE_BYTES;
+          const uint64_t dw0 = smem_desc_sw128(st);
+          const uint64_t dw1 = smem_desc_sw128(st + Cfg::W_BYTES);
+          const uint64_t db = smem_desc_sw128(st + W_OFF);
+#pragma unroll
+          for (int kk = 0; kk < Cfg::BK / 16; ++kk) {
+            const uint32_t acc = (kb | kk) != 0;
+            const uint64_t adv = (uint64_t)(kk * 32) >> 4;
+            tc_mma_bf16_pair(d0, dw0 + adv, db + adv, idesc, acc);
+            if (Cfg::kDual) tc_mma_bf16_pair(d0 + 128, dw1 + adv, db + adv, idesc, acc);
+          }
+          tc_commit_pair_mc(&empty[s], 0x3);
+          if (++s == Cfg::STAGES) { s = 0; ph ^= 1; }
+        }
+        if (!ok) break;
+        tc_commit_pair_mc(&tfull[ab], 0x3);
+      }
+      tc_commit_pair_mc(drain, 0x1);
+      mbar_wait_drain(drain, 0);
+    } else if (rank == 1 && lane == 0 && Cfg::kGather) {
+      // ---------------- relay of the peer's gather (CTA 1) ----------------
+      const uint32_t full_leader = cluster_map(&full[0], 0);
+      int s = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      for (int t = cid; t < num_tiles && ok; t += ncl) {
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(&gfull[s], ph, abort_flag, p.err)) { ok = false; break; }
+          fence_proxy_async_smem();
+          mbar_arrive_cluster(full_leader + (uint32_t)s * 8u);
+          if (++s == Cfg::STAGES) { s = 0; ph ^= 1; }
+        }
+      }
+    }
+  } else if (warp < 4) {
+    // ---------------- cp.async row gather (both CTAs) ----------------
+    if (Cfg::kGather) {
+      const int gt = threadIdx.x - 64;  // 0..63
+      const int q = gt & 7;             // 16-byte chunk of a 128-byte row
+      const int rsub = gt >> 3;         // rows rsub, rsub + 8, ...
+      const uint32_t swz = (uint32_t)((q ^ rsub) * 16);
+      const bf16* A = static_cast<const bf16*>(p.A);
+      uint64_t* done_bar = rank == 0 ? full : gfull;
+      constexpr int RI = Cfg::B_ROWS / 8;
+      int s = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      for (int t = cid; t < num_tiles && ok; t += ncl) {
+        const int rt = t / NT;
+        int g, row0, n, nmma;
+        locate_ws_tile(p, s_tiles, rt, g, row0, n, nmma);
+        const int hb = nmma >> 1;
+        const int base = (int)rank * hb;
+        const bf16* src[RI];
+#pragma unroll
+        for (int i = 0; i < RI; ++i) {
+          const int rr = base + rsub + 8 * i;
+          src[i] = (rr < n) ? A + (size_t)__ldg(p.gather + row0 + rr) * p.lda + q * 8 : A;
+        }
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait_cluster(&empty[s], ph ^ 1, abort_flag, p.err)) { ok = false; break; }
+          uint8_t* rows_smem = smem + s * Cfg::STAGE_BYTES + W_OFF;
+#pragma unroll
+          for (int i = 0; i < RI; ++i) {
+            const int r = rsub + 8 * i;
+            if (r < hb)
+              cp_async_16(rows_smem + r * 128 + swz, src[i] + kb * Cfg::BK,
+                          base + r < n ? 16u : 0u);
+          }
+          cp_async_mbar_arrive(&done_bar[s]);
+          mbar_arrive(&done_bar[s]);
+          if (++s == Cfg::STAGES) { s = 0; ph ^= 1; }
+        }
+      }
+      cp_async_wait<0>();
+    }
+  } else {
+    // ---------------- epilogue (warps 4..11 of both CTAs) ----------------
+    const int qd = warp & 3;
+    const int eg = (warp - 4) >> 2;
+    const uint32_t tempty_leader = cluster_map(&tempty[0], 0);
+    const EpiParams& e = p.epi;
+    bf16* out = static_cast<bf16*>(e.out);
+    int it = 0;
+    for (int t = cid; t < num_tiles; t += ncl, ++it) {
+      const int rt = t / NT, ft = t - (t / NT) * NT;
+      int g, row0, n, nmma;
+      locate_ws_tile(p, s_tiles, rt, g, row0, n, nmma);
+      const int ab = it & 1;
+      const uint32_t aph = (it >> 1) & 1;
+      if (!mbar_wait_cluster(&tfull[ab], aph, abort_flag, p.err)) break;
+      tc_fence_after();
+      const uint32_t tb = tmem_base + ((uint32_t)(qd * 32) << 16) + ab * Cfg::ACC_COLS;
+      const int f = ft * Cfg::FT + (int)rank * 128 + qd * 32 + lane;
+      const bool fok = f < p.F;
+      float v0[32], v1[32];
+      for (int c0 = 32 * eg; c0 < n; c0 += 64) {
+        tmem_ld_32x32(tb + c0, v0);
+        if (Cfg::kDual) tmem_ld_32x32(tb + 128 + c0, v1);
+        tc_wait_ld();
+        const int cn = min(32, n - c0);
+        float rw = 1.f;
+        if (Cfg::kEpi == EPI_SCALE_ROWS && lane < cn) rw = __ldg(e.row_w + row0 + c0 + lane);
+        bf16* o = out + (size_t)(row0 + c0) * e.ldo + (Cfg::kEpi == EPI_ACT ? e.col0 : 0) + f;
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          float v;
+          if (Cfg::kEpi == EPI_SCALE_ROWS) v = v0[c] * __shfl_sync(0xffffffffu, rw, c);
+          else v = apply_act(e.act, v0[c], Cfg::kDual ? v1[c] : 0.f);
+          if (c < cn && fok) {
+            const bf16 hi = __float2bfloat16_rn(v);
+            o[(size_t)c * e.ldo] = hi;
+            if (Cfg::kEpi == EPI_ACT && e.split_off)
+              o[(size_t)c * e.ldo + e.split_off] = __float2bfloat16_rn(v - __bfloat162float(hi));
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(tempty_leader + (uint32_t)ab * 8u);
+    }
+  }
+
+  __syncthreads();
+  cluster_sync();  // no CTA leaves while its peer may still signal its barriers
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, Cfg::TMEM_COLS);
+  }
+}
+
 }  // namespace lmoe

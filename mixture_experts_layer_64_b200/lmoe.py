@@ -20,8 +20,8 @@ LIB_PATH = os.path.join(HERE, "liblmoe.so")
 OK, ERR_INVALID_ARG, ERR_NOT_READY, ERR_CUDA, ERR_OOM, ERR_TIMEOUT, ERR_UNSUPPORTED, ERR_DEVICE = range(8)
 ACT = {"silu": 0, "swiglu": 1, "relu2": 2}
 DTYPE = {"f32": 0, "bf16": 1}
-SKIP_PROJ, DEBUG_CHECKS, FORCE_SIMT, FORCE_SWAP, FORCE_NOSWAP, FORCE_NOPAIR = (
-    0x1, 0x2, 0x4, 0x8, 0x10, 0x20)
+SKIP_PROJ, DEBUG_CHECKS, FORCE_SIMT, FORCE_SWAP, FORCE_NOSWAP, FORCE_NOPAIR, FORCE_WS_PAIR = (
+    0x1, 0x2, 0x4, 0x8, 0x10, 0x20, 0x40)
 MAX_EXPERTS, MAX_TOPK = 1024, 32
 DEVERR_WAIT_TIMEOUT, DEVERR_RANGE, DEVERR_NONFINITE = 0x1, 0x2, 0x4
 STAGES = {"logits": 0, "idx": 1, "w": 2, "offsets": 3, "perm": 4, "z": 5, "h": 6, "ys": 7, "comb": 8}

@@ -55,6 +55,26 @@ def test_route_only_bit_exact_edges(T, N, k):
     _route_case(T, N, k, seed=T * 7 + N + k)
 
 
+@pytest.mark.parametrize("T,N,k", [(200, 896, 16), (100, 512, 22), (64, 128, 8), (40, 1024, 32)])
+def test_route_only_bit_exact_crowded_logits(T, N, k):
+    """Logits on a coarse grid (six values, zeros of both signs): far more than
+    k keys sit at or above the k-th largest lane maximum, so selection takes
+    the exact radix-select branch, and ties decide most of the order."""
+    g = torch.Generator().manual_seed(T + N + k)
+    lg = (torch.randint(-3, 3, (T, N), generator=g).float() * 0.5)
+    neg = torch.rand((T, N), generator=g) < 0.5
+    lg = torch.where((lg == 0) & neg, torch.tensor(-0.0), lg)
+    L = lmoe.LatentMoELayer(64, 64, N, k, 64, act="silu", dtype="bf16")
+    L.reserve(T)
+    r = L.route_only(lg.cuda())
+    torch.cuda.synchronize()
+    o_idx, o_w, o_off, o_perm = oracle.route(lg.numpy(), k)
+    np.testing.assert_array_equal(r["idx"].cpu().numpy(), o_idx)
+    np.testing.assert_array_equal(r["offsets"].cpu().numpy(), o_off)
+    np.testing.assert_array_equal(r["perm"].cpu().numpy(), o_perm)
+    np.testing.assert_allclose(r["w"].cpu().numpy(), o_w, rtol=2e-6, atol=1e-7)
+
+
 def test_route_only_rejects_oversized_T():
     L = lmoe.LatentMoELayer(64, 64, 16, 4, 64, act="silu", dtype="bf16")
     L.reserve(8)
@@ -92,35 +112,67 @@ def test_small_layer_default_path(name):
     assert res["unique"] >= res["tokens"] * 0.9
 
 
+def paths(res):
+    """(FC1, FC2) expert kernels of the last forward."""
+    return res["expert_path"] & 7, res["expert_path"] >> 3
+
+
 @pytest.mark.parametrize("name", ["swiglu", "relu2-shared", "skip"])
-@pytest.mark.parametrize("flags", [lmoe.FORCE_SWAP, lmoe.FORCE_NOSWAP,
-                                   lmoe.FORCE_NOSWAP | lmoe.FORCE_NOPAIR, lmoe.FORCE_SIMT])
+@pytest.mark.parametrize("flags", [0, lmoe.FORCE_SWAP, lmoe.FORCE_NOSWAP, lmoe.FORCE_WS_PAIR,
+                                   lmoe.FORCE_NOPAIR, lmoe.FORCE_SIMT])
 def test_small_layer_each_expert_kernel(name, flags):
-    """Every expert kernel on the same layers (FC1, FC2): weight-stationary
-    (2, 2), token-tiled with FC2 on CTA pairs (1, 3), token-tiled on single
-    CTAs (1, 1), CUDA cores (0, 0)."""
+    """Every expert kernel on the same layers (FC1, FC2): token-tiled with FC2
+    on CTA pairs (1, 3, the default at these row counts), weight-stationary on
+    single CTAs (2, 2), weight-stationary on CTA pairs (4, 4), token-tiled on
+    single CTAs (1, 1), CUDA cores (0, 0)."""
     res = check_forward(SMALL[name], flags=flags, fixture=True)
-    want = {lmoe.FORCE_SWAP: (2, 2), lmoe.FORCE_NOSWAP: (1, 3),
-            lmoe.FORCE_NOSWAP | lmoe.FORCE_NOPAIR: (1, 1), lmoe.FORCE_SIMT: (0, 0)}[flags]
-    assert (res["expert_path"] & 3, res["expert_path"] >> 2) == want
+    want = {0: (1, 3), lmoe.FORCE_SWAP: (2, 2), lmoe.FORCE_NOSWAP: (1, 3), lmoe.FORCE_WS_PAIR: (4, 4),
+            lmoe.FORCE_NOPAIR: (1, 1), lmoe.FORCE_SIMT: (0, 0)}[flags]
+    assert paths(res) == want
+
+
+@pytest.mark.parametrize("act", ["swiglu", "relu2"])
+def test_weight_stationary_pairs_on_skewed_loads(act):
+    """Router bias that spreads the experts' loads from ~T/2 rows down to none:
+    experts with one tile, several tiles of nearly equal size (including
+    loads just past 128 and 256 rows), single rows and no rows; a feature
+    count that ends inside a CTA's half of the 256-feature tile."""
+    w = W_("ws-skew", T=1100, d=256, l=192, N=16, k=4, m=320, act=act, shared_m=0, seed=23)
+    W = workloads.make_weights(w, device="cuda")
+    b = torch.linspace(3.0, -3.0, w.N, device="cuda")
+    b[-1] = -40.0  # never chosen
+    W["bias"] = b
+    res = check_forward(w, W=W, flags=lmoe.FORCE_WS_PAIR, fixture=True,
+                        tokens=sample_tokens(w.T, 300, seed=2))
+    assert paths(res) == (4, 4)
+    L, _ = gpu_layer(w, lmoe.FORCE_WS_PAIR, W)
+    x = workloads.make_x(w, device="cuda")
+    L.forward(x)
+    torch.cuda.synchronize()
+    off = L.debug_dump("offsets", w.T).cpu().numpy()
+    loads = np.diff(off)
+    assert loads[-1] == 0 and loads.max() > 256 and ((loads > 128) & (loads < 256)).any()
 
 
 def test_pair_kernels_on_dense_prefill_shapes():
     """T >= 1024 puts the dense GEMMs (router, down-projection, shared FC1,
-    up-projection) on CTA pairs as well as the expert FC2; ragged last row
+    up-projection) on CTA pairs as well as the expert GEMMs; ragged last row
     tile."""
     w = W_("pair-dense", T=1100, d=256, l=192, N=16, k=4, m=320, act="swiglu", shared_m=256,
            seed=22)
     res = check_forward(w, fixture=True, tokens=sample_tokens(w.T, 200, seed=1))
-    assert res["expert_path"] >> 2 == 3
+    assert paths(res) == (1, 3)
+    res = check_forward(w, flags=lmoe.FORCE_WS_PAIR, fixture=True,
+                        tokens=sample_tokens(w.T, 200, seed=1))
+    assert paths(res) == (4, 4)
     res = check_forward(w, flags=lmoe.FORCE_NOPAIR, fixture=True,
                         tokens=sample_tokens(w.T, 200, seed=1))
-    assert res["expert_path"] >> 2 == 1
+    assert paths(res) == (1, 1)
 
 
 def test_tcgen05_path_is_taken_for_bf16():
     res = check_forward(SMALL["swiglu"], fixture=True)
-    assert res["expert_path"] & 3 in (1, 2)
+    assert paths(res)[0] in (1, 2, 4)
     res = check_forward(SMALL["odd-K"], fixture=True)
     assert res["expert_path"] == 0
 
@@ -189,5 +241,5 @@ def test_workload_full_size(name):
     print(name, res)
     assert res["unique"] >= 0.8 * res["tokens"]
     if w.dtype == "bf16":
-        assert res["expert_path"] & 3 in (1, 2)
+        assert paths(res)[0] in (1, 2, 4)
     torch.cuda.empty_cache()
