@@ -38,6 +38,8 @@ struct EpiParams {
   int split_off;          // EPI_ACT, bf16: > 0 also writes v - bf16(v) (rounded) at
                           // column col0 + split_off + f, so that hi + lo carries the
                           // value to ~16 significant bits through the next bf16 GEMM
+  long slice;             // split-K partials (EPI_F32_BIAS): elements between the
+                          // fp32 slices of consecutive K ranges
 };
 
 // A (possibly grouped) problem D[r, f] = sum_k A[src(r), k] * B[wrow(g, f), k]
@@ -65,6 +67,8 @@ struct GemmProblem {
   EpiParams epi;
   int tma_store;          // token-tiled kernels: write full 32-row blocks with TMA stores
                           // (the output map is the kernel's third tensor map)
+  int splits;             // dense, single-CTA token-tiled: > 1 splits K into ranges of
+  int kb_per_split;       // kb_per_split 64-wide blocks, each written as an fp32 slice
   int* err;               // device error word
 };
 

@@ -91,6 +91,8 @@ struct lmoe_layer {
   void *z = nullptr, *h = nullptr, *ys = nullptr, *cat = nullptr;
   void *x_stage = nullptr, *out_stage = nullptr;
   float* s32 = nullptr;  // [T, d] fp32 shared-expert output (projection-skip layers)
+  float* part = nullptr;  // split-K partial sums of the dense GEMMs at small T
+  size_t part_bytes = 0;
   // bookkeeping
   int last_T = -1, launches = 0, expert_path = -1;
   std::string detail;
@@ -223,7 +225,7 @@ lmoe_status launch_tc(lmoe_layer* h, const GemmCall& c, cudaStream_t st) {
   GemmProblem p = c.p;
   p.tma_store = (!Cfg::kSwap && tma_store_ok(c) && encode_out_map(&tc, c)) ? 1 : 0;
   const long NT = (c.p.F + Cfg::FT - 1) / Cfg::FT;
-  const long tiles = (long)c.p.max_row_tiles * NT;
+  const long tiles = (long)c.p.max_row_tiles * NT * std::max(1, c.p.splits);
   const int grid = (int)std::max(1L, std::min<long>(h->num_sms, tiles));
   tc_gemm_kernel<Cfg><<<grid, kTcThreads, Cfg::SMEM_BYTES, st>>>(ta, tb, tc, p);
   LMOE_CHECK_LAUNCH(h);
@@ -365,6 +367,58 @@ bool tc_eligible(const lmoe_layer* h, const GemmCall& c) {
   return true;
 }
 
+// ---- split-K for the dense GEMMs at small T ----------------------------------
+//
+// At decode sizes a dense GEMM (router, down-projection, shared FC1,
+// up-projection) has a handful of 128 x 128 output tiles over K = d or l:
+// one CTA per tile would stream K serially while most SMs idle.  The call is
+// then split over K into S ranges, each written as an fp32 slice of partial
+// sums, and splitk_reduce_kernel adds the slices in a fixed order (so results
+// are deterministic) and applies the epilogue.
+
+constexpr size_t kSplitPartBytes = 32u << 20;
+
+// Number of K ranges for a dense single-CTA call (1: no split), and the
+// 64-wide K blocks per range.
+int choose_splits(const lmoe_layer* h, const GemmCall& c, int& kbs) {
+  if (c.pair || c.swap || c.p.offsets || !h->part) return 1;
+  const bool dual = c.p.dual_offset > 0;
+  if (dual && c.p.dual_offset != c.p.F) return 1;  // gate and linear rows must be adjacent
+  const int Fp = dual ? 2 * c.p.F : c.p.F;
+  const int KB = c.p.K / 64;
+  if (Fp % 4 != 0 || KB < 4) return 1;
+  const long tiles = (long)((c.p.M + kRowTile - 1) / kRowTile) * ((Fp + 127) / 128);
+  if (tiles * 2 > h->num_sms) return 1;
+  int S = (int)std::min<long>(std::min<long>(h->num_sms / tiles, KB / 2), 16);
+  while (S > 1 && (size_t)S * c.p.M * Fp * sizeof(float) > h->part_bytes) --S;
+  if (S < 2) return 1;
+  kbs = (KB + S - 1) / S;
+  return (KB + kbs - 1) / kbs;  // every range non-empty
+}
+
+lmoe_status run_split(lmoe_layer* h, const GemmCall& c, int S, int kbs, cudaStream_t st) {
+  const bool dual = c.p.dual_offset > 0;
+  const int Fp = dual ? 2 * c.p.F : c.p.F;
+  GemmCall g = c;
+  g.kind = GK_ROUTER;  // fp32 output, no bias: the partial sums
+  g.p.F = Fp;
+  g.p.dual_offset = 0;
+  std::memset(&g.p.epi, 0, sizeof g.p.epi);
+  g.p.epi.out = h->part;
+  g.p.epi.ldo = Fp;
+  g.p.epi.slice = (long)c.p.M * Fp;
+  g.p.splits = S;
+  g.p.kb_per_split = kbs;
+  g.out_rows = c.p.M;
+  LMOE_TRY((launch_tc<TcCfg<false, false, false, 128, EPI_F32_BIAS>>(h, g, st)));
+  const int kind = c.kind == GK_ROUTER ? EPI_F32_BIAS : c.kind == GK_UP ? EPI_RESID : EPI_ACT;
+  const long n = (long)c.p.M * c.p.F;
+  splitk_reduce_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(
+      h->part, S, g.p.epi.slice, c.p.M, c.p.F, Fp, dual ? c.p.F : 0, kind, c.p.epi);
+  LMOE_CHECK_LAUNCH(h);
+  return LMOE_OK;
+}
+
 lmoe_status run_gemm(lmoe_layer* h, GemmCall c, cudaStream_t st, int* path = nullptr) {
   c.p.err = h->err;
   if (c.pair && c.p.gather != nullptr) {
@@ -394,6 +448,11 @@ lmoe_status run_gemm(lmoe_layer* h, GemmCall c, cudaStream_t st, int* path = nul
       return launch_pair_ws<TcPairWsCfg<false, false, EPI_SCALE_ROWS>>(h, c, st);
   }
   if (path) *path = c.pair ? 3 : (c.swap ? 2 : 1);
+  if (!c.pair && !c.swap && !c.p.offsets && c.kind != GK_FC1 && c.kind != GK_FC2) {
+    int kbs = 0;
+    const int S = choose_splits(h, c, kbs);
+    if (S > 1) return run_split(h, c, S, kbs, st);
+  }
   if (c.pair) {
     switch (c.kind) {
       case GK_DENSE_ACT:
@@ -676,6 +735,8 @@ void free_workspace(lmoe_layer* h) {
   free_ptr(h->x_stage);
   free_ptr(h->out_stage);
   free_ptr(h->s32);
+  free_ptr(h->part);
+  h->part_bytes = 0;
   h->max_T = 0;
 }
 
@@ -851,6 +912,10 @@ lmoe_status lmoe_reserve(lmoe_layer* h, int max_T) {
   ALLOC(h->x_stage, T * h->d * es);
   ALLOC(h->out_stage, T * h->d * es);
   if (skip && h->shared_m > 0) ALLOC(h->s32, T * h->d * sizeof(float));
+  if (h->dtype == LMOE_BF16) {
+    h->part_bytes = kSplitPartBytes;
+    ALLOC(h->part, h->part_bytes);
+  }
 #undef ALLOC
   LMOE_CUDA(h, cudaMemset(h->bitmap, 0, (size_t)h->N * W * sizeof(uint32_t)));
   LMOE_CUDA(h, cudaMemset(h->done, 0, sizeof(unsigned)));

@@ -1,6 +1,6 @@
 // Elementwise kernels: the gate-weighted combine (Eq. (1), the sum over the
-// selected experts, in latent width) and the weight repack into the K-major
-// layout the GEMMs read.
+// selected experts, in latent width), the reduction of split-K partial sums,
+// and the weight repack into the K-major layout the GEMMs read.
 #pragma once
 
 #include "common.cuh"
@@ -65,6 +65,42 @@ __global__ void __launch_bounds__(256) combine_scalar_kernel(const T* __restrict
     if (add32) acc += add32[(size_t)t * ldr + c];
     for (int j = 0; j < k; ++j) acc += to_f32<T>(ys[(size_t)slot_row[(size_t)t * k + j] * l + c]);
     out[(size_t)t * ldo + c] = from_f32<T>(acc);
+  }
+}
+
+// Second half of a split-K dense GEMM: sums the S fp32 slices of partial
+// results part[s][row][c] (c < Fp, slice = M * Fp elements apart) in slice
+// order and applies the contraction's epilogue:
+//   EPI_F32_BIAS  fp32 out[row][f] = sum (+ bias[f])
+//   EPI_ACT       bf16 out[row][col0 + f] = act(sum_f, sum_{f + dual})
+//                 (+ its rounding residue at column col0 + split_off + f)
+//   EPI_RESID     bf16 out[row][f] = resid[row][f] + sum
+// F is the number of output features (Fp = F, or 2F for a gated problem
+// whose gate and linear rows were computed as one).  One thread per output
+// element.
+__global__ void __launch_bounds__(256) splitk_reduce_kernel(const float* __restrict__ part, int S,
+                                                            long slice, int M, int F, int Fp,
+                                                            int dual, int kind, EpiParams e) {
+  const long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= (long)M * F) return;
+  const int row = (int)(i / F), f = (int)(i - (long)row * F);
+  const float* src = part + (size_t)row * Fp + f;
+  float g = 0.f, u = 0.f;
+  for (int s = 0; s < S; ++s) {
+    g += src[(size_t)s * slice];
+    if (dual) u += src[(size_t)s * slice + dual];
+  }
+  if (kind == EPI_F32_BIAS) {
+    static_cast<float*>(e.out)[(size_t)row * e.ldo + f] = g + (e.bias ? e.bias[f] : 0.f);
+  } else if (kind == EPI_ACT) {
+    const float v = apply_act(e.act, g, u);
+    const bf16 hi = __float2bfloat16_rn(v);
+    bf16* o = static_cast<bf16*>(e.out) + (size_t)row * e.ldo + e.col0 + f;
+    o[0] = hi;
+    if (e.split_off) o[e.split_off] = __float2bfloat16_rn(v - __bfloat162float(hi));
+  } else {  // EPI_RESID
+    const float r = __bfloat162float(static_cast<const bf16*>(e.resid)[(size_t)row * e.ldr + f]);
+    static_cast<bf16*>(e.out)[(size_t)row * e.ldo + f] = __float2bfloat16_rn(r + g);
   }
 }
 

@@ -72,11 +72,12 @@ struct TcCfg {
 // One row (token-tiled mode): 32 consecutive features [f, f+32) of row `row`.
 template <int kEpi, bool kGated>
 __device__ __forceinline__ void store_row32(const GemmProblem& p, int row, int f,
-                                            const float (&v0)[32], const float (&v1)[32]) {
+                                            const float (&v0)[32], const float (&v1)[32],
+                                            size_t slice_off = 0) {
   const EpiParams& e = p.epi;
   const bool full = f + 32 <= p.F;
   if (kEpi == EPI_F32_BIAS) {
-    float* o = static_cast<float*>(e.out) + (size_t)row * e.ldo + f;
+    float* o = static_cast<float*>(e.out) + slice_off + (size_t)row * e.ldo + f;
     if (full) {
 #pragma unroll
       for (int i = 0; i < 32; i += 4) {
@@ -315,7 +316,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const int num_tiles = total_row_tiles_s(p, s_tiles) * NT;
+  // Split-K (dense problems): tile t covers K blocks [kb0, kb1) of split
+  // t / tiles_per_split and writes an fp32 slice of partial sums.
+  const int S = p.splits > 1 ? p.splits : 1;
+  const int KBS = S > 1 ? p.kb_per_split : KB;
+  const int tiles_per_split = total_row_tiles_s(p, s_tiles) * NT;
+  const int num_tiles = tiles_per_split * S;
 
   if (warp == 0) {
     // ---------------- TMA producer ----------------
@@ -324,7 +330,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       uint32_t ph = 0;
       long armed = 0;
       for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
-        const int rt = t / NT, ft = t - (t / NT) * NT;
+        const int ks = t / tiles_per_split, tl = t - ks * tiles_per_split;
+        const int rt = tl / NT, ft = tl - (tl / NT) * NT;
+        const int kb0 = ks * KBS, kb1 = min(KB, kb0 + KBS);
         int g, row0, rows;
         locate_row_tile_s(p, s_tiles, rt, g, row0, rows);
         const int wrow = (int)(g * p.w_group_stride) + ft * Cfg::FT;
@@ -332,7 +340,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         uint32_t bytes = Cfg::NUM_W * Cfg::W_BYTES;
         if (!Cfg::kGather) bytes += Cfg::kSwap ? nsub * 4096 : Cfg::ACT_BYTES;
         bool ok = true;
-        for (int kb = 0; kb < KB; ++kb) {
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, p.err)) { ok = false; break; }
           uint8_t* st = smem + s * Cfg::STAGE_BYTES;
           mbar_arrive_expect_tx(&full[s], bytes);
@@ -371,7 +379,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       uint32_t ph = 0;
       int it = 0;
       for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++it) {
-        const int rt = t / NT;
+        const int ks = t / tiles_per_split, tl = t - ks * tiles_per_split;
+        const int rt = tl / NT;
+        const int kb0 = ks * KBS, kb1 = min(KB, kb0 + KBS);
         int g, row0, rows;
         locate_row_tile_s(p, s_tiles, rt, g, row0, rows);
         const int ab = it & 1;
@@ -388,7 +398,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (Cfg::kSwap) n = max(16, (rows + 15) & ~15);
         const uint32_t idesc = idesc_bf16_f32(128, n);
         bool ok = true;
-        for (int kb = 0; kb < KB; ++kb) {
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&full[s], ph, abort_flag, p.err)) { ok = false; break; }
           tc_fence_after();
           const uint8_t* st = smem + s * Cfg::STAGE_BYTES;
@@ -397,7 +407,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           const uint64_t dw1 = smem_desc_sw128(st + Cfg::ACT_BYTES + Cfg::W_BYTES);
 #pragma unroll
           for (int kk = 0; kk < Cfg::BK / 16; ++kk) {
-            const uint32_t acc = (kb | kk) != 0;
+            const uint32_t acc = (kb != kb0 || kk != 0) ? 1u : 0u;
             const uint64_t adv = (uint64_t)(kk * 32) >> 4;  // 16 bf16 = 32 bytes along K
             if (Cfg::kSwap) {
               tc_mma_bf16(d0, dw0 + adv, da + adv, idesc, acc);
@@ -433,7 +443,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       uint32_t ph = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-        const int rt = t / NT;
+        const int ks = t / tiles_per_split, tl = t - ks * tiles_per_split;
+        const int rt = tl / NT;
+        const int kb0 = ks * KBS, kb1 = min(KB, kb0 + KBS);
         int g, row0, rows;
         locate_row_tile_s(p, s_tiles, rt, g, row0, rows);
         const int nload = Cfg::kSwap ? max(16, (rows + 15) & ~15) : 128;
@@ -443,7 +455,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           const int r = rsub + 8 * i;
           src[i] = (r < rows) ? A + (size_t)__ldg(p.gather + row0 + r) * p.lda + q * 8 : A;
         }
-        for (int kb = 0; kb < KB; ++kb) {
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, p.err)) { ok = false; break; }
           uint8_t* act = smem + s * Cfg::STAGE_BYTES;
 #pragma unroll
@@ -465,7 +477,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int eg = (warp - 4) >> 2;   // warpgroup: even / odd 32-column chunks
     int it = 0;
     for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++it) {
-      const int rt = t / NT, ft = t - (t / NT) * NT;
+      const int ks = t / tiles_per_split, tl = t - ks * tiles_per_split;
+      const int rt = tl / NT, ft = tl - (tl / NT) * NT;
+      const size_t slice_off = (size_t)ks * (size_t)p.epi.slice;
       int g, row0, rows;
       locate_row_tile_s(p, s_tiles, rt, g, row0, rows);
       const int ab = it & 1;
@@ -488,7 +502,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               epi_tma_chunk32<Cfg::kEpi, Cfg::kDual>(p, &tmC, stg, lane, row0 + qd * 32, f0 + c0,
                                                      v0, v1);
             else if (r < rows)
-              store_row32<Cfg::kEpi, Cfg::kDual>(p, row0 + r, f0 + c0, v0, v1);
+              store_row32<Cfg::kEpi, Cfg::kDual>(p, row0 + r, f0 + c0, v0, v1, slice_off);
           }
         }
       } else {

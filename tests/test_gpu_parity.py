@@ -170,6 +170,24 @@ def test_pair_kernels_on_dense_prefill_shapes():
     assert paths(res) == (1, 1)
 
 
+@pytest.mark.parametrize("skip", [False, True])
+def test_split_k_dense_gemms_at_decode_size(skip):
+    """Few tokens and long K: the router, down-projection, gated shared FC1
+    (with its hi/lo split) and up-projection run as split-K GEMMs whose fp32
+    partial slices are summed in a fixed order; the projection-skip layer
+    also sends its fp32 shared-expert output through the split."""
+    w = W_("split", T=40, d=1024, l=1024 if skip else 512, N=16, k=4, m=128, act="swiglu",
+           shared_m=256, skip_proj=skip, bias="normal0.5", seed=31)
+    res = check_forward(w, fixture=True)
+    assert res["unique"] >= 0.9 * res["tokens"]
+    L, W = gpu_layer(w)
+    x = workloads.make_x(w, device="cuda")
+    a = L.forward(x)
+    b = L.forward(x)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+
+
 def test_tcgen05_path_is_taken_for_bf16():
     res = check_forward(SMALL["swiglu"], fixture=True)
     assert paths(res)[0] in (1, 2, 4)
