@@ -192,8 +192,8 @@ bool encode_out_map(CUtensorMap* map, const GemmCall& c) {
 // Whether a token-tiled call can write its output with TMA stores.
 bool tma_store_ok(const GemmCall& c) {
   const EpiParams& e = c.p.epi;
-  if (c.swap || e.split_off || c.kind == GK_ROUTER) return false;  // fp32 logits: plain stores
-  const size_t es = 2;
+  if (c.swap || e.split_off) return false;
+  const size_t es = c.kind == GK_ROUTER ? 4 : 2;
   const char* base = static_cast<const char*>(e.out) +
                      (c.kind == GK_DENSE_ACT || c.kind == GK_FC1 ? (size_t)e.col0 * es : 0);
   return aligned16(base) && ((size_t)e.ldo * es) % 16 == 0 && (c.p.F * es) % 16 == 0;
@@ -388,10 +388,10 @@ int choose_splits(const lmoe_layer* h, const GemmCall& c, int& kbs) {
   const int KB = c.p.K / 64;
   if (Fp % 4 != 0 || KB < 4) return 1;
   const long tiles = (long)((c.p.M + kRowTile - 1) / kRowTile) * ((Fp + 127) / 128);
-  if (tiles * 2 > h->num_sms) return 1;
+  if (tiles * 4 > h->num_sms) return 1;  // fewer than 4 ranges would not pay for the reduction
   int S = (int)std::min<long>(std::min<long>(h->num_sms / tiles, KB / 2), 16);
   while (S > 1 && (size_t)S * c.p.M * Fp * sizeof(float) > h->part_bytes) --S;
-  if (S < 2) return 1;
+  if (S < 4) return 1;
   kbs = (KB + S - 1) / S;
   return (KB + kbs - 1) / kbs;  // every range non-empty
 }
@@ -409,7 +409,7 @@ lmoe_status run_split(lmoe_layer* h, const GemmCall& c, int S, int kbs, cudaStre
   g.p.epi.slice = (long)c.p.M * Fp;
   g.p.splits = S;
   g.p.kb_per_split = kbs;
-  g.out_rows = c.p.M;
+  g.out_rows = (long)S * c.p.M;  // the slices stacked: rows of the output map
   LMOE_TRY((launch_tc<TcCfg<false, false, false, 128, EPI_F32_BIAS>>(h, g, st)));
   const int kind = c.kind == GK_ROUTER ? EPI_F32_BIAS : c.kind == GK_UP ? EPI_RESID : EPI_ACT;
   const long n = (long)c.p.M * c.p.F;

@@ -51,17 +51,20 @@ struct TcCfg {
   static constexpr int ACT_BYTES = ACT_ROWS * BK * 2;
   static constexpr int W_BYTES = W_ROWS * BK * 2;
   static constexpr int STAGE_BYTES = ACT_BYTES + NUM_W * W_BYTES;
-  static constexpr int STAGES_RAW = kTcSmemBudget / STAGE_BYTES;
+  // epilogue staging: one 32 x 32 box per epilogue warp (bf16 or fp32)
+  static constexpr int STG_WARP = kEpi == EPI_F32_BIAS ? 4096 : 2048;
+  static constexpr int STG_BYTES = kSwap ? 0 : kEpiWarps * STG_WARP;
+  static constexpr int STAGES_RAW = (kTcSmemBudget + kEpiWarps * 2048 - STG_BYTES) / STAGE_BYTES;
   static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
   static constexpr int ACC_N = kSwap ? 128 : W_ROWS;  // fp32 columns of one accumulator
   static constexpr int ACC_COLS = ACC_N * NUM_W;      // one TMEM buffer
   static constexpr int TMEM_COLS = 2 * ACC_COLS;      // double buffered
   static constexpr int FT = W_ROWS;                   // features per tile
   static constexpr int TABLE_BYTES = 2 * (LMOE_MAX_EXPERTS + 1) * 4;  // tile_prefix, offsets
-  static constexpr int STG_BYTES = kSwap ? 0 : kEpiWarps * 2048;  // epilogue staging (bf16 boxes)
   static constexpr int SMEM_BYTES = 1024 /*align slack*/ + STAGES * STAGE_BYTES + STG_BYTES + 512 +
                                     TABLE_BYTES;
   static_assert(TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM allocation must be a power of two");
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
   static_assert(STAGES >= 3, "pipeline too shallow");
   static_assert(!kSwap || kEpi == EPI_ACT || kEpi == EPI_SCALE_ROWS, "swap epilogues");
   static_assert(kWN_ == 128 || kWN_ == 256, "weight tile");
@@ -219,11 +222,41 @@ __device__ __forceinline__ void epi_tma_chunk32_impl(const GemmProblem& p, const
   }
 }
 
+// fp32 output (router logits, split-K partial sums): 32 rows x 32 floats,
+// 128-byte rows staged with the 128-byte swizzle (16-byte chunk c of row r at
+// r * 128 + ((c ^ (r & 7)) << 4)).
+__device__ __forceinline__ void epi_tma_chunk32_f32(const GemmProblem& p, const CUtensorMap* tmC,
+                                                    uint8_t* stg, int lane, int row_base, int f,
+                                                    const float (&v0)[32]) {
+  const float* b = p.epi.bias;
+  if (lane == 0) bulk_wait_read0();  // the previous box has left the buffer
+  __syncwarp();
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    float4 q;
+    float* qf = reinterpret_cast<float*>(&q);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int i = 4 * c + j;
+      qf[j] = v0[i] + ((b && f + i < p.F) ? __ldg(b + f + i) : 0.f);
+    }
+    *reinterpret_cast<float4*>(stg + lane * 128 + ((c ^ (lane & 7)) << 4)) = q;
+  }
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_2d(tmC, stg, f, row_base);
+    bulk_commit();
+  }
+}
+
 template <int kEpi, bool kGated>
 __device__ __forceinline__ void epi_tma_chunk32(const GemmProblem& p, const CUtensorMap* tmC,
                                                 uint8_t* stg, int lane, int row_base, int f,
                                                 const float (&v0)[32], const float (&v1)[32]) {
-  if constexpr (kEpi != EPI_F32_BIAS)
+  if constexpr (kEpi == EPI_F32_BIAS)
+    epi_tma_chunk32_f32(p, tmC, stg, lane, row_base, f, v0);
+  else
     epi_tma_chunk32_impl<kEpi, kGated>(p, tmC, stg, lane, row_base, f, v0, v1);
 }
 
@@ -492,15 +525,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (!Cfg::kSwap) {
         const int r = qd * 32 + lane;
         const bool tma = p.tma_store && rows - qd * 32 >= 32;
-        uint8_t* stg = stg_base + (warp - 4) * 2048;
+        uint8_t* stg = stg_base + (warp - 4) * Cfg::STG_WARP;
+        const int slice_rows = ks * p.M;  // split-K: the slice's rows in the output map
         for (int c0 = 32 * eg; c0 < Cfg::ACC_N; c0 += 64) {
           tmem_ld_32x32(tb + c0, v0);
           if (Cfg::kDual) tmem_ld_32x32(tb + Cfg::ACC_N + c0, v1);
           tc_wait_ld();
           if (f0 + c0 < p.F) {
             if (tma)
-              epi_tma_chunk32<Cfg::kEpi, Cfg::kDual>(p, &tmC, stg, lane, row0 + qd * 32, f0 + c0,
-                                                     v0, v1);
+              epi_tma_chunk32<Cfg::kEpi, Cfg::kDual>(p, &tmC, stg, lane, slice_rows + row0 + qd * 32,
+                                                     f0 + c0, v0, v1);
             else if (r < rows)
               store_row32<Cfg::kEpi, Cfg::kDual>(p, row0 + r, f0 + c0, v0, v1, slice_off);
           }
@@ -562,11 +596,12 @@ struct TcPairCfg {
   static constexpr int A_BYTES = 128 * BK * 2;   // this CTA's 128 rows
   static constexpr int B_BYTES = 128 * BK * 2;   // this CTA's half of the 256 weight rows
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int STAGES = 6;
+  static constexpr int STG_WARP = kEpi == EPI_F32_BIAS ? 4096 : 2048;  // one 32 x 32 box
+  static constexpr int STG_BYTES = kEpiWarps * STG_WARP;               // epilogue staging
+  static constexpr int STAGES = kEpi == EPI_F32_BIAS ? 5 : 6;
   static constexpr int ACC_N = 256;              // columns of one accumulator buffer
   static constexpr int TMEM_COLS = 512;
   static constexpr int FT = kDual ? 128 : 256;   // output features per tile
-  static constexpr int STG_BYTES = kEpiWarps * 2048;  // epilogue staging (bf16 boxes)
   static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + STG_BYTES + 512 +
                                     2 * (LMOE_MAX_EXPERTS + 1) * 4;
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
@@ -717,7 +752,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const int wrow = (int)rank * 128 + qd * 32;  // this warp's first row in the 256-row tile
       const int r = wrow + lane;
       const bool tma = p.tma_store && rows - wrow >= 32;
-      uint8_t* stg = stg_base + (warp - 4) * 2048;
+      uint8_t* stg = stg_base + (warp - 4) * Cfg::STG_WARP;
       float v0[32], v1[32];
       constexpr int NCOL = Cfg::kDual ? 128 : 256;
       for (int c0 = 32 * eg; c0 < NCOL; c0 += 64) {
