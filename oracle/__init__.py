@@ -34,7 +34,11 @@ class _Layer(ctypes.Structure):
                 ("Wg", ctypes.c_void_p), ("bias", ctypes.c_void_p),
                 ("Wdown", ctypes.c_void_p), ("Wup", ctypes.c_void_p),
                 ("W1", ctypes.c_void_p), ("W2", ctypes.c_void_p),
-                ("Ws1", ctypes.c_void_p), ("Ws2", ctypes.c_void_p)]
+                ("Ws1", ctypes.c_void_p), ("Ws2", ctypes.c_void_p),
+                ("route_mode", ctypes.c_int)]
+
+# routing variants (bits of route_mode)
+ROUTE_FULL_SOFTMAX, ROUTE_BIAS_SELECT = 1, 2
 
 
 _lib = None
@@ -50,6 +54,8 @@ def lib():
         I = ctypes.c_int
         L.oracle_router_logits.argtypes = [P, P, P, I, P, I]
         L.oracle_route.argtypes = [P, I, I, I, P, P, P, P, I]
+        L.oracle_route_ex.argtypes = [P, P, I, I, I, I, P, P, P, P, I]
+        L.oracle_route_ex.restype = I
         L.oracle_forward.argtypes = [P, P, P, I, P, P, P, P, P, I]
         L.oracle_layer.argtypes = [P, P, P, I, P, P, P, P, I]
         for f in (L.oracle_router_logits, L.oracle_route, L.oracle_forward,
@@ -97,7 +103,7 @@ class OracleLayer:
 
     def __init__(self, *, d, l, N, k, m, act, shared_m=0, dtype="bf16",
                  skip_proj=False, Wg, bias=None, Wdown=None, Wup=None,
-                 W1, W2, Ws1=None, Ws2=None):
+                 W1, W2, Ws1=None, Ws2=None, route_mode=0):
         self.d, self.l, self.N, self.k, self.m = d, l, N, k, m
         self.act, self.shared_m, self.dtype, self.skip_proj = act, shared_m, dtype, skip_proj
         keep = []
@@ -126,7 +132,7 @@ class OracleLayer:
                              int(bool(skip_proj)), _ptr(self._Wg), _ptr(self._bias),
                              _ptr(self._Wdown), _ptr(self._Wup),
                              ctypes.cast(p1, ctypes.c_void_p), ctypes.cast(p2, ctypes.c_void_p),
-                             _ptr(self._Ws1), _ptr(self._Ws2))
+                             _ptr(self._Ws1), _ptr(self._Ws2), int(route_mode))
 
     @staticmethod
     def _expert(W, e, arr):
@@ -180,8 +186,14 @@ class OracleLayer:
         return {"out": out, "logits32": lg, "idx": idx, "w": w}
 
 
-def route(logits32, k: int, nthreads: Optional[int] = None):
-    """Top-k + renormalised softmax + expert grouping on fp32 logits.
+def route(logits32, k: int, nthreads: Optional[int] = None, sel_bias=None,
+          full_softmax: bool = False):
+    """Top-k + gate weights + expert grouping on fp32 logits.
+
+    Default: selection on the logits, softmax renormalised over the k chosen.
+    ``sel_bias`` [N] fp32: select on the fp32 sum logits + sel_bias, gates
+    from the logits.  ``full_softmax``: gates are the softmax over all N
+    logits at the chosen experts.
     Returns (idx [T,k] int32, w [T,k] float64, offsets [N+1], perm [T*k])."""
     lg = np.ascontiguousarray(_host_array(logits32, "f32"), dtype=np.float32)
     T, N = lg.shape
@@ -189,8 +201,16 @@ def route(logits32, k: int, nthreads: Optional[int] = None):
     w = np.empty((T, k), dtype=np.float64)
     offsets = np.empty(N + 1, dtype=np.int32)
     perm = np.empty(T * k, dtype=np.int32)
-    rc = lib().oracle_route(_ptr(lg), T, N, k, _ptr(idx), _ptr(w), _ptr(offsets),
-                            _ptr(perm), nthreads or default_threads())
+    sb = None
+    if sel_bias is not None:
+        sb = np.ascontiguousarray(_host_array(sel_bias, "f32"), dtype=np.float32)
+    if sb is None and not full_softmax:
+        rc = lib().oracle_route(_ptr(lg), T, N, k, _ptr(idx), _ptr(w), _ptr(offsets),
+                                _ptr(perm), nthreads or default_threads())
+    else:
+        rc = lib().oracle_route_ex(_ptr(lg), _ptr(sb), T, N, k, int(bool(full_softmax)),
+                                   _ptr(idx), _ptr(w), _ptr(offsets), _ptr(perm),
+                                   nthreads or default_threads())
     if rc:
         raise OracleError(f"oracle_route failed ({rc})")
     return idx, w, offsets, perm

@@ -12,6 +12,8 @@
 //   logits   = x . Wg + b                         router on the full-width x
 //   S        = the k experts first under the order (logit desc, index asc)
 //   w_j      = exp(l_j - l_0) / sum_{j'} exp(l_j' - l_0)   over the k chosen
+//              (variants: the softmax over all N logits taken at the chosen
+//              experts; a bias that only steers the selection)
 //   z        = x . Wdown                          down-projection d -> l
 //   y_j      = act(z . W1[e_j]) . W2[e_j]         expert e_j in latent width
 //   comb     = sum_j w_j y_j                      gate-weighted sum, slot order
@@ -48,6 +50,14 @@ namespace {
 enum { OR_F32 = 0, OR_BF16 = 1 };
 enum { OR_ACT_SILU = 0, OR_ACT_SWIGLU = 1, OR_ACT_RELU2 = 2 };
 enum { OR_OK = 0, OR_ERR_ARG = 1, OR_ERR_NAN = 2, OR_ERR_MISSING = 3 };
+// Routing variants (paper Section 3 and Section 4):
+//   OR_ROUTE_FULL_SOFTMAX  gate w_j = p'_{e_j}, the softmax over all N logits
+//                          taken at the selected experts (Eq. (1) literally;
+//                          the k gates sum to less than 1)
+//   OR_ROUTE_BIAS_SELECT   the router bias only steers the selection (the
+//                          auxiliary-loss-free balancing of Section 4): experts
+//                          are chosen on l + b, the gates use l
+enum { OR_ROUTE_FULL_SOFTMAX = 1, OR_ROUTE_BIAS_SELECT = 2 };
 
 inline double widen(const void* p, int dtype, size_t i) {
   if (dtype == OR_F32) return (double)static_cast<const float*>(p)[i];
@@ -122,6 +132,7 @@ struct OracleLayer {
   const void* const* W2;   // N pointers, each [m, l]
   const void* Ws1;         // [d, ms_in] or NULL when shared_m == 0
   const void* Ws2;         // [shared_m, d]
+  int route_mode;          // OR_ROUTE_* bits (0: the default routing)
 };
 
 static int m_in_of(int act, int m) { return act == OR_ACT_SWIGLU ? 2 * m : m; }
@@ -153,47 +164,61 @@ int oracle_router_logits(const OracleLayer* L, const void* x, const int* tokens,
       const double xi = widen(x, L->dtype, (size_t)t * d + i);
       for (int e = 0; e < N; ++e) lg[e] += xi * widen(L->Wg, L->dtype, (size_t)i * N + e);
     }
-    if (L->bias)
+    if (L->bias && !(L->route_mode & OR_ROUTE_BIAS_SELECT))
       for (int e = 0; e < N; ++e) lg[e] += (double)L->bias[e];
   });
   return OR_OK;
 }
 
-// Top-k selection and renormalised gate weights on fp32 logits, followed by
-// the grouping of (token, slot) pairs by expert (paper Section 3: the top-K
-// index set and the dispatch after the down-projection).
-//   idx[t][j]   the j-th expert of token t under (logit desc, index asc);
+// Top-k selection and gate weights on fp32 logits, followed by the grouping
+// of (token, slot) pairs by expert (paper Section 3: the top-K index set and
+// the dispatch after the down-projection).
+//   key[t][e]   the selection key: the logit, or with sel_bias the fp32 sum
+//               l + b[e] (rounded once, as the CUDA library decides in fp32)
+//   idx[t][j]   the j-th expert of token t under (key desc, index asc);
 //               +0.0 and -0.0 compare equal.
-//   w[t][j]     exp(l_j - l_0) / sum_j' exp(l_j' - l_0) in float64.
+//   w[t][j]     in float64 from the fp32 logits l (never from the keys):
+//               renormalised  exp(l_j - M) / sum_{j' chosen} exp(l_j' - M),
+//               full softmax  exp(l_j - M) / sum_{e < N} exp(l_e - M),
+//               with M the largest logit of the sum (a shift that cancels).
 //   offsets[e]  number of pairs routed to experts < e (offsets[N] = T*k).
 //   perm[r]     the pair t*k+j at expert-sorted row r; rows of one expert in
 //               ascending token order.
 // Any of w/offsets/perm may be NULL.  Returns OR_ERR_NAN on a NaN logit.
-int oracle_route(const float* logits32, int T, int N, int k, int* idx, double* w,
-                 int* offsets, int* perm, int nthreads) {
+int oracle_route_ex(const float* logits32, const float* sel_bias, int T, int N, int k,
+                    int full_softmax, int* idx, double* w, int* offsets, int* perm,
+                    int nthreads) {
   if (T < 0 || N <= 0 || k <= 0 || k > N || (T > 0 && (!logits32 || !idx)))
     return OR_ERR_ARG;
   std::atomic<int> bad{0};
   parallel_for(T, nthreads, [&](long t) {
     const float* lg = logits32 + (size_t)t * N;
+    std::vector<float> key(lg, lg + N);
+    if (sel_bias)
+      for (int e = 0; e < N; ++e) key[e] = lg[e] + sel_bias[e];  // one fp32 rounding
     std::vector<int> order(N);
     for (int e = 0; e < N; ++e) {
-      if (std::isnan(lg[e])) bad = 1;
+      if (std::isnan(key[e])) bad = 1;
       order[e] = e;
     }
     if (bad) return;
     std::partial_sort(order.begin(), order.begin() + k, order.end(),
                       [&](int a, int b) {
-                        if (lg[a] != lg[b]) return lg[a] > lg[b];
+                        if (key[a] != key[b]) return key[a] > key[b];
                         return a < b;
                       });
     for (int j = 0; j < k; ++j) idx[(size_t)t * k + j] = order[j];
     if (w) {
-      const double l0 = (double)lg[order[0]];
-      double den = 0.0;
-      for (int j = 0; j < k; ++j) den += std::exp((double)lg[order[j]] - l0);
+      double M = -INFINITY, den = 0.0;
+      if (full_softmax) {
+        for (int e = 0; e < N; ++e) M = std::max(M, (double)lg[e]);
+        for (int e = 0; e < N; ++e) den += std::exp((double)lg[e] - M);
+      } else {
+        for (int j = 0; j < k; ++j) M = std::max(M, (double)lg[order[j]]);
+        for (int j = 0; j < k; ++j) den += std::exp((double)lg[order[j]] - M);
+      }
       for (int j = 0; j < k; ++j)
-        w[(size_t)t * k + j] = std::exp((double)lg[order[j]] - l0) / den;
+        w[(size_t)t * k + j] = std::exp((double)lg[order[j]] - M) / den;
     }
   });
   if (bad) return OR_ERR_NAN;
@@ -212,6 +237,12 @@ int oracle_route(const float* logits32, int T, int N, int k, int* idx, double* w
     if (offsets) offsets[N] = (int)pos;
   }
   return OR_OK;
+}
+
+// The default routing: selection on the logits, renormalised gates.
+int oracle_route(const float* logits32, int T, int N, int k, int* idx, double* w,
+                 int* offsets, int* perm, int nthreads) {
+  return oracle_route_ex(logits32, nullptr, T, N, k, 0, idx, w, offsets, perm, nthreads);
 }
 
 // Steps after routing, for S tokens (rows tokens[s] of x, or row s), given
@@ -309,7 +340,8 @@ int oracle_forward(const OracleLayer* L, const void* x, const int* tokens, int S
 }
 
 // The whole layer for S tokens from the inputs alone: fp64 logits, rounded to
-// fp32 for the selection, then oracle_route and oracle_forward.  Optional
+// fp32 for the selection, then the routing of the layer's route_mode and
+// oracle_forward.  Optional
 // outputs: logits32 [S,N], idx [S,k], w [S,k].
 int oracle_layer(const OracleLayer* L, const void* x, const int* tokens, int S,
                  double* out, float* logits32, int* idx, double* w, int nthreads) {
@@ -323,7 +355,9 @@ int oracle_layer(const OracleLayer* L, const void* x, const int* tokens, int S,
   for (size_t i = 0; i < lg.size(); ++i) lg32[i] = (float)lg[i];
   std::vector<int> id((size_t)S * k);
   std::vector<double> ww((size_t)S * k);
-  rc = oracle_route(lg32.data(), S, N, k, id.data(), ww.data(), nullptr, nullptr, nthreads);
+  const float* sel_bias = (L->route_mode & OR_ROUTE_BIAS_SELECT) ? L->bias : nullptr;
+  rc = oracle_route_ex(lg32.data(), sel_bias, S, N, k, L->route_mode & OR_ROUTE_FULL_SOFTMAX,
+                       id.data(), ww.data(), nullptr, nullptr, nthreads);
   if (rc) return rc;
   if (logits32) std::memcpy(logits32, lg32.data(), lg32.size() * sizeof(float));
   if (idx) std::memcpy(idx, id.data(), id.size() * sizeof(int));

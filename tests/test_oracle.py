@@ -150,6 +150,76 @@ def test_route_invariants_and_special_cases():
         oracle.route(np.array([[0.0, np.nan]], dtype=np.float32), 1)
 
 
+@pytest.mark.parametrize("T,N,k,seed", [(9, 16, 4, 21), (33, 128, 8, 22), (17, 896, 16, 23),
+                                        (5, 12, 12, 24)])
+def test_route_full_softmax_is_softmax_over_all_experts(T, N, k, seed):
+    """Eq. (1) read literally: the gate of a chosen expert is its entry of
+    the softmax over all N logits (scipy), so the k gates sum to below one
+    unless k = N, where the variant equals the renormalised default."""
+    lg = workloads.make_logits(T, N, seed, ties=True).numpy()
+    idx, w, offsets, perm = oracle.route(lg, k, full_softmax=True)
+    idx0, w0, off0, perm0 = oracle.route(lg, k)
+    np.testing.assert_array_equal(idx, idx0)          # the selection is unchanged
+    np.testing.assert_array_equal(perm, perm0)
+    np.testing.assert_array_equal(offsets, off0)
+    p = sp_softmax(lg.astype(f64), axis=1)
+    np.testing.assert_allclose(w, np.take_along_axis(p, idx.astype(np.int64), axis=1),
+                               rtol=1e-13, atol=1e-300)
+    if k < N:
+        assert np.all(w.sum(1) < 1.0)
+    else:
+        np.testing.assert_allclose(w, w0, rtol=1e-14)
+
+
+@pytest.mark.parametrize("full", [False, True])
+def test_route_bias_selects_only(full):
+    """Auxiliary-loss-free balancing (Section 4): the bias moves the choice,
+    computed on the fp32 sum logit + bias (brute-force sort of numpy float32
+    sums), while the gates come from the logits alone (scipy softmax)."""
+    T, N, k = 40, 64, 6
+    lg = workloads.make_logits(T, N, 31, ties=True).numpy()
+    b = (np.random.default_rng(5).normal(size=N) * 2.0).astype(np.float32)
+    idx, w, offsets, perm = oracle.route(lg, k, sel_bias=b, full_softmax=full)
+    key = lg + b[None, :]                              # float32 + float32 -> float32
+    assert key.dtype == np.float32
+    for t in range(T):
+        order = sorted(range(N), key=lambda e: (-float(key[t, e]), e))[:k]
+        assert list(idx[t]) == order
+        if full:
+            ref = sp_softmax(lg[t].astype(f64))[order]
+        else:
+            ref = sp_softmax(lg[t, order].astype(f64))
+        np.testing.assert_allclose(w[t], ref, rtol=1e-13, atol=1e-300)
+    # the bias changed the selection of some tokens (it is large on purpose)
+    assert not np.array_equal(idx, oracle.route(lg, k)[0])
+    np.testing.assert_array_equal(perm, np.argsort(idx.ravel(), kind="stable"))
+
+
+def test_layer_route_modes():
+    """The layer-level route mode: with the bias selecting only, the router
+    logits leave the bias out, and the whole layer equals the forward step
+    fed by the variant routing."""
+    L0, W = make_layer(64, 32, 12, 3, 24, "relu2", bias=True, seed=40)
+    x = rnd((10, 64), 1.0, 41)
+    for mode in (oracle.ROUTE_BIAS_SELECT, oracle.ROUTE_FULL_SOFTMAX,
+                 oracle.ROUTE_BIAS_SELECT | oracle.ROUTE_FULL_SOFTMAX):
+        L = oracle.OracleLayer(d=64, l=32, N=12, k=3, m=24, act="relu2", route_mode=mode, **W)
+        lg = L.router_logits(x)
+        plain = as64(x) @ as64(W["Wg"])
+        if mode & oracle.ROUTE_BIAS_SELECT:
+            np.testing.assert_allclose(lg, plain, rtol=1e-12, atol=1e-12)
+        else:
+            np.testing.assert_allclose(lg, plain + W["bias"].double().numpy(), rtol=1e-12,
+                                       atol=1e-12)
+        sb = W["bias"] if mode & oracle.ROUTE_BIAS_SELECT else None
+        idx, w, _, _ = oracle.route(lg.astype(np.float32), 3, sel_bias=sb,
+                                    full_softmax=bool(mode & oracle.ROUTE_FULL_SOFTMAX))
+        res = L.layer(x)
+        np.testing.assert_array_equal(res["idx"], idx)
+        np.testing.assert_allclose(res["w"], w, rtol=1e-15)
+        np.testing.assert_allclose(res["out"], L.forward(x, idx, w), rtol=1e-13, atol=1e-13)
+
+
 # ---------------------------------------------------------------------------
 # router logits: a library matmul
 # ---------------------------------------------------------------------------
