@@ -80,6 +80,19 @@ typedef enum { LMOE_F32 = 0, LMOE_BF16 = 1 } lmoe_dtype;
                                     to 128/256, but its 2-SM MMAs with N < 256
                                     run below full rate, which makes it slower
                                     at a few hundred rows per expert.           */
+#define LMOE_ROUTE_FULL_SOFTMAX 0x80u  /* gates are the softmax over all N router
+                                    logits taken at the k chosen experts (the
+                                    paper's Eq. (1) read literally: the gates
+                                    sum to less than 1) instead of the softmax
+                                    renormalised over the k chosen           */
+#define LMOE_ROUTE_BIAS_SELECT  0x100u /* the router bias only steers the choice
+                                    (auxiliary-loss-free balancing, the
+                                    paper's Section 4): experts are chosen on
+                                    the fp32 sum logit + bias, the gates use
+                                    the logit alone; lmoe_router_logits and
+                                    the logits stage then exclude the bias,
+                                    and lmoe_route_only adds the bias given to
+                                    lmoe_set_weights for the choice          */
 
 /* Limits of this build. */
 #define LMOE_MAX_EXPERTS 1024

@@ -560,7 +560,10 @@ lmoe_status run_routing(lmoe_layer* h, const float* logits, int T, int* idx, flo
   const int W = (T + 31) / 32;
   const int debug = (h->flags & LMOE_DEBUG_CHECKS) ? 1 : 0;
   {
-    const cudaError_t e = launch_topk(logits, T, h->N, h->k, idx, w, h->bitmap, W, debug, h->err, st);
+    const float* sel_bias = (h->flags & LMOE_ROUTE_BIAS_SELECT) ? h->bias : nullptr;
+    const int full = (h->flags & LMOE_ROUTE_FULL_SOFTMAX) ? 1 : 0;
+    const cudaError_t e = launch_topk(logits, T, h->N, h->k, sel_bias, full, idx, w, h->bitmap,
+                                      W, debug, h->err, st);
     if (e != cudaSuccess) return cuda_fail(h, e, "top-k launch");
     ++h->launches;
   }
@@ -579,7 +582,7 @@ lmoe_status run_router(lmoe_layer* h, const void* x, float* logits, int T, cudaS
   GemmCall c = dense_call(GK_ROUTER, T, x, h->d, h->Wg_t, h->N, h->d);
   c.p.epi.out = logits;
   c.p.epi.ldo = h->N;
-  c.p.epi.bias = h->bias;
+  c.p.epi.bias = (h->flags & LMOE_ROUTE_BIAS_SELECT) ? nullptr : h->bias;
   if (h->dtype == LMOE_BF16 && T >= 1024 && !(h->flags & (LMOE_FORCE_SIMT | LMOE_FORCE_NOPAIR)))
     make_pair(h, c);
   return run_gemm(h, c, st);
@@ -805,7 +808,8 @@ lmoe_status lmoe_create(int d, int l, int N, int k, int m, lmoe_act act, int sha
   if (!out) return LMOE_ERR_INVALID_ARG;
   *out = nullptr;
   const unsigned known = LMOE_SKIP_PROJ | LMOE_DEBUG_CHECKS | LMOE_FORCE_SIMT | LMOE_FORCE_SWAP |
-                         LMOE_FORCE_NOSWAP | LMOE_FORCE_NOPAIR | LMOE_FORCE_WS_PAIR;
+                         LMOE_FORCE_NOSWAP | LMOE_FORCE_NOPAIR | LMOE_FORCE_WS_PAIR |
+                         LMOE_ROUTE_FULL_SOFTMAX | LMOE_ROUTE_BIAS_SELECT;
   if (d <= 0 || l <= 0 || N <= 0 || k <= 0 || m <= 0 || shared_m < 0) return LMOE_ERR_INVALID_ARG;
   if (k > N || (flags & ~known)) return LMOE_ERR_INVALID_ARG;
   if (act != LMOE_ACT_SILU && act != LMOE_ACT_SWIGLU && act != LMOE_ACT_RELU2) return LMOE_ERR_INVALID_ARG;

@@ -91,14 +91,25 @@ __device__ __forceinline__ void warp_sort_desc64(unsigned long long& a, unsigned
 // decided so far); the selection is every key above tau plus the
 // lowest-indexed keys equal to tau.  Selection and order are exact integer
 // operations in both branches.
-template <int NPL>
-__global__ void __launch_bounds__(256) topk_softmax_kernel(const float* __restrict__ logits, int T,
-                                                           int N, int k, int* __restrict__ idx,
+//
+// Variants: with sel_bias the keys are the fp32 sums logit + sel_bias[e] (the
+// bias steers the choice only); the gates always come from the logits:
+// renormalised over the k chosen, or (full_softmax) the softmax over all N
+// logits taken at the chosen experts.
+template <int NPL, bool kVariant>
+__global__ void __launch_bounds__(128) topk_softmax_kernel(const float* __restrict__ logits, int T,
+                                                           int N, int k,
+                                                           const float* __restrict__ sel_bias,
+                                                           int full_softmax, int* __restrict__ idx,
                                                            float* __restrict__ w,
                                                            uint32_t* __restrict__ bitmap, int W,
                                                            int debug, int* err) {
-  __shared__ uint32_t s_hist[8][256];
-  __shared__ unsigned long long s_sel[8][64];
+  __shared__ uint32_t s_hist[4][256];
+  __shared__ unsigned long long s_sel[4][64];
+  if (!kVariant) {
+    sel_bias = nullptr;
+    full_softmax = 0;
+  }
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
   const int t = blockIdx.x * (blockDim.x >> 5) + wib;
   if (t >= T) return;
@@ -110,8 +121,9 @@ __global__ void __launch_bounds__(256) topk_softmax_kernel(const float* __restri
     const int e = lane + 32 * i;
     key[i] = 0u;  // absent experts: 0, never above a real key and never counted
     if (e < N) {
-      const float v = __ldg(lg + e);
+      float v = __ldg(lg + e);
       if (debug && !isfinite(v)) bad = true;
+      if (sel_bias) v = __fadd_rn(v, __ldg(sel_bias + e));
       key[i] = orderable_bits(v);
     }
   }
@@ -217,10 +229,27 @@ __global__ void __launch_bounds__(256) topk_softmax_kernel(const float* __restri
     warp_sort_desc64(v, b, lane);
   }
   const int e = (int)(0xFFFFFFFFu - (uint32_t)(v & 0xFFFFFFFFull));
-  const float val = from_orderable_bits((uint32_t)(v >> 32));
-  const float l0 = __shfl_sync(0xffffffffu, val, 0);
-  const float ex = lane < k ? expf(val - l0) : 0.f;
-  float sum = ex;
+  // the chosen logit of slot `lane` (the key itself unless a bias steered it)
+  float val = lane < k ? from_orderable_bits((uint32_t)(v >> 32)) : -INFINITY;
+  if (sel_bias && lane < k) val = __ldg(lg + e);
+  float M, sum;
+  if (!full_softmax) {
+    M = sel_bias ? val : __shfl_sync(0xffffffffu, val, 0);  // slot 0 holds the top logit
+    if (sel_bias) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    }
+    sum = lane < k ? expf(val - M) : 0.f;
+  } else {
+    // softmax over all N logits: max and sum of exp over the whole row
+    M = -INFINITY;
+    for (int c = lane; c < N; c += 32) M = fmaxf(M, __ldg(lg + c));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    sum = 0.f;
+    for (int c = lane; c < N; c += 32) sum += expf(__ldg(lg + c) - M);
+  }
+  const float ex = lane < k ? expf(val - M) : 0.f;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
   if (lane < k) {
@@ -232,14 +261,21 @@ __global__ void __launch_bounds__(256) topk_softmax_kernel(const float* __restri
 
 // Launches topk_softmax_kernel with the smallest multiple of 4 slots per lane
 // that covers N.
-static inline cudaError_t launch_topk(const float* logits, int T, int N, int k, int* idx, float* w,
+static inline cudaError_t launch_topk(const float* logits, int T, int N, int k,
+                                      const float* sel_bias, int full_softmax, int* idx, float* w,
                                       uint32_t* bitmap, int W, int debug, int* err,
                                       cudaStream_t st) {
-  const dim3 grid((T + 7) / 8), block(256);
-#define LMOE_TOPK_CASE(S)                                                                      \
-  case S:                                                                                      \
-    topk_softmax_kernel<S><<<grid, block, 0, st>>>(logits, T, N, k, idx, w, bitmap, W, debug, \
-                                                   err);                                       \
+  const dim3 grid((T + 3) / 4), block(128);
+  const bool var = sel_bias != nullptr || full_softmax != 0;
+#define LMOE_TOPK_CASE(S)                                                                        \
+  case S:                                                                                        \
+    if (var)                                                                                     \
+      topk_softmax_kernel<S, true><<<grid, block, 0, st>>>(logits, T, N, k, sel_bias,           \
+                                                           full_softmax, idx, w, bitmap, W,      \
+                                                           debug, err);                          \
+    else                                                                                         \
+      topk_softmax_kernel<S, false><<<grid, block, 0, st>>>(logits, T, N, k, nullptr, 0, idx, w, \
+                                                            bitmap, W, debug, err);              \
     break;
   switch ((N + 127) / 128 * 4) {
     LMOE_TOPK_CASE(4)

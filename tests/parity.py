@@ -42,7 +42,14 @@ def _cpu(t):
     return None if t is None else t.detach().to("cpu")
 
 
-def oracle_layer(w: workloads.Workload, W: Dict, experts: Optional[Iterable[int]] = None):
+def route_mode(flags: int) -> int:
+    """The oracle's routing variant bits for the library's flags."""
+    return ((oracle.ROUTE_FULL_SOFTMAX if flags & lmoe.ROUTE_FULL_SOFTMAX else 0) |
+            (oracle.ROUTE_BIAS_SELECT if flags & lmoe.ROUTE_BIAS_SELECT else 0))
+
+
+def oracle_layer(w: workloads.Workload, W: Dict, experts: Optional[Iterable[int]] = None,
+                 mode: int = 0):
     if experts is None:
         W1, W2 = _cpu(W["W1"]), _cpu(W["W2"])
     else:
@@ -53,7 +60,7 @@ def oracle_layer(w: workloads.Workload, W: Dict, experts: Optional[Iterable[int]
                               shared_m=w.shared_m, dtype=w.dtype, skip_proj=w.skip_proj,
                               Wg=_cpu(W["Wg"]), bias=_cpu(W["bias"]), Wdown=_cpu(W["Wdown"]),
                               Wup=_cpu(W["Wup"]), W1=W1, W2=W2, Ws1=_cpu(W["Ws1"]),
-                              Ws2=_cpu(W["Ws2"]))
+                              Ws2=_cpu(W["Ws2"]), route_mode=mode)
 
 
 def logit_bound(x_host: torch.Tensor, Wg_host: torch.Tensor, bias_host) -> np.ndarray:
@@ -98,10 +105,17 @@ def check_forward(w: workloads.Workload, flags: int = 0, tokens: Optional[np.nda
         tokens = np.arange(T, dtype=np.int32)
     tokens = np.asarray(tokens, dtype=np.int32)
     x_host = x.cpu()
-    O0 = oracle_layer(w, W, experts=[])
+    mode = route_mode(flags)
+    O0 = oracle_layer(w, W, experts=[], mode=mode)
     lg64 = O0.router_logits(x_host, tokens)
     lg32 = lg64.astype(np.float32)
-    o_idx, o_w, _, _ = oracle.route(lg32, w.k)
+    sel_bias = None
+    keys32 = lg32  # what the selection compares
+    if mode & oracle.ROUTE_BIAS_SELECT and W["bias"] is not None:
+        sel_bias = _cpu(W["bias"]).float().numpy()
+        keys32 = lg32 + sel_bias[None, :]
+    o_idx, o_w, _, _ = oracle.route(lg32, w.k, sel_bias=sel_bias,
+                                    full_softmax=bool(mode & oracle.ROUTE_FULL_SOFTMAX))
 
     # logits: within the accumulation bound of the oracle's
     tau = logit_bound(x_host[tokens], _cpu(W["Wg"]), _cpu(W["bias"]))
@@ -110,7 +124,7 @@ def check_forward(w: workloads.Workload, flags: int = 0, tokens: Optional[np.nda
     logit_rel = rel_l2(g_lg[tokens].astype(np.float64), lg64)
 
     # routing: unique where the oracle's top-k boundary is wider than 2 tau
-    srt = -np.sort(-lg32.astype(np.float64), axis=1)
+    srt = -np.sort(-keys32.astype(np.float64), axis=1)
     kth = srt[:, w.k - 1]
     nxt = srt[:, w.k] if w.k < w.N else np.full(len(tokens), -np.inf)
     tmax = tau.max(axis=1)
@@ -119,19 +133,19 @@ def check_forward(w: workloads.Workload, flags: int = 0, tokens: Optional[np.nda
     assert np.array_equal(gi[uniq], o_idx[uniq]), "selected experts differ on unique tokens"
     assert np.all(np.abs(g_w[tokens][uniq] - o_w[uniq]) <= 1e-3)
     for r in np.nonzero(~uniq)[0]:
-        chosen = lg32[r, gi[r]].astype(np.float64)
+        chosen = keys32[r, gi[r]].astype(np.float64)
         assert len(set(gi[r].tolist())) == w.k
         assert np.all(chosen >= kth[r] - 2 * tmax[r])
         others = np.setdiff1d(np.arange(w.N), gi[r])
         if others.size:
-            assert np.all(lg32[r, others] <= kth[r] + 2 * tmax[r])
+            assert np.all(keys32[r, others] <= kth[r] + 2 * tmax[r])
 
     # outputs of the unique tokens
     ut = tokens[uniq]
     res = {"tokens": len(tokens), "unique": int(uniq.sum()), "logit_rel_l2": logit_rel}
     if ut.size:
         experts = np.unique(o_idx[uniq])
-        O = oracle_layer(w, W, experts=experts)
+        O = oracle_layer(w, W, experts=experts, mode=mode)
         ref, z, comb = O.forward(x_host, o_idx[uniq], o_w[uniq], tokens=ut, stages=True)
         got = g_out[ut]
         res.update(compare_outputs(got, ref, w.dtype, fixture=fixture))

@@ -75,6 +75,46 @@ def test_route_only_bit_exact_crowded_logits(T, N, k):
     np.testing.assert_allclose(r["w"].cpu().numpy(), o_w, rtol=2e-6, atol=1e-7)
 
 
+ROUTE_VARIANTS = [lmoe.ROUTE_FULL_SOFTMAX, lmoe.ROUTE_BIAS_SELECT,
+                  lmoe.ROUTE_FULL_SOFTMAX | lmoe.ROUTE_BIAS_SELECT]
+
+
+@pytest.mark.parametrize("flags", ROUTE_VARIANTS)
+@pytest.mark.parametrize("T,N,k", [(300, 896, 16), (257, 512, 32), (100, 16, 4), (40, 128, 8)])
+def test_route_only_variants_bit_exact(flags, T, N, k):
+    """Routing variants on shared logits: the choice (on logit + bias in
+    fp32 when the bias selects only) bit-exact; gates from the logits alone,
+    renormalised or the softmax over all N (fp32 sum over N: 2e-5)."""
+    w_ = W_("route-var", T=T, d=64, l=64, N=N, k=k, m=64, act="silu", bias="normal0.5",
+            seed=T + N)
+    W = workloads.make_weights(w_, device="cuda")
+    W["bias"] = (torch.randn(N, generator=torch.Generator().manual_seed(N)) * 2.0).cuda()
+    L, _ = gpu_layer(w_, flags, W)
+    lg = workloads.make_logits(T, N, seed=T * 3 + k, ties=True)
+    r = L.route_only(lg.cuda())
+    torch.cuda.synchronize()
+    sb = W["bias"].cpu().numpy() if flags & lmoe.ROUTE_BIAS_SELECT else None
+    o_idx, o_w, o_off, o_perm = oracle.route(lg.numpy(), k, sel_bias=sb,
+                                             full_softmax=bool(flags & lmoe.ROUTE_FULL_SOFTMAX))
+    np.testing.assert_array_equal(r["idx"].cpu().numpy(), o_idx)
+    np.testing.assert_array_equal(r["offsets"].cpu().numpy(), o_off)
+    np.testing.assert_array_equal(r["perm"].cpu().numpy(), o_perm)
+    rtol = 2e-5 if flags & lmoe.ROUTE_FULL_SOFTMAX else 2e-6
+    np.testing.assert_allclose(r["w"].cpu().numpy(), o_w, rtol=rtol, atol=1e-9)
+    if flags & lmoe.ROUTE_BIAS_SELECT:  # the bias is large enough to move the choice
+        assert not np.array_equal(o_idx, oracle.route(lg.numpy(), k)[0])
+
+
+@pytest.mark.parametrize("flags", ROUTE_VARIANTS)
+@pytest.mark.parametrize("name", ["silu-bias", "fp32"])
+def test_forward_routing_variants(name, flags):
+    w = SMALL[name]
+    W = workloads.make_weights(w, device="cuda")
+    W["bias"] = (torch.randn(w.N, generator=torch.Generator().manual_seed(7)) * 1.5).cuda()
+    res = check_forward(w, flags=flags, W=W, fixture=True)
+    assert res["unique"] >= 0.8 * res["tokens"]
+
+
 def test_route_only_rejects_oversized_T():
     L = lmoe.LatentMoELayer(64, 64, 16, 4, 64, act="silu", dtype="bf16")
     L.reserve(8)
