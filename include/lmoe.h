@@ -158,9 +158,13 @@ lmoe_status lmoe_forward(lmoe_layer* h, const void* x, void* out, int T, lmoe_st
 /*
  * lmoe_forward_host -- lmoe_forward with HOST buffers: copies x_host (host,
  * [T, d]) into library staging memory, runs the layer and copies the result
- * to out_host (host, [T, d]), all enqueued on stream; the caller synchronises
- * the stream before reading out_host.  Pinned host memory makes the copies
- * asynchronous.  Errors: as lmoe_forward.
+ * to out_host (host, [T, d]).  The upload runs on a library-owned copy stream
+ * into one of two staging slots (alternating per call), so it overlaps the
+ * previous call's forward; the forward and the download are enqueued on
+ * stream after it.  The caller synchronises stream before reading out_host or
+ * reusing x_host.  Pinned host memory makes the copies asynchronous.  Calls
+ * on one handle must come from one host thread at a time.  Errors: as
+ * lmoe_forward.
  */
 lmoe_status lmoe_forward_host(lmoe_layer* h, const void* x_host, void* out_host, int T,
                               lmoe_stream_t stream);

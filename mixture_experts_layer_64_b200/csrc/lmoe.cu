@@ -90,6 +90,12 @@ struct lmoe_layer {
   float* row_w = nullptr;
   void *z = nullptr, *h = nullptr, *ys = nullptr, *cat = nullptr;
   void *x_stage = nullptr, *out_stage = nullptr;
+  // host entry: a second x staging slot, a copy stream for the uploads, and
+  // per slot "upload done" / "forward done reading the slot" events
+  void* x_stage2 = nullptr;
+  cudaStream_t copy_stream = nullptr;
+  cudaEvent_t ev_up[2] = {nullptr, nullptr}, ev_used[2] = {nullptr, nullptr};
+  int host_slot = 0;
   float* s32 = nullptr;  // [T, d] fp32 shared-expert output (projection-skip layers)
   float* part = nullptr;  // split-K partial sums of the dense GEMMs at small T
   size_t part_bytes = 0;
@@ -676,16 +682,22 @@ lmoe_status run_forward(lmoe_layer* h, const void* x, void* out, int T, cudaStre
     const bool vec_ok = (l % vec == 0) && (ldo % vec == 0) && aligned16(dst) && aligned16(h->ys) &&
                         (!resid || (aligned16(resid) && d % vec == 0));
     const int threads = std::min(256, std::max(32, (l / vec + 31) / 32 * 32));
+    // split a token's columns over blocks when T alone does not fill the GPU
+    const int per_block = threads * vec;
+    const int chunks = std::max(1, std::min((l + per_block - 1) / per_block,
+                                            (2 * h->num_sms + T - 1) / std::max(T, 1)));
+    const dim3 cgrid((unsigned)T, (unsigned)chunks);
     if (h->dtype == LMOE_BF16) {
       if (vec_ok)
-        combine_kernel<bf16><<<T, threads, 0, st>>>((const bf16*)h->ys, h->slot_row, k, l, (const bf16*)resid,
-                                                    d, add32, (bf16*)dst, ldo);
+        combine_kernel<bf16><<<cgrid, threads, 0, st>>>((const bf16*)h->ys, h->slot_row, k, l,
+                                                        (const bf16*)resid, d, add32, (bf16*)dst,
+                                                        ldo);
       else
         combine_scalar_kernel<bf16><<<T, 256, 0, st>>>((const bf16*)h->ys, h->slot_row, k, l,
                                                        (const bf16*)resid, d, add32, (bf16*)dst, ldo);
     } else {
       if (vec_ok)
-        combine_kernel<float><<<T, threads, 0, st>>>((const float*)h->ys, h->slot_row, k, l,
+        combine_kernel<float><<<cgrid, threads, 0, st>>>((const float*)h->ys, h->slot_row, k, l,
                                                      (const float*)resid, d, add32, (float*)dst, ldo);
       else
         combine_scalar_kernel<float><<<T, 256, 0, st>>>((const float*)h->ys, h->slot_row, k, l,
@@ -736,7 +748,16 @@ void free_workspace(lmoe_layer* h) {
   free_ptr(h->ys);
   free_ptr(h->cat);
   free_ptr(h->x_stage);
+  free_ptr(h->x_stage2);
   free_ptr(h->out_stage);
+  for (int i = 0; i < 2; ++i) {
+    if (h->ev_up[i]) cudaEventDestroy(h->ev_up[i]);
+    if (h->ev_used[i]) cudaEventDestroy(h->ev_used[i]);
+    h->ev_up[i] = h->ev_used[i] = nullptr;
+  }
+  if (h->copy_stream) cudaStreamDestroy(h->copy_stream);
+  h->copy_stream = nullptr;
+  h->host_slot = 0;
   free_ptr(h->s32);
   free_ptr(h->part);
   h->part_bytes = 0;
@@ -914,7 +935,13 @@ lmoe_status lmoe_reserve(lmoe_layer* h, int max_T) {
   ALLOC(h->ys, R * h->l * es);
   if (h->Kup > 0) ALLOC(h->cat, T * h->Kup * es);
   ALLOC(h->x_stage, T * h->d * es);
+  ALLOC(h->x_stage2, T * h->d * es);
   ALLOC(h->out_stage, T * h->d * es);
+  LMOE_CUDA(h, cudaStreamCreateWithFlags(&h->copy_stream, cudaStreamNonBlocking));
+  for (int i = 0; i < 2; ++i) {
+    LMOE_CUDA(h, cudaEventCreateWithFlags(&h->ev_up[i], cudaEventDisableTiming));
+    LMOE_CUDA(h, cudaEventCreateWithFlags(&h->ev_used[i], cudaEventDisableTiming));
+  }
   if (skip && h->shared_m > 0) ALLOC(h->s32, T * h->d * sizeof(float));
   if (h->dtype == LMOE_BF16) {
     h->part_bytes = kSplitPartBytes;
@@ -953,8 +980,20 @@ lmoe_status lmoe_forward_host(lmoe_layer* h, const void* x_host, void* out_host,
   DevGuard g(h->device);
   cudaStream_t st = (cudaStream_t)stream;
   const size_t bytes = (size_t)T * h->d * h->es;
-  LMOE_CUDA(h, cudaMemcpyAsync(h->x_stage, x_host, bytes, cudaMemcpyHostToDevice, st));
-  LMOE_TRY(run_forward(h, h->x_stage, h->out_stage, T, st));
+  // The upload runs on the library's copy stream into one of two staging
+  // slots, so that it can overlap the previous call's forward (which reads
+  // the other slot); it waits until the forward that last read this slot has
+  // finished.  The caller's stream waits for the upload; the download stays
+  // on the caller's stream, so out_host is complete when that stream is.
+  const int s = h->host_slot;
+  h->host_slot ^= 1;
+  void* xs = s ? h->x_stage2 : h->x_stage;
+  LMOE_CUDA(h, cudaStreamWaitEvent(h->copy_stream, h->ev_used[s], 0));
+  LMOE_CUDA(h, cudaMemcpyAsync(xs, x_host, bytes, cudaMemcpyHostToDevice, h->copy_stream));
+  LMOE_CUDA(h, cudaEventRecord(h->ev_up[s], h->copy_stream));
+  LMOE_CUDA(h, cudaStreamWaitEvent(st, h->ev_up[s], 0));
+  LMOE_TRY(run_forward(h, xs, h->out_stage, T, st));
+  LMOE_CUDA(h, cudaEventRecord(h->ev_used[s], st));
   LMOE_CUDA(h, cudaMemcpyAsync(out_host, h->out_stage, bytes, cudaMemcpyDeviceToHost, st));
   return LMOE_OK;
 }

@@ -10,7 +10,8 @@ namespace lmoe {
 // comb[t, c] = (resid[t, c] +) sum_{j < k} ys[slot_row[t*k + j], c], summed in
 // fp32 in slot order, rounded once.  ys rows are in expert order (as the
 // expert GEMMs wrote them); slot_row maps each (token, slot) pair to its row.
-// One block per token, VEC elements per thread per step (16-byte accesses).
+// Block (t, y) covers token t's columns y*blockDim*VEC, ... with a stride of
+// gridDim.y*blockDim*VEC: VEC elements per thread per step (16-byte accesses).
 // With add32 (fp32, row stride ldr) that addend joins the sum before the one
 // rounding: the projection-skip layer adds its shared expert this way.
 template <typename T>
@@ -22,7 +23,8 @@ __global__ void __launch_bounds__(256) combine_kernel(const T* __restrict__ ys,
   constexpr int VEC = 16 / sizeof(T);
   const int t = blockIdx.x;
   const int* rows = slot_row + (size_t)t * k;
-  for (int c = threadIdx.x * VEC; c < l; c += blockDim.x * VEC) {
+  for (int c = (blockIdx.y * blockDim.x + threadIdx.x) * VEC; c < l;
+       c += gridDim.y * blockDim.x * VEC) {
     float acc[VEC];
     if (resid) {
       const uint4 rv = *reinterpret_cast<const uint4*>(resid + (size_t)t * ldr + c);

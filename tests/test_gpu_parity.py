@@ -261,6 +261,28 @@ def test_forward_is_deterministic_and_host_entry_matches():
     assert torch.equal(oh, a.cpu())
 
 
+def test_host_entry_back_to_back_calls():
+    """Consecutive host-buffer calls alternate two staging slots and upload on
+    a copy stream while the previous forward runs: four calls with different
+    inputs and no synchronisation in between must each equal the device-buffer
+    forward of their own input."""
+    w = SMALL["relu2-shared"]
+    L, W = gpu_layer(w)
+    x0 = workloads.make_x(w, device="cuda").float()
+    xs = [(x0 * (1.0 + 0.25 * i)).roll(i, dims=0).to(torch.bfloat16).contiguous()
+          for i in range(4)]
+    ref = [L.forward(x).cpu() for x in xs]
+    torch.cuda.synchronize()
+    xh = [x.cpu().pin_memory() for x in xs]
+    oh = [torch.empty_like(h).pin_memory() for h in xh]
+    for a, b in zip(xh, oh):
+        L.forward_host(a, b)
+    torch.cuda.synchronize()
+    for i in range(4):
+        assert torch.equal(oh[i], ref[i]), i
+    assert L.last_error() == (lmoe.OK, 0)
+
+
 def test_uniform_router_is_mean_of_experts():
     """W_g = 0, k = N: every token uses every expert with weight 1/N."""
     w = W_("uniform", T=64, d=128, l=64, N=4, k=4, m=64, act="relu2", seed=19)
