@@ -96,6 +96,20 @@ WORKLOADS: Dict[str, Workload] = {
 }
 WORKLOAD_ORDER = list(WORKLOADS)
 
+
+def quantize_e4m3(W: torch.Tensor):
+    """Per-output-column fp8 E4M3 quantisation of a weight stack in the API
+    layout [..., in, out]: scale[..., o] = max_i |W[..., i, o]| / 448 (fp32,
+    1 for an all-zero column) and codes = W / scale rounded to E4M3 by
+    torch's float8_e4m3fn conversion.  Returns (codes uint8 [..., in, out],
+    scales float32 [..., out]).  Inputs for the fp8 expert weights: the
+    library and the oracle both read these codes and scales."""
+    Wf = W.float()
+    amax = Wf.abs().amax(dim=-2)
+    scale = torch.where(amax > 0, amax / 448.0, torch.ones_like(amax))
+    codes = (Wf / scale.unsqueeze(-2)).to(torch.float8_e4m3fn).view(torch.uint8)
+    return codes.contiguous(), scale.contiguous()
+
 _TID = {"x": 1, "Wg": 2, "bias": 3, "Wdown": 4, "Wup": 5, "W1": 6, "W2": 7,
         "Ws1": 8, "Ws2": 9}
 

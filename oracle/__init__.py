@@ -35,7 +35,8 @@ class _Layer(ctypes.Structure):
                 ("Wdown", ctypes.c_void_p), ("Wup", ctypes.c_void_p),
                 ("W1", ctypes.c_void_p), ("W2", ctypes.c_void_p),
                 ("Ws1", ctypes.c_void_p), ("Ws2", ctypes.c_void_p),
-                ("route_mode", ctypes.c_int)]
+                ("route_mode", ctypes.c_int),
+                ("expert_fp8", ctypes.c_int), ("W1s", ctypes.c_void_p), ("W2s", ctypes.c_void_p)]
 
 # routing variants (bits of route_mode)
 ROUTE_FULL_SOFTMAX, ROUTE_BIAS_SELECT = 1, 2
@@ -62,6 +63,8 @@ def lib():
                   L.oracle_layer, L.oracle_hardware_threads):
             f.restype = I
         L.oracle_hardware_threads.argtypes = []
+        L.oracle_e4m3_value.argtypes = [I]
+        L.oracle_e4m3_value.restype = ctypes.c_double
         _lib = L
     return _lib
 
@@ -98,12 +101,15 @@ class OracleLayer:
     """Host copy of one layer's weights, in the API layout [in, out].
 
     ``W1``/``W2`` are either full stacks ``[N, ...]`` or a mapping
-    expert -> matrix holding only the experts that will be reached.
+    expert -> matrix holding only the experts that will be reached.  With
+    ``W1s``/``W2s`` (per-expert fp32 scales per output column, ``[N, m_in]``
+    and ``[N, l]``, stacks or mappings) ``W1``/``W2`` are fp8 E4M3 codes
+    (uint8) in the same layouts.
     """
 
     def __init__(self, *, d, l, N, k, m, act, shared_m=0, dtype="bf16",
                  skip_proj=False, Wg, bias=None, Wdown=None, Wup=None,
-                 W1, W2, Ws1=None, Ws2=None, route_mode=0):
+                 W1, W2, Ws1=None, Ws2=None, route_mode=0, W1s=None, W2s=None):
         self.d, self.l, self.N, self.k, self.m = d, l, N, k, m
         self.act, self.shared_m, self.dtype, self.skip_proj = act, shared_m, dtype, skip_proj
         keep = []
@@ -120,19 +126,42 @@ class OracleLayer:
         if bias is not None:
             self._bias = np.ascontiguousarray(_host_array(bias, "f32"), dtype=np.float32)
             keep.append(self._bias)
+        fp8 = W1s is not None or W2s is not None
+        if fp8 and (W1s is None or W2s is None):
+            raise OracleError("fp8 expert weights need both W1s and W2s")
+
+        def arr8(t):  # E4M3 codes, or fp32 scales
+            if t is None:
+                return None
+            a = _host_array(t, "f32")
+            a = np.ascontiguousarray(a, dtype=np.uint8 if a.dtype == np.uint8 else np.float32)
+            keep.append(a)
+            return a
+
+        warr = arr8 if fp8 else arr
         p1 = (ctypes.c_void_p * N)()
         p2 = (ctypes.c_void_p * N)()
+        s1 = (ctypes.c_void_p * N)()
+        s2 = (ctypes.c_void_p * N)()
         for e in range(N):
-            a1 = self._expert(W1, e, arr)
-            a2 = self._expert(W2, e, arr)
+            a1 = self._expert(W1, e, warr)
+            a2 = self._expert(W2, e, warr)
+            if fp8 and ((a1 is not None and a1.dtype != np.uint8) or
+                        (a2 is not None and a2.dtype != np.uint8)):
+                raise OracleError("fp8 expert weights must be uint8 E4M3 codes")
             p1[e] = _ptr(a1)
             p2[e] = _ptr(a2)
-        self._p1, self._p2, self._keep = p1, p2, keep
+            if fp8:
+                s1[e] = _ptr(self._expert(W1s, e, arr8))
+                s2[e] = _ptr(self._expert(W2s, e, arr8))
+        self._p1, self._p2, self._s1, self._s2, self._keep = p1, p2, s1, s2, keep
         self.struct = _Layer(d, l, N, k, m, ACT_CODES[act], shared_m, DTYPE_CODES[dtype],
                              int(bool(skip_proj)), _ptr(self._Wg), _ptr(self._bias),
                              _ptr(self._Wdown), _ptr(self._Wup),
                              ctypes.cast(p1, ctypes.c_void_p), ctypes.cast(p2, ctypes.c_void_p),
-                             _ptr(self._Ws1), _ptr(self._Ws2), int(route_mode))
+                             _ptr(self._Ws1), _ptr(self._Ws2), int(route_mode),
+                             int(fp8), ctypes.cast(s1, ctypes.c_void_p),
+                             ctypes.cast(s2, ctypes.c_void_p))
 
     @staticmethod
     def _expert(W, e, arr):
@@ -214,6 +243,11 @@ def route(logits32, k: int, nthreads: Optional[int] = None, sel_bias=None,
     if rc:
         raise OracleError(f"oracle_route failed ({rc})")
     return idx, w, offsets, perm
+
+
+def e4m3_value(code: int) -> float:
+    """The exact value of one fp8 E4M3 code, as the oracle reads it."""
+    return float(lib().oracle_e4m3_value(int(code)))
 
 
 def hardware_threads() -> int:

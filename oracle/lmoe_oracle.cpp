@@ -36,7 +36,11 @@
 //
 // Weights use the API layout [in, out] row-major (y = x . W); the expert
 // stacks are passed as one pointer per expert so that a caller may supply
-// only the experts its tokens reach (the others may be NULL).
+// only the experts its tokens reach (the others may be NULL).  Expert weights
+// may instead be fp8 E4M3 codes with one fp32 scale per output column (low-
+// precision expert weights: the paper's Section 2 models FP4 weights, its
+// Section 4.3 measures FP8 quantisation): the oracle widens each code to the
+// exact value it denotes and multiplies by its column's scale.
 #include <algorithm>
 #include <atomic>
 #include <cmath>
@@ -47,7 +51,7 @@
 
 namespace {
 
-enum { OR_F32 = 0, OR_BF16 = 1 };
+enum { OR_F32 = 0, OR_BF16 = 1, OR_E4M3 = 2 };
 enum { OR_ACT_SILU = 0, OR_ACT_SWIGLU = 1, OR_ACT_RELU2 = 2 };
 enum { OR_OK = 0, OR_ERR_ARG = 1, OR_ERR_NAN = 2, OR_ERR_MISSING = 3 };
 // Routing variants (paper Section 3 and Section 4):
@@ -59,8 +63,21 @@ enum { OR_OK = 0, OR_ERR_ARG = 1, OR_ERR_NAN = 2, OR_ERR_MISSING = 3 };
 //                          are chosen on l + b, the gates use l
 enum { OR_ROUTE_FULL_SOFTMAX = 1, OR_ROUTE_BIAS_SELECT = 2 };
 
+// One fp8 E4M3 code (the OCP "E4M3FN" encoding: 1 sign, 4 exponent bits with
+// bias 7, 3 mantissa bits; exponent field 0 is subnormal, S.1111.111 is NaN,
+// no infinities; largest finite 448) as the exact double it denotes.
+inline double e4m3_value(uint8_t c) {
+  const int sgn = c >> 7, E = (c >> 3) & 15, m = c & 7;
+  double v;
+  if (E == 15 && m == 7) v = NAN;
+  else if (E == 0) v = std::ldexp((double)m, -9);           // m/8 * 2^-6
+  else v = std::ldexp(8.0 + m, E - 10);                    // (1 + m/8) * 2^(E-7)
+  return sgn ? -v : v;
+}
+
 inline double widen(const void* p, int dtype, size_t i) {
   if (dtype == OR_F32) return (double)static_cast<const float*>(p)[i];
+  if (dtype == OR_E4M3) return e4m3_value(static_cast<const uint8_t*>(p)[i]);
   uint32_t bits = (uint32_t)static_cast<const uint16_t*>(p)[i] << 16;
   float f;
   std::memcpy(&f, &bits, sizeof f);
@@ -104,12 +121,15 @@ void apply_act(int act, const double* a, int m, double* h) {
 
 // acc[p][o] = sum_i in[p][i] * W[i][o] for p in [0, P), sequential in i.
 // in: P rows of width K (double); W: [K, O] in dtype; acc: P rows of width O.
+// col_scale (fp8 weights): W[i][o] stands for code(i, o) * col_scale[o].
 void rows_times_matrix(const double* in, int P, int K, const void* W, int dtype,
-                       int O, double* acc, std::vector<double>& wrow) {
+                       int O, double* acc, std::vector<double>& wrow,
+                       const float* col_scale = nullptr) {
   std::fill(acc, acc + (size_t)P * O, 0.0);
   wrow.resize(O);
   for (int i = 0; i < K; ++i) {
-    for (int o = 0; o < O; ++o) wrow[o] = widen(W, dtype, (size_t)i * O + o);
+    for (int o = 0; o < O; ++o)
+      wrow[o] = widen(W, dtype, (size_t)i * O + o) * (col_scale ? (double)col_scale[o] : 1.0);
     for (int p = 0; p < P; ++p) {
       const double zi = in[(size_t)p * K + i];
       double* a = acc + (size_t)p * O;
@@ -133,6 +153,11 @@ struct OracleLayer {
   const void* Ws1;         // [d, ms_in] or NULL when shared_m == 0
   const void* Ws2;         // [shared_m, d]
   int route_mode;          // OR_ROUTE_* bits (0: the default routing)
+  // fp8 expert weights: W1[e] / W2[e] hold E4M3 codes in the same layouts,
+  // W1s[e] [m_in] and W2s[e] [l] one fp32 scale per output column.
+  int expert_fp8;
+  const float* const* W1s;
+  const float* const* W2s;
 };
 
 static int m_in_of(int act, int m) { return act == OR_ACT_SWIGLU ? 2 * m : m; }
@@ -267,7 +292,9 @@ int oracle_forward(const OracleLayer* L, const void* x, const int* tokens, int S
     const int e = idx[p];
     if (e < 0 || e >= N) return OR_ERR_ARG;
     if (!L->W1[e] || !L->W2[e]) return OR_ERR_MISSING;
+    if (L->expert_fp8 && (!L->W1s || !L->W2s || !L->W1s[e] || !L->W2s[e])) return OR_ERR_MISSING;
   }
+  const int edt = L->expert_fp8 ? OR_E4M3 : dt;  // the expert weights' element type
 
   // x rows in float64.
   std::vector<double> X((size_t)S * d);
@@ -303,9 +330,11 @@ int oracle_forward(const OracleLayer* L, const void* x, const int* tokens, int S
       const int s = pairs[e][q0 + p] / k;
       std::memcpy(&zin[(size_t)p * l], &Z[(size_t)s * l], l * sizeof(double));
     }
-    rows_times_matrix(zin.data(), P, l, L->W1[e], dt, m_in, a.data(), wrow);
+    rows_times_matrix(zin.data(), P, l, L->W1[e], edt, m_in, a.data(), wrow,
+                      L->expert_fp8 ? L->W1s[e] : nullptr);
     for (int p = 0; p < P; ++p) apply_act(L->act, &a[(size_t)p * m_in], m, &h[(size_t)p * m]);
-    rows_times_matrix(h.data(), P, m, L->W2[e], dt, l, y.data(), wrow);
+    rows_times_matrix(h.data(), P, m, L->W2[e], edt, l, y.data(), wrow,
+                      L->expert_fp8 ? L->W2s[e] : nullptr);
     for (int p = 0; p < P; ++p)
       std::memcpy(&Y[(size_t)pairs[e][q0 + p] * l], &y[(size_t)p * l], l * sizeof(double));
   });
@@ -366,5 +395,8 @@ int oracle_layer(const OracleLayer* L, const void* x, const int* tokens, int S,
 }
 
 int oracle_hardware_threads(void) { return (int)std::thread::hardware_concurrency(); }
+
+// The value an fp8 E4M3 code denotes (exposed for its pin).
+double oracle_e4m3_value(int code) { return e4m3_value((uint8_t)code); }
 
 }  // extern "C"

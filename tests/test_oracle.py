@@ -421,3 +421,80 @@ def test_tiny_workload_end_to_end_runs():
     r = L.layer(x)
     assert r["out"].shape == (w.T, w.d) and np.all(np.isfinite(r["out"]))
     np.testing.assert_allclose(r["w"].sum(1), 1.0, atol=1e-15)
+
+
+# ---------------------------------------------------------------------------
+# fp8 E4M3 expert weights with per-output-column scales
+# ---------------------------------------------------------------------------
+
+def test_e4m3_decode_matches_torch_for_every_code():
+    """The oracle's E4M3 decoder against torch's float8_e4m3fn conversion (a
+    library routine) for all 256 codes: 0x7F/0xFF are NaN, the rest exact."""
+    codes = torch.arange(256, dtype=torch.uint8)
+    ref = codes.view(torch.float8_e4m3fn).float().numpy().astype(f64)
+    got = np.array([oracle.e4m3_value(c) for c in range(256)])
+    nan = np.isnan(ref)
+    assert list(np.nonzero(nan)[0]) == [0x7F, 0xFF]
+    assert np.array_equal(np.isnan(got), nan)
+    np.testing.assert_array_equal(got[~nan], ref[~nan])
+    assert got[0x7E] == 448.0 and got[0x01] == 2.0 ** -9 and got[0x08] == 2.0 ** -6
+
+
+def test_quantiser_round_trip():
+    """Per-column scales map each column's largest magnitude to 448, and the
+    decoded codes times the scales stay within half an E4M3 step of W."""
+    W = rnd((3, 40, 24), 0.2, 51, "f32")
+    codes, scale = workloads.quantize_e4m3(W)
+    assert codes.dtype == torch.uint8 and scale.shape == (3, 24)
+    dec = np.vectorize(oracle.e4m3_value)(codes.numpy())
+    deq = dec * scale.numpy()[:, None, :]
+    np.testing.assert_allclose(np.abs(dec).max(axis=1), 448.0)
+    Wn = W.double().numpy()
+    # relative half-step of E4M3 (3 mantissa bits) = 2^-4, or the subnormal step
+    tol = np.maximum(np.abs(Wn) * 2.0 ** -4, scale.numpy()[:, None, :] * 2.0 ** -10)
+    assert np.all(np.abs(deq - Wn) <= tol * 1.0000001)
+
+
+@pytest.mark.parametrize("act", ["swiglu", "relu2"])
+def test_fp8_single_expert_is_dense_chain(act):
+    """N = k = 1 with fp8 experts: the layer is x + act(z (q1 s1)) (q2 s2) Wup
+    with the dequantised matrices built in numpy (codes decoded, each output
+    column times its scale)."""
+    d, l, m = 48, 32, 40
+    L0, W = make_layer(d, l, 1, 1, m, act, seed=60, dtype="f32")
+    q1, s1 = workloads.quantize_e4m3(W["W1"])
+    q2, s2 = workloads.quantize_e4m3(W["W2"])
+    L = oracle.OracleLayer(d=d, l=l, N=1, k=1, m=m, act=act, dtype="f32", Wg=W["Wg"],
+                           Wdown=W["Wdown"], Wup=W["Wup"], W1=q1, W2=q2, W1s=s1, W2s=s2)
+    x = rnd((7, d), 1.0, 61, "f32")
+    dec = np.vectorize(oracle.e4m3_value)
+    W1d = dec(q1[0].numpy()) * s1[0].double().numpy()[None, :]
+    W2d = dec(q2[0].numpy()) * s2[0].double().numpy()[None, :]
+    z = as64(x) @ as64(W["Wdown"])
+    h = np_act(act, z @ W1d, m)
+    ref = as64(x) + (h @ W2d) @ as64(W["Wup"])
+    res = L.layer(x)
+    np.testing.assert_allclose(res["out"], ref, rtol=1e-12, atol=1e-12)
+
+
+def test_fp8_layer_equals_layer_with_dequantised_weights():
+    """Many experts: the fp8 layer equals the f32 layer whose expert weights
+    are the dequantised values (rounded to fp32, hence 1e-6); a scale applied
+    per input row instead of per output column would miss by far."""
+    d, l, N, k, m = 40, 24, 6, 2, 16
+    L0, W = make_layer(d, l, N, k, m, "swiglu", dtype="f32", bias=True, seed=70)
+    q1, s1 = workloads.quantize_e4m3(W["W1"])
+    q2, s2 = workloads.quantize_e4m3(W["W2"])
+    dec = np.vectorize(oracle.e4m3_value)
+    W1d = torch.from_numpy((dec(q1.numpy()) * s1.double().numpy()[:, None, :]).astype(np.float32))
+    W2d = torch.from_numpy((dec(q2.numpy()) * s2.double().numpy()[:, None, :]).astype(np.float32))
+    common = dict(d=d, l=l, N=N, k=k, m=m, act="swiglu", dtype="f32", Wg=W["Wg"],
+                  bias=W["bias"], Wdown=W["Wdown"], Wup=W["Wup"])
+    L8 = oracle.OracleLayer(W1=q1, W2=q2, W1s=s1, W2s=s2, **common)
+    Ld = oracle.OracleLayer(W1=W1d, W2=W2d, **common)
+    x = rnd((30, d), 1.0, 71, "f32")
+    a, b = L8.layer(x), Ld.layer(x)
+    np.testing.assert_array_equal(a["idx"], b["idx"])
+    np.testing.assert_allclose(a["out"], b["out"], rtol=1e-6, atol=1e-6)
+    with pytest.raises(oracle.OracleError):
+        oracle.OracleLayer(W1=q1, W2=q2, W1s=s1, **common)
