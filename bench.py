@@ -175,8 +175,9 @@ class OracleRunner:
                          dtype=w.dtype, skip_proj=w.skip_proj, Wg=cpu(W_dev["Wg"]),
                          bias=cpu(W_dev["bias"]), Wdown=cpu(W_dev["Wdown"]),
                          Wup=cpu(W_dev["Wup"]), Ws1=cpu(W_dev["Ws1"]), Ws2=cpu(W_dev["Ws2"]))
+        self.fp8 = bool(w.expert_fp8)
         self.probe = oracle.OracleLayer(W1={}, W2={}, **self.base)
-        self.W1, self.W2 = {}, {}
+        self.W1, self.W2, self.S1, self.S2 = {}, {}, {}, {}
 
     def time_tokens(self, tokens: np.ndarray) -> float:
         """Seconds the oracle takes for the whole layer on `tokens` (routing
@@ -185,9 +186,16 @@ class OracleRunner:
         idx, _, _, _ = self.oracle.route(lg, self.w.k)
         for e in np.unique(idx).tolist():
             if e not in self.W1:
-                self.W1[e] = self.W_dev["W1"][e].cpu()
-                self.W2[e] = self.W_dev["W2"][e].cpu()
-        O = self.oracle.OracleLayer(W1=self.W1, W2=self.W2, **self.base)
+                if self.fp8:
+                    self.W1[e] = self.W_dev["W1q"][e].cpu()
+                    self.W2[e] = self.W_dev["W2q"][e].cpu()
+                    self.S1[e] = self.W_dev["W1s"][e].cpu()
+                    self.S2[e] = self.W_dev["W2s"][e].cpu()
+                else:
+                    self.W1[e] = self.W_dev["W1"][e].cpu()
+                    self.W2[e] = self.W_dev["W2"][e].cpu()
+        extra = dict(W1s=self.S1, W2s=self.S2) if self.fp8 else {}
+        O = self.oracle.OracleLayer(W1=self.W1, W2=self.W2, **extra, **self.base)
         t0 = time.perf_counter()
         O.layer(self.x, tokens=tokens)
         return time.perf_counter() - t0
@@ -221,9 +229,12 @@ def dist_env():
 
 def workload_config(w: workloads.Workload, n_gpus: int):
     c = costmodel.layer_counts(T=w.T, d=w.d, l=w.l, N=w.N, k=w.k, m=w.m, act=w.act,
-                               shared_m=w.shared_m, skip_proj=w.skip_proj)
+                               shared_m=w.shared_m, skip_proj=w.skip_proj,
+                               expert_bytes=1 if w.expert_fp8 else None)
     return {"workload": w.name, "T": w.T, "d": w.d, "l": w.l, "N": w.N, "k": w.k, "m": w.m,
             "act": w.act, "shared_m": w.shared_m, "skip_proj": w.skip_proj, "bias": w.bias,
+            "expert_weights": ("e4m3 codes, fp32 scale per output channel (widened to bf16 "
+                               "in the expert kernels)") if w.expert_fp8 else w.dtype,
             "global_batch": w.T * n_gpus, "parallelism": f"replicas{n_gpus}",
             "l2": f"inputs larger than L2: {c.expert_weight_bytes / 1e9:.2f} GB of expert "
                   "weights streamed from HBM every step"}
@@ -285,8 +296,11 @@ def run_ours(args):
     xw = w if rank == 0 else workloads.Workload(**{**w.__dict__, "seed": w.seed + 1000 * rank})
     x = workloads.make_x(xw, device=dev)
     L = lmoe.LatentMoELayer(w.d, w.l, w.N, w.k, w.m, act=w.act, shared_m=w.shared_m,
-                            dtype=w.dtype, skip_proj=w.skip_proj, flags=args.lib_flags)
+                            dtype=w.dtype, skip_proj=w.skip_proj,
+                            flags=args.lib_flags | (lmoe.EXPERTS_FP8 if w.expert_fp8 else 0))
     L.set_weights(W["Wg"], W["bias"], W["Wdown"], W["Wup"], W["W1"], W["W2"], W["Ws1"], W["Ws2"])
+    if w.expert_fp8:
+        L.set_expert_weights_fp8(W["W1q"], W["W1s"], W["W2q"], W["W2s"])
     L.reserve(w.T)
     out = torch.empty_like(x)
     stream = torch.cuda.current_stream()
@@ -358,7 +372,8 @@ def run_ours(args):
     stage_ms = {k: statistics.fmean(p[k] for p in prof) for k in prof[0]} if prof else {}
     counts = costmodel.stage_counts(T=w.T, d=w.d, l=w.l, N=w.N, k=w.k, m=w.m, act=w.act,
                                     shared_m=w.shared_m, skip_proj=w.skip_proj,
-                                    elem_bytes=4 if w.dtype == "f32" else 2, loads=loads)
+                                    elem_bytes=4 if w.dtype == "f32" else 2, loads=loads,
+                                    expert_bytes=1 if w.expert_fp8 else None)
     peaks, peak_src = load_peaks()
     roofline = None
     if stage_ms:
@@ -377,7 +392,8 @@ def run_ours(args):
                     f"({'hbm_gbs' if bound == 'hbm' else 'bf16_tflops_sustained'})",
                     "stage_ms": {k: round(v, 5) for k, v in stage_ms.items()}}
         lc = costmodel.layer_counts(T=w.T, d=w.d, l=w.l, N=w.N, k=w.k, m=w.m, act=w.act,
-                                    shared_m=w.shared_m, skip_proj=w.skip_proj, loads=loads)
+                                    shared_m=w.shared_m, skip_proj=w.skip_proj, loads=loads,
+                                    expert_bytes=1 if w.expert_fp8 else None)
         roofline["layer"] = {"alg_bytes": lc.bytes, "alg_flops": lc.flops,
                              "hbm_frac": lc.bytes / (ms_per_step / 1e3) / 1e9 / peaks["hbm_gbs"],
                              "touched_experts": lc.touched,

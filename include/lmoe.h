@@ -93,6 +93,12 @@ typedef enum { LMOE_F32 = 0, LMOE_BF16 = 1 } lmoe_dtype;
                                     the logits stage then exclude the bias,
                                     and lmoe_route_only adds the bias given to
                                     lmoe_set_weights for the choice          */
+#define LMOE_EXPERTS_FP8        0x200u /* expert weights W1 and W2 as fp8 E4M3
+                                    codes with one fp32 scale per output
+                                    channel (lmoe_set_expert_weights_fp8);
+                                    activations stay bf16 and accumulation
+                                    fp32.  bf16 layers with l and m multiples
+                                    of 64 only (else LMOE_ERR_UNSUPPORTED)   */
 
 /* Limits of this build. */
 #define LMOE_MAX_EXPERTS 1024
@@ -138,6 +144,25 @@ lmoe_status lmoe_create(int d, int l, int N, int k, int m, lmoe_act act, int sha
 lmoe_status lmoe_set_weights(lmoe_layer* h, const void* W_g, const float* bias,
                              const void* W_down, const void* W_up, const void* W1,
                              const void* W2, const void* Ws1, const void* Ws2);
+
+/*
+ * lmoe_set_expert_weights_fp8 -- the expert weights of a layer created with
+ * LMOE_EXPERTS_FP8 (low-precision expert weights: the paper's Section 2 models
+ * FP4 expert weights, its Section 4.3 measures FP8 quantisation).  Device
+ * pointers, API layout [in, out] as lmoe_set_weights:
+ *   W1q [N, l, m_in] E4M3 codes (one byte each, the OCP E4M3FN encoding),
+ *   W1s [N, m_in] fp32: W1[e][i][o] = value(W1q[e][i][o]) * W1s[e][o],
+ *   W2q [N, m, l]    E4M3 codes,
+ *   W2s [N, l] fp32: W2[e][i][o] = value(W2q[e][i][o]) * W2s[e][o].
+ * The library copies (and repacks) them; the caller keeps ownership of its
+ * buffers.  lmoe_set_weights is still required for the other weights (its W1
+ * and W2 may then be NULL); the layer is ready once both calls succeeded.
+ * Codes are widened to bf16 exactly inside the expert kernels and the scale
+ * multiplies the fp32 accumulator.  Synchronous.  Errors: INVALID_ARG (NULL
+ * pointer, layer created without LMOE_EXPERTS_FP8), CUDA, OOM.
+ */
+lmoe_status lmoe_set_expert_weights_fp8(lmoe_layer* h, const void* W1q, const float* W1s,
+                                        const void* W2q, const float* W2s);
 
 /*
  * lmoe_reserve -- size the workspace for up to max_T tokens per call.

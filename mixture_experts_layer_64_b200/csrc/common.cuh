@@ -69,6 +69,8 @@ struct GemmProblem {
                           // (the output map is the kernel's third tensor map)
   int splits;             // dense, single-CTA token-tiled: > 1 splits K into ranges of
   int kb_per_split;       // kb_per_split 64-wide blocks, each written as an fp32 slice
+  const float* w_scale;   // fp8 weights (B holds E4M3 codes): scale of weight row
+                          // g * w_group_stride + f, applied to the accumulator
   int* err;               // device error word
 };
 

@@ -76,6 +76,13 @@ struct lmoe_layer {
   void* Ws1_t = nullptr;  // [ms_in, d]
   void* W1_t = nullptr;   // [N * m_in, l]
   void* W2_t = nullptr;   // [N * l, m]
+  // fp8 expert weights (LMOE_EXPERTS_FP8): E4M3 codes in the same K-major
+  // layouts, and one fp32 scale per weight row (output channel)
+  uint8_t* W1q_t = nullptr;  // [N * m_in, l]
+  uint8_t* W2q_t = nullptr;  // [N * l, m]
+  float* W1s = nullptr;      // [N * m_in]
+  float* W2s = nullptr;      // [N * l]
+  bool fp8_set = false;
   // workspace
   int max_T = 0, W = 0;
   float* logits = nullptr;
@@ -176,6 +183,20 @@ bool encode_map(CUtensorMap* map, const void* ptr, long rows, int cols, long ld,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// fp8 E4M3 weights: rows of `cols` one-byte codes, 64-code (64-byte) boxes of
+// box_rows rows, no swizzle (the converter warps re-lay them out as bf16).
+bool encode_map_u8(CUtensorMap* map, const void* ptr, long rows, int cols, long ld, int box_rows) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)ld};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Output map of the TMA-store epilogue: 32 x 32 boxes, 64-byte swizzle for
 // bf16 (64-byte rows), 128-byte swizzle for fp32 (128-byte rows).
 bool encode_out_map(CUtensorMap* map, const GemmCall& c) {
@@ -222,7 +243,8 @@ lmoe_status launch_tc(lmoe_layer* h, const GemmCall& c, cudaStream_t st) {
     h->detail = "cuTensorMapEncodeTiled (activations) failed";
     return LMOE_ERR_CUDA;
   }
-  if (!encode_map(&tb, c.p.B, c.b_rows, c.p.K, c.p.K, Cfg::W_ROWS)) {
+  if (!(Cfg::kFp8 ? encode_map_u8(&tb, c.p.B, c.b_rows, c.p.K, c.p.K, Cfg::W_ROWS)
+                  : encode_map(&tb, c.p.B, c.b_rows, c.p.K, c.p.K, Cfg::W_ROWS))) {
     h->detail = "cuTensorMapEncodeTiled (weights) failed";
     return LMOE_ERR_CUDA;
   }
@@ -233,7 +255,7 @@ lmoe_status launch_tc(lmoe_layer* h, const GemmCall& c, cudaStream_t st) {
   const long NT = (c.p.F + Cfg::FT - 1) / Cfg::FT;
   const long tiles = (long)c.p.max_row_tiles * NT * std::max(1, c.p.splits);
   const int grid = (int)std::max(1L, std::min<long>(h->num_sms, tiles));
-  tc_gemm_kernel<Cfg><<<grid, kTcThreads, Cfg::SMEM_BYTES, st>>>(ta, tb, tc, p);
+  tc_gemm_kernel<Cfg><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, st>>>(ta, tb, tc, p);
   LMOE_CHECK_LAUNCH(h);
   return LMOE_OK;
 }
@@ -427,6 +449,27 @@ lmoe_status run_split(lmoe_layer* h, const GemmCall& c, int S, int kbs, cudaStre
 
 lmoe_status run_gemm(lmoe_layer* h, GemmCall c, cudaStream_t st, int* path = nullptr) {
   c.p.err = h->err;
+  if (c.p.w_scale) {
+    // fp8 expert weights: the single-CTA tensor-core kernel with the E4M3
+    // widening warps (weight-stationary or token-tiled)
+    if (!tc_eligible(h, c) || c.pair) {
+      h->detail = "fp8 expert weights need the single-CTA tensor-core kernel";
+      return LMOE_ERR_UNSUPPORTED;
+    }
+    const bool dual = c.p.dual_offset > 0;
+    if (path) *path = c.swap ? 2 : 1;
+    if (c.kind == GK_FC1) {
+      if (c.swap)
+        return dual ? launch_tc<TcCfg<true, true, true, 128, EPI_ACT, true>>(h, c, st)
+                    : launch_tc<TcCfg<true, true, false, 128, EPI_ACT, true>>(h, c, st);
+      return dual ? launch_tc<TcCfg<false, true, true, 128, EPI_ACT, true>>(h, c, st)
+                  : launch_tc<TcCfg<false, true, false, 256, EPI_ACT, true>>(h, c, st);
+    }
+    if (c.kind == GK_FC2)
+      return c.swap ? launch_tc<TcCfg<true, false, false, 128, EPI_SCALE_ROWS, true>>(h, c, st)
+                    : launch_tc<TcCfg<false, false, false, 256, EPI_SCALE_ROWS, true>>(h, c, st);
+    return LMOE_ERR_INVALID_ARG;
+  }
   if (c.pair && c.p.gather != nullptr) {
     // the pair kernels read activations with TMA only
     c.pair = false;
@@ -648,9 +691,12 @@ lmoe_status run_forward(lmoe_layer* h, const void* x, void* out, int T, cudaStre
   prof_mark(h, st, 5);
   {
     const void* A = skip ? x : h->z;
-    GemmCall c = grouped_call(h, GK_FC1, T, A, skip ? d : l, T, h->row_tok, h->W1_t, h->m_in, m, l);
+    const bool fp8 = (h->flags & LMOE_EXPERTS_FP8) != 0;
+    GemmCall c = grouped_call(h, GK_FC1, T, A, skip ? d : l, T, h->row_tok,
+                              fp8 ? (const void*)h->W1q_t : h->W1_t, h->m_in, m, l);
+    c.p.w_scale = fp8 ? h->W1s : nullptr;
     c.swap = swap;
-    c.ws_pair = ws_pair;
+    c.ws_pair = ws_pair && !fp8;
     c.p.dual_offset = h->act == LMOE_ACT_SWIGLU ? m : 0;
     c.p.epi.out = h->h;
     c.p.epi.ldo = m;
@@ -661,10 +707,13 @@ lmoe_status run_forward(lmoe_layer* h, const void* x, void* out, int T, cudaStre
   }
   prof_mark(h, st, 6);
   {
-    GemmCall c = grouped_call(h, GK_FC2, T, h->h, m, R, nullptr, h->W2_t, l, l, m);
-    if (pair_fc2 && !ws_pair) make_pair(h, c);
+    const bool fp8 = (h->flags & LMOE_EXPERTS_FP8) != 0;
+    GemmCall c = grouped_call(h, GK_FC2, T, h->h, m, R, nullptr,
+                              fp8 ? (const void*)h->W2q_t : h->W2_t, l, l, m);
+    c.p.w_scale = fp8 ? h->W2s : nullptr;
+    if (pair_fc2 && !ws_pair && !fp8) make_pair(h, c);  // the pair kernels read bf16 weights
     c.swap = swap;
-    c.ws_pair = ws_pair;
+    c.ws_pair = ws_pair && !fp8;
     c.p.epi.out = h->ys;
     c.p.epi.ldo = l;
     c.p.epi.row_w = h->row_w;
@@ -771,6 +820,11 @@ void free_weights(lmoe_layer* h) {
   free_ptr(h->Wu_t);
   free_ptr(h->Ws1_t);
   free_ptr(h->W1_t);
+  free_ptr(h->W1q_t);
+  free_ptr(h->W2q_t);
+  free_ptr(h->W1s);
+  free_ptr(h->W2s);
+  h->fp8_set = false;
   free_ptr(h->W2_t);
   h->weights_set = false;
 }
@@ -797,6 +851,11 @@ lmoe_status repack(lmoe_layer* h, const void* in, int rows, int cols, int batch,
 }
 
 bool valid_stream_call(const lmoe_layer* h, int T) { return h && T >= 0 && T <= h->max_T; }
+
+// Weights in place: lmoe_set_weights, and with fp8 experts their codes too.
+bool layer_ready(const lmoe_layer* h) {
+  return h->weights_set && (!(h->flags & LMOE_EXPERTS_FP8) || h->fp8_set);
+}
 
 }  // namespace
 
@@ -830,13 +889,18 @@ lmoe_status lmoe_create(int d, int l, int N, int k, int m, lmoe_act act, int sha
   *out = nullptr;
   const unsigned known = LMOE_SKIP_PROJ | LMOE_DEBUG_CHECKS | LMOE_FORCE_SIMT | LMOE_FORCE_SWAP |
                          LMOE_FORCE_NOSWAP | LMOE_FORCE_NOPAIR | LMOE_FORCE_WS_PAIR |
-                         LMOE_ROUTE_FULL_SOFTMAX | LMOE_ROUTE_BIAS_SELECT;
+                         LMOE_ROUTE_FULL_SOFTMAX | LMOE_ROUTE_BIAS_SELECT | LMOE_EXPERTS_FP8;
   if (d <= 0 || l <= 0 || N <= 0 || k <= 0 || m <= 0 || shared_m < 0) return LMOE_ERR_INVALID_ARG;
   if (k > N || (flags & ~known)) return LMOE_ERR_INVALID_ARG;
   if (act != LMOE_ACT_SILU && act != LMOE_ACT_SWIGLU && act != LMOE_ACT_RELU2) return LMOE_ERR_INVALID_ARG;
   if (dtype != LMOE_F32 && dtype != LMOE_BF16) return LMOE_ERR_INVALID_ARG;
   if ((flags & LMOE_SKIP_PROJ) && l != d) return LMOE_ERR_INVALID_ARG;
   if ((flags & LMOE_FORCE_SWAP) && (flags & LMOE_FORCE_NOSWAP)) return LMOE_ERR_INVALID_ARG;
+  // fp8 expert weights run on the tensor-core kernels only: bf16 layers whose
+  // expert GEMMs have K (l and m) a multiple of 64
+  if ((flags & LMOE_EXPERTS_FP8) &&
+      (dtype != LMOE_BF16 || (flags & LMOE_FORCE_SIMT) || l % 64 != 0 || m % 64 != 0))
+    return LMOE_ERR_UNSUPPORTED;
   if (N > LMOE_MAX_EXPERTS || k > LMOE_MAX_TOPK) return LMOE_ERR_UNSUPPORTED;
   // 32-bit row and element indices inside the kernels
   if ((long)N * (2L * m) * l >= (1L << 31) * 8L) return LMOE_ERR_UNSUPPORTED;
@@ -865,7 +929,8 @@ lmoe_status lmoe_create(int d, int l, int N, int k, int m, lmoe_act act, int sha
 lmoe_status lmoe_set_weights(lmoe_layer* h, const void* W_g, const float* bias, const void* W_down,
                              const void* W_up, const void* W1, const void* W2, const void* Ws1,
                              const void* Ws2) {
-  if (!h || !W_g || !W1 || !W2) return LMOE_ERR_INVALID_ARG;
+  const bool fp8 = h && (h->flags & LMOE_EXPERTS_FP8);
+  if (!h || !W_g || (!fp8 && (!W1 || !W2))) return LMOE_ERR_INVALID_ARG;
   const bool skip = (h->flags & LMOE_SKIP_PROJ) != 0;
   if (skip != (W_down == nullptr) || skip != (W_up == nullptr)) return LMOE_ERR_INVALID_ARG;
   if ((h->shared_m > 0) != (Ws1 != nullptr) || (h->shared_m > 0) != (Ws2 != nullptr))
@@ -876,8 +941,10 @@ lmoe_status lmoe_set_weights(lmoe_layer* h, const void* W_g, const float* bias, 
   const int d = h->d, l = h->l, N = h->N, m = h->m;
   if (!h->weights_set) {
     LMOE_CUDA(h, cudaMalloc(&h->Wg_t, (size_t)N * d * es));
-    LMOE_CUDA(h, cudaMalloc(&h->W1_t, (size_t)N * h->m_in * l * es));
-    LMOE_CUDA(h, cudaMalloc(&h->W2_t, (size_t)N * l * m * es));
+    if (!fp8) {
+      LMOE_CUDA(h, cudaMalloc(&h->W1_t, (size_t)N * h->m_in * l * es));
+      LMOE_CUDA(h, cudaMalloc(&h->W2_t, (size_t)N * l * m * es));
+    }
     if (!skip) LMOE_CUDA(h, cudaMalloc(&h->Wd_t, (size_t)l * d * es));
     if (h->Kup > 0) LMOE_CUDA(h, cudaMalloc(&h->Wu_t, (size_t)d * h->Kup * es));
     if (h->shared_m > 0) LMOE_CUDA(h, cudaMalloc(&h->Ws1_t, (size_t)h->ms_in * d * es));
@@ -888,8 +955,10 @@ lmoe_status lmoe_set_weights(lmoe_layer* h, const void* W_g, const float* bias, 
     LMOE_CUDA(h, cudaMemcpy(h->bias, bias, (size_t)N * sizeof(float), cudaMemcpyDeviceToDevice));
   }
   LMOE_TRY(repack(h, W_g, d, N, 1, h->Wg_t, d, 0));
-  LMOE_TRY(repack(h, W1, l, h->m_in, N, h->W1_t, l, 0));
-  LMOE_TRY(repack(h, W2, m, l, N, h->W2_t, m, 0));
+  if (!fp8) {
+    LMOE_TRY(repack(h, W1, l, h->m_in, N, h->W1_t, l, 0));
+    LMOE_TRY(repack(h, W2, m, l, N, h->W2_t, m, 0));
+  }
   if (!skip) {
     LMOE_TRY(repack(h, W_down, d, l, 1, h->Wd_t, d, 0));
     LMOE_TRY(repack(h, W_up, l, d, 1, h->Wu_t, h->Kup, 0));
@@ -902,6 +971,39 @@ lmoe_status lmoe_set_weights(lmoe_layer* h, const void* W_g, const float* bias, 
   }
   LMOE_CUDA(h, cudaDeviceSynchronize());
   h->weights_set = true;
+  return LMOE_OK;
+}
+
+lmoe_status lmoe_set_expert_weights_fp8(lmoe_layer* h, const void* W1q, const float* W1s,
+                                        const void* W2q, const float* W2s) {
+  if (!h || !W1q || !W1s || !W2q || !W2s) return LMOE_ERR_INVALID_ARG;
+  if (!(h->flags & LMOE_EXPERTS_FP8)) return LMOE_ERR_INVALID_ARG;
+  DevGuard g(h->device);
+  LMOE_CUDA(h, cudaDeviceSynchronize());
+  const int l = h->l, N = h->N, m = h->m, m_in = h->m_in;
+  if (!h->fp8_set) {
+    LMOE_CUDA(h, cudaMalloc(&h->W1q_t, (size_t)N * m_in * l));
+    LMOE_CUDA(h, cudaMalloc(&h->W2q_t, (size_t)N * l * m));
+    LMOE_CUDA(h, cudaMalloc(&h->W1s, (size_t)N * m_in * sizeof(float)));
+    LMOE_CUDA(h, cudaMalloc(&h->W2s, (size_t)N * l * sizeof(float)));
+  }
+  // codes [N][in][out] -> K-major [N][out][in], as the bf16 stacks
+  {
+    dim3 grid((m_in + 31) / 32, (l + 31) / 32, N), block(32, 8);
+    transpose_kernel<uint8_t><<<grid, block>>>(static_cast<const uint8_t*>(W1q), l, m_in,
+                                               (long)l * m_in, h->W1q_t, l, 0, (long)m_in * l);
+    LMOE_CUDA(h, cudaGetLastError());
+  }
+  {
+    dim3 grid((l + 31) / 32, (m + 31) / 32, N), block(32, 8);
+    transpose_kernel<uint8_t><<<grid, block>>>(static_cast<const uint8_t*>(W2q), m, l,
+                                               (long)m * l, h->W2q_t, m, 0, (long)l * m);
+    LMOE_CUDA(h, cudaGetLastError());
+  }
+  LMOE_CUDA(h, cudaMemcpy(h->W1s, W1s, (size_t)N * m_in * sizeof(float), cudaMemcpyDeviceToDevice));
+  LMOE_CUDA(h, cudaMemcpy(h->W2s, W2s, (size_t)N * l * sizeof(float), cudaMemcpyDeviceToDevice));
+  LMOE_CUDA(h, cudaDeviceSynchronize());
+  h->fp8_set = true;
   return LMOE_OK;
 }
 
@@ -962,7 +1064,7 @@ lmoe_status lmoe_reserve(lmoe_layer* h, int max_T) {
 
 lmoe_status lmoe_forward(lmoe_layer* h, const void* x, void* out, int T, lmoe_stream_t stream) {
   if (!h) return LMOE_ERR_INVALID_ARG;
-  if (!h->weights_set || h->max_T == 0) return LMOE_ERR_NOT_READY;
+  if (!layer_ready(h) || h->max_T == 0) return LMOE_ERR_NOT_READY;
   if (!valid_stream_call(h, T)) return LMOE_ERR_INVALID_ARG;
   if (T == 0) return LMOE_OK;
   if (!x || !out || x == out) return LMOE_ERR_INVALID_ARG;
@@ -973,7 +1075,7 @@ lmoe_status lmoe_forward(lmoe_layer* h, const void* x, void* out, int T, lmoe_st
 lmoe_status lmoe_forward_host(lmoe_layer* h, const void* x_host, void* out_host, int T,
                               lmoe_stream_t stream) {
   if (!h) return LMOE_ERR_INVALID_ARG;
-  if (!h->weights_set || h->max_T == 0) return LMOE_ERR_NOT_READY;
+  if (!layer_ready(h) || h->max_T == 0) return LMOE_ERR_NOT_READY;
   if (!valid_stream_call(h, T)) return LMOE_ERR_INVALID_ARG;
   if (T == 0) return LMOE_OK;
   if (!x_host || !out_host) return LMOE_ERR_INVALID_ARG;
@@ -1019,7 +1121,7 @@ lmoe_status lmoe_route_only(lmoe_layer* h, const float* logits, int T, int* idx,
 lmoe_status lmoe_router_logits(lmoe_layer* h, const void* x, float* logits, int T,
                                lmoe_stream_t stream) {
   if (!h) return LMOE_ERR_INVALID_ARG;
-  if (!h->weights_set || h->max_T == 0) return LMOE_ERR_NOT_READY;
+  if (!layer_ready(h) || h->max_T == 0) return LMOE_ERR_NOT_READY;
   if (!valid_stream_call(h, T)) return LMOE_ERR_INVALID_ARG;
   if (T == 0) return LMOE_OK;
   if (!x || !logits) return LMOE_ERR_INVALID_ARG;

@@ -19,7 +19,7 @@
 // same feature tile and accumulates them into two TMEM accumulators, so the
 // epilogue sees both halves of a feature in one thread.
 //
-// Warp roles (384 threads):
+// Warp roles (384 threads; 512 with fp8 weights):
 //   warp 0      TMA producer (weights, and contiguous activation rows)
 //   warp 1      TMEM allocation and the single-thread MMA issuer
 //   warps 2-3   cp.async row gather of activations (gathered problems),
@@ -27,6 +27,10 @@
 //   warps 4-11  epilogue, two warpgroups taking alternate 32-column chunks:
 //               tcgen05.ld -> epilogue math -> shared-memory staging -> TMA
 //               bulk stores (plain stores for partly covered row blocks)
+// With fp8 E4M3 weights (512 threads) the epilogue is one warpgroup (warps
+// 4-7) and warps 8-15 widen each stage's E4M3 weight tiles to bf16 in shared
+// memory before the MMA issuer may use the stage; the per-output-channel
+// scales multiply the fp32 accumulators in the epilogue.
 // The smem ring has STAGES stages of one 64-wide K slice each; TMEM holds two
 // accumulator buffers so the epilogue of tile i overlaps the MMAs of tile i+1.
 #pragma once
@@ -40,20 +44,27 @@ constexpr int kEpiWarps = 8;  // two warpgroups; each warp reads its TMEM lane q
 constexpr int kTcSmemBudget = 200 * 1024;
 constexpr int kGatherThreads = 64;
 
-template <bool kSwap_, bool kGather_, bool kDual_, int kWN_, int kEpi_>
+template <bool kSwap_, bool kGather_, bool kDual_, int kWN_, int kEpi_, bool kFp8_ = false>
 struct TcCfg {
-  static constexpr bool kSwap = kSwap_, kGather = kGather_, kDual = kDual_;
+  static constexpr bool kSwap = kSwap_, kGather = kGather_, kDual = kDual_, kFp8 = kFp8_;
   static constexpr int kEpi = kEpi_;
+  // warps 0-3: producer, MMA issuer, gather; then the epilogue warps (two
+  // warpgroups, or one with fp8 weights), then (fp8) the converter warps that
+  // widen the E4M3 weight tiles to bf16
+  static constexpr int EPI_WARPS = kFp8 ? 4 : kEpiWarps;
+  static constexpr int CONV_THREADS = kFp8 ? 256 : 0;
+  static constexpr int THREADS = 128 + 32 * EPI_WARPS + CONV_THREADS;
   static constexpr int BK = 64;                       // bf16 per 128-byte swizzled row
   static constexpr int ACT_ROWS = 128;
   static constexpr int W_ROWS = kSwap ? 128 : (kDual ? 128 : kWN_);
   static constexpr int NUM_W = kDual ? 2 : 1;
   static constexpr int ACT_BYTES = ACT_ROWS * BK * 2;
   static constexpr int W_BYTES = W_ROWS * BK * 2;
-  static constexpr int STAGE_BYTES = ACT_BYTES + NUM_W * W_BYTES;
+  static constexpr int W8_BYTES = kFp8 ? W_ROWS * BK : 0;  // one fp8 weight tile (64-byte rows)
+  static constexpr int STAGE_BYTES = ACT_BYTES + NUM_W * (W_BYTES + W8_BYTES);
   // epilogue staging: one 32 x 32 box per epilogue warp (bf16 or fp32)
   static constexpr int STG_WARP = kEpi == EPI_F32_BIAS ? 4096 : 2048;
-  static constexpr int STG_BYTES = kSwap ? 0 : kEpiWarps * STG_WARP;
+  static constexpr int STG_BYTES = kSwap ? 0 : EPI_WARPS * STG_WARP;
   static constexpr int STAGES_RAW = (kTcSmemBudget + kEpiWarps * 2048 - STG_BYTES) / STAGE_BYTES;
   static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
   static constexpr int ACC_N = kSwap ? 128 : W_ROWS;  // fp32 columns of one accumulator
@@ -68,7 +79,53 @@ struct TcCfg {
   static_assert(STAGES >= 3, "pipeline too shallow");
   static_assert(!kSwap || kEpi == EPI_ACT || kEpi == EPI_SCALE_ROWS, "swap epilogues");
   static_assert(kWN_ == 128 || kWN_ == 256, "weight tile");
+  static_assert(!kFp8 || kEpi == EPI_ACT || kEpi == EPI_SCALE_ROWS, "fp8 weights: expert GEMMs");
 };
+
+// ---- fp8 E4M3 weights -----------------------------------------------------------
+
+// Four E4M3 codes (byte 0 first) -> four bf16 with the same values, as two
+// bf16x2 words.  Every step is an exact hardware conversion: E4M3 pairs to
+// f16 pairs (every E4M3 value, subnormals included, is a normal f16 or
+// zero), f16 to f32, and f32 pairs to bf16 pairs (4 significant bits fit).
+__device__ __forceinline__ void e4m3x4_to_bf16x4(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  asm("{\n\t.reg .b16 l, h, a0, a1, a2, a3;\n\t.reg .b32 fl, fh;\n\t"
+      ".reg .f32 f0, f1, f2, f3;\n\t"
+      "mov.b32 {l, h}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 fl, l;\n\t"
+      "cvt.rn.f16x2.e4m3x2 fh, h;\n\t"
+      "mov.b32 {a0, a1}, fl;\n\t"
+      "mov.b32 {a2, a3}, fh;\n\t"
+      "cvt.f32.f16 f0, a0;\n\tcvt.f32.f16 f1, a1;\n\t"
+      "cvt.f32.f16 f2, a2;\n\tcvt.f32.f16 f3, a3;\n\t"
+      "cvt.rn.bf16x2.f32 %0, f1, f0;\n\t"
+      "cvt.rn.bf16x2.f32 %1, f3, f2;\n\t}"
+      : "=r"(lo), "=r"(hi)
+      : "r"(w));
+}
+
+// Widens one weight tile: W_ROWS rows of 64 E4M3 codes (64-byte rows, no
+// swizzle, as TMA stored them) into W_ROWS rows of 64 bf16 in the 128-byte
+// swizzled K-major layout the MMA reads.  ct = this thread's index among the
+// nconv converter threads; chunk c = (row, 16-byte quarter q) is handled by
+// thread c mod nconv.
+template <int W_ROWS, int kConv>
+__device__ __forceinline__ void widen_fp8_tile(const uint8_t* src, uint8_t* dst, int ct) {
+#pragma unroll
+  for (int c = ct; c < W_ROWS * 4; c += kConv) {
+    const int r = c >> 2, q = c & 3;
+    const uint4 v = *reinterpret_cast<const uint4*>(src + r * 64 + q * 16);
+    const uint32_t in[4] = {v.x, v.y, v.z, v.w};
+    uint32_t out[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) e4m3x4_to_bf16x4(in[i], out[2 * i], out[2 * i + 1]);
+    uint8_t* row = dst + r * 128;
+    const int sw = r & 7;
+    *reinterpret_cast<uint4*>(row + (((2 * q) ^ sw) << 4)) = make_uint4(out[0], out[1], out[2], out[3]);
+    *reinterpret_cast<uint4*>(row + (((2 * q + 1) ^ sw) << 4)) =
+        make_uint4(out[4], out[5], out[6], out[7]);
+  }
+}
 
 // ---- epilogue stores ----------------------------------------------------------
 
@@ -303,7 +360,7 @@ __device__ __forceinline__ int total_row_tiles_s(const GemmProblem& p, const int
 // ---- the kernel -----------------------------------------------------------------
 
 template <class Cfg>
-__global__ void __launch_bounds__(kTcThreads, 1)
+__global__ void __launch_bounds__(Cfg::THREADS, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmC, const GemmProblem p) {
   extern __shared__ uint8_t smem_raw[];
@@ -312,12 +369,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint8_t* stg_base = smem + Cfg::STAGES * Cfg::STAGE_BYTES;  // epilogue staging (1024-aligned)
   uint64_t* full = reinterpret_cast<uint64_t*>(stg_base + Cfg::STG_BYTES);
   uint64_t* empty = full + Cfg::STAGES;
-  uint64_t* tfull = empty + Cfg::STAGES;
+  uint64_t* wfull = empty + Cfg::STAGES;  // fp8 weights: the E4M3 tiles have landed
+  uint64_t* tfull = wfull + Cfg::STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* s_tiles = reinterpret_cast<int*>(stg_base + Cfg::STG_BYTES + 512);
+  static_assert(3 * Cfg::STAGES * 8 + 5 * 8 + 8 <= 512, "barrier area");
+  constexpr int W8_OFF = Cfg::ACT_BYTES + Cfg::NUM_W * Cfg::W_BYTES;  // fp8 tiles in a stage
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   load_tile_tables(p, s_tiles);
@@ -326,12 +386,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < Cfg::STAGES; ++s) {
-      mbar_init(&full[s], Cfg::kGather ? 1 + kGatherThreads : 1);
+      // producer + gather threads + (fp8) the converters, after widening
+      mbar_init(&full[s], 1 + (Cfg::kGather ? kGatherThreads : 0) + Cfg::CONV_THREADS);
       mbar_init(&empty[s], 1);
+      mbar_init(&wfull[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], kEpiWarps);
+      mbar_init(&tempty[b], Cfg::EPI_WARPS);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -370,7 +432,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         locate_row_tile_s(p, s_tiles, rt, g, row0, rows);
         const int wrow = (int)(g * p.w_group_stride) + ft * Cfg::FT;
         const int nsub = Cfg::kSwap ? (rows + 31) / 32 : 4;
-        uint32_t bytes = Cfg::NUM_W * Cfg::W_BYTES;
+        uint32_t bytes = Cfg::kFp8 ? 0u : (uint32_t)(Cfg::NUM_W * Cfg::W_BYTES);
         if (!Cfg::kGather) bytes += Cfg::kSwap ? nsub * 4096 : Cfg::ACT_BYTES;
         bool ok = true;
         for (int kb = kb0; kb < kb1; ++kb) {
@@ -378,10 +440,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           uint8_t* st = smem + s * Cfg::STAGE_BYTES;
           mbar_arrive_expect_tx(&full[s], bytes);
           ++armed;
-          tma_load_2d(&tmB, &full[s], st + Cfg::ACT_BYTES, kb * Cfg::BK, wrow);
-          if (Cfg::kDual)
-            tma_load_2d(&tmB, &full[s], st + Cfg::ACT_BYTES + Cfg::W_BYTES, kb * Cfg::BK,
-                        wrow + p.dual_offset);
+          if (Cfg::kFp8) {
+            // E4M3 tiles into the staging area; the converter warps widen them
+            mbar_arrive_expect_tx(&wfull[s], Cfg::NUM_W * Cfg::W8_BYTES);
+            tma_load_2d(&tmB, &wfull[s], st + W8_OFF, kb * Cfg::BK, wrow);
+            if (Cfg::kDual)
+              tma_load_2d(&tmB, &wfull[s], st + W8_OFF + Cfg::W8_BYTES, kb * Cfg::BK,
+                          wrow + p.dual_offset);
+          } else {
+            tma_load_2d(&tmB, &full[s], st + Cfg::ACT_BYTES, kb * Cfg::BK, wrow);
+            if (Cfg::kDual)
+              tma_load_2d(&tmB, &full[s], st + Cfg::ACT_BYTES + Cfg::W_BYTES, kb * Cfg::BK,
+                          wrow + p.dual_offset);
+          }
           if (!Cfg::kGather) {
             if (Cfg::kSwap) {
               for (int sub = 0; sub < nsub; ++sub)
@@ -395,13 +466,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (!ok) break;
       }
       if (*abort_flag) {
-        // Let every armed load land before the block frees its shared memory.
+        // Let every armed load land before the block frees its shared memory
+        // (fp8: the weight tiles complete on wfull; full may then stay short
+        // of the converters' arrivals, which the bounded wait absorbs).
         int ss = s;
         uint32_t pp = ph;
         for (long i = 0; i < armed && i < Cfg::STAGES; ++i) {
           if (ss == 0) { ss = Cfg::STAGES; pp ^= 1; }
           --ss;
-          mbar_wait_drain(&full[ss], pp);
+          if (Cfg::kFp8) mbar_wait_drain(&wfull[ss], pp);
+          if (!Cfg::kFp8 || !Cfg::kGather) mbar_wait_drain(&full[ss], pp);
         }
       }
     }
@@ -504,10 +578,39 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
       cp_async_wait<0>();
     }
+  } else if (warp >= 4 + Cfg::EPI_WARPS) {
+    // ---------------- fp8 weights: widen E4M3 tiles to bf16 ----------------
+    // Same stage sequence as the producer; each stage's tiles are widened in
+    // place (staging area -> the bf16 weight slots) and handed to the MMA
+    // issuer with a fence (generic-proxy writes -> tensor-core reads) and an
+    // arrive on full.
+    if (Cfg::kFp8) {
+      const int ct = threadIdx.x - (128 + 32 * Cfg::EPI_WARPS);
+      int s = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+        const int ks = t / tiles_per_split;
+        const int kb0 = ks * KBS, kb1 = min(KB, kb0 + KBS);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait(&wfull[s], ph, abort_flag, p.err)) { ok = false; break; }
+          uint8_t* st = smem + s * Cfg::STAGE_BYTES;
+#pragma unroll
+          for (int i = 0; i < Cfg::NUM_W; ++i)
+            widen_fp8_tile<Cfg::W_ROWS, Cfg::CONV_THREADS>(st + W8_OFF + i * Cfg::W8_BYTES,
+                                                           st + Cfg::ACT_BYTES + i * Cfg::W_BYTES,
+                                                           ct);
+          fence_proxy_async_smem();
+          mbar_arrive(&full[s]);
+          if (++s == Cfg::STAGES) { s = 0; ph ^= 1; }
+        }
+      }
+    }
   } else {
     // ---------------- epilogue (warps 4..11: two warpgroups) ----------------
     const int qd = warp & 3;          // TMEM lane quarter this warp may access
     const int eg = (warp - 4) >> 2;   // warpgroup: even / odd 32-column chunks
+    constexpr int kChunkStride = 32 * (Cfg::EPI_WARPS / 4);  // columns between a warp's chunks
     int it = 0;
     for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++it) {
       const int ks = t / tiles_per_split, tl = t - ks * tiles_per_split;
@@ -527,11 +630,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const bool tma = p.tma_store && rows - qd * 32 >= 32;
         uint8_t* stg = stg_base + (warp - 4) * Cfg::STG_WARP;
         const int slice_rows = ks * p.M;  // split-K: the slice's rows in the output map
-        for (int c0 = 32 * eg; c0 < Cfg::ACC_N; c0 += 64) {
+        for (int c0 = 32 * eg; c0 < Cfg::ACC_N; c0 += kChunkStride) {
           tmem_ld_32x32(tb + c0, v0);
           if (Cfg::kDual) tmem_ld_32x32(tb + Cfg::ACC_N + c0, v1);
           tc_wait_ld();
           if (f0 + c0 < p.F) {
+            if (Cfg::kFp8) {  // per-output-channel scales of the fp8 weights
+              const float* sc = p.w_scale + (size_t)g * p.w_group_stride + f0 + c0;
+#pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                const bool in = f0 + c0 + i < p.F;
+                v0[i] *= in ? __ldg(sc + i) : 0.f;
+                if (Cfg::kDual) v1[i] *= in ? __ldg(sc + p.dual_offset + i) : 0.f;
+              }
+            }
             if (tma)
               epi_tma_chunk32<Cfg::kEpi, Cfg::kDual>(p, &tmC, stg, lane, slice_rows + row0 + qd * 32,
                                                      f0 + c0, v0, v1);
@@ -541,7 +653,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
       } else {
         const int f = f0 + qd * 32 + lane;
-        for (int c0 = 32 * eg; c0 < rows; c0 += 64) {
+        float s0 = 1.f, s1 = 1.f;  // fp8 weights: this thread's output channel scales
+        if (Cfg::kFp8 && f < p.F) {
+          const float* sc = p.w_scale + (size_t)g * p.w_group_stride + f;
+          s0 = __ldg(sc);
+          if (Cfg::kDual) s1 = __ldg(sc + p.dual_offset);
+        }
+        for (int c0 = 32 * eg; c0 < rows; c0 += kChunkStride) {
           tmem_ld_32x32(tb + c0, v0);
           if (Cfg::kDual) tmem_ld_32x32(tb + Cfg::ACC_N + c0, v1);
           tc_wait_ld();
@@ -550,7 +668,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
             for (int c = 0; c < 32; ++c)
               if (c < cn)
-                store_elem<Cfg::kEpi>(p, row0 + c0 + c, f, v0[c], Cfg::kDual ? v1[c] : 0.f);
+                store_elem<Cfg::kEpi>(p, row0 + c0 + c, f, v0[c] * s0,
+                                      Cfg::kDual ? v1[c] * s1 : 0.f);
           }
         }
       }

@@ -23,6 +23,7 @@ DTYPE = {"f32": 0, "bf16": 1}
 SKIP_PROJ, DEBUG_CHECKS, FORCE_SIMT, FORCE_SWAP, FORCE_NOSWAP, FORCE_NOPAIR, FORCE_WS_PAIR = (
     0x1, 0x2, 0x4, 0x8, 0x10, 0x20, 0x40)
 ROUTE_FULL_SOFTMAX, ROUTE_BIAS_SELECT = 0x80, 0x100
+EXPERTS_FP8 = 0x200
 MAX_EXPERTS, MAX_TOPK = 1024, 32
 DEVERR_WAIT_TIMEOUT, DEVERR_RANGE, DEVERR_NONFINITE = 0x1, 0x2, 0x4
 STAGES = {"logits": 0, "idx": 1, "w": 2, "offsets": 3, "perm": 4, "z": 5, "h": 6, "ys": 7, "comb": 8}
@@ -30,7 +31,8 @@ EXPORTS = ["lmoe_create", "lmoe_set_weights", "lmoe_reserve", "lmoe_forward", "l
            "lmoe_route_only", "lmoe_router_logits", "lmoe_stage_bytes", "lmoe_debug_dump",
            "lmoe_last_error", "lmoe_profile_begin", "lmoe_profile_end", "lmoe_stage_name",
            "lmoe_last_launch_count", "lmoe_last_expert_path", "lmoe_status_string",
-           "lmoe_error_detail", "lmoe_destroy", "lmoe_route_only_noalloc"]
+           "lmoe_error_detail", "lmoe_destroy", "lmoe_route_only_noalloc",
+           "lmoe_set_expert_weights_fp8"]
 NOALLOC_MAX_WORDS = 262144
 
 
@@ -57,6 +59,7 @@ def lib() -> ctypes.CDLL:
         sig = {
             "lmoe_create": ([I, I, I, I, I, I, I, I, U, ctypes.POINTER(P)], I),
             "lmoe_set_weights": ([P] * 9, I),
+            "lmoe_set_expert_weights_fp8": ([P] * 5, I),
             "lmoe_reserve": ([P, I], I),
             "lmoe_forward": ([P, P, P, I, P], I),
             "lmoe_forward_host": ([P, P, P, I, P], I),
@@ -191,6 +194,18 @@ class LatentMoELayer:
         self._check(lib().lmoe_set_weights(self._h, *[_ptr(ts[k]) for k in
                                                       ("Wg", "bias", "Wdown", "Wup", "W1", "W2",
                                                        "Ws1", "Ws2")]), "lmoe_set_weights")
+
+    def set_expert_weights_fp8(self, W1q, W1s, W2q, W2s):
+        """fp8 E4M3 expert weights (layer created with EXPERTS_FP8): uint8 codes
+        W1q [N, l, m_in], W2q [N, m, l] in the API layout and fp32 scales per
+        output channel W1s [N, m_in], W2s [N, l]."""
+        N, l, m = self.N, self.l, self.m
+        ts = [self._dev(W1q, (N, l, self.m_in), torch.uint8, "W1q"),
+              self._dev(W1s, (N, self.m_in), torch.float32, "W1s"),
+              self._dev(W2q, (N, m, l), torch.uint8, "W2q"),
+              self._dev(W2s, (N, l), torch.float32, "W2s")]
+        self._check(lib().lmoe_set_expert_weights_fp8(self._h, *[_ptr(t) for t in ts]),
+                    "lmoe_set_expert_weights_fp8")
 
     def reserve(self, max_T: int):
         self._check(lib().lmoe_reserve(self._h, max_T), "lmoe_reserve")

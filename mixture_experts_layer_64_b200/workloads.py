@@ -58,6 +58,7 @@ class Workload:
     skip_proj: bool = False      # l == d and the two projections are identities
     bias: Optional[str] = None   # None, "normal0.5" or "zipf1.1"
     seed: int = 0
+    expert_fp8: bool = False     # expert weights as E4M3 codes + per-channel scales
 
     @property
     def m_in(self) -> int:
@@ -94,6 +95,13 @@ WORKLOADS: Dict[str, Workload] = {
                                       d=7168, l=1792, N=896, k=16, m=1024,
                                       act="swiglu", bias="zipf1.1", seed=4),
 }
+# Low-precision expert weights (the paper's deployment lever at decode, where
+# the expert weights are the traffic): the two decode shapes with E4M3 expert
+# weights and per-channel scales, everything else as above.
+WORKLOADS["std-moe-decode-fp8"] = replace(WORKLOADS["std-moe-decode"], name="std-moe-decode-fp8",
+                                          expert_fp8=True)
+WORKLOADS["latent-decode-fp8"] = replace(WORKLOADS["latent-decode"], name="latent-decode-fp8",
+                                         expert_fp8=True)
 WORKLOAD_ORDER = list(WORKLOADS)
 
 
@@ -178,7 +186,18 @@ def make_weights(w: Workload, device="cpu", experts: bool = True) -> Dict[str, O
                                _TID["Wdown"], 0, device, dt)
         out["Wup"] = _normal((w.l, w.d), 1.0 / math.sqrt(w.l), w.seed,
                              _TID["Wup"], 0, device, dt)
-    if experts:
+    if experts and w.expert_fp8:
+        # the same bf16 draws, quantised per expert (W1q/W2q codes, W1s/W2s
+        # scales); W1/W2 stay None
+        W1q = torch.empty((w.N, w.l, w.m_in), dtype=torch.uint8, device=device)
+        W2q = torch.empty((w.N, w.m, w.l), dtype=torch.uint8, device=device)
+        W1s = torch.empty((w.N, w.m_in), dtype=torch.float32, device=device)
+        W2s = torch.empty((w.N, w.l), dtype=torch.float32, device=device)
+        for e in range(w.N):
+            W1q[e], W1s[e] = quantize_e4m3(make_expert_W1(w, e, device))
+            W2q[e], W2s[e] = quantize_e4m3(make_expert_W2(w, e, device))
+        out.update(W1=None, W2=None, W1q=W1q, W1s=W1s, W2q=W2q, W2s=W2s)
+    elif experts:
         W1 = torch.empty((w.N, w.l, w.m_in), dtype=dt, device=device)
         W2 = torch.empty((w.N, w.m, w.l), dtype=dt, device=device)
         for e in range(w.N):

@@ -228,6 +228,60 @@ def test_split_k_dense_gemms_at_decode_size(skip):
     assert torch.equal(a, b)
 
 
+# ---------------------------------------------------------------------------
+# fp8 E4M3 expert weights (codes + per-output-channel scales)
+# ---------------------------------------------------------------------------
+
+FP8 = {
+    "swiglu": W_("f8-swiglu", T=300, d=256, l=128, N=8, k=3, m=192, act="swiglu", seed=41,
+                 expert_fp8=True),
+    "relu2-shared": W_("f8-relu2", T=260, d=256, l=192, N=6, k=2, m=320, act="relu2",
+                       shared_m=320, bias="normal0.5", seed=42, expert_fp8=True),
+    "silu-skip": W_("f8-silu-skip", T=90, d=128, l=128, N=12, k=4, m=64, act="silu",
+                    skip_proj=True, seed=43, expert_fp8=True),
+}
+
+
+@pytest.mark.parametrize("name", list(FP8))
+@pytest.mark.parametrize("flags", [0, lmoe.FORCE_SWAP, lmoe.FORCE_NOSWAP])
+def test_fp8_experts(name, flags):
+    """E4M3 expert weights widened to bf16 inside the tensor-core kernels and
+    scaled per output channel in the epilogue, against the oracle reading
+    the same codes: weight-stationary (2, 2) and token-tiled (1, 1)."""
+    res = check_forward(FP8[name], flags=flags, fixture=True)
+    assert res["unique"] >= 0.9 * res["tokens"]
+    fc1, fc2 = paths(res)
+    assert fc1 == fc2 and fc1 in (1, 2)
+    if flags == lmoe.FORCE_SWAP:
+        assert fc1 == 2
+    if flags == lmoe.FORCE_NOSWAP:
+        assert fc1 == 1
+
+
+def test_fp8_expert_api_errors():
+    w = FP8["swiglu"]
+    with pytest.raises(lmoe.LmoeError):  # fp8 experts need a bf16 layer
+        lmoe.LatentMoELayer(w.d, w.l, w.N, w.k, w.m, act=w.act, dtype="f32",
+                            flags=lmoe.EXPERTS_FP8)
+    with pytest.raises(lmoe.LmoeError):  # K of the expert GEMMs a multiple of 64
+        lmoe.LatentMoELayer(w.d, 96, w.N, w.k, w.m, act=w.act, dtype="bf16",
+                            flags=lmoe.EXPERTS_FP8)
+    W = workloads.make_weights(w, device="cuda")
+    L = lmoe.LatentMoELayer(w.d, w.l, w.N, w.k, w.m, act=w.act, dtype="bf16",
+                            flags=lmoe.EXPERTS_FP8)
+    L.set_weights(W["Wg"], W["bias"], W["Wdown"], W["Wup"], None, None, None, None)
+    L.reserve(w.T)
+    x = workloads.make_x(w, device="cuda")
+    with pytest.raises(lmoe.LmoeError):  # not ready before the fp8 experts are set
+        L.forward(x)
+    L.set_expert_weights_fp8(W["W1q"], W["W1s"], W["W2q"], W["W2s"])
+    L.forward(x)
+    torch.cuda.synchronize()
+    plain = lmoe.LatentMoELayer(w.d, w.l, w.N, w.k, w.m, act=w.act, dtype="bf16")
+    with pytest.raises(lmoe.LmoeError):  # the layer was not created for fp8 experts
+        plain.set_expert_weights_fp8(W["W1q"], W["W1s"], W["W2q"], W["W2s"])
+
+
 def test_tcgen05_path_is_taken_for_bf16():
     res = check_forward(SMALL["swiglu"], fixture=True)
     assert paths(res)[0] in (1, 2, 4)
@@ -310,7 +364,8 @@ def test_device_error_word_clean_and_profile():
 # ---------------------------------------------------------------------------
 
 FULL_SAMPLES = {"tiny-fp32": 64, "std-moe-decode": 96, "latent-decode": 96,
-                "latent-prefill-shared": 64, "latent-prefill-skewed": 48}
+                "latent-prefill-shared": 64, "latent-prefill-skewed": 48,
+                "std-moe-decode-fp8": 96, "latent-decode-fp8": 96}
 
 
 @pytest.mark.parametrize("name", workloads.WORKLOAD_ORDER)
