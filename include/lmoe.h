@@ -96,8 +96,8 @@ typedef enum { LMOE_F32 = 0, LMOE_BF16 = 1 } lmoe_dtype;
 #define LMOE_EXPERTS_FP8        0x200u /* expert weights W1 and W2 as fp8 E4M3
                                     codes with one fp32 scale per output
                                     channel (lmoe_set_expert_weights_fp8);
-                                    activations stay bf16 and accumulation
-                                    fp32.  bf16 layers with l and m multiples
+                                    the expert MMAs run on f16 operands with
+                                    fp32 accumulation.  bf16 layers with l and m multiples
                                     of 64 only (else LMOE_ERR_UNSUPPORTED)   */
 
 /* Limits of this build. */
@@ -157,8 +157,11 @@ lmoe_status lmoe_set_weights(lmoe_layer* h, const void* W_g, const float* bias,
  * The library copies (and repacks) them; the caller keeps ownership of its
  * buffers.  lmoe_set_weights is still required for the other weights (its W1
  * and W2 may then be NULL); the layer is ready once both calls succeeded.
- * Codes are widened to bf16 exactly inside the expert kernels and the scale
- * multiplies the fp32 accumulator.  Synchronous.  Errors: INVALID_ARG (NULL
+ * Inside the expert kernels the codes widen exactly to f16 and the MMAs
+ * multiply f16 operands with fp32 accumulation: the FC1 input rows are
+ * converted to f16 once per forward (exact for magnitudes in [2^-14, 65504],
+ * saturating above) and FC1 writes its output in f16; the scale multiplies
+ * the fp32 accumulator.  Synchronous.  Errors: INVALID_ARG (NULL
  * pointer, layer created without LMOE_EXPERTS_FP8), CUDA, OOM.
  */
 lmoe_status lmoe_set_expert_weights_fp8(lmoe_layer* h, const void* W1q, const float* W1s,
@@ -226,7 +229,8 @@ typedef enum {
   LMOE_STAGE_OFFSETS = 3,  /* [N+1]    int32                                 */
   LMOE_STAGE_PERM = 4,     /* [T*k]    int32 sorted row -> t*k+j             */
   LMOE_STAGE_Z = 5,        /* [T, l]   dtype  latent rows (not with SKIP)    */
-  LMOE_STAGE_H = 6,        /* [T*k, m] dtype  expert hidden rows, sorted     */
+  LMOE_STAGE_H = 6,        /* [T*k, m] dtype  expert hidden rows, sorted
+                              (f16 with LMOE_EXPERTS_FP8)                   */
   LMOE_STAGE_YS = 7,       /* [T*k, l] dtype  gate-scaled expert outputs,
                                              expert-sorted rows (as H)       */
   LMOE_STAGE_COMB = 8      /* [T, l]   dtype  combined rows (not with SKIP)  */

@@ -8,6 +8,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -75,6 +76,7 @@ struct GemmProblem {
 };
 
 constexpr int kRowTile = 128;
+constexpr int kSwapRowTile = 64;  // rows per tile (the MMA's N, at most) of the weight-stationary kernel
 
 // ---- scalar helpers ---------------------------------------------------------
 
@@ -446,6 +448,14 @@ __device__ __forceinline__ uint32_t idesc_bf16_f32(int M, int N) {
   d |= 1u << 4;                       // D format: F32
   d |= 1u << 7;                       // A format: BF16
   d |= 1u << 10;                      // B format: BF16
+  d |= (uint32_t)(N >> 3) << 17;      // N >> 3
+  d |= (uint32_t)(M >> 4) << 24;      // M >> 4
+  return d;
+}
+// The same with f16 A and B (format code 0).
+__device__ __forceinline__ uint32_t idesc_f16_f32(int M, int N) {
+  uint32_t d = 0;
+  d |= 1u << 4;                       // D format: F32
   d |= (uint32_t)(N >> 3) << 17;      // N >> 3
   d |= (uint32_t)(M >> 4) << 24;      // M >> 4
   return d;

@@ -83,6 +83,7 @@ struct lmoe_layer {
   float* W1s = nullptr;      // [N * m_in]
   float* W2s = nullptr;      // [N * l]
   bool fp8_set = false;
+  void* a16 = nullptr;       // fp8 experts: the FC1 input rows in f16 [T, l or d]
   // workspace
   int max_T = 0, W = 0;
   float* logits = nullptr;
@@ -91,6 +92,7 @@ struct lmoe_layer {
   uint32_t* bitmap = nullptr;
   uint2* wp = nullptr;
   int *counts = nullptr, *offsets = nullptr, *tile_prefix = nullptr, *tile_prefix2 = nullptr;
+  int* tile_prefix64 = nullptr;  // 64-row tile counts (weight-stationary kernel)
   unsigned* done = nullptr;
   int* err = nullptr;
   int *row_tok = nullptr, *row_slot = nullptr, *slot_row = nullptr;
@@ -449,6 +451,15 @@ lmoe_status run_split(lmoe_layer* h, const GemmCall& c, int S, int kbs, cudaStre
 
 lmoe_status run_gemm(lmoe_layer* h, GemmCall c, cudaStream_t st, int* path = nullptr) {
   c.p.err = h->err;
+  // The weight-stationary tensor-core kernel takes at most kSwapRowTile rows
+  // (its MMA N) per tile: tiles follow the 64-row prefix.
+  const auto swap_rows = [&](GemmCall& g) {
+    if (g.swap && g.p.offsets) {
+      g.p.row_tile = kSwapRowTile;
+      g.p.tile_prefix = h->tile_prefix64;
+      g.p.max_row_tiles = (int)(g.out_rows / kSwapRowTile + h->N);  // routed rows
+    }
+  };
   if (c.p.w_scale) {
     // fp8 expert weights: the single-CTA tensor-core kernel with the E4M3
     // widening warps (weight-stationary or token-tiled)
@@ -456,6 +467,7 @@ lmoe_status run_gemm(lmoe_layer* h, GemmCall c, cudaStream_t st, int* path = nul
       h->detail = "fp8 expert weights need the single-CTA tensor-core kernel";
       return LMOE_ERR_UNSUPPORTED;
     }
+    swap_rows(c);
     const bool dual = c.p.dual_offset > 0;
     if (path) *path = c.swap ? 2 : 1;
     if (c.kind == GK_FC1) {
@@ -497,6 +509,7 @@ lmoe_status run_gemm(lmoe_layer* h, GemmCall c, cudaStream_t st, int* path = nul
       return launch_pair_ws<TcPairWsCfg<false, false, EPI_SCALE_ROWS>>(h, c, st);
   }
   if (path) *path = c.pair ? 3 : (c.swap ? 2 : 1);
+  swap_rows(c);
   if (!c.pair && !c.swap && !c.p.offsets && c.kind != GK_FC1 && c.kind != GK_FC2) {
     int kbs = 0;
     const int S = choose_splits(h, c, kbs);
@@ -618,7 +631,9 @@ lmoe_status run_routing(lmoe_layer* h, const float* logits, int T, int* idx, flo
   }
   if (marks) prof_mark(h, st, 2);
   group_count_kernel<<<(h->N + 7) / 8, 256, 0, st>>>(h->bitmap, h->wp, h->N, W, h->counts, offsets,
-                                                     h->tile_prefix, tile_prefix2, h->done);
+                                                     h->tile_prefix, tile_prefix2,
+                                                     tile_prefix2 ? h->tile_prefix64 : nullptr,
+                                                     h->done);
   LMOE_CHECK_LAUNCH(h);
   const long P = (long)T * h->k;
   group_rank_kernel<<<(unsigned)((P + 255) / 256), 256, 0, st>>>(
@@ -692,6 +707,18 @@ lmoe_status run_forward(lmoe_layer* h, const void* x, void* out, int T, cudaStre
   {
     const void* A = skip ? x : h->z;
     const bool fp8 = (h->flags & LMOE_EXPERTS_FP8) != 0;
+    if (fp8) {
+      // the fp8 expert kernels multiply f16 operands: the FC1 input in f16
+      const long n = (long)T * (skip ? d : l);
+      const int vec = (n % 8 == 0 && aligned16(A) && aligned16(h->a16)) ? 1 : 0;
+      const long work = vec ? n / 8 : n;
+      const unsigned blocks = (unsigned)std::max<long>(1, std::min<long>((work + 255) / 256,
+                                                                          8L * h->num_sms));
+      bf16_to_f16_kernel<<<blocks, 256, 0, st>>>(static_cast<const bf16*>(A),
+                                                 static_cast<__half*>(h->a16), n, vec);
+      LMOE_CHECK_LAUNCH(h);
+      A = h->a16;
+    }
     GemmCall c = grouped_call(h, GK_FC1, T, A, skip ? d : l, T, h->row_tok,
                               fp8 ? (const void*)h->W1q_t : h->W1_t, h->m_in, m, l);
     c.p.w_scale = fp8 ? h->W1s : nullptr;
@@ -786,6 +813,7 @@ void free_workspace(lmoe_layer* h) {
   free_ptr(h->offsets);
   free_ptr(h->tile_prefix);
   free_ptr(h->tile_prefix2);
+  free_ptr(h->tile_prefix64);
   free_ptr(h->slot_row);
   free_ptr(h->done);
   free_ptr(h->err);
@@ -808,6 +836,7 @@ void free_workspace(lmoe_layer* h) {
   h->copy_stream = nullptr;
   h->host_slot = 0;
   free_ptr(h->s32);
+  free_ptr(h->a16);
   free_ptr(h->part);
   h->part_bytes = 0;
   h->max_T = 0;
@@ -1026,6 +1055,7 @@ lmoe_status lmoe_reserve(lmoe_layer* h, int max_T) {
   ALLOC(h->offsets, (size_t)(h->N + 1) * sizeof(int));
   ALLOC(h->tile_prefix, (size_t)(h->N + 1) * sizeof(int));
   ALLOC(h->tile_prefix2, (size_t)(h->N + 1) * sizeof(int));
+  ALLOC(h->tile_prefix64, (size_t)(h->N + 1) * sizeof(int));
   ALLOC(h->slot_row, R * sizeof(int));
   ALLOC(h->done, sizeof(unsigned));
   ALLOC(h->err, sizeof(int));
@@ -1045,6 +1075,7 @@ lmoe_status lmoe_reserve(lmoe_layer* h, int max_T) {
     LMOE_CUDA(h, cudaEventCreateWithFlags(&h->ev_used[i], cudaEventDisableTiming));
   }
   if (skip && h->shared_m > 0) ALLOC(h->s32, T * h->d * sizeof(float));
+  if (h->flags & LMOE_EXPERTS_FP8) ALLOC(h->a16, T * (skip ? h->d : h->l) * 2);
   if (h->dtype == LMOE_BF16) {
     h->part_bytes = kSplitPartBytes;
     ALLOC(h->part, h->part_bytes);
@@ -1056,6 +1087,7 @@ lmoe_status lmoe_reserve(lmoe_layer* h, int max_T) {
   LMOE_CUDA(h, cudaMemset(h->offsets, 0, (size_t)(h->N + 1) * sizeof(int)));
   LMOE_CUDA(h, cudaMemset(h->tile_prefix, 0, (size_t)(h->N + 1) * sizeof(int)));
   LMOE_CUDA(h, cudaMemset(h->tile_prefix2, 0, (size_t)(h->N + 1) * sizeof(int)));
+  LMOE_CUDA(h, cudaMemset(h->tile_prefix64, 0, (size_t)(h->N + 1) * sizeof(int)));
   LMOE_CUDA(h, cudaDeviceSynchronize());
   h->max_T = max_T;
   h->W = (int)W;

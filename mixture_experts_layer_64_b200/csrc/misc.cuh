@@ -106,6 +106,34 @@ __global__ void __launch_bounds__(256) splitk_reduce_kernel(const float* __restr
   }
 }
 
+// bf16 -> f16 for the FC1 input of a layer with fp8 expert weights (its
+// expert MMAs run on f16 operands): exact for magnitudes in [2^-14, 65504],
+// an absolute error below 2^-25 under that, saturating at +-65504 above.
+// vec: n is a multiple of 8 and both pointers 16-byte aligned.
+__global__ void __launch_bounds__(256) bf16_to_f16_kernel(const bf16* __restrict__ in,
+                                                          __half* __restrict__ out, long n,
+                                                          int vec) {
+  const long i0 = ((long)blockIdx.x * blockDim.x + threadIdx.x) * (vec ? 8 : 1);
+  const long stride = (long)gridDim.x * blockDim.x * (vec ? 8 : 1);
+  for (long i = i0; i < n; i += stride) {
+    if (vec) {
+      uint4 v = *reinterpret_cast<const uint4*>(in + i);
+      uint32_t* w = reinterpret_cast<uint32_t*>(&v);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float lo = __uint_as_float(w[j] << 16), hi = __uint_as_float(w[j] & 0xFFFF0000u);
+        uint32_t h2;
+        asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(h2) : "f"(hi), "f"(lo));
+        w[j] = h2;
+      }
+      *reinterpret_cast<uint4*>(out + i) = v;
+    } else {
+      const float f = __bfloat162float(in[i]);
+      out[i] = __float2half_rn(fminf(fmaxf(f, -65504.f), 65504.f));
+    }
+  }
+}
+
 // out[b][c][col0 + r] = in[b][r][c] for r < rows, c < cols: the [in, out]
 // API layout to the K-major [out, in] layout, batched over experts, with a
 // column offset so that two matrices can share one K-concatenated operand.

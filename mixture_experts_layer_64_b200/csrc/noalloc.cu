@@ -95,7 +95,7 @@ extern "C" lmoe_status lmoe_route_only_noalloc(const float* logits, int T, int N
     return LMOE_ERR_CUDA;
   launch_topk(logits, T, N, k, nullptr, 0, idx, w, bitmap, (int)W, 0, err, s);
   group_count_kernel<<<(N + 7) / 8, 256, 0, s>>>(bitmap, wp, N, (int)W, counts, offsets,
-                                                 tile_prefix, nullptr, done);
+                                                 tile_prefix, nullptr, nullptr, done);
   const long P = (long)T * k;
   group_rank_kernel<<<(unsigned)((P + 255) / 256), 256, 0, s>>>(idx, w, wp, offsets, T, k, N,
                                                                  (int)W, nullptr, perm, nullptr,

@@ -301,6 +301,7 @@ static __global__ void __launch_bounds__(256) group_count_kernel(uint32_t* __res
                                                           int* __restrict__ offsets,
                                                           int* __restrict__ tile_prefix,
                                                           int* __restrict__ tile_prefix2,
+                                                          int* __restrict__ tile_prefix64,
                                                           unsigned int* done) {
   const int lane = threadIdx.x & 31;
   const int e = blockIdx.x * 8 + (threadIdx.x >> 5);
@@ -332,47 +333,55 @@ static __global__ void __launch_bounds__(256) group_count_kernel(uint32_t* __res
   __syncthreads();
   if (!is_last) return;
   __threadfence();
-  // Block-wide exclusive scans of counts and of ceil(counts / 128) and
-  // ceil(counts / 256) (row tiles of single CTAs and of CTA pairs).
-  __shared__ int s_c[256], s_t[256], s_u[256];
+  // Block-wide exclusive scans of counts and of ceil(counts / 128),
+  // ceil(counts / 256) and ceil(counts / 64) (row tiles of single CTAs, of
+  // CTA pairs, and of the weight-stationary kernel).
+  __shared__ int s_c[256], s_t[256], s_u[256], s_v[256];
   const int per = (N + 255) / 256;
   const int lo = threadIdx.x * per, hi = min(N, lo + per);
-  int c_sum = 0, t_sum = 0, u_sum = 0;
+  int c_sum = 0, t_sum = 0, u_sum = 0, v_sum = 0;
   for (int i = lo; i < hi; ++i) {
     const int c = __ldcg(counts + i);
     c_sum += c;
     t_sum += (c + kRowTile - 1) / kRowTile;
     u_sum += (c + 2 * kRowTile - 1) / (2 * kRowTile);
+    v_sum += (c + kSwapRowTile - 1) / kSwapRowTile;
   }
   s_c[threadIdx.x] = c_sum;
   s_t[threadIdx.x] = t_sum;
   s_u[threadIdx.x] = u_sum;
+  s_v[threadIdx.x] = v_sum;
   __syncthreads();
   for (int o = 1; o < 256; o <<= 1) {
     const int a = threadIdx.x >= o ? s_c[threadIdx.x - o] : 0;
     const int b = threadIdx.x >= o ? s_t[threadIdx.x - o] : 0;
     const int d = threadIdx.x >= o ? s_u[threadIdx.x - o] : 0;
+    const int f = threadIdx.x >= o ? s_v[threadIdx.x - o] : 0;
     __syncthreads();
     s_c[threadIdx.x] += a;
     s_t[threadIdx.x] += b;
     s_u[threadIdx.x] += d;
+    s_v[threadIdx.x] += f;
     __syncthreads();
   }
   int c_run = s_c[threadIdx.x] - c_sum, t_run = s_t[threadIdx.x] - t_sum,
-      u_run = s_u[threadIdx.x] - u_sum;
+      u_run = s_u[threadIdx.x] - u_sum, v_run = s_v[threadIdx.x] - v_sum;
   for (int i = lo; i < hi; ++i) {
     const int c = __ldcg(counts + i);
     offsets[i] = c_run;
     tile_prefix[i] = t_run;
     if (tile_prefix2) tile_prefix2[i] = u_run;
+    if (tile_prefix64) tile_prefix64[i] = v_run;
     c_run += c;
     t_run += (c + kRowTile - 1) / kRowTile;
     u_run += (c + 2 * kRowTile - 1) / (2 * kRowTile);
+    v_run += (c + kSwapRowTile - 1) / kSwapRowTile;
   }
   if (threadIdx.x == 255) {
     offsets[N] = s_c[255];
     tile_prefix[N] = s_t[255];
     if (tile_prefix2) tile_prefix2[N] = s_u[255];
+    if (tile_prefix64) tile_prefix64[N] = s_v[255];
     *done = 0u;
   }
 }

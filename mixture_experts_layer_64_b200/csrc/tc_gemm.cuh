@@ -12,9 +12,9 @@
 //   token-tiled (kSwap = false): the MMA's M = 128 activation rows, N = the
 //     weight tile (128 or 256 features); used when groups hold many rows.
 //   weight-stationary (kSwap = true): the MMA's M = 128 weight rows
-//     (features), N = the group's rows rounded up to 16 (<= 128); used at
-//     decode sizes, where an expert sees ~16 tokens and the kernel is a
-//     stream over the expert weights.
+//     (features), N = the tile's rows rounded up to 16 (tiles of at most 64
+//     rows); used at decode sizes, where an expert sees ~16 tokens and the
+//     kernel is a stream over the expert weights.
 // Gated FC1 (SwiGLU) loads the gate rows f and the linear rows f + m of the
 // same feature tile and accumulates them into two TMEM accumulators, so the
 // epilogue sees both halves of a feature in one thread.
@@ -28,9 +28,10 @@
 //               tcgen05.ld -> epilogue math -> shared-memory staging -> TMA
 //               bulk stores (plain stores for partly covered row blocks)
 // With fp8 E4M3 weights (512 threads) the epilogue is one warpgroup (warps
-// 4-7) and warps 8-15 widen each stage's E4M3 weight tiles to bf16 in shared
-// memory before the MMA issuer may use the stage; the per-output-channel
-// scales multiply the fp32 accumulators in the epilogue.
+// 4-7) and warps 8-15 widen each stage's E4M3 weight tiles to f16 in shared
+// memory before the MMA issuer (f16 x f16 -> fp32, the activation rows
+// arrive in f16) may use the stage; the per-output-channel scales multiply
+// the fp32 accumulators in the epilogue.
 // The smem ring has STAGES stages of one 64-wide K slice each; TMEM holds two
 // accumulator buffers so the epilogue of tile i overlaps the MMAs of tile i+1.
 #pragma once
@@ -54,61 +55,73 @@ struct TcCfg {
   static constexpr int EPI_WARPS = kFp8 ? 4 : kEpiWarps;
   static constexpr int CONV_THREADS = kFp8 ? 256 : 0;
   static constexpr int THREADS = 128 + 32 * EPI_WARPS + CONV_THREADS;
+  // fp8 weights: the MMA runs on f16 operands, so the FC1 output (the FC2
+  // input) is written in f16; FC2 writes bf16
+  static constexpr bool kF16Out = kFp8 && kEpi_ == EPI_ACT;
   static constexpr int BK = 64;                       // bf16 per 128-byte swizzled row
-  static constexpr int ACT_ROWS = 128;
+  static constexpr int ACT_ROWS = kSwap ? kSwapRowTile : 128;  // activation rows per stage
   static constexpr int W_ROWS = kSwap ? 128 : (kDual ? 128 : kWN_);
   static constexpr int NUM_W = kDual ? 2 : 1;
   static constexpr int ACT_BYTES = ACT_ROWS * BK * 2;
   static constexpr int W_BYTES = W_ROWS * BK * 2;
   static constexpr int W8_BYTES = kFp8 ? W_ROWS * BK : 0;  // one fp8 weight tile (64-byte rows)
-  static constexpr int STAGE_BYTES = ACT_BYTES + NUM_W * (W_BYTES + W8_BYTES);
+  static constexpr int STAGE_BYTES = ACT_BYTES + NUM_W * W_BYTES;  // one bf16 stage
   // epilogue staging: one 32 x 32 box per epilogue warp (bf16 or fp32)
   static constexpr int STG_WARP = kEpi == EPI_F32_BIAS ? 4096 : 2048;
   static constexpr int STG_BYTES = kSwap ? 0 : EPI_WARPS * STG_WARP;
-  static constexpr int STAGES_RAW = (kTcSmemBudget + kEpiWarps * 2048 - STG_BYTES) / STAGE_BYTES;
-  static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
+  static constexpr int BUDGET = kTcSmemBudget + kEpiWarps * 2048 - STG_BYTES;
+  static constexpr int STAGES_RAW = BUDGET / STAGE_BYTES;
+  // fp8 weights: about 5/9 of the budget as widened stages (at least 3), the
+  // rest as a ring of E4M3 slots (one K slice of the NUM_W weight tiles each)
+  // that a producer lane fills ahead of the stages
+  static constexpr int STAGES_F8 = BUDGET * 5 / 9 / STAGE_BYTES;
+  static constexpr int STAGES = kFp8 ? (STAGES_F8 < 3 ? 3 : (STAGES_F8 > 8 ? 8 : STAGES_F8))
+                                     : (STAGES_RAW > 8 ? 8 : STAGES_RAW);
+  static constexpr int W8_SLOT = NUM_W * W8_BYTES;
+  static constexpr int S8_RAW = kFp8 ? (BUDGET - STAGES * STAGE_BYTES) / W8_SLOT : 0;
+  static constexpr int S8 = S8_RAW > 16 ? 16 : S8_RAW;
+  static constexpr int RING_BYTES = STAGES * STAGE_BYTES + S8 * W8_SLOT;
   static constexpr int ACC_N = kSwap ? 128 : W_ROWS;  // fp32 columns of one accumulator
   static constexpr int ACC_COLS = ACC_N * NUM_W;      // one TMEM buffer
   static constexpr int TMEM_COLS = 2 * ACC_COLS;      // double buffered
   static constexpr int FT = W_ROWS;                   // features per tile
   static constexpr int TABLE_BYTES = 2 * (LMOE_MAX_EXPERTS + 1) * 4;  // tile_prefix, offsets
-  static constexpr int SMEM_BYTES = 1024 /*align slack*/ + STAGES * STAGE_BYTES + STG_BYTES + 512 +
+  static constexpr int SMEM_BYTES = 1024 /*align slack*/ + RING_BYTES + STG_BYTES + 512 +
                                     TABLE_BYTES;
   static_assert(TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM allocation must be a power of two");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
   static_assert(STAGES >= 3, "pipeline too shallow");
+  static_assert(!kFp8 || S8 >= 2, "fp8 weight ring too shallow");
+  static_assert(2 * STAGES * 8 + 2 * S8 * 8 + 5 * 8 + 8 <= 512, "barrier area");
   static_assert(!kSwap || kEpi == EPI_ACT || kEpi == EPI_SCALE_ROWS, "swap epilogues");
   static_assert(kWN_ == 128 || kWN_ == 256, "weight tile");
   static_assert(!kFp8 || kEpi == EPI_ACT || kEpi == EPI_SCALE_ROWS, "fp8 weights: expert GEMMs");
 };
 
 // ---- fp8 E4M3 weights -----------------------------------------------------------
+//
+// The expert kernels with fp8 weights run the MMA on f16 operands: an E4M3
+// code widens to f16 in one hardware conversion per pair, and the activation
+// rows arrive in f16 (the layer converts the FC1 input once per forward, and
+// FC1 writes its output in f16).
 
-// Four E4M3 codes (byte 0 first) -> four bf16 with the same values, as two
-// bf16x2 words.  Every step is an exact hardware conversion: E4M3 pairs to
-// f16 pairs (every E4M3 value, subnormals included, is a normal f16 or
-// zero), f16 to f32, and f32 pairs to bf16 pairs (4 significant bits fit).
-__device__ __forceinline__ void e4m3x4_to_bf16x4(uint32_t w, uint32_t& lo, uint32_t& hi) {
-  asm("{\n\t.reg .b16 l, h, a0, a1, a2, a3;\n\t.reg .b32 fl, fh;\n\t"
-      ".reg .f32 f0, f1, f2, f3;\n\t"
+// Four E4M3 codes (byte 0 first) -> four f16 with the same values, as two
+// f16x2 words: one exact hardware conversion per pair (every E4M3 value,
+// subnormals included, is a normal f16 or zero).
+__device__ __forceinline__ void e4m3x4_to_f16x4(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  asm("{\n\t.reg .b16 l, h;\n\t"
       "mov.b32 {l, h}, %2;\n\t"
-      "cvt.rn.f16x2.e4m3x2 fl, l;\n\t"
-      "cvt.rn.f16x2.e4m3x2 fh, h;\n\t"
-      "mov.b32 {a0, a1}, fl;\n\t"
-      "mov.b32 {a2, a3}, fh;\n\t"
-      "cvt.f32.f16 f0, a0;\n\tcvt.f32.f16 f1, a1;\n\t"
-      "cvt.f32.f16 f2, a2;\n\tcvt.f32.f16 f3, a3;\n\t"
-      "cvt.rn.bf16x2.f32 %0, f1, f0;\n\t"
-      "cvt.rn.bf16x2.f32 %1, f3, f2;\n\t}"
+      "cvt.rn.f16x2.e4m3x2 %0, l;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %1, h;\n\t}"
       : "=r"(lo), "=r"(hi)
       : "r"(w));
 }
 
 // Widens one weight tile: W_ROWS rows of 64 E4M3 codes (64-byte rows, no
-// swizzle, as TMA stored them) into W_ROWS rows of 64 bf16 in the 128-byte
+// swizzle, as TMA stored them) into W_ROWS rows of 64 f16 in the 128-byte
 // swizzled K-major layout the MMA reads.  ct = this thread's index among the
-// nconv converter threads; chunk c = (row, 16-byte quarter q) is handled by
-// thread c mod nconv.
+// kConv converter threads; chunk c = (row, 16-byte quarter q) is handled by
+// thread c mod kConv.
 template <int W_ROWS, int kConv>
 __device__ __forceinline__ void widen_fp8_tile(const uint8_t* src, uint8_t* dst, int ct) {
 #pragma unroll
@@ -118,7 +131,7 @@ __device__ __forceinline__ void widen_fp8_tile(const uint8_t* src, uint8_t* dst,
     const uint32_t in[4] = {v.x, v.y, v.z, v.w};
     uint32_t out[8];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) e4m3x4_to_bf16x4(in[i], out[2 * i], out[2 * i + 1]);
+    for (int i = 0; i < 4; ++i) e4m3x4_to_f16x4(in[i], out[2 * i], out[2 * i + 1]);
     uint8_t* row = dst + r * 128;
     const int sw = r & 7;
     *reinterpret_cast<uint4*>(row + (((2 * q) ^ sw) << 4)) = make_uint4(out[0], out[1], out[2], out[3]);
@@ -129,8 +142,17 @@ __device__ __forceinline__ void widen_fp8_tile(const uint8_t* src, uint8_t* dst,
 
 // ---- epilogue stores ----------------------------------------------------------
 
+// The 16-bit output value of v: bf16, or (kF16) the bits of the f16 value in
+// the same storage type -- the expert FC1 of a layer with fp8 weights writes
+// its hidden rows in f16, the operand type of its FC2.
+template <bool kF16>
+__device__ __forceinline__ bf16 round_out(float v) {
+  if constexpr (kF16) return __ushort_as_bfloat16(__half_as_ushort(__float2half_rn(v)));
+  else return __float2bfloat16_rn(v);
+}
+
 // One row (token-tiled mode): 32 consecutive features [f, f+32) of row `row`.
-template <int kEpi, bool kGated>
+template <int kEpi, bool kGated, bool kF16 = false>
 __device__ __forceinline__ void store_row32(const GemmProblem& p, int row, int f,
                                             const float (&v0)[32], const float (&v1)[32],
                                             size_t slice_off = 0) {
@@ -185,11 +207,11 @@ __device__ __forceinline__ void store_row32(const GemmProblem& p, int row, int f
       bf16* qlb = reinterpret_cast<bf16*>(&ql);
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        qb[j] = __float2bfloat16_rn(r[i + j]);
-        qlb[j] = __float2bfloat16_rn(r[i + j] - __bfloat162float(qb[j]));
+        qb[j] = round_out<kF16>(r[i + j]);
+        if (!kF16) qlb[j] = __float2bfloat16_rn(r[i + j] - __bfloat162float(qb[j]));
       }
       *reinterpret_cast<uint4*>(o + i) = q;
-      if (split) *reinterpret_cast<uint4*>(o + split + i) = ql;
+      if (!kF16 && split) *reinterpret_cast<uint4*>(o + split + i) = ql;
     }
   } else {
     // ragged last chunk (F not a multiple of 32): element stores, fully
@@ -198,24 +220,24 @@ __device__ __forceinline__ void store_row32(const GemmProblem& p, int row, int f
     for (int i = 0; i < 32; ++i) {
       if (f + i < p.F) {
         float v = (kEpi == EPI_RESID) ? __bfloat162float(res[i]) + v0[i] : r[i];
-        const bf16 hi = __float2bfloat16_rn(v);
+        const bf16 hi = round_out<kF16>(v);
         o[i] = hi;
-        if (split) o[split + i] = __float2bfloat16_rn(v - __bfloat162float(hi));
+        if (!kF16 && split) o[split + i] = __float2bfloat16_rn(v - __bfloat162float(hi));
       }
     }
   }
 }
 
 // One element (weight-stationary mode): feature f of row `row`.
-template <int kEpi>
+template <int kEpi, bool kF16 = false>
 __device__ __forceinline__ void store_elem(const GemmProblem& p, int row, int f, float v0, float v1) {
   const EpiParams& e = p.epi;
   if (kEpi == EPI_ACT) {
     const float v = apply_act(e.act, v0, v1);
-    const bf16 hi = __float2bfloat16_rn(v);
+    const bf16 hi = round_out<kF16>(v);
     bf16* o = static_cast<bf16*>(e.out) + (size_t)row * e.ldo + e.col0 + f;
     o[0] = hi;
-    if (e.split_off) o[e.split_off] = __float2bfloat16_rn(v - __bfloat162float(hi));
+    if (!kF16 && e.split_off) o[e.split_off] = __float2bfloat16_rn(v - __bfloat162float(hi));
   } else {  // EPI_SCALE_ROWS
     static_cast<bf16*>(e.out)[(size_t)row * e.ldo + f] =
         __float2bfloat16_rn(v0 * __ldg(e.row_w + row));
@@ -232,7 +254,7 @@ __device__ __forceinline__ void store_elem(const GemmProblem& p, int row, int f,
 // keeps the row-per-thread writes free of bank conflicts) and one lane writes
 // the box with a bulk tensor store.  Blocks of 32 rows that a tile only partly
 // covers, and the fp32 router logits, use the plain stores.
-template <int kEpi, bool kGated>
+template <int kEpi, bool kGated, bool kF16>
 __device__ __forceinline__ void epi_tma_chunk32_impl(const GemmProblem& p, const CUtensorMap* tmC,
                                                 uint8_t* stg, int lane, int row_base, int f,
                                                 const float (&v0)[32], const float (&v1)[32]) {
@@ -268,7 +290,7 @@ __device__ __forceinline__ void epi_tma_chunk32_impl(const GemmProblem& p, const
     uint4 q;
     bf16* qb = reinterpret_cast<bf16*>(&q);
 #pragma unroll
-    for (int j = 0; j < 8; ++j) qb[j] = __float2bfloat16_rn(r[8 * c + j]);
+    for (int j = 0; j < 8; ++j) qb[j] = round_out<kF16>(r[8 * c + j]);
     *reinterpret_cast<uint4*>(stg + lane * 64 + ((c ^ ((lane >> 1) & 3)) << 4)) = q;
   }
   fence_proxy_async_smem();
@@ -307,14 +329,14 @@ __device__ __forceinline__ void epi_tma_chunk32_f32(const GemmProblem& p, const 
   }
 }
 
-template <int kEpi, bool kGated>
+template <int kEpi, bool kGated, bool kF16 = false>
 __device__ __forceinline__ void epi_tma_chunk32(const GemmProblem& p, const CUtensorMap* tmC,
                                                 uint8_t* stg, int lane, int row_base, int f,
                                                 const float (&v0)[32], const float (&v1)[32]) {
   if constexpr (kEpi == EPI_F32_BIAS)
     epi_tma_chunk32_f32(p, tmC, stg, lane, row_base, f, v0);
   else
-    epi_tma_chunk32_impl<kEpi, kGated>(p, tmC, stg, lane, row_base, f, v0, v1);
+    epi_tma_chunk32_impl<kEpi, kGated, kF16>(p, tmC, stg, lane, row_base, f, v0, v1);
 }
 
 // ---- tile lookup from shared memory -----------------------------------------------
@@ -366,18 +388,18 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint8_t* stg_base = smem + Cfg::STAGES * Cfg::STAGE_BYTES;  // epilogue staging (1024-aligned)
+  uint8_t* stg_base = smem + Cfg::RING_BYTES;  // epilogue staging (1024-aligned)
+  uint8_t* w8_ring = smem + Cfg::STAGES * Cfg::STAGE_BYTES;  // fp8 weights: E4M3 slots
   uint64_t* full = reinterpret_cast<uint64_t*>(stg_base + Cfg::STG_BYTES);
   uint64_t* empty = full + Cfg::STAGES;
-  uint64_t* wfull = empty + Cfg::STAGES;  // fp8 weights: the E4M3 tiles have landed
-  uint64_t* tfull = wfull + Cfg::STAGES;
+  uint64_t* w8full = empty + Cfg::STAGES;  // fp8: an E4M3 slot has landed
+  uint64_t* w8empty = w8full + Cfg::S8;    // fp8: an E4M3 slot has been widened
+  uint64_t* tfull = w8empty + Cfg::S8;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* s_tiles = reinterpret_cast<int*>(stg_base + Cfg::STG_BYTES + 512);
-  static_assert(3 * Cfg::STAGES * 8 + 5 * 8 + 8 <= 512, "barrier area");
-  constexpr int W8_OFF = Cfg::ACT_BYTES + Cfg::NUM_W * Cfg::W_BYTES;  // fp8 tiles in a stage
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   load_tile_tables(p, s_tiles);
@@ -387,9 +409,13 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < Cfg::STAGES; ++s) {
       // producer + gather threads + (fp8) the converters, after widening
+      // producer + gather threads + (fp8) the converters, after widening
       mbar_init(&full[s], 1 + (Cfg::kGather ? kGatherThreads : 0) + Cfg::CONV_THREADS);
       mbar_init(&empty[s], 1);
-      mbar_init(&wfull[s], 1);
+    }
+    for (int j = 0; j < Cfg::S8; ++j) {
+      mbar_init(&w8full[j], 1);
+      mbar_init(&w8empty[j], Cfg::CONV_THREADS);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
@@ -420,6 +446,42 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
 
   if (warp == 0) {
     // ---------------- TMA producer ----------------
+    // Lane 0 arms the stages (activation rows, and bf16 weights).  With fp8
+    // weights lane 1 walks the same (tile, K block) sequence on its own and
+    // keeps the E4M3 slot ring loading, limited only by the converters.
+    if (Cfg::kFp8 && lane == 1) {
+      int j = 0;
+      uint32_t jph = 0;
+      long wissued = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+        const int ks = t / tiles_per_split, tl = t - ks * tiles_per_split;
+        const int rt = tl / NT, ft = tl - (tl / NT) * NT;
+        const int kb0 = ks * KBS, kb1 = min(KB, kb0 + KBS);
+        int g, row0, rows;
+        locate_row_tile_s(p, s_tiles, rt, g, row0, rows);
+        const int wrow = (int)(g * p.w_group_stride) + ft * Cfg::FT;
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait(&w8empty[j], jph ^ 1, abort_flag, p.err)) { ok = false; break; }
+          uint8_t* slot = w8_ring + j * Cfg::W8_SLOT;
+          mbar_arrive_expect_tx(&w8full[j], Cfg::W8_SLOT);
+          tma_load_2d(&tmB, &w8full[j], slot, kb * Cfg::BK, wrow);
+          if (Cfg::kDual)
+            tma_load_2d(&tmB, &w8full[j], slot + Cfg::W8_BYTES, kb * Cfg::BK,
+                        wrow + p.dual_offset);
+          ++wissued;
+          if (++j == Cfg::S8) { j = 0; jph ^= 1; }
+        }
+      }
+      if (*abort_flag) {
+        // let the loads in flight land before the block frees its shared memory
+        for (long i = 0; i < wissued && i < Cfg::S8; ++i) {
+          if (j == 0) { j = Cfg::S8; jph ^= 1; }
+          --j;
+          mbar_wait_drain(&w8full[j], jph);
+        }
+      }
+    }
     if (lane == 0) {
       int s = 0;
       uint32_t ph = 0;
@@ -438,16 +500,10 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, p.err)) { ok = false; break; }
           uint8_t* st = smem + s * Cfg::STAGE_BYTES;
-          mbar_arrive_expect_tx(&full[s], bytes);
+          uint64_t* abar = &full[s];
+          mbar_arrive_expect_tx(abar, bytes);
           ++armed;
-          if (Cfg::kFp8) {
-            // E4M3 tiles into the staging area; the converter warps widen them
-            mbar_arrive_expect_tx(&wfull[s], Cfg::NUM_W * Cfg::W8_BYTES);
-            tma_load_2d(&tmB, &wfull[s], st + W8_OFF, kb * Cfg::BK, wrow);
-            if (Cfg::kDual)
-              tma_load_2d(&tmB, &wfull[s], st + W8_OFF + Cfg::W8_BYTES, kb * Cfg::BK,
-                          wrow + p.dual_offset);
-          } else {
+          if (!Cfg::kFp8) {
             tma_load_2d(&tmB, &full[s], st + Cfg::ACT_BYTES, kb * Cfg::BK, wrow);
             if (Cfg::kDual)
               tma_load_2d(&tmB, &full[s], st + Cfg::ACT_BYTES + Cfg::W_BYTES, kb * Cfg::BK,
@@ -456,9 +512,9 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
           if (!Cfg::kGather) {
             if (Cfg::kSwap) {
               for (int sub = 0; sub < nsub; ++sub)
-                tma_load_2d(&tmA, &full[s], st + sub * 4096, kb * Cfg::BK, row0 + sub * 32);
+                tma_load_2d(&tmA, abar, st + sub * 4096, kb * Cfg::BK, row0 + sub * 32);
             } else {
-              tma_load_2d(&tmA, &full[s], st, kb * Cfg::BK, row0);
+              tma_load_2d(&tmA, abar, st, kb * Cfg::BK, row0);
             }
           }
           if (++s == Cfg::STAGES) { s = 0; ph ^= 1; }
@@ -466,16 +522,15 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         if (!ok) break;
       }
       if (*abort_flag) {
-        // Let every armed load land before the block frees its shared memory
-        // (fp8: the weight tiles complete on wfull; full may then stay short
-        // of the converters' arrivals, which the bounded wait absorbs).
+        // Let every armed load land before the block frees its shared memory.
         int ss = s;
         uint32_t pp = ph;
         for (long i = 0; i < armed && i < Cfg::STAGES; ++i) {
           if (ss == 0) { ss = Cfg::STAGES; pp ^= 1; }
           --ss;
-          if (Cfg::kFp8) mbar_wait_drain(&wfull[ss], pp);
-          if (!Cfg::kFp8 || !Cfg::kGather) mbar_wait_drain(&full[ss], pp);
+          // (with fp8 weights full may stay short of the converters'
+          // arrivals; the bounded wait absorbs that)
+          mbar_wait_drain(&full[ss], pp);
         }
       }
     }
@@ -503,7 +558,8 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         // MMA computes both and reads the activation tile once.
         int n = Cfg::kDual ? 2 * Cfg::ACC_N : Cfg::ACC_N;
         if (Cfg::kSwap) n = max(16, (rows + 15) & ~15);
-        const uint32_t idesc = idesc_bf16_f32(128, n);
+        // fp8 weights: both operands were widened to f16
+        const uint32_t idesc = Cfg::kFp8 ? idesc_f16_f32(128, n) : idesc_bf16_f32(128, n);
         bool ok = true;
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&full[s], ph, abort_flag, p.err)) { ok = false; break; }
@@ -579,30 +635,37 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       cp_async_wait<0>();
     }
   } else if (warp >= 4 + Cfg::EPI_WARPS) {
-    // ---------------- fp8 weights: widen E4M3 tiles to bf16 ----------------
-    // Same stage sequence as the producer; each stage's tiles are widened in
-    // place (staging area -> the bf16 weight slots) and handed to the MMA
-    // issuer with a fence (generic-proxy writes -> tensor-core reads) and an
-    // arrive on full.
+    // ---------------- fp8 weights: widen to f16 ----------------
+    // Same (tile, K block) sequence as the producer: E4M3 slot j is widened
+    // into stage s's weight slots, handed to the MMA issuer with a fence
+    // (generic-proxy writes -> tensor-core reads) and an arrive on full, and
+    // the slot goes back to the producer with an arrive on w8empty.
     if (Cfg::kFp8) {
       const int ct = threadIdx.x - (128 + 32 * Cfg::EPI_WARPS);
       int s = 0;
       uint32_t ph = 0;
       bool ok = true;
+      int j = 0;
+      uint32_t jph = 0;
       for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
         const int ks = t / tiles_per_split;
         const int kb0 = ks * KBS, kb1 = min(KB, kb0 + KBS);
         for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait(&wfull[s], ph, abort_flag, p.err)) { ok = false; break; }
+          // the E4M3 slot has landed and the stage's previous MMAs are done
+          if (!mbar_wait(&w8full[j], jph, abort_flag, p.err)) { ok = false; break; }
+          if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, p.err)) { ok = false; break; }
           uint8_t* st = smem + s * Cfg::STAGE_BYTES;
+          const uint8_t* slot = w8_ring + j * Cfg::W8_SLOT;
 #pragma unroll
           for (int i = 0; i < Cfg::NUM_W; ++i)
-            widen_fp8_tile<Cfg::W_ROWS, Cfg::CONV_THREADS>(st + W8_OFF + i * Cfg::W8_BYTES,
+            widen_fp8_tile<Cfg::W_ROWS, Cfg::CONV_THREADS>(slot + i * Cfg::W8_BYTES,
                                                            st + Cfg::ACT_BYTES + i * Cfg::W_BYTES,
                                                            ct);
           fence_proxy_async_smem();
           mbar_arrive(&full[s]);
+          mbar_arrive(&w8empty[j]);
           if (++s == Cfg::STAGES) { s = 0; ph ^= 1; }
+          if (++j == Cfg::S8) { j = 0; jph ^= 1; }
         }
       }
     }
@@ -645,10 +708,11 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
               }
             }
             if (tma)
-              epi_tma_chunk32<Cfg::kEpi, Cfg::kDual>(p, &tmC, stg, lane, slice_rows + row0 + qd * 32,
-                                                     f0 + c0, v0, v1);
+              epi_tma_chunk32<Cfg::kEpi, Cfg::kDual, Cfg::kF16Out>(
+                  p, &tmC, stg, lane, slice_rows + row0 + qd * 32, f0 + c0, v0, v1);
             else if (r < rows)
-              store_row32<Cfg::kEpi, Cfg::kDual>(p, row0 + r, f0 + c0, v0, v1, slice_off);
+              store_row32<Cfg::kEpi, Cfg::kDual, Cfg::kF16Out>(p, row0 + r, f0 + c0, v0, v1,
+                                                               slice_off);
           }
         }
       } else {
@@ -668,8 +732,8 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
 #pragma unroll
             for (int c = 0; c < 32; ++c)
               if (c < cn)
-                store_elem<Cfg::kEpi>(p, row0 + c0 + c, f, v0[c] * s0,
-                                      Cfg::kDual ? v1[c] * s1 : 0.f);
+                store_elem<Cfg::kEpi, Cfg::kF16Out>(p, row0 + c0 + c, f, v0[c] * s0,
+                                                    Cfg::kDual ? v1[c] * s1 : 0.f);
           }
         }
       }
