@@ -240,8 +240,10 @@ lmoe_status launch_tc(lmoe_layer* h, const GemmCall& c, cudaStream_t st) {
   CUtensorMap ta, tb;
   std::memset(&ta, 0, sizeof ta);
   std::memset(&tb, 0, sizeof tb);
-  if (!Cfg::kGather &&
-      !encode_map(&ta, c.p.A, c.a_rows, c.p.K, c.p.lda, Cfg::kSwap ? 32 : 128)) {
+  // activations: 32- or 128-row boxes, or (gathered rows) one-row boxes for
+  // the four-row TMA gather
+  if (!encode_map(&ta, c.p.A, c.a_rows, c.p.K, c.p.lda,
+                  Cfg::kGather ? 1 : (Cfg::kSwap ? 32 : 128))) {
     h->detail = "cuTensorMapEncodeTiled (activations) failed";
     return LMOE_ERR_CUDA;
   }

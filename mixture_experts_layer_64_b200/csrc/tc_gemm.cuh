@@ -22,8 +22,10 @@
 // Warp roles (384 threads; 512 with fp8 weights):
 //   warp 0      TMA producer (weights, and contiguous activation rows)
 //   warp 1      TMEM allocation and the single-thread MMA issuer
-//   warps 2-3   cp.async row gather of activations (gathered problems),
-//               completion signalled to the MMA issuer through the mbarrier
+//   warps 2-3   row gather of activations (gathered problems): cp.async
+//               copies for token-tiled tiles, completion signalled to the MMA
+//               issuer through the mbarrier; four-row TMA gathers (warp 2)
+//               for weight-stationary tiles
 //   warps 4-11  epilogue, two warpgroups taking alternate 32-column chunks:
 //               tcgen05.ld -> epilogue math -> shared-memory staging -> TMA
 //               bulk stores (plain stores for partly covered row blocks)
@@ -409,8 +411,11 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < Cfg::STAGES; ++s) {
       // producer + gather threads + (fp8) the converters, after widening
-      // producer + gather threads + (fp8) the converters, after widening
-      mbar_init(&full[s], 1 + (Cfg::kGather ? kGatherThreads : 0) + Cfg::CONV_THREADS);
+      // the producer (its expect_tx covers the weights and the activation
+      // rows, including TMA-gathered ones) + the cp.async gather threads of
+      // token-tiled tiles + (fp8) the converters, after widening
+      mbar_init(&full[s], 1 + (Cfg::kGather && !Cfg::kSwap ? kGatherThreads : 0) +
+                              Cfg::CONV_THREADS);
       mbar_init(&empty[s], 1);
     }
     for (int j = 0; j < Cfg::S8; ++j) {
@@ -496,6 +501,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         const int nsub = Cfg::kSwap ? (rows + 31) / 32 : 4;
         uint32_t bytes = Cfg::kFp8 ? 0u : (uint32_t)(Cfg::NUM_W * Cfg::W_BYTES);
         if (!Cfg::kGather) bytes += Cfg::kSwap ? nsub * 4096 : Cfg::ACT_BYTES;
+        else if (Cfg::kSwap) bytes += max(16, (rows + 15) & ~15) * 128;  // TMA-gathered rows
         bool ok = true;
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, p.err)) { ok = false; break; }
@@ -589,14 +595,50 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       tc_commit(drain);
       mbar_wait_drain(drain, 0);
     }
+  } else if (warp < 4 && Cfg::kGather && Cfg::kSwap) {
+    // ---------------- TMA row gather (weight-stationary tiles) ----------------
+    // Lane i of warp 2 brings rows 4i..4i+3 of each stage's activation tile
+    // (at most 64 rows) with one gather4 (rows picked by token index; the
+    // tile's padding rows repeat its first row), completing on the stage's
+    // full barrier, whose expected bytes the producer has armed.  Warp 3 has
+    // no work.  (Token-tiled tiles gather 128 rows per stage with cp.async:
+    // there a four-row TMA gather cannot keep up.)
+    if (warp == 2) {
+      int s = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+        const int ks = t / tiles_per_split, tl = t - ks * tiles_per_split;
+        const int rt = tl / NT;
+        const int kb0 = ks * KBS, kb1 = min(KB, kb0 + KBS);
+        int g, row0, rows;
+        locate_row_tile_s(p, s_tiles, rt, g, row0, rows);
+        const int nload = Cfg::kSwap ? max(16, (rows + 15) & ~15) : Cfg::ACT_ROWS;
+        const bool active = 4 * lane < nload;
+        int src[4];
+        const int first = __ldg(p.gather + row0);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int r = 4 * lane + q;
+          src[q] = r < rows ? __ldg(p.gather + row0 + r) : first;
+        }
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, p.err)) { ok = false; break; }
+          if (active)
+            tma_gather4(&tmA, &full[s], smem + s * Cfg::STAGE_BYTES + lane * 4 * 128,
+                        kb * Cfg::BK, src[0], src[1], src[2], src[3]);
+          if (++s == Cfg::STAGES) { s = 0; ph ^= 1; }
+        }
+      }
+    }
   } else if (warp < 4) {
-    // ---------------- cp.async row gather ----------------
+    // ---------------- cp.async row gather (token-tiled tiles) ----------------
     // Each thread copies 16-byte chunks of the tile's rows straight into the
     // 128-byte-swizzled layout, then hands the stage to the MMA issuer with an
     // mbarrier arrive that the hardware triggers when its copies have landed.
     // The thread never waits for its own copies, so all STAGES stages can be
     // in flight.
-    if (Cfg::kGather) {
+    if (Cfg::kGather && !Cfg::kSwap) {
       const int gt = threadIdx.x - 64;  // 0..63
       const int q = gt & 7;             // 16-byte chunk of a 128-byte row
       const int rsub = gt >> 3;         // rows rsub, rsub + 8, ...
