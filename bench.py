@@ -240,6 +240,29 @@ def workload_config(w: workloads.Workload, n_gpus: int):
                   "weights streamed from HBM every step"}
 
 
+# ---------------------------------------------------------------------------
+# replicas (one process per GPU): the pieces that do not need a GPU
+# ---------------------------------------------------------------------------
+
+def replica_workload(w: workloads.Workload, rank: int) -> workloads.Workload:
+    """Rank r draws its own batch (seed + 1000 r); weights are the same."""
+    return w if rank == 0 else workloads.Workload(**{**w.__dict__, "seed": w.seed + 1000 * rank})
+
+
+def max_over_ranks(pg, value: float, device) -> float:
+    """The largest of the ranks' values (the job's time is its slowest rank)."""
+    if pg is None:
+        return float(value)
+    t = torch.tensor([value], device=device, dtype=torch.float64)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(tokens_per_rank: int, ranks: int, ms_per_step: float) -> float:
+    """Whole-job tokens/s: every rank's tokens over the slowest rank's time."""
+    return tokens_per_rank * ranks / (ms_per_step / 1000.0)
+
+
 def run_reference(args):
     ws, rank, _ = dist_env()
     if rank != 0:
@@ -293,7 +316,7 @@ def run_ours(args):
     w = workloads.WORKLOADS[args.workload]
     W = workloads.make_weights(w, device=dev)
     # each replica draws its own batch
-    xw = w if rank == 0 else workloads.Workload(**{**w.__dict__, "seed": w.seed + 1000 * rank})
+    xw = replica_workload(w, rank)
     x = workloads.make_x(xw, device=dev)
     L = lmoe.LatentMoELayer(w.d, w.l, w.N, w.k, w.m, act=w.act, shared_m=w.shared_m,
                             dtype=w.dtype, skip_proj=w.skip_proj,
@@ -334,12 +357,9 @@ def run_ours(args):
     clocks = sampler.stop() if sampler else None
     elapsed_ms = t0.elapsed_time(t1)
     prof = L.profile_end()
-    if pg:
-        tt = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
-        pg.all_reduce(tt, op=pg.ReduceOp.MAX)
-        elapsed_ms = float(tt.item())
+    elapsed_ms = max_over_ranks(pg, elapsed_ms, dev)
     ms_per_step = elapsed_ms / args.steps
-    value = w.T * ws / (ms_per_step / 1000.0)
+    value = job_throughput(w.T, ws, ms_per_step)
 
     # ---- end to end through the host-buffer entry point (pinned buffers)
     xh = x.cpu().pin_memory()
@@ -357,11 +377,7 @@ def run_ours(args):
         L.forward_host(xh, oh)
     e1.record(stream)
     torch.cuda.synchronize()
-    e_ms = e0.elapsed_time(e1) / e_steps
-    if pg:
-        tt = torch.tensor([e_ms], device=dev, dtype=torch.float64)
-        pg.all_reduce(tt, op=pg.ReduceOp.MAX)
-        e_ms = float(tt.item())
+    e_ms = max_over_ranks(pg, e0.elapsed_time(e1) / e_steps, dev)
     io_bytes = w.T * w.d * (4 if w.dtype == "f32" else 2)
 
     st, word = L.last_error()
@@ -419,7 +435,7 @@ def run_ours(args):
                 "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
                 "config": workload_config(w, ws),
-                "e2e": {"value": w.T * ws / (e_ms / 1000.0), "unit": UNIT,
+                "e2e": {"value": job_throughput(w.T, ws, e_ms), "unit": UNIT,
                         "h2d_bytes_per_step": io_bytes, "d2h_bytes_per_step": io_bytes},
                 "gpu_launches": launches_per_step * args.steps,
                 "lib_flags": args.lib_flags,
