@@ -299,6 +299,18 @@ const char* lmoe_stage_name(int stage);
 lmoe_status lmoe_route_only_noalloc(const float* logits, int T, int N, int k, int* idx, float* w,
                                     int* offsets, int* perm, lmoe_stream_t stream);
 
+/*
+ * lmoe_selftest_wait_timeout -- test hook for the bounded waits: enqueues one
+ * kernel whose thread waits on an mbarrier that nothing arrives on; after
+ * limit_us microseconds (1 .. 1e6) the wait gives up, sets
+ * LMOE_DEVERR_WAIT_TIMEOUT in the handle's device error word and the kernel
+ * returns, leaving the context usable.  lmoe_last_error then returns
+ * LMOE_ERR_TIMEOUT.  No counterpart in the paper (a property of this
+ * implementation: no wait in the library's kernels can hang a GPU).
+ * Errors: INVALID_ARG (limit out of range), NOT_READY (no workspace), CUDA.
+ */
+lmoe_status lmoe_selftest_wait_timeout(lmoe_layer* h, unsigned limit_us, lmoe_stream_t stream);
+
 /* Kernel launches the last lmoe_forward enqueued (library kernels only). */
 int lmoe_last_launch_count(const lmoe_layer* h);
 

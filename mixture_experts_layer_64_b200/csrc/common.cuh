@@ -188,14 +188,14 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;
 // flagging the error word and the block-wide abort flag) on expiry, or
 // immediately when another thread of the block has already aborted.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          int* err) {
+                                          int* err, uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 255u) == 0) {
       if (*abort_flag) return false;
-      if (globaltimer() - t0 > kWaitLimitNs) {
+      if (globaltimer() - t0 > limit_ns) {
         *abort_flag = 1;
         set_error(err, LMOE_DEVERR_WAIT_TIMEOUT);
         return false;

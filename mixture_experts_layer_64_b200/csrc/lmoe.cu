@@ -1134,6 +1134,15 @@ lmoe_status lmoe_forward_host(lmoe_layer* h, const void* x_host, void* out_host,
   return LMOE_OK;
 }
 
+lmoe_status lmoe_selftest_wait_timeout(lmoe_layer* h, unsigned limit_us, lmoe_stream_t stream) {
+  if (!h || limit_us == 0 || limit_us > 1000000u) return LMOE_ERR_INVALID_ARG;
+  if (h->max_T == 0) return LMOE_ERR_NOT_READY;
+  DevGuard g(h->device);
+  wait_selftest_kernel<<<1, 32, 0, (cudaStream_t)stream>>>(h->err, 1000ull * limit_us);
+  LMOE_CUDA(h, cudaGetLastError());
+  return LMOE_OK;
+}
+
 lmoe_status lmoe_route_only(lmoe_layer* h, const float* logits, int T, int* idx, float* w,
                             int* offsets, int* perm, lmoe_stream_t stream) {
   if (!h) return LMOE_ERR_INVALID_ARG;

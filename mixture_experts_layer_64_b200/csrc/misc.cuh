@@ -134,6 +134,21 @@ __global__ void __launch_bounds__(256) bf16_to_f16_kernel(const bf16* __restrict
   }
 }
 
+// Self-test of the bounded waits: one thread waits on an mbarrier that no
+// one arrives on; after limit_ns the wait gives up, sets the device error
+// word (LMOE_DEVERR_WAIT_TIMEOUT) and the kernel returns.
+__global__ void wait_selftest_kernel(int* err, unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_flag, err, limit_ns);
+}
+
 // out[b][c][col0 + r] = in[b][r][c] for r < rows, c < cols: the [in, out]
 // API layout to the K-major [out, in] layout, batched over experts, with a
 // column offset so that two matrices can share one K-concatenated operand.

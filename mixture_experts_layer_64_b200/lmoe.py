@@ -32,7 +32,7 @@ EXPORTS = ["lmoe_create", "lmoe_set_weights", "lmoe_reserve", "lmoe_forward", "l
            "lmoe_last_error", "lmoe_profile_begin", "lmoe_profile_end", "lmoe_stage_name",
            "lmoe_last_launch_count", "lmoe_last_expert_path", "lmoe_status_string",
            "lmoe_error_detail", "lmoe_destroy", "lmoe_route_only_noalloc",
-           "lmoe_set_expert_weights_fp8"]
+           "lmoe_set_expert_weights_fp8", "lmoe_selftest_wait_timeout"]
 NOALLOC_MAX_WORDS = 262144
 
 
@@ -60,6 +60,7 @@ def lib() -> ctypes.CDLL:
             "lmoe_create": ([I, I, I, I, I, I, I, I, U, ctypes.POINTER(P)], I),
             "lmoe_set_weights": ([P] * 9, I),
             "lmoe_set_expert_weights_fp8": ([P] * 5, I),
+            "lmoe_selftest_wait_timeout": ([P, U, P], I),
             "lmoe_reserve": ([P, I], I),
             "lmoe_forward": ([P, P, P, I, P], I),
             "lmoe_forward_host": ([P, P, P, I, P], I),
@@ -206,6 +207,12 @@ class LatentMoELayer:
               self._dev(W2s, (N, l), torch.float32, "W2s")]
         self._check(lib().lmoe_set_expert_weights_fp8(self._h, *[_ptr(t) for t in ts]),
                     "lmoe_set_expert_weights_fp8")
+
+    def selftest_wait_timeout(self, limit_us: int, stream=None):
+        """Test hook: a device wait that nothing completes gives up after
+        limit_us and flags LMOE_DEVERR_WAIT_TIMEOUT (read with last_error)."""
+        self._check(lib().lmoe_selftest_wait_timeout(self._h, limit_us, _stream(stream)),
+                    "lmoe_selftest_wait_timeout")
 
     def reserve(self, max_T: int):
         self._check(lib().lmoe_reserve(self._h, max_T), "lmoe_reserve")

@@ -337,6 +337,21 @@ def test_host_entry_back_to_back_calls():
     assert L.last_error() == (lmoe.OK, 0)
 
 
+def test_bounded_wait_gives_up_and_reports():
+    """A device wait that nothing completes gives up after its limit, the
+    error word reads LMOE_DEVERR_WAIT_TIMEOUT (status TIMEOUT), the word is
+    cleared by reading it, and the context stays usable for a forward."""
+    w = SMALL["swiglu"]
+    L, W = gpu_layer(w)
+    x = workloads.make_x(w, device="cuda")
+    L.selftest_wait_timeout(50_000)  # 50 ms
+    assert L.last_error() == (lmoe.ERR_TIMEOUT, lmoe.DEVERR_WAIT_TIMEOUT)
+    assert L.last_error() == (lmoe.OK, 0)
+    check_forward(w, layer=L, W=W, x=x, fixture=True)
+    with pytest.raises(lmoe.LmoeError):
+        L.selftest_wait_timeout(0)
+
+
 def test_uniform_router_is_mean_of_experts():
     """W_g = 0, k = N: every token uses every expert with weight 1/N."""
     w = W_("uniform", T=64, d=128, l=64, N=4, k=4, m=64, act="relu2", seed=19)
