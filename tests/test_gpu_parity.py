@@ -258,6 +258,25 @@ def test_fp8_experts(name, flags):
         assert fc1 == 1
 
 
+def test_fp8_experts_prefill_sized():
+    """fp8 weights on the token-tiled kernel over many waves of tiles (256
+    rows per expert, several feature tiles), the E4M3 slot ring cycling."""
+    w = W_("f8-prefill", T=2048, d=1024, l=512, N=32, k=4, m=512, act="swiglu",
+           shared_m=512, seed=44, expert_fp8=True)
+    res = check_forward(w, tokens=sample_tokens(w.T, 160, seed=3))
+    assert paths(res) == (1, 1)
+    assert res["unique"] >= 0.8 * res["tokens"]
+
+
+def test_ws_pair_prefill_sized():
+    """The opt-in weight-stationary CTA-pair kernel at ~500 rows per expert
+    (several nearly equal N tiles per expert, every K block, full feature
+    tiles)."""
+    w = W_("wsp-prefill", T=2048, d=512, l=512, N=16, k=4, m=512, act="swiglu", seed=45)
+    res = check_forward(w, flags=lmoe.FORCE_WS_PAIR, tokens=sample_tokens(w.T, 160, seed=4))
+    assert paths(res) == (4, 4)
+
+
 def test_fp8_expert_api_errors():
     w = FP8["swiglu"]
     with pytest.raises(lmoe.LmoeError):  # fp8 experts need a bf16 layer
