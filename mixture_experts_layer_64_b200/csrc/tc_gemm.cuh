@@ -410,17 +410,16 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < Cfg::STAGES; ++s) {
-      // producer + gather threads + (fp8) the converters, after widening
       // the producer (its expect_tx covers the weights and the activation
       // rows, including TMA-gathered ones) + the cp.async gather threads of
-      // token-tiled tiles + (fp8) the converters, after widening
+      // token-tiled tiles + (fp8) one lane per converter warp
       mbar_init(&full[s], 1 + (Cfg::kGather && !Cfg::kSwap ? kGatherThreads : 0) +
-                              Cfg::CONV_THREADS);
+                              Cfg::CONV_THREADS / 32);
       mbar_init(&empty[s], 1);
     }
     for (int j = 0; j < Cfg::S8; ++j) {
       mbar_init(&w8full[j], 1);
-      mbar_init(&w8empty[j], Cfg::CONV_THREADS);
+      mbar_init(&w8empty[j], Cfg::CONV_THREADS / 32);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
@@ -703,9 +702,14 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
             widen_fp8_tile<Cfg::W_ROWS, Cfg::CONV_THREADS>(slot + i * Cfg::W8_BYTES,
                                                            st + Cfg::ACT_BYTES + i * Cfg::W_BYTES,
                                                            ct);
+          // each thread orders its own writes for the tensor core, then one
+          // lane per warp hands the warp's part on (8 arrivals, not 256)
           fence_proxy_async_smem();
-          mbar_arrive(&full[s]);
-          mbar_arrive(&w8empty[j]);
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(&full[s]);
+            mbar_arrive(&w8empty[j]);
+          }
           if (++s == Cfg::STAGES) { s = 0; ph ^= 1; }
           if (++j == Cfg::S8) { j = 0; jph ^= 1; }
         }
