@@ -29,7 +29,9 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
+from typing import Optional
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
@@ -100,14 +102,19 @@ class ClockSampler:
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_index: int, path: Optional[str] = None):
+        """Samples every 100 ms into `path` (a temporary file when None)."""
         self.gpu = gpu_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{gpu_index}.csv")
+        self.temporary = path is None
+        if path is None:
+            fd, path = tempfile.mkstemp(prefix=f"clocks_gpu{gpu_index}_", suffix=".csv")
+            os.close(fd)
+        self.path = path
 
     def start(self):
         try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            os.makedirs(os.path.dirname(os.path.abspath(self.path)), exist_ok=True)
             self.fh = open(self.path, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
@@ -131,6 +138,8 @@ class ClockSampler:
             for r in csv.reader(fh):
                 if len(r) >= 9:
                     rows.append([c.strip() for c in r])
+        if self.temporary:
+            os.unlink(self.path)
         if not rows:
             return None
 
@@ -337,7 +346,7 @@ def run_ours(args):
     launches_per_step = L.last_launch_count
     loads = np.diff(L.debug_dump("offsets", w.T).cpu().numpy())
 
-    sampler = ClockSampler(local) if rank == 0 else None
+    sampler = ClockSampler(local, args.clocks_csv) if rank == 0 else None
     if sampler:
         sampler.start()
     # ---- timed region: K steps, stage events recorded on the launching stream
@@ -463,6 +472,8 @@ def main():
                     help="override N (reduced cases for profiler captures)")
     ap.add_argument("--topk", type=int, default=None, help="override k")
     ap.add_argument("--tokens", type=int, default=None, help="override T")
+    ap.add_argument("--clocks-csv", default=None,
+                    help="keep the raw nvidia-smi clock samples of the timed region here")
     ap.add_argument("--lib-flags", type=int, default=0,
                     help="lmoe_create flags (e.g. 32 = never use CTA pairs) for A/B runs")
     args = ap.parse_args()

@@ -55,7 +55,7 @@ typedef enum {
   LMOE_ERR_CUDA = 3,          /* a CUDA runtime or driver call failed       */
   LMOE_ERR_OOM = 4,           /* device allocation failed                   */
   LMOE_ERR_TIMEOUT = 5,       /* a device-side bounded wait gave up         */
-  LMOE_ERR_UNSUPPORTED = 6,   /* valid but outside this build's limits      */
+  LMOE_ERR_UNSUPPORTED = 6,   /* valid but outside the library's limits     */
   LMOE_ERR_DEVICE = 7         /* a device-side check failed (error word)    */
 } lmoe_status;
 
@@ -100,7 +100,7 @@ typedef enum { LMOE_F32 = 0, LMOE_BF16 = 1 } lmoe_dtype;
                                     fp32 accumulation.  bf16 layers with l and m multiples
                                     of 64 only (else LMOE_ERR_UNSUPPORTED)   */
 
-/* Limits of this build. */
+/* Limits of the library. */
 #define LMOE_MAX_EXPERTS 1024
 #define LMOE_MAX_TOPK    32
 
