@@ -99,6 +99,17 @@ typedef enum { LMOE_F32 = 0, LMOE_BF16 = 1 } lmoe_dtype;
                                     the expert MMAs run on f16 operands with
                                     fp32 accumulation.  bf16 layers with l and m multiples
                                     of 64 only (else LMOE_ERR_UNSUPPORTED)   */
+#define LMOE_SINGLE_STREAM      0x400u /* every stage of lmoe_forward on the
+                                    caller's stream.  By default the stages
+                                    that read only x (down-projection, shared
+                                    expert FC1) run on a second stream of the
+                                    handle, forked from and joined back into
+                                    the caller's stream inside the call, so
+                                    that they overlap the router and routing
+                                    steps (separate streams for the shared
+                                    expert, the optimisation proposed in the
+                                    paper's Section 4.3 after Table 5).
+                                    Results are bitwise the same either way. */
 
 /* Limits of the library. */
 #define LMOE_MAX_EXPERTS 1024
@@ -171,7 +182,10 @@ lmoe_status lmoe_set_expert_weights_fp8(lmoe_layer* h, const void* W1q, const fl
  * lmoe_reserve -- size the workspace for up to max_T tokens per call.
  * Allocates; call it before lmoe_forward / lmoe_route_only /
  * lmoe_router_logits / lmoe_forward_host.  Calling it again with a larger
- * max_T reallocates (synchronously).  Errors: INVALID_ARG (max_T < 1), OOM.
+ * max_T reallocates (synchronously).  It also creates the handle's two
+ * internal streams (the host entry's copy stream and the forward's side
+ * stream, see LMOE_SINGLE_STREAM) and their events.  Errors: INVALID_ARG
+ * (max_T < 1), OOM, CUDA.
  */
 lmoe_status lmoe_reserve(lmoe_layer* h, int max_T);
 

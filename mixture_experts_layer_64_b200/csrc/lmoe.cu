@@ -37,6 +37,10 @@ using namespace lmoe;
 namespace {
 
 constexpr int kStages = 9;  // profiled stage count (10 boundaries)
+// events per profiled forward: the 10 stage boundaries on the caller's stream,
+// then the side stream's start, "down-projection done" and end
+constexpr int kMarks = kStages + 4;
+constexpr int kSideMark0 = kStages + 1;
 const char* kStageNames[kStages] = {"router",     "topk",       "group",   "down_proj", "shared_fc1",
                                     "expert_fc1", "expert_fc2", "combine", "up_proj"};
 
@@ -108,11 +112,18 @@ struct lmoe_layer {
   float* s32 = nullptr;  // [T, d] fp32 shared-expert output (projection-skip layers)
   float* part = nullptr;  // split-K partial sums of the dense GEMMs at small T
   size_t part_bytes = 0;
+  // the stages that read only x (down-projection, shared expert FC1) run on a
+  // second stream beside the router and routing steps: the stream, its own
+  // split-K partial buffer, and the fork and join events
+  cudaStream_t side_stream = nullptr;
+  float* part_side = nullptr;
+  cudaEvent_t ev_fork = nullptr, ev_side = nullptr;
   // bookkeeping
   int last_T = -1, launches = 0, expert_path = -1;
   std::string detail;
   // profiling
   std::vector<cudaEvent_t> events;
+  std::vector<char> prof_side;  // per profiled forward: the side stream ran
   int prof_cap = 0, prof_count = 0;
   bool profiling = false;
 };
@@ -171,6 +182,7 @@ struct GemmCall {
   bool swap;    // weight-stationary expert kernels
   bool pair;    // 2-SM token-tiled kernels on CTA pairs (256-row tiles)
   bool ws_pair;  // grouped: weight-stationary kernel on CTA pairs (rows on N)
+  bool side;     // enqueued on the side stream: split-K uses the side partial buffer
 };
 
 bool encode_map(CUtensorMap* map, const void* ptr, long rows, int cols, long ld, int box_rows) {
@@ -412,8 +424,12 @@ constexpr size_t kSplitPartBytes = 32u << 20;
 
 // Number of K ranges for a dense single-CTA call (1: no split), and the
 // 64-wide K blocks per range.
+float* part_buffer(const lmoe_layer* h, const GemmCall& c) {
+  return c.side ? h->part_side : h->part;
+}
+
 int choose_splits(const lmoe_layer* h, const GemmCall& c, int& kbs) {
-  if (c.pair || c.swap || c.p.offsets || !h->part) return 1;
+  if (c.pair || c.swap || c.p.offsets || !part_buffer(h, c)) return 1;
   const bool dual = c.p.dual_offset > 0;
   if (dual && c.p.dual_offset != c.p.F) return 1;  // gate and linear rows must be adjacent
   const int Fp = dual ? 2 * c.p.F : c.p.F;
@@ -436,7 +452,8 @@ lmoe_status run_split(lmoe_layer* h, const GemmCall& c, int S, int kbs, cudaStre
   g.p.F = Fp;
   g.p.dual_offset = 0;
   std::memset(&g.p.epi, 0, sizeof g.p.epi);
-  g.p.epi.out = h->part;
+  float* part = part_buffer(h, c);
+  g.p.epi.out = part;
   g.p.epi.ldo = Fp;
   g.p.epi.slice = (long)c.p.M * Fp;
   g.p.splits = S;
@@ -446,7 +463,7 @@ lmoe_status run_split(lmoe_layer* h, const GemmCall& c, int S, int kbs, cudaStre
   const int kind = c.kind == GK_ROUTER ? EPI_F32_BIAS : c.kind == GK_UP ? EPI_RESID : EPI_ACT;
   const long n = (long)c.p.M * c.p.F;
   splitk_reduce_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(
-      h->part, S, g.p.epi.slice, c.p.M, c.p.F, Fp, dual ? c.p.F : 0, kind, c.p.epi);
+      part, S, g.p.epi.slice, c.p.M, c.p.F, Fp, dual ? c.p.F : 0, kind, c.p.epi);
   LMOE_CHECK_LAUNCH(h);
   return LMOE_OK;
 }
@@ -613,7 +630,7 @@ bool use_swap(const lmoe_layer* h, int T) {
 
 void prof_mark(lmoe_layer* h, cudaStream_t st, int i) {
   if (h->profiling && h->prof_count < h->prof_cap)
-    cudaEventRecord(h->events[(size_t)h->prof_count * (kStages + 1) + i], st);
+    cudaEventRecord(h->events[(size_t)h->prof_count * kMarks + i], st);
 }
 
 // ---- the routing steps ---------------------------------------------------------
@@ -654,17 +671,56 @@ lmoe_status run_router(lmoe_layer* h, const void* x, float* logits, int T, cudaS
   return run_gemm(h, c, st);
 }
 
+// The stages that read only x: the down-projection z = x Wdown and the shared
+// expert's FC1 (with the projection-skip layout, also its FC2 in fp32), on
+// stream s.  Marks m_z and m_end are recorded after the down-projection and
+// at the end; on the side stream, ev_side at the end as well.
+lmoe_status run_x_stages(lmoe_layer* h, const void* x, int T, bool pair_dense, bool side,
+                         cudaStream_t s, int m_z, int m_end) {
+  const bool skip = (h->flags & LMOE_SKIP_PROJ) != 0;
+  const int d = h->d, l = h->l, ms = h->shared_m;
+  if (!skip) {
+    GemmCall c = dense_call(GK_DENSE_ACT, T, x, d, h->Wd_t, l, d);
+    c.side = side;
+    c.p.epi.out = h->z;
+    c.p.epi.ldo = l;
+    if (pair_dense) make_pair(h, c);
+    LMOE_TRY(run_gemm(h, c, s));
+  }
+  prof_mark(h, s, m_z);
+  if (ms > 0) {
+    GemmCall c = dense_call(GK_DENSE_ACT, T, x, d, h->Ws1_t, ms, d);
+    c.side = side;
+    c.b_rows = h->ms_in;
+    c.p.dual_offset = h->act == LMOE_ACT_SWIGLU ? ms : 0;
+    c.p.epi.out = h->cat;
+    c.p.epi.ldo = h->Kup;
+    c.p.epi.col0 = skip ? 0 : l;
+    c.p.epi.act = h->act;
+    c.p.epi.split_off = h->split_shared ? ms : 0;
+    if (pair_dense) make_pair(h, c);
+    LMOE_TRY(run_gemm(h, c, s));
+    if (skip) {
+      // no up-projection GEMM to carry it: s = hs Ws2 in fp32, added by the
+      // combine before the output's single rounding
+      GemmCall c2 = dense_call(GK_ROUTER, T, h->cat, h->Kup, h->Wu_t, d, h->Kup);
+      c2.side = side;
+      c2.p.epi.out = h->s32;
+      c2.p.epi.ldo = d;
+      c2.p.epi.bias = nullptr;
+      LMOE_TRY(run_gemm(h, c2, s));
+    }
+  }
+  if (side) LMOE_CUDA(h, cudaEventRecord(h->ev_side, s));
+  prof_mark(h, s, m_end);
+  return LMOE_OK;
+}
+
 lmoe_status run_forward(lmoe_layer* h, const void* x, void* out, int T, cudaStream_t st) {
   h->launches = 0;
   const bool skip = (h->flags & LMOE_SKIP_PROJ) != 0;
   const int d = h->d, l = h->l, k = h->k, m = h->m, ms = h->shared_m;
   const long R = (long)T * k;
-  prof_mark(h, st, 0);
-  LMOE_TRY(run_router(h, x, h->logits, T, st));
-  prof_mark(h, st, 1);
-  LMOE_TRY(run_routing(h, h->logits, T, h->idx, h->w, h->offsets, h->row_tok, h->row_slot,
-                       h->row_w, h->slot_row, h->tile_prefix2, st, true));
-  prof_mark(h, st, 3);
   const bool swap = use_swap(h, T);
   const bool pairs_ok = h->dtype == LMOE_BF16 && !(h->flags & (LMOE_FORCE_SIMT | LMOE_FORCE_NOPAIR));
   // CTA pairs for the dense GEMMs once there are enough rows to fill them,
@@ -676,36 +732,33 @@ lmoe_status run_forward(lmoe_layer* h, const void* x, void* out, int T, cudaStre
   // MMA's N, so an expert's last tile is padded to 16 rows, not 128 or 256)
   const bool ws_pair = pairs_ok && !swap && (h->flags & LMOE_FORCE_WS_PAIR) &&
                        !(h->flags & LMOE_FORCE_NOSWAP);
-  if (!skip) {
-    GemmCall c = dense_call(GK_DENSE_ACT, T, x, d, h->Wd_t, l, d);
-    c.p.epi.out = h->z;
-    c.p.epi.ldo = l;
-    if (pair_dense) make_pair(h, c);
-    LMOE_TRY(run_gemm(h, c, st));
+  // The down-projection and the shared FC1 depend on x alone: forked onto the
+  // side stream they overlap the router GEMM and the latency-bound routing
+  // kernels (which fit on an SM beside a GEMM CTA).  st waits for the whole
+  // side stream before the expert FC1: a shared FC1 still running beside the
+  // persistent expert FC1 would hold SMs that some of its CTAs need, and
+  // those CTAs' tiles would finish last.
+  const bool side = h->side_stream && !(h->flags & LMOE_SINGLE_STREAM) && (!skip || ms > 0);
+  if (h->profiling && h->prof_count < h->prof_cap) h->prof_side[h->prof_count] = side ? 1 : 0;
+  prof_mark(h, st, 0);
+  if (side) {
+    LMOE_CUDA(h, cudaEventRecord(h->ev_fork, st));
+    LMOE_CUDA(h, cudaStreamWaitEvent(h->side_stream, h->ev_fork, 0));
+    prof_mark(h, h->side_stream, kSideMark0);
+    LMOE_TRY(run_x_stages(h, x, T, pair_dense, true, h->side_stream, kSideMark0 + 1,
+                          kSideMark0 + 2));
   }
-  prof_mark(h, st, 4);
-  if (ms > 0) {
-    GemmCall c = dense_call(GK_DENSE_ACT, T, x, d, h->Ws1_t, ms, d);
-    c.b_rows = h->ms_in;
-    c.p.dual_offset = h->act == LMOE_ACT_SWIGLU ? ms : 0;
-    c.p.epi.out = h->cat;
-    c.p.epi.ldo = h->Kup;
-    c.p.epi.col0 = skip ? 0 : l;
-    c.p.epi.act = h->act;
-    c.p.epi.split_off = h->split_shared ? ms : 0;
-    if (pair_dense) make_pair(h, c);
-    LMOE_TRY(run_gemm(h, c, st));
-    if (skip) {
-      // no up-projection GEMM to carry it: s = hs Ws2 in fp32, added by the
-      // combine before the output's single rounding
-      GemmCall c2 = dense_call(GK_ROUTER, T, h->cat, h->Kup, h->Wu_t, d, h->Kup);
-      c2.p.epi.out = h->s32;
-      c2.p.epi.ldo = d;
-      c2.p.epi.bias = nullptr;
-      LMOE_TRY(run_gemm(h, c2, st));
-    }
+  LMOE_TRY(run_router(h, x, h->logits, T, st));
+  prof_mark(h, st, 1);
+  LMOE_TRY(run_routing(h, h->logits, T, h->idx, h->w, h->offsets, h->row_tok, h->row_slot,
+                       h->row_w, h->slot_row, h->tile_prefix2, st, true));
+  prof_mark(h, st, 3);
+  if (side) {
+    LMOE_CUDA(h, cudaStreamWaitEvent(st, h->ev_side, 0));
+    prof_mark(h, st, 5);
+  } else {
+    LMOE_TRY(run_x_stages(h, x, T, pair_dense, false, st, 4, 5));
   }
-  prof_mark(h, st, 5);
   {
     const void* A = skip ? x : h->z;
     const bool fp8 = (h->flags & LMOE_EXPERTS_FP8) != 0;
@@ -836,6 +889,13 @@ void free_workspace(lmoe_layer* h) {
   }
   if (h->copy_stream) cudaStreamDestroy(h->copy_stream);
   h->copy_stream = nullptr;
+  for (cudaEvent_t* e : {&h->ev_fork, &h->ev_side}) {
+    if (*e) cudaEventDestroy(*e);
+    *e = nullptr;
+  }
+  if (h->side_stream) cudaStreamDestroy(h->side_stream);
+  h->side_stream = nullptr;
+  free_ptr(h->part_side);
   h->host_slot = 0;
   free_ptr(h->s32);
   free_ptr(h->a16);
@@ -920,7 +980,8 @@ lmoe_status lmoe_create(int d, int l, int N, int k, int m, lmoe_act act, int sha
   *out = nullptr;
   const unsigned known = LMOE_SKIP_PROJ | LMOE_DEBUG_CHECKS | LMOE_FORCE_SIMT | LMOE_FORCE_SWAP |
                          LMOE_FORCE_NOSWAP | LMOE_FORCE_NOPAIR | LMOE_FORCE_WS_PAIR |
-                         LMOE_ROUTE_FULL_SOFTMAX | LMOE_ROUTE_BIAS_SELECT | LMOE_EXPERTS_FP8;
+                         LMOE_ROUTE_FULL_SOFTMAX | LMOE_ROUTE_BIAS_SELECT | LMOE_EXPERTS_FP8 |
+                         LMOE_SINGLE_STREAM;
   if (d <= 0 || l <= 0 || N <= 0 || k <= 0 || m <= 0 || shared_m < 0) return LMOE_ERR_INVALID_ARG;
   if (k > N || (flags & ~known)) return LMOE_ERR_INVALID_ARG;
   if (act != LMOE_ACT_SILU && act != LMOE_ACT_SWIGLU && act != LMOE_ACT_RELU2) return LMOE_ERR_INVALID_ARG;
@@ -1081,7 +1142,11 @@ lmoe_status lmoe_reserve(lmoe_layer* h, int max_T) {
   if (h->dtype == LMOE_BF16) {
     h->part_bytes = kSplitPartBytes;
     ALLOC(h->part, h->part_bytes);
+    ALLOC(h->part_side, h->part_bytes);
   }
+  LMOE_CUDA(h, cudaStreamCreateWithFlags(&h->side_stream, cudaStreamNonBlocking));
+  for (cudaEvent_t* e : {&h->ev_fork, &h->ev_side})
+    LMOE_CUDA(h, cudaEventCreateWithFlags(e, cudaEventDisableTiming));
 #undef ALLOC
   LMOE_CUDA(h, cudaMemset(h->bitmap, 0, (size_t)h->N * W * sizeof(uint32_t)));
   LMOE_CUDA(h, cudaMemset(h->done, 0, sizeof(unsigned)));
@@ -1252,8 +1317,9 @@ lmoe_status lmoe_profile_begin(lmoe_layer* h, int max_forwards) {
   DevGuard g(h->device);
   LMOE_CUDA(h, cudaDeviceSynchronize());
   destroy_events(h);
-  const size_t n = (size_t)max_forwards * (kStages + 1);
+  const size_t n = (size_t)max_forwards * kMarks;
   h->events.resize(n, nullptr);
+  h->prof_side.assign((size_t)max_forwards, 0);
   for (size_t i = 0; i < n; ++i) {
     cudaError_t e = cudaEventCreate(&h->events[i]);
     if (e != cudaSuccess) {
@@ -1278,10 +1344,17 @@ lmoe_status lmoe_profile_end(lmoe_layer* h, float* ms, int capacity, int* n_forw
   int written = 0;
   for (int f = 0; f < h->prof_count; ++f) {
     if ((f + 1) * kStages > capacity) break;
+    cudaEvent_t* ev = &h->events[(size_t)f * kMarks];
     for (int s = 0; s < kStages; ++s) {
+      // with the side stream, the down-projection and shared FC1 stages are
+      // timed there (they overlap the router and routing stages)
+      int a = s, b = s + 1;
+      if (h->prof_side[f] && (s == 3 || s == 4)) {
+        a = kSideMark0 + (s - 3);
+        b = a + 1;
+      }
       float t = 0.f;
-      cudaEvent_t* ev = &h->events[(size_t)f * (kStages + 1)];
-      LMOE_CUDA(h, cudaEventElapsedTime(&t, ev[s], ev[s + 1]));
+      LMOE_CUDA(h, cudaEventElapsedTime(&t, ev[a], ev[b]));
       ms[f * kStages + s] = t;
     }
     written = f + 1;

@@ -229,6 +229,69 @@ def test_split_k_dense_gemms_at_decode_size(skip):
 
 
 # ---------------------------------------------------------------------------
+# the x-only stages on a second stream
+# ---------------------------------------------------------------------------
+
+SIDE = {
+    # split-K dense GEMMs on both streams at once (router on the caller's
+    # stream; down-projection and gated shared FC1 on the side stream)
+    "split": W_("side-split", T=40, d=1024, l=512, N=16, k=4, m=128, act="swiglu",
+                shared_m=256, bias="normal0.5", seed=31),
+    # projection-skip layer: the side stream carries the shared FC1 and its
+    # fp32 FC2, which the combine adds
+    "skip": W_("side-skip", T=40, d=1024, l=1024, N=16, k=4, m=128, act="swiglu",
+               shared_m=256, skip_proj=True, seed=32),
+    # CTA-pair dense GEMMs on both streams, ragged last row tile
+    "pairs": W_("side-pairs", T=1100, d=256, l=192, N=16, k=4, m=320, act="relu2",
+                shared_m=256, seed=33),
+    # no shared expert: only the down-projection moves
+    "no-shared": W_("side-noshared", T=300, d=256, l=128, N=8, k=3, m=192, act="swiglu",
+                    seed=34),
+}
+
+
+@pytest.mark.parametrize("name", list(SIDE))
+def test_side_stream_matches_single_stream(name):
+    """By default the down-projection and the shared FC1 run on a second
+    stream beside the router and routing steps; LMOE_SINGLE_STREAM keeps
+    every stage on the caller's stream.  The two orders give bitwise the same
+    output, also over back-to-back forwards with no synchronisation between
+    them, and the default order matches the oracle."""
+    w = SIDE[name]
+    res = check_forward(w, fixture=True, tokens=sample_tokens(w.T, 200, seed=3))
+    assert res["unique"] >= 0.9 * res["tokens"]
+    W = workloads.make_weights(w, device="cuda")
+    A, _ = gpu_layer(w, 0, W)
+    B, _ = gpu_layer(w, lmoe.SINGLE_STREAM, W)
+    x0 = workloads.make_x(w, device="cuda").float()
+    xs = [(x0 * (1.0 + 0.5 * i)).roll(3 * i, dims=0).to(torch.bfloat16).contiguous()
+          for i in range(3)]
+    outs_a = [A.forward(x) for x in xs]  # enqueued back to back
+    outs_b = [B.forward(x) for x in xs]
+    torch.cuda.synchronize()
+    for a, b in zip(outs_a, outs_b):
+        assert torch.equal(a, b)
+    assert A.last_error() == (lmoe.OK, 0) and B.last_error() == (lmoe.OK, 0)
+
+
+def test_side_stream_profile_stages():
+    """Profiled forwards time the side stream's two stages on that stream:
+    every stage time is non-negative and the down-projection and shared FC1
+    are not empty."""
+    w = SIDE["pairs"]
+    L, W = gpu_layer(w)
+    x = workloads.make_x(w, device="cuda")
+    L.profile_begin(2)
+    for _ in range(2):
+        L.forward(x)
+    prof = L.profile_end()
+    assert len(prof) == 2
+    for p in prof:
+        assert all(v >= 0 for v in p.values())
+        assert p["down_proj"] > 0 and p["shared_fc1"] > 0
+
+
+# ---------------------------------------------------------------------------
 # fp8 E4M3 expert weights (codes + per-output-channel scales)
 # ---------------------------------------------------------------------------
 
