@@ -110,6 +110,13 @@ typedef enum { LMOE_F32 = 0, LMOE_BF16 = 1 } lmoe_dtype;
                                     expert, the optimisation proposed in the
                                     paper's Section 4.3 after Table 5).
                                     Results are bitwise the same either way. */
+#define LMOE_NO_PDL             0x800u /* launch the forward's kernels without
+                                    programmatic dependent launch.  By
+                                    default each kernel may be scheduled
+                                    while its predecessor on the stream
+                                    drains, sets up its barriers and tensor
+                                    memory, and waits for the predecessor's
+                                    writes before its first global access. */
 
 /* Limits of the library. */
 #define LMOE_MAX_EXPERTS 1024

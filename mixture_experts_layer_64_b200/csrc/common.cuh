@@ -154,6 +154,41 @@ __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
                : "memory");
 }
 
+// ---- programmatic dependent launch ----------------------------------------------
+//
+// The forward's kernels are launched with programmatic stream serialisation:
+// a kernel may be scheduled while its predecessor on the stream still runs,
+// do its set-up that touches no global memory (barrier init, TMEM allocation,
+// tensor-map prefetch), and then wait in griddep_wait until the predecessor
+// has completed and its writes are visible.  Every kernel calls griddep_wait
+// before its first global load or store; launched without the attribute, the
+// wait returns at once.  griddep_launch lets the next kernel be scheduled once
+// every CTA of this grid has issued it (all of them are then resident), so a
+// waiting successor never holds resources this grid still needs.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Launches kernel `kern` on stream st, with programmatic stream serialisation
+// when pdl is set (the kernel must then call griddep_wait before touching
+// global memory, as every forward kernel does).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_kernel(bool pdl, void (*kern)(KArgs...), dim3 grid, dim3 block,
+                                 size_t smem, cudaStream_t st, Args... args) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 __device__ __forceinline__ void fence_barrier_init() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }

@@ -70,6 +70,9 @@ struct lmoe_layer {
   unsigned flags;
   int m_in, ms_in, Kup, es;  // es: element size
   bool split_shared = false;  // bf16 shared hidden carried as a hi + lo pair
+  bool pdl = true;            // forward kernels with programmatic dependent launch
+  bool pdl_hold = false;      // the next launch follows a cross-stream wait (or opens a
+                              // forward): launched with the full stream dependency
   int device = 0, num_sms = 148;
   bool weights_set = false;
   // weights, K-major
@@ -160,6 +163,15 @@ lmoe_status cuda_fail(lmoe_layer* h, cudaError_t e, const char* what) {
     if (e_ != cudaSuccess) return cuda_fail((h), e_, #call); \
   } while (0)
 
+// A launch through launch_kernel (forward kernels: programmatic stream
+// serialisation unless LMOE_NO_PDL).
+#define LMOE_LAUNCH(h, ...)                                             \
+  do {                                                                  \
+    cudaError_t e_ = launch_kernel(take_pdl(h), __VA_ARGS__);           \
+    if (e_ != cudaSuccess) return cuda_fail((h), e_, "kernel launch"); \
+    ++(h)->launches;                                                    \
+  } while (0)
+
 #define LMOE_CHECK_LAUNCH(h)                                           \
   do {                                                                 \
     cudaError_t e_ = cudaGetLastError();                               \
@@ -168,6 +180,15 @@ lmoe_status cuda_fail(lmoe_layer* h, cudaError_t e, const char* what) {
   } while (0)
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+// Whether the next launch may use programmatic dependent launch; a pending
+// hold (set after a cross-stream wait and at the start of a forward) makes
+// that one launch wait for everything before it on its stream.
+bool take_pdl(lmoe_layer* h) {
+  const bool use = h->pdl && !h->pdl_hold;
+  h->pdl_hold = false;
+  return use;
+}
 
 // ---- GEMM dispatch --------------------------------------------------------------
 
@@ -271,8 +292,8 @@ lmoe_status launch_tc(lmoe_layer* h, const GemmCall& c, cudaStream_t st) {
   const long NT = (c.p.F + Cfg::FT - 1) / Cfg::FT;
   const long tiles = (long)c.p.max_row_tiles * NT * std::max(1, c.p.splits);
   const int grid = (int)std::max(1L, std::min<long>(h->num_sms, tiles));
-  tc_gemm_kernel<Cfg><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, st>>>(ta, tb, tc, p);
-  LMOE_CHECK_LAUNCH(h);
+  LMOE_LAUNCH(h, tc_gemm_kernel<Cfg>, dim3(grid), dim3(Cfg::THREADS), Cfg::SMEM_BYTES, st, ta, tb,
+              tc, p);
   return LMOE_OK;
 }
 
@@ -300,22 +321,25 @@ lmoe_status pair_setup(lmoe_layer* h, Kern kern, int smem_bytes, int* max_cluste
   return LMOE_OK;
 }
 
-// Launches `clusters` CTA pairs of a 2-SM kernel.
+// Launches `clusters` CTA pairs of a 2-SM kernel (programmatic stream
+// serialisation unless LMOE_NO_PDL).
 template <typename Kern, typename... Args>
 lmoe_status pair_launch(lmoe_layer* h, Kern kern, int smem_bytes, long clusters, cudaStream_t st,
                         Args... args) {
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.gridDim = dim3((unsigned)(2 * clusters), 1, 1);
   cfg.blockDim = dim3(kTcThreads, 1, 1);
   cfg.dynamicSmemBytes = smem_bytes;
   cfg.stream = st;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = take_pdl(h) ? 2 : 1;
   LMOE_CUDA(h, cudaLaunchKernelEx(&cfg, kern, args...));
   ++h->launches;
   return LMOE_OK;
@@ -374,8 +398,7 @@ lmoe_status launch_simt(lmoe_layer* h, const GemmCall& c, cudaStream_t st) {
   const long NT = (c.p.F + kSimtTN - 1) / kSimtTN;
   const long blocks = (long)c.p.max_row_tiles * NT;
   if (blocks <= 0) return LMOE_OK;
-  simt_gemm_kernel<T, kDual, kEpi><<<(unsigned)blocks, 256, 0, st>>>(c.p);
-  LMOE_CHECK_LAUNCH(h);
+  LMOE_LAUNCH(h, simt_gemm_kernel<T, kDual, kEpi>, dim3((unsigned)blocks), dim3(256), 0, st, c.p);
   return LMOE_OK;
 }
 
@@ -462,9 +485,9 @@ lmoe_status run_split(lmoe_layer* h, const GemmCall& c, int S, int kbs, cudaStre
   LMOE_TRY((launch_tc<TcCfg<false, false, false, 128, EPI_F32_BIAS>>(h, g, st)));
   const int kind = c.kind == GK_ROUTER ? EPI_F32_BIAS : c.kind == GK_UP ? EPI_RESID : EPI_ACT;
   const long n = (long)c.p.M * c.p.F;
-  splitk_reduce_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(
-      part, S, g.p.epi.slice, c.p.M, c.p.F, Fp, dual ? c.p.F : 0, kind, c.p.epi);
-  LMOE_CHECK_LAUNCH(h);
+  LMOE_LAUNCH(h, splitk_reduce_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, st,
+              (const float*)part, S, g.p.epi.slice, c.p.M, c.p.F, Fp, dual ? c.p.F : 0, kind,
+              c.p.epi);
   return LMOE_OK;
 }
 
@@ -644,20 +667,18 @@ lmoe_status run_routing(lmoe_layer* h, const float* logits, int T, int* idx, flo
     const float* sel_bias = (h->flags & LMOE_ROUTE_BIAS_SELECT) ? h->bias : nullptr;
     const int full = (h->flags & LMOE_ROUTE_FULL_SOFTMAX) ? 1 : 0;
     const cudaError_t e = launch_topk(logits, T, h->N, h->k, sel_bias, full, idx, w, h->bitmap,
-                                      W, debug, h->err, st);
+                                      W, debug, h->err, st, take_pdl(h));
     if (e != cudaSuccess) return cuda_fail(h, e, "top-k launch");
     ++h->launches;
   }
   if (marks) prof_mark(h, st, 2);
-  group_count_kernel<<<(h->N + 7) / 8, 256, 0, st>>>(h->bitmap, h->wp, h->N, W, h->counts, offsets,
-                                                     h->tile_prefix, tile_prefix2,
-                                                     tile_prefix2 ? h->tile_prefix64 : nullptr,
-                                                     h->done);
-  LMOE_CHECK_LAUNCH(h);
+  LMOE_LAUNCH(h, group_count_kernel, dim3((h->N + 7) / 8), dim3(256), 0, st, h->bitmap, h->wp,
+              h->N, W, h->counts, offsets, h->tile_prefix, tile_prefix2,
+              tile_prefix2 ? h->tile_prefix64 : (int*)nullptr, h->done);
   const long P = (long)T * h->k;
-  group_rank_kernel<<<(unsigned)((P + 255) / 256), 256, 0, st>>>(
-      idx, w, h->wp, offsets, T, h->k, h->N, W, row_tok, row_slot, row_w, slot_row, debug, h->err);
-  LMOE_CHECK_LAUNCH(h);
+  LMOE_LAUNCH(h, group_rank_kernel, dim3((unsigned)((P + 255) / 256)), dim3(256), 0, st,
+              (const int*)idx, (const float*)w, (const uint2*)h->wp, (const int*)offsets, T, h->k,
+              h->N, W, row_tok, row_slot, row_w, slot_row, debug, h->err);
   return LMOE_OK;
 }
 
@@ -745,9 +766,11 @@ lmoe_status run_forward(lmoe_layer* h, const void* x, void* out, int T, cudaStre
     LMOE_CUDA(h, cudaEventRecord(h->ev_fork, st));
     LMOE_CUDA(h, cudaStreamWaitEvent(h->side_stream, h->ev_fork, 0));
     prof_mark(h, h->side_stream, kSideMark0);
+    h->pdl_hold = true;
     LMOE_TRY(run_x_stages(h, x, T, pair_dense, true, h->side_stream, kSideMark0 + 1,
                           kSideMark0 + 2));
   }
+  h->pdl_hold = true;
   LMOE_TRY(run_router(h, x, h->logits, T, st));
   prof_mark(h, st, 1);
   LMOE_TRY(run_routing(h, h->logits, T, h->idx, h->w, h->offsets, h->row_tok, h->row_slot,
@@ -755,6 +778,7 @@ lmoe_status run_forward(lmoe_layer* h, const void* x, void* out, int T, cudaStre
   prof_mark(h, st, 3);
   if (side) {
     LMOE_CUDA(h, cudaStreamWaitEvent(st, h->ev_side, 0));
+    h->pdl_hold = true;
     prof_mark(h, st, 5);
   } else {
     LMOE_TRY(run_x_stages(h, x, T, pair_dense, false, st, 4, 5));
@@ -769,9 +793,8 @@ lmoe_status run_forward(lmoe_layer* h, const void* x, void* out, int T, cudaStre
       const long work = vec ? n / 8 : n;
       const unsigned blocks = (unsigned)std::max<long>(1, std::min<long>((work + 255) / 256,
                                                                           8L * h->num_sms));
-      bf16_to_f16_kernel<<<blocks, 256, 0, st>>>(static_cast<const bf16*>(A),
-                                                 static_cast<__half*>(h->a16), n, vec);
-      LMOE_CHECK_LAUNCH(h);
+      LMOE_LAUNCH(h, bf16_to_f16_kernel, dim3(blocks), dim3(256), 0, st,
+                  static_cast<const bf16*>(A), static_cast<__half*>(h->a16), n, vec);
       A = h->a16;
     }
     GemmCall c = grouped_call(h, GK_FC1, T, A, skip ? d : l, T, h->row_tok,
@@ -818,23 +841,24 @@ lmoe_status run_forward(lmoe_layer* h, const void* x, void* out, int T, cudaStre
     const int chunks = std::max(1, std::min((l + per_block - 1) / per_block,
                                             (2 * h->num_sms + T - 1) / std::max(T, 1)));
     const dim3 cgrid((unsigned)T, (unsigned)chunks);
+    const long ldr = d;
     if (h->dtype == LMOE_BF16) {
       if (vec_ok)
-        combine_kernel<bf16><<<cgrid, threads, 0, st>>>((const bf16*)h->ys, h->slot_row, k, l,
-                                                        (const bf16*)resid, d, add32, (bf16*)dst,
-                                                        ldo);
+        LMOE_LAUNCH(h, combine_kernel<bf16>, cgrid, dim3(threads), 0, st, (const bf16*)h->ys,
+                    (const int*)h->slot_row, k, l, (const bf16*)resid, ldr, add32, (bf16*)dst, ldo);
       else
-        combine_scalar_kernel<bf16><<<T, 256, 0, st>>>((const bf16*)h->ys, h->slot_row, k, l,
-                                                       (const bf16*)resid, d, add32, (bf16*)dst, ldo);
+        LMOE_LAUNCH(h, combine_scalar_kernel<bf16>, dim3(T), dim3(256), 0, st, (const bf16*)h->ys,
+                    (const int*)h->slot_row, k, l, (const bf16*)resid, ldr, add32, (bf16*)dst, ldo);
     } else {
       if (vec_ok)
-        combine_kernel<float><<<cgrid, threads, 0, st>>>((const float*)h->ys, h->slot_row, k, l,
-                                                     (const float*)resid, d, add32, (float*)dst, ldo);
+        LMOE_LAUNCH(h, combine_kernel<float>, cgrid, dim3(threads), 0, st, (const float*)h->ys,
+                    (const int*)h->slot_row, k, l, (const float*)resid, ldr, add32, (float*)dst,
+                    ldo);
       else
-        combine_scalar_kernel<float><<<T, 256, 0, st>>>((const float*)h->ys, h->slot_row, k, l,
-                                                        (const float*)resid, d, add32, (float*)dst, ldo);
+        LMOE_LAUNCH(h, combine_scalar_kernel<float>, dim3(T), dim3(256), 0, st,
+                    (const float*)h->ys, (const int*)h->slot_row, k, l, (const float*)resid, ldr,
+                    add32, (float*)dst, ldo);
     }
-    LMOE_CHECK_LAUNCH(h);
   }
   prof_mark(h, st, 8);
   if (!skip) {
@@ -981,7 +1005,7 @@ lmoe_status lmoe_create(int d, int l, int N, int k, int m, lmoe_act act, int sha
   const unsigned known = LMOE_SKIP_PROJ | LMOE_DEBUG_CHECKS | LMOE_FORCE_SIMT | LMOE_FORCE_SWAP |
                          LMOE_FORCE_NOSWAP | LMOE_FORCE_NOPAIR | LMOE_FORCE_WS_PAIR |
                          LMOE_ROUTE_FULL_SOFTMAX | LMOE_ROUTE_BIAS_SELECT | LMOE_EXPERTS_FP8 |
-                         LMOE_SINGLE_STREAM;
+                         LMOE_SINGLE_STREAM | LMOE_NO_PDL;
   if (d <= 0 || l <= 0 || N <= 0 || k <= 0 || m <= 0 || shared_m < 0) return LMOE_ERR_INVALID_ARG;
   if (k > N || (flags & ~known)) return LMOE_ERR_INVALID_ARG;
   if (act != LMOE_ACT_SILU && act != LMOE_ACT_SWIGLU && act != LMOE_ACT_RELU2) return LMOE_ERR_INVALID_ARG;
@@ -1001,6 +1025,7 @@ lmoe_status lmoe_create(int d, int l, int N, int k, int m, lmoe_act act, int sha
   lmoe_layer* h = new lmoe_layer();
   h->d = d; h->l = l; h->N = N; h->k = k; h->m = m; h->act = act; h->shared_m = shared_m;
   h->dtype = dtype; h->flags = flags;
+  h->pdl = (flags & LMOE_NO_PDL) == 0;
   h->m_in = act == LMOE_ACT_SWIGLU ? 2 * m : m;
   h->ms_in = act == LMOE_ACT_SWIGLU ? 2 * shared_m : shared_m;
   // bf16: the shared expert's hidden activations go into the up-projection as
@@ -1222,6 +1247,7 @@ lmoe_status lmoe_route_only(lmoe_layer* h, const float* logits, int T, int* idx,
     LMOE_CUDA(h, cudaMemsetAsync(offsets, 0, (size_t)(h->N + 1) * sizeof(int), st));
     return LMOE_OK;
   }
+  h->pdl_hold = true;
   return run_routing(h, logits, T, idx, w, offsets, nullptr, perm, nullptr, nullptr, nullptr, st,
                      false);
 }
@@ -1235,6 +1261,7 @@ lmoe_status lmoe_router_logits(lmoe_layer* h, const void* x, float* logits, int 
   if (!x || !logits) return LMOE_ERR_INVALID_ARG;
   DevGuard g(h->device);
   h->launches = 0;
+  h->pdl_hold = true;
   return run_router(h, x, logits, T, (cudaStream_t)stream);
 }
 

@@ -20,6 +20,8 @@ __global__ void __launch_bounds__(256) combine_kernel(const T* __restrict__ ys,
                                                       int l, const T* __restrict__ resid, long ldr,
                                                       const float* __restrict__ add32,
                                                       T* __restrict__ out, long ldo) {
+  griddep_launch();
+  griddep_wait();  // the previous kernel's outputs are visible
   constexpr int VEC = 16 / sizeof(T);
   const int t = blockIdx.x;
   const int* rows = slot_row + (size_t)t * k;
@@ -61,6 +63,8 @@ __global__ void __launch_bounds__(256) combine_scalar_kernel(const T* __restrict
                                                              const T* __restrict__ resid, long ldr,
                                                              const float* __restrict__ add32,
                                                              T* __restrict__ out, long ldo) {
+  griddep_launch();
+  griddep_wait();  // the previous kernel's outputs are visible
   const int t = blockIdx.x;
   for (int c = threadIdx.x; c < l; c += blockDim.x) {
     float acc = resid ? to_f32<T>(resid[(size_t)t * ldr + c]) : 0.f;
@@ -83,6 +87,8 @@ __global__ void __launch_bounds__(256) combine_scalar_kernel(const T* __restrict
 __global__ void __launch_bounds__(256) splitk_reduce_kernel(const float* __restrict__ part, int S,
                                                             long slice, int M, int F, int Fp,
                                                             int dual, int kind, EpiParams e) {
+  griddep_launch();
+  griddep_wait();  // the previous kernel's outputs are visible
   const long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= (long)M * F) return;
   const int row = (int)(i / F), f = (int)(i - (long)row * F);
@@ -113,6 +119,8 @@ __global__ void __launch_bounds__(256) splitk_reduce_kernel(const float* __restr
 __global__ void __launch_bounds__(256) bf16_to_f16_kernel(const bf16* __restrict__ in,
                                                           __half* __restrict__ out, long n,
                                                           int vec) {
+  griddep_launch();
+  griddep_wait();  // the previous kernel's outputs are visible
   const long i0 = ((long)blockIdx.x * blockDim.x + threadIdx.x) * (vec ? 8 : 1);
   const long stride = (long)gridDim.x * blockDim.x * (vec ? 8 : 1);
   for (long i = i0; i < n; i += stride) {

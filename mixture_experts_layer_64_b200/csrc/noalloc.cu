@@ -93,7 +93,7 @@ extern "C" lmoe_status lmoe_route_only_noalloc(const float* logits, int T, int N
   if (cudaMemsetAsync(bitmap, 0, (size_t)N * W * sizeof(uint32_t), s) != cudaSuccess ||
       cudaMemsetAsync(done, 0, sizeof(unsigned), s) != cudaSuccess)
     return LMOE_ERR_CUDA;
-  launch_topk(logits, T, N, k, nullptr, 0, idx, w, bitmap, (int)W, 0, err, s);
+  launch_topk(logits, T, N, k, nullptr, 0, idx, w, bitmap, (int)W, 0, err, s, false);
   group_count_kernel<<<(N + 7) / 8, 256, 0, s>>>(bitmap, wp, N, (int)W, counts, offsets,
                                                  tile_prefix, nullptr, nullptr, done);
   const long P = (long)T * k;

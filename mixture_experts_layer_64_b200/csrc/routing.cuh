@@ -104,6 +104,8 @@ __global__ void __launch_bounds__(128) topk_softmax_kernel(const float* __restri
                                                            float* __restrict__ w,
                                                            uint32_t* __restrict__ bitmap, int W,
                                                            int debug, int* err) {
+  griddep_launch();
+  griddep_wait();  // the previous kernel's outputs are visible
   __shared__ uint32_t s_hist[4][256];
   __shared__ unsigned long long s_sel[4][64];
   if (!kVariant) {
@@ -260,22 +262,21 @@ __global__ void __launch_bounds__(128) topk_softmax_kernel(const float* __restri
 }
 
 // Launches topk_softmax_kernel with the smallest multiple of 4 slots per lane
-// that covers N.
+// that covers N (pdl: programmatic stream serialisation).
 static inline cudaError_t launch_topk(const float* logits, int T, int N, int k,
                                       const float* sel_bias, int full_softmax, int* idx, float* w,
                                       uint32_t* bitmap, int W, int debug, int* err,
-                                      cudaStream_t st) {
+                                      cudaStream_t st, bool pdl) {
   const dim3 grid((T + 3) / 4), block(128);
   const bool var = sel_bias != nullptr || full_softmax != 0;
-#define LMOE_TOPK_CASE(S)                                                                        \
-  case S:                                                                                        \
-    if (var)                                                                                     \
-      topk_softmax_kernel<S, true><<<grid, block, 0, st>>>(logits, T, N, k, sel_bias,           \
-                                                           full_softmax, idx, w, bitmap, W,      \
-                                                           debug, err);                          \
-    else                                                                                         \
-      topk_softmax_kernel<S, false><<<grid, block, 0, st>>>(logits, T, N, k, nullptr, 0, idx, w, \
-                                                            bitmap, W, debug, err);              \
+  cudaError_t e = cudaSuccess;
+#define LMOE_TOPK_CASE(S)                                                                   \
+  case S:                                                                                   \
+    e = var ? launch_kernel(pdl, topk_softmax_kernel<S, true>, grid, block, 0, st, logits, T, \
+                            N, k, sel_bias, full_softmax, idx, w, bitmap, W, debug, err)     \
+            : launch_kernel(pdl, topk_softmax_kernel<S, false>, grid, block, 0, st, logits,  \
+                            T, N, k, (const float*)nullptr, 0, idx, w, bitmap, W, debug,    \
+                            err);                                                           \
     break;
   switch ((N + 127) / 128 * 4) {
     LMOE_TOPK_CASE(4)
@@ -290,7 +291,7 @@ static inline cudaError_t launch_topk(const float* logits, int T, int N, int k,
       return cudaErrorInvalidValue;
   }
 #undef LMOE_TOPK_CASE
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 // Word prefix + bits: wp[e][wd] = {set bits of expert e in words < wd, word wd}.
@@ -303,6 +304,8 @@ static __global__ void __launch_bounds__(256) group_count_kernel(uint32_t* __res
                                                           int* __restrict__ tile_prefix2,
                                                           int* __restrict__ tile_prefix64,
                                                           unsigned int* done) {
+  griddep_launch();
+  griddep_wait();  // the previous kernel's outputs are visible
   const int lane = threadIdx.x & 31;
   const int e = blockIdx.x * 8 + (threadIdx.x >> 5);
   if (e < N) {
@@ -392,6 +395,8 @@ static __global__ void __launch_bounds__(256) group_rank_kernel(
     const int* __restrict__ offsets, int T, int k, int N, int W, int* __restrict__ row_tok,
     int* __restrict__ row_slot, float* __restrict__ row_w, int* __restrict__ slot_row, int debug,
     int* err) {
+  griddep_launch();
+  griddep_wait();  // the previous kernel's outputs are visible
   const long pidx = (long)blockIdx.x * blockDim.x + threadIdx.x;
   if (pidx >= (long)T * k) return;
   const int t = (int)(pidx / k);

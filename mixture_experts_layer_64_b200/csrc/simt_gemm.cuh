@@ -36,6 +36,8 @@ __device__ __forceinline__ void simt_store(const GemmProblem& p, int row, int f,
 // count return at once.
 template <typename T, bool kDual, int kEpi>
 __global__ void __launch_bounds__(256) simt_gemm_kernel(const GemmProblem p) {
+  griddep_launch();
+  griddep_wait();  // the previous kernel's outputs are visible
   __shared__ float As[kSimtTK][kSimtTM + 4];
   __shared__ float Bs[kDual ? 2 : 1][kSimtTK][kSimtTN + 4];
   const int NT = (p.F + kSimtTN - 1) / kSimtTN;

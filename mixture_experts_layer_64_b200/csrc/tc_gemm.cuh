@@ -404,7 +404,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
   int* s_tiles = reinterpret_cast<int*>(stg_base + Cfg::STG_BYTES + 512);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  load_tile_tables(p, s_tiles);
+  griddep_launch();
   const int NT = (p.F + Cfg::FT - 1) / Cfg::FT;
   const int KB = p.K / Cfg::BK;
 
@@ -438,6 +438,8 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     tmem_relinquish();
     tc_fence_before();
   }
+  griddep_wait();  // the previous kernel's outputs (tile tables, activations)
+  load_tile_tables(p, s_tiles);
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
@@ -855,7 +857,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   int* s_tiles = reinterpret_cast<int*>(stg_base + Cfg::STG_BYTES + 512);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  load_tile_tables(p, s_tiles);
+  griddep_launch();
   const uint32_t rank = cluster_ctarank();
   const int cid = (int)cluster_id_x(), ncl = (int)cluster_count_x();
   const int NT = (p.F + Cfg::FT - 1) / Cfg::FT;
@@ -883,6 +885,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     tmem_relinquish_pair();
     tc_fence_before();
   }
+  griddep_wait();  // the previous kernel's outputs (tile tables, activations)
+  load_tile_tables(p, s_tiles);
   __syncthreads();
   cluster_sync();  // both CTAs' barriers exist before any remote arrive
   tc_fence_after();
@@ -1104,7 +1108,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   static_assert(3 * Cfg::STAGES * 8 + 5 * 8 + 8 <= 512, "barrier area");
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  load_tile_tables(p, s_tiles);
+  griddep_launch();
   const uint32_t rank = cluster_ctarank();
   const int cid = (int)cluster_id_x(), ncl = (int)cluster_count_x();
   const int NT = (p.F + Cfg::FT - 1) / Cfg::FT;
@@ -1135,6 +1139,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     tmem_relinquish_pair();
     tc_fence_before();
   }
+  griddep_wait();  // the previous kernel's outputs (tile tables, activations)
+  load_tile_tables(p, s_tiles);
   __syncthreads();
   cluster_sync();  // both CTAs' barriers exist before any remote arrive
   tc_fence_after();

@@ -25,6 +25,7 @@ SKIP_PROJ, DEBUG_CHECKS, FORCE_SIMT, FORCE_SWAP, FORCE_NOSWAP, FORCE_NOPAIR, FOR
 ROUTE_FULL_SOFTMAX, ROUTE_BIAS_SELECT = 0x80, 0x100
 EXPERTS_FP8 = 0x200
 SINGLE_STREAM = 0x400
+NO_PDL = 0x800
 MAX_EXPERTS, MAX_TOPK = 1024, 32
 DEVERR_WAIT_TIMEOUT, DEVERR_RANGE, DEVERR_NONFINITE = 0x1, 0x2, 0x4
 STAGES = {"logits": 0, "idx": 1, "w": 2, "offsets": 3, "perm": 4, "z": 5, "h": 6, "ys": 7, "comb": 8}

@@ -274,6 +274,27 @@ def test_side_stream_matches_single_stream(name):
     assert A.last_error() == (lmoe.OK, 0) and B.last_error() == (lmoe.OK, 0)
 
 
+@pytest.mark.parametrize("name", ["split", "pairs"])
+def test_programmatic_launch_matches_plain_launches(name):
+    """Kernels launched with programmatic dependent launch (the default)
+    start while their predecessor drains and wait for its writes before
+    touching global memory; LMOE_NO_PDL launches each after its predecessor
+    has finished.  Back-to-back forwards give bitwise the same outputs."""
+    w = SIDE[name]
+    W = workloads.make_weights(w, device="cuda")
+    A, _ = gpu_layer(w, 0, W)
+    B, _ = gpu_layer(w, lmoe.NO_PDL | lmoe.SINGLE_STREAM, W)
+    x0 = workloads.make_x(w, device="cuda").float()
+    xs = [(x0 * (1.0 - 0.3 * i)).roll(5 * i, dims=0).to(torch.bfloat16).contiguous()
+          for i in range(3)]
+    outs_a = [A.forward(x) for x in xs]
+    outs_b = [B.forward(x) for x in xs]
+    torch.cuda.synchronize()
+    for a, b in zip(outs_a, outs_b):
+        assert torch.equal(a, b)
+    assert A.last_error() == (lmoe.OK, 0) and B.last_error() == (lmoe.OK, 0)
+
+
 def test_side_stream_profile_stages():
     """Profiled forwards time the side stream's two stages on that stream:
     every stage time is non-negative and the down-projection and shared FC1
