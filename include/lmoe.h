@@ -284,6 +284,15 @@ lmoe_status lmoe_last_error(lmoe_layer* h, int* device_error_word);
  * *n_stages, and stops recording.  Stage s is named by lmoe_stage_name(s).
  */
 lmoe_status lmoe_profile_begin(lmoe_layer* h, int max_forwards);
+/*
+ * lmoe_profile_begin_stages -- lmoe_profile_begin recording only the
+ * boundaries of the stages whose bit is set in stage_mask (bit s = stage s);
+ * lmoe_profile_end writes -1 for the other stages.  An event recorded between
+ * two kernels makes the second wait for the first to finish, so timing one
+ * stage this way leaves the other kernel boundaries free to launch early.
+ * Errors: INVALID_ARG (max_forwards < 1, stage_mask without a stage bit).
+ */
+lmoe_status lmoe_profile_begin_stages(lmoe_layer* h, int max_forwards, unsigned stage_mask);
 lmoe_status lmoe_profile_end(lmoe_layer* h, float* ms, int capacity, int* n_forwards,
                              int* n_stages);
 const char* lmoe_stage_name(int stage);

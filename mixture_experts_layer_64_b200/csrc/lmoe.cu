@@ -127,6 +127,7 @@ struct lmoe_layer {
   // profiling
   std::vector<cudaEvent_t> events;
   std::vector<char> prof_side;  // per profiled forward: the side stream ran
+  unsigned prof_mask = 0;       // the stages whose boundaries are recorded
   int prof_cap = 0, prof_count = 0;
   bool profiling = false;
 };
@@ -651,8 +652,19 @@ bool use_swap(const lmoe_layer* h, int T) {
   return (long)T * h->k < 64L * h->N;  // fewer than 64 rows per expert on average
 }
 
+// Records boundary i of the current profiled forward if a recorded stage
+// starts or ends there (boundary i of the caller's stream opens stage i and
+// closes stage i - 1; side boundary kSideMark0 + j opens stage 3 + j and
+// closes stage 2 + j, of which only the side stream's stages 3 and 4 count).
 void prof_mark(lmoe_layer* h, cudaStream_t st, int i) {
-  if (h->profiling && h->prof_count < h->prof_cap)
+  if (!h->profiling || h->prof_count >= h->prof_cap) return;
+  const int opens = i < kSideMark0 ? i : 3 + (i - kSideMark0);
+  const int closes = opens - 1;
+  const bool side = i >= kSideMark0;
+  const auto has = [&](int s) {
+    return s >= 0 && s < kStages && (!side || s == 3 || s == 4) && ((h->prof_mask >> s) & 1u);
+  };
+  if (has(opens) || has(closes))
     cudaEventRecord(h->events[(size_t)h->prof_count * kMarks + i], st);
 }
 
@@ -1340,7 +1352,12 @@ lmoe_status lmoe_last_error(lmoe_layer* h, int* device_error_word) {
 }
 
 lmoe_status lmoe_profile_begin(lmoe_layer* h, int max_forwards) {
-  if (!h || max_forwards < 1) return LMOE_ERR_INVALID_ARG;
+  return lmoe_profile_begin_stages(h, max_forwards, (1u << kStages) - 1);
+}
+
+lmoe_status lmoe_profile_begin_stages(lmoe_layer* h, int max_forwards, unsigned stage_mask) {
+  if (!h || max_forwards < 1 || (stage_mask & ((1u << kStages) - 1)) == 0)
+    return LMOE_ERR_INVALID_ARG;
   DevGuard g(h->device);
   LMOE_CUDA(h, cudaDeviceSynchronize());
   destroy_events(h);
@@ -1357,6 +1374,7 @@ lmoe_status lmoe_profile_begin(lmoe_layer* h, int max_forwards) {
   }
   h->prof_cap = max_forwards;
   h->prof_count = 0;
+  h->prof_mask = stage_mask & ((1u << kStages) - 1);
   h->profiling = true;
   return LMOE_OK;
 }
@@ -1373,6 +1391,10 @@ lmoe_status lmoe_profile_end(lmoe_layer* h, float* ms, int capacity, int* n_forw
     if ((f + 1) * kStages > capacity) break;
     cudaEvent_t* ev = &h->events[(size_t)f * kMarks];
     for (int s = 0; s < kStages; ++s) {
+      if (!((h->prof_mask >> s) & 1u)) {
+        ms[f * kStages + s] = -1.f;  // not recorded
+        continue;
+      }
       // with the side stream, the down-projection and shared FC1 stages are
       // timed there (they overlap the router and routing stages)
       int a = s, b = s + 1;

@@ -34,7 +34,8 @@ EXPORTS = ["lmoe_create", "lmoe_set_weights", "lmoe_reserve", "lmoe_forward", "l
            "lmoe_last_error", "lmoe_profile_begin", "lmoe_profile_end", "lmoe_stage_name",
            "lmoe_last_launch_count", "lmoe_last_expert_path", "lmoe_status_string",
            "lmoe_error_detail", "lmoe_destroy", "lmoe_route_only_noalloc",
-           "lmoe_set_expert_weights_fp8", "lmoe_selftest_wait_timeout"]
+           "lmoe_set_expert_weights_fp8", "lmoe_selftest_wait_timeout",
+           "lmoe_profile_begin_stages"]
 NOALLOC_MAX_WORDS = 262144
 
 
@@ -72,6 +73,7 @@ def lib() -> ctypes.CDLL:
             "lmoe_debug_dump": ([P, I, P, S, P], I),
             "lmoe_last_error": ([P, ctypes.POINTER(I)], I),
             "lmoe_profile_begin": ([P, I], I),
+            "lmoe_profile_begin_stages": ([P, I, ctypes.c_uint], I),
             "lmoe_profile_end": ([P, P, I, ctypes.POINTER(I), ctypes.POINTER(I)], I),
             "lmoe_stage_name": ([I], ctypes.c_char_p),
             "lmoe_last_launch_count": ([P], I),
@@ -292,19 +294,31 @@ class LatentMoELayer:
         st = lib().lmoe_last_error(self._h, ctypes.byref(word))
         return st, word.value
 
-    def profile_begin(self, max_forwards: int):
-        self._check(lib().lmoe_profile_begin(self._h, max_forwards), "lmoe_profile_begin")
+    def profile_begin(self, max_forwards: int, stages=None):
+        """Records stage times of the next max_forwards forwards: every stage,
+        or only the named ones (the other boundaries stay free of events)."""
+        if stages is None:
+            self._check(lib().lmoe_profile_begin(self._h, max_forwards), "lmoe_profile_begin")
+        else:
+            names = [stage_name(i) for i in range(16) if stage_name(i)]
+            mask = 0
+            for n in stages:
+                mask |= 1 << names.index(n)
+            self._check(lib().lmoe_profile_begin_stages(self._h, max_forwards, mask),
+                        "lmoe_profile_begin_stages")
         self._prof_cap = max_forwards
 
     def profile_end(self):
-        """Per-forward stage times (ms): a list of dicts stage name -> ms."""
+        """Per-forward stage times (ms): a list of dicts stage name -> ms
+        (recorded stages only)."""
         cap = self._prof_cap * 16
         buf = (ctypes.c_float * cap)()
         nf, ns = ctypes.c_int(), ctypes.c_int()
         self._check(lib().lmoe_profile_end(self._h, buf, cap, ctypes.byref(nf), ctypes.byref(ns)),
                     "lmoe_profile_end")
         names = [stage_name(i) for i in range(ns.value)]
-        return [{names[s]: buf[f * ns.value + s] for s in range(ns.value)} for f in range(nf.value)]
+        return [{names[s]: buf[f * ns.value + s] for s in range(ns.value)
+                 if buf[f * ns.value + s] >= 0} for f in range(nf.value)]
 
     @property
     def last_launch_count(self) -> int:

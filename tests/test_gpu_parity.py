@@ -295,6 +295,24 @@ def test_programmatic_launch_matches_plain_launches(name):
     assert A.last_error() == (lmoe.OK, 0) and B.last_error() == (lmoe.OK, 0)
 
 
+@pytest.mark.parametrize("stage", ["expert_fc1", "down_proj", "group"])
+def test_profile_selected_stages(stage):
+    """Profiling one stage records only its two boundaries (a side-stream
+    stage's on the side stream); the forward's output is unchanged."""
+    w = SIDE["pairs"]
+    L, W = gpu_layer(w)
+    x = workloads.make_x(w, device="cuda")
+    ref = L.forward(x)
+    L.profile_begin(3, stages=[stage])
+    outs = [L.forward(x) for _ in range(3)]
+    prof = L.profile_end()
+    assert len(prof) == 3
+    for p, o in zip(prof, outs):
+        assert list(p) == [stage] and p[stage] > 0
+        assert torch.equal(o, ref)
+    assert L.last_error() == (lmoe.OK, 0)
+
+
 def test_side_stream_profile_stages():
     """Profiled forwards time the side stream's two stages on that stream:
     every stage time is non-negative and the down-projection and shared FC1
