@@ -313,6 +313,23 @@ def test_profile_selected_stages(stage):
     assert L.last_error() == (lmoe.OK, 0)
 
 
+def test_profile_stage_mask_errors():
+    """A stage mask without a stage bit, or no forwards, is rejected before
+    anything is recorded; an unknown stage name is rejected by the binding."""
+    w = SIDE["no-shared"]
+    L, W = gpu_layer(w)
+    lib = lmoe.lib()
+    assert lib.lmoe_profile_begin_stages(L._h, 2, 0) == lmoe.ERR_INVALID_ARG
+    assert lib.lmoe_profile_begin_stages(L._h, 2, 1 << 12) == lmoe.ERR_INVALID_ARG
+    assert lib.lmoe_profile_begin_stages(L._h, 0, 1) == lmoe.ERR_INVALID_ARG
+    with pytest.raises(ValueError):
+        L.profile_begin(2, stages=["no_such_stage"])
+    x = workloads.make_x(w, device="cuda")
+    L.forward(x)
+    torch.cuda.synchronize()
+    assert L.last_error() == (lmoe.OK, 0)
+
+
 def test_side_stream_profile_stages():
     """Profiled forwards time the side stream's two stages on that stream:
     every stage time is non-negative and the down-projection and shared FC1
