@@ -1,0 +1,60 @@
+"""Host-side consistency: the binding's constants against the header, and the
+bench's use of recorded DRAM traffic."""
+import json
+import os
+import re
+
+import pytest
+
+from mixture_experts_layer_64_b200 import lmoe
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "lmoe.h")
+
+
+def header_defines():
+    text = open(HEADER).read()
+    return {m.group(1): int(m.group(2), 0)
+            for m in re.finditer(r"^#define\s+LMOE_(\w+)\s+(0x[0-9a-fA-F]+|\d+)u?\b", text, re.M)}
+
+
+def test_binding_flags_and_limits_match_the_header():
+    defs = header_defines()
+    flags = {k: v for k, v in defs.items()
+             if k in ("SKIP_PROJ", "DEBUG_CHECKS", "FORCE_SIMT", "FORCE_SWAP", "FORCE_NOSWAP",
+                      "FORCE_NOPAIR", "FORCE_WS_PAIR", "ROUTE_FULL_SOFTMAX", "ROUTE_BIAS_SELECT",
+                      "EXPERTS_FP8", "SINGLE_STREAM", "NO_PDL")}
+    assert len(flags) == 12, sorted(flags)
+    for name, value in flags.items():
+        assert getattr(lmoe, name) == value, name
+    # flags are distinct single bits
+    assert len(set(flags.values())) == len(flags)
+    assert all(v & (v - 1) == 0 for v in flags.values())
+    assert lmoe.MAX_EXPERTS == defs["MAX_EXPERTS"] and lmoe.MAX_TOPK == defs["MAX_TOPK"]
+    assert lmoe.DEVERR_WAIT_TIMEOUT == defs["DEVERR_WAIT_TIMEOUT"]
+    assert lmoe.DEVERR_RANGE == defs["DEVERR_RANGE"]
+    assert lmoe.DEVERR_NONFINITE == defs["DEVERR_NONFINITE"]
+
+
+def test_binding_stage_ids_match_the_header():
+    text = open(HEADER).read()
+    enum = {m.group(1).lower(): int(m.group(2))
+            for m in re.finditer(r"LMOE_STAGE_(\w+)\s*=\s*(\d+)", text)}
+    assert enum == lmoe.STAGES
+
+
+def test_recorded_traffic_is_used_only_on_the_captured_sources(monkeypatch):
+    import bench
+
+    with open(os.path.join(ROOT, "profiles", "traffic.json")) as fh:
+        recorded = json.load(fh)
+    entries = [(wl, st, rec) for wl, stages in recorded.items() if not wl.startswith("_")
+               for st, rec in stages.items()]
+    assert entries
+    for wl, st, rec in entries:
+        assert rec["dram_bytes_per_launch"] > 0 and os.path.exists(os.path.join(ROOT, rec["source"]))
+        monkeypatch.setattr(bench, "kernel_source_hash", lambda stage, h=rec["kernel_sources"]: h)
+        assert bench.recorded_traffic(wl, st) == rec["dram_bytes_per_launch"]
+        monkeypatch.setattr(bench, "kernel_source_hash", lambda stage: "0" * 16)
+        assert bench.recorded_traffic(wl, st) is None
+    assert bench.recorded_traffic("no-such-workload", "expert_fc1") is None
