@@ -13,9 +13,14 @@ replica on its own batch: tokens are independent, so there is no data-path
 collective; the timed region is bracketed by a barrier and
 torch.cuda.synchronize(), and the time is the max over ranks.
 
-Prints one JSON line (rank 0).  --impl reference times the CPU oracle (the
-reference arm of this method: a plain float64 C++ implementation) on a
-bounded token sample of the same workload.
+Prints one JSON line (rank 0).  With the default workload (decode, the
+headline) the line also carries "prefill": the two prefill workloads
+(latent-prefill-skewed, latent-prefill-shared) measured in the same run with
+the same steps and warm-up, each with its own clocks, roofline, expert-load
+summary, per-stage p50/p95/p99 and projection share (--no-prefill skips
+them).  --impl reference times the CPU oracle (the reference arm of this
+method: a plain float64 C++ implementation) on a bounded token sample of the
+same workload.
 """
 from __future__ import annotations
 
@@ -45,7 +50,9 @@ METRIC = "LatentMoE layer tokens/sec at decode & prefill T; HBM GB/s / tensor-pi
 UNIT = "tokens/s"
 DEFAULT_WORKLOAD = "std-moe-decode"
 EXPERT_PATHS = ["cuda-core", "tcgen05 token-tiled", "tcgen05 weight-stationary",
-                "tcgen05 token-tiled, 2-SM CTA pairs", "tcgen05 weight-stationary, 2-SM CTA pairs"]
+                "tcgen05 token-tiled, 2-SM CTA pairs", "tcgen05 weight-stationary, 2-SM CTA pairs",
+                "tcgen05 split by load: 2-SM CTA-pair token tiles above 384 rows per expert, "
+                "weight-stationary tiles of the expert's rows below"]
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 _CSRC = "mixture_experts_layer_64_b200/csrc/"
 _GEMM_SRC = (_CSRC + "common.cuh", _CSRC + "tc_gemm.cuh")
@@ -307,29 +314,47 @@ def run_reference(args):
     return 0
 
 
-def run_ours(args):
-    from mixture_experts_layer_64_b200 import build, lmoe
+PREFILL_WORKLOADS = ("latent-prefill-skewed", "latent-prefill-shared")
+NOMINAL_HBM_GBS = 8000.0  # the ~8 TB/s HBM figure the decode target is quoted against
+PROJECTION_SHARE_PAGES = 0.09  # the paper's ~9% latent-projection overhead (Section 4.3)
 
-    ws, rank, local = dist_env()
-    pg = None
-    if ws > 1:
-        import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-        pg = dist
-    else:
-        torch.cuda.set_device(0)
-    build.build_library()
-    dev = torch.device("cuda", torch.cuda.current_device())
-    w = workloads.WORKLOADS[args.workload]
+
+def percentiles(vals):
+    a = np.asarray(vals, dtype=np.float64)
+    return {"p50": round(float(np.percentile(a, 50)), 5), "p95": round(float(np.percentile(a, 95)), 5),
+            "p99": round(float(np.percentile(a, 99)), 5), "mean": round(float(a.mean()), 5)}
+
+
+def load_summary(loads: np.ndarray):
+    """Per-expert routed rows of one forward (from the offsets): touched
+    experts, the largest load, and the MMA work of tiles of 16 / 64 / 128 /
+    256 rows relative to the routed rows (padding of each expert's last tile)."""
+    c = loads[loads > 0]
+    if c.size == 0:
+        return {"touched": 0}
+    pad = {str(tile): round(float((np.ceil(c / tile) * tile).sum() / c.sum()), 4)
+           for tile in (16, 64, 128, 256)}
+    return {"touched": int(c.size), "max_rows": int(c.max()), "min_rows": int(c.min()),
+            "mean_rows_touched": round(float(c.mean()), 2), "routed_rows": int(c.sum()),
+            "rows_in_experts_over_4096": int(c[c >= 4096].sum()),
+            "experts_under_16_rows": int((c < 16).sum()), "padding_factor": pad}
+
+
+def measure(args, name: str, pg, rank: int, ws: int, local: int, dev, flags: int = 0,
+            n_prof: int = 50):
+    """Builds the workload's layer and measures it: an untimed profiled pass
+    (events at every stage boundary, n_prof forwards), the timed region of
+    args.steps forwards (events around the dominant stage only), and the
+    host-buffer entry point.  Every rank takes the same collective steps."""
+    from mixture_experts_layer_64_b200 import lmoe
+
+    w = workloads.WORKLOADS[name]
     W = workloads.make_weights(w, device=dev)
-    # each replica draws its own batch
-    xw = replica_workload(w, rank)
+    xw = replica_workload(w, rank)  # each replica draws its own batch
     x = workloads.make_x(xw, device=dev)
     L = lmoe.LatentMoELayer(w.d, w.l, w.N, w.k, w.m, act=w.act, shared_m=w.shared_m,
                             dtype=w.dtype, skip_proj=w.skip_proj,
-                            flags=args.lib_flags | (lmoe.EXPERTS_FP8 if w.expert_fp8 else 0))
+                            flags=flags | (lmoe.EXPERTS_FP8 if w.expert_fp8 else 0))
     L.set_weights(W["Wg"], W["bias"], W["Wdown"], W["Wup"], W["W1"], W["W2"], W["Ws1"], W["Ws2"])
     if w.expert_fp8:
         L.set_expert_weights_fp8(W["W1q"], W["W1s"], W["W2q"], W["W2s"])
@@ -347,15 +372,16 @@ def run_ours(args):
     loads = np.diff(L.debug_dump("offsets", w.T).cpu().numpy())
 
     # ---- stage breakdown: an untimed pass with events at every stage boundary
-    n_prof = max(3, min(args.steps, 20))
     L.profile_begin(n_prof)
     for _ in range(n_prof):
         L.forward(x, out)
     prof_all = L.profile_end()
-    stage_ms = {k: statistics.fmean(p[k] for p in prof_all) for k in prof_all[0]}
+    stage_pct = {k: percentiles([p[k] for p in prof_all]) for k in prof_all[0]}
+    stage_ms = {k: v["mean"] for k, v in stage_pct.items()}
     dom = max(stage_ms, key=stage_ms.get)
 
-    sampler = ClockSampler(local, args.clocks_csv) if rank == 0 else None
+    sampler = ClockSampler(local, args.clocks_csv if name == args.workload else None) \
+        if rank == 0 else None
     if sampler:
         sampler.start()
     # ---- timed region: K steps; events on the launching stream around the
@@ -379,7 +405,6 @@ def run_ours(args):
     prof = L.profile_end()
     elapsed_ms = max_over_ranks(pg, elapsed_ms, dev)
     ms_per_step = elapsed_ms / args.steps
-    value = job_throughput(w.T, ws, ms_per_step)
 
     # ---- end to end through the host-buffer entry point (pinned buffers)
     xh = x.cpu().pin_memory()
@@ -417,26 +442,86 @@ def run_ours(args):
         t = dom_ms / 1000.0
         ridge = peaks["bf16_tflops_sustained"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
         if by > 0 and (fl / by) < ridge:
-            ach, pk, unit, bound = by / t / 1e9, peaks["hbm_gbs"], "GB/s", "hbm"
+            ach = by / t / 1e9
+            roofline = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                        "frac": ach / peaks["hbm_gbs"],
+                        "peak_source": f"{peak_src} (hbm_gbs: a STREAM-style copy)",
+                        "frac_of_nominal": ach / NOMINAL_HBM_GBS,
+                        "nominal_note": "achieved / 8000 GB/s, the ~8 TB/s B200 HBM figure: a "
+                                        "read-only weight stream can exceed the measured copy"}
         else:
-            ach, pk, unit, bound = fl / t / 1e12, peaks["bf16_tflops_sustained"], "TFLOP/s", "tensor"
-        roofline = {"bound": bound, "achieved": ach, "peak": pk, "unit": unit, "frac": ach / pk,
-                    "traffic": recorded_traffic(w.name, dom), "kernel": dom,
-                    "algorithmic_per_launch": by if bound == "hbm" else fl,
-                    "launch_ms": dom_ms, "peak_source": f"{peak_src} "
-                    f"({'hbm_gbs' if bound == 'hbm' else 'bf16_tflops_sustained'})",
-                    "stage_ms": {k: round(v, 5) for k, v in stage_ms.items()},
-                    "stage_ms_source": f"untimed pass of {n_prof} steps with events at "
-                                       "every stage boundary"}
-        lc = costmodel.layer_counts(T=w.T, d=w.d, l=w.l, N=w.N, k=w.k, m=w.m, act=w.act,
-                                    shared_m=w.shared_m, skip_proj=w.skip_proj, loads=loads,
-                                    expert_bytes=1 if w.expert_fp8 else None)
-        roofline["layer"] = {"alg_bytes": lc.bytes, "alg_flops": lc.flops,
-                             "hbm_frac": lc.bytes / (ms_per_step / 1e3) / 1e9 / peaks["hbm_gbs"],
-                             "touched_experts": lc.touched,
-                             "t_exp_mean": round(lc.t_exp_mean, 2),
-                             "paper_intensity": costmodel.arithmetic_intensity(
-                                 lc.t_exp_mean, w.l, w.m) if lc.touched else None}
+            ach = fl / t / 1e12
+            pb, psus = peaks["bf16_tflops"], peaks["bf16_tflops_sustained"]
+            roofline = {"bound": "tensor", "achieved": ach, "peak": pb, "unit": "TFLOP/s",
+                        "frac": ach / pb,
+                        "peak_source": f"{peak_src} (bf16_tflops: cuBLAS bf16 burst)",
+                        "peak_sustained": psus, "frac_sustained": ach / psus}
+        roofline.update({"traffic": recorded_traffic(w.name, dom), "kernel": dom,
+                         "algorithmic_per_launch": by if roofline["bound"] == "hbm" else fl,
+                         "launch_ms": dom_ms})
+    lc = costmodel.layer_counts(T=w.T, d=w.d, l=w.l, N=w.N, k=w.k, m=w.m, act=w.act,
+                                shared_m=w.shared_m, skip_proj=w.skip_proj, loads=loads,
+                                expert_bytes=1 if w.expert_fp8 else None)
+    layer = {"alg_bytes": lc.bytes, "alg_flops": lc.flops,
+             "hbm_frac": lc.bytes / (ms_per_step / 1e3) / 1e9 / peaks["hbm_gbs"],
+             "tensor_frac_burst": lc.flops / (ms_per_step / 1e3) / 1e12 / peaks["bf16_tflops"],
+             "touched_experts": lc.touched, "t_exp_mean": round(lc.t_exp_mean, 2),
+             "paper_intensity": costmodel.arithmetic_intensity(lc.t_exp_mean, w.l, w.m)
+             if lc.touched else None}
+    if w.skip_proj:
+        proj = {"value": None, "note": "no projections (standard-MoE shape, l = d)"}
+    else:
+        p50 = stage_pct["down_proj"]["p50"] + stage_pct["up_proj"]["p50"]
+        proj = {"value": round(p50 / ms_per_step, 4), "pages": PROJECTION_SHARE_PAGES,
+                "down_proj_ms_p50": stage_pct["down_proj"]["p50"],
+                "up_proj_ms_p50": stage_pct["up_proj"]["p50"],
+                "note": "(down + up projection) p50 / timed step; the down-projection runs "
+                        "on a second stream beside the router and routing"}
+    res = {"workload": name, "w": w, "W": W, "x": x, "ms_per_step": ms_per_step,
+           "value": job_throughput(w.T, ws, ms_per_step),
+           "e2e": {"value": job_throughput(w.T, ws, e_ms), "unit": UNIT,
+                   "h2d_bytes_per_step": io_bytes, "d2h_bytes_per_step": io_bytes},
+           "gpu_launches": launches_per_step * args.steps, "clocks": clocks,
+           "roofline": roofline, "layer": layer, "stage_ms": stage_pct,
+           "stage_ms_source": f"untimed pass of {n_prof} forwards after {args.warmup} warm-up "
+                              "forwards, events at every stage boundary",
+           "projection_share": proj, "expert_loads": load_summary(loads),
+           "expert_path": {"fc1": EXPERT_PATHS[max(0, L.last_expert_path) & 7],
+                           "fc2": EXPERT_PATHS[max(0, L.last_expert_path) >> 3]}}
+    L.close()
+    return res
+
+
+def sub_record(r):
+    """The JSON of one measured workload beside the headline (prefill)."""
+    w = r["w"]
+    return {"workload": r["workload"], "value": r["value"], "unit": UNIT,
+            "ms_per_step": r["ms_per_step"], "config": {"T": w.T, "d": w.d, "l": w.l, "N": w.N,
+                                                        "k": w.k, "m": w.m, "act": w.act,
+                                                        "shared_m": w.shared_m, "bias": w.bias},
+            "e2e": r["e2e"], "gpu_launches": r["gpu_launches"], "clocks": r["clocks"],
+            "roofline": r["roofline"], "layer": r["layer"], "expert_loads": r["expert_loads"],
+            "projection_share": r["projection_share"], "stage_ms": r["stage_ms"],
+            "expert_path": r["expert_path"]}
+
+
+def run_ours(args):
+    from mixture_experts_layer_64_b200 import build
+
+    ws, rank, local = dist_env()
+    pg = None
+    if ws > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+        pg = dist
+    else:
+        torch.cuda.set_device(0)
+    build.build_library()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    main = measure(args, args.workload, pg, rank, ws, local, dev, flags=args.lib_flags)
+    w, W, x = main.pop("w"), main.pop("W"), main.pop("x")
 
     cpu_baseline = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
@@ -450,21 +535,37 @@ def run_ours(args):
         except Exception as e:  # the baseline is reported, never required
             cpu_baseline = {"value": None, "unit": UNIT, "cores": None, "kind": "oracle",
                             "sample": f"failed: {e}"}
+    del W, x
+    torch.cuda.empty_cache()
+
+    # ---- the prefill workloads, measured in the same run with the same steps
+    prefill = []
+    if not args.no_prefill and args.workload == DEFAULT_WORKLOAD:
+        for name in PREFILL_WORKLOADS:
+            r = measure(args, name, pg, rank, ws, local, dev, flags=args.lib_flags)
+            del r["W"], r["x"]
+            prefill.append(sub_record(r))
+            del r
+            torch.cuda.empty_cache()
 
     if rank == 0:
-        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
-                "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-                "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
-                "config": workload_config(w, ws),
-                "e2e": {"value": job_throughput(w.T, ws, e_ms), "unit": UNIT,
-                        "h2d_bytes_per_step": io_bytes, "d2h_bytes_per_step": io_bytes},
-                "gpu_launches": launches_per_step * args.steps,
-                "lib_flags": args.lib_flags,
-                "roofline": roofline, "cpu_baseline": cpu_baseline, "clocks": clocks,
-                "expert_path": {"fc1": EXPERT_PATHS[max(0, L.last_expert_path) & 7],
-                                "fc2": EXPERT_PATHS[max(0, L.last_expert_path) >> 3]}}
+        roofline = main["roofline"]
+        if roofline is not None:
+            roofline = dict(roofline, stage_ms={k: v["mean"] for k, v in main["stage_ms"].items()},
+                            layer=main["layer"])
+        line = {"metric": METRIC, "value": main["value"], "unit": UNIT, "n_gpus": ws,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": main["ms_per_step"],
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": w.dtype, "data": "synthetic", "config": workload_config(w, ws),
+                "e2e": main["e2e"], "gpu_launches": main["gpu_launches"],
+                "lib_flags": args.lib_flags, "roofline": roofline, "cpu_baseline": cpu_baseline,
+                "clocks": main["clocks"], "expert_path": main["expert_path"],
+                "stage_ms": main["stage_ms"], "stage_ms_source": main["stage_ms_source"],
+                "projection_share": main["projection_share"],
+                "expert_loads": main["expert_loads"]}
+        if prefill:
+            line["prefill"] = prefill
         print(json.dumps(line), flush=True)
-    L.close()
     if pg:
         pg.barrier()
         pg.destroy_process_group()
@@ -480,6 +581,8 @@ def main():
     ap.add_argument("--workload", choices=workloads.WORKLOAD_ORDER, default=DEFAULT_WORKLOAD)
 
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true",
+                    help="skip the prefill workloads measured beside the default decode line")
     ap.add_argument("--experts", type=int, default=None,
                     help="override N (reduced cases for profiler captures)")
     ap.add_argument("--topk", type=int, default=None, help="override k")

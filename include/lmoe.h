@@ -117,6 +117,39 @@ typedef enum { LMOE_F32 = 0, LMOE_BF16 = 1 } lmoe_dtype;
                                     drains, sets up its barriers and tensor
                                     memory, and waits for the predecessor's
                                     writes before its first global access. */
+#define LMOE_LOAD_SPLIT         0x1000u /* prefill (token-tiled) expert GEMMs
+                                    split by load: the experts with more
+                                    than 384 rows on CTA pairs (256-row token
+                                    tiles; FC1 gathers its rows by token in
+                                    both CTAs), the others on single-CTA
+                                    weight-stationary tiles of their rows
+                                    rounded up to 16 (at most 128 rows for a
+                                    gated FC1, 256 otherwise), so an expert
+                                    with few rows pays neither a 128- nor a
+                                    256-row tile.  Off by default: FC1 on
+                                    single-CTA 128-row tiles and FC2 on CTA
+                                    pairs for every expert.  Results are the
+                                    same either way up to the order of fp32
+                                    sums inside the tensor cores. */
+#define LMOE_NO_STREAM_K        0x2000u /* decode (weight-stationary) expert
+                                    FC1 in whole tiles per CTA.  By
+                                    default, with at least two tiles per
+                                    CTA, the (tile, K block) units are dealt
+                                    out in equal ranges, one per CTA, so the
+                                    weight stream ends on every SM at the
+                                    same time; a tile that straddles two
+                                    ranges is summed from its two fp32 parts
+                                    (in a fixed way: the result does not
+                                    depend on timing).  Needs 2 x (SMs + 1)
+                                    x 64 KB of workspace. */
+
+#define LMOE_SORTED_ROWS        0x4000u /* copy the expert FC1's input rows
+                                    into expert order (T*k rows of the
+                                    latent width, a workspace of that size)
+                                    before FC1, which then loads them as
+                                    contiguous tiles by TMA instead of
+                                    gathering them by token.  Off by
+                                    default.  Results are the same. */
 
 /* Limits of the library. */
 #define LMOE_MAX_EXPERTS 1024
@@ -298,6 +331,85 @@ lmoe_status lmoe_profile_end(lmoe_layer* h, float* ms, int capacity, int* n_forw
 const char* lmoe_stage_name(int stage);
 
 /*
+ * ---- Expert parallelism: dispatch and combine in latent space ----
+ *
+ * The paper's deployment analysis (LatentMoE, Section 2.2 "Communication
+ * Bottleneck"; Section 3, the paragraph after Eq. (1)) splits the N experts
+ * over `world` GPUs and moves, per token, its routed rows to the GPUs that
+ * own its experts and the expert outputs back; LatentMoE does both in the
+ * latent width l instead of d, so both all-to-alls carry d / l times fewer
+ * bytes.  These calls run one rank's compute; the caller moves the rows
+ * between ranks (an all-to-all: NCCL through torch.distributed, see
+ * mixture_experts_layer_64_b200/ep.py).  Rows a rank receives must be in
+ * its own device memory before lmoe_ep_experts reads them.
+ *
+ * Ownership: N % world == 0 and rank r owns the n = N / world experts
+ * [r n, (r + 1) n).  Every rank's handle holds the weights of all N experts
+ * (lmoe_set_weights); lmoe_ep_experts reads those of its own n only.
+ * Per call, on every rank:
+ *   1 lmoe_ep_dispatch: router, top-k, grouping, down-projection (and the
+ *     shared expert's first matrix).  send_rows[r] = the latent row of the
+ *     token of sorted row r (rows sorted by expert, then token; with
+ *     LMOE_SKIP_PROJ the token's row of x), send_gates[r] = its gate,
+ *     expert_counts[e] = the rows routed to expert e.  The rows for rank q are
+ *     the contiguous block of its experts.
+ *   2 (caller) every rank sends rank q the n counts of q's experts: rank q
+ *     holds recv_counts[s][e] (s = source rank); then the row blocks and
+ *     gates, sources in rank order.
+ *   3 lmoe_ep_experts: the n local experts' FFNs on the received rows, with
+ *     each row's gate applied; out_rows[i] belongs to received row i.
+ *   4 (caller) the reverse exchange: each source receives back its rows in
+ *     the order it sent them (its send_rows order).
+ *   5 lmoe_ep_combine: per token the sum of its k returned rows, the
+ *     up-projection, the shared expert and the residual.
+ * Steps 1 and 5 pair up on one handle (5 uses 1's routing); one dispatch at
+ * a time per handle.  All pointers are device pointers, rows in the layer
+ * dtype with row stride l (d with LMOE_SKIP_PROJ), counts int32.
+ */
+
+/* Sizes the expert-side workspace for up to max_recv_rows received rows per
+ * call (at most world * T * k).  Allocates.  Errors: INVALID_ARG, NOT_READY
+ * (call lmoe_reserve first), OOM, CUDA. */
+lmoe_status lmoe_ep_reserve(lmoe_layer* h, int max_recv_rows);
+
+/* Step 1.  send_rows [T*k, l], send_gates [T*k] fp32, expert_counts [N]
+ * int32: device outputs owned by the caller.  0 < T <= reserved max_T.
+ * Errors: NOT_READY, INVALID_ARG, UNSUPPORTED (fp8 expert weights), CUDA. */
+lmoe_status lmoe_ep_dispatch(lmoe_layer* h, const void* x, int T, void* send_rows,
+                             float* send_gates, int* expert_counts, lmoe_stream_t stream);
+
+/* Step 3.  recv_counts: HOST array [world, n] int32, recv_counts[s][e] =
+ * the rows source rank s sent for local expert e (the caller has them: they
+ * size the all-to-all); Rr = their sum <= the reserved max_recv_rows.
+ * recv_rows [Rr, l] and recv_gates [Rr] (device) in received order: sources
+ * in rank order, each source's rows as it sent them.  out_rows [Rr, l]
+ * (device): the gate-scaled expert outputs in received order.  The local
+ * experts' kernels are chosen from the mean received rows per local expert
+ * as in lmoe_forward.  The small grouping tables are uploaded from a
+ * library-owned pinned buffer (the call waits for the previous call's upload
+ * before rewriting it).  Errors: NOT_READY (no lmoe_ep_reserve),
+ * INVALID_ARG (sizes, NULL, negative counts, N % world != 0),
+ * UNSUPPORTED (Rr over the reserved size; fp8 expert weights), CUDA. */
+lmoe_status lmoe_ep_experts(lmoe_layer* h, const void* recv_rows, const float* recv_gates,
+                            const int* recv_counts, int rank, int world, void* out_rows,
+                            lmoe_stream_t stream);
+
+/* Step 5.  back_rows [T*k, l] in the dispatch's send order; x the same
+ * [T, d] input as the dispatch, out [T, d].  Errors: NOT_READY (no matching
+ * dispatch), INVALID_ARG, CUDA. */
+lmoe_status lmoe_ep_combine(lmoe_layer* h, const void* x, const void* back_rows, void* out, int T,
+                            lmoe_stream_t stream);
+
+/* Host-side plan of step 3 (no GPU, host pointers): the order in which the
+ * received rows are grouped by local expert -- experts in order, then
+ * sources in rank order, each source's rows as sent.  recv_counts [world,
+ * n]; offsets [n + 1] (offsets[n] = Rr); perm [Rr]: grouped row -> received
+ * row.  lmoe_ep_experts builds the same order on the device.  Errors:
+ * INVALID_ARG (bad sizes, NULL, negative counts). */
+lmoe_status lmoe_ep_local_plan(const int* recv_counts, int world, int n_local, int* offsets,
+                               int* perm);
+
+/*
  * lmoe_route_only_noalloc -- lmoe_route_only without a handle and without
  * allocating device memory.  The paper has no counterpart: this is an
  * interface for callers, not a step of the method.
@@ -315,19 +427,29 @@ const char* lmoe_stage_name(int stage);
  *   N * ceil(T / 32) <= LMOE_NOALLOC_MAX_WORDS (e.g. T <= 8192 with N = 1024,
  *   T <= 16384 with N = 512); beyond them it returns LMOE_ERR_UNSUPPORTED and
  *   enqueues nothing.
- *   Setup: the first call on a device looks up the array's device address
- *   (cudaGetSymbolAddress) with that device current; make that first call
- *   before any stream capture.
+ *   Setup: every call looks up the array's device address
+ *   (cudaGetSymbolAddress) on the current device, so it stays valid across a
+ *   device reset; the first call on a device also loads the module there:
+ *   make that first call before any stream capture.  The current device
+ *   must be the one that holds the pointers and the stream.
  *   Sharing: every call uses the same array and clears the parts that must
  *   start at zero, so calls that overlap on the GPU (other streams, other
  *   host threads) race and must be serialised by the caller.
+ * error_word: a caller-owned device int, or NULL.  When given, the call
+ * zeroes it on the stream and runs the kernels with the device checks of
+ * LMOE_DEBUG_CHECKS: a non-finite logit sets LMOE_DEVERR_NONFINITE and an
+ * expert index out of range LMOE_DEVERR_RANGE in it.  The call itself does
+ * not synchronise: read the word once the stream has completed.  With NULL
+ * no checks run, and non-finite logits give indices that are in range but
+ * otherwise unspecified.
  * Errors: INVALID_ARG (bad sizes, NULL pointers), UNSUPPORTED (over the
- * limits), CUDA.
+ * limits), CUDA (a failed enqueue: the outputs are then not written).
  */
 #define LMOE_NOALLOC_MAX_WORDS     262144u
 #define LMOE_NOALLOC_SCRATCH_BYTES 3211264u
 lmoe_status lmoe_route_only_noalloc(const float* logits, int T, int N, int k, int* idx, float* w,
-                                    int* offsets, int* perm, lmoe_stream_t stream);
+                                    int* offsets, int* perm, int* error_word,
+                                    lmoe_stream_t stream);
 
 /*
  * lmoe_selftest_wait_timeout -- test hook for the bounded waits: enqueues one
@@ -348,7 +470,10 @@ int lmoe_last_launch_count(const lmoe_layer* h);
  * in bits 3-5, each: 0 CUDA-core, 1 tcgen05 token-tiled, 2 tcgen05
  * weight-stationary (swap-AB), 3 tcgen05 token-tiled on CTA pairs (2-SM MMA),
  * 4 tcgen05 weight-stationary on CTA pairs (the expert's rows as the MMA's N,
- * split into tiles of nearly equal size in units of 16 rows). */
+ * split into tiles of nearly equal size in units of 16 rows), 5 tcgen05
+ * split by load (CTA-pair token tiles for the experts with more than 384
+ * rows, single-CTA weight-stationary tiles of up to 128 / 256 rows for the
+ * others). */
 int lmoe_last_expert_path(const lmoe_layer* h);
 
 const char* lmoe_status_string(lmoe_status s);

@@ -73,10 +73,25 @@ struct GemmProblem {
   const float* w_scale;   // fp8 weights (B holds E4M3 codes): scale of weight row
                           // g * w_group_stride + f, applied to the accumulator
   int* err;               // device error word
+  int stream_k;           // weight-stationary decode tiles: stream-K work split
+  float* sk_part;         // stream-K: 2 fp32 slots of kSkSlotFloats per CTA boundary
+  int* sk_count;          // stream-K: one arrival counter per boundary (zero between launches)
 };
 
 constexpr int kRowTile = 128;
 constexpr int kSwapRowTile = 64;  // rows per tile (the MMA's N, at most) of the weight-stationary kernel
+// One stream-K partial accumulator of a weight-stationary tile: up to 64 rows
+// x (gate, linear) x 128 features, fp32.
+constexpr int kSkSlotFloats = kSwapRowTile * 2 * 128;
+// Experts with more than this many rows run their prefill expert GEMMs on CTA
+// pairs (256-row token tiles); the others on weight-stationary tiles whose
+// row count is the expert's, rounded up to 16.  A pair tile issues its MMAs
+// about a third faster than a single-CTA tile, but pads the expert's last
+// tile to 256 rows: up to ~384 rows the exact-size tiles do less work.
+#ifndef LMOE_PAIR_MIN_ROWS
+#define LMOE_PAIR_MIN_ROWS 384
+#endif
+constexpr int kPairMinRows = LMOE_PAIR_MIN_ROWS;
 
 // ---- scalar helpers ---------------------------------------------------------
 

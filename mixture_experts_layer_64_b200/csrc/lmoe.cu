@@ -27,6 +27,7 @@
 
 #include "../../include/lmoe.h"
 #include "common.cuh"
+#include "ep.cuh"
 #include "misc.cuh"
 #include "routing.cuh"
 #include "simt_gemm.cuh"
@@ -65,6 +66,15 @@ EncodeTiledFn get_encode_fn() {
 
 }  // namespace
 
+// The row grouping an expert GEMM runs over: G groups (experts e0 .. e0 +
+// G - 1 of the weight stacks), their row offsets, and the tile counts of each
+// tile size (exclusive prefixes over the groups, see group_count_kernel).
+struct Grouping {
+  int G = 0, e0 = 0;
+  const int *offsets = nullptr, *tp128 = nullptr, *tp256 = nullptr, *tp64 = nullptr;
+  const int *big256 = nullptr, *small128 = nullptr, *small256 = nullptr;
+};
+
 struct lmoe_layer {
   int d, l, N, k, m, act, shared_m, dtype;
   unsigned flags;
@@ -91,6 +101,7 @@ struct lmoe_layer {
   float* W2s = nullptr;      // [N * l]
   bool fp8_set = false;
   void* a16 = nullptr;       // fp8 experts: the FC1 input rows in f16 [T, l or d]
+  void* zs = nullptr;        // LMOE_SORTED_ROWS: the FC1 input rows in expert order [T*k, l or d]
   // workspace
   int max_T = 0, W = 0;
   float* logits = nullptr;
@@ -100,6 +111,28 @@ struct lmoe_layer {
   uint2* wp = nullptr;
   int *counts = nullptr, *offsets = nullptr, *tile_prefix = nullptr, *tile_prefix2 = nullptr;
   int* tile_prefix64 = nullptr;  // 64-row tile counts (weight-stationary kernel)
+  // prefill expert GEMMs split by load: 256-row tiles of the experts with
+  // more than kPairMinRows rows (CTA pairs), 128- and 256-row tiles of the
+  // others (weight-stationary, single CTA)
+  int *big_prefix2 = nullptr, *small_prefix = nullptr, *small_prefix2 = nullptr;
+  // stream-K split of the weight-stationary decode GEMMs: two partial
+  // accumulator slots and one arrival counter per boundary between CTAs
+  float* sk_part = nullptr;
+  int* sk_count = nullptr;
+  // the forward's expert grouping (all N experts, the routing's prefixes)
+  Grouping fwd_grp;
+  // expert parallelism: the received rows' grouping over the local experts
+  // and the expert-side workspace (lmoe_ep_reserve)
+  Grouping ep_grp;
+  int ep_max_rows = 0;
+  int* ep_tab = nullptr;        // device: counts [N] | src_start [N+1] | roff [N] | goff [N] |
+                                // offsets [N+1] | 6 tile prefixes [N+1]
+  int* ep_tab_host = nullptr;   // pinned staging of the first four tables
+  cudaEvent_t ep_uploaded = nullptr;  // the last upload from ep_tab_host has been read
+  int *ep_perm = nullptr, *ep_inv = nullptr;  // grouped row <-> received row
+  float* ep_gates = nullptr;                  // gates in grouped order
+  void *ep_h = nullptr, *ep_ys = nullptr;     // FC1 output, FC2 output (grouped)
+  int ep_T = -1;                              // the pending dispatch's T (-1: none)
   unsigned* done = nullptr;
   int* err = nullptr;
   int *row_tok = nullptr, *row_slot = nullptr, *slot_row = nullptr;
@@ -204,7 +237,10 @@ struct GemmCall {
   bool swap;    // weight-stationary expert kernels
   bool pair;    // 2-SM token-tiled kernels on CTA pairs (256-row tiles)
   bool ws_pair;  // grouped: weight-stationary kernel on CTA pairs (rows on N)
+  int wide;      // grouped, swap: weight-stationary tiles of up to 128 / 256 rows
+                 // (0: the decode kernel's 64-row tiles)
   bool side;     // enqueued on the side stream: split-K uses the side partial buffer
+  const Grouping* grp;  // grouped calls: the grouping (tile prefixes)
 };
 
 bool encode_map(CUtensorMap* map, const void* ptr, long rows, int cols, long ld, int box_rows) {
@@ -354,7 +390,8 @@ lmoe_status launch_pair(lmoe_layer* h, const GemmCall& c, cudaStream_t st) {
   CUtensorMap ta, tb;
   std::memset(&ta, 0, sizeof ta);
   std::memset(&tb, 0, sizeof tb);
-  if (!encode_map(&ta, c.p.A, c.a_rows, c.p.K, c.p.lda, 128) ||
+  // gathered rows (kGather) are fetched by cp.async: no activation map
+  if ((!Cfg::kGather && !encode_map(&ta, c.p.A, c.a_rows, c.p.K, c.p.lda, 128)) ||
       !encode_map(&tb, c.p.B, c.b_rows, c.p.K, c.p.K, 128)) {
     h->detail = "cuTensorMapEncodeTiled failed";
     return LMOE_ERR_CUDA;
@@ -386,9 +423,9 @@ lmoe_status launch_pair_ws(lmoe_layer* h, const GemmCall& c, cudaStream_t st) {
     return LMOE_ERR_CUDA;
   }
   GemmProblem p = c.p;
-  p.tile_prefix = Cfg::NMAX == 2 * kRowTile ? h->tile_prefix2 : h->tile_prefix;
+  p.tile_prefix = Cfg::NMAX == 2 * kRowTile ? c.grp->tp256 : c.grp->tp128;
   p.row_tile = Cfg::NMAX;
-  const long max_row_tiles = (long)c.out_rows / Cfg::NMAX + h->N;
+  const long max_row_tiles = (long)c.out_rows / Cfg::NMAX + c.grp->G;
   const long NT = (c.p.F + Cfg::FT - 1) / Cfg::FT;
   const long clusters = std::max(1L, std::min<long>(max_clusters, max_row_tiles * NT));
   return pair_launch(h, tc_gemm_pair_ws_kernel<Cfg>, Cfg::SMEM_BYTES, clusters, st, ta, tb, p);
@@ -468,6 +505,26 @@ int choose_splits(const lmoe_layer* h, const GemmCall& c, int& kbs) {
   return (KB + kbs - 1) / kbs;  // every range non-empty
 }
 
+// First half of a split-K call: the S fp32 slices of partial sums in the
+// call's partial buffer (slice = M * Fp floats apart).
+lmoe_status run_split_partials(lmoe_layer* h, const GemmCall& c, int S, int kbs,
+                               cudaStream_t st) {
+  const bool dual = c.p.dual_offset > 0;
+  const int Fp = dual ? 2 * c.p.F : c.p.F;
+  GemmCall g = c;
+  g.kind = GK_ROUTER;  // fp32 output, no bias: the partial sums
+  g.p.F = Fp;
+  g.p.dual_offset = 0;
+  std::memset(&g.p.epi, 0, sizeof g.p.epi);
+  g.p.epi.out = part_buffer(h, c);
+  g.p.epi.ldo = Fp;
+  g.p.epi.slice = (long)c.p.M * Fp;
+  g.p.splits = S;
+  g.p.kb_per_split = kbs;
+  g.out_rows = (long)S * c.p.M;  // the slices stacked: rows of the output map
+  return launch_tc<TcCfg<false, false, false, 128, EPI_F32_BIAS>>(h, g, st);
+}
+
 lmoe_status run_split(lmoe_layer* h, const GemmCall& c, int S, int kbs, cudaStream_t st) {
   const bool dual = c.p.dual_offset > 0;
   const int Fp = dual ? 2 * c.p.F : c.p.F;
@@ -497,10 +554,17 @@ lmoe_status run_gemm(lmoe_layer* h, GemmCall c, cudaStream_t st, int* path = nul
   // The weight-stationary tensor-core kernel takes at most kSwapRowTile rows
   // (its MMA N) per tile: tiles follow the 64-row prefix.
   const auto swap_rows = [&](GemmCall& g) {
-    if (g.swap && g.p.offsets) {
+    if (g.swap && g.p.offsets && !g.wide) {
       g.p.row_tile = kSwapRowTile;
-      g.p.tile_prefix = h->tile_prefix64;
-      g.p.max_row_tiles = (int)(g.out_rows / kSwapRowTile + h->N);  // routed rows
+      g.p.tile_prefix = g.grp->tp64;
+      g.p.max_row_tiles = (int)(g.out_rows / kSwapRowTile + g.grp->G);  // routed rows
+      // the expert FC1 (the longer weight stream, with the fewer tiles per
+      // CTA): stream-K over (tile, K block) units once there are two tiles
+      // per CTA (decided in the kernel from the tile count).  For FC2, whose
+      // tiles are short and many, the whole-tile split measured faster.
+      g.p.stream_k = (h->sk_part && g.kind == GK_FC1) ? 1 : 0;
+      g.p.sk_part = h->sk_part;
+      g.p.sk_count = h->sk_count;
     }
   };
   if (c.p.w_scale) {
@@ -525,19 +589,19 @@ lmoe_status run_gemm(lmoe_layer* h, GemmCall c, cudaStream_t st, int* path = nul
                     : launch_tc<TcCfg<false, false, false, 256, EPI_SCALE_ROWS, true>>(h, c, st);
     return LMOE_ERR_INVALID_ARG;
   }
-  if (c.pair && c.p.gather != nullptr) {
-    // the pair kernels read activations with TMA only
+  if (c.pair && c.p.gather != nullptr && c.kind != GK_FC1) {
+    // the pair kernels gather rows by index only for the expert FC1
     c.pair = false;
     c.p.row_tile = kRowTile;
-    c.p.tile_prefix = h->tile_prefix;
+    c.p.tile_prefix = c.grp ? c.grp->tp128 : nullptr;
   }
   if (!tc_eligible(h, c)) {
-    if (c.pair) {  // the CUDA-core kernel tiles by 128 rows
+    if (c.pair || c.wide) {  // the CUDA-core kernel tiles by 128 rows
       c.pair = false;
       c.p.row_tile = kRowTile;
-      c.p.tile_prefix = h->tile_prefix;
+      c.p.tile_prefix = c.grp ? c.grp->tp128 : nullptr;
       if (!c.p.offsets) c.p.max_row_tiles = (c.p.M + kRowTile - 1) / kRowTile;
-      else c.p.max_row_tiles = (int)((c.a_rows + kRowTile - 1) / kRowTile + h->N);
+      else c.p.max_row_tiles = (int)((c.out_rows + kRowTile - 1) / kRowTile + c.grp->G);
     }
     if (path) *path = 0;
     return h->dtype == LMOE_F32 ? dispatch_simt<float>(h, c, st) : dispatch_simt<bf16>(h, c, st);
@@ -548,8 +612,26 @@ lmoe_status run_gemm(lmoe_layer* h, GemmCall c, cudaStream_t st, int* path = nul
     if (c.kind == GK_FC1 && c.p.gather)
       return dual ? launch_pair_ws<TcPairWsCfg<true, true, EPI_ACT>>(h, c, st)
                   : launch_pair_ws<TcPairWsCfg<true, false, EPI_ACT>>(h, c, st);
+    if (c.kind == GK_FC1)  // rows already in expert order (LMOE_SORTED_ROWS)
+      return dual ? launch_pair_ws<TcPairWsCfg<false, true, EPI_ACT>>(h, c, st)
+                  : launch_pair_ws<TcPairWsCfg<false, false, EPI_ACT>>(h, c, st);
     if (c.kind == GK_FC2 && !c.p.gather)
       return launch_pair_ws<TcPairWsCfg<false, false, EPI_SCALE_ROWS>>(h, c, st);
+  }
+  if (c.swap && c.wide && c.p.offsets) {
+    // weight-stationary tiles of up to 128 (gated FC1: two accumulators) or
+    // 256 rows, rows gathered by cp.async (FC1) or loaded by TMA (FC2)
+    if (path) *path = 2;
+    if (c.kind == GK_FC1 && c.p.gather && c.wide == (dual ? 128 : 256))
+      return dual ? launch_tc<TcCfg<true, true, true, 128, EPI_ACT, false, 128>>(h, c, st)
+                  : launch_tc<TcCfg<true, true, false, 128, EPI_ACT, false, 256>>(h, c, st);
+    if (c.kind == GK_FC1 && c.wide == (dual ? 128 : 256))  // rows in expert order
+      return dual ? launch_tc<TcCfg<true, false, true, 128, EPI_ACT, false, 128>>(h, c, st)
+                  : launch_tc<TcCfg<true, false, false, 128, EPI_ACT, false, 256>>(h, c, st);
+    if (c.kind == GK_FC2 && !c.p.gather && !dual && c.wide == 256)
+      return launch_tc<TcCfg<true, false, false, 128, EPI_SCALE_ROWS, false, 256>>(h, c, st);
+    h->detail = "no wide weight-stationary kernel for this call";
+    return LMOE_ERR_INVALID_ARG;
   }
   if (path) *path = c.pair ? 3 : (c.swap ? 2 : 1);
   swap_rows(c);
@@ -561,7 +643,12 @@ lmoe_status run_gemm(lmoe_layer* h, GemmCall c, cudaStream_t st, int* path = nul
   if (c.pair) {
     switch (c.kind) {
       case GK_DENSE_ACT:
+        return dual ? launch_pair<TcPairCfg<true, EPI_ACT>>(h, c, st)
+                    : launch_pair<TcPairCfg<false, EPI_ACT>>(h, c, st);
       case GK_FC1:
+        if (c.p.gather)
+          return dual ? launch_pair<TcPairCfg<true, EPI_ACT, true>>(h, c, st)
+                      : launch_pair<TcPairCfg<false, EPI_ACT, true>>(h, c, st);
         return dual ? launch_pair<TcPairCfg<true, EPI_ACT>>(h, c, st)
                     : launch_pair<TcPairCfg<false, EPI_ACT>>(h, c, st);
       case GK_FC2: return launch_pair<TcPairCfg<false, EPI_SCALE_ROWS>>(h, c, st);
@@ -575,6 +662,13 @@ lmoe_status run_gemm(lmoe_layer* h, GemmCall c, cudaStream_t st, int* path = nul
       return dual ? launch_tc<TcCfg<false, false, true, 128, EPI_ACT>>(h, c, st)
                   : launch_tc<TcCfg<false, false, false, 256, EPI_ACT>>(h, c, st);
     case GK_FC1:
+      if (!c.p.gather) {  // rows already in expert order (LMOE_SORTED_ROWS)
+        if (c.swap)
+          return dual ? launch_tc<TcCfg<true, false, true, 128, EPI_ACT>>(h, c, st)
+                      : launch_tc<TcCfg<true, false, false, 128, EPI_ACT>>(h, c, st);
+        return dual ? launch_tc<TcCfg<false, false, true, 128, EPI_ACT>>(h, c, st)
+                    : launch_tc<TcCfg<false, false, false, 256, EPI_ACT>>(h, c, st);
+      }
       if (c.swap)
         return dual ? launch_tc<TcCfg<true, true, true, 128, EPI_ACT>>(h, c, st)
                     : launch_tc<TcCfg<true, true, false, 128, EPI_ACT>>(h, c, st);
@@ -613,43 +707,71 @@ void make_pair(const lmoe_layer* h, GemmCall& c) {
   c.pair = true;
   c.p.row_tile = 2 * kRowTile;
   if (c.p.offsets) {
-    c.p.tile_prefix = h->tile_prefix2;
-    const long R = (long)c.a_rows;
-    c.p.max_row_tiles = (int)((R + 2 * kRowTile - 1) / (2 * kRowTile) + h->N);
+    c.p.tile_prefix = c.grp->tp256;
+    const long R = (long)c.out_rows;
+    c.p.max_row_tiles = (int)((R + 2 * kRowTile - 1) / (2 * kRowTile) + c.grp->G);
   } else {
     c.p.max_row_tiles = (c.p.M + 2 * kRowTile - 1) / (2 * kRowTile);
   }
 }
 
-GemmCall grouped_call(const lmoe_layer* h, GemmKind kind, int T, const void* A, long lda,
-                      long a_rows, const int* gather, const void* B, long stride, int F, int K) {
+// A grouped expert GEMM over the R rows of grouping g: the weights of the
+// group's experts start at expert g.e0 of the stack B (elem_bytes each).
+GemmCall grouped_call(const Grouping& g, GemmKind kind, long R, const void* A, long lda,
+                      long a_rows, const int* gather, const void* B, size_t elem_bytes,
+                      long stride, int F, int K) {
   GemmCall c;
   std::memset(&c, 0, sizeof c);
-  const long R = (long)T * h->k;
   c.kind = kind;
-  c.p.offsets = h->offsets;
-  c.p.tile_prefix = h->tile_prefix;
-  c.p.G = h->N;
-  c.p.max_row_tiles = (int)((R + kRowTile - 1) / kRowTile + h->N);
+  c.grp = &g;
+  c.p.offsets = g.offsets;
+  c.p.tile_prefix = g.tp128;
+  c.p.G = g.G;
+  c.p.max_row_tiles = (int)((R + kRowTile - 1) / kRowTile + g.G);
   c.p.row_tile = kRowTile;
   c.p.A = A;
   c.p.lda = lda;
   c.p.gather = gather;
-  c.p.B = B;
+  c.p.B = static_cast<const char*>(B) + (size_t)g.e0 * stride * K * elem_bytes;
   c.p.w_group_stride = stride;
   c.p.F = F;
   c.p.K = K;
   c.a_rows = a_rows;
-  c.b_rows = (long)h->N * stride;
+  c.b_rows = (long)g.G * stride;
   c.out_rows = R;
   c.p.epi.act = ACT_NONE;
   return c;
 }
 
-bool use_swap(const lmoe_layer* h, int T) {
+// A prefill expert GEMM split by load: the experts with more than
+// kPairMinRows rows on CTA pairs (256-row token tiles; FC1 gathers its rows
+// by token in both CTAs), the others on single-CTA weight-stationary tiles
+// of the expert's rows rounded up to 16 (at most 128 rows for the gated FC1,
+// whose two accumulators share the tensor memory, 256 otherwise).  Two
+// launches that write disjoint rows of the output; the tile counts of each
+// come from the grouping step's big / small prefixes.
+lmoe_status run_split_by_load(lmoe_layer* h, const GemmCall& c, cudaStream_t st, int* path) {
+  GemmCall big = c;
+  make_pair(h, big);
+  big.p.tile_prefix = c.grp->big256;
+  LMOE_TRY(run_gemm(h, big, st));
+  GemmCall small = c;
+  small.pair = false;
+  small.swap = true;
+  const bool dual = c.kind == GK_FC1 && c.p.dual_offset > 0;
+  small.wide = dual ? 128 : 256;
+  small.p.row_tile = small.wide;
+  small.p.tile_prefix = dual ? c.grp->small128 : c.grp->small256;
+  small.p.max_row_tiles = (int)(c.out_rows / small.wide + c.grp->G);
+  LMOE_TRY(run_gemm(h, small, st));
+  *path = 5;
+  return LMOE_OK;
+}
+
+bool use_swap(const lmoe_layer* h, long R, int G) {
   if (h->flags & LMOE_FORCE_SWAP) return true;
   if (h->flags & LMOE_FORCE_NOSWAP) return false;
-  return (long)T * h->k < 64L * h->N;  // fewer than 64 rows per expert on average
+  return R < 64L * G;  // fewer than 64 rows per expert on average
 }
 
 // Records boundary i of the current profiled forward if a recorded stage
@@ -670,23 +792,54 @@ void prof_mark(lmoe_layer* h, cudaStream_t st, int i) {
 
 // ---- the routing steps ---------------------------------------------------------
 
+// Whether the routing runs with the default variant (renormalised gates over
+// logits that include the bias).
+bool default_routing(const lmoe_layer* h) {
+  return !(h->flags & (LMOE_ROUTE_BIAS_SELECT | LMOE_ROUTE_FULL_SOFTMAX));
+}
+
+// Top-k and grouping.  part_S > 0: the logits are still the router's S
+// split-K partial slices in h->part, summed (with the bias) by the top-k
+// kernel, which writes them to `logits`.
 lmoe_status run_routing(lmoe_layer* h, const float* logits, int T, int* idx, float* w,
                         int* offsets, int* row_tok, int* row_slot, float* row_w, int* slot_row,
-                        int* tile_prefix2, cudaStream_t st, bool marks) {
+                        int* tile_prefix2, cudaStream_t st, bool marks, int part_S = 0) {
   const int W = (T + 31) / 32;
   const int debug = (h->flags & LMOE_DEBUG_CHECKS) ? 1 : 0;
   {
-    const float* sel_bias = (h->flags & LMOE_ROUTE_BIAS_SELECT) ? h->bias : nullptr;
-    const int full = (h->flags & LMOE_ROUTE_FULL_SOFTMAX) ? 1 : 0;
-    const cudaError_t e = launch_topk(logits, T, h->N, h->k, sel_bias, full, idx, w, h->bitmap,
-                                      W, debug, h->err, st, take_pdl(h));
+    TopkArgs a;
+    std::memset(&a, 0, sizeof a);
+    a.logits = logits;
+    a.T = T;
+    a.N = h->N;
+    a.k = h->k;
+    a.sel_bias = (h->flags & LMOE_ROUTE_BIAS_SELECT) ? h->bias : nullptr;
+    a.full_softmax = (h->flags & LMOE_ROUTE_FULL_SOFTMAX) ? 1 : 0;
+    a.idx = idx;
+    a.w = w;
+    a.bitmap = h->bitmap;
+    a.W = W;
+    a.debug = debug;
+    a.err = h->err;
+    if (part_S > 0) {
+      a.logits = nullptr;
+      a.part = h->part;
+      a.S = part_S;
+      a.slice = (long)T * h->N;
+      a.pbias = h->bias;
+      a.logits_out = const_cast<float*>(logits);
+    }
+    const cudaError_t e = launch_topk_args(a, st, take_pdl(h));
     if (e != cudaSuccess) return cuda_fail(h, e, "top-k launch");
     ++h->launches;
   }
   if (marks) prof_mark(h, st, 2);
   LMOE_LAUNCH(h, group_count_kernel, dim3((h->N + 7) / 8), dim3(256), 0, st, h->bitmap, h->wp,
               h->N, W, h->counts, offsets, h->tile_prefix, tile_prefix2,
-              tile_prefix2 ? h->tile_prefix64 : (int*)nullptr, h->done);
+              tile_prefix2 ? h->tile_prefix64 : (int*)nullptr, h->done,
+              tile_prefix2 ? h->big_prefix2 : (int*)nullptr,
+              tile_prefix2 ? h->small_prefix : (int*)nullptr,
+              tile_prefix2 ? h->small_prefix2 : (int*)nullptr);
   const long P = (long)T * h->k;
   LMOE_LAUNCH(h, group_rank_kernel, dim3((unsigned)((P + 255) / 256)), dim3(256), 0, st,
               (const int*)idx, (const float*)w, (const uint2*)h->wp, (const int*)offsets, T, h->k,
@@ -694,13 +847,30 @@ lmoe_status run_routing(lmoe_layer* h, const float* logits, int T, int* idx, flo
   return LMOE_OK;
 }
 
-lmoe_status run_router(lmoe_layer* h, const void* x, float* logits, int T, cudaStream_t st) {
+// The router GEMM.  With part_S (the forward, default routing) a call that
+// splits K leaves its partial slices in h->part for the top-k kernel to sum:
+// *part_S = the number of slices, else 0 and the logits are written.
+lmoe_status run_router(lmoe_layer* h, const void* x, float* logits, int T, cudaStream_t st,
+                       int* part_S = nullptr) {
   GemmCall c = dense_call(GK_ROUTER, T, x, h->d, h->Wg_t, h->N, h->d);
   c.p.epi.out = logits;
   c.p.epi.ldo = h->N;
   c.p.epi.bias = (h->flags & LMOE_ROUTE_BIAS_SELECT) ? nullptr : h->bias;
   if (h->dtype == LMOE_BF16 && T >= 1024 && !(h->flags & (LMOE_FORCE_SIMT | LMOE_FORCE_NOPAIR)))
     make_pair(h, c);
+  if (part_S) {
+    *part_S = 0;
+    c.p.err = h->err;
+    int kbs = 0;
+    if (!c.pair && default_routing(h) && tc_eligible(h, c)) {
+      const int S = choose_splits(h, c, kbs);
+      if (S > 1) {
+        LMOE_TRY(run_split_partials(h, c, S, kbs, st));
+        *part_S = S;
+        return LMOE_OK;
+      }
+    }
+  }
   return run_gemm(h, c, st);
 }
 
@@ -749,22 +919,19 @@ lmoe_status run_x_stages(lmoe_layer* h, const void* x, int T, bool pair_dense, b
   return LMOE_OK;
 }
 
-lmoe_status run_forward(lmoe_layer* h, const void* x, void* out, int T, cudaStream_t st) {
-  h->launches = 0;
+// Whether CTA pairs may be used at all, and for the dense GEMMs of T tokens.
+bool pairs_allowed(const lmoe_layer* h) {
+  return h->dtype == LMOE_BF16 && !(h->flags & (LMOE_FORCE_SIMT | LMOE_FORCE_NOPAIR));
+}
+bool pair_dense_for(const lmoe_layer* h, int T) { return pairs_allowed(h) && T >= 1024; }
+
+// Everything before the expert GEMMs: router, top-k, grouping (on the
+// caller's stream) and the x-only stages (down-projection, shared FC1; on
+// the side stream, joined before returning).  Profile marks 0-5.
+lmoe_status run_front(lmoe_layer* h, const void* x, int T, cudaStream_t st) {
   const bool skip = (h->flags & LMOE_SKIP_PROJ) != 0;
-  const int d = h->d, l = h->l, k = h->k, m = h->m, ms = h->shared_m;
-  const long R = (long)T * k;
-  const bool swap = use_swap(h, T);
-  const bool pairs_ok = h->dtype == LMOE_BF16 && !(h->flags & (LMOE_FORCE_SIMT | LMOE_FORCE_NOPAIR));
-  // CTA pairs for the dense GEMMs once there are enough rows to fill them,
-  // and for the token-tiled expert FC2 (its input rows are contiguous; the
-  // expert FC1 gathers its rows by token and stays on single CTAs)
-  const bool pair_dense = pairs_ok && T >= 1024;
-  const bool pair_fc2 = pairs_ok && !swap;
-  // on request: the expert GEMMs weight-stationary on CTA pairs (rows on the
-  // MMA's N, so an expert's last tile is padded to 16 rows, not 128 or 256)
-  const bool ws_pair = pairs_ok && !swap && (h->flags & LMOE_FORCE_WS_PAIR) &&
-                       !(h->flags & LMOE_FORCE_NOSWAP);
+  const int ms = h->shared_m;
+  const bool pair_dense = pair_dense_for(h, T);
   // The down-projection and the shared FC1 depend on x alone: forked onto the
   // side stream they overlap the router GEMM and the latency-bound routing
   // kernels (which fit on an SM beside a GEMM CTA).  st waits for the whole
@@ -783,10 +950,11 @@ lmoe_status run_forward(lmoe_layer* h, const void* x, void* out, int T, cudaStre
                           kSideMark0 + 2));
   }
   h->pdl_hold = true;
-  LMOE_TRY(run_router(h, x, h->logits, T, st));
+  int part_S = 0;
+  LMOE_TRY(run_router(h, x, h->logits, T, st, &part_S));
   prof_mark(h, st, 1);
   LMOE_TRY(run_routing(h, h->logits, T, h->idx, h->w, h->offsets, h->row_tok, h->row_slot,
-                       h->row_w, h->slot_row, h->tile_prefix2, st, true));
+                       h->row_w, h->slot_row, h->tile_prefix2, st, true, part_S));
   prof_mark(h, st, 3);
   if (side) {
     LMOE_CUDA(h, cudaStreamWaitEvent(st, h->ev_side, 0));
@@ -795,12 +963,37 @@ lmoe_status run_forward(lmoe_layer* h, const void* x, void* out, int T, cudaStre
   } else {
     LMOE_TRY(run_x_stages(h, x, T, pair_dense, false, st, 4, 5));
   }
+  return LMOE_OK;
+}
+
+// The two expert GEMMs over grouping g (R rows): hbuf[r] = act(A[src(r)]
+// W1[e]) with src = gather (or r), ysbuf[r] = row_w[r] * (hbuf[r] W2[e]).
+// Kernels: weight-stationary below 64 rows per expert on average, else
+// token-tiled (FC1 on single CTAs, FC2 on CTA pairs; or split by load).
+// Profile mark 6 between the two.  Sets h->expert_path.
+lmoe_status run_expert_gemms(lmoe_layer* h, const Grouping& g, const void* A, long lda, long a_rows,
+                             const int* gather, long R, void* hbuf, void* ysbuf,
+                             const float* row_w, cudaStream_t st) {
+  const int l = h->l, m = h->m;
+  const bool skip = (h->flags & LMOE_SKIP_PROJ) != 0;
+  const int cols = skip ? h->d : l;
+  const bool swap = use_swap(h, R, g.G);
+  const bool pairs_ok = pairs_allowed(h);
+  const bool fp8 = (h->flags & LMOE_EXPERTS_FP8) != 0;
+  // token-tiled expert GEMMs with FC1 on single CTAs and FC2 on CTA pairs,
+  // or (LMOE_LOAD_SPLIT) split by load: experts with many rows on CTA pairs,
+  // the rest on weight-stationary single-CTA tiles
+  const bool load_split = pairs_ok && !swap && !fp8 && (h->flags & LMOE_LOAD_SPLIT) &&
+                          !(h->flags & LMOE_FORCE_WS_PAIR) && l % 64 == 0 && m % 64 == 0;
+  const bool pair_fc2 = pairs_ok && !swap;
+  // on request: the expert GEMMs weight-stationary on CTA pairs (rows on the
+  // MMA's N, so an expert's last tile is padded to 16 rows, not 128 or 256)
+  const bool ws_pair = pairs_ok && !swap && (h->flags & LMOE_FORCE_WS_PAIR) &&
+                       !(h->flags & LMOE_FORCE_NOSWAP);
   {
-    const void* A = skip ? x : h->z;
-    const bool fp8 = (h->flags & LMOE_EXPERTS_FP8) != 0;
     if (fp8) {
       // the fp8 expert kernels multiply f16 operands: the FC1 input in f16
-      const long n = (long)T * (skip ? d : l);
+      const long n = a_rows * cols;
       const int vec = (n % 8 == 0 && aligned16(A) && aligned16(h->a16)) ? 1 : 0;
       const long work = vec ? n / 8 : n;
       const unsigned blocks = (unsigned)std::max<long>(1, std::min<long>((work + 255) / 256,
@@ -809,35 +1002,67 @@ lmoe_status run_forward(lmoe_layer* h, const void* x, void* out, int T, cudaStre
                   static_cast<const bf16*>(A), static_cast<__half*>(h->a16), n, vec);
       A = h->a16;
     }
-    GemmCall c = grouped_call(h, GK_FC1, T, A, skip ? d : l, T, h->row_tok,
-                              fp8 ? (const void*)h->W1q_t : h->W1_t, h->m_in, m, l);
-    c.p.w_scale = fp8 ? h->W1s : nullptr;
+    const bool sorted = (h->flags & LMOE_SORTED_ROWS) && h->dtype == LMOE_BF16 && !fp8 && gather;
+    if (sorted) {
+      // the FC1 input rows copied into expert order: FC1 then loads them as
+      // contiguous tiles (by TMA) like FC2 does its input
+      const int vec = (cols % 8 == 0 && lda % 8 == 0 && aligned16(A) && aligned16(h->zs)) ? 1 : 0;
+      const unsigned blocks =
+          (unsigned)std::max<long>(1, std::min<long>((R + 7) / 8, 8L * h->num_sms));
+      LMOE_LAUNCH(h, gather_rows_kernel, dim3(blocks), dim3(256), 0, st,
+                  static_cast<const uint16_t*>(A), lda, gather, R, cols,
+                  static_cast<uint16_t*>(h->zs), vec);
+      A = h->zs;
+      lda = cols;
+      a_rows = R;
+      gather = nullptr;
+    }
+    GemmCall c = grouped_call(g, GK_FC1, R, A, lda, a_rows, gather,
+                              fp8 ? (const void*)h->W1q_t : h->W1_t, fp8 ? 1 : h->es, h->m_in,
+                              m, l);
+    c.p.w_scale = fp8 ? h->W1s + (size_t)g.e0 * h->m_in : nullptr;
     c.swap = swap;
     c.ws_pair = ws_pair && !fp8;
     c.p.dual_offset = h->act == LMOE_ACT_SWIGLU ? m : 0;
-    c.p.epi.out = h->h;
+    c.p.epi.out = hbuf;
     c.p.epi.ldo = m;
     c.p.epi.act = h->act;
     int path = 0;
-    LMOE_TRY(run_gemm(h, c, st, &path));
+    if (load_split) LMOE_TRY(run_split_by_load(h, c, st, &path));
+    else LMOE_TRY(run_gemm(h, c, st, &path));
     h->expert_path = path;
   }
   prof_mark(h, st, 6);
   {
-    const bool fp8 = (h->flags & LMOE_EXPERTS_FP8) != 0;
-    GemmCall c = grouped_call(h, GK_FC2, T, h->h, m, R, nullptr,
-                              fp8 ? (const void*)h->W2q_t : h->W2_t, l, l, m);
-    c.p.w_scale = fp8 ? h->W2s : nullptr;
-    if (pair_fc2 && !ws_pair && !fp8) make_pair(h, c);  // the pair kernels read bf16 weights
+    GemmCall c = grouped_call(g, GK_FC2, R, hbuf, m, R, nullptr,
+                              fp8 ? (const void*)h->W2q_t : h->W2_t, fp8 ? 1 : h->es, l, l, m);
+    c.p.w_scale = fp8 ? h->W2s + (size_t)g.e0 * l : nullptr;
     c.swap = swap;
     c.ws_pair = ws_pair && !fp8;
-    c.p.epi.out = h->ys;
+    c.p.epi.out = ysbuf;
     c.p.epi.ldo = l;
-    c.p.epi.row_w = h->row_w;
+    c.p.epi.row_w = row_w;
     int path = 0;
-    LMOE_TRY(run_gemm(h, c, st, &path));
+    if (load_split) {
+      LMOE_TRY(run_split_by_load(h, c, st, &path));
+    } else {
+      if (pair_fc2 && !ws_pair && !fp8) make_pair(h, c);  // the pair kernels read bf16 weights
+      LMOE_TRY(run_gemm(h, c, st, &path));
+    }
     h->expert_path |= path << 3;
   }
+  return LMOE_OK;
+}
+
+// Everything after the expert GEMMs: the gate-weighted sum of each token's k
+// rows of ys (rows in the grouping's order, found through slot_row), then the
+// up-projection with the shared expert and the residual (or, skipping the
+// projections, the residual and the fp32 shared output in the combine).
+// Profile marks 7-9.
+lmoe_status run_back(lmoe_layer* h, const void* x, const void* ys, void* out, int T,
+                     cudaStream_t st) {
+  const bool skip = (h->flags & LMOE_SKIP_PROJ) != 0;
+  const int d = h->d, l = h->l, k = h->k, ms = h->shared_m;
   prof_mark(h, st, 7);
   {
     const void* resid = skip ? x : nullptr;
@@ -845,7 +1070,7 @@ lmoe_status run_forward(lmoe_layer* h, const void* x, void* out, int T, cudaStre
     void* dst = skip ? out : h->cat;
     const long ldo = skip ? d : h->Kup;
     const int vec = 16 / h->es;
-    const bool vec_ok = (l % vec == 0) && (ldo % vec == 0) && aligned16(dst) && aligned16(h->ys) &&
+    const bool vec_ok = (l % vec == 0) && (ldo % vec == 0) && aligned16(dst) && aligned16(ys) &&
                         (!resid || (aligned16(resid) && d % vec == 0));
     const int threads = std::min(256, std::max(32, (l / vec + 31) / 32 * 32));
     // split a token's columns over blocks when T alone does not fill the GPU
@@ -856,19 +1081,19 @@ lmoe_status run_forward(lmoe_layer* h, const void* x, void* out, int T, cudaStre
     const long ldr = d;
     if (h->dtype == LMOE_BF16) {
       if (vec_ok)
-        LMOE_LAUNCH(h, combine_kernel<bf16>, cgrid, dim3(threads), 0, st, (const bf16*)h->ys,
+        LMOE_LAUNCH(h, combine_kernel<bf16>, cgrid, dim3(threads), 0, st, (const bf16*)ys,
                     (const int*)h->slot_row, k, l, (const bf16*)resid, ldr, add32, (bf16*)dst, ldo);
       else
-        LMOE_LAUNCH(h, combine_scalar_kernel<bf16>, dim3(T), dim3(256), 0, st, (const bf16*)h->ys,
+        LMOE_LAUNCH(h, combine_scalar_kernel<bf16>, dim3(T), dim3(256), 0, st, (const bf16*)ys,
                     (const int*)h->slot_row, k, l, (const bf16*)resid, ldr, add32, (bf16*)dst, ldo);
     } else {
       if (vec_ok)
-        LMOE_LAUNCH(h, combine_kernel<float>, cgrid, dim3(threads), 0, st, (const float*)h->ys,
+        LMOE_LAUNCH(h, combine_kernel<float>, cgrid, dim3(threads), 0, st, (const float*)ys,
                     (const int*)h->slot_row, k, l, (const float*)resid, ldr, add32, (float*)dst,
                     ldo);
       else
         LMOE_LAUNCH(h, combine_scalar_kernel<float>, dim3(T), dim3(256), 0, st,
-                    (const float*)h->ys, (const int*)h->slot_row, k, l, (const float*)resid, ldr,
+                    (const float*)ys, (const int*)h->slot_row, k, l, (const float*)resid, ldr,
                     add32, (float*)dst, ldo);
     }
   }
@@ -879,10 +1104,21 @@ lmoe_status run_forward(lmoe_layer* h, const void* x, void* out, int T, cudaStre
     c.p.epi.ldo = d;
     c.p.epi.resid = x;
     c.p.epi.ldr = d;
-    if (pair_dense) make_pair(h, c);
+    if (pair_dense_for(h, T)) make_pair(h, c);
     LMOE_TRY(run_gemm(h, c, st));
   }
   prof_mark(h, st, 9);
+  return LMOE_OK;
+}
+
+lmoe_status run_forward(lmoe_layer* h, const void* x, void* out, int T, cudaStream_t st) {
+  h->launches = 0;
+  const bool skip = (h->flags & LMOE_SKIP_PROJ) != 0;
+  const long R = (long)T * h->k;
+  LMOE_TRY(run_front(h, x, T, st));
+  LMOE_TRY(run_expert_gemms(h, h->fwd_grp, skip ? x : h->z, skip ? h->d : h->l, T, h->row_tok, R,
+                            h->h, h->ys, h->row_w, st));
+  LMOE_TRY(run_back(h, x, h->ys, out, T, st));
   if (h->profiling && h->prof_count < h->prof_cap) ++h->prof_count;
   h->last_T = T;
   return LMOE_OK;
@@ -905,6 +1141,11 @@ void free_workspace(lmoe_layer* h) {
   free_ptr(h->tile_prefix);
   free_ptr(h->tile_prefix2);
   free_ptr(h->tile_prefix64);
+  free_ptr(h->big_prefix2);
+  free_ptr(h->small_prefix);
+  free_ptr(h->small_prefix2);
+  free_ptr(h->sk_part);
+  free_ptr(h->sk_count);
   free_ptr(h->slot_row);
   free_ptr(h->done);
   free_ptr(h->err);
@@ -935,9 +1176,56 @@ void free_workspace(lmoe_layer* h) {
   h->host_slot = 0;
   free_ptr(h->s32);
   free_ptr(h->a16);
+  free_ptr(h->zs);
   free_ptr(h->part);
   h->part_bytes = 0;
   h->max_T = 0;
+}
+
+void free_ep(lmoe_layer* h) {
+  free_ptr(h->ep_tab);
+  if (h->ep_tab_host) cudaFreeHost(h->ep_tab_host);
+  h->ep_tab_host = nullptr;
+  if (h->ep_uploaded) cudaEventDestroy(h->ep_uploaded);
+  h->ep_uploaded = nullptr;
+  free_ptr(h->ep_perm);
+  free_ptr(h->ep_inv);
+  free_ptr(h->ep_gates);
+  free_ptr(h->ep_h);
+  free_ptr(h->ep_ys);
+  h->ep_max_rows = 0;
+}
+
+// Host tables of the received rows (see lmoe_ep_experts): per local expert
+// its total rows and grouped offset; per (source, expert) block its start in
+// the received order (roff, source-major) and in the grouped order (goff,
+// expert-major); each source's first received row (src_start).  Returns the
+// total, or -1 for a negative count.
+long ep_host_tables(const int* rc, int world, int n, int* counts, int* offsets, int* src_start,
+                    int* roff, int* goff) {
+  long run = 0;
+  for (int s = 0; s < world; ++s) {
+    src_start[s] = (int)run;
+    for (int e = 0; e < n; ++e) {
+      if (rc[(size_t)s * n + e] < 0) return -1;
+      roff[(size_t)s * n + e] = (int)run;
+      run += rc[(size_t)s * n + e];
+    }
+  }
+  src_start[world] = (int)run;
+  long g = 0;
+  for (int e = 0; e < n; ++e) {
+    offsets[e] = (int)g;
+    long c = 0;
+    for (int s = 0; s < world; ++s) {
+      goff[(size_t)e * world + s] = (int)(g + c);
+      c += rc[(size_t)s * n + e];
+    }
+    counts[e] = (int)c;
+    g += c;
+  }
+  offsets[n] = (int)g;
+  return run;
 }
 
 void free_weights(lmoe_layer* h) {
@@ -1017,7 +1305,8 @@ lmoe_status lmoe_create(int d, int l, int N, int k, int m, lmoe_act act, int sha
   const unsigned known = LMOE_SKIP_PROJ | LMOE_DEBUG_CHECKS | LMOE_FORCE_SIMT | LMOE_FORCE_SWAP |
                          LMOE_FORCE_NOSWAP | LMOE_FORCE_NOPAIR | LMOE_FORCE_WS_PAIR |
                          LMOE_ROUTE_FULL_SOFTMAX | LMOE_ROUTE_BIAS_SELECT | LMOE_EXPERTS_FP8 |
-                         LMOE_SINGLE_STREAM | LMOE_NO_PDL;
+                         LMOE_SINGLE_STREAM | LMOE_NO_PDL | LMOE_LOAD_SPLIT |
+                         LMOE_NO_STREAM_K | LMOE_SORTED_ROWS;
   if (d <= 0 || l <= 0 || N <= 0 || k <= 0 || m <= 0 || shared_m < 0) return LMOE_ERR_INVALID_ARG;
   if (k > N || (flags & ~known)) return LMOE_ERR_INVALID_ARG;
   if (act != LMOE_ACT_SILU && act != LMOE_ACT_SWIGLU && act != LMOE_ACT_RELU2) return LMOE_ERR_INVALID_ARG;
@@ -1156,6 +1445,13 @@ lmoe_status lmoe_reserve(lmoe_layer* h, int max_T) {
   ALLOC(h->tile_prefix, (size_t)(h->N + 1) * sizeof(int));
   ALLOC(h->tile_prefix2, (size_t)(h->N + 1) * sizeof(int));
   ALLOC(h->tile_prefix64, (size_t)(h->N + 1) * sizeof(int));
+  ALLOC(h->big_prefix2, (size_t)(h->N + 1) * sizeof(int));
+  ALLOC(h->small_prefix, (size_t)(h->N + 1) * sizeof(int));
+  ALLOC(h->small_prefix2, (size_t)(h->N + 1) * sizeof(int));
+  if (h->dtype == LMOE_BF16 && !(h->flags & LMOE_NO_STREAM_K)) {
+    ALLOC(h->sk_part, (size_t)2 * (h->num_sms + 1) * kSkSlotFloats * sizeof(float));
+    ALLOC(h->sk_count, (size_t)(h->num_sms + 1) * sizeof(int));
+  }
   ALLOC(h->slot_row, R * sizeof(int));
   ALLOC(h->done, sizeof(unsigned));
   ALLOC(h->err, sizeof(int));
@@ -1176,6 +1472,7 @@ lmoe_status lmoe_reserve(lmoe_layer* h, int max_T) {
   }
   if (skip && h->shared_m > 0) ALLOC(h->s32, T * h->d * sizeof(float));
   if (h->flags & LMOE_EXPERTS_FP8) ALLOC(h->a16, T * (skip ? h->d : h->l) * 2);
+  if (h->flags & LMOE_SORTED_ROWS) ALLOC(h->zs, R * (skip ? h->d : h->l) * 2);
   if (h->dtype == LMOE_BF16) {
     h->part_bytes = kSplitPartBytes;
     ALLOC(h->part, h->part_bytes);
@@ -1192,9 +1489,23 @@ lmoe_status lmoe_reserve(lmoe_layer* h, int max_T) {
   LMOE_CUDA(h, cudaMemset(h->tile_prefix, 0, (size_t)(h->N + 1) * sizeof(int)));
   LMOE_CUDA(h, cudaMemset(h->tile_prefix2, 0, (size_t)(h->N + 1) * sizeof(int)));
   LMOE_CUDA(h, cudaMemset(h->tile_prefix64, 0, (size_t)(h->N + 1) * sizeof(int)));
+  LMOE_CUDA(h, cudaMemset(h->big_prefix2, 0, (size_t)(h->N + 1) * sizeof(int)));
+  LMOE_CUDA(h, cudaMemset(h->small_prefix, 0, (size_t)(h->N + 1) * sizeof(int)));
+  LMOE_CUDA(h, cudaMemset(h->small_prefix2, 0, (size_t)(h->N + 1) * sizeof(int)));
+  if (h->sk_count) LMOE_CUDA(h, cudaMemset(h->sk_count, 0, (size_t)(h->num_sms + 1) * sizeof(int)));
   LMOE_CUDA(h, cudaDeviceSynchronize());
   h->max_T = max_T;
   h->W = (int)W;
+  Grouping& fg = h->fwd_grp;
+  fg.G = h->N;
+  fg.e0 = 0;
+  fg.offsets = h->offsets;
+  fg.tp128 = h->tile_prefix;
+  fg.tp256 = h->tile_prefix2;
+  fg.tp64 = h->tile_prefix64;
+  fg.big256 = h->big_prefix2;
+  fg.small128 = h->small_prefix;
+  fg.small256 = h->small_prefix2;
   return LMOE_OK;
 }
 
@@ -1413,6 +1724,171 @@ lmoe_status lmoe_profile_end(lmoe_layer* h, float* ms, int capacity, int* n_forw
   return LMOE_OK;
 }
 
+// ---- expert parallelism ------------------------------------------------------
+
+lmoe_status lmoe_ep_local_plan(const int* recv_counts, int world, int n_local, int* offsets,
+                               int* perm) {
+  if (!recv_counts || !offsets || world < 1 || n_local < 1) return LMOE_ERR_INVALID_ARG;
+  std::vector<int> counts(n_local), src(world + 1), roff((size_t)world * n_local),
+      goff((size_t)world * n_local);
+  const long Rr = ep_host_tables(recv_counts, world, n_local, counts.data(), offsets, src.data(),
+                                 roff.data(), goff.data());
+  if (Rr < 0 || Rr > INT32_MAX) return LMOE_ERR_INVALID_ARG;
+  if (Rr > 0 && !perm) return LMOE_ERR_INVALID_ARG;
+  for (int s = 0; s < world; ++s)
+    for (int e = 0; e < n_local; ++e) {
+      const int c = recv_counts[(size_t)s * n_local + e];
+      for (int i = 0; i < c; ++i) perm[goff[(size_t)e * world + s] + i] = roff[(size_t)s * n_local + e] + i;
+    }
+  return LMOE_OK;
+}
+
+lmoe_status lmoe_ep_reserve(lmoe_layer* h, int max_recv_rows) {
+  if (!h || max_recv_rows < 1) return LMOE_ERR_INVALID_ARG;
+  if (h->max_T == 0) return LMOE_ERR_NOT_READY;
+  if (max_recv_rows <= h->ep_max_rows) return LMOE_OK;
+  DevGuard g(h->device);
+  LMOE_CUDA(h, cudaDeviceSynchronize());
+  free_ep(h);
+  const size_t N = h->N, Rr = max_recv_rows, es = h->es;
+  const size_t tab = 4 * (N + 1) + 7 * (N + 1);
+#define ALLOC(ptr, bytes) LMOE_CUDA(h, cudaMalloc((void**)&(ptr), std::max<size_t>(bytes, 16)))
+  ALLOC(h->ep_tab, tab * sizeof(int));
+  LMOE_CUDA(h, cudaMallocHost((void**)&h->ep_tab_host, 4 * (N + 1) * sizeof(int)));
+  LMOE_CUDA(h, cudaEventCreateWithFlags(&h->ep_uploaded, cudaEventDisableTiming));
+  ALLOC(h->ep_perm, Rr * sizeof(int));
+  ALLOC(h->ep_inv, Rr * sizeof(int));
+  ALLOC(h->ep_gates, Rr * sizeof(float));
+  ALLOC(h->ep_h, Rr * h->m * es);
+  ALLOC(h->ep_ys, Rr * h->l * es);
+#undef ALLOC
+  LMOE_CUDA(h, cudaMemset(h->ep_tab, 0, tab * sizeof(int)));
+  h->ep_max_rows = max_recv_rows;
+  return LMOE_OK;
+}
+
+lmoe_status lmoe_ep_dispatch(lmoe_layer* h, const void* x, int T, void* send_rows,
+                             float* send_gates, int* expert_counts, lmoe_stream_t stream) {
+  if (!h) return LMOE_ERR_INVALID_ARG;
+  if (!layer_ready(h) || h->max_T == 0) return LMOE_ERR_NOT_READY;
+  if (h->flags & LMOE_EXPERTS_FP8) return LMOE_ERR_UNSUPPORTED;
+  if (T < 1 || T > h->max_T || !x || !send_rows || !send_gates || !expert_counts)
+    return LMOE_ERR_INVALID_ARG;
+  DevGuard g(h->device);
+  cudaStream_t st = (cudaStream_t)stream;
+  const bool prof = h->profiling;  // profiling covers lmoe_forward only
+  h->profiling = false;
+  h->launches = 0;
+  const lmoe_status r = run_front(h, x, T, st);
+  h->profiling = prof;
+  LMOE_TRY(r);
+  const bool skip = (h->flags & LMOE_SKIP_PROJ) != 0;
+  const int cols = skip ? h->d : h->l;
+  const void* A = skip ? x : h->z;
+  const long R = (long)T * h->k;
+  const int vec = (cols % 8 == 0 && aligned16(A) && aligned16(send_rows)) ? 1 : 0;
+  const unsigned blocks = (unsigned)std::max<long>(1, std::min<long>((R + 7) / 8, 8L * h->num_sms));
+  if (h->dtype == LMOE_BF16) {
+    LMOE_LAUNCH(h, gather_rows_kernel, dim3(blocks), dim3(256), 0, st,
+                static_cast<const uint16_t*>(A), (long)cols, (const int*)h->row_tok, R, cols,
+                static_cast<uint16_t*>(send_rows), vec);
+  } else {  // fp32 rows: two 16-bit halves per element
+    LMOE_LAUNCH(h, gather_rows_kernel, dim3(blocks), dim3(256), 0, st,
+                static_cast<const uint16_t*>(A), 2L * cols, (const int*)h->row_tok, R, 2 * cols,
+                static_cast<uint16_t*>(send_rows), vec);
+  }
+  LMOE_CUDA(h, cudaMemcpyAsync(send_gates, h->row_w, R * sizeof(float), cudaMemcpyDeviceToDevice,
+                               st));
+  LMOE_CUDA(h, cudaMemcpyAsync(expert_counts, h->counts, (size_t)h->N * sizeof(int),
+                               cudaMemcpyDeviceToDevice, st));
+  h->ep_T = T;
+  h->pdl_hold = true;  // the next launch follows memcpys: full stream order
+  return LMOE_OK;
+}
+
+lmoe_status lmoe_ep_experts(lmoe_layer* h, const void* recv_rows, const float* recv_gates,
+                            const int* recv_counts, int rank, int world, void* out_rows,
+                            lmoe_stream_t stream) {
+  if (!h) return LMOE_ERR_INVALID_ARG;
+  if (!layer_ready(h)) return LMOE_ERR_NOT_READY;
+  if (h->ep_max_rows == 0) return LMOE_ERR_NOT_READY;
+  if (h->flags & LMOE_EXPERTS_FP8) return LMOE_ERR_UNSUPPORTED;
+  if (!recv_counts || world < 1 || rank < 0 || rank >= world || h->N % world != 0)
+    return LMOE_ERR_INVALID_ARG;
+  const int n = h->N / world;
+  DevGuard g(h->device);
+  cudaStream_t st = (cudaStream_t)stream;
+  // host tables into the pinned staging buffer (after its previous upload)
+  LMOE_CUDA(h, cudaEventSynchronize(h->ep_uploaded));
+  const size_t N1 = (size_t)h->N + 1;
+  int* hc = h->ep_tab_host;  // counts [n] | src_start [world+1] | roff [world n] | goff [n world]
+  std::vector<int> offsets(n + 1);
+  const long Rr = ep_host_tables(recv_counts, world, n, hc, offsets.data(), hc + N1, hc + 2 * N1,
+                                 hc + 3 * N1);
+  if (Rr < 0) return LMOE_ERR_INVALID_ARG;
+  if (Rr > h->ep_max_rows) return LMOE_ERR_UNSUPPORTED;
+  if (Rr > 0 && (!recv_rows || !recv_gates || !out_rows)) return LMOE_ERR_INVALID_ARG;
+  h->launches = 0;
+  if (Rr == 0) return LMOE_OK;
+  int* dt = h->ep_tab;
+  LMOE_CUDA(h, cudaMemcpyAsync(dt, hc, 4 * N1 * sizeof(int), cudaMemcpyHostToDevice, st));
+  LMOE_CUDA(h, cudaEventRecord(h->ep_uploaded, st));
+  int* d_offsets = dt + 4 * N1;
+  int* pref = dt + 5 * N1;  // tp128, tp256, tp64, big256, small128, small256
+  h->pdl_hold = true;  // after a memcpy: full stream order
+  LMOE_LAUNCH(h, ep_scan_kernel, dim3(1), dim3(256), 0, st, (const int*)dt, n, d_offsets, pref,
+              pref + N1, pref + 2 * N1, pref + 3 * N1, pref + 4 * N1, pref + 5 * N1);
+  const unsigned pblocks =
+      (unsigned)std::max<long>(1, std::min<long>((Rr + 255) / 256, 8L * h->num_sms));
+  LMOE_LAUNCH(h, ep_perm_kernel, dim3(pblocks), dim3(256), 0, st, Rr, world, n,
+              (const int*)(dt + N1), (const int*)(dt + 2 * N1), (const int*)(dt + 3 * N1),
+              recv_gates, h->ep_perm, h->ep_inv, h->ep_gates);
+  Grouping& eg = h->ep_grp;
+  eg.G = n;
+  eg.e0 = rank * n;
+  eg.offsets = d_offsets;
+  eg.tp128 = pref;
+  eg.tp256 = pref + N1;
+  eg.tp64 = pref + 2 * N1;
+  eg.big256 = pref + 3 * N1;
+  eg.small128 = pref + 4 * N1;
+  eg.small256 = pref + 5 * N1;
+  const bool skip = (h->flags & LMOE_SKIP_PROJ) != 0;
+  const int cols = skip ? h->d : h->l;
+  const bool prof = h->profiling;
+  h->profiling = false;
+  const lmoe_status r = run_expert_gemms(h, eg, recv_rows, cols, Rr, h->ep_perm, Rr, h->ep_h,
+                                         h->ep_ys, h->ep_gates, st);
+  h->profiling = prof;
+  LMOE_TRY(r);
+  // the outputs back in received order
+  const int l = h->l;
+  const int vec = (l % 8 == 0 && aligned16(out_rows)) ? 1 : 0;
+  const unsigned blocks = (unsigned)std::max<long>(1, std::min<long>((Rr + 7) / 8, 8L * h->num_sms));
+  const int ecols = h->dtype == LMOE_BF16 ? l : 2 * l;
+  LMOE_LAUNCH(h, gather_rows_kernel, dim3(blocks), dim3(256), 0, st,
+              static_cast<const uint16_t*>(h->ep_ys), (long)ecols, (const int*)h->ep_inv, Rr, ecols,
+              static_cast<uint16_t*>(out_rows), vec);
+  return LMOE_OK;
+}
+
+lmoe_status lmoe_ep_combine(lmoe_layer* h, const void* x, const void* back_rows, void* out, int T,
+                            lmoe_stream_t stream) {
+  if (!h) return LMOE_ERR_INVALID_ARG;
+  if (h->ep_T < 0 || T != h->ep_T) return LMOE_ERR_NOT_READY;
+  if (!x || !back_rows || !out || x == out) return LMOE_ERR_INVALID_ARG;
+  DevGuard g(h->device);
+  const bool prof = h->profiling;
+  h->profiling = false;
+  h->launches = 0;
+  h->pdl_hold = true;  // the rows arrived by copies the library does not see
+  const lmoe_status r = run_back(h, x, back_rows, out, T, (cudaStream_t)stream);
+  h->profiling = prof;
+  h->ep_T = -1;
+  h->last_T = T;
+  return r;
+}
+
 int lmoe_last_launch_count(const lmoe_layer* h) { return h ? h->launches : 0; }
 int lmoe_last_expert_path(const lmoe_layer* h) { return h ? h->expert_path : -1; }
 
@@ -1423,6 +1899,7 @@ void lmoe_destroy(lmoe_layer* h) {
     cudaDeviceSynchronize();
     destroy_events(h);
     free_workspace(h);
+    free_ep(h);
     free_weights(h);
   }
   delete h;

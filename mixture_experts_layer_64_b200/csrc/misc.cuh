@@ -112,6 +112,31 @@ __global__ void __launch_bounds__(256) splitk_reduce_kernel(const float* __restr
   }
 }
 
+// dst[r] = src[row_tok[r]] for the R expert-sorted rows of 16-bit elements
+// (cols per row): the FC1 input rows in expert order, so that the expert
+// GEMM loads them as contiguous tiles instead of gathering them by token.
+// One warp per row, 16-byte vectors when cols is a multiple of 8 and both
+// row strides keep 16-byte alignment.
+__global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __restrict__ src,
+                                                          long lds, const int* __restrict__ row_tok,
+                                                          long R, int cols,
+                                                          uint16_t* __restrict__ dst, int vec) {
+  griddep_launch();
+  griddep_wait();  // the previous kernel's outputs are visible
+  const int lane = threadIdx.x & 31;
+  const long warps = (long)gridDim.x * (blockDim.x >> 5);
+  for (long r = (long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < R; r += warps) {
+    const uint16_t* s = src + (size_t)__ldg(row_tok + r) * lds;
+    uint16_t* d = dst + (size_t)r * cols;
+    if (vec) {
+      for (int c = lane * 8; c < cols; c += 256)
+        *reinterpret_cast<uint4*>(d + c) = __ldg(reinterpret_cast<const uint4*>(s + c));
+    } else {
+      for (int c = lane; c < cols; c += 32) d[c] = s[c];
+    }
+  }
+}
+
 // bf16 -> f16 for the FC1 input of a layer with fp8 expert weights (its
 // expert MMAs run on f16 operands): exact for magnitudes in [2^-14, 65504],
 // an absolute error below 2^-25 under that, saturating at +-65504 above.

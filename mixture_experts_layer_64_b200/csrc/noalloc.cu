@@ -16,8 +16,6 @@
 // zero before using them.
 #include <cuda_runtime.h>
 
-#include <mutex>
-
 #include "../../include/lmoe.h"
 #include "common.cuh"
 #include "routing.cuh"
@@ -28,7 +26,7 @@ namespace {
 
 // Layout of the scratch array for one call with W = ceil(T/32) words per
 // expert: bitmap [N*W] u32 | word prefixes [N*W] uint2 | counts [N] |
-// tile counts [N+1] | done counter | error word.
+// tile counts [N+1] | done counter.
 constexpr size_t kMaxWords = LMOE_NOALLOC_MAX_WORDS;
 constexpr size_t kBitmapBytes = kMaxWords * sizeof(uint32_t);
 constexpr size_t kPrefixBytes = kMaxWords * sizeof(uint2);
@@ -43,30 +41,22 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[LMOE_NOALLOC_SC
 
 namespace {
 
-constexpr int kMaxDevices = 64;
-std::mutex g_setup_mutex;
-unsigned char* g_scratch_addr[kMaxDevices] = {};
-
 // Device address of the scratch array on the current device.  In host code
 // the array's name is only a host-side stand-in, so the address comes from
-// cudaGetSymbolAddress, once per device, with that device current.
+// cudaGetSymbolAddress with the device current.  It is looked up on every
+// call (cheap once the module is loaded there), so a device reset, after
+// which the module and its array may sit elsewhere, leaves no stale address.
 lmoe_status scratch_for_current_device(unsigned char** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return LMOE_ERR_CUDA;
-  std::lock_guard<std::mutex> lock(g_setup_mutex);
-  if (!g_scratch_addr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return LMOE_ERR_CUDA;
-    g_scratch_addr[dev] = static_cast<unsigned char*>(p);
-  }
-  *out = g_scratch_addr[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return LMOE_ERR_CUDA;
+  *out = static_cast<unsigned char*>(p);
   return LMOE_OK;
 }
 
 }  // namespace
 
 extern "C" lmoe_status lmoe_route_only_noalloc(const float* logits, int T, int N, int k, int* idx,
-                                               float* w, int* offsets, int* perm,
+                                               float* w, int* offsets, int* perm, int* error_word,
                                                lmoe_stream_t stream) {
   if (N <= 0 || k <= 0 || k > N || T < 0 || !offsets) return LMOE_ERR_INVALID_ARG;
   if (T > 0 && (!logits || !idx || !w || !perm)) return LMOE_ERR_INVALID_ARG;
@@ -77,6 +67,8 @@ extern "C" lmoe_status lmoe_route_only_noalloc(const float* logits, int T, int N
   lmoe_status st = scratch_for_current_device(&base);
   if (st != LMOE_OK) return st;
   cudaStream_t s = (cudaStream_t)stream;
+  if (error_word && cudaMemsetAsync(error_word, 0, sizeof(int), s) != cudaSuccess)
+    return LMOE_ERR_CUDA;
   if (T == 0) {
     return cudaMemsetAsync(offsets, 0, (size_t)(N + 1) * sizeof(int), s) == cudaSuccess
                ? LMOE_OK : LMOE_ERR_CUDA;
@@ -85,20 +77,24 @@ extern "C" lmoe_status lmoe_route_only_noalloc(const float* logits, int T, int N
   uint2* wp = reinterpret_cast<uint2*>(base + kBitmapBytes);
   int* counts = reinterpret_cast<int*>(base + kBitmapBytes + kPrefixBytes);
   int* tile_prefix = reinterpret_cast<int*>(base + kBitmapBytes + kPrefixBytes + kCountBytes);
-  unsigned char* tail = base + kBitmapBytes + kPrefixBytes + kCountBytes + kTileBytes;
-  unsigned* done = reinterpret_cast<unsigned*>(tail);
-  int* err = reinterpret_cast<int*>(tail + 8);
+  unsigned* done =
+      reinterpret_cast<unsigned*>(base + kBitmapBytes + kPrefixBytes + kCountBytes + kTileBytes);
+  // With an error word the kernels run their device checks and flag into it.
+  const int debug = error_word ? 1 : 0;
   // The array keeps whatever the previous call left: clear the bitmap rows
   // this call sets bits in, and the block counter of the grouping scan.
   if (cudaMemsetAsync(bitmap, 0, (size_t)N * W * sizeof(uint32_t), s) != cudaSuccess ||
       cudaMemsetAsync(done, 0, sizeof(unsigned), s) != cudaSuccess)
     return LMOE_ERR_CUDA;
-  launch_topk(logits, T, N, k, nullptr, 0, idx, w, bitmap, (int)W, 0, err, s, false);
+  if (launch_topk(logits, T, N, k, nullptr, 0, idx, w, bitmap, (int)W, debug, error_word, s,
+                  false) != cudaSuccess)
+    return LMOE_ERR_CUDA;
   group_count_kernel<<<(N + 7) / 8, 256, 0, s>>>(bitmap, wp, N, (int)W, counts, offsets,
                                                  tile_prefix, nullptr, nullptr, done);
+  if (cudaGetLastError() != cudaSuccess) return LMOE_ERR_CUDA;
   const long P = (long)T * k;
   group_rank_kernel<<<(unsigned)((P + 255) / 256), 256, 0, s>>>(idx, w, wp, offsets, T, k, N,
                                                                  (int)W, nullptr, perm, nullptr,
-                                                                 nullptr, 0, err);
+                                                                 nullptr, debug, error_word);
   return cudaGetLastError() == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA;
 }

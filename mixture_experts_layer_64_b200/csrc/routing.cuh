@@ -76,6 +76,96 @@ __device__ __forceinline__ void warp_sort_desc64(unsigned long long& a, unsigned
   }
 }
 
+// Exclusive scans over the experts of their loads and tile counts (the
+// prefixes listed at group_count_kernel), by one block of up to 256 threads;
+// the counts were written by other blocks (read through L2).  NULL outputs
+// are skipped; entry N of each is the total.
+static __device__ __noinline__ void scan_loads_block(const int* counts, int N, int* offsets,
+                                              int* tile_prefix, int* tile_prefix2,
+                                              int* tile_prefix64, int* big_prefix2,
+                                              int* small_prefix, int* small_prefix2) {
+  constexpr int kQ = 7;
+  __shared__ int s_q[kQ][256];
+  const int nt = blockDim.x;
+  const int per = (N + nt - 1) / nt;
+  const int lo = threadIdx.x * per, hi = min(N, lo + per);
+  const auto tiles_of = [](int c, int* q) {
+    q[0] = c;
+    q[1] = (c + kRowTile - 1) / kRowTile;
+    q[2] = (c + 2 * kRowTile - 1) / (2 * kRowTile);
+    q[3] = (c + kSwapRowTile - 1) / kSwapRowTile;
+    q[4] = c > kPairMinRows ? q[2] : 0;
+    q[5] = c > kPairMinRows ? 0 : q[1];
+    q[6] = c > kPairMinRows ? 0 : q[2];
+  };
+  int sum[kQ] = {0, 0, 0, 0, 0, 0, 0};
+  for (int i = lo; i < hi; ++i) {
+    int q[kQ];
+    tiles_of(__ldcg(counts + i), q);
+#pragma unroll
+    for (int j = 0; j < kQ; ++j) sum[j] += q[j];
+  }
+#pragma unroll
+  for (int j = 0; j < kQ; ++j) s_q[j][threadIdx.x] = sum[j];
+  __syncthreads();
+  for (int o = 1; o < nt; o <<= 1) {
+    int add[kQ];
+#pragma unroll
+    for (int j = 0; j < kQ; ++j) add[j] = threadIdx.x >= o ? s_q[j][threadIdx.x - o] : 0;
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < kQ; ++j) s_q[j][threadIdx.x] += add[j];
+    __syncthreads();
+  }
+  int run[kQ];
+#pragma unroll
+  for (int j = 0; j < kQ; ++j) run[j] = s_q[j][threadIdx.x] - sum[j];
+  int* out[kQ] = {offsets,     tile_prefix,  tile_prefix2, tile_prefix64,
+                  big_prefix2, small_prefix, small_prefix2};
+  for (int i = lo; i < hi; ++i) {
+    int q[kQ];
+    tiles_of(__ldcg(counts + i), q);
+#pragma unroll
+    for (int j = 0; j < kQ; ++j) {
+      if (out[j]) out[j][i] = run[j];
+      run[j] += q[j];
+    }
+  }
+  if (threadIdx.x == nt - 1) {
+#pragma unroll
+    for (int j = 0; j < kQ; ++j)
+      if (out[j]) out[j][N] = s_q[j][nt - 1];
+  }
+  __syncthreads();
+}
+
+// The sorted row of pair pidx = t * k + j: offsets[e] + the number of tokens
+// below t routed to e (word prefix + popcount of the lower bits), and the
+// maps between rows, tokens, pairs and gates.  debug: range checks that flag
+// LMOE_DEVERR_RANGE and skip the pair.
+__device__ __forceinline__ void rank_pair(long pidx, const int* idx, const float* w,
+                                          const uint2* wp, const int* offsets, int T, int k, int N,
+                                          int W, int* row_tok, int* row_slot, float* row_w,
+                                          int* slot_row, int debug, int* err) {
+  const int t = (int)(pidx / k);
+  const int e = idx[pidx];
+  if (debug && (e < 0 || e >= N)) {
+    set_error(err, LMOE_DEVERR_RANGE);
+    return;
+  }
+  const uint2 x = wp[(size_t)e * W + (t >> 5)];
+  const int rank = (int)x.x + __popc(x.y & ((1u << (t & 31)) - 1u));
+  const int row = offsets[e] + rank;
+  if (debug && (row < 0 || row >= T * k)) {
+    set_error(err, LMOE_DEVERR_RANGE);
+    return;
+  }
+  if (row_tok) row_tok[row] = t;
+  if (slot_row) slot_row[pidx] = row;
+  row_slot[row] = (int)pidx;
+  if (row_w) row_w[row] = w[pidx];
+}
+
 // logits [T, N] fp32 -> idx [T, k], w [T, k]; bitmap [N, W] gets bit t of
 // token t set in the row of every chosen expert (W = ceil(T/32) words).
 //
@@ -96,26 +186,35 @@ __device__ __forceinline__ void warp_sort_desc64(unsigned long long& a, unsigned
 // bias steers the choice only); the gates always come from the logits:
 // renormalised over the k chosen, or (full_softmax) the softmax over all N
 // logits taken at the chosen experts.
+//
+// Fusion at decode sizes (default routing only): with part the logits are
+// the sums of the router's split-K partial slices (+ bias), written to
+// logits_out as the separate reduction would.
+struct TopkArgs {
+  const float* logits;  // [T, N], or NULL with part
+  int T, N, k;
+  const float* sel_bias;  // variants only
+  int full_softmax;       // variants only
+  int* idx;
+  float* w;
+  uint32_t* bitmap;  // [N, W]
+  int W, debug;
+  int* err;
+  // fused split-K reduction of the router logits
+  const float* part;  // S slices of [T, N] partial sums, `slice` floats apart
+  int S;
+  long slice;
+  const float* pbias;  // [N] or NULL
+  float* logits_out;   // [T, N]
+};
+
 template <int NPL, bool kVariant>
-__global__ void __launch_bounds__(128) topk_softmax_kernel(const float* __restrict__ logits, int T,
-                                                           int N, int k,
-                                                           const float* __restrict__ sel_bias,
-                                                           int full_softmax, int* __restrict__ idx,
-                                                           float* __restrict__ w,
-                                                           uint32_t* __restrict__ bitmap, int W,
-                                                           int debug, int* err) {
-  griddep_launch();
-  griddep_wait();  // the previous kernel's outputs are visible
-  __shared__ uint32_t s_hist[4][256];
-  __shared__ unsigned long long s_sel[4][64];
-  if (!kVariant) {
-    sel_bias = nullptr;
-    full_softmax = 0;
-  }
-  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
-  const int t = blockIdx.x * (blockDim.x >> 5) + wib;
-  if (t >= T) return;
-  const float* lg = logits + (size_t)t * N;
+__device__ __forceinline__ void topk_token(const TopkArgs& a, int t, int lane, uint32_t* s_hist,
+                                           unsigned long long* s_sel) {
+  const int N = a.N, k = a.k;
+  const float* sel_bias = kVariant ? a.sel_bias : nullptr;
+  const int full_softmax = kVariant ? a.full_softmax : 0;
+  const float* lg = a.logits + (size_t)t * N;
   uint32_t key[NPL];
   bool bad = false;
 #pragma unroll
@@ -123,13 +222,23 @@ __global__ void __launch_bounds__(128) topk_softmax_kernel(const float* __restri
     const int e = lane + 32 * i;
     key[i] = 0u;  // absent experts: 0, never above a real key and never counted
     if (e < N) {
-      float v = __ldg(lg + e);
-      if (debug && !isfinite(v)) bad = true;
+      float v;
+      if (a.part) {
+        // the router's split-K partial sums, added in slice order, then the
+        // bias: the same fp32 operations as the separate reduction
+        v = 0.f;
+        for (int sl = 0; sl < a.S; ++sl) v += __ldg(a.part + (size_t)sl * a.slice + (size_t)t * N + e);
+        v = v + (a.pbias ? __ldg(a.pbias + e) : 0.f);
+        a.logits_out[(size_t)t * N + e] = v;
+      } else {
+        v = __ldg(lg + e);
+      }
+      if (a.debug && !isfinite(v)) bad = true;
       if (sel_bias) v = __fadd_rn(v, __ldg(sel_bias + e));
       key[i] = orderable_bits(v);
     }
   }
-  if (debug && __any_sync(0xffffffffu, bad) && lane == 0) set_error(err, LMOE_DEVERR_NONFINITE);
+  if (a.debug && __any_sync(0xffffffffu, bad) && lane == 0) set_error(a.err, LMOE_DEVERR_NONFINITE);
 
   uint32_t lmax = 0u;
 #pragma unroll
@@ -143,7 +252,7 @@ __global__ void __launch_bounds__(128) topk_softmax_kernel(const float* __restri
 
   if (ncand > 64) {
     // radix select of the k-th largest key
-    uint32_t* hist = s_hist[wib];
+    uint32_t* hist = s_hist;
     uint32_t tau = 0u, tmask = 0u;
     int kk = k;  // rank of tau among the keys that match the decided digits
 #pragma unroll 1
@@ -208,7 +317,7 @@ __global__ void __launch_bounds__(128) topk_softmax_kernel(const float* __restri
     ncand = k;
   }
 
-  // compact the selected keys into s_sel[wib][0..ncand) (lane-major), then sort
+  // compact the selected keys into s_sel[0..ncand) (lane-major), then sort
   const uint32_t cnt = __popc(sel);
   uint32_t incl = cnt;
 #pragma unroll
@@ -220,14 +329,14 @@ __global__ void __launch_bounds__(128) topk_softmax_kernel(const float* __restri
 #pragma unroll
   for (int i = 0; i < NPL; ++i)
     if ((sel >> i) & 1u)
-      s_sel[wib][pos++] = ((unsigned long long)key[i] << 32) |
+      s_sel[pos++] = ((unsigned long long)key[i] << 32) |
                           (0xFFFFFFFFu - (uint32_t)(lane + 32 * i));
   __syncwarp();
-  unsigned long long v = lane < ncand ? s_sel[wib][lane] : 0ull;
+  unsigned long long v = lane < ncand ? s_sel[lane] : 0ull;
   if (ncand <= 32) {
     v = warp_sort_desc32(v, lane);
   } else {
-    unsigned long long b = lane + 32 < ncand ? s_sel[wib][lane + 32] : 0ull;
+    unsigned long long b = lane + 32 < ncand ? s_sel[lane + 32] : 0ull;
     warp_sort_desc64(v, b, lane);
   }
   const int e = (int)(0xFFFFFFFFu - (uint32_t)(v & 0xFFFFFFFFull));
@@ -255,30 +364,36 @@ __global__ void __launch_bounds__(128) topk_softmax_kernel(const float* __restri
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
   if (lane < k) {
-    idx[(size_t)t * k + lane] = e;
-    w[(size_t)t * k + lane] = ex / sum;
-    atomicOr(bitmap + (size_t)e * W + (t >> 5), 1u << (t & 31));
+    a.idx[(size_t)t * k + lane] = e;
+    a.w[(size_t)t * k + lane] = ex / sum;
+    atomicOr(a.bitmap + (size_t)e * a.W + (t >> 5), 1u << (t & 31));
   }
+}
+
+template <int NPL, bool kVariant>
+__global__ void __launch_bounds__(128) topk_softmax_kernel(const TopkArgs a) {
+  griddep_launch();
+  griddep_wait();  // the previous kernel's outputs are visible
+  __shared__ uint32_t s_hist[4][256];
+  __shared__ unsigned long long s_sel[4][64];
+  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+  const int t = blockIdx.x * (blockDim.x >> 5) + wib;
+  if (t < a.T) topk_token<NPL, kVariant>(a, t, lane, s_hist[wib], s_sel[wib]);
 }
 
 // Launches topk_softmax_kernel with the smallest multiple of 4 slots per lane
 // that covers N (pdl: programmatic stream serialisation).
-static inline cudaError_t launch_topk(const float* logits, int T, int N, int k,
-                                      const float* sel_bias, int full_softmax, int* idx, float* w,
-                                      uint32_t* bitmap, int W, int debug, int* err,
-                                      cudaStream_t st, bool pdl) {
-  const dim3 grid((T + 3) / 4), block(128);
-  const bool var = sel_bias != nullptr || full_softmax != 0;
+static inline cudaError_t launch_topk_args(const TopkArgs& a, cudaStream_t st, bool pdl) {
+  const dim3 grid((a.T + 3) / 4), block(128);
+  const bool var = a.sel_bias != nullptr || a.full_softmax != 0;
+  if (var && a.part) return cudaErrorInvalidValue;  // the fused reduction: default routing only
   cudaError_t e = cudaSuccess;
 #define LMOE_TOPK_CASE(S)                                                                   \
   case S:                                                                                   \
-    e = var ? launch_kernel(pdl, topk_softmax_kernel<S, true>, grid, block, 0, st, logits, T, \
-                            N, k, sel_bias, full_softmax, idx, w, bitmap, W, debug, err)     \
-            : launch_kernel(pdl, topk_softmax_kernel<S, false>, grid, block, 0, st, logits,  \
-                            T, N, k, (const float*)nullptr, 0, idx, w, bitmap, W, debug,    \
-                            err);                                                           \
+    e = var ? launch_kernel(pdl, topk_softmax_kernel<S, true>, grid, block, 0, st, a)       \
+            : launch_kernel(pdl, topk_softmax_kernel<S, false>, grid, block, 0, st, a);     \
     break;
-  switch ((N + 127) / 128 * 4) {
+  switch ((a.N + 127) / 128 * 4) {
     LMOE_TOPK_CASE(4)
     LMOE_TOPK_CASE(8)
     LMOE_TOPK_CASE(12)
@@ -294,8 +409,42 @@ static inline cudaError_t launch_topk(const float* logits, int T, int N, int k,
   return e != cudaSuccess ? e : cudaGetLastError();
 }
 
+// The plain top-k launch (no fusion): logits in, indices, gates and bitmaps out.
+static inline cudaError_t launch_topk(const float* logits, int T, int N, int k,
+                                      const float* sel_bias, int full_softmax, int* idx, float* w,
+                                      uint32_t* bitmap, int W, int debug, int* err,
+                                      cudaStream_t st, bool pdl) {
+  TopkArgs a;
+  memset(&a, 0, sizeof a);
+  a.logits = logits;
+  a.T = T;
+  a.N = N;
+  a.k = k;
+  a.sel_bias = sel_bias;
+  a.full_softmax = full_softmax;
+  a.idx = idx;
+  a.w = w;
+  a.bitmap = bitmap;
+  a.W = W;
+  a.debug = debug;
+  a.err = err;
+  return launch_topk_args(a, st, pdl);
+}
+
 // Word prefix + bits: wp[e][wd] = {set bits of expert e in words < wd, word wd}.
 // Also zeroes the bitmap.  The last block scans the loads.
+//
+// Tile prefixes (exclusive scans over experts, entry N = the total):
+//   tile_prefix      128-row tiles of every expert (single-CTA token tiles)
+//   tile_prefix2     256-row tiles of every expert (CTA-pair token tiles)
+//   tile_prefix64    64-row tiles of every expert (weight-stationary tiles)
+//   big_prefix2      256-row tiles of the experts with > kPairMinRows rows
+//   small_prefix     128-row tiles of the other experts
+//   small_prefix2    256-row tiles of the other experts
+// The last three split a prefill expert GEMM by load: experts with many rows
+// go to the CTA-pair kernel (their last tile's padding is small against
+// their rows), the rest to weight-stationary tiles of up to 128 (gated) or
+// 256 rows, padded to a multiple of 16 rows.  NULL pointers skip a prefix.
 static __global__ void __launch_bounds__(256) group_count_kernel(uint32_t* __restrict__ bitmap,
                                                           uint2* __restrict__ wp, int N, int W,
                                                           int* __restrict__ counts,
@@ -303,7 +452,10 @@ static __global__ void __launch_bounds__(256) group_count_kernel(uint32_t* __res
                                                           int* __restrict__ tile_prefix,
                                                           int* __restrict__ tile_prefix2,
                                                           int* __restrict__ tile_prefix64,
-                                                          unsigned int* done) {
+                                                          unsigned int* done,
+                                                          int* __restrict__ big_prefix2 = nullptr,
+                                                          int* __restrict__ small_prefix = nullptr,
+                                                          int* __restrict__ small_prefix2 = nullptr) {
   griddep_launch();
   griddep_wait();  // the previous kernel's outputs are visible
   const int lane = threadIdx.x & 31;
@@ -336,57 +488,9 @@ static __global__ void __launch_bounds__(256) group_count_kernel(uint32_t* __res
   __syncthreads();
   if (!is_last) return;
   __threadfence();
-  // Block-wide exclusive scans of counts and of ceil(counts / 128),
-  // ceil(counts / 256) and ceil(counts / 64) (row tiles of single CTAs, of
-  // CTA pairs, and of the weight-stationary kernel).
-  __shared__ int s_c[256], s_t[256], s_u[256], s_v[256];
-  const int per = (N + 255) / 256;
-  const int lo = threadIdx.x * per, hi = min(N, lo + per);
-  int c_sum = 0, t_sum = 0, u_sum = 0, v_sum = 0;
-  for (int i = lo; i < hi; ++i) {
-    const int c = __ldcg(counts + i);
-    c_sum += c;
-    t_sum += (c + kRowTile - 1) / kRowTile;
-    u_sum += (c + 2 * kRowTile - 1) / (2 * kRowTile);
-    v_sum += (c + kSwapRowTile - 1) / kSwapRowTile;
-  }
-  s_c[threadIdx.x] = c_sum;
-  s_t[threadIdx.x] = t_sum;
-  s_u[threadIdx.x] = u_sum;
-  s_v[threadIdx.x] = v_sum;
-  __syncthreads();
-  for (int o = 1; o < 256; o <<= 1) {
-    const int a = threadIdx.x >= o ? s_c[threadIdx.x - o] : 0;
-    const int b = threadIdx.x >= o ? s_t[threadIdx.x - o] : 0;
-    const int d = threadIdx.x >= o ? s_u[threadIdx.x - o] : 0;
-    const int f = threadIdx.x >= o ? s_v[threadIdx.x - o] : 0;
-    __syncthreads();
-    s_c[threadIdx.x] += a;
-    s_t[threadIdx.x] += b;
-    s_u[threadIdx.x] += d;
-    s_v[threadIdx.x] += f;
-    __syncthreads();
-  }
-  int c_run = s_c[threadIdx.x] - c_sum, t_run = s_t[threadIdx.x] - t_sum,
-      u_run = s_u[threadIdx.x] - u_sum, v_run = s_v[threadIdx.x] - v_sum;
-  for (int i = lo; i < hi; ++i) {
-    const int c = __ldcg(counts + i);
-    offsets[i] = c_run;
-    tile_prefix[i] = t_run;
-    if (tile_prefix2) tile_prefix2[i] = u_run;
-    if (tile_prefix64) tile_prefix64[i] = v_run;
-    c_run += c;
-    t_run += (c + kRowTile - 1) / kRowTile;
-    u_run += (c + 2 * kRowTile - 1) / (2 * kRowTile);
-    v_run += (c + kSwapRowTile - 1) / kSwapRowTile;
-  }
-  if (threadIdx.x == 255) {
-    offsets[N] = s_c[255];
-    tile_prefix[N] = s_t[255];
-    if (tile_prefix2) tile_prefix2[N] = s_u[255];
-    if (tile_prefix64) tile_prefix64[N] = s_v[255];
-    *done = 0u;
-  }
+  scan_loads_block(counts, N, offsets, tile_prefix, tile_prefix2, tile_prefix64, big_prefix2,
+                   small_prefix, small_prefix2);
+  if (threadIdx.x == 0) *done = 0u;
 }
 
 // row(t, j) = offsets[e] + rank of t among the tokens routed to e.
@@ -399,23 +503,7 @@ static __global__ void __launch_bounds__(256) group_rank_kernel(
   griddep_wait();  // the previous kernel's outputs are visible
   const long pidx = (long)blockIdx.x * blockDim.x + threadIdx.x;
   if (pidx >= (long)T * k) return;
-  const int t = (int)(pidx / k);
-  const int e = __ldg(idx + pidx);
-  if (debug && (e < 0 || e >= N)) {
-    set_error(err, LMOE_DEVERR_RANGE);
-    return;
-  }
-  const uint2 x = __ldg(wp + (size_t)e * W + (t >> 5));
-  const int rank = (int)x.x + __popc(x.y & ((1u << (t & 31)) - 1u));
-  const int row = __ldg(offsets + e) + rank;
-  if (debug && (row < 0 || row >= T * k)) {
-    set_error(err, LMOE_DEVERR_RANGE);
-    return;
-  }
-  if (row_tok) row_tok[row] = t;
-  if (slot_row) slot_row[pidx] = row;
-  row_slot[row] = (int)pidx;
-  if (row_w) row_w[row] = __ldg(w + pidx);
+  rank_pair(pidx, idx, w, wp, offsets, T, k, N, W, row_tok, row_slot, row_w, slot_row, debug, err);
 }
 
 }  // namespace lmoe

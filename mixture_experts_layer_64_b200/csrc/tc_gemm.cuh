@@ -47,10 +47,19 @@ constexpr int kEpiWarps = 8;  // two warpgroups; each warp reads its TMEM lane q
 constexpr int kTcSmemBudget = 200 * 1024;
 constexpr int kGatherThreads = 64;
 
-template <bool kSwap_, bool kGather_, bool kDual_, int kWN_, int kEpi_, bool kFp8_ = false>
+template <bool kSwap_, bool kGather_, bool kDual_, int kWN_, int kEpi_, bool kFp8_ = false,
+          int kSwapRows_ = kSwapRowTile>
 struct TcCfg {
   static constexpr bool kSwap = kSwap_, kGather = kGather_, kDual = kDual_, kFp8 = kFp8_;
   static constexpr int kEpi = kEpi_;
+  // weight-stationary tiles: rows per tile (the MMA's N) at most.  Up to 64
+  // rows (decode) the gathered rows arrive by four-row TMA gathers; wider
+  // tiles (prefill experts with up to a few hundred rows, 128 or 256 rows
+  // per tile) gather them with cp.async like the token-tiled kernel.
+  static constexpr int kSwapRows = kSwapRows_;
+  static constexpr bool kWideSwap = kSwap && kSwapRows > kSwapRowTile;
+  // activation rows gathered by cp.async threads (warps 2-3)
+  static constexpr bool kCpGather = kGather && (!kSwap || kWideSwap);
   // warps 0-3: producer, MMA issuer, gather; then the epilogue warps (two
   // warpgroups, or one with fp8 weights), then (fp8) the converter warps that
   // widen the E4M3 weight tiles to bf16
@@ -61,7 +70,7 @@ struct TcCfg {
   // input) is written in f16; FC2 writes bf16
   static constexpr bool kF16Out = kFp8 && kEpi_ == EPI_ACT;
   static constexpr int BK = 64;                       // bf16 per 128-byte swizzled row
-  static constexpr int ACT_ROWS = kSwap ? kSwapRowTile : 128;  // activation rows per stage
+  static constexpr int ACT_ROWS = kSwap ? kSwapRows : 128;  // activation rows per stage
   static constexpr int W_ROWS = kSwap ? 128 : (kDual ? 128 : kWN_);
   static constexpr int NUM_W = kDual ? 2 : 1;
   static constexpr int ACT_BYTES = ACT_ROWS * BK * 2;
@@ -83,7 +92,7 @@ struct TcCfg {
   static constexpr int S8_RAW = kFp8 ? (BUDGET - STAGES * STAGE_BYTES) / W8_SLOT : 0;
   static constexpr int S8 = S8_RAW > 16 ? 16 : S8_RAW;
   static constexpr int RING_BYTES = STAGES * STAGE_BYTES + S8 * W8_SLOT;
-  static constexpr int ACC_N = kSwap ? 128 : W_ROWS;  // fp32 columns of one accumulator
+  static constexpr int ACC_N = kSwap ? (kSwapRows > 128 ? kSwapRows : 128) : W_ROWS;  // fp32 columns of one accumulator
   static constexpr int ACC_COLS = ACC_N * NUM_W;      // one TMEM buffer
   static constexpr int TMEM_COLS = 2 * ACC_COLS;      // double buffered
   static constexpr int FT = W_ROWS;                   // features per tile
@@ -94,10 +103,12 @@ struct TcCfg {
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
   static_assert(STAGES >= 3, "pipeline too shallow");
   static_assert(!kFp8 || S8 >= 2, "fp8 weight ring too shallow");
-  static_assert(2 * STAGES * 8 + 2 * S8 * 8 + 5 * 8 + 8 <= 512, "barrier area");
+  static_assert(2 * STAGES * 8 + 2 * S8 * 8 + 6 * 8 + 16 <= 512, "barrier area");
   static_assert(!kSwap || kEpi == EPI_ACT || kEpi == EPI_SCALE_ROWS, "swap epilogues");
   static_assert(kWN_ == 128 || kWN_ == 256, "weight tile");
   static_assert(!kFp8 || kEpi == EPI_ACT || kEpi == EPI_SCALE_ROWS, "fp8 weights: expert GEMMs");
+  static_assert(kSwapRows == kSwapRowTile || kSwapRows == 128 || kSwapRows == 256, "swap rows");
+  static_assert(!kWideSwap || !kFp8, "wide weight-stationary tiles: bf16 weights");
 };
 
 // ---- fp8 E4M3 weights -----------------------------------------------------------
@@ -381,6 +392,56 @@ __device__ __forceinline__ int total_row_tiles_s(const GemmProblem& p, const int
   return s_tiles[p.G];
 }
 
+// ---- the work of one CTA ---------------------------------------------------------
+//
+// Tile-granular: tiles blockIdx.x, blockIdx.x + gridDim.x, ...; with split-K
+// tile t covers the K blocks of split t / tiles_per_split.
+// Stream-K (weight-stationary decode GEMMs, p.stream_k, and at least two
+// tiles per CTA): the (tile, K block) units are dealt out in equal
+// contiguous ranges, one per CTA, so that the weight stream ends on every SM
+// at the same time instead of in a last partial wave of whole tiles.  A
+// tile whose K blocks straddle two ranges is computed in two parts: the
+// "head" (its first K blocks, at the end of one CTA's range) and the "tail"
+// (the rest, at the start of the next CTA's range).  Each part writes its
+// fp32 accumulator to a slot; whichever arrives second adds the other's part
+// and runs the epilogue.  Two fp32 terms add the same in either order, so the
+// result does not depend on which part finishes first, and no CTA waits for
+// another.
+struct TileWalk {
+  int num_tiles, tiles_per_split, KB, KBS;
+  long u_end;  // stream-K: end of this CTA's unit range; -1: tile-granular
+};
+
+__device__ __forceinline__ long walk_start(const TileWalk& w) {
+  if (w.u_end < 0) return blockIdx.x;
+  const long total = (long)w.num_tiles * w.KB;
+  const long per = (total + gridDim.x - 1) / gridDim.x;
+  return min(total, (long)blockIdx.x * per);
+}
+
+// The next segment: tile tl (row tile * NT + feature tile), split ks, K
+// blocks [kb0, kb1).
+__device__ __forceinline__ bool walk_next(const TileWalk& w, long& it, int& tl, int& ks, int& kb0,
+                                          int& kb1) {
+  if (w.u_end >= 0) {
+    if (it >= w.u_end) return false;
+    tl = (int)(it / w.KB);
+    kb0 = (int)(it - (long)tl * w.KB);
+    kb1 = (int)min((long)w.KB, (long)kb0 + (w.u_end - it));
+    ks = 0;
+    it += kb1 - kb0;
+    return true;
+  }
+  if (it >= w.num_tiles) return false;
+  const int t = (int)it;
+  ks = t / w.tiles_per_split;
+  tl = t - ks * w.tiles_per_split;
+  kb0 = ks * w.KBS;
+  kb1 = min(w.KB, kb0 + w.KBS);
+  it += gridDim.x;
+  return true;
+}
+
 // ---- the kernel -----------------------------------------------------------------
 
 template <class Cfg>
@@ -399,8 +460,10 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
   uint64_t* tfull = w8empty + Cfg::S8;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* epibar = drain + 1;  // stream-K: the epilogue warps meet here
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(epibar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* sk_order = reinterpret_cast<volatile int*>(tmem_slot + 2);  // stream-K
   int* s_tiles = reinterpret_cast<int*>(stg_base + Cfg::STG_BYTES + 512);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -413,8 +476,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       // the producer (its expect_tx covers the weights and the activation
       // rows, including TMA-gathered ones) + the cp.async gather threads of
       // token-tiled tiles + (fp8) one lane per converter warp
-      mbar_init(&full[s], 1 + (Cfg::kGather && !Cfg::kSwap ? kGatherThreads : 0) +
-                              Cfg::CONV_THREADS / 32);
+      mbar_init(&full[s], 1 + (Cfg::kCpGather ? kGatherThreads : 0) + Cfg::CONV_THREADS / 32);
       mbar_init(&empty[s], 1);
     }
     for (int j = 0; j < Cfg::S8; ++j) {
@@ -426,6 +488,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       mbar_init(&tempty[b], Cfg::EPI_WARPS);
     }
     mbar_init(drain, 1);
+    mbar_init(epibar, Cfg::EPI_WARPS);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -449,6 +512,12 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
   const int KBS = S > 1 ? p.kb_per_split : KB;
   const int tiles_per_split = total_row_tiles_s(p, s_tiles) * NT;
   const int num_tiles = tiles_per_split * S;
+  TileWalk walk{num_tiles, tiles_per_split, KB, KBS, -1};
+  if (Cfg::kSwap && !Cfg::kWideSwap && p.stream_k && S == 1 && num_tiles >= 2 * (int)gridDim.x) {
+    const long total = (long)num_tiles * KB;
+    const long per = (total + gridDim.x - 1) / gridDim.x;
+    walk.u_end = min(total, (long)(blockIdx.x + 1) * per);
+  }
 
   if (warp == 0) {
     // ---------------- TMA producer ----------------
@@ -460,10 +529,9 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       uint32_t jph = 0;
       long wissued = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-        const int ks = t / tiles_per_split, tl = t - ks * tiles_per_split;
+      int tl, ks, kb0, kb1;
+      for (long wi = walk_start(walk); ok && walk_next(walk, wi, tl, ks, kb0, kb1);) {
         const int rt = tl / NT, ft = tl - (tl / NT) * NT;
-        const int kb0 = ks * KBS, kb1 = min(KB, kb0 + KBS);
         int g, row0, rows;
         locate_row_tile_s(p, s_tiles, rt, g, row0, rows);
         const int wrow = (int)(g * p.w_group_stride) + ft * Cfg::FT;
@@ -492,17 +560,16 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       int s = 0;
       uint32_t ph = 0;
       long armed = 0;
-      for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
-        const int ks = t / tiles_per_split, tl = t - ks * tiles_per_split;
+      int tl, ks, kb0, kb1;
+      for (long wi = walk_start(walk); walk_next(walk, wi, tl, ks, kb0, kb1);) {
         const int rt = tl / NT, ft = tl - (tl / NT) * NT;
-        const int kb0 = ks * KBS, kb1 = min(KB, kb0 + KBS);
         int g, row0, rows;
         locate_row_tile_s(p, s_tiles, rt, g, row0, rows);
         const int wrow = (int)(g * p.w_group_stride) + ft * Cfg::FT;
         const int nsub = Cfg::kSwap ? (rows + 31) / 32 : 4;
         uint32_t bytes = Cfg::kFp8 ? 0u : (uint32_t)(Cfg::NUM_W * Cfg::W_BYTES);
         if (!Cfg::kGather) bytes += Cfg::kSwap ? nsub * 4096 : Cfg::ACT_BYTES;
-        else if (Cfg::kSwap) bytes += max(16, (rows + 15) & ~15) * 128;  // TMA-gathered rows
+        else if (!Cfg::kCpGather) bytes += max(16, (rows + 15) & ~15) * 128;  // TMA-gathered rows
         bool ok = true;
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, p.err)) { ok = false; break; }
@@ -547,10 +614,9 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       int s = 0;
       uint32_t ph = 0;
       int it = 0;
-      for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++it) {
-        const int ks = t / tiles_per_split, tl = t - ks * tiles_per_split;
+      int tl, ks, kb0, kb1;
+      for (long wi = walk_start(walk); walk_next(walk, wi, tl, ks, kb0, kb1); ++it) {
         const int rt = tl / NT;
-        const int kb0 = ks * KBS, kb1 = min(KB, kb0 + KBS);
         int g, row0, rows;
         locate_row_tile_s(p, s_tiles, rt, g, row0, rows);
         const int ab = it & 1;
@@ -596,7 +662,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       tc_commit(drain);
       mbar_wait_drain(drain, 0);
     }
-  } else if (warp < 4 && Cfg::kGather && Cfg::kSwap) {
+  } else if (warp < 4 && Cfg::kGather && !Cfg::kCpGather) {
     // ---------------- TMA row gather (weight-stationary tiles) ----------------
     // Lane i of warp 2 brings rows 4i..4i+3 of each stage's activation tile
     // (at most 64 rows) with one gather4 (rows picked by token index; the
@@ -608,10 +674,9 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       int s = 0;
       uint32_t ph = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-        const int ks = t / tiles_per_split, tl = t - ks * tiles_per_split;
+      int tl, ks, kb0, kb1;
+      for (long wi = walk_start(walk); ok && walk_next(walk, wi, tl, ks, kb0, kb1);) {
         const int rt = tl / NT;
-        const int kb0 = ks * KBS, kb1 = min(KB, kb0 + KBS);
         int g, row0, rows;
         locate_row_tile_s(p, s_tiles, rt, g, row0, rows);
         const int nload = Cfg::kSwap ? max(16, (rows + 15) & ~15) : Cfg::ACT_ROWS;
@@ -633,13 +698,15 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       }
     }
   } else if (warp < 4) {
-    // ---------------- cp.async row gather (token-tiled tiles) ----------------
+    // ---------------- cp.async row gather (token-tiled and wide tiles) ----------------
     // Each thread copies 16-byte chunks of the tile's rows straight into the
     // 128-byte-swizzled layout, then hands the stage to the MMA issuer with an
     // mbarrier arrive that the hardware triggers when its copies have landed.
     // The thread never waits for its own copies, so all STAGES stages can be
-    // in flight.
-    if (Cfg::kGather && !Cfg::kSwap) {
+    // in flight.  Rows past the tile's end up to the MMA's row count are
+    // zero-filled.
+    if (Cfg::kCpGather) {
+      constexpr int RI = Cfg::ACT_ROWS / 8;  // rows per thread
       const int gt = threadIdx.x - 64;  // 0..63
       const int q = gt & 7;             // 16-byte chunk of a 128-byte row
       const int rsub = gt >> 3;         // rows rsub, rsub + 8, ...
@@ -648,16 +715,15 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       int s = 0;
       uint32_t ph = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-        const int ks = t / tiles_per_split, tl = t - ks * tiles_per_split;
+      int tl, ks, kb0, kb1;
+      for (long wi = walk_start(walk); ok && walk_next(walk, wi, tl, ks, kb0, kb1);) {
         const int rt = tl / NT;
-        const int kb0 = ks * KBS, kb1 = min(KB, kb0 + KBS);
         int g, row0, rows;
         locate_row_tile_s(p, s_tiles, rt, g, row0, rows);
         const int nload = Cfg::kSwap ? max(16, (rows + 15) & ~15) : 128;
-        const bf16* src[16];
+        const bf16* src[RI];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
+        for (int i = 0; i < RI; ++i) {
           const int r = rsub + 8 * i;
           src[i] = (r < rows) ? A + (size_t)__ldg(p.gather + row0 + r) * p.lda + q * 8 : A;
         }
@@ -665,7 +731,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
           if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, p.err)) { ok = false; break; }
           uint8_t* act = smem + s * Cfg::STAGE_BYTES;
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
+          for (int i = 0; i < RI; ++i) {
             const int r = rsub + 8 * i;
             if (r < nload)
               cp_async_16(act + r * 128 + swz, src[i] + kb * Cfg::BK, r < rows ? 16u : 0u);
@@ -690,9 +756,8 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       bool ok = true;
       int j = 0;
       uint32_t jph = 0;
-      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-        const int ks = t / tiles_per_split;
-        const int kb0 = ks * KBS, kb1 = min(KB, kb0 + KBS);
+      int tl, ks, kb0, kb1;
+      for (long wi = walk_start(walk); ok && walk_next(walk, wi, tl, ks, kb0, kb1);) {
         for (int kb = kb0; kb < kb1; ++kb) {
           // the E4M3 slot has landed and the stage's previous MMAs are done
           if (!mbar_wait(&w8full[j], jph, abort_flag, p.err)) { ok = false; break; }
@@ -723,8 +788,9 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     const int eg = (warp - 4) >> 2;   // warpgroup: even / odd 32-column chunks
     constexpr int kChunkStride = 32 * (Cfg::EPI_WARPS / 4);  // columns between a warp's chunks
     int it = 0;
-    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++it) {
-      const int ks = t / tiles_per_split, tl = t - ks * tiles_per_split;
+    uint32_t sk_ph = 0;  // stream-K: phase of epibar
+    int tl, ks, kb0, kb1;
+    for (long wi = walk_start(walk); walk_next(walk, wi, tl, ks, kb0, kb1); ++it) {
       const int rt = tl / NT, ft = tl - (tl / NT) * NT;
       const size_t slice_off = (size_t)ks * (size_t)p.epi.slice;
       int g, row0, rows;
@@ -765,23 +831,78 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         }
       } else {
         const int f = f0 + qd * 32 + lane;
+        const int fl = qd * 32 + lane;  // this thread's feature within the tile
         float s0 = 1.f, s1 = 1.f;  // fp8 weights: this thread's output channel scales
         if (Cfg::kFp8 && f < p.F) {
           const float* sc = p.w_scale + (size_t)g * p.w_group_stride + f;
           s0 = __ldg(sc);
           if (Cfg::kDual) s1 = __ldg(sc + p.dual_offset);
         }
-        for (int c0 = 32 * eg; c0 < rows; c0 += kChunkStride) {
-          tmem_ld_32x32(tb + c0, v0);
-          if (Cfg::kDual) tmem_ld_32x32(tb + Cfg::ACC_N + c0, v1);
-          tc_wait_ld();
-          if (f < p.F) {
+        // Stream-K: a tile computed in two parts (see TileWalk).  Both parts
+        // write their fp32 accumulators to their slot; the second to arrive
+        // adds the other's and finishes the tile.
+        bool finish = true;
+        const float* other = nullptr;
+        if (!Cfg::kWideSwap && walk.u_end >= 0 && (kb0 > 0 || kb1 < KB)) {
+          const int part = kb0 > 0 ? 1 : 0;  // 1: tail (this range's start), 0: head (its end)
+          const int b = part ? (int)blockIdx.x : (int)blockIdx.x + 1;  // the range boundary
+          float* mine = p.sk_part + ((size_t)b * 2 + part) * kSkSlotFloats;
+          other = p.sk_part + ((size_t)b * 2 + (part ^ 1)) * kSkSlotFloats;
+          for (int c0 = 32 * eg; c0 < rows; c0 += kChunkStride) {
+            tmem_ld_32x32(tb + c0, v0);
+            if (Cfg::kDual) tmem_ld_32x32(tb + Cfg::ACC_N + c0, v1);
+            tc_wait_ld();
             const int cn = min(32, rows - c0);
 #pragma unroll
-            for (int c = 0; c < 32; ++c)
-              if (c < cn)
-                store_elem<Cfg::kEpi, Cfg::kF16Out>(p, row0 + c0 + c, f, v0[c] * s0,
-                                                    Cfg::kDual ? v1[c] * s1 : 0.f);
+            for (int c = 0; c < 32; ++c) {
+              if (c < cn) {
+                mine[(size_t)(c0 + c) * 256 + fl] = v0[c];
+                if (Cfg::kDual) mine[(size_t)(c0 + c) * 256 + 128 + fl] = v1[c];
+              }
+            }
+          }
+          // every epilogue thread's part is written and fenced before the
+          // arrival is counted (bounded waits on an mbarrier, not bar.sync,
+          // so that an aborting block cannot strand the other warps)
+          __threadfence();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(epibar);
+          if (!mbar_wait(epibar, sk_ph, abort_flag, p.err)) break;
+          sk_ph ^= 1;
+          if (threadIdx.x == 128) {  // the first epilogue thread
+            const int old = atomicAdd(p.sk_count + b, 1);
+            if (old == 1) p.sk_count[b] = 0;  // both parts are in: reset for the next launch
+            *sk_order = old;
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(epibar);
+          if (!mbar_wait(epibar, sk_ph, abort_flag, p.err)) break;
+          sk_ph ^= 1;
+          finish = *sk_order == 1;
+          if (finish) __threadfence();
+        }
+        if (finish) {
+          for (int c0 = 32 * eg; c0 < rows; c0 += kChunkStride) {
+            tmem_ld_32x32(tb + c0, v0);
+            if (Cfg::kDual) tmem_ld_32x32(tb + Cfg::ACC_N + c0, v1);
+            tc_wait_ld();
+            const int cn = min(32, rows - c0);
+            if (other) {
+#pragma unroll
+              for (int c = 0; c < 32; ++c) {
+                if (c < cn) {
+                  v0[c] += __ldcg(other + (size_t)(c0 + c) * 256 + fl);
+                  if (Cfg::kDual) v1[c] += __ldcg(other + (size_t)(c0 + c) * 256 + 128 + fl);
+                }
+              }
+            }
+            if (f < p.F) {
+#pragma unroll
+              for (int c = 0; c < 32; ++c)
+                if (c < cn)
+                  store_elem<Cfg::kEpi, Cfg::kF16Out>(p, row0 + c0 + c, f, v0[c] * s0,
+                                                      Cfg::kDual ? v1[c] * s1 : 0.f);
+            }
           }
         }
       }
@@ -815,13 +936,19 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
 // Synchronisation: both CTAs' TMA loads complete on the leader's `full`
 // barrier (2-SM TMA); the leader's MMA commits arrive on `empty` and `tfull`
 // in both CTAs (multicast commit); both CTAs' epilogue warps arrive on the
-// leader's `tempty` (remote arrive).  Activations are always TMA tiles of
-// contiguous rows (dense GEMMs, and the expert FC2 whose input rows are
-// already in expert order).
+// leader's `tempty` (remote arrive).  Activations are TMA tiles of contiguous
+// rows (dense GEMMs, and the expert FC2 whose input rows are already in
+// expert order), or (kGather, the expert FC1 of experts with many rows) rows
+// fetched by token index with cp.async by warps 2-3 of each CTA: the
+// leader's gather completes on its own `full` barrier, the peer's on its
+// local `gfull` barrier, and the peer's warp 1 relays each completed stage to
+// the leader's `full` with a remote arrive (cp.async can only signal the
+// executing CTA's barriers).
 
-template <bool kDual_, int kEpi_>
+template <bool kDual_, int kEpi_, bool kGather_ = false>
 struct TcPairCfg {
   static constexpr bool kDual = kDual_;
+  static constexpr bool kGather = kGather_;
   static constexpr int kEpi = kEpi_;
   static constexpr int BK = 64;
   static constexpr int A_BYTES = 128 * BK * 2;   // this CTA's 128 rows
@@ -849,12 +976,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint8_t* stg_base = smem + Cfg::STAGES * Cfg::STAGE_BYTES;  // epilogue staging (1024-aligned)
   uint64_t* full = reinterpret_cast<uint64_t*>(stg_base + Cfg::STG_BYTES);
   uint64_t* empty = full + Cfg::STAGES;
-  uint64_t* tfull = empty + Cfg::STAGES;
+  uint64_t* gfull = empty + Cfg::STAGES;  // kGather, peer CTA: its own gather's completion
+  uint64_t* tfull = gfull + Cfg::STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* s_tiles = reinterpret_cast<int*>(stg_base + Cfg::STG_BYTES + 512);
+  static_assert(3 * Cfg::STAGES * 8 + 5 * 8 + 8 <= 512, "barrier area");
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   griddep_launch();
@@ -865,8 +994,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < Cfg::STAGES; ++s) {
-      mbar_init(&full[s], 1);
+      // leader: the producer's expect_tx arrive, and (kGather) its own gather
+      // threads and the peer's relay
+      mbar_init(&full[s], Cfg::kGather ? 2 + kGatherThreads : 1);
       mbar_init(&empty[s], 1);
+      mbar_init(&gfull[s], kGatherThreads);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
@@ -877,7 +1009,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     fence_barrier_init();
   }
   if (warp == 0 && lane == 0) {
-    prefetch_tensormap(&tmA);
+    if (!Cfg::kGather) prefetch_tensormap(&tmA);
     prefetch_tensormap(&tmB);
   }
   if (warp == 1) {
@@ -897,6 +1029,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // ---------------- TMA producer (both CTAs) ----------------
     if (lane == 0) {
       const uint32_t full_leader = cluster_map(&full[0], 0);
+      // bytes the leader's barrier counts per stage: both CTAs' TMA loads
+      constexpr uint32_t kTx = Cfg::kGather ? 2 * Cfg::B_BYTES : 2 * Cfg::STAGE_BYTES;
       int s = 0;
       uint32_t ph = 0;
       long armed = 0;
@@ -912,11 +1046,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           if (!mbar_wait_cluster(&empty[s], ph ^ 1, abort_flag, p.err)) { ok = false; break; }
           uint8_t* st = smem + s * Cfg::STAGE_BYTES;
           if (rank == 0) {
-            mbar_arrive_expect_tx(&full[s], 2 * Cfg::STAGE_BYTES);
+            mbar_arrive_expect_tx(&full[s], kTx);
             ++armed;
           }
           const uint32_t fb = full_leader + (uint32_t)s * 8u;
-          tma_load_2d_pair(&tmA, fb, st, kb * Cfg::BK, arow);
+          if (!Cfg::kGather) tma_load_2d_pair(&tmA, fb, st, kb * Cfg::BK, arow);
           tma_load_2d_pair(&tmB, fb, st + Cfg::A_BYTES, kb * Cfg::BK, wrow);
           if (++s == Cfg::STAGES) { s = 0; ph ^= 1; }
         }
@@ -948,6 +1082,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         bool ok = true;
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait_cluster(&full[s], ph, abort_flag, p.err)) { ok = false; break; }
+          // gathered rows were written by cp.async (generic proxy): order
+          // them before the tensor core's reads
+          if (Cfg::kGather) fence_proxy_async_smem();
           tc_fence_after();
           const uint8_t* st = smem + s * Cfg::STAGE_BYTES;
           const uint64_t da = smem_desc_sw128(st);
@@ -965,6 +1102,60 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
       tc_commit_pair_mc(drain, 0x1);
       mbar_wait_drain(drain, 0);
+    } else if (Cfg::kGather && rank == 1 && lane == 0) {
+      // ---------------- relay of the peer's gather (CTA 1) ----------------
+      const uint32_t full_leader = cluster_map(&full[0], 0);
+      int s = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      for (int t = cid; t < num_tiles && ok; t += ncl) {
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(&gfull[s], ph, abort_flag, p.err)) { ok = false; break; }
+          fence_proxy_async_smem();
+          mbar_arrive_cluster(full_leader + (uint32_t)s * 8u);
+          if (++s == Cfg::STAGES) { s = 0; ph ^= 1; }
+        }
+      }
+    }
+  } else if (warp < 4) {
+    // ---------------- cp.async row gather (kGather, both CTAs) ----------------
+    // This CTA's 128 rows of the 256-row tile, fetched by token index into
+    // the 128-byte-swizzled A stage; rows past the tile's end are zero-filled.
+    if (Cfg::kGather) {
+      const int gt = threadIdx.x - 64;  // 0..63
+      const int q = gt & 7;             // 16-byte chunk of a 128-byte row
+      const int rsub = gt >> 3;         // rows rsub, rsub + 8, ...
+      const uint32_t swz = (uint32_t)((q ^ rsub) * 16);
+      const bf16* A = static_cast<const bf16*>(p.A);
+      uint64_t* done_bar = rank == 0 ? full : gfull;
+      int s = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      for (int t = cid; t < num_tiles && ok; t += ncl) {
+        const int rt = t / NT;
+        int g, row0, rows;
+        locate_row_tile_s(p, s_tiles, rt, g, row0, rows);
+        const int base = (int)rank * 128;
+        const bf16* src[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int r = base + rsub + 8 * i;
+          src[i] = (r < rows) ? A + (size_t)__ldg(p.gather + row0 + r) * p.lda + q * 8 : A;
+        }
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait_cluster(&empty[s], ph ^ 1, abort_flag, p.err)) { ok = false; break; }
+          uint8_t* act = smem + s * Cfg::STAGE_BYTES;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int r = rsub + 8 * i;
+            cp_async_16(act + r * 128 + swz, src[i] + kb * Cfg::BK, base + r < rows ? 16u : 0u);
+          }
+          cp_async_mbar_arrive(&done_bar[s]);
+          mbar_arrive(&done_bar[s]);
+          if (++s == Cfg::STAGES) { s = 0; ph ^= 1; }
+        }
+      }
+      cp_async_wait<0>();
     }
   } else if (warp >= 4) {
     // ---------------- epilogue (warps 4..11 of both CTAs) ----------------

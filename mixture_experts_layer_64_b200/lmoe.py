@@ -26,6 +26,9 @@ ROUTE_FULL_SOFTMAX, ROUTE_BIAS_SELECT = 0x80, 0x100
 EXPERTS_FP8 = 0x200
 SINGLE_STREAM = 0x400
 NO_PDL = 0x800
+LOAD_SPLIT = 0x1000
+NO_STREAM_K = 0x2000
+SORTED_ROWS = 0x4000
 MAX_EXPERTS, MAX_TOPK = 1024, 32
 DEVERR_WAIT_TIMEOUT, DEVERR_RANGE, DEVERR_NONFINITE = 0x1, 0x2, 0x4
 STAGES = {"logits": 0, "idx": 1, "w": 2, "offsets": 3, "perm": 4, "z": 5, "h": 6, "ys": 7, "comb": 8}
@@ -81,7 +84,12 @@ def lib() -> ctypes.CDLL:
             "lmoe_status_string": ([I], ctypes.c_char_p),
             "lmoe_error_detail": ([P], ctypes.c_char_p),
             "lmoe_destroy": ([P], None),
-            "lmoe_route_only_noalloc": ([P, I, I, I, P, P, P, P, P], I),
+            "lmoe_route_only_noalloc": ([P, I, I, I, P, P, P, P, P, P], I),
+            "lmoe_ep_reserve": ([P, I], I),
+            "lmoe_ep_dispatch": ([P, P, I, P, P, P, P], I),
+            "lmoe_ep_experts": ([P, P, P, P, I, I, P, P], I),
+            "lmoe_ep_combine": ([P, P, P, P, I, P], I),
+            "lmoe_ep_local_plan": ([P, I, I, P, P], I),
         }
         for name, (args, res) in sig.items():
             f = getattr(L, name)
@@ -108,25 +116,50 @@ def _stream(stream: Optional[torch.cuda.Stream]):
     return ctypes.c_void_p(s.cuda_stream)
 
 
-def route_only_noalloc(logits: torch.Tensor, k: int, stream=None) -> Dict[str, torch.Tensor]:
+def ep_local_plan(recv_counts) -> Dict[str, "np.ndarray"]:
+    """lmoe_ep_local_plan (host only): the grouped order of the rows a rank
+    receives, from recv_counts [world, n] (host).  Returns offsets [n + 1]
+    and perm (grouped row -> received row)."""
+    import numpy as np
+    rc = np.ascontiguousarray(np.asarray(recv_counts, dtype=np.int32))
+    world, n = rc.shape
+    offsets = np.zeros(n + 1, dtype=np.int32)
+    perm = np.zeros(max(1, int(rc.sum())), dtype=np.int32)
+    st = lib().lmoe_ep_local_plan(rc.ctypes.data_as(ctypes.c_void_p), world, n,
+                                  offsets.ctypes.data_as(ctypes.c_void_p),
+                                  perm.ctypes.data_as(ctypes.c_void_p))
+    if st != OK:
+        raise LmoeError(st, "lmoe_ep_local_plan")
+    return {"offsets": offsets, "perm": perm[:int(rc.sum())]}
+
+
+def route_only_noalloc(logits: torch.Tensor, k: int, stream=None,
+                       checks: bool = False) -> Dict[str, torch.Tensor]:
     """lmoe_route_only_noalloc: the routing steps without a layer handle and
     without any device allocation inside the library (its scratch is a fixed
     device array; calls overlapping on the GPU race).  The outputs are
-    allocated here by torch, as a caller that owns its memory would."""
+    allocated here by torch, as a caller that owns its memory would.  With
+    checks=True a device error word is passed too (returned as
+    "error_word", readable once the stream has completed)."""
     if logits.dtype != torch.float32 or logits.dim() != 2 or not logits.is_cuda:
         raise ValueError("logits must be a [T, N] fp32 CUDA tensor")
     logits = logits.contiguous()
     T, N = logits.shape
     dev = logits.device
-    idx = torch.empty((T, k), dtype=torch.int32, device=dev)
-    w = torch.empty((T, k), dtype=torch.float32, device=dev)
-    offsets = torch.empty((N + 1,), dtype=torch.int32, device=dev)
-    perm = torch.empty((T * k,), dtype=torch.int32, device=dev)
-    st = lib().lmoe_route_only_noalloc(_ptr(logits), T, N, k, _ptr(idx), _ptr(w), _ptr(offsets),
-                                       _ptr(perm), _stream(stream))
+    with torch.cuda.device(dev):
+        idx = torch.empty((T, k), dtype=torch.int32, device=dev)
+        w = torch.empty((T, k), dtype=torch.float32, device=dev)
+        offsets = torch.empty((N + 1,), dtype=torch.int32, device=dev)
+        perm = torch.empty((T * k,), dtype=torch.int32, device=dev)
+        word = torch.empty((1,), dtype=torch.int32, device=dev) if checks else None
+        st = lib().lmoe_route_only_noalloc(_ptr(logits), T, N, k, _ptr(idx), _ptr(w),
+                                           _ptr(offsets), _ptr(perm), _ptr(word), _stream(stream))
     if st != OK:
         raise LmoeError(st, "lmoe_route_only_noalloc")
-    return {"idx": idx, "w": w, "offsets": offsets, "perm": perm}
+    res = {"idx": idx, "w": w, "offsets": offsets, "perm": perm}
+    if checks:
+        res["error_word"] = word
+    return res
 
 
 class LatentMoELayer:
@@ -319,6 +352,54 @@ class LatentMoELayer:
         names = [stage_name(i) for i in range(ns.value)]
         return [{names[s]: buf[f * ns.value + s] for s in range(ns.value)
                  if buf[f * ns.value + s] >= 0} for f in range(nf.value)]
+
+    # -- expert parallelism (dispatch / experts / combine in latent space) ----
+    def ep_reserve(self, max_recv_rows: int):
+        self._check(lib().lmoe_ep_reserve(self._h, max_recv_rows), "lmoe_ep_reserve")
+
+    def ep_dispatch(self, x: torch.Tensor, stream=None):
+        """Step 1: (send_rows [T*k, l], send_gates [T*k], expert_counts [N]) on
+        the device, rows sorted by expert then token."""
+        T = x.shape[0]
+        x = self._dev(x, (T, self.d), name="x")
+        cols = self.d if self.flags & SKIP_PROJ else self.l
+        rows = torch.empty((T * self.k, cols), dtype=self.torch_dtype, device=self.device)
+        gates = torch.empty((T * self.k,), dtype=torch.float32, device=self.device)
+        counts = torch.empty((self.N,), dtype=torch.int32, device=self.device)
+        self._check(lib().lmoe_ep_dispatch(self._h, _ptr(x), T, _ptr(rows), _ptr(gates),
+                                           _ptr(counts), _stream(stream)), "lmoe_ep_dispatch")
+        return rows, gates, counts
+
+    def ep_experts(self, recv_rows: torch.Tensor, recv_gates: torch.Tensor, recv_counts,
+                   rank: int, world: int, stream=None) -> torch.Tensor:
+        """Step 3: the local experts on the received rows; recv_counts is a
+        host array-like [world, N / world].  Returns out_rows (received order)."""
+        rc = torch.as_tensor(recv_counts, dtype=torch.int32).reshape(world, self.N // world)
+        rc = rc.contiguous()
+        Rr = int(rc.sum())
+        cols = self.d if self.flags & SKIP_PROJ else self.l
+        out = torch.empty((Rr, cols), dtype=self.torch_dtype, device=self.device)
+        if Rr:
+            recv_rows = self._dev(recv_rows, (Rr, cols), name="recv_rows")
+            recv_gates = self._dev(recv_gates, (Rr,), torch.float32, "recv_gates")
+        self._check(lib().lmoe_ep_experts(self._h, _ptr(recv_rows) if Rr else None,
+                                          _ptr(recv_gates) if Rr else None,
+                                          ctypes.c_void_p(rc.data_ptr()), rank, world,
+                                          _ptr(out) if Rr else None, _stream(stream)),
+                    "lmoe_ep_experts")
+        return out
+
+    def ep_combine(self, x: torch.Tensor, back_rows: torch.Tensor, out=None, stream=None):
+        """Step 5: out = x + the layer, from the returned rows (send order)."""
+        T = x.shape[0]
+        x = self._dev(x, (T, self.d), name="x")
+        cols = self.d if self.flags & SKIP_PROJ else self.l
+        back_rows = self._dev(back_rows, (T * self.k, cols), name="back_rows")
+        if out is None:
+            out = torch.empty_like(x)
+        self._check(lib().lmoe_ep_combine(self._h, _ptr(x), _ptr(back_rows), _ptr(out), T,
+                                          _stream(stream)), "lmoe_ep_combine")
+        return out
 
     @property
     def last_launch_count(self) -> int:

@@ -159,15 +159,17 @@ def paths(res):
 
 @pytest.mark.parametrize("name", ["swiglu", "relu2-shared", "skip"])
 @pytest.mark.parametrize("flags", [0, lmoe.FORCE_SWAP, lmoe.FORCE_NOSWAP, lmoe.FORCE_WS_PAIR,
-                                   lmoe.FORCE_NOPAIR, lmoe.FORCE_SIMT])
+                                   lmoe.FORCE_NOPAIR, lmoe.FORCE_SIMT, lmoe.LOAD_SPLIT])
 def test_small_layer_each_expert_kernel(name, flags):
     """Every expert kernel on the same layers (FC1, FC2): token-tiled with FC2
-    on CTA pairs (1, 3, the default at these row counts), weight-stationary on
-    single CTAs (2, 2), weight-stationary on CTA pairs (4, 4), token-tiled on
-    single CTAs (1, 1), CUDA cores (0, 0)."""
+    on CTA pairs (1, 3, the default at these row counts), weight-stationary
+    on single CTAs (2, 2), weight-stationary on CTA pairs (4, 4), token-tiled
+    on single CTAs (1, 1), CUDA cores (0, 0), and split by load (5, 5: CTA
+    pairs with FC1's rows gathered in both CTAs for the experts above 384
+    rows, weight-stationary tiles of up to 128 / 256 rows for the rest)."""
     res = check_forward(SMALL[name], flags=flags, fixture=True)
     want = {0: (1, 3), lmoe.FORCE_SWAP: (2, 2), lmoe.FORCE_NOSWAP: (1, 3), lmoe.FORCE_WS_PAIR: (4, 4),
-            lmoe.FORCE_NOPAIR: (1, 1), lmoe.FORCE_SIMT: (0, 0)}[flags]
+            lmoe.FORCE_NOPAIR: (1, 1), lmoe.FORCE_SIMT: (0, 0), lmoe.LOAD_SPLIT: (5, 5)}[flags]
     assert paths(res) == want
 
 
@@ -194,6 +196,69 @@ def test_weight_stationary_pairs_on_skewed_loads(act):
     assert loads[-1] == 0 and loads.max() > 256 and ((loads > 128) & (loads < 256)).any()
 
 
+@pytest.mark.parametrize("name", ["swiglu", "relu2-shared", "skip"])
+@pytest.mark.parametrize("flags", [lmoe.SORTED_ROWS, lmoe.SORTED_ROWS | lmoe.LOAD_SPLIT,
+                                   lmoe.SORTED_ROWS | lmoe.FORCE_SWAP,
+                                   lmoe.SORTED_ROWS | lmoe.FORCE_WS_PAIR])
+def test_sorted_fc1_rows_each_expert_kernel(name, flags):
+    """LMOE_SORTED_ROWS: the FC1 input rows copied into expert order, FC1 on
+    the TMA-fed variants of every expert kernel."""
+    res = check_forward(SMALL[name], flags=flags, fixture=True)
+    want = {lmoe.SORTED_ROWS: (1, 3), lmoe.SORTED_ROWS | lmoe.LOAD_SPLIT: (5, 5),
+            lmoe.SORTED_ROWS | lmoe.FORCE_SWAP: (2, 2),
+            lmoe.SORTED_ROWS | lmoe.FORCE_WS_PAIR: (4, 4)}[flags]
+    assert paths(res) == want
+
+
+@pytest.mark.parametrize("act", ["swiglu", "relu2"])
+@pytest.mark.parametrize("sorted_rows", [False, True])
+def test_load_split_on_skewed_loads(act, sorted_rows):
+    """The token-tiled expert GEMMs split by load (LMOE_LOAD_SPLIT) on loads
+    from ~T/2 rows down to none: experts above 384 rows on CTA pairs (several 256-row tiles, a ragged
+    last tile, FC1 rows gathered by token in both CTAs), the others on
+    weight-stationary tiles of their rows (several tiles past 128 / 256
+    rows); an expert with no rows in either kernel."""
+    w = W_("split-skew", T=1100, d=256, l=192, N=16, k=4, m=320, act=act, shared_m=0, seed=24)
+    W = workloads.make_weights(w, device="cuda")
+    b = torch.linspace(3.0, -3.0, w.N, device="cuda")
+    b[-1] = -40.0  # never chosen
+    W["bias"] = b
+    L, _ = gpu_layer(w, lmoe.LOAD_SPLIT | (lmoe.SORTED_ROWS if sorted_rows else 0), W)
+    x = workloads.make_x(w, device="cuda")
+    res = check_forward(w, W=W, layer=L, x=x, fixture=True, tokens=sample_tokens(w.T, 300, seed=3))
+    assert paths(res) == (5, 5)
+    loads = np.diff(L.debug_dump("offsets", w.T).cpu().numpy())
+    print("loads", loads.tolist())
+    assert loads[-1] == 0 and loads.max() > 512
+    assert ((loads > 0) & (loads <= 128)).any() and ((loads > 128) & (loads <= 384)).any()
+
+
+@pytest.mark.parametrize("act", ["swiglu", "relu2"])
+def test_stream_k_decode_tiles(act):
+    """Weight-stationary decode GEMMs with more than two tiles per CTA take
+    the stream-K split (tiles straddling two CTAs' ranges summed from two
+    fp32 parts): parity with the oracle, bitwise the same over repeated
+    forwards, and within the tolerance of the whole-tile path
+    (LMOE_NO_STREAM_K)."""
+    w = W_("streamk", T=256, d=256, l=512, N=80, k=4, m=512, act=act, seed=25)
+    W = workloads.make_weights(w, device="cuda")
+    L, _ = gpu_layer(w, 0, W)
+    x = workloads.make_x(w, device="cuda")
+    res = check_forward(w, W=W, layer=L, x=x, fixture=True)
+    assert paths(res) == (2, 2)
+    a = L.forward(x).clone()
+    b = L.forward(x).clone()
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+    L2, _ = gpu_layer(w, lmoe.NO_STREAM_K, W)
+    res2 = check_forward(w, W=W, layer=L2, x=x, fixture=True)
+    assert paths(res2) == (2, 2)
+    c = L2.forward(x)
+    torch.cuda.synchronize()
+    assert (a.float() - c.float()).abs().max().item() <= 2e-2
+    assert L.last_error() == (lmoe.OK, 0) and L2.last_error() == (lmoe.OK, 0)
+
+
 def test_pair_kernels_on_dense_prefill_shapes():
     """T >= 1024 puts the dense GEMMs (router, down-projection, shared FC1,
     up-projection) on CTA pairs as well as the expert GEMMs; ragged last row
@@ -202,6 +267,9 @@ def test_pair_kernels_on_dense_prefill_shapes():
            seed=22)
     res = check_forward(w, fixture=True, tokens=sample_tokens(w.T, 200, seed=1))
     assert paths(res) == (1, 3)
+    res = check_forward(w, flags=lmoe.LOAD_SPLIT, fixture=True,
+                        tokens=sample_tokens(w.T, 200, seed=1))
+    assert paths(res) == (5, 5)
     res = check_forward(w, flags=lmoe.FORCE_WS_PAIR, fixture=True,
                         tokens=sample_tokens(w.T, 200, seed=1))
     assert paths(res) == (4, 4)
@@ -422,7 +490,7 @@ def test_fp8_expert_api_errors():
 
 def test_tcgen05_path_is_taken_for_bf16():
     res = check_forward(SMALL["swiglu"], fixture=True)
-    assert paths(res)[0] in (1, 2, 4)
+    assert paths(res)[0] in (1, 2, 4, 5)
     res = check_forward(SMALL["odd-K"], fixture=True)
     assert res["expert_path"] == 0
 
@@ -490,6 +558,36 @@ def test_bounded_wait_gives_up_and_reports():
         L.selftest_wait_timeout(0)
 
 
+def test_debug_checks_flag_non_finite_logits():
+    """LMOE_DEBUG_CHECKS: a NaN or an infinite router logit fed to
+    lmoe_route_only sets LMOE_DEVERR_NONFINITE in the device error word
+    (status DEVICE), with every index still in range; the word is cleared by
+    reading it, and finite logits leave it at 0.  Without the flag the same
+    logits set nothing."""
+    T, N, k = 96, 128, 8
+    lg = workloads.make_logits(T, N, seed=31, ties=False)
+    bad = lg.clone()
+    bad[3, 7] = float("nan")
+    bad[50, 0] = float("inf")
+    L = lmoe.LatentMoELayer(64, 64, N, k, 64, act="silu", dtype="bf16", flags=lmoe.DEBUG_CHECKS)
+    L.reserve(T)
+    L.route_only(lg.cuda())
+    assert L.last_error() == (lmoe.OK, 0)
+    r = L.route_only(bad.cuda())
+    assert L.last_error() == (lmoe.ERR_DEVICE, lmoe.DEVERR_NONFINITE)
+    idx = r["idx"].cpu().numpy()
+    assert idx.min() >= 0 and idx.max() < N
+    assert L.last_error() == (lmoe.OK, 0)
+    r = L.route_only(lg.cuda())  # finite again: the routing is the oracle's
+    o_idx = oracle.route(lg.numpy(), k)[0]
+    np.testing.assert_array_equal(r["idx"].cpu().numpy(), o_idx)
+    assert L.last_error() == (lmoe.OK, 0)
+    L2 = lmoe.LatentMoELayer(64, 64, N, k, 64, act="silu", dtype="bf16")
+    L2.reserve(T)
+    L2.route_only(bad.cuda())
+    assert L2.last_error() == (lmoe.OK, 0)
+
+
 def test_uniform_router_is_mean_of_experts():
     """W_g = 0, k = N: every token uses every expert with weight 1/N."""
     w = W_("uniform", T=64, d=128, l=64, N=4, k=4, m=64, act="relu2", seed=19)
@@ -509,6 +607,8 @@ def test_device_error_word_clean_and_profile():
     prof = L.profile_end()
     assert len(prof) == 3 and all(v >= 0 for p in prof for v in p.values())
     assert L.last_error() == (lmoe.OK, 0)
+    # router, top-k, grouping count and rank, down-projection, expert FC1,
+    # expert FC2, combine, up-projection
     assert L.last_launch_count >= 8
 
 
@@ -521,13 +621,31 @@ FULL_SAMPLES = {"tiny-fp32": 64, "std-moe-decode": 96, "latent-decode": 96,
                 "std-moe-decode-fp8": 96, "latent-decode-fp8": 96}
 
 
+def edge_tokens_of_largest_experts(L, T: int, n_experts: int = 2, per_end: int = 3):
+    """Tokens in the first and last row tiles of the most loaded experts (rows
+    within an expert are in ascending token order): the lowest and highest
+    token indices routed to each of them."""
+    idx = L.debug_dump("idx", T).cpu().numpy()
+    loads = np.bincount(idx.ravel(), minlength=L.N)
+    out = []
+    for e in np.argsort(-loads, kind="stable")[:n_experts]:
+        toks = np.nonzero((idx == e).any(axis=1))[0]
+        out += toks[:per_end].tolist() + toks[-per_end:].tolist()
+    return out
+
+
 @pytest.mark.parametrize("name", workloads.WORKLOAD_ORDER)
 def test_workload_full_size(name):
     w = workloads.WORKLOADS[name]
     toks = sample_tokens(w.T, FULL_SAMPLES[name], seed=w.seed)
-    res = check_forward(w, tokens=toks)
+    L, W = gpu_layer(w)
+    x = workloads.make_x(w, device="cuda")
+    L.forward(x)
+    torch.cuda.synchronize()
+    toks = np.unique(np.concatenate([toks, edge_tokens_of_largest_experts(L, w.T)])).astype(np.int32)
+    res = check_forward(w, tokens=toks, layer=L, W=W, x=x)
     print(name, res)
     assert res["unique"] >= 0.8 * res["tokens"]
     if w.dtype == "bf16":
-        assert paths(res)[0] in (1, 2, 4)
+        assert paths(res)[0] in (1, 2, 4, 5)
     torch.cuda.empty_cache()

@@ -23,8 +23,9 @@ def test_binding_flags_and_limits_match_the_header():
     flags = {k: v for k, v in defs.items()
              if k in ("SKIP_PROJ", "DEBUG_CHECKS", "FORCE_SIMT", "FORCE_SWAP", "FORCE_NOSWAP",
                       "FORCE_NOPAIR", "FORCE_WS_PAIR", "ROUTE_FULL_SOFTMAX", "ROUTE_BIAS_SELECT",
-                      "EXPERTS_FP8", "SINGLE_STREAM", "NO_PDL")}
-    assert len(flags) == 12, sorted(flags)
+                      "EXPERTS_FP8", "SINGLE_STREAM", "NO_PDL", "LOAD_SPLIT",
+                      "NO_STREAM_K", "SORTED_ROWS")}
+    assert len(flags) == 15, sorted(flags)
     for name, value in flags.items():
         assert getattr(lmoe, name) == value, name
     # flags are distinct single bits

@@ -3,31 +3,39 @@ allocate device memory (an inference server that owns all of HBM through its
 own pool, or code where cudaMalloc's implicit synchronisation is not allowed).
 
 It must give what lmoe_route_only gives (bit-exact indices, offsets and
-permutation; gates within the routing tolerance), call after call, with its
-scratch in the library's fixed device array: a second call must see no stale
-state from the first, and must not change the device's free memory.  The
-file is named to be collected last."""
+permutation; gates within the routing tolerance), and what the CPU oracle's
+routing gives, call after call, with its scratch in the library's fixed
+device array: a second call must see no stale state from the first, and must
+not change the device's free memory.  With an error word it runs the device
+checks and reports a non-finite logit there.  The file is named to be
+collected last."""
 import ctypes
 
 import numpy as np
 import pytest
 import torch
 
+import oracle
 from mixture_experts_layer_64_b200 import lmoe, workloads
 
 pytestmark = pytest.mark.gpu
 
 
-def _noalloc_via_cabi(logits: torch.Tensor, k: int):
+def _outputs(T: int, N: int, k: int, dev):
+    return {"idx": torch.full((T, k), -1, dtype=torch.int32, device=dev),
+            "w": torch.full((T, k), -1.0, dtype=torch.float32, device=dev),
+            "offsets": torch.full((N + 1,), -1, dtype=torch.int32, device=dev),
+            "perm": torch.full((T * k,), -1, dtype=torch.int32, device=dev)}
+
+
+def _noalloc_via_cabi(logits: torch.Tensor, k: int, out=None, word=None):
+    """Calls the entry point through the C ABI on caller-owned outputs."""
     T, N = logits.shape
-    dev = logits.device
-    out = {"idx": torch.full((T, k), -1, dtype=torch.int32, device=dev),
-           "w": torch.full((T, k), -1.0, dtype=torch.float32, device=dev),
-           "offsets": torch.full((N + 1,), -1, dtype=torch.int32, device=dev),
-           "perm": torch.full((T * k,), -1, dtype=torch.int32, device=dev)}
-    p = lambda t: ctypes.c_void_p(t.data_ptr())
+    if out is None:
+        out = _outputs(T, N, k, logits.device)
+    p = lambda t: ctypes.c_void_p(None if t is None else t.data_ptr())
     st = lmoe.lib().lmoe_route_only_noalloc(p(logits), T, N, k, p(out["idx"]), p(out["w"]),
-                                            p(out["offsets"]), p(out["perm"]),
+                                            p(out["offsets"]), p(out["perm"]), p(word),
                                             ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
     return st, out
 
@@ -61,19 +69,58 @@ def test_noalloc_matches_route_only_on_two_calls_in_a_row():
         refs.append((lg, k, r))
     torch.cuda.synchronize()
     for i, (lg, k, ref) in enumerate(refs):
+        out = _outputs(lg.shape[0], lg.shape[1], k, lg.device)  # the caller's memory, first
+        torch.cuda.synchronize()
         free_before = torch.cuda.mem_get_info()[0]
-        st, got = _noalloc_via_cabi(lg, k)
+        st, got = _noalloc_via_cabi(lg, k, out)
+        free_after = torch.cuda.mem_get_info()[0]
         torch.cuda.synchronize()
         assert st == lmoe.OK, lmoe.status_string(st)
         _same(got, ref)
         if i > 0:  # set-up (symbol lookup, module load) happened on the first call
-            assert torch.cuda.mem_get_info()[0] == free_before
+            assert free_after == free_before
     # and once more with the first problem again, after the second
     lg, k, ref = refs[0]
     st, got = _noalloc_via_cabi(lg, k)
     torch.cuda.synchronize()
     assert st == lmoe.OK
     _same(got, ref)
+
+
+def test_noalloc_matches_the_oracle_routing():
+    torch.cuda.set_device(0)
+    T, N, k = 257, 512, 22
+    lg = workloads.make_logits(T, N, seed=5, ties=True)
+    st, got = _noalloc_via_cabi(lg.cuda(), k)
+    torch.cuda.synchronize()
+    assert st == lmoe.OK
+    o_idx, o_w, o_off, o_perm = oracle.route(lg.numpy(), k)
+    np.testing.assert_array_equal(got["idx"].cpu().numpy(), o_idx)
+    np.testing.assert_array_equal(got["offsets"].cpu().numpy(), o_off)
+    np.testing.assert_array_equal(got["perm"].cpu().numpy(), o_perm)
+    np.testing.assert_allclose(got["w"].cpu().numpy(), o_w, rtol=2e-6, atol=1e-7)
+
+
+def test_noalloc_error_word_reports_a_non_finite_logit():
+    torch.cuda.set_device(0)
+    T, N, k = 64, 128, 8
+    lg = workloads.make_logits(T, N, seed=9, ties=False).cuda()
+    word = torch.full((1,), -1, dtype=torch.int32, device="cuda")
+    st, got = _noalloc_via_cabi(lg, k, word=word)
+    torch.cuda.synchronize()
+    assert st == lmoe.OK and int(word.item()) == 0  # cleared by the call, nothing flagged
+    bad = lg.clone()
+    bad[5, 17] = float("nan")
+    st, got = _noalloc_via_cabi(bad, k, word=word)
+    torch.cuda.synchronize()
+    assert st == lmoe.OK
+    assert int(word.item()) & lmoe.DEVERR_NONFINITE
+    idx = got["idx"].cpu().numpy()
+    assert idx.min() >= 0 and idx.max() < N  # indices stay in range
+    # the next clean call clears the word again
+    st, _ = _noalloc_via_cabi(lg, k, word=word)
+    torch.cuda.synchronize()
+    assert st == lmoe.OK and int(word.item()) == 0
 
 
 def test_noalloc_rejects_sizes_beyond_its_scratch():
