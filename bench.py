@@ -15,10 +15,11 @@ torch.cuda.synchronize(), and the time is the max over ranks.
 
 Prints one JSON line (rank 0).  With the default workload (decode, the
 headline) the line also carries "prefill": the two prefill workloads
-(latent-prefill-skewed, latent-prefill-shared) measured in the same run with
-the same steps and warm-up, each with its own clocks, roofline, expert-load
-summary, per-stage p50/p95/p99 and projection share (--no-prefill skips
-them).  --impl reference times the CPU oracle (the reference arm of this
+(latent-prefill-skewed, latent-prefill-shared), and "decode_variants": the
+latent decode workload and both decode workloads with fp8 expert weights,
+measured in the same run with the same steps and warm-up, each with its own
+clocks, roofline, expert-load summary, per-stage p50/p95/p99 and projection
+share (--no-prefill skips them).  --impl reference times the CPU oracle (the reference arm of this
 method: a plain float64 C++ implementation) on a bounded token sample of the
 same workload.
 """
@@ -315,6 +316,8 @@ def run_reference(args):
 
 
 PREFILL_WORKLOADS = ("latent-prefill-skewed", "latent-prefill-shared")
+# the other decode workloads, measured beside the headline in the same run
+DECODE_WORKLOADS = ("latent-decode", "std-moe-decode-fp8", "latent-decode-fp8")
 NOMINAL_HBM_GBS = 8000.0  # the ~8 TB/s HBM figure the decode target is quoted against
 PROJECTION_SHARE_PAGES = 0.09  # the paper's ~9% latent-projection overhead (Section 4.3)
 
@@ -498,7 +501,10 @@ def sub_record(r):
     return {"workload": r["workload"], "value": r["value"], "unit": UNIT,
             "ms_per_step": r["ms_per_step"], "config": {"T": w.T, "d": w.d, "l": w.l, "N": w.N,
                                                         "k": w.k, "m": w.m, "act": w.act,
-                                                        "shared_m": w.shared_m, "bias": w.bias},
+                                                        "shared_m": w.shared_m, "bias": w.bias,
+                                                        "skip_proj": w.skip_proj,
+                                                        "expert_weights": "e4m3" if w.expert_fp8
+                                                        else w.dtype},
             "e2e": r["e2e"], "gpu_launches": r["gpu_launches"], "clocks": r["clocks"],
             "roofline": r["roofline"], "layer": r["layer"], "expert_loads": r["expert_loads"],
             "projection_share": r["projection_share"], "stage_ms": r["stage_ms"],
@@ -538,15 +544,17 @@ def run_ours(args):
     del W, x
     torch.cuda.empty_cache()
 
-    # ---- the prefill workloads, measured in the same run with the same steps
-    prefill = []
+    # ---- the prefill workloads (and the other decode workloads), measured in
+    # the same run with the same steps
+    extra = {"prefill": [], "decode_variants": []}
     if not args.no_prefill and args.workload == DEFAULT_WORKLOAD:
-        for name in PREFILL_WORKLOADS:
-            r = measure(args, name, pg, rank, ws, local, dev, flags=args.lib_flags)
-            del r["W"], r["x"]
-            prefill.append(sub_record(r))
-            del r
-            torch.cuda.empty_cache()
+        for key, names in (("prefill", PREFILL_WORKLOADS), ("decode_variants", DECODE_WORKLOADS)):
+            for name in names:
+                r = measure(args, name, pg, rank, ws, local, dev, flags=args.lib_flags)
+                del r["W"], r["x"]
+                extra[key].append(sub_record(r))
+                del r
+                torch.cuda.empty_cache()
 
     if rank == 0:
         roofline = main["roofline"]
@@ -563,8 +571,9 @@ def run_ours(args):
                 "stage_ms": main["stage_ms"], "stage_ms_source": main["stage_ms_source"],
                 "projection_share": main["projection_share"],
                 "expert_loads": main["expert_loads"]}
-        if prefill:
-            line["prefill"] = prefill
+        for key, recs in extra.items():
+            if recs:
+                line[key] = recs
         print(json.dumps(line), flush=True)
     if pg:
         pg.barrier()
@@ -582,7 +591,8 @@ def main():
 
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true",
-                    help="skip the prefill workloads measured beside the default decode line")
+                    help="skip the prefill and other decode workloads measured beside the "
+                         "default decode line")
     ap.add_argument("--experts", type=int, default=None,
                     help="override N (reduced cases for profiler captures)")
     ap.add_argument("--topk", type=int, default=None, help="override k")

@@ -133,16 +133,15 @@ typedef enum { LMOE_F32 = 0, LMOE_BF16 = 1 } lmoe_dtype;
                                     sums inside the tensor cores. */
 #define LMOE_NO_STREAM_K        0x2000u /* decode (weight-stationary) expert
                                     FC1 in whole tiles per CTA.  By
-                                    default, with at least two tiles per
-                                    CTA, the (tile, K block) units are dealt
-                                    out in equal ranges, one per CTA, so the
-                                    weight stream ends on every SM at the
-                                    same time; a tile that straddles two
-                                    ranges is summed from its two fp32 parts
-                                    (in a fixed way: the result does not
-                                    depend on timing).  Needs 2 x (SMs + 1)
-                                    x 64 KB of workspace. */
-
+                                    default, with 2 to 16 tiles per CTA, the
+                                    (tile, K block) units are dealt out in
+                                    equal ranges, one per CTA, so the weight
+                                    stream ends on every SM at the same
+                                    time; a tile that straddles two ranges
+                                    is summed from its two fp32 parts (in a
+                                    fixed way: the result does not depend on
+                                    timing).  Needs 2 x (SMs + 1) x 64 KB of
+                                    workspace. */
 #define LMOE_SORTED_ROWS        0x4000u /* copy the expert FC1's input rows
                                     into expert order (T*k rows of the
                                     latent width, a workspace of that size)

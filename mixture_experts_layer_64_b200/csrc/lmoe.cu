@@ -256,8 +256,11 @@ bool encode_map(CUtensorMap* map, const void* ptr, long rows, int cols, long ld,
 }
 
 // fp8 E4M3 weights: rows of `cols` one-byte codes, 64-code (64-byte) boxes of
-// box_rows rows, no swizzle (the converter warps re-lay them out as bf16).
-bool encode_map_u8(CUtensorMap* map, const void* ptr, long rows, int cols, long ld, int box_rows) {
+// box_rows rows, no swizzle (the converter warps re-lay them out as f16 in
+// shared memory), or the 64-byte swizzle (sw64: the converters of the
+// weight-stationary kernels read one row per thread into tensor memory).
+bool encode_map_u8(CUtensorMap* map, const void* ptr, long rows, int cols, long ld, int box_rows,
+                   bool sw64) {
   EncodeTiledFn fn = get_encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
@@ -265,7 +268,8 @@ bool encode_map_u8(CUtensorMap* map, const void* ptr, long rows, int cols, long 
   cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            sw64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_NONE,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -317,7 +321,7 @@ lmoe_status launch_tc(lmoe_layer* h, const GemmCall& c, cudaStream_t st) {
     h->detail = "cuTensorMapEncodeTiled (activations) failed";
     return LMOE_ERR_CUDA;
   }
-  if (!(Cfg::kFp8 ? encode_map_u8(&tb, c.p.B, c.b_rows, c.p.K, c.p.K, Cfg::W_ROWS)
+  if (!(Cfg::kFp8 ? encode_map_u8(&tb, c.p.B, c.b_rows, c.p.K, c.p.K, Cfg::W_ROWS, Cfg::kTmemA)
                   : encode_map(&tb, c.p.B, c.b_rows, c.p.K, c.p.K, Cfg::W_ROWS))) {
     h->detail = "cuTensorMapEncodeTiled (weights) failed";
     return LMOE_ERR_CUDA;
@@ -505,26 +509,6 @@ int choose_splits(const lmoe_layer* h, const GemmCall& c, int& kbs) {
   return (KB + kbs - 1) / kbs;  // every range non-empty
 }
 
-// First half of a split-K call: the S fp32 slices of partial sums in the
-// call's partial buffer (slice = M * Fp floats apart).
-lmoe_status run_split_partials(lmoe_layer* h, const GemmCall& c, int S, int kbs,
-                               cudaStream_t st) {
-  const bool dual = c.p.dual_offset > 0;
-  const int Fp = dual ? 2 * c.p.F : c.p.F;
-  GemmCall g = c;
-  g.kind = GK_ROUTER;  // fp32 output, no bias: the partial sums
-  g.p.F = Fp;
-  g.p.dual_offset = 0;
-  std::memset(&g.p.epi, 0, sizeof g.p.epi);
-  g.p.epi.out = part_buffer(h, c);
-  g.p.epi.ldo = Fp;
-  g.p.epi.slice = (long)c.p.M * Fp;
-  g.p.splits = S;
-  g.p.kb_per_split = kbs;
-  g.out_rows = (long)S * c.p.M;  // the slices stacked: rows of the output map
-  return launch_tc<TcCfg<false, false, false, 128, EPI_F32_BIAS>>(h, g, st);
-}
-
 lmoe_status run_split(lmoe_layer* h, const GemmCall& c, int S, int kbs, cudaStream_t st) {
   const bool dual = c.p.dual_offset > 0;
   const int Fp = dual ? 2 * c.p.F : c.p.F;
@@ -558,10 +542,9 @@ lmoe_status run_gemm(lmoe_layer* h, GemmCall c, cudaStream_t st, int* path = nul
       g.p.row_tile = kSwapRowTile;
       g.p.tile_prefix = g.grp->tp64;
       g.p.max_row_tiles = (int)(g.out_rows / kSwapRowTile + g.grp->G);  // routed rows
-      // the expert FC1 (the longer weight stream, with the fewer tiles per
-      // CTA): stream-K over (tile, K block) units once there are two tiles
-      // per CTA (decided in the kernel from the tile count).  For FC2, whose
-      // tiles are short and many, the whole-tile split measured faster.
+      // the expert FC1 (the longer weight stream): stream-K over (tile, K
+      // block) units when there are 2 to 16 tiles per CTA (decided in the
+      // kernel from the tile count).  On FC2 it measured slower.
       g.p.stream_k = (h->sk_part && g.kind == GK_FC1) ? 1 : 0;
       g.p.sk_part = h->sk_part;
       g.p.sk_count = h->sk_count;
@@ -792,18 +775,10 @@ void prof_mark(lmoe_layer* h, cudaStream_t st, int i) {
 
 // ---- the routing steps ---------------------------------------------------------
 
-// Whether the routing runs with the default variant (renormalised gates over
-// logits that include the bias).
-bool default_routing(const lmoe_layer* h) {
-  return !(h->flags & (LMOE_ROUTE_BIAS_SELECT | LMOE_ROUTE_FULL_SOFTMAX));
-}
-
-// Top-k and grouping.  part_S > 0: the logits are still the router's S
-// split-K partial slices in h->part, summed (with the bias) by the top-k
-// kernel, which writes them to `logits`.
+// Top-k and grouping.
 lmoe_status run_routing(lmoe_layer* h, const float* logits, int T, int* idx, float* w,
                         int* offsets, int* row_tok, int* row_slot, float* row_w, int* slot_row,
-                        int* tile_prefix2, cudaStream_t st, bool marks, int part_S = 0) {
+                        int* tile_prefix2, cudaStream_t st, bool marks) {
   const int W = (T + 31) / 32;
   const int debug = (h->flags & LMOE_DEBUG_CHECKS) ? 1 : 0;
   {
@@ -821,14 +796,6 @@ lmoe_status run_routing(lmoe_layer* h, const float* logits, int T, int* idx, flo
     a.W = W;
     a.debug = debug;
     a.err = h->err;
-    if (part_S > 0) {
-      a.logits = nullptr;
-      a.part = h->part;
-      a.S = part_S;
-      a.slice = (long)T * h->N;
-      a.pbias = h->bias;
-      a.logits_out = const_cast<float*>(logits);
-    }
     const cudaError_t e = launch_topk_args(a, st, take_pdl(h));
     if (e != cudaSuccess) return cuda_fail(h, e, "top-k launch");
     ++h->launches;
@@ -847,30 +814,13 @@ lmoe_status run_routing(lmoe_layer* h, const float* logits, int T, int* idx, flo
   return LMOE_OK;
 }
 
-// The router GEMM.  With part_S (the forward, default routing) a call that
-// splits K leaves its partial slices in h->part for the top-k kernel to sum:
-// *part_S = the number of slices, else 0 and the logits are written.
-lmoe_status run_router(lmoe_layer* h, const void* x, float* logits, int T, cudaStream_t st,
-                       int* part_S = nullptr) {
+lmoe_status run_router(lmoe_layer* h, const void* x, float* logits, int T, cudaStream_t st) {
   GemmCall c = dense_call(GK_ROUTER, T, x, h->d, h->Wg_t, h->N, h->d);
   c.p.epi.out = logits;
   c.p.epi.ldo = h->N;
   c.p.epi.bias = (h->flags & LMOE_ROUTE_BIAS_SELECT) ? nullptr : h->bias;
   if (h->dtype == LMOE_BF16 && T >= 1024 && !(h->flags & (LMOE_FORCE_SIMT | LMOE_FORCE_NOPAIR)))
     make_pair(h, c);
-  if (part_S) {
-    *part_S = 0;
-    c.p.err = h->err;
-    int kbs = 0;
-    if (!c.pair && default_routing(h) && tc_eligible(h, c)) {
-      const int S = choose_splits(h, c, kbs);
-      if (S > 1) {
-        LMOE_TRY(run_split_partials(h, c, S, kbs, st));
-        *part_S = S;
-        return LMOE_OK;
-      }
-    }
-  }
   return run_gemm(h, c, st);
 }
 
@@ -950,11 +900,10 @@ lmoe_status run_front(lmoe_layer* h, const void* x, int T, cudaStream_t st) {
                           kSideMark0 + 2));
   }
   h->pdl_hold = true;
-  int part_S = 0;
-  LMOE_TRY(run_router(h, x, h->logits, T, st, &part_S));
+  LMOE_TRY(run_router(h, x, h->logits, T, st));
   prof_mark(h, st, 1);
   LMOE_TRY(run_routing(h, h->logits, T, h->idx, h->w, h->offsets, h->row_tok, h->row_slot,
-                       h->row_w, h->slot_row, h->tile_prefix2, st, true, part_S));
+                       h->row_w, h->slot_row, h->tile_prefix2, st, true));
   prof_mark(h, st, 3);
   if (side) {
     LMOE_CUDA(h, cudaStreamWaitEvent(st, h->ev_side, 0));

@@ -186,12 +186,8 @@ __device__ __forceinline__ void rank_pair(long pidx, const int* idx, const float
 // bias steers the choice only); the gates always come from the logits:
 // renormalised over the k chosen, or (full_softmax) the softmax over all N
 // logits taken at the chosen experts.
-//
-// Fusion at decode sizes (default routing only): with part the logits are
-// the sums of the router's split-K partial slices (+ bias), written to
-// logits_out as the separate reduction would.
 struct TopkArgs {
-  const float* logits;  // [T, N], or NULL with part
+  const float* logits;  // [T, N]
   int T, N, k;
   const float* sel_bias;  // variants only
   int full_softmax;       // variants only
@@ -200,12 +196,6 @@ struct TopkArgs {
   uint32_t* bitmap;  // [N, W]
   int W, debug;
   int* err;
-  // fused split-K reduction of the router logits
-  const float* part;  // S slices of [T, N] partial sums, `slice` floats apart
-  int S;
-  long slice;
-  const float* pbias;  // [N] or NULL
-  float* logits_out;   // [T, N]
 };
 
 template <int NPL, bool kVariant>
@@ -222,17 +212,7 @@ __device__ __forceinline__ void topk_token(const TopkArgs& a, int t, int lane, u
     const int e = lane + 32 * i;
     key[i] = 0u;  // absent experts: 0, never above a real key and never counted
     if (e < N) {
-      float v;
-      if (a.part) {
-        // the router's split-K partial sums, added in slice order, then the
-        // bias: the same fp32 operations as the separate reduction
-        v = 0.f;
-        for (int sl = 0; sl < a.S; ++sl) v += __ldg(a.part + (size_t)sl * a.slice + (size_t)t * N + e);
-        v = v + (a.pbias ? __ldg(a.pbias + e) : 0.f);
-        a.logits_out[(size_t)t * N + e] = v;
-      } else {
-        v = __ldg(lg + e);
-      }
+      float v = __ldg(lg + e);
       if (a.debug && !isfinite(v)) bad = true;
       if (sel_bias) v = __fadd_rn(v, __ldg(sel_bias + e));
       key[i] = orderable_bits(v);
@@ -386,7 +366,6 @@ __global__ void __launch_bounds__(128) topk_softmax_kernel(const TopkArgs a) {
 static inline cudaError_t launch_topk_args(const TopkArgs& a, cudaStream_t st, bool pdl) {
   const dim3 grid((a.T + 3) / 4), block(128);
   const bool var = a.sel_bias != nullptr || a.full_softmax != 0;
-  if (var && a.part) return cudaErrorInvalidValue;  // the fused reduction: default routing only
   cudaError_t e = cudaSuccess;
 #define LMOE_TOPK_CASE(S)                                                                   \
   case S:                                                                                   \

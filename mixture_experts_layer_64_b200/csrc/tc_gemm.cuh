@@ -76,7 +76,12 @@ struct TcCfg {
   static constexpr int ACT_BYTES = ACT_ROWS * BK * 2;
   static constexpr int W_BYTES = W_ROWS * BK * 2;
   static constexpr int W8_BYTES = kFp8 ? W_ROWS * BK : 0;  // one fp8 weight tile (64-byte rows)
-  static constexpr int STAGE_BYTES = ACT_BYTES + NUM_W * W_BYTES;  // one bf16 stage
+  // fp8 weights on weight-stationary tiles (decode): the converter warps
+  // widen each E4M3 weight tile into tensor memory, and the MMA takes its A
+  // operand (the weights) from there, so the widened tiles cost no shared
+  // memory bandwidth; the stage ring holds the activation rows only.
+  static constexpr bool kTmemA = kSwap && kFp8;
+  static constexpr int STAGE_BYTES = ACT_BYTES + (kTmemA ? 0 : NUM_W * W_BYTES);  // one stage
   // epilogue staging: one 32 x 32 box per epilogue warp (bf16 or fp32)
   static constexpr int STG_WARP = kEpi == EPI_F32_BIAS ? 4096 : 2048;
   static constexpr int STG_BYTES = kSwap ? 0 : EPI_WARPS * STG_WARP;
@@ -86,24 +91,36 @@ struct TcCfg {
   // rest as a ring of E4M3 slots (one K slice of the NUM_W weight tiles each)
   // that a producer lane fills ahead of the stages
   static constexpr int STAGES_F8 = BUDGET * 5 / 9 / STAGE_BYTES;
-  static constexpr int STAGES = kFp8 ? (STAGES_F8 < 3 ? 3 : (STAGES_F8 > 8 ? 8 : STAGES_F8))
-                                     : (STAGES_RAW > 8 ? 8 : STAGES_RAW);
+  // kTmemA: fp32 accumulators of at most 64 rows (two buffers), then a ring
+  // of widened A tiles (64 f16-wide K = 32 columns per weight tile), apart
+  // from the deeper ring of activation-row stages in shared memory, so that
+  // the rows of a K step are in place before its weights are widened
+  static constexpr int A_COLS = kTmemA ? 32 * NUM_W : 0;
+  static constexpr int STAGES_TA = kTmemA ? (512 - 2 * kSwapRowTile * NUM_W) / A_COLS : 0;
+  static constexpr int STAGES_A = kTmemA ? (STAGES_TA > 8 ? 8 : STAGES_TA) : 1;
+  static constexpr int STAGES = kTmemA ? 8
+                                : kFp8 ? (STAGES_F8 < 3 ? 3 : (STAGES_F8 > 8 ? 8 : STAGES_F8))
+                                       : (STAGES_RAW > 8 ? 8 : STAGES_RAW);
   static constexpr int W8_SLOT = NUM_W * W8_BYTES;
-  static constexpr int S8_RAW = kFp8 ? (BUDGET - STAGES * STAGE_BYTES) / W8_SLOT : 0;
-  static constexpr int S8 = S8_RAW > 16 ? 16 : S8_RAW;
+  static constexpr int S8_RAW = kFp8 ? (BUDGET - STAGES * STAGE_BYTES) / W8_SLOT : 0;  // E4M3 slots
+  static constexpr int S8 = S8_RAW > (kTmemA ? 12 : 16) ? (kTmemA ? 12 : 16) : S8_RAW;
   static constexpr int RING_BYTES = STAGES * STAGE_BYTES + S8 * W8_SLOT;
-  static constexpr int ACC_N = kSwap ? (kSwapRows > 128 ? kSwapRows : 128) : W_ROWS;  // fp32 columns of one accumulator
+  static constexpr int ACC_N = kTmemA ? kSwapRowTile
+                              : kSwap ? (kSwapRows > 128 ? kSwapRows : 128) : W_ROWS;  // fp32 columns of one accumulator
   static constexpr int ACC_COLS = ACC_N * NUM_W;      // one TMEM buffer
-  static constexpr int TMEM_COLS = 2 * ACC_COLS;      // double buffered
+  static constexpr int TMEM_COLS = kTmemA ? 512 : 2 * ACC_COLS;  // double buffered (+ A stages)
+  static constexpr int A_COL0 = 2 * ACC_COLS;         // kTmemA: first column of the A stages
   static constexpr int FT = W_ROWS;                   // features per tile
   static constexpr int TABLE_BYTES = 2 * (LMOE_MAX_EXPERTS + 1) * 4;  // tile_prefix, offsets
   static constexpr int SMEM_BYTES = 1024 /*align slack*/ + RING_BYTES + STG_BYTES + 512 +
                                     TABLE_BYTES;
   static_assert(TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM allocation must be a power of two");
+  static_assert(!kTmemA || A_COL0 + STAGES_A * A_COLS <= 512, "tensor memory: A stages");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
   static_assert(STAGES >= 3, "pipeline too shallow");
   static_assert(!kFp8 || S8 >= 2, "fp8 weight ring too shallow");
-  static_assert(2 * STAGES * 8 + 2 * S8 * 8 + 6 * 8 + 16 <= 512, "barrier area");
+  static_assert(2 * STAGES * 8 + 2 * S8 * 8 + (kTmemA ? 2 * STAGES_A * 8 : 0) + 6 * 8 + 16 <= 512,
+                "barrier area");
   static_assert(!kSwap || kEpi == EPI_ACT || kEpi == EPI_SCALE_ROWS, "swap epilogues");
   static_assert(kWN_ == 128 || kWN_ == 256, "weight tile");
   static_assert(!kFp8 || kEpi == EPI_ACT || kEpi == EPI_SCALE_ROWS, "fp8 weights: expert GEMMs");
@@ -150,6 +167,24 @@ __device__ __forceinline__ void widen_fp8_tile(const uint8_t* src, uint8_t* dst,
     *reinterpret_cast<uint4*>(row + (((2 * q) ^ sw) << 4)) = make_uint4(out[0], out[1], out[2], out[3]);
     *reinterpret_cast<uint4*>(row + (((2 * q + 1) ^ sw) << 4)) =
         make_uint4(out[4], out[5], out[6], out[7]);
+  }
+}
+
+// Widens row r of an E4M3 weight tile (64-byte rows of 64 codes, stored by
+// TMA with the 64-byte swizzle: 16-byte chunk c of row r sits at chunk
+// c ^ ((r >> 1) & 3)) into 32 words of f16 pairs, K ascending (element 2i in
+// the low half of word i).  With the swizzle a warp's 32 consecutive rows
+// read all 32 banks evenly.
+__device__ __forceinline__ void widen_fp8_row_sw64(const uint8_t* tile, int r,
+                                                   uint32_t (&out)[32]) {
+  const int x = (r >> 1) & 3;
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const uint4 v = *reinterpret_cast<const uint4*>(tile + r * 64 + ((c ^ x) << 4));
+    e4m3x4_to_f16x4(v.x, out[8 * c + 0], out[8 * c + 1]);
+    e4m3x4_to_f16x4(v.y, out[8 * c + 2], out[8 * c + 3]);
+    e4m3x4_to_f16x4(v.z, out[8 * c + 4], out[8 * c + 5]);
+    e4m3x4_to_f16x4(v.w, out[8 * c + 6], out[8 * c + 7]);
   }
 }
 
@@ -457,7 +492,9 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
   uint64_t* empty = full + Cfg::STAGES;
   uint64_t* w8full = empty + Cfg::STAGES;  // fp8: an E4M3 slot has landed
   uint64_t* w8empty = w8full + Cfg::S8;    // fp8: an E4M3 slot has been widened
-  uint64_t* tfull = w8empty + Cfg::S8;
+  uint64_t* afull = w8empty + Cfg::S8;     // kTmemA: an A stage has been widened
+  uint64_t* aempty = afull + (Cfg::kTmemA ? Cfg::STAGES_A : 0);  // kTmemA: its MMAs are done
+  uint64_t* tfull = aempty + (Cfg::kTmemA ? Cfg::STAGES_A : 0);
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
   uint64_t* epibar = drain + 1;  // stream-K: the epilogue warps meet here
@@ -476,8 +513,15 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       // the producer (its expect_tx covers the weights and the activation
       // rows, including TMA-gathered ones) + the cp.async gather threads of
       // token-tiled tiles + (fp8) one lane per converter warp
-      mbar_init(&full[s], 1 + (Cfg::kCpGather ? kGatherThreads : 0) + Cfg::CONV_THREADS / 32);
+      mbar_init(&full[s], 1 + (Cfg::kCpGather ? kGatherThreads : 0) +
+                              (Cfg::kTmemA ? 0 : Cfg::CONV_THREADS / 32));
       mbar_init(&empty[s], 1);
+    }
+    if (Cfg::kTmemA) {
+      for (int a = 0; a < Cfg::STAGES_A; ++a) {
+        mbar_init(&afull[a], Cfg::CONV_THREADS / 32);
+        mbar_init(&aempty[a], 1);
+      }
     }
     for (int j = 0; j < Cfg::S8; ++j) {
       mbar_init(&w8full[j], 1);
@@ -513,7 +557,12 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
   const int tiles_per_split = total_row_tiles_s(p, s_tiles) * NT;
   const int num_tiles = tiles_per_split * S;
   TileWalk walk{num_tiles, tiles_per_split, KB, KBS, -1};
-  if (Cfg::kSwap && !Cfg::kWideSwap && p.stream_k && S == 1 && num_tiles >= 2 * (int)gridDim.x) {
+  // stream-K only with few waves of tiles (2 to 16 per CTA): with more, the
+  // last partial wave is a small share and the contiguous per-CTA ranges
+  // (each SM on its own stretch of weights) measured slower than all SMs
+  // sweeping consecutive tiles together
+  if (Cfg::kSwap && !Cfg::kWideSwap && p.stream_k && S == 1 && num_tiles >= 2 * (int)gridDim.x &&
+      num_tiles < 16 * (int)gridDim.x) {
     const long total = (long)num_tiles * KB;
     const long per = (total + gridDim.x - 1) / gridDim.x;
     walk.u_end = min(total, (long)(blockIdx.x + 1) * per);
@@ -611,8 +660,8 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
-      int s = 0;
-      uint32_t ph = 0;
+      int s = 0, sa = 0;  // activation stage, (kTmemA) A stage
+      uint32_t ph = 0, pha = 0;
       int it = 0;
       int tl, ks, kb0, kb1;
       for (long wi = walk_start(walk); walk_next(walk, wi, tl, ks, kb0, kb1); ++it) {
@@ -636,6 +685,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         bool ok = true;
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&full[s], ph, abort_flag, p.err)) { ok = false; break; }
+          if (Cfg::kTmemA && !mbar_wait(&afull[sa], pha, abort_flag, p.err)) { ok = false; break; }
           tc_fence_after();
           const uint8_t* st = smem + s * Cfg::STAGE_BYTES;
           const uint64_t da = smem_desc_sw128(st);
@@ -645,7 +695,13 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
           for (int kk = 0; kk < Cfg::BK / 16; ++kk) {
             const uint32_t acc = (kb != kb0 || kk != 0) ? 1u : 0u;
             const uint64_t adv = (uint64_t)(kk * 32) >> 4;  // 16 bf16 = 32 bytes along K
-            if (Cfg::kSwap) {
+            if (Cfg::kTmemA) {
+              // the widened weights of stage s in tensor memory: 8 columns
+              // (16 f16) per K step, the linear half 32 columns further
+              const uint32_t a0 = tmem_base + Cfg::A_COL0 + sa * Cfg::A_COLS + kk * 8;
+              tc_mma_f16_tmem_a(d0, a0, da + adv, idesc, acc);
+              if (Cfg::kDual) tc_mma_f16_tmem_a(d1, a0 + 32, da + adv, idesc, acc);
+            } else if (Cfg::kSwap) {
               tc_mma_bf16(d0, dw0 + adv, da + adv, idesc, acc);
               if (Cfg::kDual) tc_mma_bf16(d1, dw1 + adv, da + adv, idesc, acc);
             } else {
@@ -654,6 +710,10 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
           }
           tc_commit(&empty[s]);
           if (++s == Cfg::STAGES) { s = 0; ph ^= 1; }
+          if (Cfg::kTmemA) {
+            tc_commit(&aempty[sa]);
+            if (++sa == Cfg::STAGES_A) { sa = 0; pha ^= 1; }
+          }
         }
         if (!ok) break;
         tc_commit(&tfull[ab]);
@@ -749,7 +809,51 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     // into stage s's weight slots, handed to the MMA issuer with a fence
     // (generic-proxy writes -> tensor-core reads) and an arrive on full, and
     // the slot goes back to the producer with an arrive on w8empty.
-    if (Cfg::kFp8) {
+    if (Cfg::kTmemA) {
+      // Weight-stationary tiles: converter warp w (8 of them) widens the
+      // rows of its TMEM lane quarter (w % 4; a warp may only access its own
+      // quarter) of weight tile w / 4 (gated: the gate and the linear tile;
+      // ungated: warps 0-3 the one tile) into A stage a of tensor memory,
+      // then waits for its stores and hands the stage on.
+      const int cw = warp - (4 + Cfg::EPI_WARPS);  // 0..7
+      const int qd = warp & 3;
+      const int half = cw >> 2;
+      const int r = qd * 32 + lane;  // this thread's weight row (TMEM lane)
+      int a = 0;
+      uint32_t pha = 0;
+      bool ok = true;
+      int j = 0;
+      uint32_t jph = 0;
+      int tl, ks, kb0, kb1;
+      for (long wi = walk_start(walk); ok && walk_next(walk, wi, tl, ks, kb0, kb1);) {
+        for (int kb = kb0; kb < kb1; ++kb) {
+          // the E4M3 slot has landed and the A stage's previous MMAs are done
+          if (!mbar_wait(&w8full[j], jph, abort_flag, p.err)) { ok = false; break; }
+          if (!mbar_wait(&aempty[a], pha ^ 1, abort_flag, p.err)) { ok = false; break; }
+          tc_fence_after();
+          const uint8_t* slot = w8_ring + j * Cfg::W8_SLOT;
+          const uint32_t ta = tmem_base + ((uint32_t)(qd * 32) << 16) + Cfg::A_COL0 +
+                              a * Cfg::A_COLS;
+          uint32_t v[32];
+          if (Cfg::kDual) {
+            widen_fp8_row_sw64(slot + half * Cfg::W8_BYTES, r, v);
+            tmem_st_32x32(ta + half * 32, v);
+          } else if (half == 0) {
+            widen_fp8_row_sw64(slot, r, v);
+            tmem_st_32x32(ta, v);
+          }
+          tc_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(&afull[a]);
+            mbar_arrive(&w8empty[j]);
+          }
+          if (++a == Cfg::STAGES_A) { a = 0; pha ^= 1; }
+          if (++j == Cfg::S8) { j = 0; jph ^= 1; }
+        }
+      }
+    } else if (Cfg::kFp8) {
       const int ct = threadIdx.x - (128 + 32 * Cfg::EPI_WARPS);
       int s = 0;
       uint32_t ph = 0;

@@ -68,10 +68,15 @@ def _emulated_ep(w, world, flags=0):
 
 
 def _close(res, ref, tol=2e-2):
+    """Within the stated bf16 tolerance of lmoe_forward's output, plus one
+    bf16 step of the output (2^(floor(log2|ref|) - 7)): the expert GEMMs of
+    the two paths may split a tile's K sum differently, and a last-bit
+    difference in a bf16 intermediate can move the stored output by one
+    step (0.03125 in [4, 8))."""
     a, b = res.double().cpu(), ref.double().cpu()
     err = (a - b).abs()
-    small = b.abs() < 8.0
-    assert float(err[small].max()) <= tol, float(err[small].max())
+    step = torch.exp2(torch.floor(torch.log2(b.abs().clamp_min(2.0 ** -100))) - 7)
+    assert bool((err <= tol + step).all()), float((err - step).max())
     assert float(torch.linalg.norm(a - b) / torch.linalg.norm(b)) <= 5e-3
 
 
