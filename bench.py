@@ -16,10 +16,13 @@ torch.cuda.synchronize(), and the time is the max over ranks.
 Prints one JSON line (rank 0).  With the default workload (decode, the
 headline) the line also carries "prefill": the two prefill workloads
 (latent-prefill-skewed, latent-prefill-shared), and "decode_variants": the
-latent decode workload and both decode workloads with fp8 expert weights,
-measured in the same run with the same steps and warm-up, each with its own
-clocks, roofline, expert-load summary, per-stage p50/p95/p99 and projection
-share (--no-prefill skips them).  --impl reference times the CPU oracle (the reference arm of this
+latent decode workload and both decode workloads with fp8 (E4M3) and with
+fp4 (MXFP4) expert weights, each with its own clocks, roofline, expert-load
+summary, per-stage p50/p95/p99 and projection share; and "variant_sweep": the
+standard MoE, l-MoE_eff and l-MoE_acc (LatentMoE, Section 3, Eq. (1) and
+(2)) at a decode and a prefill batch, with the weight and dispatch bytes
+each loads.  All are measured in the same run with the same steps and
+warm-up (--no-prefill skips them).  --impl reference times the CPU oracle (the reference arm of this
 method: a plain float64 C++ implementation) on a bounded token sample of the
 same workload.
 """
@@ -192,9 +195,13 @@ class OracleRunner:
                          dtype=w.dtype, skip_proj=w.skip_proj, Wg=cpu(W_dev["Wg"]),
                          bias=cpu(W_dev["bias"]), Wdown=cpu(W_dev["Wdown"]),
                          Wup=cpu(W_dev["Wup"]), Ws1=cpu(W_dev["Ws1"]), Ws2=cpu(W_dev["Ws2"]))
-        self.fp8 = bool(w.expert_fp8)
+        # low-precision experts: the codes plus their scales (fp8: per channel
+        # W1s / W2s) or block exponents (fp4: W1e / W2e)
+        self.skeys = (("W1s", "W2s") if w.expert_fp8 else ("W1e", "W2e") if w.expert_fp4
+                      else ())
         self.probe = oracle.OracleLayer(W1={}, W2={}, **self.base)
-        self.W1, self.W2, self.S1, self.S2 = {}, {}, {}, {}
+        self.W1, self.W2 = {}, {}
+        self.S = {k: {} for k in self.skeys}
 
     def time_tokens(self, tokens: np.ndarray) -> float:
         """Seconds the oracle takes for the whole layer on `tokens` (routing
@@ -203,16 +210,12 @@ class OracleRunner:
         idx, _, _, _ = self.oracle.route(lg, self.w.k)
         for e in np.unique(idx).tolist():
             if e not in self.W1:
-                if self.fp8:
-                    self.W1[e] = self.W_dev["W1q"][e].cpu()
-                    self.W2[e] = self.W_dev["W2q"][e].cpu()
-                    self.S1[e] = self.W_dev["W1s"][e].cpu()
-                    self.S2[e] = self.W_dev["W2s"][e].cpu()
-                else:
-                    self.W1[e] = self.W_dev["W1"][e].cpu()
-                    self.W2[e] = self.W_dev["W2"][e].cpu()
-        extra = dict(W1s=self.S1, W2s=self.S2) if self.fp8 else {}
-        O = self.oracle.OracleLayer(W1=self.W1, W2=self.W2, **extra, **self.base)
+                q = "q" if self.skeys else ""
+                self.W1[e] = self.W_dev["W1" + q][e].cpu()
+                self.W2[e] = self.W_dev["W2" + q][e].cpu()
+                for k in self.skeys:
+                    self.S[k][e] = self.W_dev[k][e].cpu()
+        O = self.oracle.OracleLayer(W1=self.W1, W2=self.W2, **self.S, **self.base)
         t0 = time.perf_counter()
         O.layer(self.x, tokens=tokens)
         return time.perf_counter() - t0
@@ -247,11 +250,10 @@ def dist_env():
 def workload_config(w: workloads.Workload, n_gpus: int):
     c = costmodel.layer_counts(T=w.T, d=w.d, l=w.l, N=w.N, k=w.k, m=w.m, act=w.act,
                                shared_m=w.shared_m, skip_proj=w.skip_proj,
-                               expert_bytes=1 if w.expert_fp8 else None)
+                               expert_format=w.expert_format)
     return {"workload": w.name, "T": w.T, "d": w.d, "l": w.l, "N": w.N, "k": w.k, "m": w.m,
             "act": w.act, "shared_m": w.shared_m, "skip_proj": w.skip_proj, "bias": w.bias,
-            "expert_weights": ("e4m3 codes, fp32 scale per output channel (widened to bf16 "
-                               "in the expert kernels)") if w.expert_fp8 else w.dtype,
+            "expert_weights": EXPERT_WEIGHTS.get(w.expert_format, w.dtype),
             "global_batch": w.T * n_gpus, "parallelism": f"replicas{n_gpus}",
             "l2": f"inputs larger than L2: {c.expert_weight_bytes / 1e9:.2f} GB of expert "
                   "weights streamed from HBM every step"}
@@ -317,7 +319,12 @@ def run_reference(args):
 
 PREFILL_WORKLOADS = ("latent-prefill-skewed", "latent-prefill-shared")
 # the other decode workloads, measured beside the headline in the same run
-DECODE_WORKLOADS = ("latent-decode", "std-moe-decode-fp8", "latent-decode-fp8")
+DECODE_WORKLOADS = ("latent-decode", "std-moe-decode-fp8", "latent-decode-fp8",
+                    "std-moe-decode-fp4", "latent-decode-fp4")
+EXPERT_WEIGHTS = {"e4m3": "e4m3 codes, fp32 scale per output channel (widened to f16 in the "
+                          "expert kernels)",
+                  "mxfp4": "MXFP4: e2m1 codes, one e8m0 exponent per 32 inputs (widened to f16 "
+                           "in the expert kernels)"}
 NOMINAL_HBM_GBS = 8000.0  # the ~8 TB/s HBM figure the decode target is quoted against
 PROJECTION_SHARE_PAGES = 0.09  # the paper's ~9% latent-projection overhead (Section 4.3)
 
@@ -357,10 +364,13 @@ def measure(args, name: str, pg, rank: int, ws: int, local: int, dev, flags: int
     x = workloads.make_x(xw, device=dev)
     L = lmoe.LatentMoELayer(w.d, w.l, w.N, w.k, w.m, act=w.act, shared_m=w.shared_m,
                             dtype=w.dtype, skip_proj=w.skip_proj,
-                            flags=flags | (lmoe.EXPERTS_FP8 if w.expert_fp8 else 0))
+                            flags=flags | (lmoe.EXPERTS_FP8 if w.expert_fp8 else 0) |
+                            (lmoe.EXPERTS_FP4 if w.expert_fp4 else 0))
     L.set_weights(W["Wg"], W["bias"], W["Wdown"], W["Wup"], W["W1"], W["W2"], W["Ws1"], W["Ws2"])
     if w.expert_fp8:
         L.set_expert_weights_fp8(W["W1q"], W["W1s"], W["W2q"], W["W2s"])
+    if w.expert_fp4:
+        L.set_expert_weights_fp4(W["W1q"], W["W1e"], W["W2q"], W["W2e"])
     L.reserve(w.T)
     out = torch.empty_like(x)
     stream = torch.cuda.current_stream()
@@ -437,7 +447,7 @@ def measure(args, name: str, pg, rank: int, ws: int, local: int, dev, flags: int
     counts = costmodel.stage_counts(T=w.T, d=w.d, l=w.l, N=w.N, k=w.k, m=w.m, act=w.act,
                                     shared_m=w.shared_m, skip_proj=w.skip_proj,
                                     elem_bytes=4 if w.dtype == "f32" else 2, loads=loads,
-                                    expert_bytes=1 if w.expert_fp8 else None)
+                                    expert_format=w.expert_format)
     peaks, peak_src = load_peaks()
     roofline = None
     if dom_ms > 0:
@@ -464,7 +474,7 @@ def measure(args, name: str, pg, rank: int, ws: int, local: int, dev, flags: int
                          "launch_ms": dom_ms})
     lc = costmodel.layer_counts(T=w.T, d=w.d, l=w.l, N=w.N, k=w.k, m=w.m, act=w.act,
                                 shared_m=w.shared_m, skip_proj=w.skip_proj, loads=loads,
-                                expert_bytes=1 if w.expert_fp8 else None)
+                                expert_format=w.expert_format)
     layer = {"alg_bytes": lc.bytes, "alg_flops": lc.flops,
              "hbm_frac": lc.bytes / (ms_per_step / 1e3) / 1e9 / peaks["hbm_gbs"],
              "tensor_frac_burst": lc.flops / (ms_per_step / 1e3) / 1e12 / peaks["bf16_tflops"],
@@ -503,12 +513,47 @@ def sub_record(r):
                                                         "k": w.k, "m": w.m, "act": w.act,
                                                         "shared_m": w.shared_m, "bias": w.bias,
                                                         "skip_proj": w.skip_proj,
-                                                        "expert_weights": "e4m3" if w.expert_fp8
-                                                        else w.dtype},
+                                                        "expert_weights": w.expert_format
+                                                        or w.dtype},
             "e2e": r["e2e"], "gpu_launches": r["gpu_launches"], "clocks": r["clocks"],
             "roofline": r["roofline"], "layer": r["layer"], "expert_loads": r["expert_loads"],
             "projection_share": r["projection_share"], "stage_ms": r["stage_ms"],
             "expert_path": r["expert_path"]}
+
+
+def sweep_point(variant: str, r) -> dict:
+    """One point of the LatentMoE variant sweep: the measured step and the
+    costs the paper's Table 1 compares: the expert weight bytes one token
+    activates (its k experts: the memory cost of the latency regime), the
+    bytes of one token's dispatch to its experts (one direction), the expert
+    FLOPs per token; beside them the expert weight bytes the step loads (the
+    touched experts: at batch sizes that touch every expert this is the whole
+    expert set, the same for all three variants)."""
+    w = r["w"] if "w" in r else workloads.WORKLOADS[r["workload"]]
+    touched = r["expert_loads"].get("touched", 0)
+    m_in = 2 * w.m if w.act == "swiglu" else w.m
+    return {"variant": variant, "workload": w.name, "T": w.T, "d": w.d, "l": w.l, "N": w.N,
+            "k": w.k, "m": w.m, "value": r["value"], "unit": UNIT,
+            "ms_per_step": r["ms_per_step"], "touched_experts": touched,
+            "expert_weight_bytes": touched * (w.l * m_in + w.m * w.l) * 2,
+            "active_weight_bytes_per_token": w.k * (w.l * m_in + w.m * w.l) * 2,
+            "dispatch_bytes_per_token": w.k * w.l * 2,
+            "expert_flops_per_token": 2.0 * w.k * (w.l * m_in + w.m * w.l),
+            "expert_ms": {k: r["stage_ms"][k]["p50"] for k in ("expert_fc1", "expert_fc2")}}
+
+
+def variant_sweep(points) -> dict:
+    """Ratios of each variant to the standard point of its batch size."""
+    std = points[0]
+    for p in points:
+        p["vs_standard"] = {key: round(p[key] / std[key], 4) if std[key] else None
+                            for key in ("ms_per_step", "expert_weight_bytes",
+                                        "active_weight_bytes_per_token",
+                                        "dispatch_bytes_per_token", "expert_flops_per_token")}
+    return {"points": points,
+            "paper": "Table 1: per token, l-MoE_eff cuts the active weight bytes and the "
+                     "dispatch bytes by alpha = d / l = 4 at 1 / alpha the expert FLOPs; "
+                     "l-MoE_acc keeps both costs and the FLOPs of the standard layer"}
 
 
 def run_ours(args):
@@ -528,6 +573,7 @@ def run_ours(args):
     dev = torch.device("cuda", torch.cuda.current_device())
     main = measure(args, args.workload, pg, rank, ws, local, dev, flags=args.lib_flags)
     w, W, x = main.pop("w"), main.pop("W"), main.pop("x")
+    main_point = sweep_point("standard", dict(main, w=w))
 
     cpu_baseline = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
@@ -546,7 +592,7 @@ def run_ours(args):
 
     # ---- the prefill workloads (and the other decode workloads), measured in
     # the same run with the same steps
-    extra = {"prefill": [], "decode_variants": []}
+    extra = {"prefill": [], "decode_variants": [], "variant_sweep": {}}
     if not args.no_prefill and args.workload == DEFAULT_WORKLOAD:
         for key, names in (("prefill", PREFILL_WORKLOADS), ("decode_variants", DECODE_WORKLOADS)):
             for name in names:
@@ -555,6 +601,20 @@ def run_ours(args):
                 extra[key].append(sub_record(r))
                 del r
                 torch.cuda.empty_cache()
+        # the paper's variants on the same kernels (the standard decode point
+        # is the headline workload measured above)
+        for batch, *names in workloads.VARIANT_SWEEP:
+            points = []
+            for variant, name in zip(("standard", "l-MoE_eff", "l-MoE_acc"), names):
+                if name == args.workload:
+                    points.append(main_point)
+                    continue
+                r = measure(args, name, pg, rank, ws, local, dev, flags=args.lib_flags)
+                del r["W"], r["x"]
+                points.append(sweep_point(variant, r))
+                del r
+                torch.cuda.empty_cache()
+            extra["variant_sweep"][batch] = variant_sweep(points)
 
     if rank == 0:
         roofline = main["roofline"]

@@ -149,6 +149,19 @@ typedef enum { LMOE_F32 = 0, LMOE_BF16 = 1 } lmoe_dtype;
                                     contiguous tiles by TMA instead of
                                     gathering them by token.  Off by
                                     default.  Results are the same. */
+#define LMOE_EXPERTS_FP4        0x8000u /* expert weights W1 and W2 as block-
+                                    scaled fp4 (MXFP4: E2M1 codes, one E8M0
+                                    exponent per 32 input channels;
+                                    lmoe_set_expert_weights_fp4), the format
+                                    the paper's Section 2 models its experts
+                                    in.  The expert MMAs run on f16 operands
+                                    with fp32 accumulation, on the weight-
+                                    stationary kernels at every batch size.
+                                    bf16 layers with l and m multiples of
+                                    512, not with LMOE_EXPERTS_FP8 or
+                                    LMOE_FORCE_SIMT (else
+                                    LMOE_ERR_UNSUPPORTED); no expert
+                                    parallelism.                             */
 
 /* Limits of the library. */
 #define LMOE_MAX_EXPERTS 1024
@@ -218,6 +231,32 @@ lmoe_status lmoe_set_expert_weights_fp8(lmoe_layer* h, const void* W1q, const fl
                                         const void* W2q, const float* W2s);
 
 /*
+ * lmoe_set_expert_weights_fp4 -- the expert weights of a layer created with
+ * LMOE_EXPERTS_FP4, in the OCP microscaling format MXFP4 (the FP4 expert
+ * weights the paper's Section 2 assumes for its models).  Device pointers,
+ * OUTPUT-major (each weight row is one output channel, its input channels
+ * contiguous), uint8:
+ *   W1q [N, m_in, l / 2]  E2M1 code pairs: byte j of row o holds input
+ *                         channels 2j (low nibble) and 2j + 1 (high nibble),
+ *   W1e [N, m_in, l / 32] E8M0 exponents: byte b of row o scales input
+ *                         channels [32 b, 32 b + 32) by 2^(byte - 127),
+ *   W2q [N, l, m / 2], W2e [N, l, m / 32] the same for FC2,
+ * so W1[e][i][o] = e2m1(code of channel i in row o) * 2^(W1e[e][o][i/32] - 127)
+ * (E2M1: sign, 2 exponent bits, 1 mantissa bit; magnitudes 0, 0.5, 1, 1.5, 2,
+ * 3, 4, 6).  Every exponent byte must lie in [104, 140] (scales 2^-23 ..
+ * 2^13, where code x scale is an f16 value; else LMOE_ERR_UNSUPPORTED).  The
+ * library copies them (the caller keeps its buffers); lmoe_set_weights is
+ * still required for the other weights (its W1 and W2 may be NULL).  Inside
+ * the expert kernels each 32-channel block widens exactly to f16 in tensor
+ * memory; the MMAs multiply f16 operands with fp32 accumulation, the FC1
+ * input rows are converted to f16 once per forward and FC1 writes its output
+ * in f16 (as with LMOE_EXPERTS_FP8).  Synchronous.  Errors: INVALID_ARG (NULL
+ * pointer, layer created without LMOE_EXPERTS_FP4), UNSUPPORTED, CUDA, OOM.
+ */
+lmoe_status lmoe_set_expert_weights_fp4(lmoe_layer* h, const void* W1q, const void* W1e,
+                                        const void* W2q, const void* W2e);
+
+/*
  * lmoe_reserve -- size the workspace for up to max_T tokens per call.
  * Allocates; call it before lmoe_forward / lmoe_route_only /
  * lmoe_router_logits / lmoe_forward_host.  Calling it again with a larger
@@ -283,7 +322,7 @@ typedef enum {
   LMOE_STAGE_PERM = 4,     /* [T*k]    int32 sorted row -> t*k+j             */
   LMOE_STAGE_Z = 5,        /* [T, l]   dtype  latent rows (not with SKIP)    */
   LMOE_STAGE_H = 6,        /* [T*k, m] dtype  expert hidden rows, sorted
-                              (f16 with LMOE_EXPERTS_FP8)                   */
+                              (f16 with LMOE_EXPERTS_FP8 / _FP4)            */
   LMOE_STAGE_YS = 7,       /* [T*k, l] dtype  gate-scaled expert outputs,
                                              expert-sorted rows (as H)       */
   LMOE_STAGE_COMB = 8      /* [T, l]   dtype  combined rows (not with SKIP)  */

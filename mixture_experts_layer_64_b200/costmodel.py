@@ -77,14 +77,30 @@ class LayerCounts:
     t_exp_mean: float
 
 
+# Low-precision expert weight formats: (bytes per weight, scale bytes per
+# output channel, scale bytes per weight).  e4m3: one byte per code and an fp32
+# scale per output channel; mxfp4: half a byte per E2M1 code and one E8M0 byte
+# per 32 weights.
+EXPERT_FORMATS = {"e4m3": (1.0, 4.0, 0.0), "mxfp4": (0.5, 0.0, 1.0 / 32)}
+
+
+def expert_matrix_bytes(touched: int, K: int, O: int, elem_bytes: float,
+                        expert_format: Optional[str] = None) -> float:
+    """Bytes of `touched` expert matrices of K inputs x O outputs."""
+    if expert_format is None:
+        return touched * K * O * float(elem_bytes)
+    per_w, per_ch, scale_per_w = EXPERT_FORMATS[expert_format]
+    return touched * (K * O * (per_w + scale_per_w) + O * per_ch)
+
+
 def layer_counts(*, T: int, d: int, l: int, N: int, k: int, m: int, act: str,
                  shared_m: int = 0, skip_proj: bool = False, elem_bytes: int = 2,
                  loads: Optional[Sequence[int]] = None,
-                 expert_bytes: Optional[float] = None) -> LayerCounts:
+                 expert_format: Optional[str] = None) -> LayerCounts:
     """Counts for one pass over T tokens.  ``loads`` are the per-expert row
-    counts (default: every expert touched).  ``expert_bytes``: bytes per
-    expert weight when it differs from elem_bytes (1 for fp8 codes; their
-    per-channel fp32 scales are counted too)."""
+    counts (default: every expert touched).  ``expert_format``: the expert
+    weights' low-precision format (a key of EXPERT_FORMATS, scales counted
+    too), else elem_bytes per weight."""
     m_in = 2 * m if act == "swiglu" else m
     ms_in = 2 * shared_m if act == "swiglu" else shared_m
     R = T * k
@@ -96,9 +112,8 @@ def layer_counts(*, T: int, d: int, l: int, N: int, k: int, m: int, act: str,
     proj_flops = 0.0 if skip_proj else 2.0 * (2.0 * T * d * l)
     shared_flops = 2.0 * T * (d * ms_in + shared_m * d)
     flops = router_flops + proj_flops + fc1_flops + fc2_flops + shared_flops
-    xb = eb if expert_bytes is None else expert_bytes
-    w1 = touched * l * m_in * xb + (touched * m_in * 4 if expert_bytes is not None else 0)
-    w2 = touched * m * l * xb + (touched * l * 4 if expert_bytes is not None else 0)
+    w1 = expert_matrix_bytes(touched, l, m_in, eb, expert_format)
+    w2 = expert_matrix_bytes(touched, m, l, eb, expert_format)
     other_w = d * N * eb + (0 if skip_proj else 2 * d * l * eb) + (d * ms_in + shared_m * d) * eb
     io = 2.0 * T * d * eb
     byts = w1 + w2 + other_w + io
@@ -115,21 +130,19 @@ def layer_counts(*, T: int, d: int, l: int, N: int, k: int, m: int, act: str,
 def stage_counts(*, T: int, d: int, l: int, N: int, k: int, m: int, act: str,
                  shared_m: int = 0, skip_proj: bool = False, elem_bytes: int = 2,
                  loads: Optional[Sequence[int]] = None,
-                 expert_bytes: Optional[float] = None):
+                 expert_format: Optional[str] = None):
     """Algorithmic (flops, bytes) of each launch stage of one forward pass:
     every operand read once and every result written once; expert weights
-    only for touched experts (``expert_bytes`` per weight plus fp32 scales per
-    output channel when given, as for fp8 codes).  Keys follow the library's
-    stage names."""
+    only for touched experts (in ``expert_format`` with its scales when
+    given).  Keys follow the library's stage names."""
     m_in = 2 * m if act == "swiglu" else m
     ms_in = 2 * shared_m if act == "swiglu" else shared_m
     R = T * k
     eb = elem_bytes
     touched = N if loads is None else sum(1 for c in loads if c > 0)
     kup = (0 if skip_proj else l) + shared_m
-    xb = eb if expert_bytes is None else expert_bytes
-    sc1 = touched * m_in * 4.0 if expert_bytes is not None else 0.0
-    sc2 = touched * l * 4.0 if expert_bytes is not None else 0.0
+    w1 = expert_matrix_bytes(touched, l, m_in, eb, expert_format)
+    w2 = expert_matrix_bytes(touched, m, l, eb, expert_format)
     s = {
         "router": (2.0 * T * d * N, T * d * eb + N * d * eb + T * N * 4.0),
         "topk": (0.0, T * N * 4.0 + R * 8.0),
@@ -138,8 +151,8 @@ def stage_counts(*, T: int, d: int, l: int, N: int, k: int, m: int, act: str,
                       (2.0 * T * d * l, T * d * eb + d * l * eb + T * l * eb)),
         "shared_fc1": ((0.0, 0.0) if not shared_m else
                        (2.0 * T * d * ms_in, T * d * eb + d * ms_in * eb + T * shared_m * eb)),
-        "expert_fc1": (2.0 * R * l * m_in, touched * l * m_in * xb + sc1 + T * l * eb + R * m * eb),
-        "expert_fc2": (2.0 * R * m * l, touched * m * l * xb + sc2 + R * m * eb + R * l * eb),
+        "expert_fc1": (2.0 * R * l * m_in, w1 + T * l * eb + R * m * eb),
+        "expert_fc2": (2.0 * R * m * l, w2 + R * m * eb + R * l * eb),
         "combine": (0.0, R * l * eb + T * l * eb + (T * d * eb if skip_proj else 0.0)),
         "up_proj": ((0.0, 0.0) if kup == 0 else
                     (2.0 * T * kup * d, T * kup * eb + kup * d * eb + 2.0 * T * d * eb)),

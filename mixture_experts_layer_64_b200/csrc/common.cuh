@@ -73,6 +73,8 @@ struct GemmProblem {
   const float* w_scale;   // fp8 weights (B holds E4M3 codes): scale of weight row
                           // g * w_group_stride + f, applied to the accumulator
   int* err;               // device error word
+  const uint8_t* w_exp;   // fp4 weights (B holds E2M1 code pairs, K / 2 bytes per row):
+                          // E8M0 block exponents, K / 32 bytes per weight row
   int stream_k;           // weight-stationary decode tiles: stream-K work split
   float* sk_part;         // stream-K: 2 fp32 slots of kSkSlotFloats per CTA boundary
   int* sk_count;          // stream-K: one arrival counter per boundary (zero between launches)

@@ -100,7 +100,14 @@ struct lmoe_layer {
   float* W1s = nullptr;      // [N * m_in]
   float* W2s = nullptr;      // [N * l]
   bool fp8_set = false;
-  void* a16 = nullptr;       // fp8 experts: the FC1 input rows in f16 [T, l or d]
+  // block-scaled fp4 expert weights (LMOE_EXPERTS_FP4): E2M1 code pairs and
+  // E8M0 block exponents, K-major as the caller passes them
+  uint8_t* W1q4_t = nullptr;  // [N * m_in, l / 2]
+  uint8_t* W1e_t = nullptr;   // [N * m_in, l / 32]
+  uint8_t* W2q4_t = nullptr;  // [N * l, m / 2]
+  uint8_t* W2e_t = nullptr;   // [N * l, m / 32]
+  bool fp4_set = false;
+  void* a16 = nullptr;       // fp8 / fp4 experts: the FC1 input rows in f16 [T, l or d]
   void* zs = nullptr;        // LMOE_SORTED_ROWS: the FC1 input rows in expert order [T*k, l or d]
   // workspace
   int max_T = 0, W = 0;
@@ -273,6 +280,23 @@ bool encode_map_u8(CUtensorMap* map, const void* ptr, long rows, int cols, long 
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// fp4 weights: rows of `cols` bytes (code pairs, or block exponents), boxes of
+// box_cols bytes x box_rows rows, with the 32-byte swizzle (code pairs: the
+// converters read one 32-byte row per thread) or none (exponents).
+bool encode_map_fp4(CUtensorMap* map, const void* ptr, long rows, int cols, int box_cols,
+                    int box_rows, bool sw32) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)cols};
+  cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            sw32 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Output map of the TMA-store epilogue: 32 x 32 boxes, 64-byte swizzle for
 // bf16 (64-byte rows), 128-byte swizzle for fp32 (128-byte rows).
 bool encode_out_map(CUtensorMap* map, const GemmCall& c) {
@@ -321,8 +345,11 @@ lmoe_status launch_tc(lmoe_layer* h, const GemmCall& c, cudaStream_t st) {
     h->detail = "cuTensorMapEncodeTiled (activations) failed";
     return LMOE_ERR_CUDA;
   }
-  if (!(Cfg::kFp8 ? encode_map_u8(&tb, c.p.B, c.b_rows, c.p.K, c.p.K, Cfg::W_ROWS, Cfg::kTmemA)
-                  : encode_map(&tb, c.p.B, c.b_rows, c.p.K, c.p.K, Cfg::W_ROWS))) {
+  const bool wmap =
+      Cfg::kFp4 ? encode_map_fp4(&tb, c.p.B, c.b_rows, c.p.K / 2, 32, Cfg::W_ROWS, true)
+      : Cfg::kFp8 ? encode_map_u8(&tb, c.p.B, c.b_rows, c.p.K, c.p.K, Cfg::W_ROWS, Cfg::kTmemA)
+                  : encode_map(&tb, c.p.B, c.b_rows, c.p.K, c.p.K, Cfg::W_ROWS);
+  if (!wmap) {
     h->detail = "cuTensorMapEncodeTiled (weights) failed";
     return LMOE_ERR_CUDA;
   }
@@ -330,6 +357,13 @@ lmoe_status launch_tc(lmoe_layer* h, const GemmCall& c, cudaStream_t st) {
   std::memset(&tc, 0, sizeof tc);
   GemmProblem p = c.p;
   p.tma_store = (!Cfg::kSwap && tma_store_ok(c) && encode_out_map(&tc, c)) ? 1 : 0;
+  // fp4 weights: the weight-stationary kernel's third map holds the block
+  // exponents (it stores no output tiles by TMA)
+  if (Cfg::kFp4 &&
+      !encode_map_fp4(&tc, c.p.w_exp, c.b_rows, c.p.K / 32, 16, Cfg::W_ROWS, false)) {
+    h->detail = "cuTensorMapEncodeTiled (fp4 exponents) failed";
+    return LMOE_ERR_CUDA;
+  }
   const long NT = (c.p.F + Cfg::FT - 1) / Cfg::FT;
   const long tiles = (long)c.p.max_row_tiles * NT * std::max(1, c.p.splits);
   const int grid = (int)std::max(1L, std::min<long>(h->num_sms, tiles));
@@ -550,6 +584,23 @@ lmoe_status run_gemm(lmoe_layer* h, GemmCall c, cudaStream_t st, int* path = nul
       g.p.sk_count = h->sk_count;
     }
   };
+  if (c.p.w_exp) {
+    // fp4 expert weights: the weight-stationary kernel, weights widened into
+    // tensor memory, at every batch size
+    if (!tc_eligible(h, c) || !c.swap || c.pair) {
+      h->detail = "fp4 expert weights need the weight-stationary tensor-core kernel";
+      return LMOE_ERR_UNSUPPORTED;
+    }
+    swap_rows(c);
+    const bool dual = c.p.dual_offset > 0;
+    if (path) *path = 2;
+    if (c.kind == GK_FC1)
+      return dual ? launch_tc<TcCfg<true, true, true, 128, EPI_ACT, true, kSwapRowTile, true>>(h, c, st)
+                  : launch_tc<TcCfg<true, true, false, 128, EPI_ACT, true, kSwapRowTile, true>>(h, c, st);
+    if (c.kind == GK_FC2)
+      return launch_tc<TcCfg<true, false, false, 128, EPI_SCALE_ROWS, true, kSwapRowTile, true>>(h, c, st);
+    return LMOE_ERR_INVALID_ARG;
+  }
   if (c.p.w_scale) {
     // fp8 expert weights: the single-CTA tensor-core kernel with the E4M3
     // widening warps (weight-stationary or token-tiled)
@@ -926,13 +977,16 @@ lmoe_status run_expert_gemms(lmoe_layer* h, const Grouping& g, const void* A, lo
   const int l = h->l, m = h->m;
   const bool skip = (h->flags & LMOE_SKIP_PROJ) != 0;
   const int cols = skip ? h->d : l;
-  const bool swap = use_swap(h, R, g.G);
-  const bool pairs_ok = pairs_allowed(h);
   const bool fp8 = (h->flags & LMOE_EXPERTS_FP8) != 0;
+  const bool fp4 = (h->flags & LMOE_EXPERTS_FP4) != 0;
+  const bool lowp = fp8 || fp4;  // f16 FC1 input and output
+  // fp4 weights run on the weight-stationary kernels at every size
+  const bool swap = fp4 || use_swap(h, R, g.G);
+  const bool pairs_ok = pairs_allowed(h);
   // token-tiled expert GEMMs with FC1 on single CTAs and FC2 on CTA pairs,
   // or (LMOE_LOAD_SPLIT) split by load: experts with many rows on CTA pairs,
   // the rest on weight-stationary single-CTA tiles
-  const bool load_split = pairs_ok && !swap && !fp8 && (h->flags & LMOE_LOAD_SPLIT) &&
+  const bool load_split = pairs_ok && !swap && !lowp && (h->flags & LMOE_LOAD_SPLIT) &&
                           !(h->flags & LMOE_FORCE_WS_PAIR) && l % 64 == 0 && m % 64 == 0;
   const bool pair_fc2 = pairs_ok && !swap;
   // on request: the expert GEMMs weight-stationary on CTA pairs (rows on the
@@ -940,8 +994,8 @@ lmoe_status run_expert_gemms(lmoe_layer* h, const Grouping& g, const void* A, lo
   const bool ws_pair = pairs_ok && !swap && (h->flags & LMOE_FORCE_WS_PAIR) &&
                        !(h->flags & LMOE_FORCE_NOSWAP);
   {
-    if (fp8) {
-      // the fp8 expert kernels multiply f16 operands: the FC1 input in f16
+    if (lowp) {
+      // the fp8 / fp4 expert kernels multiply f16 operands: the FC1 input in f16
       const long n = a_rows * cols;
       const int vec = (n % 8 == 0 && aligned16(A) && aligned16(h->a16)) ? 1 : 0;
       const long work = vec ? n / 8 : n;
@@ -951,7 +1005,7 @@ lmoe_status run_expert_gemms(lmoe_layer* h, const Grouping& g, const void* A, lo
                   static_cast<const bf16*>(A), static_cast<__half*>(h->a16), n, vec);
       A = h->a16;
     }
-    const bool sorted = (h->flags & LMOE_SORTED_ROWS) && h->dtype == LMOE_BF16 && !fp8 && gather;
+    const bool sorted = (h->flags & LMOE_SORTED_ROWS) && h->dtype == LMOE_BF16 && !lowp && gather;
     if (sorted) {
       // the FC1 input rows copied into expert order: FC1 then loads them as
       // contiguous tiles (by TMA) like FC2 does its input
@@ -966,12 +1020,16 @@ lmoe_status run_expert_gemms(lmoe_layer* h, const Grouping& g, const void* A, lo
       a_rows = R;
       gather = nullptr;
     }
+    // (fp4: the weight rows hold l / 2 bytes; the expert offset g.e0 is 0,
+    // expert parallelism takes no fp4 layers)
     GemmCall c = grouped_call(g, GK_FC1, R, A, lda, a_rows, gather,
-                              fp8 ? (const void*)h->W1q_t : h->W1_t, fp8 ? 1 : h->es, h->m_in,
-                              m, l);
+                              fp4 ? (const void*)h->W1q4_t
+                                  : fp8 ? (const void*)h->W1q_t : h->W1_t,
+                              fp8 ? 1 : h->es, h->m_in, m, l);
     c.p.w_scale = fp8 ? h->W1s + (size_t)g.e0 * h->m_in : nullptr;
+    c.p.w_exp = fp4 ? h->W1e_t : nullptr;
     c.swap = swap;
-    c.ws_pair = ws_pair && !fp8;
+    c.ws_pair = ws_pair && !lowp;
     c.p.dual_offset = h->act == LMOE_ACT_SWIGLU ? m : 0;
     c.p.epi.out = hbuf;
     c.p.epi.ldo = m;
@@ -984,10 +1042,13 @@ lmoe_status run_expert_gemms(lmoe_layer* h, const Grouping& g, const void* A, lo
   prof_mark(h, st, 6);
   {
     GemmCall c = grouped_call(g, GK_FC2, R, hbuf, m, R, nullptr,
-                              fp8 ? (const void*)h->W2q_t : h->W2_t, fp8 ? 1 : h->es, l, l, m);
+                              fp4 ? (const void*)h->W2q4_t
+                                  : fp8 ? (const void*)h->W2q_t : h->W2_t,
+                              fp8 ? 1 : h->es, l, l, m);
     c.p.w_scale = fp8 ? h->W2s + (size_t)g.e0 * l : nullptr;
+    c.p.w_exp = fp4 ? h->W2e_t : nullptr;
     c.swap = swap;
-    c.ws_pair = ws_pair && !fp8;
+    c.ws_pair = ws_pair && !lowp;
     c.p.epi.out = ysbuf;
     c.p.epi.ldo = l;
     c.p.epi.row_w = row_w;
@@ -995,7 +1056,7 @@ lmoe_status run_expert_gemms(lmoe_layer* h, const Grouping& g, const void* A, lo
     if (load_split) {
       LMOE_TRY(run_split_by_load(h, c, st, &path));
     } else {
-      if (pair_fc2 && !ws_pair && !fp8) make_pair(h, c);  // the pair kernels read bf16 weights
+      if (pair_fc2 && !ws_pair && !lowp) make_pair(h, c);  // the pair kernels read bf16 weights
       LMOE_TRY(run_gemm(h, c, st, &path));
     }
     h->expert_path |= path << 3;
@@ -1186,6 +1247,11 @@ void free_weights(lmoe_layer* h) {
   free_ptr(h->W1_t);
   free_ptr(h->W1q_t);
   free_ptr(h->W2q_t);
+  free_ptr(h->W1q4_t);
+  free_ptr(h->W1e_t);
+  free_ptr(h->W2q4_t);
+  free_ptr(h->W2e_t);
+  h->fp4_set = false;
   free_ptr(h->W1s);
   free_ptr(h->W2s);
   h->fp8_set = false;
@@ -1218,7 +1284,8 @@ bool valid_stream_call(const lmoe_layer* h, int T) { return h && T >= 0 && T <= 
 
 // Weights in place: lmoe_set_weights, and with fp8 experts their codes too.
 bool layer_ready(const lmoe_layer* h) {
-  return h->weights_set && (!(h->flags & LMOE_EXPERTS_FP8) || h->fp8_set);
+  return h->weights_set && (!(h->flags & LMOE_EXPERTS_FP8) || h->fp8_set) &&
+         (!(h->flags & LMOE_EXPERTS_FP4) || h->fp4_set);
 }
 
 }  // namespace
@@ -1254,6 +1321,7 @@ lmoe_status lmoe_create(int d, int l, int N, int k, int m, lmoe_act act, int sha
   const unsigned known = LMOE_SKIP_PROJ | LMOE_DEBUG_CHECKS | LMOE_FORCE_SIMT | LMOE_FORCE_SWAP |
                          LMOE_FORCE_NOSWAP | LMOE_FORCE_NOPAIR | LMOE_FORCE_WS_PAIR |
                          LMOE_ROUTE_FULL_SOFTMAX | LMOE_ROUTE_BIAS_SELECT | LMOE_EXPERTS_FP8 |
+                         LMOE_EXPERTS_FP4 |
                          LMOE_SINGLE_STREAM | LMOE_NO_PDL | LMOE_LOAD_SPLIT |
                          LMOE_NO_STREAM_K | LMOE_SORTED_ROWS;
   if (d <= 0 || l <= 0 || N <= 0 || k <= 0 || m <= 0 || shared_m < 0) return LMOE_ERR_INVALID_ARG;
@@ -1264,6 +1332,12 @@ lmoe_status lmoe_create(int d, int l, int N, int k, int m, lmoe_act act, int sha
   if ((flags & LMOE_FORCE_SWAP) && (flags & LMOE_FORCE_NOSWAP)) return LMOE_ERR_INVALID_ARG;
   // fp8 expert weights run on the tensor-core kernels only: bf16 layers whose
   // expert GEMMs have K (l and m) a multiple of 64
+  // fp4 expert weights: bf16 layers whose K (l and m) rows of block exponents
+  // are whole 16-byte boxes (K a multiple of 512); not with fp8
+  if ((flags & LMOE_EXPERTS_FP4) &&
+      (dtype != LMOE_BF16 || (flags & (LMOE_FORCE_SIMT | LMOE_EXPERTS_FP8)) || l % 512 != 0 ||
+       m % 512 != 0))
+    return LMOE_ERR_UNSUPPORTED;
   if ((flags & LMOE_EXPERTS_FP8) &&
       (dtype != LMOE_BF16 || (flags & LMOE_FORCE_SIMT) || l % 64 != 0 || m % 64 != 0))
     return LMOE_ERR_UNSUPPORTED;
@@ -1296,7 +1370,7 @@ lmoe_status lmoe_create(int d, int l, int N, int k, int m, lmoe_act act, int sha
 lmoe_status lmoe_set_weights(lmoe_layer* h, const void* W_g, const float* bias, const void* W_down,
                              const void* W_up, const void* W1, const void* W2, const void* Ws1,
                              const void* Ws2) {
-  const bool fp8 = h && (h->flags & LMOE_EXPERTS_FP8);
+  const bool fp8 = h && (h->flags & (LMOE_EXPERTS_FP8 | LMOE_EXPERTS_FP4));
   if (!h || !W_g || (!fp8 && (!W1 || !W2))) return LMOE_ERR_INVALID_ARG;
   const bool skip = (h->flags & LMOE_SKIP_PROJ) != 0;
   if (skip != (W_down == nullptr) || skip != (W_up == nullptr)) return LMOE_ERR_INVALID_ARG;
@@ -1374,6 +1448,42 @@ lmoe_status lmoe_set_expert_weights_fp8(lmoe_layer* h, const void* W1q, const fl
   return LMOE_OK;
 }
 
+lmoe_status lmoe_set_expert_weights_fp4(lmoe_layer* h, const void* W1q, const void* W1e,
+                                        const void* W2q, const void* W2e) {
+  if (!h || !W1q || !W1e || !W2q || !W2e) return LMOE_ERR_INVALID_ARG;
+  if (!(h->flags & LMOE_EXPERTS_FP4)) return LMOE_ERR_INVALID_ARG;
+  DevGuard g(h->device);
+  const size_t N = h->N, l = h->l, m = h->m, m_in = h->m_in;
+  const size_t e1 = N * m_in * (l / 32), e2 = N * l * (m / 32);
+  // every block exponent must keep code x 2^(e - 127) an f16 value
+  {
+    std::vector<uint8_t> ex(std::max(e1, e2));
+    for (int i = 0; i < 2; ++i) {
+      const size_t n = i ? e2 : e1;
+      LMOE_CUDA(h, cudaMemcpy(ex.data(), i ? W2e : W1e, n, cudaMemcpyDeviceToHost));
+      for (size_t j = 0; j < n; ++j)
+        if (ex[j] < 127 - 23 || ex[j] > 127 + 13) {
+          h->detail = "fp4 block exponent outside [2^-23, 2^13]";
+          return LMOE_ERR_UNSUPPORTED;
+        }
+    }
+  }
+  LMOE_CUDA(h, cudaDeviceSynchronize());
+  if (!h->fp4_set) {
+    LMOE_CUDA(h, cudaMalloc(&h->W1q4_t, N * m_in * (l / 2)));
+    LMOE_CUDA(h, cudaMalloc(&h->W1e_t, e1));
+    LMOE_CUDA(h, cudaMalloc(&h->W2q4_t, N * l * (m / 2)));
+    LMOE_CUDA(h, cudaMalloc(&h->W2e_t, e2));
+  }
+  LMOE_CUDA(h, cudaMemcpy(h->W1q4_t, W1q, N * m_in * (l / 2), cudaMemcpyDeviceToDevice));
+  LMOE_CUDA(h, cudaMemcpy(h->W1e_t, W1e, e1, cudaMemcpyDeviceToDevice));
+  LMOE_CUDA(h, cudaMemcpy(h->W2q4_t, W2q, N * l * (m / 2), cudaMemcpyDeviceToDevice));
+  LMOE_CUDA(h, cudaMemcpy(h->W2e_t, W2e, e2, cudaMemcpyDeviceToDevice));
+  LMOE_CUDA(h, cudaDeviceSynchronize());
+  h->fp4_set = true;
+  return LMOE_OK;
+}
+
 lmoe_status lmoe_reserve(lmoe_layer* h, int max_T) {
   if (!h || max_T < 1) return LMOE_ERR_INVALID_ARG;
   if (max_T <= h->max_T) return LMOE_OK;
@@ -1420,7 +1530,7 @@ lmoe_status lmoe_reserve(lmoe_layer* h, int max_T) {
     LMOE_CUDA(h, cudaEventCreateWithFlags(&h->ev_used[i], cudaEventDisableTiming));
   }
   if (skip && h->shared_m > 0) ALLOC(h->s32, T * h->d * sizeof(float));
-  if (h->flags & LMOE_EXPERTS_FP8) ALLOC(h->a16, T * (skip ? h->d : h->l) * 2);
+  if (h->flags & (LMOE_EXPERTS_FP8 | LMOE_EXPERTS_FP4)) ALLOC(h->a16, T * (skip ? h->d : h->l) * 2);
   if (h->flags & LMOE_SORTED_ROWS) ALLOC(h->zs, R * (skip ? h->d : h->l) * 2);
   if (h->dtype == LMOE_BF16) {
     h->part_bytes = kSplitPartBytes;
@@ -1720,7 +1830,7 @@ lmoe_status lmoe_ep_dispatch(lmoe_layer* h, const void* x, int T, void* send_row
                              float* send_gates, int* expert_counts, lmoe_stream_t stream) {
   if (!h) return LMOE_ERR_INVALID_ARG;
   if (!layer_ready(h) || h->max_T == 0) return LMOE_ERR_NOT_READY;
-  if (h->flags & LMOE_EXPERTS_FP8) return LMOE_ERR_UNSUPPORTED;
+  if (h->flags & (LMOE_EXPERTS_FP8 | LMOE_EXPERTS_FP4)) return LMOE_ERR_UNSUPPORTED;
   if (T < 1 || T > h->max_T || !x || !send_rows || !send_gates || !expert_counts)
     return LMOE_ERR_INVALID_ARG;
   DevGuard g(h->device);
@@ -1761,7 +1871,7 @@ lmoe_status lmoe_ep_experts(lmoe_layer* h, const void* recv_rows, const float* r
   if (!h) return LMOE_ERR_INVALID_ARG;
   if (!layer_ready(h)) return LMOE_ERR_NOT_READY;
   if (h->ep_max_rows == 0) return LMOE_ERR_NOT_READY;
-  if (h->flags & LMOE_EXPERTS_FP8) return LMOE_ERR_UNSUPPORTED;
+  if (h->flags & (LMOE_EXPERTS_FP8 | LMOE_EXPERTS_FP4)) return LMOE_ERR_UNSUPPORTED;
   if (!recv_counts || world < 1 || rank < 0 || rank >= world || h->N % world != 0)
     return LMOE_ERR_INVALID_ARG;
   const int n = h->N / world;

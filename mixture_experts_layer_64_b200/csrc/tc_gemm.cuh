@@ -46,9 +46,18 @@ constexpr int kTcThreads = 384;
 constexpr int kEpiWarps = 8;  // two warpgroups; each warp reads its TMEM lane quarter (warp % 4)
 constexpr int kTcSmemBudget = 200 * 1024;
 constexpr int kGatherThreads = 64;
+#ifndef LMOE_TMEMA_ACC_BUFS
+#define LMOE_TMEMA_ACC_BUFS 2
+#endif
+#ifndef LMOE_TMEMA_STAGES
+#define LMOE_TMEMA_STAGES 8
+#endif
+#ifndef LMOE_TMEMA_S8CAP
+#define LMOE_TMEMA_S8CAP 12
+#endif
 
 template <bool kSwap_, bool kGather_, bool kDual_, int kWN_, int kEpi_, bool kFp8_ = false,
-          int kSwapRows_ = kSwapRowTile>
+          int kSwapRows_ = kSwapRowTile, bool kFp4_ = false>
 struct TcCfg {
   static constexpr bool kSwap = kSwap_, kGather = kGather_, kDual = kDual_, kFp8 = kFp8_;
   static constexpr int kEpi = kEpi_;
@@ -75,7 +84,13 @@ struct TcCfg {
   static constexpr int NUM_W = kDual ? 2 : 1;
   static constexpr int ACT_BYTES = ACT_ROWS * BK * 2;
   static constexpr int W_BYTES = W_ROWS * BK * 2;
-  static constexpr int W8_BYTES = kFp8 ? W_ROWS * BK : 0;  // one fp8 weight tile (64-byte rows)
+  // low-precision weights: block-scaled FP4 (kFp4: E2M1 code pairs, 32-byte
+  // rows per 64-wide K slice, then the tile's E8M0 exponents, a 16-byte box
+  // per row) or fp8 E4M3 (64-byte rows)
+  static constexpr bool kFp4 = kFp4_;
+  static constexpr int W4_CODES = kFp4 ? W_ROWS * BK / 2 : 0;  // one fp4 weight tile's codes
+  static constexpr int W4_EXPS = kFp4 ? W_ROWS * 16 : 0;       // ... and its exponent box
+  static constexpr int W8_BYTES = kFp4 ? W4_CODES + W4_EXPS : kFp8 ? W_ROWS * BK : 0;
   // fp8 weights on weight-stationary tiles (decode): the converter warps
   // widen each E4M3 weight tile into tensor memory, and the MMA takes its A
   // operand (the weights) from there, so the widened tiles cost no shared
@@ -96,20 +111,27 @@ struct TcCfg {
   // from the deeper ring of activation-row stages in shared memory, so that
   // the rows of a K step are in place before its weights are widened
   static constexpr int A_COLS = kTmemA ? 32 * NUM_W : 0;
-  static constexpr int STAGES_TA = kTmemA ? (512 - 2 * kSwapRowTile * NUM_W) / A_COLS : 0;
+  static constexpr int ACC_BUFS = kTmemA ? LMOE_TMEMA_ACC_BUFS : 2;  // accumulator buffers
+  static constexpr int STAGES_TA =
+      kTmemA ? (512 - ACC_BUFS * kSwapRowTile * NUM_W) / A_COLS : 0;
   static constexpr int STAGES_A = kTmemA ? (STAGES_TA > 8 ? 8 : STAGES_TA) : 1;
-  static constexpr int STAGES = kTmemA ? 8
+  // kTmemA: converter warps per K step (unit).  Gated tiles: all eight
+  // (warps 0-3 the gate tile, 4-7 the linear one); ungated tiles: the two
+  // groups of four take alternate units, so two units widen at once.
+  static constexpr int CONV_PER_UNIT = kTmemA ? (kDual ? 8 : 4) : (kFp8 ? 8 : 0);
+  static constexpr int STAGES = kTmemA ? LMOE_TMEMA_STAGES
                                 : kFp8 ? (STAGES_F8 < 3 ? 3 : (STAGES_F8 > 8 ? 8 : STAGES_F8))
                                        : (STAGES_RAW > 8 ? 8 : STAGES_RAW);
   static constexpr int W8_SLOT = NUM_W * W8_BYTES;
   static constexpr int S8_RAW = kFp8 ? (BUDGET - STAGES * STAGE_BYTES) / W8_SLOT : 0;  // E4M3 slots
-  static constexpr int S8 = S8_RAW > (kTmemA ? 12 : 16) ? (kTmemA ? 12 : 16) : S8_RAW;
+  static constexpr int S8_CAP = kTmemA ? LMOE_TMEMA_S8CAP : 16;
+  static constexpr int S8 = S8_RAW > S8_CAP ? S8_CAP : S8_RAW;
   static constexpr int RING_BYTES = STAGES * STAGE_BYTES + S8 * W8_SLOT;
   static constexpr int ACC_N = kTmemA ? kSwapRowTile
                               : kSwap ? (kSwapRows > 128 ? kSwapRows : 128) : W_ROWS;  // fp32 columns of one accumulator
   static constexpr int ACC_COLS = ACC_N * NUM_W;      // one TMEM buffer
   static constexpr int TMEM_COLS = kTmemA ? 512 : 2 * ACC_COLS;  // double buffered (+ A stages)
-  static constexpr int A_COL0 = 2 * ACC_COLS;         // kTmemA: first column of the A stages
+  static constexpr int A_COL0 = ACC_BUFS * ACC_COLS;  // kTmemA: first column of the A stages
   static constexpr int FT = W_ROWS;                   // features per tile
   static constexpr int TABLE_BYTES = 2 * (LMOE_MAX_EXPERTS + 1) * 4;  // tile_prefix, offsets
   static constexpr int SMEM_BYTES = 1024 /*align slack*/ + RING_BYTES + STG_BYTES + 512 +
@@ -119,6 +141,8 @@ struct TcCfg {
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
   static_assert(STAGES >= 3, "pipeline too shallow");
   static_assert(!kFp8 || S8 >= 2, "fp8 weight ring too shallow");
+  static_assert(!kTmemA || (S8 >= 2 && STAGES_A >= 2), "tensor-memory A rings too shallow");
+  static_assert(ACC_BUFS == 1 || ACC_BUFS == 2, "accumulator buffers");
   static_assert(2 * STAGES * 8 + 2 * S8 * 8 + (kTmemA ? 2 * STAGES_A * 8 : 0) + 6 * 8 + 16 <= 512,
                 "barrier area");
   static_assert(!kSwap || kEpi == EPI_ACT || kEpi == EPI_SCALE_ROWS, "swap epilogues");
@@ -126,6 +150,7 @@ struct TcCfg {
   static_assert(!kFp8 || kEpi == EPI_ACT || kEpi == EPI_SCALE_ROWS, "fp8 weights: expert GEMMs");
   static_assert(kSwapRows == kSwapRowTile || kSwapRows == 128 || kSwapRows == 256, "swap rows");
   static_assert(!kWideSwap || !kFp8, "wide weight-stationary tiles: bf16 weights");
+  static_assert(!kFp4 || (kFp8 && kSwap), "fp4 weights: the weight-stationary tensor-memory path");
 };
 
 // ---- fp8 E4M3 weights -----------------------------------------------------------
@@ -185,6 +210,53 @@ __device__ __forceinline__ void widen_fp8_row_sw64(const uint8_t* tile, int r,
     e4m3x4_to_f16x4(v.y, out[8 * c + 2], out[8 * c + 3]);
     e4m3x4_to_f16x4(v.z, out[8 * c + 4], out[8 * c + 5]);
     e4m3x4_to_f16x4(v.w, out[8 * c + 6], out[8 * c + 7]);
+  }
+}
+
+// 2^e as an f16, for e in [-24, 15], built from the binary16 encoding: a
+// normal number (biased exponent e + 15, zero mantissa) for e >= -14, else
+// the subnormal with the single mantissa bit e + 24.
+__device__ __forceinline__ __half pow2_half(int e) {
+  const unsigned short bits =
+      e >= -14 ? (unsigned short)((e + 15) << 10) : (unsigned short)(1u << (e + 24));
+  return __ushort_as_half(bits);
+}
+
+// Widens row r of an MXFP4 weight tile for one 64-wide K slice: 32 bytes of
+// E2M1 code pairs (TMA-stored with the 32-byte swizzle: 16-byte chunk c of
+// row r sits at chunk c ^ ((r >> 2) & 1)) and the row's two E8M0 block
+// exponents, at byte `eoff` of its 16-byte exponent row.  Each code widens
+// exactly to f16 (cvt.rn.f16x2.e2m1x2), then takes its block's power of two
+// (an exact f16 multiply: the exponents are limited so that every product is
+// an f16 value).  Output as widen_fp8_row_sw64: 32 words of f16 pairs, K
+// ascending.
+__device__ __forceinline__ void widen_fp4_row_sw32(const uint8_t* codes, const uint8_t* exps, int r,
+                                                   int eoff, uint32_t (&out)[32]) {
+  const int x = (r >> 2) & 1;
+#pragma unroll
+  for (int c = 0; c < 2; ++c) {  // chunk c: K elements 32c .. 32c + 31, block c
+    const uint4 v = *reinterpret_cast<const uint4*>(codes + r * 32 + ((c ^ x) << 4));
+    const __half2 sc = __half2half2(pow2_half((int)exps[r * 16 + eoff + c] - 127));
+    const uint32_t in[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {  // 8 codes: bytes b0..b3, low nibble first
+      uint32_t w0, w1, w2, w3;
+      asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+          "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+          "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+          "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+          "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
+          "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+          : "=r"(w0), "=r"(w1), "=r"(w2), "=r"(w3)
+          : "r"(in[q]));
+      const uint32_t ws[4] = {w0, w1, w2, w3};
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        __half2 h = *reinterpret_cast<const __half2*>(&ws[b]);
+        h = __hmul2(h, sc);
+        out[16 * c + 4 * q + b] = *reinterpret_cast<const uint32_t*>(&h);
+      }
+    }
   }
 }
 
@@ -519,13 +591,13 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     }
     if (Cfg::kTmemA) {
       for (int a = 0; a < Cfg::STAGES_A; ++a) {
-        mbar_init(&afull[a], Cfg::CONV_THREADS / 32);
+        mbar_init(&afull[a], Cfg::CONV_PER_UNIT);
         mbar_init(&aempty[a], 1);
       }
     }
     for (int j = 0; j < Cfg::S8; ++j) {
       mbar_init(&w8full[j], 1);
-      mbar_init(&w8empty[j], Cfg::CONV_THREADS / 32);
+      mbar_init(&w8empty[j], Cfg::CONV_PER_UNIT);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
@@ -539,6 +611,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
   if (warp == 0 && lane == 0) {
     if (!Cfg::kGather) prefetch_tensormap(&tmA);
     prefetch_tensormap(&tmB);
+    if (Cfg::kFp4) prefetch_tensormap(&tmC);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
@@ -588,10 +661,25 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
           if (!mbar_wait(&w8empty[j], jph ^ 1, abort_flag, p.err)) { ok = false; break; }
           uint8_t* slot = w8_ring + j * Cfg::W8_SLOT;
           mbar_arrive_expect_tx(&w8full[j], Cfg::W8_SLOT);
-          tma_load_2d(&tmB, &w8full[j], slot, kb * Cfg::BK, wrow);
-          if (Cfg::kDual)
-            tma_load_2d(&tmB, &w8full[j], slot + Cfg::W8_BYTES, kb * Cfg::BK,
-                        wrow + p.dual_offset);
+          if (Cfg::kFp4) {
+            // code pairs (32 bytes per row of the K slice), then the exponent
+            // box holding this slice's two exponents (16-byte aligned start;
+            // tmC is the exponent map in the weight-stationary kernels)
+            const int ex = (kb * 2) & ~15;
+            tma_load_2d(&tmB, &w8full[j], slot, kb * (Cfg::BK / 2), wrow);
+            tma_load_2d(&tmC, &w8full[j], slot + Cfg::W4_CODES, ex, wrow);
+            if (Cfg::kDual) {
+              tma_load_2d(&tmB, &w8full[j], slot + Cfg::W8_BYTES, kb * (Cfg::BK / 2),
+                          wrow + p.dual_offset);
+              tma_load_2d(&tmC, &w8full[j], slot + Cfg::W8_BYTES + Cfg::W4_CODES, ex,
+                          wrow + p.dual_offset);
+            }
+          } else {
+            tma_load_2d(&tmB, &w8full[j], slot, kb * Cfg::BK, wrow);
+            if (Cfg::kDual)
+              tma_load_2d(&tmB, &w8full[j], slot + Cfg::W8_BYTES, kb * Cfg::BK,
+                          wrow + p.dual_offset);
+          }
           ++wissued;
           if (++j == Cfg::S8) { j = 0; jph ^= 1; }
         }
@@ -668,8 +756,8 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         const int rt = tl / NT;
         int g, row0, rows;
         locate_row_tile_s(p, s_tiles, rt, g, row0, rows);
-        const int ab = it & 1;
-        const uint32_t aph = (it >> 1) & 1;
+        const int ab = Cfg::ACC_BUFS == 2 ? (it & 1) : 0;
+        const uint32_t aph = Cfg::ACC_BUFS == 2 ? (uint32_t)(it >> 1) & 1 : (uint32_t)it & 1;
         if (!mbar_wait(&tempty[ab], aph ^ 1, abort_flag, p.err)) break;
         tc_fence_after();
         const uint32_t d0 = tmem_base + ab * Cfg::ACC_COLS;
@@ -813,42 +901,44 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       // Weight-stationary tiles: converter warp w (8 of them) widens the
       // rows of its TMEM lane quarter (w % 4; a warp may only access its own
       // quarter) of weight tile w / 4 (gated: the gate and the linear tile;
-      // ungated: warps 0-3 the one tile) into A stage a of tensor memory,
-      // then waits for its stores and hands the stage on.
+      // ungated: group w / 4 takes every other unit) into A stage a of
+      // tensor memory, then waits for its stores and hands the stage on.
+      // Units are the walk's K steps in order; every warp advances the slot
+      // and stage counters over all of them.
       const int cw = warp - (4 + Cfg::EPI_WARPS);  // 0..7
       const int qd = warp & 3;
       const int half = cw >> 2;
       const int r = qd * 32 + lane;  // this thread's weight row (TMEM lane)
-      int a = 0;
-      uint32_t pha = 0;
+      int a = 0, j = 0, par = 0;
+      uint32_t pha = 0, jph = 0;
       bool ok = true;
-      int j = 0;
-      uint32_t jph = 0;
       int tl, ks, kb0, kb1;
       for (long wi = walk_start(walk); ok && walk_next(walk, wi, tl, ks, kb0, kb1);) {
         for (int kb = kb0; kb < kb1; ++kb) {
-          // the E4M3 slot has landed and the A stage's previous MMAs are done
-          if (!mbar_wait(&w8full[j], jph, abort_flag, p.err)) { ok = false; break; }
-          if (!mbar_wait(&aempty[a], pha ^ 1, abort_flag, p.err)) { ok = false; break; }
-          tc_fence_after();
-          const uint8_t* slot = w8_ring + j * Cfg::W8_SLOT;
-          const uint32_t ta = tmem_base + ((uint32_t)(qd * 32) << 16) + Cfg::A_COL0 +
-                              a * Cfg::A_COLS;
-          uint32_t v[32];
-          if (Cfg::kDual) {
-            widen_fp8_row_sw64(slot + half * Cfg::W8_BYTES, r, v);
-            tmem_st_32x32(ta + half * 32, v);
-          } else if (half == 0) {
-            widen_fp8_row_sw64(slot, r, v);
+          if (Cfg::kDual || par == half) {
+            // the slot has landed and the A stage's previous MMAs are done
+            if (!mbar_wait(&w8full[j], jph, abort_flag, p.err)) { ok = false; break; }
+            if (!mbar_wait(&aempty[a], pha ^ 1, abort_flag, p.err)) { ok = false; break; }
+            tc_fence_after();
+            const uint8_t* tile =
+                w8_ring + j * Cfg::W8_SLOT + (Cfg::kDual ? half : 0) * Cfg::W8_BYTES;
+            const uint32_t ta = tmem_base + ((uint32_t)(qd * 32) << 16) + Cfg::A_COL0 +
+                                a * Cfg::A_COLS + (Cfg::kDual ? half * 32 : 0);
+            uint32_t v[32];
+            if (Cfg::kFp4)
+              widen_fp4_row_sw32(tile, tile + Cfg::W4_CODES, r, (kb * 2) & 15, v);
+            else
+              widen_fp8_row_sw64(tile, r, v);
             tmem_st_32x32(ta, v);
+            tc_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+              mbar_arrive(&afull[a]);
+              mbar_arrive(&w8empty[j]);
+            }
           }
-          tc_wait_st();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) {
-            mbar_arrive(&afull[a]);
-            mbar_arrive(&w8empty[j]);
-          }
+          par ^= 1;
           if (++a == Cfg::STAGES_A) { a = 0; pha ^= 1; }
           if (++j == Cfg::S8) { j = 0; jph ^= 1; }
         }
@@ -899,8 +989,8 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       const size_t slice_off = (size_t)ks * (size_t)p.epi.slice;
       int g, row0, rows;
       locate_row_tile_s(p, s_tiles, rt, g, row0, rows);
-      const int ab = it & 1;
-      const uint32_t aph = (it >> 1) & 1;
+      const int ab = Cfg::ACC_BUFS == 2 ? (it & 1) : 0;
+      const uint32_t aph = Cfg::ACC_BUFS == 2 ? (uint32_t)(it >> 1) & 1 : (uint32_t)it & 1;
       if (!mbar_wait(&tfull[ab], aph, abort_flag, p.err)) break;
       tc_fence_after();
       const uint32_t tb = tmem_base + ((uint32_t)(qd * 32) << 16) + ab * Cfg::ACC_COLS;
@@ -937,7 +1027,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         const int f = f0 + qd * 32 + lane;
         const int fl = qd * 32 + lane;  // this thread's feature within the tile
         float s0 = 1.f, s1 = 1.f;  // fp8 weights: this thread's output channel scales
-        if (Cfg::kFp8 && f < p.F) {
+        if (Cfg::kFp8 && p.w_scale && f < p.F) {
           const float* sc = p.w_scale + (size_t)g * p.w_group_stride + f;
           s0 = __ldg(sc);
           if (Cfg::kDual) s1 = __ldg(sc + p.dual_offset);

@@ -29,6 +29,7 @@ NO_PDL = 0x800
 LOAD_SPLIT = 0x1000
 NO_STREAM_K = 0x2000
 SORTED_ROWS = 0x4000
+EXPERTS_FP4 = 0x8000
 MAX_EXPERTS, MAX_TOPK = 1024, 32
 DEVERR_WAIT_TIMEOUT, DEVERR_RANGE, DEVERR_NONFINITE = 0x1, 0x2, 0x4
 STAGES = {"logits": 0, "idx": 1, "w": 2, "offsets": 3, "perm": 4, "z": 5, "h": 6, "ys": 7, "comb": 8}
@@ -37,7 +38,8 @@ EXPORTS = ["lmoe_create", "lmoe_set_weights", "lmoe_reserve", "lmoe_forward", "l
            "lmoe_last_error", "lmoe_profile_begin", "lmoe_profile_end", "lmoe_stage_name",
            "lmoe_last_launch_count", "lmoe_last_expert_path", "lmoe_status_string",
            "lmoe_error_detail", "lmoe_destroy", "lmoe_route_only_noalloc",
-           "lmoe_set_expert_weights_fp8", "lmoe_selftest_wait_timeout",
+           "lmoe_set_expert_weights_fp8", "lmoe_set_expert_weights_fp4",
+           "lmoe_selftest_wait_timeout",
            "lmoe_profile_begin_stages"]
 NOALLOC_MAX_WORDS = 262144
 
@@ -66,6 +68,7 @@ def lib() -> ctypes.CDLL:
             "lmoe_create": ([I, I, I, I, I, I, I, I, U, ctypes.POINTER(P)], I),
             "lmoe_set_weights": ([P] * 9, I),
             "lmoe_set_expert_weights_fp8": ([P] * 5, I),
+            "lmoe_set_expert_weights_fp4": ([P] * 5, I),
             "lmoe_selftest_wait_timeout": ([P, U, P], I),
             "lmoe_reserve": ([P, I], I),
             "lmoe_forward": ([P, P, P, I, P], I),
@@ -244,6 +247,19 @@ class LatentMoELayer:
               self._dev(W2s, (N, l), torch.float32, "W2s")]
         self._check(lib().lmoe_set_expert_weights_fp8(self._h, *[_ptr(t) for t in ts]),
                     "lmoe_set_expert_weights_fp8")
+
+    def set_expert_weights_fp4(self, W1q, W1e, W2q, W2e):
+        """MXFP4 expert weights (layer created with EXPERTS_FP4), output-major
+        uint8: code pairs W1q [N, m_in, l / 2], W2q [N, l, m / 2] (low nibble =
+        even input channel) and E8M0 block exponents W1e [N, m_in, l / 32],
+        W2e [N, l, m / 32]."""
+        N, l, m, mi = self.N, self.l, self.m, self.m_in
+        ts = [self._dev(W1q, (N, mi, l // 2), torch.uint8, "W1q"),
+              self._dev(W1e, (N, mi, l // 32), torch.uint8, "W1e"),
+              self._dev(W2q, (N, l, m // 2), torch.uint8, "W2q"),
+              self._dev(W2e, (N, l, m // 32), torch.uint8, "W2e")]
+        self._check(lib().lmoe_set_expert_weights_fp4(self._h, *[_ptr(t) for t in ts]),
+                    "lmoe_set_expert_weights_fp4")
 
     def selftest_wait_timeout(self, limit_us: int, stream=None):
         """Test hook: a device wait that nothing completes gives up after

@@ -59,10 +59,16 @@ class Workload:
     bias: Optional[str] = None   # None, "normal0.5" or "zipf1.1"
     seed: int = 0
     expert_fp8: bool = False     # expert weights as E4M3 codes + per-channel scales
+    expert_fp4: bool = False     # expert weights as MXFP4 (E2M1 codes + block exponents)
 
     @property
     def m_in(self) -> int:
         return 2 * self.m if self.act == "swiglu" else self.m
+
+    @property
+    def expert_format(self) -> Optional[str]:
+        """The expert weights' low-precision format (costmodel.EXPERT_FORMATS)."""
+        return "e4m3" if self.expert_fp8 else "mxfp4" if self.expert_fp4 else None
 
     @property
     def ms_in(self) -> int:
@@ -102,6 +108,33 @@ WORKLOADS["std-moe-decode-fp8"] = replace(WORKLOADS["std-moe-decode"], name="std
                                           expert_fp8=True)
 WORKLOADS["latent-decode-fp8"] = replace(WORKLOADS["latent-decode"], name="latent-decode-fp8",
                                          expert_fp8=True)
+# ... and with block-scaled FP4 expert weights (the precision of the paper's
+# GB200 roofline analysis)
+WORKLOADS["std-moe-decode-fp4"] = replace(WORKLOADS["std-moe-decode"], name="std-moe-decode-fp4",
+                                          expert_fp4=True)
+WORKLOADS["latent-decode-fp4"] = replace(WORKLOADS["latent-decode"], name="latent-decode-fp4",
+                                         expert_fp4=True)
+# The paper's two LatentMoE variants against the standard MoE they derive from
+# (LatentMoE, Section 3, Eq. (1) and Eq. (2); Table 1): the standard layer
+# (d = 4096, N = 128 experts, top-8, m = 1536, no projections), l-MoE_eff
+# (latent l = d / 4, N' = 4 N, k' = k) and l-MoE_acc (l = d / 4, N' = 4 N,
+# k' = 4 k), on the same kernels, at a decode and a prefill batch.  No router
+# bias, so all three see the same routing statistics.  The standard decode
+# point is std-moe-decode itself.
+_SWEEP = dict(d=4096, m=1536, act="swiglu")
+WORKLOADS["l-moe-eff-decode"] = Workload("l-moe-eff-decode", T=256, l=1024, N=512, k=8,
+                                         seed=11, **_SWEEP)
+WORKLOADS["l-moe-acc-decode"] = Workload("l-moe-acc-decode", T=256, l=1024, N=512, k=32,
+                                         seed=12, **_SWEEP)
+WORKLOADS["std-moe-prefill"] = Workload("std-moe-prefill", T=4096, l=4096, N=128, k=8,
+                                        skip_proj=True, seed=13, **_SWEEP)
+WORKLOADS["l-moe-eff-prefill"] = Workload("l-moe-eff-prefill", T=4096, l=1024, N=512, k=8,
+                                          seed=14, **_SWEEP)
+WORKLOADS["l-moe-acc-prefill"] = Workload("l-moe-acc-prefill", T=4096, l=1024, N=512, k=32,
+                                          seed=15, **_SWEEP)
+# (variant, standard point, l-MoE_eff point, l-MoE_acc point) per batch size
+VARIANT_SWEEP = (("decode", "std-moe-decode", "l-moe-eff-decode", "l-moe-acc-decode"),
+                 ("prefill", "std-moe-prefill", "l-moe-eff-prefill", "l-moe-acc-prefill"))
 WORKLOAD_ORDER = list(WORKLOADS)
 
 
@@ -117,6 +150,42 @@ def quantize_e4m3(W: torch.Tensor):
     scale = torch.where(amax > 0, amax / 448.0, torch.ones_like(amax))
     codes = (Wf / scale.unsqueeze(-2)).to(torch.float8_e4m3fn).view(torch.uint8)
     return codes.contiguous(), scale.contiguous()
+
+# MXFP4: the eight magnitudes of an E2M1 code, and the midpoints between
+# neighbours (a value on a midpoint goes to the neighbour whose code is even,
+# i.e. whose mantissa bit is 0)
+_E2M1_MIDPOINTS = (0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0)
+
+
+def quantize_mxfp4(W: torch.Tensor):
+    """Block-scaled FP4 (OCP MX: E2M1 elements, one E8M0 scale per 32
+    elements) of a weight stack in the API layout [..., in, out], blocks of
+    32 consecutive inputs of each output column.  Per block: scale exponent
+    e = floor(log2(amax)) - 2 (2 = the largest E2M1 exponent; e = -23 for an
+    all-zero block), clamped to [-23, 13] so that every scaled code is an f16
+    value; elements round to nearest on the E2M1 grid, ties to the even code,
+    saturating at 6.  Returns (codes uint8 [..., out, in / 2], element 2j in
+    the low nibble of byte j; exponents uint8 [..., out, in / 32] = e + 127),
+    output-major as the kernels read them.  Inputs for the fp4 expert
+    weights: the library and the oracle both read these codes."""
+    Wt = W.float().transpose(-1, -2)
+    *lead, O, I = Wt.shape
+    if I % 32:
+        raise ValueError("the input width must be a multiple of 32")
+    blk = Wt.reshape(*lead, O, I // 32, 32)
+    amax = blk.abs().amax(dim=-1)
+    e = torch.where(amax > 0, torch.floor(torch.log2(amax)) - 2, torch.full_like(amax, -23.0))
+    e = e.clamp(-23.0, 13.0)
+    v = blk / torch.exp2(e).unsqueeze(-1)
+    a = v.abs()
+    mids = torch.tensor(_E2M1_MIDPOINTS, dtype=torch.float32, device=W.device)
+    idx = torch.searchsorted(mids, a.contiguous(), right=False)  # midpoints strictly below a
+    tie = (idx < 7) & (a == mids[idx.clamp(max=6)])
+    idx = torch.where(tie & (idx % 2 == 1), idx + 1, idx)
+    code = (idx | torch.where(v < 0, 8, 0)).to(torch.uint8).reshape(*lead, O, I)
+    packed = (code[..., 0::2] | (code[..., 1::2] << 4)).contiguous()
+    return packed, (e + 127).to(torch.uint8).contiguous()
+
 
 _TID = {"x": 1, "Wg": 2, "bias": 3, "Wdown": 4, "Wup": 5, "W1": 6, "W2": 7,
         "Ws1": 8, "Ws2": 9}
@@ -186,7 +255,18 @@ def make_weights(w: Workload, device="cpu", experts: bool = True) -> Dict[str, O
                                _TID["Wdown"], 0, device, dt)
         out["Wup"] = _normal((w.l, w.d), 1.0 / math.sqrt(w.l), w.seed,
                              _TID["Wup"], 0, device, dt)
-    if experts and w.expert_fp8:
+    if experts and w.expert_fp4:
+        # the same bf16 draws, as MXFP4 per expert, output-major: W1q [N, m_in,
+        # l / 2] and W1e [N, m_in, l / 32], W2q [N, l, m / 2] and W2e [N, l, m / 32]
+        W1q = torch.empty((w.N, w.m_in, w.l // 2), dtype=torch.uint8, device=device)
+        W2q = torch.empty((w.N, w.l, w.m // 2), dtype=torch.uint8, device=device)
+        W1e = torch.empty((w.N, w.m_in, w.l // 32), dtype=torch.uint8, device=device)
+        W2e = torch.empty((w.N, w.l, w.m // 32), dtype=torch.uint8, device=device)
+        for e in range(w.N):
+            W1q[e], W1e[e] = quantize_mxfp4(make_expert_W1(w, e, device))
+            W2q[e], W2e[e] = quantize_mxfp4(make_expert_W2(w, e, device))
+        out.update(W1=None, W2=None, W1q=W1q, W1e=W1e, W2q=W2q, W2e=W2e)
+    elif experts and w.expert_fp8:
         # the same bf16 draws, quantised per expert (W1q/W2q codes, W1s/W2s
         # scales); W1/W2 stay None
         W1q = torch.empty((w.N, w.l, w.m_in), dtype=torch.uint8, device=device)

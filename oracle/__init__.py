@@ -36,7 +36,8 @@ class _Layer(ctypes.Structure):
                 ("W1", ctypes.c_void_p), ("W2", ctypes.c_void_p),
                 ("Ws1", ctypes.c_void_p), ("Ws2", ctypes.c_void_p),
                 ("route_mode", ctypes.c_int),
-                ("expert_fp8", ctypes.c_int), ("W1s", ctypes.c_void_p), ("W2s", ctypes.c_void_p)]
+                ("expert_fp8", ctypes.c_int), ("W1s", ctypes.c_void_p), ("W2s", ctypes.c_void_p),
+                ("expert_fp4", ctypes.c_int), ("W1e", ctypes.c_void_p), ("W2e", ctypes.c_void_p)]
 
 # routing variants (bits of route_mode)
 ROUTE_FULL_SOFTMAX, ROUTE_BIAS_SELECT = 1, 2
@@ -65,6 +66,8 @@ def lib():
         L.oracle_hardware_threads.argtypes = []
         L.oracle_e4m3_value.argtypes = [I]
         L.oracle_e4m3_value.restype = ctypes.c_double
+        L.oracle_e2m1_value.argtypes = [I]
+        L.oracle_e2m1_value.restype = ctypes.c_double
         _lib = L
     return _lib
 
@@ -104,12 +107,16 @@ class OracleLayer:
     expert -> matrix holding only the experts that will be reached.  With
     ``W1s``/``W2s`` (per-expert fp32 scales per output column, ``[N, m_in]``
     and ``[N, l]``, stacks or mappings) ``W1``/``W2`` are fp8 E4M3 codes
-    (uint8) in the same layouts.
+    (uint8) in the same layouts.  With ``W1e``/``W2e`` (per-expert E8M0
+    block exponents, ``[N, m_in, l / 32]`` and ``[N, l, m / 32]``)
+    ``W1``/``W2`` are MXFP4 E2M1 code pairs stored output-major,
+    ``[N, m_in, l / 2]`` and ``[N, l, m / 2]`` (uint8).
     """
 
     def __init__(self, *, d, l, N, k, m, act, shared_m=0, dtype="bf16",
                  skip_proj=False, Wg, bias=None, Wdown=None, Wup=None,
-                 W1, W2, Ws1=None, Ws2=None, route_mode=0, W1s=None, W2s=None):
+                 W1, W2, Ws1=None, Ws2=None, route_mode=0, W1s=None, W2s=None,
+                 W1e=None, W2e=None):
         self.d, self.l, self.N, self.k, self.m = d, l, N, k, m
         self.act, self.shared_m, self.dtype, self.skip_proj = act, shared_m, dtype, skip_proj
         keep = []
@@ -129,6 +136,9 @@ class OracleLayer:
         fp8 = W1s is not None or W2s is not None
         if fp8 and (W1s is None or W2s is None):
             raise OracleError("fp8 expert weights need both W1s and W2s")
+        fp4 = W1e is not None or W2e is not None
+        if fp4 and (W1e is None or W2e is None or fp8):
+            raise OracleError("fp4 expert weights need both W1e and W2e (and no fp8 scales)")
 
         def arr8(t):  # E4M3 codes, or fp32 scales
             if t is None:
@@ -138,30 +148,38 @@ class OracleLayer:
             keep.append(a)
             return a
 
-        warr = arr8 if fp8 else arr
+        warr = arr8 if (fp8 or fp4) else arr
         p1 = (ctypes.c_void_p * N)()
         p2 = (ctypes.c_void_p * N)()
         s1 = (ctypes.c_void_p * N)()
         s2 = (ctypes.c_void_p * N)()
+        e1 = (ctypes.c_void_p * N)()
+        e2 = (ctypes.c_void_p * N)()
         for e in range(N):
             a1 = self._expert(W1, e, warr)
             a2 = self._expert(W2, e, warr)
-            if fp8 and ((a1 is not None and a1.dtype != np.uint8) or
-                        (a2 is not None and a2.dtype != np.uint8)):
-                raise OracleError("fp8 expert weights must be uint8 E4M3 codes")
+            if (fp8 or fp4) and ((a1 is not None and a1.dtype != np.uint8) or
+                                 (a2 is not None and a2.dtype != np.uint8)):
+                raise OracleError("fp8 / fp4 expert weights must be uint8 codes")
             p1[e] = _ptr(a1)
             p2[e] = _ptr(a2)
             if fp8:
                 s1[e] = _ptr(self._expert(W1s, e, arr8))
                 s2[e] = _ptr(self._expert(W2s, e, arr8))
+            if fp4:
+                e1[e] = _ptr(self._expert(W1e, e, arr8))
+                e2[e] = _ptr(self._expert(W2e, e, arr8))
         self._p1, self._p2, self._s1, self._s2, self._keep = p1, p2, s1, s2, keep
+        self._e1, self._e2 = e1, e2
         self.struct = _Layer(d, l, N, k, m, ACT_CODES[act], shared_m, DTYPE_CODES[dtype],
                              int(bool(skip_proj)), _ptr(self._Wg), _ptr(self._bias),
                              _ptr(self._Wdown), _ptr(self._Wup),
                              ctypes.cast(p1, ctypes.c_void_p), ctypes.cast(p2, ctypes.c_void_p),
                              _ptr(self._Ws1), _ptr(self._Ws2), int(route_mode),
                              int(fp8), ctypes.cast(s1, ctypes.c_void_p),
-                             ctypes.cast(s2, ctypes.c_void_p))
+                             ctypes.cast(s2, ctypes.c_void_p),
+                             int(fp4), ctypes.cast(e1, ctypes.c_void_p),
+                             ctypes.cast(e2, ctypes.c_void_p))
 
     @staticmethod
     def _expert(W, e, arr):
@@ -248,6 +266,11 @@ def route(logits32, k: int, nthreads: Optional[int] = None, sel_bias=None,
 def e4m3_value(code: int) -> float:
     """The exact value of one fp8 E4M3 code, as the oracle reads it."""
     return float(lib().oracle_e4m3_value(int(code)))
+
+
+def e2m1_value(code: int) -> float:
+    """The exact value of one fp4 E2M1 code, as the oracle reads it."""
+    return float(lib().oracle_e2m1_value(int(code)))
 
 
 def hardware_threads() -> int:

@@ -40,7 +40,11 @@
 // may instead be fp8 E4M3 codes with one fp32 scale per output column (low-
 // precision expert weights: the paper's Section 2 models FP4 weights, its
 // Section 4.3 measures FP8 quantisation): the oracle widens each code to the
-// exact value it denotes and multiplies by its column's scale.
+// exact value it denotes and multiplies by its column's scale.  Or they may
+// be block-scaled FP4 (MXFP4: E2M1 codes, two per byte, with one power-of-two
+// scale per 32 consecutive input elements of each output column), stored
+// output-major: the oracle decodes each code and multiplies by its block's
+// power of two.
 #include <algorithm>
 #include <atomic>
 #include <cmath>
@@ -73,6 +77,24 @@ inline double e4m3_value(uint8_t c) {
   else if (E == 0) v = std::ldexp((double)m, -9);           // m/8 * 2^-6
   else v = std::ldexp(8.0 + m, E - 10);                    // (1 + m/8) * 2^(E-7)
   return sgn ? -v : v;
+}
+
+// One fp4 E2M1 code (the OCP microscaling element format: 1 sign, 2 exponent
+// bits with bias 1, 1 mantissa bit; exponent field 0 is subnormal; no
+// infinities or NaN; largest 6) as the exact double it denotes.
+inline double e2m1_value(int c) {
+  const int sgn = (c >> 3) & 1, E = (c >> 1) & 3, m = c & 1;
+  const double v = E == 0 ? 0.5 * m : std::ldexp(1.0 + 0.5 * m, E - 1);
+  return sgn ? -v : v;
+}
+
+// W[i][o] of an MXFP4 matrix with K inputs, stored output-major: codes
+// q[o][i / 2] (element i in the low nibble when i is even), block exponents
+// e[o][i / 32] (E8M0: the scale is 2^(e - 127)).
+inline double mxfp4_value(const uint8_t* q, const uint8_t* e, int K, int o, int i) {
+  const uint8_t b = q[(size_t)o * (K / 2) + i / 2];
+  const int code = (i & 1) ? (b >> 4) : (b & 15);
+  return std::ldexp(e2m1_value(code), (int)e[(size_t)o * (K / 32) + i / 32] - 127);
 }
 
 inline double widen(const void* p, int dtype, size_t i) {
@@ -122,14 +144,18 @@ void apply_act(int act, const double* a, int m, double* h) {
 // acc[p][o] = sum_i in[p][i] * W[i][o] for p in [0, P), sequential in i.
 // in: P rows of width K (double); W: [K, O] in dtype; acc: P rows of width O.
 // col_scale (fp8 weights): W[i][o] stands for code(i, o) * col_scale[o].
+// blk_exp (MXFP4 weights, W holding the output-major codes): W[i][o] stands
+// for mxfp4_value(W, blk_exp, K, o, i).
 void rows_times_matrix(const double* in, int P, int K, const void* W, int dtype,
                        int O, double* acc, std::vector<double>& wrow,
-                       const float* col_scale = nullptr) {
+                       const float* col_scale = nullptr, const uint8_t* blk_exp = nullptr) {
   std::fill(acc, acc + (size_t)P * O, 0.0);
   wrow.resize(O);
   for (int i = 0; i < K; ++i) {
     for (int o = 0; o < O; ++o)
-      wrow[o] = widen(W, dtype, (size_t)i * O + o) * (col_scale ? (double)col_scale[o] : 1.0);
+      wrow[o] = blk_exp ? mxfp4_value(static_cast<const uint8_t*>(W), blk_exp, K, o, i)
+                        : widen(W, dtype, (size_t)i * O + o) *
+                              (col_scale ? (double)col_scale[o] : 1.0);
     for (int p = 0; p < P; ++p) {
       const double zi = in[(size_t)p * K + i];
       double* a = acc + (size_t)p * O;
@@ -158,6 +184,12 @@ struct OracleLayer {
   int expert_fp8;
   const float* const* W1s;
   const float* const* W2s;
+  // MXFP4 expert weights: W1[e] [m_in, l / 2] and W2[e] [l, m / 2] hold
+  // E2M1 code pairs output-major, W1e[e] [m_in, l / 32] and W2e[e]
+  // [l, m / 32] one E8M0 block exponent per 32 inputs of each output column.
+  int expert_fp4;
+  const uint8_t* const* W1e;
+  const uint8_t* const* W2e;
 };
 
 static int m_in_of(int act, int m) { return act == OR_ACT_SWIGLU ? 2 * m : m; }
@@ -293,7 +325,9 @@ int oracle_forward(const OracleLayer* L, const void* x, const int* tokens, int S
     if (e < 0 || e >= N) return OR_ERR_ARG;
     if (!L->W1[e] || !L->W2[e]) return OR_ERR_MISSING;
     if (L->expert_fp8 && (!L->W1s || !L->W2s || !L->W1s[e] || !L->W2s[e])) return OR_ERR_MISSING;
+    if (L->expert_fp4 && (!L->W1e || !L->W2e || !L->W1e[e] || !L->W2e[e])) return OR_ERR_MISSING;
   }
+  if (L->expert_fp4 && (l % 32 != 0 || m % 32 != 0)) return OR_ERR_ARG;
   const int edt = L->expert_fp8 ? OR_E4M3 : dt;  // the expert weights' element type
 
   // x rows in float64.
@@ -331,10 +365,12 @@ int oracle_forward(const OracleLayer* L, const void* x, const int* tokens, int S
       std::memcpy(&zin[(size_t)p * l], &Z[(size_t)s * l], l * sizeof(double));
     }
     rows_times_matrix(zin.data(), P, l, L->W1[e], edt, m_in, a.data(), wrow,
-                      L->expert_fp8 ? L->W1s[e] : nullptr);
+                      L->expert_fp8 ? L->W1s[e] : nullptr,
+                      L->expert_fp4 ? L->W1e[e] : nullptr);
     for (int p = 0; p < P; ++p) apply_act(L->act, &a[(size_t)p * m_in], m, &h[(size_t)p * m]);
     rows_times_matrix(h.data(), P, m, L->W2[e], edt, l, y.data(), wrow,
-                      L->expert_fp8 ? L->W2s[e] : nullptr);
+                      L->expert_fp8 ? L->W2s[e] : nullptr,
+                      L->expert_fp4 ? L->W2e[e] : nullptr);
     for (int p = 0; p < P; ++p)
       std::memcpy(&Y[(size_t)pairs[e][q0 + p] * l], &y[(size_t)p * l], l * sizeof(double));
   });
@@ -398,5 +434,8 @@ int oracle_hardware_threads(void) { return (int)std::thread::hardware_concurrenc
 
 // The value an fp8 E4M3 code denotes (exposed for its pin).
 double oracle_e4m3_value(int code) { return e4m3_value((uint8_t)code); }
+
+// The value an fp4 E2M1 code denotes (exposed for its pin).
+double oracle_e2m1_value(int code) { return e2m1_value(code & 15); }
 
 }  // extern "C"

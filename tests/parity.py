@@ -31,13 +31,15 @@ F32_REL_L2 = 1e-5                       # stated tolerance for the fp32 layer
 def gpu_layer(w: workloads.Workload, flags: int = 0, W: Optional[Dict] = None):
     if W is None:
         W = workloads.make_weights(w, device="cuda")
-    fp8 = bool(w.expert_fp8)
+    fp8, fp4 = bool(w.expert_fp8), bool(w.expert_fp4)
+    flags |= (lmoe.EXPERTS_FP8 if fp8 else 0) | (lmoe.EXPERTS_FP4 if fp4 else 0)
     L = lmoe.LatentMoELayer(w.d, w.l, w.N, w.k, w.m, act=w.act, shared_m=w.shared_m,
-                            dtype=w.dtype, flags=flags | (lmoe.EXPERTS_FP8 if fp8 else 0),
-                            skip_proj=w.skip_proj)
+                            dtype=w.dtype, flags=flags, skip_proj=w.skip_proj)
     L.set_weights(W["Wg"], W["bias"], W["Wdown"], W["Wup"], W["W1"], W["W2"], W["Ws1"], W["Ws2"])
     if fp8:
         L.set_expert_weights_fp8(W["W1q"], W["W1s"], W["W2q"], W["W2s"])
+    if fp4:
+        L.set_expert_weights_fp4(W["W1q"], W["W1e"], W["W2q"], W["W2e"])
     L.reserve(w.T)
     return L, W
 
@@ -54,20 +56,18 @@ def route_mode(flags: int) -> int:
 
 def oracle_layer(w: workloads.Workload, W: Dict, experts: Optional[Iterable[int]] = None,
                  mode: int = 0):
-    fp8 = bool(w.expert_fp8)
-    k1, k2 = ("W1q", "W2q") if fp8 else ("W1", "W2")
+    fp8, fp4 = bool(w.expert_fp8), bool(w.expert_fp4)
+    k1, k2 = ("W1q", "W2q") if (fp8 or fp4) else ("W1", "W2")
+    ks = ("W1s", "W2s") if fp8 else ("W1e", "W2e") if fp4 else ()
     extra = {}
     if experts is None:
         W1, W2 = _cpu(W[k1]), _cpu(W[k2])
-        if fp8:
-            extra = dict(W1s=_cpu(W["W1s"]), W2s=_cpu(W["W2s"]))
+        extra = {k: _cpu(W[k]) for k in ks}
     else:
         ex = sorted(set(int(e) for e in experts))
         W1 = {e: _cpu(W[k1][e]) for e in ex}
         W2 = {e: _cpu(W[k2][e]) for e in ex}
-        if fp8:
-            extra = dict(W1s={e: _cpu(W["W1s"][e]) for e in ex},
-                         W2s={e: _cpu(W["W2s"][e]) for e in ex})
+        extra = {k: {e: _cpu(W[k][e]) for e in ex} for k in ks}
     return oracle.OracleLayer(**extra, d=w.d, l=w.l, N=w.N, k=w.k, m=w.m, act=w.act,
                               shared_m=w.shared_m, dtype=w.dtype, skip_proj=w.skip_proj,
                               Wg=_cpu(W["Wg"]), bias=_cpu(W["bias"]), Wdown=_cpu(W["Wdown"]),

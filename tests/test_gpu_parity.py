@@ -491,6 +491,100 @@ def test_fp8_expert_api_errors():
         plain.set_expert_weights_fp8(W["W1q"], W["W1s"], W["W2q"], W["W2s"])
 
 
+FP4 = {
+    "swiglu": W_("f4-swiglu", T=300, d=256, l=512, N=8, k=3, m=512, act="swiglu", seed=51,
+                 expert_fp4=True),
+    "relu2-shared": W_("f4-relu2", T=200, d=512, l=512, N=6, k=2, m=1024, act="relu2",
+                       shared_m=256, bias="normal0.5", seed=52, expert_fp4=True),
+    "silu-skip": W_("f4-silu-skip", T=90, d=512, l=512, N=12, k=4, m=512, act="silu",
+                    skip_proj=True, seed=53, expert_fp4=True),
+    # decode-like: 64 experts x 8 weight tiles of FC1, 2 to 16 tiles per CTA
+    # (stream-K), K = 1024 (exponent boxes at two offsets)
+    "decode-like": W_("f4-decode", T=64, d=1024, l=1024, N=64, k=8, m=512, act="swiglu",
+                      bias="normal0.5", seed=54, expert_fp4=True),
+}
+
+
+@pytest.mark.parametrize("name", list(FP4))
+def test_fp4_experts(name):
+    """MXFP4 expert weights (E2M1 codes, one power-of-two scale per 32
+    inputs) widened in tensor memory on the weight-stationary kernels,
+    against the oracle on the same codes and exponents."""
+    res = check_forward(FP4[name], fixture=True)
+    assert res["unique"] >= 0.9 * res["tokens"]
+    assert paths(res) == (2, 2)
+
+
+def test_fp4_experts_prefill_sized():
+    """fp4 weights at prefill size (the weight-stationary kernels tile up to
+    64 rows of an expert at a time: several row tiles per expert)."""
+    w = W_("f4-prefill", T=1024, d=512, l=512, N=16, k=4, m=512, act="swiglu",
+           shared_m=512, seed=55, expert_fp4=True)
+    res = check_forward(w, tokens=sample_tokens(w.T, 160, seed=5))
+    assert paths(res) == (2, 2)
+    assert res["unique"] >= 0.8 * res["tokens"]
+
+
+@pytest.mark.parametrize("low", [True, False])
+def test_fp4_extreme_block_exponents(low):
+    """FC2 blocks at one end of the accepted exponent range: scales 2^-23 ..
+    2^-21 (codes x scale are f16 subnormals) or 2^11 .. 2^13 (up to 6 x 2^13
+    = 49152), and all-zero blocks in both matrices.  The combined rows are
+    compared relatively (rel-L2 of the comb stage), so a widening that
+    flushed or clipped these values fails even where the residual hides them
+    in the output.  FC1 keeps its quantised exponents: its output is stored
+    in f16, so scales that overflow f16 there are outside the layer's range
+    whatever the widening does."""
+    w = W_("f4-extreme", T=200, d=512, l=512, N=8, k=2, m=512, act="silu", seed=56,
+           expert_fp4=True)
+    W = workloads.make_weights(w, device="cuda")
+    g = torch.Generator(device="cpu").manual_seed(7)
+    base = 127 - 23 if low else 127 + 11
+    W["W2e"] = (base + torch.randint(0, 3, W["W2e"].shape, generator=g)).to(torch.uint8).cuda()
+    for key in ("W1q", "W2q"):  # all-zero blocks: 32 codes = 16 bytes of a row
+        q = W[key].cpu()
+        q[:, :3, 16:32] = 0
+        W[key] = q.to("cuda")
+    res = check_forward(w, W=W, fixture=True)
+    assert res["unique"] >= 0.9 * res["tokens"]
+    assert "comb_rel_l2" in res
+
+
+def test_fp4_expert_api_errors():
+    w = FP4["swiglu"]
+    for kw in (dict(dtype="f32"), dict(l=384), dict(m=256)):  # bf16, l and m multiples of 512
+        a = dict(d=w.d, l=w.l, m=w.m, dtype="bf16")
+        a.update(kw)
+        with pytest.raises(lmoe.LmoeError):
+            lmoe.LatentMoELayer(a["d"], a["l"], w.N, w.k, a["m"], act=w.act, dtype=a["dtype"],
+                                flags=lmoe.EXPERTS_FP4)
+    with pytest.raises(lmoe.LmoeError):  # not with fp8
+        lmoe.LatentMoELayer(w.d, w.l, w.N, w.k, w.m, act=w.act, dtype="bf16",
+                            flags=lmoe.EXPERTS_FP4 | lmoe.EXPERTS_FP8)
+    W = workloads.make_weights(w, device="cuda")
+    L = lmoe.LatentMoELayer(w.d, w.l, w.N, w.k, w.m, act=w.act, dtype="bf16",
+                            flags=lmoe.EXPERTS_FP4)
+    L.set_weights(W["Wg"], W["bias"], W["Wdown"], W["Wup"], None, None, None, None)
+    L.reserve(w.T)
+    x = workloads.make_x(w, device="cuda")
+    with pytest.raises(lmoe.LmoeError):  # not ready before the fp4 experts are set
+        L.forward(x)
+    bad = W["W1e"].clone()
+    bad[0, 0, 0] = 127 + 14  # a scale of 2^14: 6 x 2^14 is no f16 value
+    with pytest.raises(lmoe.LmoeError):
+        L.set_expert_weights_fp4(W["W1q"], bad, W["W2q"], W["W2e"])
+    L.set_expert_weights_fp4(W["W1q"], W["W1e"], W["W2q"], W["W2e"])
+    L.forward(x)
+    torch.cuda.synchronize()
+    assert L.last_error() == (lmoe.OK, 0)
+    L.ep_reserve(w.T * w.k)
+    with pytest.raises(lmoe.LmoeError):  # no expert parallelism for fp4 layers
+        L.ep_dispatch(x)
+    plain = lmoe.LatentMoELayer(w.d, w.l, w.N, w.k, w.m, act=w.act, dtype="bf16")
+    with pytest.raises(lmoe.LmoeError):  # the layer was not created for fp4 experts
+        plain.set_expert_weights_fp4(W["W1q"], W["W1e"], W["W2q"], W["W2e"])
+
+
 def test_tcgen05_path_is_taken_for_bf16():
     res = check_forward(SMALL["swiglu"], fixture=True)
     assert paths(res)[0] in (1, 2, 4, 5)
@@ -621,7 +715,10 @@ def test_device_error_word_clean_and_profile():
 
 FULL_SAMPLES = {"tiny-fp32": 64, "std-moe-decode": 96, "latent-decode": 96,
                 "latent-prefill-shared": 64, "latent-prefill-skewed": 48,
-                "std-moe-decode-fp8": 96, "latent-decode-fp8": 96}
+                "std-moe-decode-fp8": 96, "latent-decode-fp8": 96,
+                "std-moe-decode-fp4": 96, "latent-decode-fp4": 96,
+                "l-moe-eff-decode": 64, "l-moe-acc-decode": 64, "std-moe-prefill": 48,
+                "l-moe-eff-prefill": 48, "l-moe-acc-prefill": 48}
 
 
 def edge_tokens_of_largest_experts(L, T: int, n_experts: int = 2, per_end: int = 3):

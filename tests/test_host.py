@@ -24,8 +24,8 @@ def test_binding_flags_and_limits_match_the_header():
              if k in ("SKIP_PROJ", "DEBUG_CHECKS", "FORCE_SIMT", "FORCE_SWAP", "FORCE_NOSWAP",
                       "FORCE_NOPAIR", "FORCE_WS_PAIR", "ROUTE_FULL_SOFTMAX", "ROUTE_BIAS_SELECT",
                       "EXPERTS_FP8", "SINGLE_STREAM", "NO_PDL", "LOAD_SPLIT",
-                      "NO_STREAM_K", "SORTED_ROWS")}
-    assert len(flags) == 15, sorted(flags)
+                      "NO_STREAM_K", "SORTED_ROWS", "EXPERTS_FP4")}
+    assert len(flags) == 16, sorted(flags)
     for name, value in flags.items():
         assert getattr(lmoe, name) == value, name
     # flags are distinct single bits
@@ -59,3 +59,33 @@ def test_recorded_traffic_is_used_only_on_the_captured_sources(monkeypatch):
         monkeypatch.setattr(bench, "kernel_source_hash", lambda stage: "0" * 16)
         assert bench.recorded_traffic(wl, st) is None
     assert bench.recorded_traffic("no-such-workload", "expert_fc1") is None
+
+
+def test_variant_sweep_costs_follow_the_paper():
+    """The sweep's cost columns for the paper's variants (LatentMoE, Section 3,
+    Table 1): per token, l-MoE_eff activates 1/alpha of the standard layer's
+    expert weight bytes and dispatches 1/alpha of its bytes at 1/alpha of its
+    expert FLOPs; l-MoE_acc matches the standard layer in all three."""
+    import bench
+    from mixture_experts_layer_64_b200 import workloads
+
+    for batch, *names in workloads.VARIANT_SWEEP:
+        pts = []
+        for variant, name in zip(("standard", "l-MoE_eff", "l-MoE_acc"), names):
+            w = workloads.WORKLOADS[name]
+            r = {"w": w, "expert_loads": {"touched": w.N}, "value": 1.0, "ms_per_step": 1.0,
+                 "stage_ms": {"expert_fc1": {"p50": 0.5}, "expert_fc2": {"p50": 0.25}}}
+            pts.append(bench.sweep_point(variant, r))
+        out = bench.variant_sweep(pts)["points"]
+        alpha = out[0]["d"] / out[1]["l"]
+        assert alpha == 4
+        for key in ("active_weight_bytes_per_token", "dispatch_bytes_per_token",
+                    "expert_flops_per_token"):
+            assert out[0]["vs_standard"][key] == 1.0
+            assert out[1]["vs_standard"][key] == 1 / alpha, (batch, key)
+            assert out[2]["vs_standard"][key] == 1.0, (batch, key)
+        # every expert touched: all three load the same expert set (alpha N
+        # experts of 1 / alpha the size)
+        assert [p["vs_standard"]["expert_weight_bytes"] for p in out] == [1.0, 1.0, 1.0]
+        assert out[1]["N"] == out[2]["N"] == alpha * out[0]["N"]
+        assert out[2]["k"] == alpha * out[1]["k"] == alpha * out[0]["k"]

@@ -498,3 +498,104 @@ def test_fp8_layer_equals_layer_with_dequantised_weights():
     np.testing.assert_allclose(a["out"], b["out"], rtol=1e-6, atol=1e-6)
     with pytest.raises(oracle.OracleError):
         oracle.OracleLayer(W1=q1, W2=q2, W1s=s1, **common)
+
+
+# ---------------------------------------------------------------------------
+# block-scaled FP4 (MXFP4) expert weights
+# ---------------------------------------------------------------------------
+
+# E2M1 (the OCP microscaling FP4 element): 1 sign, 2 exponent bits (bias 1),
+# 1 mantissa bit, exponent 0 subnormal -- written out from that definition
+E2M1_TABLE = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+
+
+def test_e2m1_decode_is_the_format_table():
+    got = [oracle.e2m1_value(c) for c in range(16)]
+    assert got[:8] == E2M1_TABLE
+    assert got[8:] == [-v for v in E2M1_TABLE]
+    assert np.signbit(got[8])  # code 8 is -0
+
+
+def _np_dequant_mxfp4(q, e):
+    """numpy decode of output-major MXFP4 (codes [..., out, in/2], exponents
+    [..., out, in/32]) back to the API layout [..., in, out]."""
+    q = np.asarray(q, dtype=np.uint8)
+    lo, hi = q & 15, q >> 4
+    codes = np.stack([lo, hi], axis=-1).reshape(*q.shape[:-1], q.shape[-1] * 2)
+    mag = np.array(E2M1_TABLE)[codes & 7] * np.where(codes & 8, -1.0, 1.0)
+    scale = np.exp2(np.asarray(e, dtype=np.float64) - 127.0)
+    vals = mag * np.repeat(scale, 32, axis=-1)
+    return np.swapaxes(vals, -1, -2)
+
+
+def test_mxfp4_quantiser_round_trip():
+    """Each block's scale maps its largest magnitude into [4, 8) (saturating
+    at 6), the dequantised codes stay within half a grid step of W, values on
+    the grid come back exactly and midpoints go to the even code."""
+    W = rnd((3, 64, 24), 0.2, 81, "f32")
+    q, e = workloads.quantize_mxfp4(W)
+    assert q.shape == (3, 24, 32) and e.shape == (3, 24, 2) and q.dtype == torch.uint8
+    deq = _np_dequant_mxfp4(q.numpy(), e.numpy())
+    Wn = W.double().numpy()
+    blk = np.abs(Wn).reshape(3, 2, 32, 24).max(axis=2)                 # [3, 2 blocks, 24]
+    sc = np.exp2(np.swapaxes(e.numpy().astype(np.float64) - 127.0, -1, -2))  # [3, 2, 24]
+    assert np.all((blk / sc >= 4.0) & (blk / sc < 8.0))
+    # half the grid step at the value's magnitude; above 6 the code saturates
+    X = np.repeat(sc, 32, axis=1)
+    v = np.abs(Wn) / X
+    step = np.where(v >= 4.0, 2.0, np.where(v >= 2.0, 1.0, 0.5))
+    bound = np.where(v > 6.0, (v - 6.0) * X, step / 2 * X)
+    assert np.all(np.abs(deq - Wn) <= bound * 1.0000001 + 1e-300)
+    # grid values and midpoints (scale 1: the block's largest magnitude in [4, 8))
+    vals = torch.tensor([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0, 0.25, 0.75, 1.25, 1.75,
+                         2.5, 3.5, 5.0, -0.75, -5.0, 7.9, -1.5, 0.5, 0.0, 1.0, 2.0, 3.0,
+                         4.0, 6.0, -6.0, 0.1, 0.3, 2.9, 3.1, 5.1]).reshape(32, 1)
+    q1, e1 = workloads.quantize_mxfp4(vals)
+    assert int(e1[0, 0]) == 127
+    got = _np_dequant_mxfp4(q1.numpy(), e1.numpy())[:, 0]
+    want = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0, 0.0, 1.0, 1.0, 2.0, 2.0, 4.0, 4.0, -1.0,
+            -4.0, 6.0, -1.5, 0.5, 0.0, 1.0, 2.0, 3.0, 4.0, 6.0, -6.0, 0.0, 0.5, 3.0, 3.0, 6.0]
+    assert got.tolist() == want
+
+
+@pytest.mark.parametrize("act", ["swiglu", "relu2"])
+def test_fp4_single_expert_is_dense_chain(act):
+    """N = k = 1 with MXFP4 experts: the layer is x + act(z W1d) W2d Wup with
+    the matrices decoded in numpy (nibbles through the format table, each
+    block of 32 inputs times its power of two)."""
+    d, l, m = 48, 64, 96
+    L0, W = make_layer(d, l, 1, 1, m, act, seed=82, dtype="f32")
+    q1, e1 = workloads.quantize_mxfp4(W["W1"])
+    q2, e2 = workloads.quantize_mxfp4(W["W2"])
+    L = oracle.OracleLayer(d=d, l=l, N=1, k=1, m=m, act=act, dtype="f32", Wg=W["Wg"],
+                           Wdown=W["Wdown"], Wup=W["Wup"], W1=q1, W2=q2, W1e=e1, W2e=e2)
+    x = rnd((7, d), 1.0, 83, "f32")
+    W1d = _np_dequant_mxfp4(q1[0].numpy(), e1[0].numpy())
+    W2d = _np_dequant_mxfp4(q2[0].numpy(), e2[0].numpy())
+    z = as64(x) @ as64(W["Wdown"])
+    h = np_act(act, z @ W1d, m)
+    ref = as64(x) + (h @ W2d) @ as64(W["Wup"])
+    res = L.layer(x)
+    np.testing.assert_allclose(res["out"], ref, rtol=1e-12, atol=1e-12)
+
+
+def test_fp4_layer_equals_layer_with_dequantised_weights():
+    """Many experts: the MXFP4 layer equals the f32 layer whose expert weights
+    are the decoded values (exact in fp32); exponents applied per output
+    column instead of per block of inputs would miss."""
+    d, l, N, k, m = 40, 64, 6, 2, 32
+    L0, W = make_layer(d, l, N, k, m, "swiglu", dtype="f32", bias=True, seed=84)
+    q1, e1 = workloads.quantize_mxfp4(W["W1"])
+    q2, e2 = workloads.quantize_mxfp4(W["W2"])
+    W1d = torch.from_numpy(_np_dequant_mxfp4(q1.numpy(), e1.numpy()).astype(np.float32))
+    W2d = torch.from_numpy(_np_dequant_mxfp4(q2.numpy(), e2.numpy()).astype(np.float32))
+    common = dict(d=d, l=l, N=N, k=k, m=m, act="swiglu", dtype="f32", Wg=W["Wg"],
+                  bias=W["bias"], Wdown=W["Wdown"], Wup=W["Wup"])
+    L4 = oracle.OracleLayer(W1=q1, W2=q2, W1e=e1, W2e=e2, **common)
+    Ld = oracle.OracleLayer(W1=W1d, W2=W2d, **common)
+    x = rnd((30, d), 1.0, 85, "f32")
+    a, b = L4.layer(x), Ld.layer(x)
+    np.testing.assert_array_equal(a["idx"], b["idx"])
+    np.testing.assert_allclose(a["out"], b["out"], rtol=1e-12, atol=1e-12)
+    with pytest.raises(oracle.OracleError):
+        oracle.OracleLayer(W1=q1, W2=q2, W1e=e1, **common)
