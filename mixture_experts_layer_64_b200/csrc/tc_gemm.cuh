@@ -641,58 +641,64 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     walk.u_end = min(total, (long)(blockIdx.x + 1) * per);
   }
 
-  if (warp == 0) {
-    // ---------------- TMA producer ----------------
-    // Lane 0 arms the stages (activation rows, and bf16 weights).  With fp8
-    // weights lane 1 walks the same (tile, K block) sequence on its own and
-    // keeps the E4M3 slot ring loading, limited only by the converters.
-    if (Cfg::kFp8 && lane == 1) {
-      int j = 0;
-      uint32_t jph = 0;
-      long wissued = 0;
-      bool ok = true;
-      int tl, ks, kb0, kb1;
-      for (long wi = walk_start(walk); ok && walk_next(walk, wi, tl, ks, kb0, kb1);) {
-        const int rt = tl / NT, ft = tl - (tl / NT) * NT;
-        int g, row0, rows;
-        locate_row_tile_s(p, s_tiles, rt, g, row0, rows);
-        const int wrow = (int)(g * p.w_group_stride) + ft * Cfg::FT;
-        for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait(&w8empty[j], jph ^ 1, abort_flag, p.err)) { ok = false; break; }
-          uint8_t* slot = w8_ring + j * Cfg::W8_SLOT;
-          mbar_arrive_expect_tx(&w8full[j], Cfg::W8_SLOT);
-          if (Cfg::kFp4) {
-            // code pairs (32 bytes per row of the K slice), then the exponent
-            // box holding this slice's two exponents (16-byte aligned start;
-            // tmC is the exponent map in the weight-stationary kernels)
-            const int ex = (kb * 2) & ~15;
-            tma_load_2d(&tmB, &w8full[j], slot, kb * (Cfg::BK / 2), wrow);
-            tma_load_2d(&tmC, &w8full[j], slot + Cfg::W4_CODES, ex, wrow);
-            if (Cfg::kDual) {
-              tma_load_2d(&tmB, &w8full[j], slot + Cfg::W8_BYTES, kb * (Cfg::BK / 2),
-                          wrow + p.dual_offset);
-              tma_load_2d(&tmC, &w8full[j], slot + Cfg::W8_BYTES + Cfg::W4_CODES, ex,
-                          wrow + p.dual_offset);
-            }
-          } else {
-            tma_load_2d(&tmB, &w8full[j], slot, kb * Cfg::BK, wrow);
-            if (Cfg::kDual)
-              tma_load_2d(&tmB, &w8full[j], slot + Cfg::W8_BYTES, kb * Cfg::BK,
-                          wrow + p.dual_offset);
+  // The fp8 / fp4 weight slot producer: walks the (tile, K block) sequence on
+  // its own and keeps the slot ring loading, limited only by the converters.
+  // It runs alone in warp 3 on the weight-stationary tensor-memory tiles
+  // (where warp 3 has no other work), else in lane 1 of the producer warp.
+  const auto w8_producer = [&]() {
+    int j = 0;
+    uint32_t jph = 0;
+    long wissued = 0;
+    bool ok = true;
+    int tl, ks, kb0, kb1;
+    for (long wi = walk_start(walk); ok && walk_next(walk, wi, tl, ks, kb0, kb1);) {
+      const int rt = tl / NT, ft = tl - (tl / NT) * NT;
+      int g, row0, rows;
+      locate_row_tile_s(p, s_tiles, rt, g, row0, rows);
+      const int wrow = (int)(g * p.w_group_stride) + ft * Cfg::FT;
+      for (int kb = kb0; kb < kb1; ++kb) {
+        if (!mbar_wait(&w8empty[j], jph ^ 1, abort_flag, p.err)) { ok = false; break; }
+        uint8_t* slot = w8_ring + j * Cfg::W8_SLOT;
+        mbar_arrive_expect_tx(&w8full[j], Cfg::W8_SLOT);
+        if (Cfg::kFp4) {
+          // code pairs (32 bytes per row of the K slice), then the exponent
+          // box holding this slice's two exponents (16-byte aligned start;
+          // tmC is the exponent map in the weight-stationary kernels)
+          const int ex = (kb * 2) & ~15;
+          tma_load_2d(&tmB, &w8full[j], slot, kb * (Cfg::BK / 2), wrow);
+          tma_load_2d(&tmC, &w8full[j], slot + Cfg::W4_CODES, ex, wrow);
+          if (Cfg::kDual) {
+            tma_load_2d(&tmB, &w8full[j], slot + Cfg::W8_BYTES, kb * (Cfg::BK / 2),
+                        wrow + p.dual_offset);
+            tma_load_2d(&tmC, &w8full[j], slot + Cfg::W8_BYTES + Cfg::W4_CODES, ex,
+                        wrow + p.dual_offset);
           }
-          ++wissued;
-          if (++j == Cfg::S8) { j = 0; jph ^= 1; }
+        } else {
+          tma_load_2d(&tmB, &w8full[j], slot, kb * Cfg::BK, wrow);
+          if (Cfg::kDual)
+            tma_load_2d(&tmB, &w8full[j], slot + Cfg::W8_BYTES, kb * Cfg::BK,
+                        wrow + p.dual_offset);
         }
-      }
-      if (*abort_flag) {
-        // let the loads in flight land before the block frees its shared memory
-        for (long i = 0; i < wissued && i < Cfg::S8; ++i) {
-          if (j == 0) { j = Cfg::S8; jph ^= 1; }
-          --j;
-          mbar_wait_drain(&w8full[j], jph);
-        }
+        ++wissued;
+        if (++j == Cfg::S8) { j = 0; jph ^= 1; }
       }
     }
+    if (*abort_flag) {
+      // let the loads in flight land before the block frees its shared memory
+      for (long i = 0; i < wissued && i < Cfg::S8; ++i) {
+        if (j == 0) { j = Cfg::S8; jph ^= 1; }
+        --j;
+        mbar_wait_drain(&w8full[j], jph);
+      }
+    }
+  };
+  if (Cfg::kTmemA && warp == 3) {
+    if (lane == 0) w8_producer();
+  } else if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    // Lane 0 arms the stages (activation rows, and bf16 weights); with fp8
+    // weights on token tiles lane 1 runs the weight slot producer.
+    if (Cfg::kFp8 && !Cfg::kTmemA && lane == 1) w8_producer();
     if (lane == 0) {
       int s = 0;
       uint32_t ph = 0;
@@ -816,7 +822,8 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     // (at most 64 rows) with one gather4 (rows picked by token index; the
     // tile's padding rows repeat its first row), completing on the stage's
     // full barrier, whose expected bytes the producer has armed.  Warp 3 has
-    // no work.  (Token-tiled tiles gather 128 rows per stage with cp.async:
+    // no work here (with fp8 / fp4 weights it runs the weight slot producer).
+    // (Token-tiled tiles gather 128 rows per stage with cp.async:
     // there a four-row TMA gather cannot keep up.)
     if (warp == 2) {
       int s = 0;
