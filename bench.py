@@ -20,7 +20,7 @@ latent decode workload and both decode workloads with fp8 (E4M3) and with
 fp4 (MXFP4) expert weights, each with its own clocks, roofline, expert-load
 summary, per-stage p50/p95/p99 and projection share; and "variant_sweep": the
 standard MoE, l-MoE_eff and l-MoE_acc (LatentMoE, Section 3, Eq. (1) and
-(2)) at a decode and a prefill batch, with the weight and dispatch bytes
+(2)) at a latency-bound, a decode and a prefill batch, with the weight and dispatch bytes
 each loads.  All are measured in the same run with the same steps and
 warm-up (--no-prefill skips them).  --impl reference times the CPU oracle (the reference arm of this
 method: a plain float64 C++ implementation) on a bounded token sample of the

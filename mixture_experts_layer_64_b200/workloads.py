@@ -118,7 +118,7 @@ WORKLOADS["latent-decode-fp4"] = replace(WORKLOADS["latent-decode"], name="laten
 # (LatentMoE, Section 3, Eq. (1) and Eq. (2); Table 1): the standard layer
 # (d = 4096, N = 128 experts, top-8, m = 1536, no projections), l-MoE_eff
 # (latent l = d / 4, N' = 4 N, k' = k) and l-MoE_acc (l = d / 4, N' = 4 N,
-# k' = 4 k), on the same kernels, at a decode and a prefill batch.  No router
+# k' = 4 k), on the same kernels, at decode and prefill batches.  No router
 # bias, so all three see the same routing statistics.  The standard decode
 # point is std-moe-decode itself.
 _SWEEP = dict(d=4096, m=1536, act="swiglu")
@@ -132,8 +132,17 @@ WORKLOADS["l-moe-eff-prefill"] = Workload("l-moe-eff-prefill", T=4096, l=1024, N
                                           seed=14, **_SWEEP)
 WORKLOADS["l-moe-acc-prefill"] = Workload("l-moe-acc-prefill", T=4096, l=1024, N=512, k=32,
                                           seed=15, **_SWEEP)
-# (variant, standard point, l-MoE_eff point, l-MoE_acc point) per batch size
-VARIANT_SWEEP = (("decode", "std-moe-decode", "l-moe-eff-decode", "l-moe-acc-decode"),
+# ... and at a latency-bound batch of 8 tokens, where a step touches fewer
+# experts than there are (the regime of the paper's per-token memory cost)
+WORKLOADS["std-moe-latency"] = Workload("std-moe-latency", T=8, l=4096, N=128, k=8,
+                                        skip_proj=True, seed=16, **_SWEEP)
+WORKLOADS["l-moe-eff-latency"] = Workload("l-moe-eff-latency", T=8, l=1024, N=512, k=8,
+                                          seed=17, **_SWEEP)
+WORKLOADS["l-moe-acc-latency"] = Workload("l-moe-acc-latency", T=8, l=1024, N=512, k=32,
+                                          seed=18, **_SWEEP)
+# (batch, standard point, l-MoE_eff point, l-MoE_acc point) per batch size
+VARIANT_SWEEP = (("latency", "std-moe-latency", "l-moe-eff-latency", "l-moe-acc-latency"),
+                 ("decode", "std-moe-decode", "l-moe-eff-decode", "l-moe-acc-decode"),
                  ("prefill", "std-moe-prefill", "l-moe-eff-prefill", "l-moe-acc-prefill"))
 WORKLOAD_ORDER = list(WORKLOADS)
 

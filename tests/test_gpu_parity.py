@@ -718,7 +718,8 @@ FULL_SAMPLES = {"tiny-fp32": 64, "std-moe-decode": 96, "latent-decode": 96,
                 "std-moe-decode-fp8": 96, "latent-decode-fp8": 96,
                 "std-moe-decode-fp4": 96, "latent-decode-fp4": 96,
                 "l-moe-eff-decode": 64, "l-moe-acc-decode": 64, "std-moe-prefill": 48,
-                "l-moe-eff-prefill": 48, "l-moe-acc-prefill": 48}
+                "l-moe-eff-prefill": 48, "l-moe-acc-prefill": 48, "std-moe-latency": 8,
+                "l-moe-eff-latency": 8, "l-moe-acc-latency": 8}
 
 
 def edge_tokens_of_largest_experts(L, T: int, n_experts: int = 2, per_end: int = 3):
