@@ -847,6 +847,7 @@ lmoe_status run_routing(lmoe_layer* h, const float* logits, int T, int* idx, flo
     a.W = W;
     a.debug = debug;
     a.err = h->err;
+    a.sms = h->num_sms;  // one wave of blocks; their warps stride over the tokens
     const cudaError_t e = launch_topk_args(a, st, take_pdl(h));
     if (e != cudaSuccess) return cuda_fail(h, e, "top-k launch");
     ++h->launches;

@@ -196,10 +196,25 @@ struct TopkArgs {
   uint32_t* bitmap;  // [N, W]
   int W, debug;
   int* err;
+  int sms;  // > 0: at most the blocks resident on this many SMs, warps striding over tokens
 };
 
+// Token t's logits, slot i of lane = expert lane + 32 i (0 past N).  Issued
+// ahead of their use, so that a warp's next token loads while it ranks the
+// current one.
+template <int NPL>
+__device__ __forceinline__ void topk_fetch(const TopkArgs& a, int t, int lane, float (&raw)[NPL]) {
+  const float* lg = a.logits + (size_t)t * a.N;
+#pragma unroll
+  for (int i = 0; i < NPL; ++i) {
+    const int e = lane + 32 * i;
+    raw[i] = e < a.N ? __ldg(lg + e) : 0.f;
+  }
+}
+
 template <int NPL, bool kVariant>
-__device__ __forceinline__ void topk_token(const TopkArgs& a, int t, int lane, uint32_t* s_hist,
+__device__ __forceinline__ void topk_token(const TopkArgs& a, int t, int lane,
+                                           const float (&raw)[NPL], uint32_t* s_hist,
                                            unsigned long long* s_sel) {
   const int N = a.N, k = a.k;
   const float* sel_bias = kVariant ? a.sel_bias : nullptr;
@@ -212,7 +227,7 @@ __device__ __forceinline__ void topk_token(const TopkArgs& a, int t, int lane, u
     const int e = lane + 32 * i;
     key[i] = 0u;  // absent experts: 0, never above a real key and never counted
     if (e < N) {
-      float v = __ldg(lg + e);
+      float v = raw[i];
       if (a.debug && !isfinite(v)) bad = true;
       if (sel_bias) v = __fadd_rn(v, __ldg(sel_bias + e));
       key[i] = orderable_bits(v);
@@ -357,20 +372,49 @@ __global__ void __launch_bounds__(128) topk_softmax_kernel(const TopkArgs a) {
   __shared__ uint32_t s_hist[4][256];
   __shared__ unsigned long long s_sel[4][64];
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
-  const int t = blockIdx.x * (blockDim.x >> 5) + wib;
-  if (t < a.T) topk_token<NPL, kVariant>(a, t, lane, s_hist[wib], s_sel[wib]);
+  // each warp takes tokens t, t + stride, ...; the next token's logits are
+  // in flight while the current one is ranked
+  const int stride = gridDim.x * (blockDim.x >> 5);
+  int t = blockIdx.x * (blockDim.x >> 5) + wib;
+  float raw[NPL];
+  if (t < a.T) topk_fetch<NPL>(a, t, lane, raw);
+  while (t < a.T) {
+    const int tn = t + stride;
+    float next[NPL];
+    if (tn < a.T) topk_fetch<NPL>(a, tn, lane, next);
+    topk_token<NPL, kVariant>(a, t, lane, raw, s_hist[wib], s_sel[wib]);
+    if (tn < a.T) {
+#pragma unroll
+      for (int i = 0; i < NPL; ++i) raw[i] = next[i];
+    }
+    t = tn;
+  }
 }
 
 // Launches topk_softmax_kernel with the smallest multiple of 4 slots per lane
 // that covers N (pdl: programmatic stream serialisation).
+template <int NPL, bool kVariant>
+static inline cudaError_t launch_topk_npl(const TopkArgs& a, cudaStream_t st, bool pdl) {
+  const auto kern = topk_softmax_kernel<NPL, kVariant>;
+  int blocks = (a.T + 3) / 4;
+  if (a.sms > 0 && blocks > a.sms) {
+    // the blocks one wave holds (per instantiation; registers differ with NPL)
+    static const int occ = [&] {
+      int n = 0;
+      return cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, 128, 0) == cudaSuccess && n > 0
+                 ? n : 1;
+    }();
+    if (blocks > a.sms * occ) blocks = a.sms * occ;
+  }
+  return launch_kernel(pdl, kern, dim3(blocks), dim3(128), 0, st, a);
+}
+
 static inline cudaError_t launch_topk_args(const TopkArgs& a, cudaStream_t st, bool pdl) {
-  const dim3 grid((a.T + 3) / 4), block(128);
   const bool var = a.sel_bias != nullptr || a.full_softmax != 0;
   cudaError_t e = cudaSuccess;
 #define LMOE_TOPK_CASE(S)                                                                   \
   case S:                                                                                   \
-    e = var ? launch_kernel(pdl, topk_softmax_kernel<S, true>, grid, block, 0, st, a)       \
-            : launch_kernel(pdl, topk_softmax_kernel<S, false>, grid, block, 0, st, a);     \
+    e = var ? launch_topk_npl<S, true>(a, st, pdl) : launch_topk_npl<S, false>(a, st, pdl); \
     break;
   switch ((a.N + 127) / 128 * 4) {
     LMOE_TOPK_CASE(4)
