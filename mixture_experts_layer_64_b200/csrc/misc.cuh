@@ -41,11 +41,22 @@ __global__ void __launch_bounds__(256) combine_kernel(const T* __restrict__ ys,
 #pragma unroll
       for (int v = 0; v < VEC; ++v) acc[v] += add32[(size_t)t * ldr + c + v];
     }
-    for (int j = 0; j < k; ++j) {
-      const uint4 yv = __ldg(reinterpret_cast<const uint4*>(ys + (size_t)__ldg(rows + j) * l + c));
-      const T* yb = reinterpret_cast<const T*>(&yv);
+    // the k rows in groups of 8: a group's loads are all in flight before
+    // the first is added (the sum still runs in slot order)
+    for (int j0 = 0; j0 < k; j0 += 8) {
+      uint4 yv[8];
 #pragma unroll
-      for (int v = 0; v < VEC; ++v) acc[v] += to_f32<T>(yb[v]);
+      for (int jj = 0; jj < 8; ++jj)
+        if (j0 + jj < k)
+          yv[jj] = __ldg(reinterpret_cast<const uint4*>(ys + (size_t)__ldg(rows + j0 + jj) * l + c));
+#pragma unroll
+      for (int jj = 0; jj < 8; ++jj) {
+        if (j0 + jj < k) {
+          const T* yb = reinterpret_cast<const T*>(&yv[jj]);
+#pragma unroll
+          for (int v = 0; v < VEC; ++v) acc[v] += to_f32<T>(yb[v]);
+        }
+      }
     }
     uint4 ov;
     T* ob = reinterpret_cast<T*>(&ov);
