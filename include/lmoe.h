@@ -163,6 +163,15 @@ typedef enum { LMOE_F32 = 0, LMOE_BF16 = 1 } lmoe_dtype;
                                     LMOE_ERR_UNSUPPORTED); no expert
                                     parallelism.                             */
 
+#define LMOE_FC2_SPLIT          0x10000u /* prefill expert FC2 on CTA pairs:
+                                    where an expert's rows past its whole
+                                    256-row tiles are at most 128, they run
+                                    on one 128-row single-CTA tile in a
+                                    second launch (padding to 128 rows
+                                    instead of 256); everything else stays
+                                    on the pairs.  Results are within the
+                                    bf16 tolerance of the default path. */
+
 /* Limits of the library. */
 #define LMOE_MAX_EXPERTS 1024
 #define LMOE_MAX_TOPK    32

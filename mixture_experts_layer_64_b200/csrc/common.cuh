@@ -78,6 +78,9 @@ struct GemmProblem {
   int stream_k;           // weight-stationary decode tiles: stream-K work split
   float* sk_part;         // stream-K: 2 fp32 slots of kSkSlotFloats per CTA boundary
   int* sk_count;          // stream-K: one arrival counter per boundary (zero between launches)
+  int rem_of;             // > 0 (grouped): the tiles cover only each group's last
+                          // rows % rem_of rows (its whole rem_of-row tiles run in
+                          // another launch); tile_prefix counts those tiles
 };
 
 constexpr int kRowTile = 128;
@@ -140,7 +143,9 @@ __device__ __forceinline__ void locate_row_tile(const GemmProblem& p, int rt, in
     if (__ldg(p.tile_prefix + mid) <= rt) lo = mid; else hi = mid - 1;
   }
   g = lo;
-  const int start = __ldg(p.offsets + g), end = __ldg(p.offsets + g + 1);
+  int start = __ldg(p.offsets + g);
+  const int end = __ldg(p.offsets + g + 1);
+  if (p.rem_of > 0) start = end - (end - start) % p.rem_of;
   row0 = start + (rt - __ldg(p.tile_prefix + g)) * p.row_tile;
   rows = min(p.row_tile, end - row0);
 }

@@ -73,6 +73,11 @@ struct Grouping {
   int G = 0, e0 = 0;
   const int *offsets = nullptr, *tp128 = nullptr, *tp256 = nullptr, *tp64 = nullptr;
   const int *big256 = nullptr, *small128 = nullptr, *small256 = nullptr;
+  // the split expert FC2 (LMOE_FC2_SPLIT): 256-row pair tiles of every
+  // group (the last one only if more than 128 rows are left for it), and
+  // one 128-row tile of the last rows % 256 of the groups where those are
+  // at most 128
+  const int *full256 = nullptr, *rem128 = nullptr;
 };
 
 struct lmoe_layer {
@@ -122,6 +127,9 @@ struct lmoe_layer {
   // more than kPairMinRows rows (CTA pairs), 128- and 256-row tiles of the
   // others (weight-stationary, single CTA)
   int *big_prefix2 = nullptr, *small_prefix = nullptr, *small_prefix2 = nullptr;
+  // the expert FC2 split into whole 256-row pair tiles and 128-row tiles of
+  // the rest (LMOE_FC2_SPLIT)
+  int *full_prefix2 = nullptr, *rem_prefix = nullptr;
   // stream-K split of the weight-stationary decode GEMMs: two partial
   // accumulator slots and one arrival counter per boundary between CTAs
   float* sk_part = nullptr;
@@ -858,7 +866,9 @@ lmoe_status run_routing(lmoe_layer* h, const float* logits, int T, int* idx, flo
               tile_prefix2 ? h->tile_prefix64 : (int*)nullptr, h->done,
               tile_prefix2 ? h->big_prefix2 : (int*)nullptr,
               tile_prefix2 ? h->small_prefix : (int*)nullptr,
-              tile_prefix2 ? h->small_prefix2 : (int*)nullptr);
+              tile_prefix2 ? h->small_prefix2 : (int*)nullptr,
+              tile_prefix2 ? h->full_prefix2 : (int*)nullptr,
+              tile_prefix2 ? h->rem_prefix : (int*)nullptr);
   const long P = (long)T * h->k;
   LMOE_LAUNCH(h, group_rank_kernel, dim3((unsigned)((P + 255) / 256)), dim3(256), 0, st,
               (const int*)idx, (const float*)w, (const uint2*)h->wp, (const int*)offsets, T, h->k,
@@ -1056,6 +1066,23 @@ lmoe_status run_expert_gemms(lmoe_layer* h, const Grouping& g, const void* A, lo
     int path = 0;
     if (load_split) {
       LMOE_TRY(run_split_by_load(h, c, st, &path));
+    } else if (pair_fc2 && !ws_pair && !lowp && (h->flags & LMOE_FC2_SPLIT) && g.full256 &&
+               g.rem128) {
+      // an expert's last rows past its whole 256-row tiles, when at most 128,
+      // on one 128-row single-CTA tile (padding to 128 rows instead of 256);
+      // everything else on CTA pairs (two launches writing disjoint rows of ys)
+      GemmCall full = c;
+      make_pair(h, full);
+      full.p.tile_prefix = g.full256;
+      full.p.max_row_tiles = (int)(R / (2 * kRowTile) + 1);
+      LMOE_TRY(run_gemm(h, full, st, &path));
+      GemmCall rest = c;
+      rest.p.tile_prefix = g.rem128;
+      rest.p.row_tile = kRowTile;
+      rest.p.rem_of = 2 * kRowTile;
+      rest.p.max_row_tiles = 2 * g.G;
+      int p2 = 0;
+      LMOE_TRY(run_gemm(h, rest, st, &p2));
     } else {
       if (pair_fc2 && !ws_pair && !lowp) make_pair(h, c);  // the pair kernels read bf16 weights
       LMOE_TRY(run_gemm(h, c, st, &path));
@@ -1155,6 +1182,8 @@ void free_workspace(lmoe_layer* h) {
   free_ptr(h->big_prefix2);
   free_ptr(h->small_prefix);
   free_ptr(h->small_prefix2);
+  free_ptr(h->full_prefix2);
+  free_ptr(h->rem_prefix);
   free_ptr(h->sk_part);
   free_ptr(h->sk_count);
   free_ptr(h->slot_row);
@@ -1324,7 +1353,7 @@ lmoe_status lmoe_create(int d, int l, int N, int k, int m, lmoe_act act, int sha
                          LMOE_ROUTE_FULL_SOFTMAX | LMOE_ROUTE_BIAS_SELECT | LMOE_EXPERTS_FP8 |
                          LMOE_EXPERTS_FP4 |
                          LMOE_SINGLE_STREAM | LMOE_NO_PDL | LMOE_LOAD_SPLIT |
-                         LMOE_NO_STREAM_K | LMOE_SORTED_ROWS;
+                         LMOE_NO_STREAM_K | LMOE_SORTED_ROWS | LMOE_FC2_SPLIT;
   if (d <= 0 || l <= 0 || N <= 0 || k <= 0 || m <= 0 || shared_m < 0) return LMOE_ERR_INVALID_ARG;
   if (k > N || (flags & ~known)) return LMOE_ERR_INVALID_ARG;
   if (act != LMOE_ACT_SILU && act != LMOE_ACT_SWIGLU && act != LMOE_ACT_RELU2) return LMOE_ERR_INVALID_ARG;
@@ -1508,6 +1537,8 @@ lmoe_status lmoe_reserve(lmoe_layer* h, int max_T) {
   ALLOC(h->big_prefix2, (size_t)(h->N + 1) * sizeof(int));
   ALLOC(h->small_prefix, (size_t)(h->N + 1) * sizeof(int));
   ALLOC(h->small_prefix2, (size_t)(h->N + 1) * sizeof(int));
+  ALLOC(h->full_prefix2, (size_t)(h->N + 1) * sizeof(int));
+  ALLOC(h->rem_prefix, (size_t)(h->N + 1) * sizeof(int));
   if (h->dtype == LMOE_BF16 && !(h->flags & LMOE_NO_STREAM_K)) {
     ALLOC(h->sk_part, (size_t)2 * (h->num_sms + 1) * kSkSlotFloats * sizeof(float));
     ALLOC(h->sk_count, (size_t)(h->num_sms + 1) * sizeof(int));
@@ -1552,6 +1583,8 @@ lmoe_status lmoe_reserve(lmoe_layer* h, int max_T) {
   LMOE_CUDA(h, cudaMemset(h->big_prefix2, 0, (size_t)(h->N + 1) * sizeof(int)));
   LMOE_CUDA(h, cudaMemset(h->small_prefix, 0, (size_t)(h->N + 1) * sizeof(int)));
   LMOE_CUDA(h, cudaMemset(h->small_prefix2, 0, (size_t)(h->N + 1) * sizeof(int)));
+  LMOE_CUDA(h, cudaMemset(h->full_prefix2, 0, (size_t)(h->N + 1) * sizeof(int)));
+  LMOE_CUDA(h, cudaMemset(h->rem_prefix, 0, (size_t)(h->N + 1) * sizeof(int)));
   if (h->sk_count) LMOE_CUDA(h, cudaMemset(h->sk_count, 0, (size_t)(h->num_sms + 1) * sizeof(int)));
   LMOE_CUDA(h, cudaDeviceSynchronize());
   h->max_T = max_T;
@@ -1566,6 +1599,8 @@ lmoe_status lmoe_reserve(lmoe_layer* h, int max_T) {
   fg.big256 = h->big_prefix2;
   fg.small128 = h->small_prefix;
   fg.small256 = h->small_prefix2;
+  fg.full256 = h->full_prefix2;
+  fg.rem128 = h->rem_prefix;
   return LMOE_OK;
 }
 

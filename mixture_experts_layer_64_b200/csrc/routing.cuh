@@ -83,8 +83,10 @@ __device__ __forceinline__ void warp_sort_desc64(unsigned long long& a, unsigned
 static __device__ __noinline__ void scan_loads_block(const int* counts, int N, int* offsets,
                                               int* tile_prefix, int* tile_prefix2,
                                               int* tile_prefix64, int* big_prefix2,
-                                              int* small_prefix, int* small_prefix2) {
-  constexpr int kQ = 7;
+                                              int* small_prefix, int* small_prefix2,
+                                              int* full_prefix2 = nullptr,
+                                              int* rem_prefix = nullptr) {
+  constexpr int kQ = 9;
   __shared__ int s_q[kQ][256];
   const int nt = blockDim.x;
   const int per = (N + nt - 1) / nt;
@@ -97,8 +99,15 @@ static __device__ __noinline__ void scan_loads_block(const int* counts, int N, i
     q[4] = c > kPairMinRows ? q[2] : 0;
     q[5] = c > kPairMinRows ? 0 : q[1];
     q[6] = c > kPairMinRows ? 0 : q[2];
+    // pair tiles of the split FC2: the whole 256-row tiles, and the last
+    // rows if more than 128 of them are left (a 256-row tile pads them no
+    // worse than two 128-row tiles); at most 128 left rows take one 128-row
+    // single-CTA tile instead (half the padding)
+    const int r = c % (2 * kRowTile);
+    q[7] = c / (2 * kRowTile) + (r > kRowTile ? 1 : 0);
+    q[8] = (r > 0 && r <= kRowTile) ? 1 : 0;
   };
-  int sum[kQ] = {0, 0, 0, 0, 0, 0, 0};
+  int sum[kQ] = {0, 0, 0, 0, 0, 0, 0, 0, 0};
   for (int i = lo; i < hi; ++i) {
     int q[kQ];
     tiles_of(__ldcg(counts + i), q);
@@ -120,8 +129,8 @@ static __device__ __noinline__ void scan_loads_block(const int* counts, int N, i
   int run[kQ];
 #pragma unroll
   for (int j = 0; j < kQ; ++j) run[j] = s_q[j][threadIdx.x] - sum[j];
-  int* out[kQ] = {offsets,     tile_prefix,  tile_prefix2, tile_prefix64,
-                  big_prefix2, small_prefix, small_prefix2};
+  int* out[kQ] = {offsets,      tile_prefix,   tile_prefix2, tile_prefix64, big_prefix2,
+                  small_prefix, small_prefix2, full_prefix2, rem_prefix};
   for (int i = lo; i < hi; ++i) {
     int q[kQ];
     tiles_of(__ldcg(counts + i), q);
@@ -478,7 +487,9 @@ static __global__ void __launch_bounds__(256) group_count_kernel(uint32_t* __res
                                                           unsigned int* done,
                                                           int* __restrict__ big_prefix2 = nullptr,
                                                           int* __restrict__ small_prefix = nullptr,
-                                                          int* __restrict__ small_prefix2 = nullptr) {
+                                                          int* __restrict__ small_prefix2 = nullptr,
+                                                          int* __restrict__ full_prefix2 = nullptr,
+                                                          int* __restrict__ rem_prefix = nullptr) {
   griddep_launch();
   griddep_wait();  // the previous kernel's outputs are visible
   const int lane = threadIdx.x & 31;
@@ -512,7 +523,7 @@ static __global__ void __launch_bounds__(256) group_count_kernel(uint32_t* __res
   if (!is_last) return;
   __threadfence();
   scan_loads_block(counts, N, offsets, tile_prefix, tile_prefix2, tile_prefix64, big_prefix2,
-                   small_prefix, small_prefix2);
+                   small_prefix, small_prefix2, full_prefix2, rem_prefix);
   if (threadIdx.x == 0) *done = 0u;
 }
 

@@ -490,7 +490,9 @@ __device__ __forceinline__ void locate_row_tile_s(const GemmProblem& p, const in
     if (tp[mid] <= rt) lo = mid; else hi = mid - 1;
   }
   g = lo;
-  row0 = off[g] + (rt - tp[g]) * p.row_tile;
+  // (rem_of: only the group's last rows % rem_of rows)
+  const int start = p.rem_of > 0 ? off[g + 1] - (off[g + 1] - off[g]) % p.rem_of : off[g];
+  row0 = start + (rt - tp[g]) * p.row_tile;
   rows = min(p.row_tile, off[g + 1] - row0);
 }
 

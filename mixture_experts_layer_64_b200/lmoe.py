@@ -30,6 +30,7 @@ LOAD_SPLIT = 0x1000
 NO_STREAM_K = 0x2000
 SORTED_ROWS = 0x4000
 EXPERTS_FP4 = 0x8000
+FC2_SPLIT = 0x10000
 MAX_EXPERTS, MAX_TOPK = 1024, 32
 DEVERR_WAIT_TIMEOUT, DEVERR_RANGE, DEVERR_NONFINITE = 0x1, 0x2, 0x4
 STAGES = {"logits": 0, "idx": 1, "w": 2, "offsets": 3, "perm": 4, "z": 5, "h": 6, "ys": 7, "comb": 8}

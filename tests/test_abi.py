@@ -68,7 +68,7 @@ def test_status_strings_and_stage_names(L):
     (256, 64, 16, 4, 128, 0, -1, 0, 0),       # negative shared width
     (256, 64, 16, 4, 128, 0, 0, 0, 1),        # skip flag with l != d
     (256, 256, 16, 4, 128, 0, 0, 0, 0x8 | 0x10),  # contradictory forcing flags
-    (256, 256, 16, 4, 128, 0, 0, 0, 0x10000),  # unknown flag
+    (256, 256, 16, 4, 128, 0, 0, 0, 0x20000),  # unknown flag
 ])
 def test_create_rejects_bad_arguments(L, args):
     h = ctypes.c_void_p(123)

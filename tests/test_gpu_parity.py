@@ -234,6 +234,50 @@ def test_load_split_on_skewed_loads(act, sorted_rows):
 
 
 @pytest.mark.parametrize("act", ["swiglu", "relu2"])
+def test_fc2_split_on_skewed_loads(act):
+    """LMOE_FC2_SPLIT: an expert's rows past its whole 256-row tiles of the
+    expert FC2, when at most 128, on one 128-row single-CTA tile, the rest on
+    CTA pairs (loads from ~T/2 rows down to none: several whole tiles,
+    remainders on either side of 128, experts below 256 rows)."""
+    w = W_("fc2-split", T=1100, d=256, l=192, N=16, k=4, m=320, act=act, shared_m=0, seed=26)
+    W = workloads.make_weights(w, device="cuda")
+    b = torch.linspace(3.0, -3.0, w.N, device="cuda")
+    b[-1] = -40.0  # never chosen
+    W["bias"] = b
+    L, _ = gpu_layer(w, lmoe.FC2_SPLIT, W)
+    x = workloads.make_x(w, device="cuda")
+    res = check_forward(w, W=W, layer=L, x=x, fixture=True, tokens=sample_tokens(w.T, 300, seed=4))
+    assert paths(res) == (1, 3)
+    loads = np.diff(L.debug_dump("offsets", w.T).cpu().numpy())
+    assert loads[-1] == 0 and loads.max() > 512
+    assert ((loads > 0) & (loads < 256)).any() and (loads % 256 != 0).any()
+    # the same layer without the split: the same routing, outputs within the
+    # bf16 tolerance (the remainder rows run through other MMA shapes)
+    L2, _ = gpu_layer(w, 0, W)
+    a, b2 = L.forward(x), L2.forward(x)
+    torch.cuda.synchronize()
+    assert torch.equal(L.debug_dump("idx", w.T), L2.debug_dump("idx", w.T))
+    err = (a.double() - b2.double()).abs()
+    assert float(err.max()) <= 2e-2 + float(b2.double().abs().max()) * 2 ** -7
+
+
+def test_fc2_split_full_size_skewed():
+    """LMOE_FC2_SPLIT on latent-prefill-skewed at full size, sampled tokens
+    plus the first and last tokens of the most loaded experts."""
+    w = workloads.WORKLOADS["latent-prefill-skewed"]
+    L, W = gpu_layer(w, lmoe.FC2_SPLIT)
+    x = workloads.make_x(w, device="cuda")
+    L.forward(x)
+    torch.cuda.synchronize()
+    toks = np.unique(np.concatenate([sample_tokens(w.T, 32, seed=w.seed + 1),
+                                     edge_tokens_of_largest_experts(L, w.T)])).astype(np.int32)
+    res = check_forward(w, tokens=toks, layer=L, W=W, x=x)
+    assert res["unique"] >= 0.8 * res["tokens"]
+    assert paths(res) == (1, 3)
+    torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("act", ["swiglu", "relu2"])
 def test_stream_k_decode_tiles(act):
     """The weight-stationary decode FC1 with 2 to 16 tiles per CTA takes the
     stream-K split (tiles straddling two CTAs' ranges summed from two fp32

@@ -24,8 +24,8 @@ def test_binding_flags_and_limits_match_the_header():
              if k in ("SKIP_PROJ", "DEBUG_CHECKS", "FORCE_SIMT", "FORCE_SWAP", "FORCE_NOSWAP",
                       "FORCE_NOPAIR", "FORCE_WS_PAIR", "ROUTE_FULL_SOFTMAX", "ROUTE_BIAS_SELECT",
                       "EXPERTS_FP8", "SINGLE_STREAM", "NO_PDL", "LOAD_SPLIT",
-                      "NO_STREAM_K", "SORTED_ROWS", "EXPERTS_FP4")}
-    assert len(flags) == 16, sorted(flags)
+                      "NO_STREAM_K", "SORTED_ROWS", "EXPERTS_FP4", "FC2_SPLIT")}
+    assert len(flags) == 17, sorted(flags)
     for name, value in flags.items():
         assert getattr(lmoe, name) == value, name
     # flags are distinct single bits
