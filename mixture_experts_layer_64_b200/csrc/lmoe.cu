@@ -334,14 +334,19 @@ bool tma_store_ok(const GemmCall& c) {
   return aligned16(base) && ((size_t)e.ldo * es) % 16 == 0 && (c.p.F * es) % 16 == 0;
 }
 
+// Function attributes and occupancy are per device: the launch helpers
+// keep what they set up per device ordinal (below kMaxDevices).
+constexpr int kMaxDevices = 64;
+
 template <class Cfg>
 lmoe_status launch_tc(lmoe_layer* h, const GemmCall& c, cudaStream_t st) {
-  static bool attr_done = false;
-  if (!attr_done) {
+  static bool attr_done[kMaxDevices] = {};
+  bool& done = attr_done[h->device % kMaxDevices];
+  if (!done) {
     LMOE_CUDA(h, cudaFuncSetAttribute(tc_gemm_kernel<Cfg>,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       Cfg::SMEM_BYTES));
-    attr_done = true;
+    done = true;
   }
   CUtensorMap ta, tb;
   std::memset(&ta, 0, sizeof ta);
@@ -430,7 +435,8 @@ lmoe_status pair_launch(lmoe_layer* h, Kern kern, int smem_bytes, long clusters,
 
 template <class Cfg>
 lmoe_status launch_pair(lmoe_layer* h, const GemmCall& c, cudaStream_t st) {
-  static int max_clusters = 0;
+  static int clusters_of[kMaxDevices] = {};
+  int& max_clusters = clusters_of[h->device % kMaxDevices];
   if (max_clusters == 0)
     LMOE_TRY(pair_setup(h, tc_gemm_pair_kernel<Cfg>, Cfg::SMEM_BYTES, &max_clusters));
   CUtensorMap ta, tb;
@@ -457,7 +463,8 @@ lmoe_status launch_pair(lmoe_layer* h, const GemmCall& c, cudaStream_t st) {
 // tile prefix of the grouping step.
 template <class Cfg>
 lmoe_status launch_pair_ws(lmoe_layer* h, const GemmCall& c, cudaStream_t st) {
-  static int max_clusters = 0;
+  static int clusters_of[kMaxDevices] = {};
+  int& max_clusters = clusters_of[h->device % kMaxDevices];
   if (max_clusters == 0)
     LMOE_TRY(pair_setup(h, tc_gemm_pair_ws_kernel<Cfg>, Cfg::SMEM_BYTES, &max_clusters));
   CUtensorMap ta, tb;

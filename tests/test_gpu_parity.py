@@ -794,3 +794,37 @@ def test_workload_full_size(name):
     if w.dtype == "bf16":
         assert paths(res)[0] in (1, 2, 4, 5)
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("name", ["swiglu-shared", "decode-like"])
+def test_forward_captures_into_a_cuda_graph(name):
+    """lmoe_forward enqueues only kernels, copies and cross-stream events (no
+    allocation, no synchronisation), so a caller can capture it into a CUDA
+    graph (side stream, programmatic dependent launch and split-K / stream-K
+    included) and replay it: each replay equals the eager forward bit for
+    bit, also on new inputs written into the captured input buffer."""
+    w = SMALL["swiglu-shared"] if name == "swiglu-shared" else W_(
+        "graph-decode", T=64, d=1024, l=512, N=64, k=8, m=512, act="swiglu",
+        bias="normal0.5", seed=57)
+    L, W = gpu_layer(w)
+    x = workloads.make_x(w, device="cuda")
+    x2 = workloads.make_x(W_(**{**w.__dict__, "seed": w.seed + 99}), device="cuda")
+    ref1 = L.forward(x).clone()
+    ref2 = L.forward(x2).clone()
+    xin, out = x.clone(), torch.empty_like(x)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):  # warm-up on a side stream, as torch asks before capture
+        L.forward(xin, out)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        L.forward(xin, out)
+    for src, ref in ((x, ref1), (x2, ref2), (x, ref1)):
+        xin.copy_(src)
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(out, ref)
+    assert L.last_error() == (lmoe.OK, 0)
+    del g
