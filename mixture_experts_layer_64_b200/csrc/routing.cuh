@@ -254,6 +254,35 @@ __device__ __forceinline__ void topk_token(const TopkArgs& a, int t, int lane,
     if (lane + 32 * i < N && key[i] >= theta) sel |= 1u << i;
   int ncand = (int)__reduce_add_sync(0xffffffffu, (uint32_t)__popc(sel));
 
+  if (ncand > 64 && k <= 64) {
+    // A tighter lower bound on the k-th largest key: the k-th largest of the
+    // lanes' two largest keys (a sub-multiset of the keys, so at most the
+    // k-th largest of them all).  With k near 32 the lane maxima alone bound
+    // it poorly (the k-th of 32 maxima is their smallest).
+    uint32_t top2 = 0u;
+    bool seen = false;  // one instance of the lane maximum skipped
+#pragma unroll
+    for (int i = 0; i < NPL; ++i) {
+      if (lane + 32 * i < N) {
+        if (!seen && key[i] == lmax) seen = true;
+        else top2 = max(top2, key[i]);
+      }
+    }
+    unsigned long long a = lmax, b = top2;
+    warp_sort_desc64(a, b, lane);  // position p: lane p's a (p < 32), lane p - 32's b
+    const uint32_t theta2 =
+        (uint32_t)__shfl_sync(0xffffffffu, (k - 1) < 32 ? a : b, (k - 1) & 31);
+    uint32_t sel2 = 0;
+#pragma unroll
+    for (int i = 0; i < NPL; ++i)
+      if (lane + 32 * i < N && key[i] >= theta2) sel2 |= 1u << i;
+    const int n2 = (int)__reduce_add_sync(0xffffffffu, (uint32_t)__popc(sel2));
+    if (n2 <= 64) {
+      sel = sel2;
+      ncand = n2;
+    }
+  }
+
   if (ncand > 64) {
     // radix select of the k-th largest key
     uint32_t* hist = s_hist;
