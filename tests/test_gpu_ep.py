@@ -128,3 +128,33 @@ def test_expert_parallel_errors():
         L.ep_experts(None, None, np.zeros((3, 5), dtype=np.int32), 0, 3)
     with pytest.raises(lmoe.LmoeError):  # combine without a dispatch
         L.ep_combine(x, torch.zeros((w.T * w.k, w.l), dtype=torch.bfloat16, device="cuda"))
+
+
+def test_expert_parallel_layer_over_nccl_world_one():
+    """ExpertParallelLayer through a real NCCL process group of one rank (the
+    only size a one-GPU run can form; the gloo tests cover the exchange plan
+    at world sizes 2 and 4): dispatch, the count and row all-to-alls, the
+    experts and the combine equal lmoe_forward on the same tokens."""
+    import os
+    import socket
+    import torch.distributed as dist
+    from mixture_experts_layer_64_b200.ep import ExpertParallelLayer
+
+    w = EP["latent-relu2-shared"]
+    L, W = gpu_layer(w)
+    x = workloads.make_x(w, device="cuda")
+    ref = L.forward(x).clone()
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    store = dist.TCPStore("127.0.0.1", port, 1, True)
+    dist.init_process_group("nccl", store=store, rank=0, world_size=1,
+                            device_id=torch.device("cuda", torch.cuda.current_device()))
+    try:
+        ep_layer = ExpertParallelLayer(L, max_recv_rows=w.T * w.k)
+        out = ep_layer(x)
+        torch.cuda.synchronize()
+    finally:
+        dist.destroy_process_group()
+    _close(out, ref)
+    assert L.last_error() == (lmoe.OK, 0)
