@@ -1065,7 +1065,11 @@ lmoe_status run_expert_gemms(lmoe_layer* h, const Grouping& g, const void* A, lo
                               fp8 ? 1 : h->es, l, l, m);
     c.p.w_scale = fp8 ? h->W2s + (size_t)g.e0 * l : nullptr;
     c.p.w_exp = fp4 ? h->W2e_t : nullptr;
-    c.swap = swap;
+    // fp8 FC2 on token tiles at every size (unless weight-stationary tiles are
+    // forced): one 128 x 256 MMA per K step covers 256 output features where
+    // the 16-row weight-stationary tiles issue two, and at decode the MMA
+    // count, not HBM, sets the pace of the widened fp8 kernels
+    c.swap = swap && !(fp8 && !(h->flags & LMOE_FORCE_SWAP));
     c.ws_pair = ws_pair && !lowp;
     c.p.epi.out = ysbuf;
     c.p.epi.ldo = l;

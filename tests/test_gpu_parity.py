@@ -479,17 +479,17 @@ FP8 = {
 @pytest.mark.parametrize("name", list(FP8))
 @pytest.mark.parametrize("flags", [0, lmoe.FORCE_SWAP, lmoe.FORCE_NOSWAP])
 def test_fp8_experts(name, flags):
-    """E4M3 expert weights widened to bf16 inside the tensor-core kernels and
+    """E4M3 expert weights widened to f16 inside the tensor-core kernels and
     scaled per output channel in the epilogue, against the oracle reading
-    the same codes: weight-stationary (2, 2) and token-tiled (1, 1)."""
+    the same codes: FC1 weight-stationary or token-tiled by size with FC2 on
+    token tiles (default), both weight-stationary (2, 2), both token-tiled
+    (1, 1)."""
     res = check_forward(FP8[name], flags=flags, fixture=True)
     assert res["unique"] >= 0.9 * res["tokens"]
     fc1, fc2 = paths(res)
-    assert fc1 == fc2 and fc1 in (1, 2)
-    if flags == lmoe.FORCE_SWAP:
-        assert fc1 == 2
-    if flags == lmoe.FORCE_NOSWAP:
-        assert fc1 == 1
+    assert fc1 in (1, 2)
+    want = {0: (fc1, 1), lmoe.FORCE_SWAP: (2, 2), lmoe.FORCE_NOSWAP: (1, 1)}[flags]
+    assert (fc1, fc2) == want
 
 
 def test_fp8_experts_prefill_sized():
