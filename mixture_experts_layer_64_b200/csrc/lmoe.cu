@@ -359,7 +359,7 @@ lmoe_status launch_tc(lmoe_layer* h, const GemmCall& c, cudaStream_t st) {
     return LMOE_ERR_CUDA;
   }
   const bool wmap =
-      Cfg::kFp4 ? encode_map_fp4(&tb, c.p.B, c.b_rows, c.p.K / 2, 32, Cfg::W_ROWS, true)
+      Cfg::kFp4 ? encode_map_fp4(&tb, c.p.B, c.b_rows, c.p.K / 2, 32, Cfg::W_ROWS, Cfg::kTmemA)
       : Cfg::kFp8 ? encode_map_u8(&tb, c.p.B, c.b_rows, c.p.K, c.p.K, Cfg::W_ROWS, Cfg::kTmemA)
                   : encode_map(&tb, c.p.B, c.b_rows, c.p.K, c.p.K, Cfg::W_ROWS);
   if (!wmap) {
@@ -369,9 +369,9 @@ lmoe_status launch_tc(lmoe_layer* h, const GemmCall& c, cudaStream_t st) {
   CUtensorMap tc;
   std::memset(&tc, 0, sizeof tc);
   GemmProblem p = c.p;
-  p.tma_store = (!Cfg::kSwap && tma_store_ok(c) && encode_out_map(&tc, c)) ? 1 : 0;
-  // fp4 weights: the weight-stationary kernel's third map holds the block
-  // exponents (it stores no output tiles by TMA)
+  p.tma_store = (!Cfg::kSwap && !Cfg::kFp4 && tma_store_ok(c) && encode_out_map(&tc, c)) ? 1 : 0;
+  // fp4 weights: the kernel's third map holds the block exponents (its
+  // epilogue then stores with plain stores)
   if (Cfg::kFp4 &&
       !encode_map_fp4(&tc, c.p.w_exp, c.b_rows, c.p.K / 32, 16, Cfg::W_ROWS, false)) {
     h->detail = "cuTensorMapEncodeTiled (fp4 exponents) failed";
@@ -600,11 +600,17 @@ lmoe_status run_gemm(lmoe_layer* h, GemmCall c, cudaStream_t st, int* path = nul
     }
   };
   if (c.p.w_exp) {
-    // fp4 expert weights: the weight-stationary kernel, weights widened into
-    // tensor memory, at every batch size
-    if (!tc_eligible(h, c) || !c.swap || c.pair) {
-      h->detail = "fp4 expert weights need the weight-stationary tensor-core kernel";
+    // fp4 expert weights: FC1 on the weight-stationary kernel (weights widened
+    // into tensor memory) at every batch size, FC2 on it or on token tiles
+    // (weights widened into shared memory)
+    if (!tc_eligible(h, c) || c.pair || (!c.swap && c.kind != GK_FC2)) {
+      h->detail = "fp4 expert weights: no tensor-core kernel for this call";
       return LMOE_ERR_UNSUPPORTED;
+    }
+    if (!c.swap) {
+      if (path) *path = 1;
+      return launch_tc<TcCfg<false, false, false, 256, EPI_SCALE_ROWS, true, kSwapRowTile, true>>(
+          h, c, st);
     }
     swap_rows(c);
     const bool dual = c.p.dual_offset > 0;
@@ -1065,11 +1071,11 @@ lmoe_status run_expert_gemms(lmoe_layer* h, const Grouping& g, const void* A, lo
                               fp8 ? 1 : h->es, l, l, m);
     c.p.w_scale = fp8 ? h->W2s + (size_t)g.e0 * l : nullptr;
     c.p.w_exp = fp4 ? h->W2e_t : nullptr;
-    // fp8 FC2 on token tiles at every size (unless weight-stationary tiles are
-    // forced): one 128 x 256 MMA per K step covers 256 output features where
-    // the 16-row weight-stationary tiles issue two, and at decode the MMA
-    // count, not HBM, sets the pace of the widened fp8 kernels
-    c.swap = swap && !(fp8 && !(h->flags & LMOE_FORCE_SWAP));
+    // fp8 / fp4 FC2 on token tiles at every size (unless weight-stationary
+    // tiles are forced): one 128 x 256 MMA per K step covers 256 output
+    // features where the 16-row weight-stationary tiles issue two, and at
+    // decode the MMA count, not HBM, sets the pace of the widened kernels
+    c.swap = swap && !(lowp && !(h->flags & LMOE_FORCE_SWAP));
     c.ws_pair = ws_pair && !lowp;
     c.p.epi.out = ysbuf;
     c.p.epi.ldo = l;

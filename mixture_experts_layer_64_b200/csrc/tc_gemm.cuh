@@ -87,7 +87,7 @@ struct TcCfg {
   // low-precision weights: block-scaled FP4 (kFp4: E2M1 code pairs, 32-byte
   // rows per 64-wide K slice, then the tile's E8M0 exponents, a 16-byte box
   // per row) or fp8 E4M3 (64-byte rows)
-  static constexpr bool kFp4 = kFp4_;
+  static constexpr bool kFp4 = kFp4_;  // (with kFp8: fp4 reuses the widening paths)
   static constexpr int W4_CODES = kFp4 ? W_ROWS * BK / 2 : 0;  // one fp4 weight tile's codes
   static constexpr int W4_EXPS = kFp4 ? W_ROWS * 16 : 0;       // ... and its exponent box
   static constexpr int W8_BYTES = kFp4 ? W4_CODES + W4_EXPS : kFp8 ? W_ROWS * BK : 0;
@@ -119,6 +119,10 @@ struct TcCfg {
   // (warps 0-3 the gate tile, 4-7 the linear one); ungated tiles: the two
   // groups of four take alternate units, so two units widen at once.
   static constexpr int CONV_PER_UNIT = kTmemA ? (kDual ? 8 : 4) : (kFp8 ? 8 : 0);
+  // fp8 / fp4: the weight slot producer has warp 3 to itself where that warp
+  // gathers no rows (weight-stationary tiles, and token tiles of contiguous
+  // rows), else it shares the producer warp (lane 1)
+  static constexpr bool kW8Warp3 = kFp8 && (kTmemA || !kCpGather);
   static constexpr int STAGES = kTmemA ? LMOE_TMEMA_STAGES
                                 : kFp8 ? (STAGES_F8 < 3 ? 3 : (STAGES_F8 > 8 ? 8 : STAGES_F8))
                                        : (STAGES_RAW > 8 ? 8 : STAGES_RAW);
@@ -150,7 +154,7 @@ struct TcCfg {
   static_assert(!kFp8 || kEpi == EPI_ACT || kEpi == EPI_SCALE_ROWS, "fp8 weights: expert GEMMs");
   static_assert(kSwapRows == kSwapRowTile || kSwapRows == 128 || kSwapRows == 256, "swap rows");
   static_assert(!kWideSwap || !kFp8, "wide weight-stationary tiles: bf16 weights");
-  static_assert(!kFp4 || (kFp8 && kSwap), "fp4 weights: the weight-stationary tensor-memory path");
+  static_assert(!kFp4 || kFp8, "fp4 weights: the widening (fp8) kernel paths");
 };
 
 // ---- fp8 E4M3 weights -----------------------------------------------------------
@@ -222,14 +226,34 @@ __device__ __forceinline__ __half pow2_half(int e) {
   return __ushort_as_half(bits);
 }
 
+// Eight E2M1 codes (four bytes, the low nibble of each byte first) as four
+// words of f16 pairs, each exact (cvt.rn.f16x2.e2m1x2) and then scaled by
+// the block's power of two sc (an exact f16 multiply: the exponents are
+// limited so that every product is an f16 value).
+__device__ __forceinline__ void e2m1x8_to_f16x8(uint32_t codes, __half2 sc, uint32_t* out) {
+  uint32_t w0, w1, w2, w3;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+      : "=r"(w0), "=r"(w1), "=r"(w2), "=r"(w3)
+      : "r"(codes));
+  const uint32_t ws[4] = {w0, w1, w2, w3};
+#pragma unroll
+  for (int b = 0; b < 4; ++b) {
+    __half2 h = *reinterpret_cast<const __half2*>(&ws[b]);
+    h = __hmul2(h, sc);
+    out[b] = *reinterpret_cast<const uint32_t*>(&h);
+  }
+}
+
 // Widens row r of an MXFP4 weight tile for one 64-wide K slice: 32 bytes of
 // E2M1 code pairs (TMA-stored with the 32-byte swizzle: 16-byte chunk c of
 // row r sits at chunk c ^ ((r >> 2) & 1)) and the row's two E8M0 block
-// exponents, at byte `eoff` of its 16-byte exponent row.  Each code widens
-// exactly to f16 (cvt.rn.f16x2.e2m1x2), then takes its block's power of two
-// (an exact f16 multiply: the exponents are limited so that every product is
-// an f16 value).  Output as widen_fp8_row_sw64: 32 words of f16 pairs, K
-// ascending.
+// exponents, at byte `eoff` of its 16-byte exponent row.  Output as
+// widen_fp8_row_sw64: 32 words of f16 pairs, K ascending.
 __device__ __forceinline__ void widen_fp4_row_sw32(const uint8_t* codes, const uint8_t* exps, int r,
                                                    int eoff, uint32_t (&out)[32]) {
   const int x = (r >> 2) & 1;
@@ -237,26 +261,37 @@ __device__ __forceinline__ void widen_fp4_row_sw32(const uint8_t* codes, const u
   for (int c = 0; c < 2; ++c) {  // chunk c: K elements 32c .. 32c + 31, block c
     const uint4 v = *reinterpret_cast<const uint4*>(codes + r * 32 + ((c ^ x) << 4));
     const __half2 sc = __half2half2(pow2_half((int)exps[r * 16 + eoff + c] - 127));
-    const uint32_t in[4] = {v.x, v.y, v.z, v.w};
+    e2m1x8_to_f16x8(v.x, sc, &out[16 * c + 0]);
+    e2m1x8_to_f16x8(v.y, sc, &out[16 * c + 4]);
+    e2m1x8_to_f16x8(v.z, sc, &out[16 * c + 8]);
+    e2m1x8_to_f16x8(v.w, sc, &out[16 * c + 12]);
+  }
+}
+
+// Widens an MXFP4 weight tile (W_ROWS rows of 32 code bytes, unswizzled, and
+// a 16-byte exponent row each) for one 64-wide K slice to f16 in the
+// 128-byte-swizzled K-major layout of a stage, by kConv converter threads:
+// chunk c = (row, 32-element block h) is handled by thread c mod kConv and
+// writes the block's four 16-byte chunks.
+template <int W_ROWS, int kConv>
+__device__ __forceinline__ void widen_fp4_tile(const uint8_t* codes, const uint8_t* exps, int eoff,
+                                               uint8_t* dst, int ct) {
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {  // 8 codes: bytes b0..b3, low nibble first
-      uint32_t w0, w1, w2, w3;
-      asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
-          "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
-          "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
-          "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
-          "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
-          "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
-          : "=r"(w0), "=r"(w1), "=r"(w2), "=r"(w3)
-          : "r"(in[q]));
-      const uint32_t ws[4] = {w0, w1, w2, w3};
+  for (int c = ct; c < W_ROWS * 2; c += kConv) {
+    const int r = c >> 1, hb = c & 1;
+    const uint4 v = *reinterpret_cast<const uint4*>(codes + r * 32 + hb * 16);
+    const __half2 sc = __half2half2(pow2_half((int)exps[r * 16 + eoff + hb] - 127));
+    uint32_t out[16];
+    e2m1x8_to_f16x8(v.x, sc, &out[0]);
+    e2m1x8_to_f16x8(v.y, sc, &out[4]);
+    e2m1x8_to_f16x8(v.z, sc, &out[8]);
+    e2m1x8_to_f16x8(v.w, sc, &out[12]);
+    uint8_t* row = dst + r * 128;
+    const int sw = r & 7;
 #pragma unroll
-      for (int b = 0; b < 4; ++b) {
-        __half2 h = *reinterpret_cast<const __half2*>(&ws[b]);
-        h = __hmul2(h, sc);
-        out[16 * c + 4 * q + b] = *reinterpret_cast<const uint32_t*>(&h);
-      }
-    }
+    for (int i = 0; i < 4; ++i)
+      *reinterpret_cast<uint4*>(row + (((4 * hb + i) ^ sw) << 4)) =
+          make_uint4(out[4 * i], out[4 * i + 1], out[4 * i + 2], out[4 * i + 3]);
   }
 }
 
@@ -645,8 +680,8 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
 
   // The fp8 / fp4 weight slot producer: walks the (tile, K block) sequence on
   // its own and keeps the slot ring loading, limited only by the converters.
-  // It runs alone in warp 3 on the weight-stationary tensor-memory tiles
-  // (where warp 3 has no other work), else in lane 1 of the producer warp.
+  // It runs alone in warp 3 where that warp has no other work (kW8Warp3),
+  // else in lane 1 of the producer warp.
   const auto w8_producer = [&]() {
     int j = 0;
     uint32_t jph = 0;
@@ -694,13 +729,14 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       }
     }
   };
-  if (Cfg::kTmemA && warp == 3) {
+  if (Cfg::kW8Warp3 && warp == 3) {
     if (lane == 0) w8_producer();
   } else if (warp == 0) {
     // ---------------- TMA producer ----------------
     // Lane 0 arms the stages (activation rows, and bf16 weights); with fp8
-    // weights on token tiles lane 1 runs the weight slot producer.
-    if (Cfg::kFp8 && !Cfg::kTmemA && lane == 1) w8_producer();
+    // weights on token tiles of gathered rows lane 1 runs the weight slot
+    // producer.
+    if (Cfg::kFp8 && !Cfg::kW8Warp3 && lane == 1) w8_producer();
     if (lane == 0) {
       int s = 0;
       uint32_t ph = 0;
@@ -968,10 +1004,16 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
           uint8_t* st = smem + s * Cfg::STAGE_BYTES;
           const uint8_t* slot = w8_ring + j * Cfg::W8_SLOT;
 #pragma unroll
-          for (int i = 0; i < Cfg::NUM_W; ++i)
-            widen_fp8_tile<Cfg::W_ROWS, Cfg::CONV_THREADS>(slot + i * Cfg::W8_BYTES,
-                                                           st + Cfg::ACT_BYTES + i * Cfg::W_BYTES,
-                                                           ct);
+          for (int i = 0; i < Cfg::NUM_W; ++i) {
+            if (Cfg::kFp4)
+              widen_fp4_tile<Cfg::W_ROWS, Cfg::CONV_THREADS>(
+                  slot + i * Cfg::W8_BYTES, slot + i * Cfg::W8_BYTES + Cfg::W4_CODES, (kb * 2) & 15,
+                  st + Cfg::ACT_BYTES + i * Cfg::W_BYTES, ct);
+            else
+              widen_fp8_tile<Cfg::W_ROWS, Cfg::CONV_THREADS>(slot + i * Cfg::W8_BYTES,
+                                                             st + Cfg::ACT_BYTES + i * Cfg::W_BYTES,
+                                                             ct);
+          }
           // each thread orders its own writes for the tensor core, then one
           // lane per warp hands the warp's part on (8 arrivals, not 256)
           fence_proxy_async_smem();
@@ -1015,7 +1057,9 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
           if (Cfg::kDual) tmem_ld_32x32(tb + Cfg::ACC_N + c0, v1);
           tc_wait_ld();
           if (f0 + c0 < p.F) {
-            if (Cfg::kFp8) {  // per-output-channel scales of the fp8 weights
+            // per-output-channel scales of the fp8 weights (fp4 weights have
+            // none: their block exponents were applied while widening)
+            if (Cfg::kFp8 && !Cfg::kFp4) {
               const float* sc = p.w_scale + (size_t)g * p.w_group_stride + f0 + c0;
 #pragma unroll
               for (int i = 0; i < 32; ++i) {
@@ -1036,7 +1080,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         const int f = f0 + qd * 32 + lane;
         const int fl = qd * 32 + lane;  // this thread's feature within the tile
         float s0 = 1.f, s1 = 1.f;  // fp8 weights: this thread's output channel scales
-        if (Cfg::kFp8 && p.w_scale && f < p.F) {
+        if (Cfg::kFp8 && !Cfg::kFp4 && f < p.F) {
           const float* sc = p.w_scale + (size_t)g * p.w_group_stride + f;
           s0 = __ldg(sc);
           if (Cfg::kDual) s1 = __ldg(sc + p.dual_offset);

@@ -550,13 +550,15 @@ FP4 = {
 
 
 @pytest.mark.parametrize("name", list(FP4))
-def test_fp4_experts(name):
+@pytest.mark.parametrize("flags", [0, lmoe.FORCE_SWAP])
+def test_fp4_experts(name, flags):
     """MXFP4 expert weights (E2M1 codes, one power-of-two scale per 32
-    inputs) widened in tensor memory on the weight-stationary kernels,
-    against the oracle on the same codes and exponents."""
-    res = check_forward(FP4[name], fixture=True)
+    inputs), against the oracle on the same codes and exponents: FC1 widened
+    in tensor memory on the weight-stationary kernel, FC2 widened in shared
+    memory on token tiles (default) or in tensor memory (FORCE_SWAP)."""
+    res = check_forward(FP4[name], flags=flags, fixture=True)
     assert res["unique"] >= 0.9 * res["tokens"]
-    assert paths(res) == (2, 2)
+    assert paths(res) == ((2, 2) if flags else (2, 1))
 
 
 def test_fp4_experts_prefill_sized():
@@ -565,7 +567,7 @@ def test_fp4_experts_prefill_sized():
     w = W_("f4-prefill", T=1024, d=512, l=512, N=16, k=4, m=512, act="swiglu",
            shared_m=512, seed=55, expert_fp4=True)
     res = check_forward(w, tokens=sample_tokens(w.T, 160, seed=5))
-    assert paths(res) == (2, 2)
+    assert paths(res) == (2, 1)
     assert res["unique"] >= 0.8 * res["tokens"]
 
 
