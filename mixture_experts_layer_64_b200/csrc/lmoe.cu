@@ -732,7 +732,13 @@ lmoe_status run_gemm(lmoe_layer* h, GemmCall c, cudaStream_t st, int* path = nul
     case GK_FC2:
       return c.swap ? launch_tc<TcCfg<true, false, false, 128, EPI_SCALE_ROWS>>(h, c, st)
                     : launch_tc<TcCfg<false, false, false, 256, EPI_SCALE_ROWS>>(h, c, st);
-    case GK_UP: return launch_tc<TcCfg<false, false, false, 256, EPI_RESID>>(h, c, st);
+    case GK_UP:
+      // decode sizes: 128-wide tiles where 256-wide ones would leave more
+      // than half the SMs idle (twice the CTAs, each with half the loads and
+      // half the epilogue)
+      if (!c.p.offsets && 2L * c.p.max_row_tiles * ((c.p.F + 255) / 256) <= h->num_sms)
+        return launch_tc<TcCfg<false, false, false, 128, EPI_RESID>>(h, c, st);
+      return launch_tc<TcCfg<false, false, false, 256, EPI_RESID>>(h, c, st);
   }
   return LMOE_ERR_INVALID_ARG;
 }
