@@ -125,7 +125,7 @@ struct TcCfg {
   static constexpr bool kW8Warp3 = kFp8 && (kTmemA || !kCpGather);
   static constexpr int STAGES = kTmemA ? LMOE_TMEMA_STAGES
                                 : kFp8 ? (STAGES_F8 < 3 ? 3 : (STAGES_F8 > 8 ? 8 : STAGES_F8))
-                                       : (STAGES_RAW > 8 ? 8 : STAGES_RAW);
+                                       : (STAGES_RAW > 12 ? 12 : STAGES_RAW);
   static constexpr int W8_SLOT = NUM_W * W8_BYTES;
   static constexpr int S8_RAW = kFp8 ? (BUDGET - STAGES * STAGE_BYTES) / W8_SLOT : 0;  // E4M3 slots
   static constexpr int S8_CAP = kTmemA ? LMOE_TMEMA_S8CAP : 16;
