@@ -71,8 +71,11 @@ struct TcCfg {
   static constexpr bool kCpGather = kGather && (!kSwap || kWideSwap);
   // warps 0-3: producer, MMA issuer, gather; then the epilogue warps (two
   // warpgroups, or one with fp8 weights), then (fp8) the converter warps that
-  // widen the E4M3 weight tiles to bf16
-  static constexpr int EPI_WARPS = kFp8 ? 4 : kEpiWarps;
+  // widen the E4M3 weight tiles to bf16.  The ungated token-tiled expert FC1
+  // (128 x 256 tiles, eight 32-column chunks per TMEM lane quarter) takes
+  // three warpgroups, so that a warp drains three chunks of a tile, not
+  // four, while the next tile's MMAs run.
+  static constexpr int EPI_WARPS = kFp8 ? 4 : (!kSwap && kGather && !kDual) ? 12 : kEpiWarps;
   static constexpr int CONV_THREADS = kFp8 ? 256 : 0;
   static constexpr int THREADS = 128 + 32 * EPI_WARPS + CONV_THREADS;
   // fp8 weights: the MMA runs on f16 operands, so the FC1 output (the FC2
@@ -1028,9 +1031,9 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       }
     }
   } else {
-    // ---------------- epilogue (warps 4..11: two warpgroups) ----------------
+    // ---------------- epilogue (warps 4.. : two or three warpgroups) ----------------
     const int qd = warp & 3;          // TMEM lane quarter this warp may access
-    const int eg = (warp - 4) >> 2;   // warpgroup: even / odd 32-column chunks
+    const int eg = (warp - 4) >> 2;   // warpgroup: every (EPI_WARPS / 4)-th 32-column chunk
     constexpr int kChunkStride = 32 * (Cfg::EPI_WARPS / 4);  // columns between a warp's chunks
     int it = 0;
     uint32_t sk_ph = 0;  // stream-K: phase of epibar
