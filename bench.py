@@ -108,49 +108,125 @@ def recorded_traffic(workload: str, stage: str):
 # clocks during the timed region
 # ---------------------------------------------------------------------------
 
+def gpu_uuid(dev) -> Optional[str]:
+    """The CUDA device's UUID as NVML spells it (without its "GPU-" prefix)."""
+    try:
+        return str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        return None
+
+
 class ClockSampler:
+    """SM clock, power and clock-event (throttle) reasons of one GPU while the
+    timed region runs.  NVML is read in a thread every 20 ms (read-only
+    queries; the device is found by its UUID, since NVML does not follow
+    CUDA_VISIBLE_DEVICES); without NVML the nvidia-smi query loop runs
+    instead, and timing starts only once its first sample has landed."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    PERIOD_S = 0.02
 
-    def __init__(self, gpu_index: int, path: Optional[str] = None):
-        """Samples every 100 ms into `path` (a temporary file when None)."""
+    def __init__(self, gpu_index: int, path: Optional[str] = None, uuid: Optional[str] = None):
+        """Rows go to `path` as CSV (nvidia-smi's columns) when given."""
         self.gpu = gpu_index
-        self.proc = None
-        self.temporary = path is None
-        if path is None:
-            fd, path = tempfile.mkstemp(prefix=f"clocks_gpu{gpu_index}_", suffix=".csv")
-            os.close(fd)
+        self.uuid = uuid
         self.path = path
+        self.proc = None
+        self.thread = None
+        self.rows = []
+
+    # ---- NVML thread
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        if self.uuid:
+            for u in (self.uuid, "GPU-" + self.uuid):
+                try:
+                    return pynvml, pynvml.nvmlDeviceGetHandleByUUID(u)
+                except pynvml.NVMLError:
+                    pass
+        return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
+
+    def _nvml_row(self, nv, h):
+        sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+        mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+        pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+        try:
+            rs = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+        except AttributeError:
+            rs = nv.nvmlDeviceGetCurrentClocksThrottleReasons(h)
+        bits = (nv.nvmlClocksEventReasonHwSlowdown, nv.nvmlClocksEventReasonHwThermalSlowdown,
+                nv.nvmlClocksEventReasonSwThermalSlowdown, nv.nvmlClocksEventReasonSwPowerCap)
+        flags = ["Active" if rs & b else "Not Active" for b in bits]
+        return [str(self.gpu), str(sm), str(mx), f"{pw:.2f}", hex(rs)] + flags
+
+    def _loop(self, nv, h):
+        while not self.done.is_set():
+            try:
+                self.rows.append(self._nvml_row(nv, h))
+            except Exception:
+                pass
+            self.done.wait(self.PERIOD_S)
 
     def start(self):
+        import threading
         try:
-            os.makedirs(os.path.dirname(os.path.abspath(self.path)), exist_ok=True)
-            self.fh = open(self.path, "w")
+            nv, h = self._nvml_handle()
+            self.rows.append(self._nvml_row(nv, h))
+            self.done = threading.Event()
+            self.thread = threading.Thread(target=self._loop, args=(nv, h), daemon=True)
+            self.thread.start()
+            return
+        except Exception:
+            self.thread = None
+        # fallback: nvidia-smi's query loop, into a file
+        try:
+            self.smi_path = self.path
+            if self.smi_path is None:
+                fd, self.smi_path = tempfile.mkstemp(prefix=f"clocks_gpu{self.gpu}_", suffix=".csv")
+                os.close(fd)
+            self.fh = open(self.smi_path, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
                  "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=self.fh, stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
-        time.sleep(0.3)
+            return
+        t_end = time.time() + 5.0
+        while time.time() < t_end and not self._smi_rows():
+            time.sleep(0.02)
+
+    def _smi_rows(self):
+        try:
+            with open(self.smi_path) as fh:
+                return [[c.strip() for c in r] for r in csv.reader(fh) if len(r) >= 9]
+        except OSError:
+            return []
 
     def stop(self):
-        if self.proc is None:
+        if self.thread is not None:
+            time.sleep(self.PERIOD_S)
+            self.done.set()
+            self.thread.join(timeout=2)
+            rows = list(self.rows)
+            if self.path:
+                with open(self.path, "w") as fh:
+                    fh.writelines(", ".join(r) + "\n" for r in rows)
+        elif self.proc is not None:
+            time.sleep(0.15)  # one more sample after the timed region
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.fh.close()
+            rows = self._smi_rows()
+            if self.path is None:
+                os.unlink(self.smi_path)
+        else:
             return None
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        self.fh.close()
-        rows = []
-        with open(self.path) as fh:
-            for r in csv.reader(fh):
-                if len(r) >= 9:
-                    rows.append([c.strip() for c in r])
-        if self.temporary:
-            os.unlink(self.path)
         if not rows:
             return None
 
@@ -171,7 +247,8 @@ class ClockSampler:
                           if rows[i][5 + j].lower().startswith("active")})
         return {"sm_mhz": statistics.median(sm[i] for i in load),
                 "sm_max_mhz": max(x for x in mx if x == x) if any(x == x for x in mx) else None,
-                "reasons": reasons, "samples": len(rows), "samples_under_load": len(load)}
+                "reasons": reasons, "samples": len(rows), "samples_under_load": len(load),
+                "source": "nvml" if self.thread is not None else "nvidia-smi"}
 
 
 # ---------------------------------------------------------------------------
@@ -393,8 +470,8 @@ def measure(args, name: str, pg, rank: int, ws: int, local: int, dev, flags: int
     stage_ms = {k: v["mean"] for k, v in stage_pct.items()}
     dom = max(stage_ms, key=stage_ms.get)
 
-    sampler = ClockSampler(local, args.clocks_csv if name == args.workload else None) \
-        if rank == 0 else None
+    sampler = ClockSampler(local, args.clocks_csv if name == args.workload else None,
+                           gpu_uuid(dev)) if rank == 0 else None
     if sampler:
         sampler.start()
     # ---- timed region: K steps; events on the launching stream around the

@@ -3,6 +3,7 @@ bench's use of recorded DRAM traffic."""
 import json
 import os
 import re
+import sys
 
 import pytest
 
@@ -89,3 +90,44 @@ def test_variant_sweep_costs_follow_the_paper():
         assert [p["vs_standard"]["expert_weight_bytes"] for p in out] == [1.0, 1.0, 1.0]
         assert out[1]["N"] == out[2]["N"] == alpha * out[0]["N"]
         assert out[2]["k"] == alpha * out[1]["k"] == alpha * out[0]["k"]
+
+
+def test_clock_sampler_reads_nvml_in_a_thread(monkeypatch):
+    """The bench's clock record from a fake NVML (read-only queries): the
+    median SM clock of the samples under load (the top half by power), the
+    maximum clock, and the throttle reasons active under load by name."""
+    import time
+    import types
+    import bench
+
+    fake = types.ModuleType("pynvml")
+    fake.NVMLError = type("NVMLError", (Exception,), {})
+    fake.NVML_CLOCK_SM = 1
+    fake.nvmlClocksEventReasonSwPowerCap = 0x4
+    fake.nvmlClocksEventReasonHwSlowdown = 0x8
+    fake.nvmlClocksEventReasonSwThermalSlowdown = 0x20
+    fake.nvmlClocksEventReasonHwThermalSlowdown = 0x40
+    state = {"n": 0}
+
+    def clock(h, kind):
+        state["n"] += 1
+        return 1800 if state["n"] % 2 else 1965  # alternating samples
+
+    fake.nvmlInit = lambda: None
+    fake.nvmlDeviceGetHandleByUUID = lambda u: ("uuid", u)
+    fake.nvmlDeviceGetHandleByIndex = lambda i: ("index", i)
+    fake.nvmlDeviceGetClockInfo = clock
+    fake.nvmlDeviceGetMaxClockInfo = lambda h, kind: 1965
+    # power follows the clock: the 1965 MHz samples are the loaded ones
+    fake.nvmlDeviceGetPowerUsage = lambda h: 900000 if state["n"] % 2 == 0 else 300000
+    fake.nvmlDeviceGetCurrentClocksEventReasons = lambda h: 0x4 if state["n"] % 2 == 0 else 0x0
+    monkeypatch.setitem(sys.modules, "pynvml", fake)
+
+    s = bench.ClockSampler(0, None, "00000000-0000-0000-0000-000000000000")
+    s.start()
+    time.sleep(0.15)
+    rec = s.stop()
+    assert rec["source"] == "nvml"
+    assert rec["samples"] >= 3 and rec["samples_under_load"] == max(1, rec["samples"] // 2)
+    assert rec["sm_max_mhz"] == 1965
+    assert rec["sm_mhz"] == 1965 and rec["reasons"] == ["sw_power_cap"]
