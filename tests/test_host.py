@@ -131,3 +131,19 @@ def test_clock_sampler_reads_nvml_in_a_thread(monkeypatch):
     assert rec["samples"] >= 3 and rec["samples_under_load"] == max(1, rec["samples"] // 2)
     assert rec["sm_max_mhz"] == 1965
     assert rec["sm_mhz"] == 1965 and rec["reasons"] == ["sw_power_cap"]
+
+
+def test_clock_sampler_without_nvml_or_nvidia_smi(monkeypatch, tmp_path):
+    """Without NVML the sampler falls back to the nvidia-smi query loop; if
+    that command is missing too, the record is None (and start/stop neither
+    raise nor wait long)."""
+    import time
+    import bench
+
+    monkeypatch.setitem(sys.modules, "pynvml", None)  # import pynvml raises ImportError
+    monkeypatch.setenv("PATH", str(tmp_path))          # no nvidia-smi on the path
+    s = bench.ClockSampler(0, str(tmp_path / "clocks.csv"))
+    t0 = time.time()
+    s.start()
+    rec = s.stop()
+    assert rec is None and time.time() - t0 < 5.0
